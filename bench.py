@@ -1,0 +1,558 @@
+#!/usr/bin/env python
+"""Benchmark of the paged decode-attention hot path on B200.
+
+One step = one decode step of the workload over one layer: host bookkeeping
+(append one token to every sequence, pack block tables / lengths / slots),
+host-to-device copy of that metadata, copy-on-write copies if any,
+``reshape_and_cache`` of the new tokens, ``paged_attention_decode`` (with the
+split-context reduce). Metric: KV GB/s = algorithmic bytes of the attention
+call (K and V of every context token, q, out, block-table entries, lengths)
+per second of step time, plus context tokens per second.
+
+Default workload: OPT-13B geometry, one layer - 64 sequences, 40 heads x 128,
+block size 16, context lengths U[1, 2048], pool 1.25x the need, fp16,
+partitions of 512 tokens. Inputs are synthetic and resident in HBM before the
+timed region; the KV pool (about 1.7 GB) exceeds L2, so no flush is needed.
+
+Every step grows each sequence by one token. So that the timed lengths stay
+those of the workload whatever the step count, the loop round-robins over R
+identical copies of the one-layer workload (as a model's layers would), and
+each copy starts short by half the steps it will take, so its lengths during
+timing are centred on the configured ones.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                       [--workload opt13b|gqa_long_bs16|gqa_long_bs32]
+For N > 1 launch with torchrun; every rank runs an independent shard (its own
+pool and batch: weak scaling, no data-path collective).
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+from workloads.values import K_STREAM, Q_STREAM, V_STREAM, normal_bits, value_seed_words  # noqa: E402
+
+METRIC = "paged decode attention: KV GB/s (% of HBM peak) and seq-tokens/s per layer"
+UNIT = "GB/s"
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def algorithmic_bytes(lens, g):
+    """Bytes one attention call must move: K and V of every context token, q, out,
+    block-table entries and context lengths."""
+    lens = np.asarray(lens, dtype=np.int64)
+    e = g.elem_bytes
+    kv = int(lens.sum()) * g.num_kv_heads * g.head_dim * e * 2
+    qo = len(lens) * g.num_q_heads * g.head_dim * e * 2
+    meta = 4 * int(np.sum(-(-lens // g.block_size))) + 4 * len(lens)
+    return kv + qo + meta
+
+
+# ---------------------------------------------------------------- clocks (NVML)
+class ClockSampler:
+    """Samples SM clock and throttle reasons of one GPU every few ms while running."""
+
+    REASONS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
+               "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80}
+
+    def __init__(self, torch_device):
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._h = None
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            import torch
+
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(torch_device).uuid)
+            self._h = pynvml.nvmlDeviceGetHandleByUUID(uuid.encode())
+            self._nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # pragma: no cover - depends on the box
+            self.error = repr(e)
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                fn = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                    nv.nvmlDeviceGetCurrentClocksThrottleReasons
+                r = fn(self._h)
+                for name, bit in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self._h is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._h is not None:
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                    "samples": 0}
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------- distributed
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def dist_max(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def dist_sum(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+# ---------------------------------------------------------------- our arm
+class Replica:
+    """One copy of the one-layer workload: host pool, sequences, device KV pool."""
+
+    def __init__(self, wl, start_lens, device, prefill_k, prefill_v):
+        import torch
+        import paged_kv_cache_319_b200 as kvp
+
+        g = wl.geometry
+        self.pool = kvp.BlockPool(wl.num_blocks, g.block_size, g.num_kv_heads, g.head_dim, g.dtype,
+                                  wl.free_order)
+        self.seqs = np.array([self.pool.create() for _ in start_lens], dtype=np.int64)
+        slots = []
+        for s, L in zip(self.seqs, start_lens):
+            slots.extend(self.pool.append(int(s), int(L)))
+        tdt = torch.float16 if g.dtype == "f16" else torch.bfloat16
+        shape = (wl.num_blocks, g.num_kv_heads, g.block_size, g.head_dim)
+        self.k = torch.zeros(shape, dtype=tdt, device=device)
+        self.v = torch.zeros(shape, dtype=tdt, device=device)
+        st = torch.tensor(slots, dtype=torch.int64, device=device)
+        kvp.reshape_and_cache(prefill_k, prefill_v, self.k, self.v, st)
+        self.lens = np.asarray(start_lens, dtype=np.int64)
+
+
+def to_dev(bits, dtype, device):
+    import torch
+
+    t = torch.from_numpy(np.ascontiguousarray(bits).view(np.int16))
+    return t.view(torch.float16 if dtype == "f16" else torch.bfloat16).to(device)
+
+
+def run_ours(args, world, rank, local):
+    import torch
+    import paged_kv_cache_319_b200 as kvp
+
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    wl = workloads.by_name(args.workload)
+    g = wl.geometry
+    part = wl.partition_size if args.partition is None else args.partition
+    ctx = np.asarray(wl.info["context_lens"], dtype=np.int64)
+    S = len(ctx)
+    W, K = args.warmup, args.steps
+
+    # Replicas: none grows by more than ~64 tokens over warm-up, timing and the
+    # end-to-end pass; each starts short by its warm-up steps plus half its
+    # timed steps, so the timed lengths are centred on the configured ones.
+    K_e2e = max(1, min(K, 64))
+    pool_bytes = 2 * wl.num_blocks * g.num_kv_heads * g.block_size * g.head_dim * g.elem_bytes
+    free_b = torch.cuda.mem_get_info(device)[0]
+    r_cap = max(1, int(0.6 * free_b // pool_bytes))
+    R = max(1, min(r_cap, math.ceil((W + K + K_e2e) / 64)))
+    shift = math.ceil(W / R) + math.ceil(K / R) // 2
+    start = np.maximum(ctx - shift, 1)
+    grow = math.ceil((W + K + K_e2e) / R) + 1
+    need_end = int(np.sum(-(-(start + grow) // g.block_size)))
+    if need_end > wl.num_blocks:
+        raise SystemExit(f"pool of {wl.num_blocks} blocks too small for {W + K} steps")
+
+    seed_rank = wl.value_seed + 7919 * rank
+    n_pre = int(start.sum())
+    pk = to_dev(normal_bits(value_seed_words(seed_rank, K_STREAM, 0), (max(n_pre, 1), g.num_kv_heads, g.head_dim), g.dtype), g.dtype, device)
+    pv = to_dev(normal_bits(value_seed_words(seed_rank, V_STREAM, 0), (max(n_pre, 1), g.num_kv_heads, g.head_dim), g.dtype), g.dtype, device)
+    reps = [Replica(wl, start, device, pk[:n_pre], pv[:n_pre]) for _ in range(R)]
+    del pk, pv
+
+    # per-step inputs, resident in HBM (a cycle of NI sets)
+    NI = min(W + K, 32)
+    qs = [to_dev(normal_bits(value_seed_words(seed_rank, Q_STREAM, 1 + i), (S, g.num_q_heads, g.head_dim), g.dtype), g.dtype, device) for i in range(NI)]
+    kn = [to_dev(normal_bits(value_seed_words(seed_rank, K_STREAM, 1 + i), (S, g.num_kv_heads, g.head_dim), g.dtype), g.dtype, device) for i in range(NI)]
+    vn = [to_dev(normal_bits(value_seed_words(seed_rank, V_STREAM, 1 + i), (S, g.num_kv_heads, g.head_dim), g.dtype), g.dtype, device) for i in range(NI)]
+
+    max_ctx_total = int(start.max()) + grow
+    MB = -(-max_ctx_total // g.block_size)
+    NBUF = 3
+    pin = lambda shape, dt: torch.empty(shape, dtype=dt, pin_memory=True)
+    slot_h = [pin((S,), torch.int64) for _ in range(NBUF)]
+    tab_h = [pin((S, MB), torch.int32) for _ in range(NBUF)]
+    len_h = [pin((S,), torch.int32) for _ in range(NBUF)]
+    slot_d = [torch.empty((S,), dtype=torch.int64, device=device) for _ in range(NBUF)]
+    tab_d = [torch.empty((S, MB), dtype=torch.int32, device=device) for _ in range(NBUF)]
+    len_d = [torch.empty((S,), dtype=torch.int32, device=device) for _ in range(NBUF)]
+    done = [None] * NBUF
+    out = torch.empty((S, g.num_q_heads, g.head_dim), dtype=qs[0].dtype, device=device)
+    ws_bytes = kvp.decode_workspace_bytes(S, g.num_q_heads, g.head_dim, max_ctx_total, part)
+    ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    step_bytes, step_tokens, launches = [], [], []
+    ev_pairs = []
+
+    def step(i, timed):
+        rep = reps[i % R]
+        b = i % NBUF
+        if done[b] is not None:
+            done[b].synchronize()
+        slots_np = slot_h[b].numpy()
+        rep.pool.append_batch(rep.seqs, 1, out=slots_np)
+        copies = rep.pool.take_copies()
+        rep.pool.build_batch(rep.seqs, MB, tab_h[b].numpy(), len_h[b].numpy())
+        rep.lens += 1
+        slot_d[b].copy_(slot_h[b], non_blocking=True)
+        tab_d[b].copy_(tab_h[b], non_blocking=True)
+        len_d[b].copy_(len_h[b], non_blocking=True)
+        n_launch = 0
+        if copies:
+            pairs = torch.tensor(copies, dtype=torch.int32).to(device, non_blocking=True)
+            kvp.copy_blocks(rep.k, rep.v, pairs)
+            n_launch += 1
+        j = i % NI
+        kvp.reshape_and_cache(kn[j], vn[j], rep.k, rep.v, slot_d[b])
+        n_launch += 1
+        if timed:
+            e0 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+        kvp.paged_attention_decode(qs[j], rep.k, rep.v, tab_d[b], len_d[b], wl.scale, out,
+                                   max_context_len=max_ctx_total, partition_size=part,
+                                   workspace=ws)
+        n_launch += 2 if (part and int(rep.lens.max()) > part) else 1
+        if timed:
+            e1 = torch.cuda.Event(enable_timing=True)
+            e1.record(stream)
+            ev_pairs.append((e0, e1))
+            step_bytes.append(algorithmic_bytes(rep.lens, g))
+            step_tokens.append(int(rep.lens.sum()))
+            launches.append(n_launch)
+        ev = torch.cuda.Event()
+        ev.record(stream)
+        done[b] = ev
+
+    for i in range(W):
+        step(i, False)
+    torch.cuda.synchronize(device)
+    kvp.check_device_error(device)
+    barrier(world)
+    torch.cuda.synchronize(device)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(device) as clk:
+        t0.record(stream)
+        for i in range(W, W + K):
+            step(i, True)
+        t1.record(stream)
+        torch.cuda.synchronize(device)
+    kvp.check_device_error(device)
+    barrier(world)
+    elapsed_ms = t0.elapsed_time(t1)
+    max_ms = dist_max(elapsed_ms, world)
+    total_bytes = dist_sum(float(sum(step_bytes)), world)
+    total_tokens = dist_sum(float(sum(step_tokens)), world)
+    dec_ms = [a.elapsed_time(b) for a, b in ev_pairs]
+    dec_avg_ms = sum(dec_ms) / len(dec_ms)
+    dec_bytes_avg = sum(step_bytes) / len(step_bytes)
+    achieved = dec_bytes_avg / (dec_avg_ms * 1e-3) / 1e9
+
+    # ---- end to end through the public API with host buffers
+    e2e = run_e2e(args, wl, reps, device, seed_rank, MB, max_ctx_total, part, ws, world)
+
+    peak, peak_kind = peaks()
+    value = total_bytes / (max_ms * 1e-3) / 1e9
+    res = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": K,
+        "warmup": W,
+        "ms_per_step": round(max_ms / K, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": g.dtype,
+        "data": "synthetic (seeded N(0,1) q/K/V; lengths and placement as configured)",
+        "config": {
+            "workload": wl.description,
+            "name": wl.name,
+            "num_seqs_per_gpu": S,
+            "num_q_heads": g.num_q_heads,
+            "num_kv_heads": g.num_kv_heads,
+            "head_dim": g.head_dim,
+            "block_size": g.block_size,
+            "partition_size": part,
+            "mean_context_len_timed": round(float(np.mean(step_tokens)) / S, 1),
+            "replicas": R,
+            "l2": "inputs larger than L2 (KV pool %.2f GB per replica)" % (pool_bytes / 1e9),
+            "parallelism": f"replicas x{world} (independent shards, no collective)",
+        },
+        "seq_tokens_per_s": round(total_tokens / (max_ms * 1e-3), 1),
+        "decode_tokens_per_s": round(world * S * K / (max_ms * 1e-3), 1),
+        "hbm_frac_of_step": round(value / peak, 4),
+        "gpu_launches": int(sum(launches)),
+        "roofline": {
+            "kernel": "paged_attention_decode (pass 1 + split reduce)",
+            "bound": "hbm",
+            "achieved": round(achieved, 1),
+            "peak": peak,
+            "peak_source": peak_kind,
+            "unit": "GB/s",
+            "frac": round(achieved / peak, 4),
+            "frac_of_nominal_8tbs": round(achieved / 8000.0, 4),
+            "traffic": None,
+            "avg_launch_us": round(dec_avg_ms * 1e3, 2),
+            "algorithmic_bytes_per_launch": int(dec_bytes_avg),
+        },
+        "e2e": e2e,
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline(wl, budget_s=args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+
+
+def run_e2e(args, wl, reps, device, seed_rank, MB, max_ctx_total, part, ws, world):
+    """Same metric with host inputs: per step, pinned host -> device copies of q, the
+    new K/V and the metadata, the kernels, and the output copied back, synchronised."""
+    import torch
+    import paged_kv_cache_319_b200 as kvp
+
+    g = wl.geometry
+    S = len(reps[0].seqs)
+    K = max(1, min(args.steps, 64))
+    R = len(reps)
+    pin = lambda t: t.pin_memory()
+    host_q = pin(torch.from_numpy(normal_bits(value_seed_words(seed_rank, Q_STREAM, 999), (S, g.num_q_heads, g.head_dim), g.dtype).view(np.int16)))
+    host_k = pin(torch.from_numpy(normal_bits(value_seed_words(seed_rank, K_STREAM, 999), (S, g.num_kv_heads, g.head_dim), g.dtype).view(np.int16)))
+    host_v = pin(torch.from_numpy(normal_bits(value_seed_words(seed_rank, V_STREAM, 999), (S, g.num_kv_heads, g.head_dim), g.dtype).view(np.int16)))
+    tdt = torch.float16 if g.dtype == "f16" else torch.bfloat16
+    host_out = torch.empty((S, g.num_q_heads, g.head_dim), dtype=torch.int16).pin_memory()
+    slot_h = torch.empty((S,), dtype=torch.int64).pin_memory()
+    tab_h = torch.empty((S, MB), dtype=torch.int32).pin_memory()
+    len_h = torch.empty((S,), dtype=torch.int32).pin_memory()
+    q_d = torch.empty((S, g.num_q_heads, g.head_dim), dtype=tdt, device=device)
+    k_d = torch.empty((S, g.num_kv_heads, g.head_dim), dtype=tdt, device=device)
+    v_d = torch.empty_like(k_d)
+    out = torch.empty_like(q_d)
+    slot_d = torch.empty((S,), dtype=torch.int64, device=device)
+    tab_d = torch.empty((S, MB), dtype=torch.int32, device=device)
+    len_d = torch.empty((S,), dtype=torch.int32, device=device)
+    h2d = (host_q.numel() + host_k.numel() + host_v.numel()) * 2 + slot_h.numel() * 8 + \
+        (tab_h.numel() + len_h.numel()) * 4
+    d2h = host_out.numel() * 2
+    total_bytes = 0
+    barrier(world)
+    torch.cuda.synchronize(device)
+    t = time.perf_counter()
+    for i in range(K):
+        rep = reps[i % R]
+        rep.pool.append_batch(rep.seqs, 1, out=slot_h.numpy())
+        copies = rep.pool.take_copies()
+        rep.pool.build_batch(rep.seqs, MB, tab_h.numpy(), len_h.numpy())
+        rep.lens += 1
+        q_d.view(torch.int16).copy_(host_q, non_blocking=True)
+        k_d.view(torch.int16).copy_(host_k, non_blocking=True)
+        v_d.view(torch.int16).copy_(host_v, non_blocking=True)
+        slot_d.copy_(slot_h, non_blocking=True)
+        tab_d.copy_(tab_h, non_blocking=True)
+        len_d.copy_(len_h, non_blocking=True)
+        if copies:
+            kvp.copy_blocks(rep.k, rep.v, torch.tensor(copies, dtype=torch.int32).to(device))
+        kvp.reshape_and_cache(k_d, v_d, rep.k, rep.v, slot_d)
+        kvp.paged_attention_decode(q_d, rep.k, rep.v, tab_d, len_d, wl.scale, out,
+                                   max_context_len=max_ctx_total, partition_size=part, workspace=ws)
+        host_out.copy_(out.view(torch.int16), non_blocking=True)
+        torch.cuda.current_stream(device).synchronize()
+        total_bytes += algorithmic_bytes(rep.lens, g)
+    el = time.perf_counter() - t
+    el = dist_max(el, world)
+    total_bytes = dist_sum(float(total_bytes), world)
+    return {"value": round(total_bytes / el / 1e9, 2), "unit": UNIT, "steps": K,
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+
+
+# ---------------------------------------------------------------- CPU oracle
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+
+        return max([d.get("num_threads", 1) for d in threadpool_info()] or [1])
+    except Exception:
+        return int(os.environ.get("OMP_NUM_THREADS", "1"))
+
+
+def cpu_baseline(wl, budget_s=15.0, seqs_per_step=None):
+    """The fp64 oracle on the host: gather + softmax(qK^T)V per sequence, timed on a
+    bounded sample of the workload's decode step (the first sequences of the batch)."""
+    from oracle.replay import OracleReplay
+
+    rp = OracleReplay(wl)
+    rp.run()
+    (i, seqs, tables, lens), = rp.attends[-1:]
+    g = wl.geometry
+    done, nbytes = 0, 0
+    t0 = time.perf_counter()
+    order = list(range(len(lens)))
+    while time.perf_counter() - t0 < budget_s and done < len(order):
+        s = order[done]
+        rp.decode(i, tables, lens, seqs=[s], split=False)
+        nbytes += algorithmic_bytes([lens[s]], g)
+        done += 1
+    el = time.perf_counter() - t0
+    return {"value": round(nbytes / el / 1e9, 4), "unit": UNIT,
+            "cores": len(os.sched_getaffinity(0)), "blas_threads": cpu_threads(), "kind": "oracle",
+            "sample": f"{done} of {len(lens)} sequences of one decode step ({wl.name}), "
+                      f"{nbytes / 1e9:.3f} GB of K/V, {el:.1f} s"}
+
+
+def run_reference(args, world, rank):
+    """The oracle as the reference arm: each step is a bounded sample of the workload."""
+    if rank != 0:
+        return
+    from oracle.replay import OracleReplay
+
+    wl = workloads.by_name(args.workload)
+    rp = OracleReplay(wl)
+    rp.run()
+    (i, seqs, tables, lens), = rp.attends[-1:]
+    g = wl.geometry
+    per_step = max(1, min(len(lens), args.ref_seqs_per_step))
+    order = np.argsort(np.asarray(lens))[::-1][: len(lens)].tolist()
+
+    def one(k):
+        sel = [order[(k * per_step + j) % len(order)] for j in range(per_step)]
+        rp.decode(i, tables, lens, seqs=sel, split=False)
+        return algorithmic_bytes([lens[s] for s in sel], g)
+
+    for k in range(args.warmup):
+        one(k)
+    t0 = time.perf_counter()
+    nbytes = sum(one(args.warmup + k) for k in range(args.steps))
+    el = time.perf_counter() - t0
+    value = nbytes / el / 1e9
+    res = {
+        "metric": METRIC, "value": round(value, 4), "unit": UNIT, "impl": "reference",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(el * 1e3 / args.steps, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.description, "name": wl.name},
+        "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "kind": "oracle",
+                         "cores": len(os.sched_getaffinity(0)), "blas_threads": cpu_threads(),
+                         "sample": f"{per_step} sequence(s) of one decode step per step"},
+        "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(res), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="opt13b",
+                    choices=["opt13b", "gqa_long_bs16", "gqa_long_bs32"])
+    ap.add_argument("--partition", type=int, default=None)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--ref-seqs-per-step", type=int, default=1)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        # The oracle needs no GPU and no process group: rank 0 runs, the others exit.
+        run_reference(args, int(os.environ.get("WORLD_SIZE", "1")),
+                      int(os.environ.get("RANK", "0")))
+        return
+    world, rank, local = dist_setup()
+    try:
+        run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

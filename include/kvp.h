@@ -1,0 +1,278 @@
+/*
+ * kvp.h - C ABI of libkvp: a paged KV cache and its decode-attention path for
+ * NVIDIA B200 (sm_100a).
+ *
+ * The method (sources cited by page title and section):
+ *
+ *  - The KV cache of each sequence is cut into fixed-size blocks; a
+ *    per-sequence block table maps logical block numbers to physical blocks,
+ *    which are taken from a shared pool only when the sequence grows into them,
+ *    and the attention kernel follows the block table instead of assuming a
+ *    contiguous cache. ["Your GPU was mostly empty: how PagedAttention turned
+ *    KV cache waste into 2-4x throughput", section "The OS already solved this
+ *    in the 1960s"; "vLLM and PagedAttention", section "Architecture, step by
+ *    step", steps 1-3]
+ *  - Blocks are shared between sequences by reference count; a block is copied
+ *    only when a sequence writes into a block that is shared (block-level
+ *    copy-on-write, as with fork()). ["Your GPU was mostly empty", section
+ *    "Paging's second gift: copy-on-write"]
+ *  - A block that no live sequence references returns to the shared pool.
+ *    ["PagedAttention: KV cache memory management", sections "How logical
+ *    blocks, physical blocks and the block table work" and "A request
+ *    lifecycle: allocation, growth, sharing and release"]
+ *
+ * Conventions for every call:
+ *  - Returns KVP_OK (0) or a negative KVP_ERR_* status; no C++ exception
+ *    crosses this boundary. kvp_last_error_message() describes the last
+ *    failure of the calling thread.
+ *  - A failed host call leaves all state unchanged.
+ *  - Host metadata (block tables, reference counts, free list) is owned by the
+ *    pool handle. A pool is not thread-safe: one thread at a time per pool.
+ *  - Device buffers are owned by the caller and passed as raw device pointers;
+ *    no call allocates or frees device memory. `stream` is a cudaStream_t
+ *    (NULL = the legacy default stream). Device calls are asynchronous with
+ *    respect to the host: they validate their arguments, launch, and return.
+ *  - Device-side index checks (block ids, slots, context lengths) never fault:
+ *    an out-of-range index is skipped and recorded in a device error word that
+ *    kvp_check_device_error() reads back.
+ *
+ * KV cache layout (the pages fix none; this is the library's choice):
+ *   k_cache, v_cache : [num_blocks][num_kv_heads][block_size][head_dim],
+ *   row-major, separate K and V buffers, elements fp16 or bf16. One
+ *   (physical block, KV head) tile is one contiguous block_size*head_dim run.
+ *   Token slot s lives in physical block s / block_size at offset
+ *   s % block_size.
+ */
+#ifndef KVP_H_
+#define KVP_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define KVP_API __attribute__((visibility("default")))
+#else
+#define KVP_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes ------------------------------------------------------- */
+#define KVP_OK 0
+#define KVP_ERR_INVALID (-1)  /* bad argument or unsupported geometry        */
+#define KVP_ERR_OOM (-2)      /* the pool has too few free blocks            */
+#define KVP_ERR_NO_SEQ (-3)   /* no live sequence with that id               */
+#define KVP_ERR_CUDA (-4)     /* a CUDA runtime call failed                  */
+#define KVP_ERR_BOUNDS (-5)   /* a device kernel met an out-of-range index   */
+#define KVP_ERR_CAPACITY (-6) /* an output buffer is too small              */
+
+/* ---- element types ------------------------------------------------------ */
+#define KVP_F16 0
+#define KVP_BF16 1
+
+typedef struct kvp_pool kvp_pool;
+typedef void* kvp_stream_t; /* a cudaStream_t */
+
+typedef struct kvp_pool_stats {
+  int64_t num_blocks;
+  int64_t num_free;         /* blocks on the free list                      */
+  int64_t num_used;         /* blocks with reference count > 0              */
+  int64_t num_shared;       /* blocks with reference count > 1              */
+  int64_t waste_slots;      /* sum over live sequences of unused slots in   */
+                            /* their last block                             */
+  int64_t cow_copies_total; /* copy-on-write copies queued since creation   */
+  int64_t num_seqs;         /* live sequences                               */
+} kvp_pool_stats;
+
+/* =========================================================================
+ * Host: block pool and sequences (integer bookkeeping)
+ * ========================================================================= */
+
+/* Creates a pool of `num_blocks` physical blocks of `block_size` token slots
+ * for a layer group with `num_kv_heads` KV heads of `head_dim` elements of
+ * `dtype`. The free list is a stack: the first block handed out is
+ * free_order[0], then free_order[1], ... `free_order` must be a permutation of
+ * 0..num_blocks-1 (it is copied); NULL means 0, 1, 2, ... Block placement is
+ * then fully determined by the call sequence.
+ * Errors: KVP_ERR_INVALID (non-positive sizes, not a permutation, bad dtype). */
+KVP_API int kv_pool_create(int32_t num_blocks, int32_t block_size, int32_t num_kv_heads,
+                   int32_t head_dim, int32_t dtype, const int32_t* free_order,
+                   kvp_pool** out);
+
+/* Frees the pool and all its host metadata. NULL is accepted. */
+KVP_API int kv_pool_destroy(kvp_pool* pool);
+
+/* Number of free blocks. */
+KVP_API int kv_pool_num_free(const kvp_pool* pool, int32_t* n);
+
+/* Free blocks in hand-out order (next block first) into out[0..cap); *n gets
+ * the count. KVP_ERR_CAPACITY (with *n set) if cap is too small. */
+KVP_API int kv_pool_free_list(const kvp_pool* pool, int32_t* out, int32_t cap, int32_t* n);
+
+/* Reference count of one block. KVP_ERR_INVALID if block is out of range. */
+KVP_API int kv_pool_refcount(const kvp_pool* pool, int32_t block, int32_t* rc);
+
+/* Reference counts of all blocks into out[0..num_blocks). */
+KVP_API int kv_pool_refcounts(const kvp_pool* pool, int32_t* out, int32_t cap);
+
+/* Counters of the pool (see kvp_pool_stats). */
+KVP_API int kv_pool_stats(const kvp_pool* pool, kvp_pool_stats* out);
+
+/* New empty sequence (no blocks). Ids count up from 0 and are never reused;
+ * a fork also takes the next id. */
+KVP_API int kv_seq_create(kvp_pool* pool, int64_t* seq_id);
+
+/* Appends n_tokens >= 0 tokens to `seq`, one after another, and writes each
+ * token's flat slot (physical_block * block_size + offset) to slots_out
+ * (may be NULL when n_tokens == 0). A token at a block boundary takes a new
+ * block from the free list; a token that lands in a partly filled last block
+ * that other sequences also reference first takes a private copy: a new block
+ * is taken, the pair (old, new) is queued for copy_blocks, the old block loses
+ * one reference and the table entry moves to the new block.
+ * Errors: KVP_ERR_NO_SEQ, KVP_ERR_INVALID (n_tokens < 0), KVP_ERR_OOM when the
+ * free list cannot supply every block the call needs (nothing changes). */
+KVP_API int kv_seq_append(kvp_pool* pool, int64_t seq, int32_t n_tokens, int64_t* slots_out);
+
+/* Appends n_each tokens to every sequence of seqs[0..num_seqs), in that order;
+ * the result equals num_seqs successive kv_seq_append calls.
+ * slots_out[i*n_each + j] is token j of seqs[i]. All or nothing: on
+ * KVP_ERR_OOM / KVP_ERR_NO_SEQ nothing changes. */
+KVP_API int kv_seq_append_batch(kvp_pool* pool, const int64_t* seqs, int32_t num_seqs,
+                        int32_t n_each, int64_t* slots_out);
+
+/* New sequence sharing every block of `parent` (each block gains one
+ * reference); the child has the parent's length. */
+KVP_API int kv_seq_fork(kvp_pool* pool, int64_t parent, int64_t* child);
+
+/* Ends `seq`: each block of its table, in logical order, loses one reference;
+ * a block that reaches zero is pushed onto the free list. */
+KVP_API int kv_seq_release(kvp_pool* pool, int64_t seq);
+
+/* Length (tokens) of `seq`. */
+KVP_API int kv_seq_len(const kvp_pool* pool, int64_t seq, int32_t* len);
+
+/* Block table of `seq` into out[0..cap); *n gets its length.
+ * KVP_ERR_CAPACITY (with *n set) if cap is too small. */
+KVP_API int kv_seq_block_table(const kvp_pool* pool, int64_t seq, int32_t* out, int32_t cap,
+                       int32_t* n);
+
+/* Moves the queued copy-on-write pairs, in creation order, into
+ * pairs[2*i] = src, pairs[2*i+1] = dst, and clears the queue. KVP_ERR_CAPACITY
+ * (with *n set, queue kept) if cap (pairs) is too small. */
+KVP_API int kv_pool_take_copies(kvp_pool* pool, int32_t* pairs, int32_t cap, int32_t* n);
+
+/* Like kv_pool_take_copies but leaves the queue as it is. */
+KVP_API int kv_pool_pending_copies(const kvp_pool* pool, int32_t* pairs, int32_t cap, int32_t* n);
+
+/* Packs the batch metadata the decode kernels read: block_tables is
+ * [num_seqs][max_blocks] (row i = table of seqs[i], padded with -1) and
+ * context_lens[i] = length of seqs[i]. Host buffers; copy them to the device.
+ * KVP_ERR_CAPACITY if a table is longer than max_blocks. */
+KVP_API int kv_build_batch(const kvp_pool* pool, const int64_t* seqs, int32_t num_seqs,
+                   int32_t max_blocks, int32_t* block_tables, int32_t* context_lens);
+
+/* Capacity model: KV bytes per token of a model with `hidden` = heads *
+ * head_dim and `layers` layers at `elem_bytes` bytes per value, i.e.
+ * 2 * hidden * layers * elem_bytes (one key and one value vector per token
+ * and layer). ["Your GPU was mostly empty", section "Why the KV cache is an
+ * allocator problem", OPT-13B worked example] */
+KVP_API int64_t kvp_kv_bytes_per_token(int64_t hidden, int64_t layers, int64_t elem_bytes);
+
+/* =========================================================================
+ * Device: sm_100a kernels on caller-owned memory, on the caller's stream
+ * ========================================================================= */
+
+/* Writes each new token's keys and values to its slot: for t < num_tokens
+ * with s = slot_mapping[t] >= 0,
+ *   k_cache[s / block_size][h][s % block_size][:] = k_new[t][h][:]  (all h)
+ * and likewise for V. A negative slot marks padding and is skipped; a slot
+ * >= num_blocks * block_size is skipped and sets KVP_ERR_BOUNDS in the device
+ * error word. If two tokens name one slot, the result is one of them.
+ * ["PagedAttention: KV cache memory management", section "A request
+ * lifecycle: allocation, growth, sharing and release": decode appends new
+ * cache state]
+ * k_new, v_new: device [num_tokens][num_kv_heads][head_dim], dtype.
+ * slot_mapping: device int64 [num_tokens]. head_dim * 2 bytes must be a
+ * multiple of 16. */
+KVP_API int reshape_and_cache(const void* k_new, const void* v_new, void* k_cache, void* v_cache,
+                      const int64_t* slot_mapping, int32_t num_tokens, int32_t num_kv_heads,
+                      int32_t head_dim, int32_t block_size, int32_t num_blocks, int32_t dtype,
+                      kvp_stream_t stream);
+
+/* Block-level copy-on-write copies: for each i < num_pairs, with
+ * src = pairs[2*i], dst = pairs[2*i+1], the whole physical block dst of K and
+ * of V (all KV heads, all slots: block_elems = num_kv_heads * block_size *
+ * head_dim elements) becomes a copy of block src. Destinations must be
+ * distinct and no destination may be a source. Out-of-range ids are skipped
+ * and set KVP_ERR_BOUNDS in the device error word. ["Your GPU was mostly
+ * empty", section "Paging's second gift: copy-on-write"]
+ * pairs: device int32 [num_pairs][2]. block_elems * 2 bytes must be a
+ * multiple of 16. */
+KVP_API int copy_blocks(void* k_cache, void* v_cache, const int32_t* pairs, int32_t num_pairs,
+                int32_t num_blocks, int64_t block_elems, int32_t dtype, kvp_stream_t stream);
+
+/* Bytes of device workspace paged_attention_decode needs for this batch
+ * shape: 0 when partition_size == 0 or when no sequence can have more than one
+ * partition (max_context_len <= partition_size); else room for, per
+ * (sequence, query head, partition), a running max, an exponent sum and
+ * head_dim fp32 partial outputs, with P = ceil(max_context_len /
+ * partition_size) partitions: about num_seqs * num_q_heads * P *
+ * (head_dim + 2) * 4 bytes. */
+KVP_API size_t kvp_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, int32_t head_dim,
+                                  int32_t max_context_len, int32_t partition_size);
+
+/* Decode attention over the paged cache. For sequence s and query head h,
+ * with KV head g = h / (num_q_heads / num_kv_heads) and ctx = context_lens[s]:
+ *   key j    = k_cache[block_tables[s][j / block_size]][g][j % block_size][:]
+ *   value j  = v_cache[...same...]
+ *   out[s][h] = sum_j softmax_j(scale * q[s][h] . key j) * value j,  j < ctx.
+ * The kernel follows the block table ["vLLM and PagedAttention", section
+ * "Architecture, step by step", step 3]; the result is the same as attention
+ * over a contiguous cache ["Your GPU was mostly empty", section "The OS
+ * already solved this in the 1960s"]. ctx == 0 gives a zero row.
+ * Split context: with partition_size > 0 (a multiple of block_size; the
+ * grouped-query tensor-core path needs a multiple of 128), each sequence's
+ * tokens are cut into partitions of that many tokens; each partition
+ * produces its running max, exponent sum and unnormalised output in
+ * `workspace`, and a second kernel merges them by the log-sum-exp identity.
+ * Sequences with one partition write `out` directly. partition_size == 0
+ * processes each (sequence, head) in one pass and needs no workspace.
+ * q: device [num_seqs][num_q_heads][head_dim]; out: same shape and dtype.
+ * block_tables: device int32 [num_seqs][max_blocks_per_seq];
+ * context_lens: device int32 [num_seqs]; every context_lens[s] must be
+ * <= max_context_len <= max_blocks_per_seq * block_size (larger values are
+ * clamped and set KVP_ERR_BOUNDS). workspace: device, >=
+ * kvp_decode_workspace_bytes(...) bytes, 256-byte aligned, contents ignored.
+ * Supported: head_dim 64 or 128; block_size 8, 16 or 32; num_q_heads a
+ * multiple of num_kv_heads. Grouped-query batches (num_q_heads >
+ * num_kv_heads, group <= 16) run on the tensor cores and need head_dim 128
+ * and block_size 16 or 32; one query head per KV head runs on the CUDA cores.
+ * Accumulation is fp32; out is rounded to nearest even.
+ * Errors: KVP_ERR_INVALID (unsupported geometry, misaligned pointers,
+ * workspace too small), KVP_ERR_CUDA (launch failure). */
+KVP_API int paged_attention_decode(const void* q, const void* k_cache, const void* v_cache,
+                           const int32_t* block_tables, const int32_t* context_lens,
+                           int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
+                           int32_t head_dim, int32_t block_size, int32_t num_blocks,
+                           int32_t max_blocks_per_seq, int32_t max_context_len, float scale,
+                           int32_t partition_size, void* workspace, size_t workspace_bytes,
+                           void* out, int32_t dtype, kvp_stream_t stream);
+
+/* Synchronises `stream`, then reads and clears the device error word of the
+ * current device: KVP_OK, or KVP_ERR_BOUNDS if a kernel skipped an
+ * out-of-range index since the last check (the message names the first). */
+KVP_API int kvp_check_device_error(kvp_stream_t stream);
+
+/* Description of the calling thread's last failure ("" if none). */
+KVP_API const char* kvp_last_error_message(void);
+
+/* Library version string. */
+KVP_API const char* kvp_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVP_H_ */

@@ -1,0 +1,280 @@
+"""Paged KV cache and decode attention for NVIDIA B200 (sm_100a).
+
+Python binding of libkvp (C ABI in ``include/kvp.h``). This module only
+marshals arguments: every step of the path - block bookkeeping, cache
+writes, copy-on-write copies, attention - runs in the native library. There
+is no Python or CPU fallback; calls fail loudly if ``libkvp.so`` is missing.
+
+Host side: :class:`BlockPool` (fixed-size physical blocks, per-sequence block
+tables, allocation on growth, fork with refcounted copy-on-write, release).
+Device side (torch CUDA tensors, the current torch stream):
+:func:`reshape_and_cache`, :func:`copy_blocks`, :func:`paged_attention_decode`.
+"""
+
+from __future__ import annotations
+
+import ctypes as C
+
+import numpy as np
+
+from ._lib import (KVP_BF16, KVP_F16, KvpError, P_i32, P_i64, PoolStats, check, lib)
+
+__all__ = [
+    "BlockPool", "KvpError", "reshape_and_cache", "copy_blocks", "paged_attention_decode",
+    "decode_workspace_bytes", "check_device_error", "kv_bytes_per_token", "version",
+    "KVP_F16", "KVP_BF16",
+]
+
+_DTYPES = {"f16": KVP_F16, "bf16": KVP_BF16}
+
+
+def version() -> str:
+    return lib().kvp_version().decode()
+
+
+def kv_bytes_per_token(hidden: int, layers: int, elem_bytes: int) -> int:
+    return int(lib().kvp_kv_bytes_per_token(hidden, layers, elem_bytes))
+
+
+def _i32p(a: np.ndarray):
+    return a.ctypes.data_as(P_i32)
+
+
+def _i64p(a: np.ndarray):
+    return a.ctypes.data_as(P_i64)
+
+
+class BlockPool:
+    """Host-side block allocator of one KV pool (wraps ``kv_pool_*`` / ``kv_seq_*``)."""
+
+    def __init__(self, num_blocks: int, block_size: int, num_kv_heads: int, head_dim: int,
+                 dtype: str = "f16", free_order=None):
+        self.num_blocks = int(num_blocks)
+        self.block_size = int(block_size)
+        self._h = C.c_void_p()
+        order = None
+        if free_order is not None:
+            order = np.ascontiguousarray(np.asarray(free_order, dtype=np.int32))
+            if order.shape != (self.num_blocks,):
+                raise ValueError("free_order must have num_blocks entries")
+        check(lib().kv_pool_create(num_blocks, block_size, num_kv_heads, head_dim, _DTYPES[dtype],
+                                   _i32p(order) if order is not None else None, C.byref(self._h)))
+
+    def close(self):
+        if self._h:
+            lib().kv_pool_destroy(self._h)
+            self._h = C.c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    # ---- sequences ----------------------------------------------------------
+    def create(self) -> int:
+        sid = C.c_int64()
+        check(lib().kv_seq_create(self._h, C.byref(sid)))
+        return sid.value
+
+    def append(self, seq: int, n: int) -> list[int]:
+        out = np.empty(max(int(n), 0), dtype=np.int64)
+        check(lib().kv_seq_append(self._h, seq, int(n), _i64p(out) if n > 0 else None))
+        return out.tolist()
+
+    def append_batch(self, seqs, n_each: int = 1, out: np.ndarray | None = None) -> np.ndarray:
+        s = np.ascontiguousarray(np.asarray(seqs, dtype=np.int64))
+        if out is None:
+            out = np.empty(len(s) * n_each, dtype=np.int64)
+        check(lib().kv_seq_append_batch(self._h, _i64p(s), len(s), int(n_each), _i64p(out)))
+        return out
+
+    def fork(self, parent: int) -> int:
+        cid = C.c_int64()
+        check(lib().kv_seq_fork(self._h, parent, C.byref(cid)))
+        return cid.value
+
+    def release(self, seq: int) -> None:
+        check(lib().kv_seq_release(self._h, seq))
+
+    def seq_len(self, seq: int) -> int:
+        n = C.c_int32()
+        check(lib().kv_seq_len(self._h, seq, C.byref(n)))
+        return n.value
+
+    def block_table(self, seq: int) -> list[int]:
+        n = C.c_int32()
+        rc = lib().kv_seq_block_table(self._h, seq, None, 0, C.byref(n))
+        if rc not in (0, -6):
+            check(rc)
+        out = np.empty(n.value, dtype=np.int32)
+        check(lib().kv_seq_block_table(self._h, seq, _i32p(out), n.value, C.byref(n)))
+        return out.tolist()
+
+    # ---- pool ---------------------------------------------------------------------
+    def num_free(self) -> int:
+        n = C.c_int32()
+        check(lib().kv_pool_num_free(self._h, C.byref(n)))
+        return n.value
+
+    def free_list(self) -> list[int]:
+        out = np.empty(self.num_blocks, dtype=np.int32)
+        n = C.c_int32()
+        check(lib().kv_pool_free_list(self._h, _i32p(out), self.num_blocks, C.byref(n)))
+        return out[:n.value].tolist()
+
+    def refcount(self, block: int) -> int:
+        r = C.c_int32()
+        check(lib().kv_pool_refcount(self._h, block, C.byref(r)))
+        return r.value
+
+    def refcounts(self) -> list[int]:
+        out = np.empty(self.num_blocks, dtype=np.int32)
+        check(lib().kv_pool_refcounts(self._h, _i32p(out), self.num_blocks))
+        return out.tolist()
+
+    def stats(self) -> dict:
+        s = PoolStats()
+        check(lib().kv_pool_stats(self._h, C.byref(s)))
+        return {f: getattr(s, f) for f, _ in PoolStats._fields_}
+
+    def _pairs(self, fn) -> list[tuple[int, int]]:
+        n = C.c_int32()
+        rc = fn(self._h, None, 0, C.byref(n))
+        if rc not in (0, -6):
+            check(rc)
+        buf = np.empty(2 * max(n.value, 1), dtype=np.int32)
+        check(fn(self._h, _i32p(buf), n.value, C.byref(n)))
+        return [(int(buf[2 * i]), int(buf[2 * i + 1])) for i in range(n.value)]
+
+    def take_copies(self) -> list[tuple[int, int]]:
+        return self._pairs(lib().kv_pool_take_copies)
+
+    def pending_copies(self) -> list[tuple[int, int]]:
+        return self._pairs(lib().kv_pool_pending_copies)
+
+    def build_batch(self, seqs, max_blocks: int, tables: np.ndarray | None = None,
+                    lens: np.ndarray | None = None):
+        """Block tables ``int32 [n, max_blocks]`` (padded with -1) and lengths ``int32 [n]``."""
+        s = np.ascontiguousarray(np.asarray(seqs, dtype=np.int64))
+        if tables is None:
+            tables = np.empty((len(s), max_blocks), dtype=np.int32)
+        if lens is None:
+            lens = np.empty(len(s), dtype=np.int32)
+        check(lib().kv_build_batch(self._h, _i64p(s), len(s), int(max_blocks), _i32p(tables),
+                                   _i32p(lens)))
+        return tables, lens
+
+
+# ---- device operations (torch tensors on a CUDA device) -------------------------------
+def _torch():
+    import torch
+
+    return torch
+
+
+def _code(t) -> int:
+    torch = _torch()
+    if t.dtype == torch.float16:
+        return KVP_F16
+    if t.dtype == torch.bfloat16:
+        return KVP_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _cuda(*ts):
+    dev = ts[0].device
+    for t in ts:
+        if not t.is_cuda or t.device != dev:
+            raise ValueError("all tensors must be on the same CUDA device")
+        if not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+    return dev
+
+
+def _stream(dev) -> C.c_void_p:
+    return C.c_void_p(_torch().cuda.current_stream(dev).cuda_stream)
+
+
+def reshape_and_cache(k_new, v_new, k_cache, v_cache, slot_mapping) -> None:
+    """Writes ``k_new/v_new [T, Hkv, D]`` into ``k_cache/v_cache [NB, Hkv, bs, D]`` at ``slot_mapping [T]``."""
+    torch = _torch()
+    dev = _cuda(k_new, v_new, k_cache, v_cache, slot_mapping)
+    if slot_mapping.dtype != torch.int64:
+        raise TypeError("slot_mapping must be int64")
+    T, Hkv, D = k_new.shape
+    NB, Hkv2, bs, D2 = k_cache.shape
+    if (Hkv, D) != (Hkv2, D2) or v_new.shape != k_new.shape or v_cache.shape != k_cache.shape:
+        raise ValueError("shape mismatch")
+    if not (k_new.dtype == v_new.dtype == k_cache.dtype == v_cache.dtype):
+        raise TypeError("dtype mismatch")
+    check(lib().reshape_and_cache(k_new.data_ptr(), v_new.data_ptr(), k_cache.data_ptr(),
+                                  v_cache.data_ptr(), slot_mapping.data_ptr(), T, Hkv, D, bs, NB,
+                                  _code(k_cache), _stream(dev)))
+
+
+def copy_blocks(k_cache, v_cache, pairs) -> None:
+    """Copy-on-write block copies; ``pairs`` is a CUDA ``int32 [n, 2]`` of (src, dst)."""
+    torch = _torch()
+    dev = _cuda(k_cache, v_cache, pairs)
+    if pairs.dtype != torch.int32 or pairs.dim() != 2 or pairs.shape[1] != 2:
+        raise TypeError("pairs must be int32 [n, 2]")
+    NB = k_cache.shape[0]
+    elems = k_cache[0].numel()
+    check(lib().copy_blocks(k_cache.data_ptr(), v_cache.data_ptr(), pairs.data_ptr(),
+                            pairs.shape[0], NB, elems, _code(k_cache), _stream(dev)))
+
+
+def decode_workspace_bytes(num_seqs: int, num_q_heads: int, head_dim: int, max_context_len: int,
+                           partition_size: int) -> int:
+    return int(lib().kvp_decode_workspace_bytes(num_seqs, num_q_heads, head_dim, max_context_len,
+                                                partition_size))
+
+
+def paged_attention_decode(q, k_cache, v_cache, block_tables, context_lens, scale: float,
+                           out=None, *, max_context_len: int | None = None,
+                           partition_size: int = 0, workspace=None):
+    """Decode attention over the paged cache; returns ``out [S, Hq, D]`` (dtype of q).
+
+    ``max_context_len`` bounds every ``context_lens`` entry (default: the
+    block-table capacity); ``partition_size > 0`` selects the split-context
+    kernel pair. A workspace is allocated with torch when needed and none is given.
+    """
+    torch = _torch()
+    dev = _cuda(q, k_cache, v_cache, block_tables, context_lens)
+    if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32:
+        raise TypeError("block_tables and context_lens must be int32")
+    S, Hq, D = q.shape
+    NB, Hkv, bs, D2 = k_cache.shape
+    if D2 != D or v_cache.shape != k_cache.shape or q.dtype != k_cache.dtype:
+        raise ValueError("q / cache mismatch")
+    MB = block_tables.shape[1] if block_tables.dim() == 2 else 0
+    if block_tables.shape[0] != S or context_lens.shape != (S,):
+        raise ValueError("batch metadata mismatch")
+    mcl = MB * bs if max_context_len is None else int(max_context_len)
+    if out is None:
+        out = torch.empty_like(q)
+    else:
+        _cuda(out)
+        if out.shape != q.shape or out.dtype != q.dtype:
+            raise ValueError("out mismatch")
+    need = decode_workspace_bytes(S, Hq, D, mcl, partition_size)
+    ws_ptr, ws_bytes = None, 0
+    if need:
+        if workspace is None:
+            workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+        _cuda(workspace)
+        ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()
+    check(lib().paged_attention_decode(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
+                                       block_tables.data_ptr(), context_lens.data_ptr(), S, Hq,
+                                       Hkv, D, bs, NB, max(MB, 1), mcl, float(scale),
+                                       int(partition_size), ws_ptr, ws_bytes, out.data_ptr(),
+                                       _code(q), _stream(dev)))
+    return out
+
+
+def check_device_error(device=None) -> None:
+    """Synchronises the current stream and raises if a kernel recorded an out-of-range index."""
+    torch = _torch()
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    check(lib().kvp_check_device_error(_stream(dev)))

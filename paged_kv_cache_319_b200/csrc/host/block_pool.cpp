@@ -1,0 +1,364 @@
+// Host-side paged KV block pool: free list, per-sequence block tables,
+// reference counts, copy-on-write queue.
+//
+// Method: fixed-size blocks taken only when a sequence grows into them, a
+// block table per sequence ["Your GPU was mostly empty", section "The OS
+// already solved this in the 1960s"; "vLLM and PagedAttention", section
+// "Architecture, step by step", steps 1-2]; sharing by reference count with a
+// copy only when a sequence writes into a shared block ["Your GPU was mostly
+// empty", section "Paging's second gift: copy-on-write"]; blocks no sequence
+// references go back to the shared pool ["PagedAttention: KV cache memory
+// management", section "A request lifecycle: allocation, growth, sharing and
+// release"].
+//
+// Policy (the pages leave it open; fixed here so placement is reproducible):
+// the free list is a LIFO stack seeded with the caller's order (first pop =
+// free_order[0]); release walks a table in logical order and pushes blocks
+// that reach zero; copy-on-write fires only on a write into a partly filled
+// last block whose count is > 1, and the writer gets the new block.
+//
+// Every mutating call first checks that it can succeed (block need vs free
+// count, ids), then mutates, so a failed call changes nothing.
+
+#include <cstdint>
+#include <cstring>
+#include <new>
+#include <unordered_map>
+#include <utility>
+#include <vector>
+
+#include "../status.h"
+
+struct kvp_pool {
+  int32_t num_blocks = 0;
+  int32_t block_size = 0;
+  int32_t num_kv_heads = 0;
+  int32_t head_dim = 0;
+  int32_t dtype = 0;
+  std::vector<int32_t> free_stack;  // back() is the next block handed out
+  std::vector<int32_t> rc;
+  struct Seq {
+    std::vector<int32_t> table;
+    int32_t len = 0;
+  };
+  std::unordered_map<int64_t, Seq> seqs;
+  std::vector<std::pair<int32_t, int32_t>> pending;  // (src, dst) copy-on-write pairs
+  int64_t next_seq = 0;
+  int64_t cow_total = 0;
+
+  Seq* find(int64_t id) {
+    auto it = seqs.find(id);
+    return it == seqs.end() ? nullptr : &it->second;
+  }
+  const Seq* find(int64_t id) const {
+    auto it = seqs.find(id);
+    return it == seqs.end() ? nullptr : &it->second;
+  }
+
+  static int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+  // Blocks an append of n tokens to s takes, given the last block's count.
+  int64_t need_for(const Seq& s, int32_t n, int32_t last_rc) const {
+    int64_t need = ceil_div(int64_t(s.len) + n, block_size) - ceil_div(s.len, block_size);
+    if (n > 0 && s.len % block_size != 0 && last_rc > 1) need += 1;
+    return need;
+  }
+
+  // Appends n tokens; the caller has checked that the free list suffices.
+  void append_unchecked(Seq& s, int32_t n, int64_t* slots) {
+    for (int32_t i = 0; i < n; ++i) {
+      const int32_t pos = s.len;
+      if (pos % block_size == 0) {
+        const int32_t b = free_stack.back();
+        free_stack.pop_back();
+        rc[b] = 1;
+        s.table.push_back(b);
+      } else if (rc[s.table.back()] > 1) {
+        const int32_t src = s.table.back();
+        const int32_t dst = free_stack.back();
+        free_stack.pop_back();
+        pending.emplace_back(src, dst);
+        ++cow_total;
+        rc[src] -= 1;
+        rc[dst] = 1;
+        s.table.back() = dst;
+      }
+      slots[i] = int64_t(s.table[pos / block_size]) * block_size + pos % block_size;
+      s.len = pos + 1;
+    }
+  }
+};
+
+namespace kvp {
+std::string& last_error() {
+  static thread_local std::string msg;
+  return msg;
+}
+}  // namespace kvp
+
+using kvp::fail;
+
+extern "C" {
+
+const char* kvp_last_error_message(void) { return kvp::last_error().c_str(); }
+
+const char* kvp_version(void) { return "libkvp 0.1.0 (sm_100a)"; }
+
+int64_t kvp_kv_bytes_per_token(int64_t hidden, int64_t layers, int64_t elem_bytes) {
+  return 2 * hidden * layers * elem_bytes;
+}
+
+int kv_pool_create(int32_t num_blocks, int32_t block_size, int32_t num_kv_heads,
+                   int32_t head_dim, int32_t dtype, const int32_t* free_order, kvp_pool** out) {
+  if (!out) return fail(KVP_ERR_INVALID, "kv_pool_create: out is NULL");
+  if (num_blocks <= 0 || block_size <= 0 || num_kv_heads <= 0 || head_dim <= 0)
+    return fail(KVP_ERR_INVALID, "kv_pool_create: sizes must be positive");
+  if (dtype != KVP_F16 && dtype != KVP_BF16)
+    return fail(KVP_ERR_INVALID, "kv_pool_create: dtype must be KVP_F16 or KVP_BF16");
+  if (int64_t(num_blocks) * block_size > (int64_t(1) << 40))
+    return fail(KVP_ERR_INVALID, "kv_pool_create: pool too large");
+  kvp_pool* p = new (std::nothrow) kvp_pool();
+  if (!p) return fail(KVP_ERR_OOM, "kv_pool_create: host allocation failed");
+  try {
+    p->num_blocks = num_blocks;
+    p->block_size = block_size;
+    p->num_kv_heads = num_kv_heads;
+    p->head_dim = head_dim;
+    p->dtype = dtype;
+    p->rc.assign(num_blocks, 0);
+    p->free_stack.resize(num_blocks);
+    if (free_order) {
+      std::vector<char> seen(num_blocks, 0);
+      for (int32_t i = 0; i < num_blocks; ++i) {
+        const int32_t b = free_order[i];
+        if (b < 0 || b >= num_blocks || seen[b]) {
+          delete p;
+          return fail(KVP_ERR_INVALID, "kv_pool_create: free_order is not a permutation");
+        }
+        seen[b] = 1;
+      }
+    }
+    for (int32_t i = 0; i < num_blocks; ++i)
+      p->free_stack[num_blocks - 1 - i] = free_order ? free_order[i] : i;
+  } catch (...) {
+    delete p;
+    return fail(KVP_ERR_OOM, "kv_pool_create: host allocation failed");
+  }
+  *out = p;
+  return KVP_OK;
+}
+
+int kv_pool_destroy(kvp_pool* pool) {
+  delete pool;
+  return KVP_OK;
+}
+
+int kv_pool_num_free(const kvp_pool* pool, int32_t* n) {
+  if (!pool || !n) return fail(KVP_ERR_INVALID, "kv_pool_num_free: NULL argument");
+  *n = int32_t(pool->free_stack.size());
+  return KVP_OK;
+}
+
+int kv_pool_free_list(const kvp_pool* pool, int32_t* out, int32_t cap, int32_t* n) {
+  if (!pool || !n) return fail(KVP_ERR_INVALID, "kv_pool_free_list: NULL argument");
+  const int32_t cnt = int32_t(pool->free_stack.size());
+  *n = cnt;
+  if (cap < cnt || (cnt && !out)) return fail(KVP_ERR_CAPACITY, "kv_pool_free_list: cap %d < %d", cap, cnt);
+  for (int32_t i = 0; i < cnt; ++i) out[i] = pool->free_stack[cnt - 1 - i];
+  return KVP_OK;
+}
+
+int kv_pool_refcount(const kvp_pool* pool, int32_t block, int32_t* rc) {
+  if (!pool || !rc) return fail(KVP_ERR_INVALID, "kv_pool_refcount: NULL argument");
+  if (block < 0 || block >= pool->num_blocks)
+    return fail(KVP_ERR_INVALID, "kv_pool_refcount: block %d out of range", block);
+  *rc = pool->rc[block];
+  return KVP_OK;
+}
+
+int kv_pool_refcounts(const kvp_pool* pool, int32_t* out, int32_t cap) {
+  if (!pool || !out) return fail(KVP_ERR_INVALID, "kv_pool_refcounts: NULL argument");
+  if (cap < pool->num_blocks) return fail(KVP_ERR_CAPACITY, "kv_pool_refcounts: cap too small");
+  std::memcpy(out, pool->rc.data(), sizeof(int32_t) * pool->num_blocks);
+  return KVP_OK;
+}
+
+int kv_pool_stats(const kvp_pool* pool, kvp_pool_stats* out) {
+  if (!pool || !out) return fail(KVP_ERR_INVALID, "kv_pool_stats: NULL argument");
+  kvp_pool_stats s{};
+  s.num_blocks = pool->num_blocks;
+  s.num_free = int64_t(pool->free_stack.size());
+  for (int32_t c : pool->rc) {
+    s.num_used += c > 0;
+    s.num_shared += c > 1;
+  }
+  for (const auto& kv : pool->seqs)
+    s.waste_slots += int64_t(kv.second.table.size()) * pool->block_size - kv.second.len;
+  s.cow_copies_total = pool->cow_total;
+  s.num_seqs = int64_t(pool->seqs.size());
+  *out = s;
+  return KVP_OK;
+}
+
+int kv_seq_create(kvp_pool* pool, int64_t* seq_id) {
+  if (!pool || !seq_id) return fail(KVP_ERR_INVALID, "kv_seq_create: NULL argument");
+  try {
+    pool->seqs.emplace(pool->next_seq, kvp_pool::Seq{});
+  } catch (...) {
+    return fail(KVP_ERR_OOM, "kv_seq_create: host allocation failed");
+  }
+  *seq_id = pool->next_seq++;
+  return KVP_OK;
+}
+
+int kv_seq_append(kvp_pool* pool, int64_t seq, int32_t n_tokens, int64_t* slots_out) {
+  if (!pool) return fail(KVP_ERR_INVALID, "kv_seq_append: NULL pool");
+  kvp_pool::Seq* s = pool->find(seq);
+  if (!s) return fail(KVP_ERR_NO_SEQ, "kv_seq_append: no live sequence %lld", (long long)seq);
+  if (n_tokens < 0) return fail(KVP_ERR_INVALID, "kv_seq_append: n_tokens < 0");
+  if (n_tokens > 0 && !slots_out) return fail(KVP_ERR_INVALID, "kv_seq_append: slots_out is NULL");
+  if (int64_t(s->len) + n_tokens > INT32_MAX) return fail(KVP_ERR_INVALID, "kv_seq_append: length overflow");
+  const int32_t last_rc = s->table.empty() ? 0 : pool->rc[s->table.back()];
+  const int64_t need = pool->need_for(*s, n_tokens, last_rc);
+  if (need > int64_t(pool->free_stack.size()))
+    return fail(KVP_ERR_OOM, "kv_seq_append: need %lld blocks, %zu free", (long long)need,
+                pool->free_stack.size());
+  try {
+    s->table.reserve(s->table.size() + size_t(need));
+    pool->pending.reserve(pool->pending.size() + 1);
+  } catch (...) {
+    return fail(KVP_ERR_OOM, "kv_seq_append: host allocation failed");
+  }
+  pool->append_unchecked(*s, n_tokens, slots_out);
+  return KVP_OK;
+}
+
+int kv_seq_append_batch(kvp_pool* pool, const int64_t* seqs, int32_t num_seqs, int32_t n_each,
+                        int64_t* slots_out) {
+  if (!pool) return fail(KVP_ERR_INVALID, "kv_seq_append_batch: NULL pool");
+  if (num_seqs < 0 || n_each < 0) return fail(KVP_ERR_INVALID, "kv_seq_append_batch: negative size");
+  if (num_seqs == 0 || n_each == 0) return KVP_OK;
+  if (!seqs || !slots_out) return fail(KVP_ERR_INVALID, "kv_seq_append_batch: NULL argument");
+  // Exact block need of the whole batch: a copy-on-write by an earlier
+  // sequence lowers the count a later sharer of the same last block sees.
+  std::unordered_map<int32_t, int32_t> rc_after;
+  std::vector<kvp_pool::Seq*> ptrs(num_seqs);
+  int64_t need = 0;
+  for (int32_t i = 0; i < num_seqs; ++i) {
+    kvp_pool::Seq* s = pool->find(seqs[i]);
+    if (!s) return fail(KVP_ERR_NO_SEQ, "kv_seq_append_batch: no live sequence %lld", (long long)seqs[i]);
+    for (int32_t j = 0; j < i; ++j)
+      if (ptrs[j] == s) return fail(KVP_ERR_INVALID, "kv_seq_append_batch: duplicate sequence");
+    ptrs[i] = s;
+    if (int64_t(s->len) + n_each > INT32_MAX) return fail(KVP_ERR_INVALID, "kv_seq_append_batch: overflow");
+    int32_t last_rc = 0;
+    if (!s->table.empty()) {
+      const int32_t last = s->table.back();
+      auto it = rc_after.find(last);
+      last_rc = it == rc_after.end() ? pool->rc[last] : it->second;
+      if (s->len % pool->block_size != 0 && last_rc > 1) rc_after[last] = last_rc - 1;
+    }
+    need += pool->need_for(*s, n_each, last_rc);
+  }
+  if (need > int64_t(pool->free_stack.size()))
+    return fail(KVP_ERR_OOM, "kv_seq_append_batch: need %lld blocks, %zu free", (long long)need,
+                pool->free_stack.size());
+  for (int32_t i = 0; i < num_seqs; ++i)
+    pool->append_unchecked(*ptrs[i], n_each, slots_out + int64_t(i) * n_each);
+  return KVP_OK;
+}
+
+int kv_seq_fork(kvp_pool* pool, int64_t parent, int64_t* child) {
+  if (!pool || !child) return fail(KVP_ERR_INVALID, "kv_seq_fork: NULL argument");
+  const kvp_pool::Seq* p = pool->find(parent);
+  if (!p) return fail(KVP_ERR_NO_SEQ, "kv_seq_fork: no live sequence %lld", (long long)parent);
+  try {
+    kvp_pool::Seq c = *p;
+    pool->seqs.emplace(pool->next_seq, std::move(c));
+  } catch (...) {
+    return fail(KVP_ERR_OOM, "kv_seq_fork: host allocation failed");
+  }
+  for (int32_t b : pool->seqs[pool->next_seq].table) pool->rc[b] += 1;
+  *child = pool->next_seq++;
+  return KVP_OK;
+}
+
+int kv_seq_release(kvp_pool* pool, int64_t seq) {
+  if (!pool) return fail(KVP_ERR_INVALID, "kv_seq_release: NULL pool");
+  auto it = pool->seqs.find(seq);
+  if (it == pool->seqs.end()) return fail(KVP_ERR_NO_SEQ, "kv_seq_release: no live sequence %lld", (long long)seq);
+  for (int32_t b : it->second.table) {
+    if (--pool->rc[b] == 0) pool->free_stack.push_back(b);
+  }
+  pool->seqs.erase(it);
+  return KVP_OK;
+}
+
+int kv_seq_len(const kvp_pool* pool, int64_t seq, int32_t* len) {
+  if (!pool || !len) return fail(KVP_ERR_INVALID, "kv_seq_len: NULL argument");
+  const kvp_pool::Seq* s = pool->find(seq);
+  if (!s) return fail(KVP_ERR_NO_SEQ, "kv_seq_len: no live sequence %lld", (long long)seq);
+  *len = s->len;
+  return KVP_OK;
+}
+
+int kv_seq_block_table(const kvp_pool* pool, int64_t seq, int32_t* out, int32_t cap, int32_t* n) {
+  if (!pool || !n) return fail(KVP_ERR_INVALID, "kv_seq_block_table: NULL argument");
+  const kvp_pool::Seq* s = pool->find(seq);
+  if (!s) return fail(KVP_ERR_NO_SEQ, "kv_seq_block_table: no live sequence %lld", (long long)seq);
+  const int32_t cnt = int32_t(s->table.size());
+  *n = cnt;
+  if (cap < cnt || (cnt && !out)) return fail(KVP_ERR_CAPACITY, "kv_seq_block_table: cap %d < %d", cap, cnt);
+  if (cnt) std::memcpy(out, s->table.data(), sizeof(int32_t) * cnt);
+  return KVP_OK;
+}
+
+static int copy_pairs_out(const kvp_pool* pool, int32_t* pairs, int32_t cap, int32_t* n,
+                          const char* who) {
+  if (!pool || !n) return fail(KVP_ERR_INVALID, "%s: NULL argument", who);
+  const int32_t cnt = int32_t(pool->pending.size());
+  *n = cnt;
+  if (cap < cnt || (cnt && !pairs)) return fail(KVP_ERR_CAPACITY, "%s: cap %d < %d", who, cap, cnt);
+  for (int32_t i = 0; i < cnt; ++i) {
+    pairs[2 * i] = pool->pending[i].first;
+    pairs[2 * i + 1] = pool->pending[i].second;
+  }
+  return KVP_OK;
+}
+
+int kv_pool_take_copies(kvp_pool* pool, int32_t* pairs, int32_t cap, int32_t* n) {
+  const int rc = copy_pairs_out(pool, pairs, cap, n, "kv_pool_take_copies");
+  if (rc == KVP_OK) pool->pending.clear();
+  return rc;
+}
+
+int kv_pool_pending_copies(const kvp_pool* pool, int32_t* pairs, int32_t cap, int32_t* n) {
+  return copy_pairs_out(pool, pairs, cap, n, "kv_pool_pending_copies");
+}
+
+int kv_build_batch(const kvp_pool* pool, const int64_t* seqs, int32_t num_seqs, int32_t max_blocks,
+                   int32_t* block_tables, int32_t* context_lens) {
+  if (!pool) return fail(KVP_ERR_INVALID, "kv_build_batch: NULL pool");
+  if (num_seqs < 0 || max_blocks < 0) return fail(KVP_ERR_INVALID, "kv_build_batch: negative size");
+  if (num_seqs == 0) return KVP_OK;
+  if (!seqs || !context_lens || (max_blocks && !block_tables))
+    return fail(KVP_ERR_INVALID, "kv_build_batch: NULL argument");
+  for (int32_t i = 0; i < num_seqs; ++i) {
+    const kvp_pool::Seq* s = pool->find(seqs[i]);
+    if (!s) return fail(KVP_ERR_NO_SEQ, "kv_build_batch: no live sequence %lld", (long long)seqs[i]);
+    if (int32_t(s->table.size()) > max_blocks)
+      return fail(KVP_ERR_CAPACITY, "kv_build_batch: table of %lld has %zu > %d blocks",
+                  (long long)seqs[i], s->table.size(), max_blocks);
+  }
+  for (int32_t i = 0; i < num_seqs; ++i) {
+    const kvp_pool::Seq* s = pool->find(seqs[i]);
+    int32_t* row = block_tables + int64_t(i) * max_blocks;
+    const int32_t cnt = int32_t(s->table.size());
+    if (cnt) std::memcpy(row, s->table.data(), sizeof(int32_t) * cnt);
+    for (int32_t j = cnt; j < max_blocks; ++j) row[j] = -1;
+    context_lens[i] = s->len;
+  }
+  return KVP_OK;
+}
+
+}  // extern "C"

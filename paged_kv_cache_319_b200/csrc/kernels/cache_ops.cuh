@@ -1,0 +1,73 @@
+// reshape_and_cache and copy_blocks: the two writes into the paged KV pool.
+//
+// Both are pure data movement, bound by HBM bandwidth. Every thread moves
+// 16-byte vectors; a warp covers contiguous 512-byte spans, so loads and
+// stores are fully coalesced. Out-of-range indices are skipped and recorded.
+#pragma once
+
+#include "common.cuh"
+
+namespace kvp {
+namespace dev {
+
+// New tokens' K and V rows go to their slots: decode appends new cache state
+// ["PagedAttention: KV cache memory management", section "A request
+// lifecycle: allocation, growth, sharing and release"].
+// k_new/v_new: [T][Hkv][D]; cache: [NB][Hkv][bs][D]. Thread-iteration c moves
+// the 16-byte chunk j = c % cpr of row (t, h) = c / cpr, where cpr = D / 8
+// chunks per row; cpr and block_size are powers of two (shifts), and the
+// host guarantees T * Hkv * cpr < 2^31.
+__global__ void __launch_bounds__(256) reshape_and_cache_kernel(
+    const uint4* __restrict__ k_new, const uint4* __restrict__ v_new, uint4* __restrict__ k_cache,
+    uint4* __restrict__ v_cache, const int64_t* __restrict__ slot_mapping, uint32_t num_chunks,
+    uint32_t num_kv_heads, uint32_t log2_cpr, uint32_t log2_bs, int64_t num_slots) {
+  const uint32_t stride = gridDim.x * blockDim.x;
+  const uint32_t cpr_mask = (1u << log2_cpr) - 1u;
+  for (uint32_t c = blockIdx.x * blockDim.x + threadIdx.x; c < num_chunks; c += stride) {
+    const uint32_t row = c >> log2_cpr;
+    const uint32_t j = c & cpr_mask;
+    const uint32_t t = row / num_kv_heads;
+    const uint32_t h = row - t * num_kv_heads;
+    const int64_t s = __ldg(slot_mapping + t);
+    if (s < 0) continue;  // padding token
+    if (s >= num_slots) {
+      if (h == 0 && j == 0) record_error(KVP_DEVERR_SLOT, uint64_t(t));
+      continue;
+    }
+    const int64_t blk = s >> log2_bs;
+    const int64_t off = s & ((int64_t(1) << log2_bs) - 1);
+    const int64_t dst = (((blk * num_kv_heads + h) << log2_bs) + off) * (int64_t(1) << log2_cpr) + j;
+    const uint4 kv = __ldg(k_new + c);
+    const uint4 vv = __ldg(v_new + c);
+    k_cache[dst] = kv;
+    v_cache[dst] = vv;
+  }
+}
+
+// Block-level copy-on-write: block dst of K and V becomes a copy of block src
+// ["Your GPU was mostly empty", section "Paging's second gift: copy-on-write"].
+// grid.y = pair, grid.z = 0 (K) / 1 (V); grid.x strides over the block's chunks.
+__global__ void __launch_bounds__(256) copy_blocks_kernel(uint4* __restrict__ k_cache,
+                                                          uint4* __restrict__ v_cache,
+                                                          const int32_t* __restrict__ pairs,
+                                                          int64_t chunks_per_block,
+                                                          int32_t num_blocks) {
+  const int32_t i = blockIdx.y;
+  const int32_t src = __ldg(pairs + 2 * i);
+  const int32_t dst = __ldg(pairs + 2 * i + 1);
+  if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) {
+    if (blockIdx.x == 0 && blockIdx.z == 0 && threadIdx.x == 0)
+      record_error(KVP_DEVERR_PAIR, uint64_t(i));
+    return;
+  }
+  uint4* base = blockIdx.z == 0 ? k_cache : v_cache;
+  const uint4* s = base + int64_t(src) * chunks_per_block;
+  uint4* d = base + int64_t(dst) * chunks_per_block;
+  const int64_t stride = int64_t(gridDim.x) * blockDim.x;
+  for (int64_t c = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; c < chunks_per_block;
+       c += stride)
+    d[c] = s[c];
+}
+
+}  // namespace dev
+}  // namespace kvp

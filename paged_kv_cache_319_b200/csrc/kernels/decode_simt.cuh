@@ -1,0 +1,390 @@
+// Paged decode attention on the CUDA cores, one CTA per (partition, query
+// head, sequence), and the log-sum-exp merge of split partitions.
+//
+// What it computes: for sequence s and query head h (KV head g = h / G), the
+// keys and values of tokens j < ctx are found through the block table -
+// physical block block_tables[s][j / bs], slot j % bs - and the output is
+// softmax(scale * q K^T) V, the same result as over a contiguous cache ["vLLM
+// and PagedAttention", section "Architecture, step by step", step 3; "Your
+// GPU was mostly empty", section "The OS already solved this in the 1960s"].
+//
+// How: each warp of the CTA owns every NW-th block of the partition and runs
+// its own TMA pipeline of NST stages: one elected lane issues two 2-D tensor
+// loads (K tile, V tile: block_size rows x head_dim, 128-byte swizzled) per
+// block onto the stage's mbarrier. A (block, KV head) tile is one contiguous
+// block_size * head_dim run of the cache, so every load is one dense 2-4 KiB
+// burst. The warp keeps a running max m, a per-lane exponent sum and an fp32
+// accumulator (online softmax in the log2 domain, q pre-scaled by
+// scale * log2 e). QK: two lanes per key row, 16-byte swizzled reads (no
+// bank conflicts), one shuffle to join the halves; row max by a single
+// integer max-reduction. PV: each lane owns head_dim / 32 output dims and
+// broadcasts p by shuffle. At the end the warps merge through shared memory
+// and the CTA writes either the normalised output or, for split sequences,
+// (m, l, acc) to the workspace.
+#pragma once
+
+#include <math.h>
+
+#include "common.cuh"
+
+namespace kvp {
+namespace dev {
+
+struct DecodeArgs {
+  const void* q;                // [S][Hq][D]
+  void* out;                    // [S][Hq][D]
+  const int32_t* block_tables;  // [S][max_blocks_per_seq]
+  const int32_t* context_lens;  // [S]
+  float* ws_ml;                 // [S][Hq][pmax][2] = (m in log2 units, l)
+  float* ws_acc;                // [S][Hq][pmax][D], unnormalised
+  int32_t num_seqs;
+  int32_t num_q_heads;
+  int32_t num_kv_heads;
+  int32_t num_blocks;
+  int32_t max_blocks_per_seq;
+  int32_t max_context_len;
+  int32_t part_blocks;  // partition length in blocks (whole context when unsplit)
+  int32_t part_tokens;  // part_blocks * block_size
+  int32_t pmax;         // partitions per (sequence, head) in grid and workspace
+  float scale_log2;     // scale * log2(e)
+};
+
+__device__ __forceinline__ uint8_t* align_1024(uint8_t* p) {
+  const uint32_t a = smem_u32(p);
+  return p + ((1024u - (a & 1023u)) & 1023u);
+}
+
+// Clamped context length of sequence s (records out-of-range values once).
+__device__ __forceinline__ int32_t load_ctx(const DecodeArgs& a, int32_t s, bool report) {
+  int32_t ctx = __ldg(a.context_lens + s);
+  if (ctx < 0 || ctx > a.max_context_len) {
+    if (report) record_error(KVP_DEVERR_CTX, uint64_t(s));
+    ctx = ctx < 0 ? 0 : a.max_context_len;
+  }
+  return ctx;
+}
+
+template <typename T, int D, int BS, int NW, int NST>
+struct SimtCfg {
+  static constexpr int kRegions = D / 64;          // 128-byte row regions (1 or 2)
+  static constexpr int kTileBytes = BS * D * 2;    // one (block, KV head) tile
+  static constexpr int kChunksPerRow = D / 8;      // 16-byte chunks per row
+  static constexpr int kChunksPerLane = kChunksPerRow / 2;
+  static constexpr int kPasses = (BS + 15) / 16;   // 16 rows per QK pass
+  static constexpr int kDimsPerLane = D / 32;
+  static constexpr int kTileArea = NW * NST * 2 * kTileBytes;
+  static constexpr int kBarArea = NW * NST * 8;
+  static constexpr int kMergeArea = NW * (D + 2) * 4;
+  static constexpr int kSmemBytes = 1024 + kTileArea + kBarArea + kMergeArea;
+  static_assert(D == 64 || D == 128, "head_dim 64 or 128");
+  static_assert(BS == 8 || BS == 16 || BS == 32, "block_size 8, 16 or 32");
+  static_assert(NST >= 1 && NST <= 32, "stages");
+};
+
+template <typename T, int D, int BS, int NW, int NST>
+__global__ void __launch_bounds__(NW * 32) decode_simt_kernel(
+    const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
+    const DecodeArgs a) {
+  using C = SimtCfg<T, D, BS, NW, NST>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align_1024(smem_raw);
+  uint8_t* tiles = smem;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kTileArea);
+  float* mg_m = reinterpret_cast<float*>(smem + C::kTileArea + C::kBarArea);
+  float* mg_l = mg_m + NW;
+  float* mg_acc = mg_l + NW;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int p = blockIdx.x;
+  const int h = blockIdx.y;
+  const int s = blockIdx.z;
+
+  const int32_t ctx = load_ctx(a, s, p == 0 && h == 0 && threadIdx.x == 0);
+  const int32_t nblk = (ctx + BS - 1) / BS;
+  const int32_t nparts = (nblk + a.part_blocks - 1) / a.part_blocks;
+  const int32_t b0 = p * a.part_blocks;
+  if (p > 0 && b0 >= nblk) return;  // empty partition (p == 0 always writes its row)
+  const int32_t b1 = min(nblk, b0 + a.part_blocks);
+  const int32_t g = h / (a.num_q_heads / a.num_kv_heads);
+  const int32_t* table = a.block_tables + int64_t(s) * a.max_blocks_per_seq;
+
+  // Blocks of this warp: b0 + warp + NW * i, i < nw.
+  const int32_t span = b1 - b0;
+  const int32_t nw = span > warp ? (span - warp + NW - 1) / NW : 0;
+
+  uint64_t* my_bars = bars + warp * NST;
+  uint8_t* my_tiles = tiles + size_t(warp) * NST * 2 * C::kTileBytes;
+  if (lane == 0) {
+    for (int i = 0; i < NST; ++i) mbar_init(&my_bars[i], 1);
+    fence_mbar_init();
+  }
+  if (lane == 0) {
+    prefetch_tensormap(&kmap);
+    prefetch_tensormap(&vmap);
+  }
+  __syncwarp();
+
+  const uint64_t policy = l2_policy_evict_first();
+  const int32_t rows_total = a.num_blocks * a.num_kv_heads * BS;
+
+  // Register cache of 32 block ids: lane l holds id of index base + l.
+  int32_t id_base = 0;
+  int32_t my_id = -1;
+  auto load_ids = [&](int32_t base) {
+    const int32_t idx = base + lane;
+    my_id = idx < nw ? __ldg(table + b0 + warp + NW * idx) : -1;
+  };
+  load_ids(0);
+
+  auto issue = [&](int32_t i, int32_t id) {  // lane 0 only
+    const int stage = i % NST;
+    uint8_t* kt = my_tiles + size_t(stage) * 2 * C::kTileBytes;
+    uint8_t* vt = kt + C::kTileBytes;
+    int32_t row;
+    if (id < 0 || id >= a.num_blocks) {
+      record_error(KVP_DEVERR_BLOCK_ID, (uint64_t(s) << 32) | uint32_t(b0 + warp + NW * i));
+      row = rows_total;  // out of the tensor: the load fills zeros
+    } else {
+      row = (id * a.num_kv_heads + g) * BS;
+    }
+    mbar_arrive_expect_tx(&my_bars[stage], 2 * C::kTileBytes);
+#pragma unroll
+    for (int r = 0; r < C::kRegions; ++r) {
+      tma_load_2d(kt + r * BS * 128, &kmap, &my_bars[stage], r * 64, row, policy);
+      tma_load_2d(vt + r * BS * 128, &vmap, &my_bars[stage], r * 64, row, policy);
+    }
+  };
+
+  {
+    const int npro = nw < NST ? nw : NST;
+    for (int i = 0; i < npro; ++i) {
+      const int32_t id = __shfl_sync(0xffffffffu, my_id, i);
+      if (lane == 0) issue(i, id);
+    }
+  }
+
+  // q of this head, pre-scaled: lane part (lane >> 4) covers chunks
+  // [part * kChunksPerLane, (part + 1) * kChunksPerLane) of the row.
+  const int part = lane >> 4;
+  float qf[C::kChunksPerLane * 8];
+  {
+    const uint4* qrow = reinterpret_cast<const uint4*>(static_cast<const T*>(a.q) +
+                                                       (int64_t(s) * a.num_q_heads + h) * D);
+#pragma unroll
+    for (int c = 0; c < C::kChunksPerLane; ++c) {
+      const uint4 v = __ldg(qrow + part * C::kChunksPerLane + c);
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = Elem<T>::to_float2(w[e]);
+        qf[c * 8 + 2 * e] = f.x * a.scale_log2;
+        qf[c * 8 + 2 * e + 1] = f.y * a.scale_log2;
+      }
+    }
+  }
+
+  float m_run = -INFINITY;
+  float l_lane = 0.f;
+  float acc[C::kDimsPerLane];
+#pragma unroll
+  for (int e = 0; e < C::kDimsPerLane; ++e) acc[e] = 0.f;
+
+  bool aborted = false;
+  int32_t i_fail = 0;
+  for (int32_t i = 0; i < nw; ++i) {
+    const int stage = i % NST;
+    const uint32_t phase = uint32_t(i / NST) & 1u;
+    if (!__all_sync(0xffffffffu, mbar_wait(&my_bars[stage], phase, 0x5100u + stage))) {
+      aborted = true;
+      i_fail = i;
+      break;
+    }
+    const uint8_t* kt = my_tiles + size_t(stage) * 2 * C::kTileBytes;
+    const uint8_t* vt = kt + C::kTileBytes;
+    const int32_t tok0 = (b0 + warp + NW * i) * BS;
+    const int32_t nvalid = min(BS, ctx - tok0);
+
+    // ---- scores: row r = pass * 16 + (lane & 15), half `part` of its chunks
+    float sc[C::kPasses];
+#pragma unroll
+    for (int ps = 0; ps < C::kPasses; ++ps) {
+      const int r = ps * 16 + (lane & 15);
+      float d0 = 0.f, d1 = 0.f, d2 = 0.f, d3 = 0.f;
+      if (r < BS) {
+#pragma unroll
+        for (int c = 0; c < C::kChunksPerLane; ++c) {
+          const int lc = part * C::kChunksPerLane + c;
+          const int region = lc >> 3;
+          const int cc = lc & 7;
+          const uint4 kv = *reinterpret_cast<const uint4*>(kt + region * BS * 128 + r * 128 +
+                                                           ((cc ^ (r & 7)) << 4));
+          const float2 f0 = Elem<T>::to_float2(kv.x);
+          const float2 f1 = Elem<T>::to_float2(kv.y);
+          const float2 f2 = Elem<T>::to_float2(kv.z);
+          const float2 f3 = Elem<T>::to_float2(kv.w);
+          d0 = fmaf(qf[c * 8 + 0], f0.x, d0);
+          d1 = fmaf(qf[c * 8 + 1], f0.y, d1);
+          d2 = fmaf(qf[c * 8 + 2], f1.x, d2);
+          d3 = fmaf(qf[c * 8 + 3], f1.y, d3);
+          d0 = fmaf(qf[c * 8 + 4], f2.x, d0);
+          d1 = fmaf(qf[c * 8 + 5], f2.y, d1);
+          d2 = fmaf(qf[c * 8 + 6], f3.x, d2);
+          d3 = fmaf(qf[c * 8 + 7], f3.y, d3);
+        }
+      }
+      float dot = (d0 + d1) + (d2 + d3);
+      dot += __shfl_xor_sync(0xffffffffu, dot, 16);
+      sc[ps] = r < nvalid ? dot : -INFINITY;
+    }
+
+    // ---- online softmax update (log2 domain)
+    float tmax = sc[0];
+#pragma unroll
+    for (int ps = 1; ps < C::kPasses; ++ps) tmax = fmaxf(tmax, sc[ps]);
+    tmax = warp_max(tmax);
+    const float m_new = fmaxf(m_run, tmax);
+    const float alpha = m_run == -INFINITY ? 0.f : exp2f(m_run - m_new);
+    float pr[C::kPasses];
+    float psum = 0.f;
+#pragma unroll
+    for (int ps = 0; ps < C::kPasses; ++ps) {
+      pr[ps] = sc[ps] == -INFINITY ? 0.f : exp2f(sc[ps] - m_new);
+      psum += pr[ps];
+    }
+    l_lane = l_lane * alpha + (lane < 16 ? psum : 0.f);
+#pragma unroll
+    for (int e = 0; e < C::kDimsPerLane; ++e) acc[e] *= alpha;
+    m_run = m_new;
+
+    // ---- acc += p V: lane owns dims [lane * kDimsPerLane, +kDimsPerLane)
+    {
+      constexpr int DPL = C::kDimsPerLane;
+      const int d0 = lane * DPL;
+      const int region = d0 >> 6;
+      const int cc = (d0 & 63) >> 3;
+      const int pos = d0 & 7;
+#pragma unroll
+      for (int r = 0; r < BS; ++r) {
+        const float pv = __shfl_sync(0xffffffffu, pr[r >> 4], r & 15);
+        if (r < nvalid) {
+          const uint8_t* src = vt + region * BS * 128 + r * 128 + ((cc ^ (r & 7)) << 4) + pos * 2;
+          if constexpr (DPL == 4) {
+            const uint2 v = *reinterpret_cast<const uint2*>(src);
+            const float2 f0 = Elem<T>::to_float2(v.x);
+            const float2 f1 = Elem<T>::to_float2(v.y);
+            acc[0] = fmaf(pv, f0.x, acc[0]);
+            acc[1] = fmaf(pv, f0.y, acc[1]);
+            acc[2] = fmaf(pv, f1.x, acc[2]);
+            acc[3] = fmaf(pv, f1.y, acc[3]);
+          } else {
+            const uint32_t v = *reinterpret_cast<const uint32_t*>(src);
+            const float2 f0 = Elem<T>::to_float2(v);
+            acc[0] = fmaf(pv, f0.x, acc[0]);
+            acc[1] = fmaf(pv, f0.y, acc[1]);
+          }
+        }
+      }
+    }
+
+    // ---- refill this stage with block i + NST
+    const int32_t nxt = i + NST;
+    if (nxt < nw && nxt >= id_base + 32) {
+      id_base += 32;
+      load_ids(id_base);
+    }
+    const int32_t id = __shfl_sync(0xffffffffu, my_id, (nxt - id_base) & 31);
+    __syncwarp();
+    if (lane == 0 && nxt < nw) {
+      fence_proxy_async_smem();
+      issue(nxt, id);
+    }
+  }
+
+  if (aborted) {
+    // Drain this warp's loads still in flight before the CTA exits.
+    if (lane == 0) {
+      for (int32_t i = i_fail; i < nw && i < i_fail + NST; ++i)
+        mbar_wait(&my_bars[i % NST], uint32_t(i / NST) & 1u, 0x5200u);
+    }
+    m_run = -INFINITY;
+  }
+
+  // ---- merge the warps
+#pragma unroll
+  for (int o = 8; o >= 1; o >>= 1) l_lane += __shfl_xor_sync(0xffffffffu, l_lane, o);
+  if (lane == 0) {
+    mg_m[warp] = m_run;
+    mg_l[warp] = l_lane;
+  }
+#pragma unroll
+  for (int e = 0; e < C::kDimsPerLane; ++e) mg_acc[warp * D + lane * C::kDimsPerLane + e] = acc[e];
+  const int any_abort = __syncthreads_or(aborted ? 1 : 0);
+
+  const int64_t row_sh = int64_t(s) * a.num_q_heads + h;
+  float M = -INFINITY;
+#pragma unroll
+  for (int w = 0; w < NW; ++w) M = fmaxf(M, mg_m[w]);
+  float wgt[NW];
+  float L = 0.f;
+#pragma unroll
+  for (int w = 0; w < NW; ++w) {
+    wgt[w] = (mg_m[w] == -INFINITY || M == -INFINITY) ? 0.f : exp2f(mg_m[w] - M);
+    L += mg_l[w] * wgt[w];
+  }
+  for (int t = threadIdx.x; t < D; t += NW * 32) {
+    float o = 0.f;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) o = fmaf(mg_acc[w * D + t], wgt[w], o);
+    if (nparts <= 1) {
+      const float y = (L > 0.f && !any_abort) ? o / L : 0.f;
+      static_cast<uint16_t*>(a.out)[row_sh * D + t] = Elem<T>::from_float(y);
+    } else {
+      a.ws_acc[(row_sh * a.pmax + p) * D + t] = o;
+    }
+  }
+  if (nparts > 1 && threadIdx.x == 0) {
+    a.ws_ml[(row_sh * a.pmax + p) * 2 + 0] = any_abort ? -INFINITY : M;
+    a.ws_ml[(row_sh * a.pmax + p) * 2 + 1] = any_abort ? 0.f : L;
+  }
+}
+
+// Log-sum-exp merge of the partitions of split sequences: M = max_p m_p,
+// L = sum_p l_p 2^(m_p - M), out = sum_p 2^(m_p - M) acc_p / L.
+// grid (Hq, S), D threads; sequences with a single partition were written by
+// the partition kernel and are skipped.
+template <typename T, int D>
+__global__ void __launch_bounds__(D) decode_reduce_kernel(const DecodeArgs a) {
+  extern __shared__ float wsh[];  // [pmax] weights
+  const int h = blockIdx.x;
+  const int s = blockIdx.y;
+  const int32_t ctx = load_ctx(a, s, false);
+  const int32_t nparts = (ctx + a.part_tokens - 1) / a.part_tokens;
+  if (nparts <= 1) return;
+  const int64_t row_sh = int64_t(s) * a.num_q_heads + h;
+  const float* ml = a.ws_ml + row_sh * a.pmax * 2;
+  __shared__ float red[2];
+  if (threadIdx.x == 0) {
+    float M = -INFINITY;
+    for (int p = 0; p < nparts; ++p) M = fmaxf(M, ml[2 * p]);
+    float L = 0.f;
+    for (int p = 0; p < nparts; ++p) {
+      const float w = (ml[2 * p] == -INFINITY || M == -INFINITY) ? 0.f : exp2f(ml[2 * p] - M);
+      wsh[p] = w;
+      L += ml[2 * p + 1] * w;
+    }
+    red[0] = L;
+  }
+  __syncthreads();
+  const float L = red[0];
+  const float* acc = a.ws_acc + row_sh * a.pmax * D;
+  for (int t = threadIdx.x; t < D; t += blockDim.x) {
+    float o = 0.f;
+    for (int p = 0; p < nparts; ++p) o = fmaf(acc[int64_t(p) * D + t], wsh[p], o);
+    const float y = L > 0.f ? o / L : 0.f;
+    static_cast<uint16_t*>(a.out)[row_sh * D + t] = Elem<T>::from_float(y);
+  }
+}
+
+}  // namespace dev
+}  // namespace kvp

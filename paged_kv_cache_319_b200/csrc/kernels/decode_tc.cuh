@@ -1,0 +1,559 @@
+// Paged decode attention for grouped-query heads on the 5th-generation tensor
+// cores (tcgen05, accumulators in tensor memory).
+//
+// What it computes is the same as the CUDA-core kernel: for sequence s and
+// query head h with KV head g = h / G, softmax(scale * q K^T) V over the keys
+// and values found through the block table ["vLLM and PagedAttention",
+// section "Architecture, step by step", step 3]. With G query heads sharing a
+// KV head, QK^T and PV are small dense contractions, so they run as MMAs with
+// the token axis as the 128-row M dimension (operands swapped):
+//
+//   S^T [128 tokens x N] = K_tile [128 x 128 dims] . Q_g^T [128 dims x N]
+//   O^T [128 dims x N]  += V_tile^T [128 dims x 128 tokens] . P^T [128 x N]
+//
+// with N = 16 columns (the G real heads; the rest are ignored).
+//
+// Structure: a persistent CTA per SM walks its share of work units
+// (sequence, KV head, partition); a unit is cut into chunks of up to 512
+// tokens (4 M-tiles). Warp roles:
+//   warp 0  producer: 2-D TMA loads (128-byte swizzle) of Q (per unit) and of
+//           K then V tiles (per chunk) into a 5-stage ring of 32 KiB stages;
+//           a stage is 128 tokens = 128 / block_size cache blocks, each block
+//           tile landing at its rows of the stage.
+//   warp 1  MMA issuer (one thread) and tensor-memory owner: per chunk, QK^T
+//           into a double-buffered S region, then PV into a double-buffered O
+//           region; tcgen05.commit releases ring stages and signals softmax.
+//   warps 2-5  softmax and epilogue (thread = TMEM lane = token row for S,
+//           head-dim row for O): chunk max per head, p = 2^(s - m) rounded to
+//           the input type into a shared-memory P^T buffer, then the chunk's
+//           O is merged into fp32 registers by the log-sum-exp rule; the unit
+//           ends by writing the normalised output or (m, l, acc) for the
+//           split-context reduce.
+// The exponent sum l is accumulated from the same rounded p that the MMA
+// uses, so the weights stay a normalised average.
+#pragma once
+
+#include <type_traits>
+
+#include "common.cuh"
+#include "decode_simt.cuh"
+
+namespace kvp {
+namespace dev {
+
+namespace tc {
+
+constexpr int kD = 128;             // head_dim
+constexpr int kN = 16;              // MMA N (query heads of a group, padded)
+constexpr int kTileTok = 128;       // MMA M: tokens per tile
+constexpr int kChunkTiles = 4;      // tiles per chunk (512 tokens)
+constexpr int kChunkTok = kTileTok * kChunkTiles;
+constexpr int kStages = 5;
+constexpr int kStageBytes = kTileTok * kD * 2;       // 32 KiB
+constexpr int kRegionBytes = kTileTok * 128;         // 16 KiB: 64 dims of 128 tokens
+constexpr int kQBytes = kN * kD * 2;                 // 4 KiB
+constexpr int kPBytes = kChunkTok * kN * 2;          // 16 KiB
+constexpr int kTmemCols = 256;
+constexpr int kSCol = 0;                             // S buffers: [0, 128)
+constexpr int kOCol = 128;                           // O buffers: [128, 160)
+constexpr int kThreads = 192;
+constexpr int kSoftmaxThreads = 128;
+
+// Shared-memory layout (offsets from a 1024-aligned base).
+constexpr int kOffRing = 0;
+constexpr int kOffQ = kOffRing + kStages * kStageBytes;
+constexpr int kOffP = kOffQ + 2 * kQBytes;
+constexpr int kOffBar = kOffP + 2 * kPBytes;
+constexpr int kNumBars = 2 * kStages + 2 * 10;
+constexpr int kOffRed = kOffBar + kNumBars * 8;               // [2 halves][4 warps][kN] maxima
+constexpr int kOffRedL = kOffRed + 2 * 4 * kN * 4;            // [2 halves][4 warps][kN] sums
+constexpr int kOffTmemPtr = kOffRedL + 2 * 4 * kN * 4;
+constexpr int kSmemBytes = 1024 + kOffTmemPtr + 16;
+// The softmax warps wait for a chunk's last V tile (to zero rows past the end
+// of the sequence) before the PV MMAs free any stage of that chunk, so the
+// ring must hold a chunk's K tiles plus that V tile.
+static_assert(kStages >= kChunkTiles, "ring too shallow for one chunk");
+static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
+
+// tcgen05 instruction descriptor, kind::f16, fp32 accumulate, M = 128, N = 16.
+__host__ __device__ constexpr uint32_t idesc_f16(uint32_t ab_fmt, uint32_t a_mn, uint32_t b_mn) {
+  return (1u << 4) | (ab_fmt << 7) | (ab_fmt << 10) | (a_mn << 15) | (b_mn << 16) |
+         (uint32_t(kN >> 3) << 17) | (uint32_t(kTileTok >> 4) << 24);
+}
+
+// Shared-memory matrix descriptor (sm_100 format, version 1).
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo,
+                                              uint32_t layout) {
+  return uint64_t((addr & 0x3FFFFu) >> 4) | (uint64_t((lbo >> 4) & 0x3FFFu) << 16) |
+         (uint64_t((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (uint64_t(layout) << 61);
+}
+constexpr uint32_t kLayoutNone = 0;
+constexpr uint32_t kLayoutSw128 = 2;
+
+template <int NG>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, float (&v)[NG]) {
+  uint32_t r[NG];
+  if constexpr (NG == 4) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(taddr)
+                 : "memory");
+  } else if constexpr (NG == 8) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                   "=r"(r[6]), "=r"(r[7])
+                 : "r"(taddr)
+                 : "memory");
+  } else {
+    static_assert(NG == 16, "group padded to 4, 8 or 16");
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+        "%11, %12, %13, %14, %15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr)
+        : "memory");
+  }
+#pragma unroll
+  for (int j = 0; j < NG; ++j) v[j] = __uint_as_float(r[j]);
+}
+
+// Work unit u -> (s, g, p) over the grid pmax x Hkv x S (p fastest).
+struct Unit {
+  int32_t s, g, p;
+  int32_t tok_begin, tok_end;  // token range of the unit
+  int32_t ctx;
+  int32_t nparts;
+};
+
+__device__ __forceinline__ bool decode_unit(const DecodeArgs& a, int64_t u, Unit& w) {
+  const int64_t per_seq = int64_t(a.pmax) * a.num_kv_heads;
+  w.s = int32_t(u / per_seq);
+  const int32_t rem = int32_t(u - int64_t(w.s) * per_seq);
+  w.g = rem / a.pmax;
+  w.p = rem - w.g * a.pmax;
+  w.ctx = load_ctx(a, w.s, false);
+  w.nparts = (w.ctx + a.part_tokens - 1) / a.part_tokens;
+  if (w.p > 0 && w.p >= w.nparts) return false;  // empty (p == 0 always runs)
+  w.tok_begin = w.p * a.part_tokens;
+  w.tok_end = min(w.ctx, w.tok_begin + a.part_tokens);
+  if (w.tok_end < w.tok_begin) w.tok_end = w.tok_begin;
+  return true;
+}
+
+__device__ __forceinline__ int32_t chunks_of(const Unit& w) {
+  return (w.tok_end - w.tok_begin + kChunkTok - 1) / kChunkTok;
+}
+__device__ __forceinline__ int32_t tiles_of(const Unit& w, int32_t c) {
+  const int32_t c0 = w.tok_begin + c * kChunkTok;
+  const int32_t c1 = min(w.tok_end, c0 + kChunkTok);
+  return (c1 - c0 + kTileTok - 1) / kTileTok;
+}
+
+}  // namespace tc
+
+template <typename T, int BS, int NG>
+__global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
+    const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
+    const __grid_constant__ CUtensorMap qmap, const DecodeArgs a, int64_t num_units) {
+  using namespace tc;
+  static_assert(BS == 16 || BS == 32, "block_size 16 or 32");
+  constexpr int kBlocksPerTile = kTileTok / BS;
+  constexpr uint32_t kFmt = std::is_same<T, __half>::value ? 0u : 1u;
+  constexpr uint32_t kIdescQK = idesc_f16(kFmt, 0, 0);  // A = K (K-major), B = Q (K-major)
+  constexpr uint32_t kIdescPV = idesc_f16(kFmt, 1, 0);  // A = V^T (MN-major), B = P^T (K-major)
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align_1024(smem_raw);
+  uint8_t* ring = smem + kOffRing;
+  uint8_t* qbuf = smem + kOffQ;
+  uint8_t* pbuf = smem + kOffP;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
+  uint64_t* full = bars;                   // [kStages]
+  uint64_t* empty = bars + kStages;        // [kStages]
+  uint64_t* q_full = empty + kStages;      // [2]
+  uint64_t* q_empty = q_full + 2;          // [2]
+  uint64_t* s_full = q_empty + 2;          // [2]
+  uint64_t* s_free = s_full + 2;           // [2]
+  uint64_t* p_full = s_free + 2;           // [2]
+  uint64_t* p_free = p_full + 2;           // [2]
+  uint64_t* o_full = p_free + 2;           // [2]
+  uint64_t* o_free = o_full + 2;           // [2]
+  uint64_t* red_bar = o_free + 2;          // [2] chunk maxima of the 4 softmax warps
+  uint64_t* lred_bar = red_bar + 2;        // [2] unit sums of the 4 softmax warps
+  float* red = reinterpret_cast<float*>(smem + kOffRed);
+  float* redl = reinterpret_cast<float*>(smem + kOffRedL);
+  uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + kOffTmemPtr);
+  __shared__ int abort_flag;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&q_full[i], 1);
+      mbar_init(&q_empty[i], 1);
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_free[i], 4);
+      mbar_init(&p_full[i], 4);
+      mbar_init(&p_free[i], 1);
+      mbar_init(&o_full[i], 1);
+      mbar_init(&o_free[i], 4);
+      mbar_init(&red_bar[i], 4);
+      mbar_init(&lred_bar[i], 4);
+    }
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  // P^T buffers start as zeros (rows of padded heads are never written).
+  for (int i = threadIdx.x; i < 2 * kPBytes / 16; i += blockDim.x)
+    reinterpret_cast<uint4*>(pbuf)[i] = make_uint4(0, 0, 0, 0);
+  fence_proxy_async_smem();
+  if (warp == 1) {
+    tmem_alloc(tmem_ptr, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_ptr;
+
+  const int32_t G = a.num_q_heads / a.num_kv_heads;
+  const int32_t rows_total = a.num_blocks * a.num_kv_heads * BS;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      prefetch_tensormap(&kmap);
+      prefetch_tensormap(&vmap);
+      prefetch_tensormap(&qmap);
+    }
+    const uint64_t pol_kv = l2_policy_evict_first();
+    const uint64_t pol_q = l2_policy_evict_last();
+    uint32_t ctr = 0;   // ring tiles issued
+    uint32_t ucnt = 0;  // units started
+    bool ok = true;
+    for (int64_t u = blockIdx.x; u < num_units && ok; u += gridDim.x) {
+      tc::Unit w;
+      if (!tc::decode_unit(a, u, w)) continue;
+      const int32_t nch = tc::chunks_of(w);
+      if (nch == 0) continue;
+      const uint32_t qb = ucnt & 1u;
+      if (lane == 0) {
+        ok = mbar_wait(&q_empty[qb], ((ucnt >> 1) & 1u) ^ 1u, 0x7100u);
+        if (ok) {
+          mbar_arrive_expect_tx(&q_full[qb], kQBytes);
+          const int32_t qrow = w.s * a.num_q_heads + w.g * G;
+          tma_load_2d(qbuf + qb * kQBytes, &qmap, &q_full[qb], 0, qrow, pol_q);
+          tma_load_2d(qbuf + qb * kQBytes + kN * 128, &qmap, &q_full[qb], 64, qrow, pol_q);
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      ++ucnt;
+      const int32_t* table = a.block_tables + int64_t(w.s) * a.max_blocks_per_seq;
+      for (int32_t c = 0; c < nch && ok; ++c) {
+        const int32_t ntile = tc::tiles_of(w, c);
+        const int32_t blk0 = (w.tok_begin + c * kChunkTok) / BS;
+        const int32_t nblk_seq = (w.ctx + BS - 1) / BS;
+        // lane j holds the id of block blk0 + j (one chunk = 512 / BS <= 32 blocks)
+        const int32_t bidx = blk0 + lane;
+        int32_t id = -1;
+        if (lane < ntile * kBlocksPerTile && bidx < nblk_seq) {
+          id = __ldg(table + bidx);
+          if (id < 0 || id >= a.num_blocks) {
+            record_error(KVP_DEVERR_BLOCK_ID, (uint64_t(w.s) << 32) | uint32_t(bidx));
+            id = -1;
+          }
+        }
+        const int32_t row = id < 0 ? rows_total : (id * a.num_kv_heads + w.g) * BS;
+        for (int kv = 0; kv < 2 && ok; ++kv) {
+          const CUtensorMap* map = kv == 0 ? &kmap : &vmap;
+          for (int32_t t = 0; t < ntile && ok; ++t, ++ctr) {
+            const uint32_t st = ctr % kStages;
+            if (lane == 0) {
+              ok = mbar_wait(&empty[st], ((ctr / kStages) & 1u) ^ 1u, 0x7200u);
+              if (ok) mbar_arrive_expect_tx(&full[st], kStageBytes);
+            }
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) break;
+            const int j = lane - t * kBlocksPerTile;  // block j of this tile
+            if (j >= 0 && j < kBlocksPerTile) {
+              uint8_t* dst = ring + st * kStageBytes + j * BS * 128;
+              tma_load_2d(dst, map, &full[st], 0, row, pol_kv);
+              tma_load_2d(dst + kRegionBytes, map, &full[st], 64, row, pol_kv);
+            }
+            __syncwarp();
+          }
+        }
+      }
+    }
+    if (!ok) {
+      atomicExch(&abort_flag, 1);
+      if (lane == 0)  // drain the loads that may still be in flight
+        for (uint32_t i = ctr > kStages ? ctr - kStages : 0; i < ctr; ++i)
+          mbar_wait(&full[i % kStages], (i / kStages) & 1u, 0x7300u);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    uint32_t ctr = 0, ucnt = 0, cc = 0;
+    bool ok = true;
+    for (int64_t u = blockIdx.x; u < num_units && ok; u += gridDim.x) {
+      tc::Unit w;
+      if (!tc::decode_unit(a, u, w)) continue;
+      const int32_t nch = tc::chunks_of(w);
+      if (nch == 0) continue;  // nothing to multiply; the producer loads no Q for it
+      const uint32_t qb = ucnt & 1u;
+      if (lane == 0) ok = mbar_wait(&q_full[qb], (ucnt >> 1) & 1u, 0x7400u);
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      const uint32_t q_addr = smem_u32(qbuf + qb * kQBytes);
+      for (int32_t c = 0; c < nch && ok; ++c, ++cc) {
+        const uint32_t b = cc & 1u;
+        const uint32_t use = cc >> 1;
+        const int32_t ntile = tc::tiles_of(w, c);
+        if (lane == 0) {
+          // ---- S^T = K Q^T, one tile of 128 tokens at a time
+          ok = mbar_wait(&s_free[b], (use & 1u) ^ 1u, 0x7500u);
+          tc_fence_after();
+          for (int32_t t = 0; t < ntile && ok; ++t, ++ctr) {
+            const uint32_t st = ctr % kStages;
+            ok = mbar_wait(&full[st], (ctr / kStages) & 1u, 0x7600u);
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t k_addr = smem_u32(ring + st * kStageBytes);
+            const uint32_t d_tmem = tmem_base + kSCol + b * (kChunkTiles * kN) + t * kN;
+#pragma unroll
+            for (int kk = 0; kk < kD / 16; ++kk) {
+              const uint32_t off = (kk >> 2) * kRegionBytes + (kk & 3) * 32;
+              const uint32_t qoff = (kk >> 2) * (kN * 128) + (kk & 3) * 32;
+              umma_f16_ss(d_tmem, smem_desc(k_addr + off, 16, 1024, kLayoutSw128),
+                          smem_desc(q_addr + qoff, 16, 1024, kLayoutSw128), kIdescQK, kk > 0);
+            }
+            umma_commit(&empty[st]);
+          }
+          if (ok) {
+            umma_commit(&s_full[b]);
+            if (c == nch - 1) umma_commit(&q_empty[qb]);
+          }
+          // ---- O^T += V^T P^T
+          if (ok) ok = mbar_wait(&p_full[b], use & 1u, 0x7700u);
+          if (ok) ok = mbar_wait(&o_free[b], (use & 1u) ^ 1u, 0x7800u);
+          tc_fence_after();
+          const uint32_t p_addr = smem_u32(pbuf + b * kPBytes);
+          const uint32_t o_tmem = tmem_base + kOCol + b * kN;
+          for (int32_t t = 0; t < ntile && ok; ++t, ++ctr) {
+            const uint32_t st = ctr % kStages;
+            ok = mbar_wait(&full[st], (ctr / kStages) & 1u, 0x7900u);
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t v_addr = smem_u32(ring + st * kStageBytes);
+#pragma unroll
+            for (int kk = 0; kk < kTileTok / 16; ++kk) {
+              const uint32_t pk = (t * kTileTok + kk * 16) / 8 * 256;
+              umma_f16_ss(o_tmem, smem_desc(v_addr + kk * 2048, kRegionBytes, 1024, kLayoutSw128),
+                          smem_desc(p_addr + pk, 256, 128, kLayoutNone), kIdescPV,
+                          (t > 0 || kk > 0) ? 1u : 0u);
+            }
+            umma_commit(&empty[st]);
+          }
+          if (ok) {
+            umma_commit(&o_full[b]);
+            umma_commit(&p_free[b]);
+          }
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+      }
+      ++ucnt;
+    }
+    if (!ok) atomicExch(&abort_flag, 1);
+  } else {
+    // ------------------------------------------------------------ softmax + epilogue
+    // All waits here are bounded mbarrier waits made warp-uniform; the four
+    // warps exchange maxima and sums through shared memory guarded by count-4
+    // mbarriers on alternating halves (no unbounded named barriers).
+    const int quarter = warp & 3;          // TMEM lanes 32*quarter .. +31
+    const int r = quarter * 32 + lane;     // token row (S) / head-dim row (O)
+    const uint32_t lane_addr = uint32_t(quarter * 32) << 16;
+    const int wi = warp - 2;               // softmax warp index 0..3
+    auto wait_all = [&](uint64_t* bar, uint32_t parity, uint32_t where) {
+      return __all_sync(0xffffffffu, mbar_wait(bar, parity, where)) != 0;
+    };
+    uint32_t ctr = 0, cc = 0, ucnt = 0;
+    bool ok = true;
+    for (int64_t u = blockIdx.x; u < num_units && ok; u += gridDim.x) {
+      tc::Unit w;
+      if (!tc::decode_unit(a, u, w)) continue;
+      float acc[NG], m_run[NG], l_thr[NG];
+#pragma unroll
+      for (int j = 0; j < NG; ++j) {
+        acc[j] = 0.f;
+        m_run[j] = -INFINITY;
+        l_thr[j] = 0.f;
+      }
+      const int32_t nch = tc::chunks_of(w);
+      for (int32_t c = 0; c < nch && ok; ++c, ++cc) {
+        const uint32_t b = cc & 1u;
+        const uint32_t use = cc >> 1;
+        const int32_t ntile = tc::tiles_of(w, c);
+        const int32_t ctok0 = w.tok_begin + c * kChunkTok;
+        const int32_t ctok1 = min(w.tok_end, ctok0 + kChunkTok);
+        // ---- scores of this thread's tokens (row r of each tile)
+        ok = wait_all(&s_full[b], use & 1u, 0x7a00u);
+        if (!ok) break;
+        tc_fence_after();
+        float sv[kChunkTiles][NG];
+#pragma unroll
+        for (int t = 0; t < kChunkTiles; ++t) {
+          if (t < ntile) {
+            tmem_ld_cols<NG>(tmem_base + lane_addr + kSCol + b * (kChunkTiles * kN) + t * kN,
+                             sv[t]);
+          } else {
+#pragma unroll
+            for (int j = 0; j < NG; ++j) sv[t][j] = -INFINITY;
+          }
+        }
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s_free[b]);
+        float cmax[NG];
+#pragma unroll
+        for (int j = 0; j < NG; ++j) cmax[j] = -INFINITY;
+#pragma unroll
+        for (int t = 0; t < kChunkTiles; ++t) {
+          const bool valid = t < ntile && ctok0 + t * kTileTok + r < ctok1;
+#pragma unroll
+          for (int j = 0; j < NG; ++j) {
+            sv[t][j] = valid ? sv[t][j] * a.scale_log2 : -INFINITY;
+            cmax[j] = fmaxf(cmax[j], sv[t][j]);
+          }
+        }
+        float* redm = red + b * 4 * kN;
+#pragma unroll
+        for (int j = 0; j < NG; ++j) {
+          cmax[j] = warp_max(cmax[j]);
+          if (lane == 0) redm[wi * kN + j] = cmax[j];
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&red_bar[b]);
+        ok = wait_all(&red_bar[b], use & 1u, 0x7a80u);
+        if (!ok) break;
+#pragma unroll
+        for (int j = 0; j < NG; ++j)
+          cmax[j] = fmaxf(fmaxf(redm[j], redm[kN + j]), fmaxf(redm[2 * kN + j], redm[3 * kN + j]));
+        // ---- p = 2^(s - m), rounded to the input type, into P^T (K-major, no swizzle)
+        ok = wait_all(&p_free[b], (use & 1u) ^ 1u, 0x7b00u);
+        if (!ok) break;
+        uint8_t* pb = pbuf + b * kPBytes;
+        float psum[NG];
+#pragma unroll
+        for (int j = 0; j < NG; ++j) psum[j] = 0.f;
+#pragma unroll
+        for (int t = 0; t < kChunkTiles; ++t) {
+          if (t < ntile) {
+            const int tok = t * kTileTok + r;  // token within the chunk
+            uint8_t* prow = pb + (tok >> 3) * 256 + (tok & 7) * 2;
+#pragma unroll
+            for (int j = 0; j < NG; ++j) {
+              const float pf = sv[t][j] == -INFINITY ? 0.f : exp2f(sv[t][j] - cmax[j]);
+              const uint16_t pbits = Elem<T>::from_float(pf);
+              psum[j] += Elem<T>::to_float2(uint32_t(pbits)).x;
+              *reinterpret_cast<uint16_t*>(prow + (j >> 3) * 128 + (j & 7) * 16) = pbits;
+            }
+          }
+        }
+        // Tokens past the end of the sequence in the chunk's last tile: their V
+        // rows hold whatever the pool had there; zero them before the PV MMA
+        // (p is already 0 for them, but 0 * inf would still be NaN).
+        {
+          const int32_t last_tile = (ctok1 - 1 - ctok0) / kTileTok;
+          const bool past_end = ctok0 + last_tile * kTileTok + r >= ctok1;
+          const uint32_t vctr = ctr + ntile + last_tile;
+          const uint32_t st = vctr % kStages;
+          if (__any_sync(0xffffffffu, past_end)) {
+            ok = wait_all(&full[st], (vctr / kStages) & 1u, 0x7c00u);
+            if (ok && past_end) {
+              uint8_t* vrow = ring + st * kStageBytes + r * 128;
+#pragma unroll
+              for (int q = 0; q < 8; ++q) {
+                reinterpret_cast<uint4*>(vrow)[q] = make_uint4(0, 0, 0, 0);
+                reinterpret_cast<uint4*>(vrow + kRegionBytes)[q] = make_uint4(0, 0, 0, 0);
+              }
+            }
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_full[b]);
+        if (!ok) break;
+        ctr += 2 * ntile;
+        // ---- merge this chunk's O into the running output
+        ok = wait_all(&o_full[b], use & 1u, 0x7d00u);
+        if (!ok) break;
+        tc_fence_after();
+        float ov[NG];
+        tmem_ld_cols<NG>(tmem_base + lane_addr + kOCol + b * kN, ov);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&o_free[b]);
+#pragma unroll
+        for (int j = 0; j < NG; ++j) {
+          const float mn = fmaxf(m_run[j], cmax[j]);
+          const float fo = m_run[j] == -INFINITY ? 0.f : exp2f(m_run[j] - mn);
+          const float fc = cmax[j] == -INFINITY ? 0.f : exp2f(cmax[j] - mn);
+          acc[j] = acc[j] * fo + ov[j] * fc;
+          l_thr[j] = l_thr[j] * fo + psum[j] * fc;
+          m_run[j] = mn;
+        }
+      }
+      if (!ok) break;
+      // ---- unit epilogue: l over all 128 rows, then write
+      const uint32_t ub = ucnt & 1u;
+      float* rl = redl + ub * 4 * kN;
+#pragma unroll
+      for (int j = 0; j < NG; ++j) {
+        float v = l_thr[j];
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        if (lane == 0) rl[wi * kN + j] = v;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&lred_bar[ub]);
+      ok = wait_all(&lred_bar[ub], (ucnt >> 1) & 1u, 0x7e00u);
+      ++ucnt;
+      if (!ok) break;
+      const int32_t h0 = w.g * G;
+#pragma unroll
+      for (int j = 0; j < NG; ++j) {
+        const float L = (rl[j] + rl[kN + j]) + (rl[2 * kN + j] + rl[3 * kN + j]);
+        if (j < G) {
+          const int64_t row_sh = int64_t(w.s) * a.num_q_heads + h0 + j;
+          if (w.nparts <= 1) {
+            const float y = L > 0.f ? acc[j] / L : 0.f;
+            static_cast<uint16_t*>(a.out)[row_sh * kD + r] = Elem<T>::from_float(y);
+          } else {
+            a.ws_acc[(row_sh * a.pmax + w.p) * kD + r] = acc[j];
+            if (r == 0) {
+              a.ws_ml[(row_sh * a.pmax + w.p) * 2 + 0] = m_run[j];
+              a.ws_ml[(row_sh * a.pmax + w.p) * 2 + 1] = L;
+            }
+          }
+        }
+      }
+    }
+    if (!ok) atomicExch(&abort_flag, 1);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem_base, kTmemCols);
+}
+
+}  // namespace dev
+}  // namespace kvp

@@ -1,0 +1,361 @@
+// Device entry points of libkvp (C ABI): argument checks, TMA tensor maps,
+// kernel selection by geometry, launches on the caller's stream.
+//
+// All device code lives in this one translation unit (the kernels are
+// headers) so the device error word is a single symbol per GPU.
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "kernels/cache_ops.cuh"
+#include "kernels/common.cuh"
+#include "kernels/decode_simt.cuh"
+#include "kernels/decode_tc.cuh"
+#include "status.h"
+
+using kvp::fail;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+int cuda_fail(cudaError_t e, const char* what) {
+  return fail(KVP_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+int current_device() {
+  int d = 0;
+  cudaGetDevice(&d);
+  return d;
+}
+
+int sm_count() {
+  static std::atomic<int> cache[kMaxDevices];
+  const int d = current_device();
+  if (d < 0 || d >= kMaxDevices) return 148;
+  int n = cache[d].load(std::memory_order_relaxed);
+  if (n == 0) {
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, d);
+    if (n <= 0) n = 148;
+    cache[d].store(n, std::memory_order_relaxed);
+  }
+  return n;
+}
+
+// Raises a kernel's dynamic shared-memory limit once per device.
+template <typename K>
+cudaError_t ensure_smem(K kernel, int bytes) {
+  static std::atomic<uint64_t> done{0};
+  const int d = current_device();
+  const uint64_t bit = d < 64 ? (1ull << d) : 0;
+  if (bit && (done.load(std::memory_order_relaxed) & bit)) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_relaxed);
+  return e;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2-D view [rows][cols] of 2-byte elements with a {64, box_rows} box and
+// 128-byte swizzle; out-of-range rows read as zeros.
+int make_map(CUtensorMap* map, const void* base, int32_t dtype, uint64_t rows, uint64_t cols,
+             uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return fail(KVP_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  const CUtensorMapDataType dt =
+      dtype == KVP_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  CUresult r = fn(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(KVP_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", int(r));
+  return KVP_OK;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+int ilog2(int64_t v) {
+  int l = 0;
+  while ((int64_t(1) << l) < v) ++l;
+  return (int64_t(1) << l) == v ? l : -1;
+}
+
+struct Workspace {
+  size_t ml_bytes, acc_bytes, total;
+};
+
+Workspace ws_layout(int64_t S, int64_t Hq, int64_t D, int64_t pmax) {
+  Workspace w{};
+  if (pmax <= 1) return w;
+  auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
+  w.ml_bytes = up(size_t(S * Hq * pmax * 2 * 4));
+  w.acc_bytes = up(size_t(S * Hq * pmax * D * 4));
+  w.total = w.ml_bytes + w.acc_bytes;
+  return w;
+}
+
+// ---- decode launches ----------------------------------------------------------
+template <typename T, int D, int BS>
+int launch_simt(const CUtensorMap& km, const CUtensorMap& vm, const kvp::dev::DecodeArgs& a,
+                cudaStream_t st) {
+  constexpr int NW = 4, NST = 3;
+  using C = kvp::dev::SimtCfg<T, D, BS, NW, NST>;
+  auto k = kvp::dev::decode_simt_kernel<T, D, BS, NW, NST>;
+  cudaError_t e = ensure_smem(k, C::kSmemBytes);
+  if (e != cudaSuccess) return cuda_fail(e, "decode (CUDA cores): smem attribute");
+  dim3 grid(a.pmax, a.num_q_heads, a.num_seqs);
+  k<<<grid, NW * 32, C::kSmemBytes, st>>>(km, vm, a);
+  e = cudaGetLastError();
+  return e == cudaSuccess ? KVP_OK : cuda_fail(e, "decode (CUDA cores): launch");
+}
+
+template <typename T, int BS, int NG>
+int launch_tc(const CUtensorMap& km, const CUtensorMap& vm, const CUtensorMap& qm,
+              const kvp::dev::DecodeArgs& a, cudaStream_t st) {
+  auto k = kvp::dev::decode_tc_kernel<T, BS, NG>;
+  cudaError_t e = ensure_smem(k, kvp::dev::tc::kSmemBytes);
+  if (e != cudaSuccess) return cuda_fail(e, "decode (tensor cores): smem attribute");
+  const int64_t units = int64_t(a.num_seqs) * a.num_kv_heads * a.pmax;
+  const int grid = int(units < sm_count() ? units : sm_count());
+  k<<<grid, kvp::dev::tc::kThreads, kvp::dev::tc::kSmemBytes, st>>>(km, vm, qm, a, units);
+  e = cudaGetLastError();
+  return e == cudaSuccess ? KVP_OK : cuda_fail(e, "decode (tensor cores): launch");
+}
+
+template <typename T, int D>
+int launch_reduce(const kvp::dev::DecodeArgs& a, cudaStream_t st) {
+  auto k = kvp::dev::decode_reduce_kernel<T, D>;
+  dim3 grid(a.num_q_heads, a.num_seqs);
+  k<<<grid, D, size_t(a.pmax) * 4, st>>>(a);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? KVP_OK : cuda_fail(e, "decode reduce: launch");
+}
+
+template <typename T, int D>
+int simt_by_bs(int bs, const CUtensorMap& km, const CUtensorMap& vm, const kvp::dev::DecodeArgs& a,
+               cudaStream_t st) {
+  switch (bs) {
+    case 8: return launch_simt<T, D, 8>(km, vm, a, st);
+    case 16: return launch_simt<T, D, 16>(km, vm, a, st);
+    case 32: return launch_simt<T, D, 32>(km, vm, a, st);
+  }
+  return fail(KVP_ERR_INVALID, "block_size %d not supported", bs);
+}
+
+template <typename T>
+int tc_dispatch(int bs, int G, const CUtensorMap& km, const CUtensorMap& vm, const CUtensorMap& qm,
+                const kvp::dev::DecodeArgs& a, cudaStream_t st) {
+  const int ng = G <= 4 ? 4 : (G <= 8 ? 8 : 16);
+  if (bs == 16) {
+    if (ng == 4) return launch_tc<T, 16, 4>(km, vm, qm, a, st);
+    if (ng == 8) return launch_tc<T, 16, 8>(km, vm, qm, a, st);
+    return launch_tc<T, 16, 16>(km, vm, qm, a, st);
+  }
+  if (ng == 4) return launch_tc<T, 32, 4>(km, vm, qm, a, st);
+  if (ng == 8) return launch_tc<T, 32, 8>(km, vm, qm, a, st);
+  return launch_tc<T, 32, 16>(km, vm, qm, a, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+int reshape_and_cache(const void* k_new, const void* v_new, void* k_cache, void* v_cache,
+                      const int64_t* slot_mapping, int32_t num_tokens, int32_t num_kv_heads,
+                      int32_t head_dim, int32_t block_size, int32_t num_blocks, int32_t dtype,
+                      kvp_stream_t stream) {
+  if (num_tokens < 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 || num_blocks <= 0)
+    return fail(KVP_ERR_INVALID, "reshape_and_cache: bad sizes");
+  if (dtype != KVP_F16 && dtype != KVP_BF16) return fail(KVP_ERR_INVALID, "reshape_and_cache: bad dtype");
+  const int lcpr = ilog2(head_dim / 8);
+  const int lbs = ilog2(block_size);
+  if (head_dim % 8 || lcpr < 0 || lbs < 0)
+    return fail(KVP_ERR_INVALID, "reshape_and_cache: head_dim/8 and block_size must be powers of two");
+  if (num_tokens == 0) return KVP_OK;
+  if (!k_new || !v_new || !k_cache || !v_cache || !slot_mapping)
+    return fail(KVP_ERR_INVALID, "reshape_and_cache: NULL pointer");
+  if (!aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
+      !aligned(slot_mapping, 8))
+    return fail(KVP_ERR_INVALID, "reshape_and_cache: misaligned pointer");
+  const int64_t chunks = int64_t(num_tokens) * num_kv_heads * (head_dim / 8);
+  if (chunks >= (int64_t(1) << 31)) return fail(KVP_ERR_INVALID, "reshape_and_cache: too many tokens in one call");
+  const int threads = 256;
+  int64_t blocks = (chunks + threads - 1) / threads;
+  const int64_t cap = int64_t(sm_count()) * 16;
+  if (blocks > cap) blocks = cap;
+  kvp::dev::reshape_and_cache_kernel<<<int(blocks), threads, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new), static_cast<uint4*>(k_cache),
+      static_cast<uint4*>(v_cache), slot_mapping, uint32_t(chunks), uint32_t(num_kv_heads),
+      uint32_t(lcpr), uint32_t(lbs), int64_t(num_blocks) * block_size);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? KVP_OK : cuda_fail(e, "reshape_and_cache: launch");
+}
+
+int copy_blocks(void* k_cache, void* v_cache, const int32_t* pairs, int32_t num_pairs,
+                int32_t num_blocks, int64_t block_elems, int32_t dtype, kvp_stream_t stream) {
+  if (num_pairs < 0 || num_blocks <= 0 || block_elems <= 0)
+    return fail(KVP_ERR_INVALID, "copy_blocks: bad sizes");
+  if (dtype != KVP_F16 && dtype != KVP_BF16) return fail(KVP_ERR_INVALID, "copy_blocks: bad dtype");
+  if ((block_elems * 2) % 16) return fail(KVP_ERR_INVALID, "copy_blocks: block bytes not a multiple of 16");
+  if (num_pairs == 0) return KVP_OK;
+  if (num_pairs > 65535) return fail(KVP_ERR_INVALID, "copy_blocks: more than 65535 pairs in one call");
+  if (!k_cache || !v_cache || !pairs) return fail(KVP_ERR_INVALID, "copy_blocks: NULL pointer");
+  if (!aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(pairs, 4))
+    return fail(KVP_ERR_INVALID, "copy_blocks: misaligned pointer");
+  const int64_t chunks = block_elems * 2 / 16;
+  int gx = int((chunks + 255) / 256);
+  if (gx > 64) gx = 64;
+  dim3 grid(gx, num_pairs, 2);
+  kvp::dev::copy_blocks_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), pairs, chunks, num_blocks);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? KVP_OK : cuda_fail(e, "copy_blocks: launch");
+}
+
+size_t kvp_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, int32_t head_dim,
+                                  int32_t max_context_len, int32_t partition_size) {
+  if (partition_size <= 0 || num_seqs <= 0 || num_q_heads <= 0 || head_dim <= 0 || max_context_len <= 0)
+    return 0;
+  const int64_t pmax = (int64_t(max_context_len) + partition_size - 1) / partition_size;
+  return ws_layout(num_seqs, num_q_heads, head_dim, pmax).total;
+}
+
+int paged_attention_decode(const void* q, const void* k_cache, const void* v_cache,
+                           const int32_t* block_tables, const int32_t* context_lens,
+                           int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
+                           int32_t head_dim, int32_t block_size, int32_t num_blocks,
+                           int32_t max_blocks_per_seq, int32_t max_context_len, float scale,
+                           int32_t partition_size, void* workspace, size_t workspace_bytes,
+                           void* out, int32_t dtype, kvp_stream_t stream) {
+  if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_blocks <= 0 ||
+      max_blocks_per_seq <= 0 || max_context_len < 0 || partition_size < 0)
+    return fail(KVP_ERR_INVALID, "paged_attention_decode: bad sizes");
+  if (num_q_heads % num_kv_heads) return fail(KVP_ERR_INVALID, "paged_attention_decode: num_q_heads %% num_kv_heads != 0");
+  if (head_dim != 64 && head_dim != 128) return fail(KVP_ERR_INVALID, "paged_attention_decode: head_dim must be 64 or 128");
+  if (block_size != 8 && block_size != 16 && block_size != 32)
+    return fail(KVP_ERR_INVALID, "paged_attention_decode: block_size must be 8, 16 or 32");
+  if (dtype != KVP_F16 && dtype != KVP_BF16) return fail(KVP_ERR_INVALID, "paged_attention_decode: bad dtype");
+  if (int64_t(max_context_len) > int64_t(max_blocks_per_seq) * block_size)
+    return fail(KVP_ERR_INVALID, "paged_attention_decode: max_context_len > max_blocks_per_seq * block_size");
+  if (int64_t(num_blocks) * num_kv_heads * block_size >= (int64_t(1) << 31))
+    return fail(KVP_ERR_INVALID, "paged_attention_decode: pool too large for 32-bit row coordinates");
+  if (partition_size % block_size) return fail(KVP_ERR_INVALID, "paged_attention_decode: partition_size must be a multiple of block_size");
+  if (!std::isfinite(scale)) return fail(KVP_ERR_INVALID, "paged_attention_decode: scale not finite");
+  if (num_seqs == 0) return KVP_OK;
+  if (!q || !k_cache || !v_cache || !block_tables || !context_lens || !out)
+    return fail(KVP_ERR_INVALID, "paged_attention_decode: NULL pointer");
+  if (!aligned(q, 16) || !aligned(out, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
+      !aligned(block_tables, 4) || !aligned(context_lens, 4))
+    return fail(KVP_ERR_INVALID, "paged_attention_decode: misaligned pointer");
+
+  const int G = num_q_heads / num_kv_heads;
+  const bool tensor_cores = G > 1 && G <= 16 && head_dim == 128 && (block_size == 16 || block_size == 32);
+  if (tensor_cores && partition_size % 128)
+    return fail(KVP_ERR_INVALID, "paged_attention_decode: grouped-query path needs partition_size %% 128 == 0");
+
+  const int32_t ctx_cap = max_context_len > 0 ? max_context_len : 1;
+  int32_t part_tokens, pmax;
+  if (partition_size > 0) {
+    part_tokens = partition_size;
+    pmax = (ctx_cap + partition_size - 1) / partition_size;
+  } else {
+    part_tokens = ((ctx_cap + block_size - 1) / block_size) * block_size;
+    pmax = 1;
+  }
+  const Workspace wl = ws_layout(num_seqs, num_q_heads, head_dim, pmax);
+  if (wl.total) {
+    if (!workspace || workspace_bytes < wl.total)
+      return fail(KVP_ERR_INVALID, "paged_attention_decode: workspace of %zu bytes needed", wl.total);
+    if (!aligned(workspace, 256)) return fail(KVP_ERR_INVALID, "paged_attention_decode: workspace not 256-byte aligned");
+  }
+
+  kvp::dev::DecodeArgs a{};
+  a.q = q;
+  a.out = out;
+  a.block_tables = block_tables;
+  a.context_lens = context_lens;
+  a.ws_ml = wl.total ? static_cast<float*>(workspace) : nullptr;
+  a.ws_acc = wl.total ? reinterpret_cast<float*>(static_cast<char*>(workspace) + wl.ml_bytes) : nullptr;
+  a.num_seqs = num_seqs;
+  a.num_q_heads = num_q_heads;
+  a.num_kv_heads = num_kv_heads;
+  a.num_blocks = num_blocks;
+  a.max_blocks_per_seq = max_blocks_per_seq;
+  a.max_context_len = max_context_len;
+  a.part_blocks = part_tokens / block_size;
+  a.part_tokens = part_tokens;
+  a.pmax = pmax;
+  a.scale_log2 = scale * 1.4426950408889634f;
+
+  const uint64_t rows = uint64_t(num_blocks) * num_kv_heads * block_size;
+  CUtensorMap km, vm;
+  int rc = make_map(&km, k_cache, dtype, rows, head_dim, block_size);
+  if (rc) return rc;
+  rc = make_map(&vm, v_cache, dtype, rows, head_dim, block_size);
+  if (rc) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+  if (tensor_cores) {
+    CUtensorMap qm;
+    rc = make_map(&qm, q, dtype, uint64_t(num_seqs) * num_q_heads, head_dim, kvp::dev::tc::kN);
+    if (rc) return rc;
+    rc = dtype == KVP_F16 ? tc_dispatch<__half>(block_size, G, km, vm, qm, a, st)
+                          : tc_dispatch<__nv_bfloat16>(block_size, G, km, vm, qm, a, st);
+  } else if (head_dim == 128) {
+    rc = dtype == KVP_F16 ? simt_by_bs<__half, 128>(block_size, km, vm, a, st)
+                          : simt_by_bs<__nv_bfloat16, 128>(block_size, km, vm, a, st);
+  } else {
+    rc = dtype == KVP_F16 ? simt_by_bs<__half, 64>(block_size, km, vm, a, st)
+                          : simt_by_bs<__nv_bfloat16, 64>(block_size, km, vm, a, st);
+  }
+  if (rc || pmax <= 1) return rc;
+  if (head_dim == 128)
+    return dtype == KVP_F16 ? launch_reduce<__half, 128>(a, st) : launch_reduce<__nv_bfloat16, 128>(a, st);
+  return dtype == KVP_F16 ? launch_reduce<__half, 64>(a, st) : launch_reduce<__nv_bfloat16, 64>(a, st);
+}
+
+int kvp_check_device_error(kvp_stream_t stream) {
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "kvp_check_device_error: stream synchronize");
+  unsigned long long v = 0;
+  e = cudaMemcpyFromSymbol(&v, kvp::dev::g_error_word, sizeof(v));
+  if (e != cudaSuccess) return cuda_fail(e, "kvp_check_device_error: read");
+  if (v == 0) return KVP_OK;
+  const unsigned long long zero = 0;
+  e = cudaMemcpyToSymbol(kvp::dev::g_error_word, &zero, sizeof(zero));
+  if (e != cudaSuccess) return cuda_fail(e, "kvp_check_device_error: clear");
+  const unsigned kind = unsigned(v >> 56);
+  const unsigned long long payload = v & ((1ull << 56) - 1);
+  static const char* names[] = {"none", "slot out of range (token index)",
+                                "block table entry out of range (seq << 32 | logical block)",
+                                "context length out of range (sequence)",
+                                "copy pair out of range (pair index)", "bounded wait timed out (site)"};
+  const char* name = kind < 6 ? names[kind] : "unknown";
+  if (kind == kvp::dev::KVP_DEVERR_TIMEOUT)
+    return fail(KVP_ERR_CUDA, "device: %s 0x%llx", name, payload);
+  return fail(KVP_ERR_BOUNDS, "device: %s %llu", name, payload);
+}
+
+}  // extern "C"

@@ -1,0 +1,128 @@
+"""Runs a workload's operation schedule through libkvp on one GPU.
+
+The host allocator (:class:`BlockPool`) turns create / append / fork /
+release into block tables, slots and copy-on-write pairs; at each ``sync``
+the pending copies run (``copy_blocks``) and then every token appended since
+the previous sync is written to its slot (``reshape_and_cache``); at each
+``attend`` the batch's block tables and lengths go to the device and
+``paged_attention_decode`` runs. Per-step order: copies, then scatter, then
+attention, because a new token may land in a block copied in the same step.
+
+Inputs (K/V of appended tokens, q of each attend) are drawn from
+:mod:`workloads` keyed by the op's index, the same draws any other consumer
+of the schedule sees.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+from workloads.values import K_STREAM, Q_STREAM, V_STREAM, normal_bits, value_seed_words
+
+from . import BlockPool, copy_blocks, paged_attention_decode, reshape_and_cache
+
+
+def bits_to_tensor(bits: np.ndarray, dtype: str, device):
+    import torch
+
+    t = torch.from_numpy(np.ascontiguousarray(bits).view(np.int16))
+    t = t.view(torch.float16 if dtype == "f16" else torch.bfloat16)
+    return t.to(device, non_blocking=False)
+
+
+class DeviceReplay:
+    def __init__(self, wl, device="cuda", keep_outputs: bool = True):
+        import torch
+
+        g = wl.geometry
+        self.wl, self.g = wl, g
+        self.device = torch.device(device)
+        self.tdtype = torch.float16 if g.dtype == "f16" else torch.bfloat16
+        self.pool = BlockPool(wl.num_blocks, g.block_size, g.num_kv_heads, g.head_dim, g.dtype,
+                              wl.free_order)
+        shape = (wl.num_blocks, g.num_kv_heads, g.block_size, g.head_dim)
+        self.k_cache = torch.zeros(shape, dtype=self.tdtype, device=self.device)
+        self.v_cache = torch.zeros(shape, dtype=self.tdtype, device=self.device)
+        self.ids: dict[int, int] = {}
+        self._pending = []
+        self.events = []
+        self.attends = []          # (op_index, seq ids, tables, lens)
+        self.outputs = {}          # op_index -> out tensor
+        self.keep_outputs = keep_outputs
+        self.next_index = 0
+
+    def kv_values(self, op_index: int, n: int):
+        g = self.g
+        shape = (n, g.num_kv_heads, g.head_dim)
+        k = normal_bits(value_seed_words(self.wl.value_seed, K_STREAM, op_index), shape, g.dtype)
+        v = normal_bits(value_seed_words(self.wl.value_seed, V_STREAM, op_index), shape, g.dtype)
+        return k, v
+
+    def q_values(self, op_index: int, num_seqs: int):
+        g = self.g
+        shape = (num_seqs, g.num_q_heads, g.head_dim)
+        return normal_bits(value_seed_words(self.wl.value_seed, Q_STREAM, op_index), shape, g.dtype)
+
+    def run(self, ops=None, start_index=None, attend_kwargs=None):
+        ops = self.wl.ops if ops is None else ops
+        i = self.next_index if start_index is None else start_index
+        for op in ops:
+            self._apply(i, op, attend_kwargs or {})
+            i += 1
+        self.next_index = i
+
+    def _apply(self, i, op, kw):
+        import torch
+
+        kind = op[0]
+        pool = self.pool
+        if kind == "create":
+            self.ids[op[1]] = pool.create()
+            self.events.append((i, "create", self.ids[op[1]]))
+        elif kind == "append":
+            slots = pool.append(self.ids[op[1]], op[2])
+            self._pending.append((slots, i, op[2]))
+            self.events.append((i, "append", slots))
+        elif kind == "fork":
+            self.ids[op[2]] = pool.fork(self.ids[op[1]])
+            self.events.append((i, "fork", self.ids[op[2]]))
+        elif kind == "release":
+            pool.release(self.ids[op[1]])
+            self.events.append((i, "release", None))
+        elif kind == "sync":
+            copies = pool.take_copies()
+            self.events.append((i, "sync", copies))
+            if copies:
+                pairs = torch.tensor(copies, dtype=torch.int32, device=self.device)
+                copy_blocks(self.k_cache, self.v_cache, pairs)
+            work = [(s, j, n) for s, j, n in self._pending if n]
+            if work:
+                ks, vs, sl = [], [], []
+                for slots, j, n in work:
+                    k, v = self.kv_values(j, n)
+                    ks.append(k)
+                    vs.append(v)
+                    sl.extend(slots)
+                k_new = bits_to_tensor(np.concatenate(ks), self.g.dtype, self.device)
+                v_new = bits_to_tensor(np.concatenate(vs), self.g.dtype, self.device)
+                slot_t = torch.tensor(sl, dtype=torch.int64, device=self.device)
+                reshape_and_cache(k_new, v_new, self.k_cache, self.v_cache, slot_t)
+            self._pending = []
+        elif kind == "attend":
+            seqs = [self.ids[h] for h in op[1]]
+            lens_host = [pool.seq_len(s) for s in seqs]
+            bs = self.g.block_size
+            max_blocks = max(1, max(-(-L // bs) for L in lens_host))
+            tables, lens = pool.build_batch(seqs, max_blocks)
+            self.attends.append((i, seqs, tables, lens))
+            q = bits_to_tensor(self.q_values(i, len(seqs)), self.g.dtype, self.device)
+            bt = torch.from_numpy(tables).to(self.device)
+            cl = torch.from_numpy(lens).to(self.device)
+            part = kw.get("partition_size", self.wl.partition_size)
+            out = paged_attention_decode(q, self.k_cache, self.v_cache, bt, cl, self.wl.scale,
+                                         max_context_len=int(lens.max()) if len(lens) else 0,
+                                         partition_size=part)
+            if self.keep_outputs:
+                self.outputs[i] = out
+        else:
+            raise ValueError(f"unknown op {op!r}")
