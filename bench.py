@@ -148,26 +148,30 @@ def dist_setup():
     return world, rank, local
 
 
-def dist_max(x: float, world: int) -> float:
+def _reduce(x: float, world: int, op: str) -> float:
+    """All-reduce of one timing number across ranks (CPU tensor under gloo)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
 
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dev = "cpu" if dist.get_backend() == "gloo" else "cuda"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX if op == "max" else dist.ReduceOp.SUM)
     return float(t.item())
+
+
+def dist_max(x: float, world: int) -> float:
+    return _reduce(x, world, "max")
 
 
 def dist_sum(x: float, world: int) -> float:
-    if world == 1:
-        return x
-    import torch
-    import torch.distributed as dist
+    return _reduce(x, world, "sum")
 
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.SUM)
-    return float(t.item())
+
+def shard_value_seed(value_seed: int, rank: int) -> int:
+    """Each rank's independent shard draws its own values; lengths and schedule are shared."""
+    return value_seed + 7919 * rank
 
 
 def barrier(world):
@@ -236,7 +240,7 @@ def run_ours(args, world, rank, local):
     if need_end > wl.num_blocks:
         raise SystemExit(f"pool of {wl.num_blocks} blocks too small for {W + K} steps")
 
-    seed_rank = wl.value_seed + 7919 * rank
+    seed_rank = shard_value_seed(wl.value_seed, rank)
     n_pre = int(start.sum())
     pk = to_dev(normal_bits(value_seed_words(seed_rank, K_STREAM, 0), (max(n_pre, 1), g.num_kv_heads, g.head_dim), g.dtype), g.dtype, device)
     pv = to_dev(normal_bits(value_seed_words(seed_rank, V_STREAM, 0), (max(n_pre, 1), g.num_kv_heads, g.head_dim), g.dtype), g.dtype, device)

@@ -48,37 +48,47 @@ constexpr int kN = 16;              // MMA N (query heads of a group, padded)
 constexpr int kTileTok = 128;       // MMA M: tokens per tile
 constexpr int kChunkTiles = 4;      // tiles per chunk (512 tokens)
 constexpr int kChunkTok = kTileTok * kChunkTiles;
-constexpr int kStages = 5;
 constexpr int kStageBytes = kTileTok * kD * 2;       // 32 KiB
 constexpr int kRegionBytes = kTileTok * 128;         // 16 KiB: 64 dims of 128 tokens
 constexpr int kQBytes = kN * kD * 2;                 // 4 KiB
-constexpr int kPBytes = kChunkTok * kN * 2;          // 16 KiB
 constexpr int kTmemCols = 256;
 constexpr int kSCol = 0;                             // S buffers: [0, 128)
-constexpr int kOCol = 128;                           // O buffers: [128, 160)
+constexpr int kOCol = 128;                           // O buffers: [128, 128 + 2 * kNPV)
 constexpr int kThreads = 192;
 constexpr int kSoftmaxThreads = 128;
 
-// Shared-memory layout (offsets from a 1024-aligned base).
-constexpr int kOffRing = 0;
-constexpr int kOffQ = kOffRing + kStages * kStageBytes;
-constexpr int kOffP = kOffQ + 2 * kQBytes;
-constexpr int kOffBar = kOffP + 2 * kPBytes;
-constexpr int kNumBars = 2 * kStages + 2 * 10;
-constexpr int kOffRed = kOffBar + kNumBars * 8;               // [2 halves][4 warps][kN] maxima
-constexpr int kOffRedL = kOffRed + 2 * 4 * kN * 4;            // [2 halves][4 warps][kN] sums
-constexpr int kOffTmemPtr = kOffRedL + 2 * 4 * kN * 4;
-constexpr int kSmemBytes = 1024 + kOffTmemPtr + 16;
-// The softmax warps wait for a chunk's last V tile (to zero rows past the end
-// of the sequence) before the PV MMAs free any stage of that chunk, so the
-// ring must hold a chunk's K tiles plus that V tile.
-static_assert(kStages >= kChunkTiles, "ring too shallow for one chunk");
-static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
+// Layout for a group width NG (query heads per KV head, padded to 4, 8 or 16).
+// P^T holds p split into a high part and a low part, both in the input type
+// (rows [0, NG) and [NG, 2 NG)): the PV MMA multiplies V by hi + lo, which
+// carries p to about 16 significant bits instead of the 8 of one bf16.
+template <int NG>
+struct Cfg {
+  static constexpr int kNPV = 2 * NG <= 16 ? 16 : 32;  // N of the PV MMA
+  static constexpr int kStages = NG <= 8 ? 5 : 4;
+  static constexpr int kPBytes = kChunkTok * kNPV * 2;
+  static constexpr int kPLbo = kNPV * 16;               // bytes between 8-token groups of P^T
+  static constexpr int kOffRing = 0;
+  static constexpr int kOffQ = kOffRing + kStages * kStageBytes;
+  static constexpr int kOffP = kOffQ + 2 * kQBytes;
+  static constexpr int kOffBar = kOffP + 2 * kPBytes;
+  static constexpr int kNumBars = 2 * kStages + 2 * 10;
+  static constexpr int kOffRed = kOffBar + kNumBars * 8;     // [2 halves][4 warps][kN] maxima
+  static constexpr int kOffRedL = kOffRed + 2 * 4 * kN * 4;  // [2 halves][4 warps][kN] sums
+  static constexpr int kOffTmemPtr = kOffRedL + 2 * 4 * kN * 4;
+  static constexpr int kSmemBytes = 1024 + kOffTmemPtr + 16;
+  // The softmax warps wait for a chunk's last V tile (to zero rows past the
+  // end of the sequence) before the PV MMAs free any stage of that chunk, so
+  // the ring must hold a chunk's K tiles plus that V tile.
+  static_assert(kStages >= kChunkTiles, "ring too shallow for one chunk");
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
+  static_assert(kOCol + 2 * kNPV <= kTmemCols, "tensor memory budget");
+};
 
-// tcgen05 instruction descriptor, kind::f16, fp32 accumulate, M = 128, N = 16.
-__host__ __device__ constexpr uint32_t idesc_f16(uint32_t ab_fmt, uint32_t a_mn, uint32_t b_mn) {
+// tcgen05 instruction descriptor, kind::f16, fp32 accumulate, M = 128.
+__host__ __device__ constexpr uint32_t idesc_f16(uint32_t ab_fmt, uint32_t a_mn, uint32_t b_mn,
+                                                 uint32_t n) {
   return (1u << 4) | (ab_fmt << 7) | (ab_fmt << 10) | (a_mn << 15) | (b_mn << 16) |
-         (uint32_t(kN >> 3) << 17) | (uint32_t(kTileTok >> 4) << 24);
+         ((n >> 3) << 17) | (uint32_t(kTileTok >> 4) << 24);
 }
 
 // Shared-memory matrix descriptor (sm_100 format, version 1).
@@ -104,8 +114,22 @@ __device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, float (&v)[NG]) {
                    "=r"(r[6]), "=r"(r[7])
                  : "r"(taddr)
                  : "memory");
+  } else if constexpr (NG == 32) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+        "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
+        "%28, %29, %30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+          "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+          "=r"(r[31])
+        : "r"(taddr)
+        : "memory");
   } else {
-    static_assert(NG == 16, "group padded to 4, 8 or 16");
+    static_assert(NG == 16, "4, 8, 16 or 32 columns");
+
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
         "%11, %12, %13, %14, %15}, [%16];"
@@ -159,17 +183,23 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
     const __grid_constant__ CUtensorMap qmap, const DecodeArgs a, int64_t num_units) {
   using namespace tc;
   static_assert(BS == 16 || BS == 32, "block_size 16 or 32");
+  using L = tc::Cfg<NG>;
+  constexpr int kStages = L::kStages;
+  constexpr int kPBytes = L::kPBytes;
+  constexpr int kNPV = L::kNPV;
   constexpr int kBlocksPerTile = kTileTok / BS;
   constexpr uint32_t kFmt = std::is_same<T, __half>::value ? 0u : 1u;
-  constexpr uint32_t kIdescQK = idesc_f16(kFmt, 0, 0);  // A = K (K-major), B = Q (K-major)
-  constexpr uint32_t kIdescPV = idesc_f16(kFmt, 1, 0);  // A = V^T (MN-major), B = P^T (K-major)
+  // A = K (K-major), B = Q (K-major), N = 16
+  constexpr uint32_t kIdescQK = idesc_f16(kFmt, 0, 0, kN);
+  // A = V^T (MN-major), B = P^T (K-major, hi and lo rows), N = kNPV
+  constexpr uint32_t kIdescPV = idesc_f16(kFmt, 1, 0, kNPV);
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align_1024(smem_raw);
-  uint8_t* ring = smem + kOffRing;
-  uint8_t* qbuf = smem + kOffQ;
-  uint8_t* pbuf = smem + kOffP;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
+  uint8_t* ring = smem + L::kOffRing;
+  uint8_t* qbuf = smem + L::kOffQ;
+  uint8_t* pbuf = smem + L::kOffP;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kOffBar);
   uint64_t* full = bars;                   // [kStages]
   uint64_t* empty = bars + kStages;        // [kStages]
   uint64_t* q_full = empty + kStages;      // [2]
@@ -182,9 +212,9 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
   uint64_t* o_free = o_full + 2;           // [2]
   uint64_t* red_bar = o_free + 2;          // [2] chunk maxima of the 4 softmax warps
   uint64_t* lred_bar = red_bar + 2;        // [2] unit sums of the 4 softmax warps
-  float* red = reinterpret_cast<float*>(smem + kOffRed);
-  float* redl = reinterpret_cast<float*>(smem + kOffRedL);
-  uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + kOffTmemPtr);
+  float* red = reinterpret_cast<float*>(smem + L::kOffRed);
+  float* redl = reinterpret_cast<float*>(smem + L::kOffRedL);
+  uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + L::kOffTmemPtr);
   __shared__ int abort_flag;
 
   const int warp = threadIdx.x >> 5;
@@ -344,7 +374,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
           if (ok) ok = mbar_wait(&o_free[b], (use & 1u) ^ 1u, 0x7800u);
           tc_fence_after();
           const uint32_t p_addr = smem_u32(pbuf + b * kPBytes);
-          const uint32_t o_tmem = tmem_base + kOCol + b * kN;
+          const uint32_t o_tmem = tmem_base + kOCol + b * kNPV;
           for (int32_t t = 0; t < ntile && ok; ++t, ++ctr) {
             const uint32_t st = ctr % kStages;
             ok = mbar_wait(&full[st], (ctr / kStages) & 1u, 0x7900u);
@@ -353,9 +383,9 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
             const uint32_t v_addr = smem_u32(ring + st * kStageBytes);
 #pragma unroll
             for (int kk = 0; kk < kTileTok / 16; ++kk) {
-              const uint32_t pk = (t * kTileTok + kk * 16) / 8 * 256;
+              const uint32_t pk = (t * kTileTok + kk * 16) / 8 * L::kPLbo;
               umma_f16_ss(o_tmem, smem_desc(v_addr + kk * 2048, kRegionBytes, 1024, kLayoutSw128),
-                          smem_desc(p_addr + pk, 256, 128, kLayoutNone), kIdescPV,
+                          smem_desc(p_addr + pk, L::kPLbo, 128, kLayoutNone), kIdescPV,
                           (t > 0 || kk > 0) ? 1u : 0u);
             }
             umma_commit(&empty[st]);
@@ -456,13 +486,17 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
         for (int t = 0; t < kChunkTiles; ++t) {
           if (t < ntile) {
             const int tok = t * kTileTok + r;  // token within the chunk
-            uint8_t* prow = pb + (tok >> 3) * 256 + (tok & 7) * 2;
+            uint8_t* prow = pb + (tok >> 3) * L::kPLbo + (tok & 7) * 2;
 #pragma unroll
             for (int j = 0; j < NG; ++j) {
               const float pf = sv[t][j] == -INFINITY ? 0.f : exp2f(sv[t][j] - cmax[j]);
-              const uint16_t pbits = Elem<T>::from_float(pf);
-              psum[j] += Elem<T>::to_float2(uint32_t(pbits)).x;
-              *reinterpret_cast<uint16_t*>(prow + (j >> 3) * 128 + (j & 7) * 16) = pbits;
+              const uint16_t hi = Elem<T>::from_float(pf);
+              const float hf = Elem<T>::to_float2(uint32_t(hi)).x;
+              const uint16_t lo = Elem<T>::from_float(pf - hf);
+              psum[j] += hf + Elem<T>::to_float2(uint32_t(lo)).x;
+              const int jl = NG + j;
+              *reinterpret_cast<uint16_t*>(prow + (j >> 3) * 128 + (j & 7) * 16) = hi;
+              *reinterpret_cast<uint16_t*>(prow + (jl >> 3) * 128 + (jl & 7) * 16) = lo;
             }
           }
         }
@@ -495,8 +529,11 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
         ok = wait_all(&o_full[b], use & 1u, 0x7d00u);
         if (!ok) break;
         tc_fence_after();
+        float ov2[2 * NG];  // [hi columns | lo columns]
+        tmem_ld_cols<2 * NG>(tmem_base + lane_addr + kOCol + b * kNPV, ov2);
         float ov[NG];
-        tmem_ld_cols<NG>(tmem_base + lane_addr + kOCol + b * kN, ov);
+#pragma unroll
+        for (int j = 0; j < NG; ++j) ov[j] = ov2[j] + ov2[NG + j];
         tmem_ld_wait();
         tc_fence_before();
         __syncwarp();

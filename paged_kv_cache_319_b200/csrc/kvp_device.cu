@@ -13,6 +13,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <unordered_map>
 
 #include "kernels/cache_ops.cuh"
 #include "kernels/common.cuh"
@@ -49,15 +50,24 @@ int sm_count() {
   return n;
 }
 
-// Raises a kernel's dynamic shared-memory limit once per device.
+// Raises a kernel's dynamic shared-memory limit once per (kernel, device).
 template <typename K>
 cudaError_t ensure_smem(K kernel, int bytes) {
-  static std::atomic<uint64_t> done{0};
+  static std::mutex mu;
+  static std::unordered_map<const void*, uint64_t> done;  // kernel -> device bit mask
   const int d = current_device();
   const uint64_t bit = d < 64 ? (1ull << d) : 0;
-  if (bit && (done.load(std::memory_order_relaxed) & bit)) return cudaSuccess;
+  const void* key = reinterpret_cast<const void*>(kernel);
+  {
+    std::lock_guard<std::mutex> g(mu);
+    auto it = done.find(key);
+    if (bit && it != done.end() && (it->second & bit)) return cudaSuccess;
+  }
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-  if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_relaxed);
+  if (e == cudaSuccess && bit) {
+    std::lock_guard<std::mutex> g(mu);
+    done[key] |= bit;
+  }
   return e;
 }
 
@@ -135,11 +145,12 @@ template <typename T, int BS, int NG>
 int launch_tc(const CUtensorMap& km, const CUtensorMap& vm, const CUtensorMap& qm,
               const kvp::dev::DecodeArgs& a, cudaStream_t st) {
   auto k = kvp::dev::decode_tc_kernel<T, BS, NG>;
-  cudaError_t e = ensure_smem(k, kvp::dev::tc::kSmemBytes);
+  constexpr int smem = kvp::dev::tc::Cfg<NG>::kSmemBytes;
+  cudaError_t e = ensure_smem(k, smem);
   if (e != cudaSuccess) return cuda_fail(e, "decode (tensor cores): smem attribute");
   const int64_t units = int64_t(a.num_seqs) * a.num_kv_heads * a.pmax;
   const int grid = int(units < sm_count() ? units : sm_count());
-  k<<<grid, kvp::dev::tc::kThreads, kvp::dev::tc::kSmemBytes, st>>>(km, vm, qm, a, units);
+  k<<<grid, kvp::dev::tc::kThreads, smem, st>>>(km, vm, qm, a, units);
   e = cudaGetLastError();
   return e == cudaSuccess ? KVP_OK : cuda_fail(e, "decode (tensor cores): launch");
 }
