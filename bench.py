@@ -60,6 +60,35 @@ def peaks():
         return 6650.0, "fallback"
 
 
+# DRAM traffic (read + write) of one launch of each decode kernel, as a multiple of
+# its algorithmic bytes, from the ncu captures summarised in profiles/; valid only
+# while the kernel source hashes to the value it had when captured.
+PROFILED_TRAFFIC = {
+    "decode_simt": {"ratio": (1.242983e9 + 9.548288e6) / 1.235123281e9, "sha": "5d4d20f128bed01d",
+                    "files": ["common.cuh", "decode_simt.cuh"]},
+    "decode_tc": {"ratio": (701.80096e6 + 6.554368e6) / 701466464.0, "sha": "9917bd6aa78b9c79",
+                  "files": ["common.cuh", "decode_simt.cuh", "decode_tc.cuh"]},
+}
+
+
+def kernel_sha(files):
+    import hashlib
+
+    d = os.path.join(ROOT, "paged_kv_cache_319_b200", "csrc", "kernels")
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(d, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_per_launch(kernel, alg_bytes):
+    p = PROFILED_TRAFFIC[kernel]
+    if kernel_sha(p["files"]) != p["sha"]:
+        return None
+    return int(p["ratio"] * alg_bytes)
+
+
 def algorithmic_bytes(lens, g):
     """Bytes one attention call must move: K and V of every context token, q, out,
     block-table entries and context lengths."""
@@ -72,63 +101,87 @@ def algorithmic_bytes(lens, g):
 
 
 # ---------------------------------------------------------------- clocks (NVML)
-class ClockSampler:
-    """Samples SM clock and throttle reasons of one GPU every few ms while running."""
+REASON_BITS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+               "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80}
 
-    REASONS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
-               "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80}
+
+def _clock_worker(uuid, stop, out):
+    """Child process: samples the SM clock and throttle reasons every ~1 ms."""
+    try:
+        import pynvml as nv
+
+        nv.nvmlInit()
+        h = nv.nvmlDeviceGetHandleByUUID(uuid.encode())
+        reasons_fn = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        out.put(("max", nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)))
+        out.put(("ready", None))
+        buf = []
+        while not stop.is_set():
+            buf.append((time.time(), nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM), reasons_fn(h)))
+            time.sleep(0.001)
+        out.put(("samples", buf))
+    except Exception as e:  # pragma: no cover - depends on the box
+        out.put(("error", repr(e)))
+        out.put(("samples", []))
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons of one GPU from a separate process (no
+    GIL contention) and keeps the samples taken inside the ``with`` block."""
 
     def __init__(self, torch_device):
+        import multiprocessing as mp
+
+        import torch
+
+        self.uuid = "GPU-" + str(torch.cuda.get_device_properties(torch_device).uuid)
+        ctx = mp.get_context("spawn")
+        self._stop = ctx.Event()
+        self._q = ctx.Queue()
+        self._p = ctx.Process(target=_clock_worker, args=(self.uuid, self._stop, self._q),
+                              daemon=True)
+        self._p.start()
+        self.max_mhz, self.error, self.window = None, None, (0.0, 0.0)
+        while True:  # wait until the child samples
+            kind, v = self._q.get(timeout=60)
+            if kind == "max":
+                self.max_mhz = v
+            elif kind == "error":
+                self.error = v
+            if kind in ("ready", "samples"):
+                break
         self.samples = []
-        self.reasons = set()
-        self.max_mhz = None
-        self._stop = threading.Event()
-        self._h = None
-        try:
-            import pynvml
-
-            pynvml.nvmlInit()
-            import torch
-
-            uuid = "GPU-" + str(torch.cuda.get_device_properties(torch_device).uuid)
-            self._h = pynvml.nvmlDeviceGetHandleByUUID(uuid.encode())
-            self._nv = pynvml
-            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
-        except Exception as e:  # pragma: no cover - depends on the box
-            self.error = repr(e)
-
-    def _run(self):
-        nv = self._nv
-        while not self._stop.is_set():
-            try:
-                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
-                fn = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
-                    nv.nvmlDeviceGetCurrentClocksThrottleReasons
-                r = fn(self._h)
-                for name, bit in self.REASONS.items():
-                    if r & bit:
-                        self.reasons.add(name)
-            except Exception:
-                pass
-            time.sleep(0.002)
 
     def __enter__(self):
-        if self._h is not None:
-            self._t = threading.Thread(target=self._run, daemon=True)
-            self._t.start()
+        self._t0 = time.time()
         return self
 
     def __exit__(self, *a):
+        self.window = (self._t0, time.time())
         self._stop.set()
-        if self._h is not None:
-            self._t.join()
+        try:
+            while True:
+                kind, v = self._q.get(timeout=30)
+                if kind == "samples":
+                    self.samples = v
+                    break
+                if kind == "error":
+                    self.error = v
+        except Exception:
+            pass
+        self._p.join(timeout=10)
 
     def summary(self):
-        if not self.samples:
-            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
-                    "samples": 0}
-        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
-                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+        t0, t1 = self.window
+        inside = [(c, r) for t, c, r in self.samples if t0 <= t <= t1]
+        reasons = sorted({n for _, r in inside for n, b in REASON_BITS.items() if r & b})
+        res = {"sm_mhz": float(statistics.median([c for c, _ in inside])) if inside else None,
+               "sm_max_mhz": self.max_mhz, "reasons": reasons, "samples": len(inside),
+               "window_ms": round((t1 - t0) * 1e3, 1)}
+        if self.error:
+            res["error"] = self.error
+        return res
 
 
 # ---------------------------------------------------------------- distributed
@@ -181,6 +234,11 @@ def barrier(world):
         dist.barrier()
 
 
+def make_workload(args):
+    kw = {} if getattr(args, "num_seqs", None) is None else {"num_seqs": args.num_seqs}
+    return workloads.by_name(args.workload, **kw)
+
+
 # ---------------------------------------------------------------- our arm
 class Replica:
     """One copy of the one-layer workload: host pool, sequences, device KV pool."""
@@ -218,7 +276,7 @@ def run_ours(args, world, rank, local):
 
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
-    wl = workloads.by_name(args.workload)
+    wl = make_workload(args)
     g = wl.geometry
     part = wl.partition_size if args.partition is None else args.partition
     ctx = np.asarray(wl.info["context_lens"], dtype=np.int64)
@@ -311,6 +369,7 @@ def run_ours(args, world, rank, local):
         ev.record(stream)
         done[b] = ev
 
+    clk = ClockSampler(device)  # started before warm-up so the GPU is not idle before timing
     for i in range(W):
         step(i, False)
     torch.cuda.synchronize(device)
@@ -319,7 +378,7 @@ def run_ours(args, world, rank, local):
     torch.cuda.synchronize(device)
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
-    with ClockSampler(device) as clk:
+    with clk:
         t0.record(stream)
         for i in range(W, W + K):
             step(i, True)
@@ -331,6 +390,7 @@ def run_ours(args, world, rank, local):
     max_ms = dist_max(elapsed_ms, world)
     total_bytes = dist_sum(float(sum(step_bytes)), world)
     total_tokens = dist_sum(float(sum(step_tokens)), world)
+    kernel_name = "decode_tc" if g.num_q_heads > g.num_kv_heads else "decode_simt"
     dec_ms = [a.elapsed_time(b) for a, b in ev_pairs]
     dec_avg_ms = sum(dec_ms) / len(dec_ms)
     dec_bytes_avg = sum(step_bytes) / len(step_bytes)
@@ -373,7 +433,7 @@ def run_ours(args, world, rank, local):
         "hbm_frac_of_step": round(value / peak, 4),
         "gpu_launches": int(sum(launches)),
         "roofline": {
-            "kernel": "paged_attention_decode (pass 1 + split reduce)",
+            "kernel": f"paged_attention_decode: {kernel_name} + decode_reduce_kernel",
             "bound": "hbm",
             "achieved": round(achieved, 1),
             "peak": peak,
@@ -381,7 +441,9 @@ def run_ours(args, world, rank, local):
             "unit": "GB/s",
             "frac": round(achieved / peak, 4),
             "frac_of_nominal_8tbs": round(achieved / 8000.0, 4),
-            "traffic": None,
+            "traffic": traffic_per_launch(kernel_name, dec_bytes_avg),
+            "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum of one launch "
+                              "(profiles/), scaled by algorithmic bytes; null if the kernel changed",
             "avg_launch_us": round(dec_avg_ms * 1e3, 2),
             "algorithmic_bytes_per_launch": int(dec_bytes_avg),
         },
@@ -494,7 +556,7 @@ def run_reference(args, world, rank):
         return
     from oracle.replay import OracleReplay
 
-    wl = workloads.by_name(args.workload)
+    wl = make_workload(args)
     rp = OracleReplay(wl)
     rp.run()
     (i, seqs, tables, lens), = rp.attends[-1:]
@@ -537,6 +599,8 @@ def main():
     ap.add_argument("--workload", default="opt13b",
                     choices=["opt13b", "gqa_long_bs16", "gqa_long_bs32"])
     ap.add_argument("--partition", type=int, default=None)
+    ap.add_argument("--num-seqs", type=int, default=None,
+                    help="smaller batch of the same workload (profiling small cases)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--ref-seqs-per-step", type=int, default=1)

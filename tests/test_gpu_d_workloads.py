@@ -16,7 +16,10 @@ import workloads
 pytestmark = pytest.mark.gpu
 
 
-def replay_pair(wl):
+def replay_pair(wl, rows_of=None):
+    """Runs both sides. The oracle decodes each attend op when it happens (later
+    steps may reuse released blocks), on the rows ``rows_of(lens)`` (default: all);
+    the references are returned by op index."""
     from paged_kv_cache_319_b200.replay import DeviceReplay
     import paged_kv_cache_319_b200 as kvp
 
@@ -24,8 +27,14 @@ def replay_pair(wl):
     dev.run()
     kvp.check_device_error()
     ora = OracleReplay(wl)
-    ora.run()
-    return dev, ora
+    refs = {}
+
+    def on_attend(i, seqs, tables, lens):
+        rows = None if rows_of is None else rows_of(lens)
+        refs[i] = (rows, ora.decode(i, tables, lens.tolist(), seqs=rows))
+
+    ora.run(attend=on_attend)
+    return dev, ora, refs
 
 
 def bookkeeping_equal(dev, ora):
@@ -48,17 +57,17 @@ def pools_equal(dev, ora):
                                      ("beam", {"steps": 16})])
 def test_small_workloads_every_output(name, kw):
     wl = workloads.by_name(name, **kw)
-    dev, ora = replay_pair(wl)
+    dev, ora, refs = replay_pair(wl)
     bookkeeping_equal(dev, ora)
     pools_equal(dev, ora)
-    for (i, seqs, t, l) in ora.attends:
-        ref = ora.decode(i, t, l)
+    assert refs
+    for i, (rows, ref) in refs.items():
         check_close(to_bits(dev.outputs[i]), ref, wl.geometry.dtype)
 
 
 def test_sharing_b_made_the_expected_copies():
     wl = workloads.sharing_sampling("B")
-    dev, _ = replay_pair(wl)
+    dev, _, _ = replay_pair(wl)
     copies = [p for (_, k, payload) in dev.events if k == "sync" for p in payload]
     assert len(copies) == 8 * 7
     st = dev.pool.stats()
@@ -76,34 +85,29 @@ def sampled(lens, n=6):
 
 def test_opt13b_full_size():
     wl = workloads.opt13b()
-    dev, ora = replay_pair(wl)
+    dev, ora, refs = replay_pair(wl, lambda l: sampled(l, 8))
     bookkeeping_equal(dev, ora)
     pools_equal(dev, ora)
-    (i, seqs, t, l), = ora.attends
-    rows = sampled(l, 8)
-    ref = ora.decode(i, t, l, seqs=rows)
+    (i, (rows, ref)), = refs.items()
     err, rel = check_close(to_bits(dev.outputs[i]), ref, "f16", rows=rows)
     assert err < 2e-3
 
 
 def test_llama13b_churn():
     wl = workloads.llama13b_churn(steps=4)
-    dev, ora = replay_pair(wl)
+    dev, ora, refs = replay_pair(wl, lambda l: sampled(l, 6))
     bookkeeping_equal(dev, ora)
     pools_equal(dev, ora)
-    for (i, seqs, t, l) in ora.attends:
-        rows = sampled(l, 6)
-        ref = ora.decode(i, t, l, seqs=rows)
+    assert len(refs) == 4
+    for i, (rows, ref) in refs.items():
         check_close(to_bits(dev.outputs[i]), ref, "f16", rows=rows)
 
 
 @pytest.mark.parametrize("bs", [16, 32])
 def test_gqa_long_full_size(bs):
     wl = workloads.gqa_long(bs)
-    dev, ora = replay_pair(wl)
+    dev, ora, refs = replay_pair(wl, lambda l: sampled(l, 2))
     bookkeeping_equal(dev, ora)
-    (i, seqs, t, l), = ora.attends
-    rows = sampled(l, 2)
-    ref = ora.decode(i, t, l, seqs=rows)
+    (i, (rows, ref)), = refs.items()
     err, rel = check_close(to_bits(dev.outputs[i]), ref, "bf16", rows=rows)
     assert err < 2e-3
