@@ -260,6 +260,38 @@ KVP_API int paged_attention_decode(const void* q, const void* k_cache, const voi
                            int32_t partition_size, void* workspace, size_t workspace_bytes,
                            void* out, int32_t dtype, kvp_stream_t stream);
 
+/* Largest split-context scratch, in bytes, that paged_attention_decode_noalloc
+ * can serve from its built-in area (40 MiB). */
+#define KVP_STATIC_SCRATCH_BYTES (40u * 1024u * 1024u)
+
+/* paged_attention_decode without a workspace argument, for callers that cannot
+ * allocate device memory: for example a serving engine whose allocator has
+ * already reserved all free device memory for its KV pool, or a latency-
+ * critical path that cannot afford cudaMalloc's implicit synchronisation. The
+ * paper has no counterpart to this entry point; it is a convenience of this
+ * library.
+ * The split-context scratch lives in one static device array of
+ * KVP_STATIC_SCRATCH_BYTES inside the library; every GPU that loads the
+ * library holds that memory until the process exits. The call allocates
+ * nothing: inputs and outputs are the caller's, as for
+ * paged_attention_decode, and the arguments and results are the same.
+ * The first call on a device looks up the array's device address on that
+ * device (with it current); make that first call before any stream capture.
+ * All calls share the one array and it keeps the last call's contents;
+ * nothing in it needs to start at zero (each call writes every partial it
+ * later reads), but calls whose kernels overlap on the GPU (different streams,
+ * or several host threads) race on it and must be serialised by the caller.
+ * Errors: those of paged_attention_decode, and KVP_ERR_INVALID when the batch
+ * needs more scratch than KVP_STATIC_SCRATCH_BYTES (kvp_decode_workspace_bytes
+ * gives the need; the message states both sizes). */
+KVP_API int paged_attention_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,
+                           const int32_t* block_tables, const int32_t* context_lens,
+                           int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
+                           int32_t head_dim, int32_t block_size, int32_t num_blocks,
+                           int32_t max_blocks_per_seq, int32_t max_context_len, float scale,
+                           int32_t partition_size, void* out, int32_t dtype,
+                           kvp_stream_t stream);
+
 /* Synchronises `stream`, then reads and clears the device error word of the
  * current device: KVP_OK, or KVP_ERR_BOUNDS if a kernel skipped an
  * out-of-range index since the last check (the message names the first). */

@@ -17,6 +17,7 @@ KVP_ERR_BOUNDS = -5
 KVP_ERR_CAPACITY = -6
 KVP_F16 = 0
 KVP_BF16 = 1
+KVP_STATIC_SCRATCH_BYTES = 40 * 1024 * 1024  # include/kvp.h
 
 ERROR_KINDS = {
     KVP_ERR_INVALID: "invalid",
@@ -71,6 +72,8 @@ SIGNATURES = {
     "kvp_decode_workspace_bytes": (sz, [i32, i32, i32, i32, i32]),
     "paged_attention_decode": (C.c_int, [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32,
                                          i32, f32, i32, vp, sz, vp, i32, vp]),
+    "paged_attention_decode_noalloc": (C.c_int, [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,
+                                                 i32, i32, f32, i32, vp, i32, vp]),
     "kvp_check_device_error": (C.c_int, [vp]),
     "kvp_last_error_message": (C.c_char_p, []),
     "kvp_version": (C.c_char_p, []),

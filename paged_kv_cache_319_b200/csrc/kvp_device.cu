@@ -370,3 +370,57 @@ int kvp_check_device_error(kvp_stream_t stream) {
 }
 
 }  // extern "C"
+
+// ---- decode for callers that cannot allocate device memory ------------------------
+// The split-context scratch of paged_attention_decode_noalloc: one static array
+// in this module, so every GPU that loads the library holds it until exit. Host
+// code must not pass the symbol itself to a kernel (on the host it names a
+// host-side stand-in); its device address is looked up once per device below.
+static __device__ __align__(256) unsigned char g_static_decode_scratch[KVP_STATIC_SCRATCH_BYTES];
+
+namespace {
+
+std::mutex g_static_scratch_mu;
+void* g_static_scratch_ptr[kMaxDevices] = {};
+
+// Device address of the static scratch on the current device (looked up on the
+// first call for each device, with that device current).
+int static_scratch_address(void** out) {
+  const int d = current_device();
+  if (d < 0 || d >= kMaxDevices) return fail(KVP_ERR_INVALID, "device index %d out of range", d);
+  std::lock_guard<std::mutex> g(g_static_scratch_mu);
+  if (!g_static_scratch_ptr[d]) {
+    void* p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_static_decode_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "paged_attention_decode_noalloc: scratch address");
+    g_static_scratch_ptr[d] = p;
+  }
+  *out = g_static_scratch_ptr[d];
+  return KVP_OK;
+}
+
+}  // namespace
+
+extern "C" int paged_attention_decode_noalloc(
+    const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
+    const int32_t* context_lens, int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
+    int32_t head_dim, int32_t block_size, int32_t num_blocks, int32_t max_blocks_per_seq,
+    int32_t max_context_len, float scale, int32_t partition_size, void* out, int32_t dtype,
+    kvp_stream_t stream) {
+  const size_t need = kvp_decode_workspace_bytes(num_seqs, num_q_heads, head_dim, max_context_len,
+                                                 partition_size);
+  if (need > size_t(KVP_STATIC_SCRATCH_BYTES))
+    return fail(KVP_ERR_INVALID,
+                "paged_attention_decode_noalloc: this batch needs %zu bytes of split-context "
+                "scratch; the static area holds %zu (use paged_attention_decode with a workspace)",
+                need, size_t(KVP_STATIC_SCRATCH_BYTES));
+  void* ws = nullptr;
+  if (need > 0) {
+    const int rc = static_scratch_address(&ws);
+    if (rc) return rc;
+  }
+  return paged_attention_decode(q, k_cache, v_cache, block_tables, context_lens, num_seqs,
+                                num_q_heads, num_kv_heads, head_dim, block_size, num_blocks,
+                                max_blocks_per_seq, max_context_len, scale, partition_size, ws,
+                                need > 0 ? size_t(KVP_STATIC_SCRATCH_BYTES) : 0, out, dtype, stream);
+}
