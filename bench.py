@@ -260,7 +260,7 @@ class Replica:
         self.v = torch.zeros(shape, dtype=tdt, device=device)
         st = torch.tensor(slots, dtype=torch.int64, device=device)
         kvp.reshape_and_cache(prefill_k, prefill_v, self.k, self.v, st)
-        self.lens = np.asarray(start_lens, dtype=np.int64)
+        self.lens = np.array(start_lens, dtype=np.int64)  # own copy per replica
 
 
 def to_dev(bits, dtype, device):
@@ -362,8 +362,10 @@ def run_ours(args, world, rank, local):
             e1 = torch.cuda.Event(enable_timing=True)
             e1.record(stream)
             ev_pairs.append((e0, e1))
-            step_bytes.append(algorithmic_bytes(rep.lens, g))
-            step_tokens.append(int(rep.lens.sum()))
+            packed = len_h[b].numpy()  # the lengths this step's kernels read
+            assert np.array_equal(packed, rep.lens)
+            step_bytes.append(algorithmic_bytes(packed, g))
+            step_tokens.append(int(packed.sum()))
             launches.append(n_launch)
         ev = torch.cuda.Event()
         ev.record(stream)
@@ -508,7 +510,7 @@ def run_e2e(args, wl, reps, device, seed_rank, MB, max_ctx_total, part, ws, worl
                                    max_context_len=max_ctx_total, partition_size=part, workspace=ws)
         host_out.copy_(out.view(torch.int16), non_blocking=True)
         torch.cuda.current_stream(device).synchronize()
-        total_bytes += algorithmic_bytes(rep.lens, g)
+        total_bytes += algorithmic_bytes(len_h.numpy(), g)
     el = time.perf_counter() - t
     el = dist_max(el, world)
     total_bytes = dist_sum(float(total_bytes), world)

@@ -23,6 +23,15 @@
 
 using kvp::fail;
 
+// Launch shape of the CUDA-core decode kernel: warps per CTA and TMA stages per
+// warp (shared memory per CTA = warps x stages x 2 tiles + merge area).
+#ifndef KVP_SIMT_WARPS
+#define KVP_SIMT_WARPS 4
+#endif
+#ifndef KVP_SIMT_STAGES
+#define KVP_SIMT_STAGES 3
+#endif
+
 namespace {
 
 constexpr int kMaxDevices = 64;
@@ -130,7 +139,7 @@ Workspace ws_layout(int64_t S, int64_t Hq, int64_t D, int64_t pmax) {
 template <typename T, int D, int BS>
 int launch_simt(const CUtensorMap& km, const CUtensorMap& vm, const kvp::dev::DecodeArgs& a,
                 cudaStream_t st) {
-  constexpr int NW = 4, NST = 3;
+  constexpr int NW = KVP_SIMT_WARPS, NST = KVP_SIMT_STAGES;
   using C = kvp::dev::SimtCfg<T, D, BS, NW, NST>;
   auto k = kvp::dev::decode_simt_kernel<T, D, BS, NW, NST>;
   cudaError_t e = ensure_smem(k, C::kSmemBytes);
