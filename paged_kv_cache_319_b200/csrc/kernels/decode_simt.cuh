@@ -100,6 +100,9 @@ __global__ void __launch_bounds__(NW * 32) decode_simt_kernel(
   const int h = blockIdx.y;
   const int s = blockIdx.z;
 
+  // The split-context reduce may be scheduled as soon as every CTA of this grid
+  // has started; it waits for this grid to complete before reading partials.
+  pdl_trigger();
   const int32_t ctx = load_ctx(a, s, p == 0 && h == 0 && threadIdx.x == 0);
   const int32_t nblk = (ctx + BS - 1) / BS;
   const int32_t nparts = (nblk + a.part_blocks - 1) / a.part_blocks;
@@ -356,6 +359,7 @@ __global__ void __launch_bounds__(NW * 32) decode_simt_kernel(
 template <typename T, int D>
 __global__ void __launch_bounds__(D) decode_reduce_kernel(const DecodeArgs a) {
   extern __shared__ float wsh[];  // [pmax] weights
+  pdl_wait();  // launched programmatically: the partition kernel must be complete
   const int h = blockIdx.x;
   const int s = blockIdx.y;
   const int32_t ctx = load_ctx(a, s, false);

@@ -219,6 +219,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  pdl_trigger();  // the split-context reduce waits for this grid to complete
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStages; ++i) {

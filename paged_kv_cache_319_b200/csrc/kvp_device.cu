@@ -24,12 +24,16 @@
 using kvp::fail;
 
 // Launch shape of the CUDA-core decode kernel: warps per CTA and TMA stages per
-// warp (shared memory per CTA = warps x stages x 2 tiles + merge area).
+// warp (shared memory per CTA = warps x stages x 2 tiles + merge area). The
+// kernel is bound by per-warp latency more than by bytes in flight: on the
+// OPT-13B geometry, 4 warps x 2 stages (67 KB, 3 CTAs = 12 warps per SM) ran
+// at 190.5 us per call against 231.9 us for 4 x 3 (2 CTAs per SM). Tiles of
+// 8 KB (block size 32) use half the warps to keep about 64 KB per CTA.
 #ifndef KVP_SIMT_WARPS
 #define KVP_SIMT_WARPS 4
 #endif
 #ifndef KVP_SIMT_STAGES
-#define KVP_SIMT_STAGES 3
+#define KVP_SIMT_STAGES 2
 #endif
 
 namespace {
@@ -139,7 +143,8 @@ Workspace ws_layout(int64_t S, int64_t Hq, int64_t D, int64_t pmax) {
 template <typename T, int D, int BS>
 int launch_simt(const CUtensorMap& km, const CUtensorMap& vm, const kvp::dev::DecodeArgs& a,
                 cudaStream_t st) {
-  constexpr int NW = KVP_SIMT_WARPS, NST = KVP_SIMT_STAGES;
+  constexpr int NW = (BS * D * 2 >= 8192 && KVP_SIMT_WARPS > 1) ? KVP_SIMT_WARPS / 2 : KVP_SIMT_WARPS;
+  constexpr int NST = KVP_SIMT_STAGES;
   using C = kvp::dev::SimtCfg<T, D, BS, NW, NST>;
   auto k = kvp::dev::decode_simt_kernel<T, D, BS, NW, NST>;
   cudaError_t e = ensure_smem(k, C::kSmemBytes);
@@ -166,10 +171,20 @@ int launch_tc(const CUtensorMap& km, const CUtensorMap& vm, const CUtensorMap& q
 
 template <typename T, int D>
 int launch_reduce(const kvp::dev::DecodeArgs& a, cudaStream_t st) {
-  auto k = kvp::dev::decode_reduce_kernel<T, D>;
-  dim3 grid(a.num_q_heads, a.num_seqs);
-  k<<<grid, D, size_t(a.pmax) * 4, st>>>(a);
-  cudaError_t e = cudaGetLastError();
+  // Programmatic dependent launch: the reduce's launch overlaps the tail of the
+  // partition kernel; the kernel itself waits (griddepcontrol.wait) for it.
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(a.num_q_heads, a.num_seqs);
+  cfg.blockDim = dim3(D);
+  cfg.dynamicSmemBytes = size_t(a.pmax) * 4;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kvp::dev::decode_reduce_kernel<T, D>, a);
+  if (e == cudaSuccess) e = cudaGetLastError();
   return e == cudaSuccess ? KVP_OK : cuda_fail(e, "decode reduce: launch");
 }
 
