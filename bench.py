@@ -64,7 +64,7 @@ def peaks():
 # its algorithmic bytes, from the ncu captures summarised in profiles/; valid only
 # while the kernel source hashes to the value it had when captured.
 PROFILED_TRAFFIC = {
-    "decode_simt": {"ratio": (1.242983e9 + 9.548288e6) / 1.235123281e9, "sha": "5d4d20f128bed01d",
+    "decode_simt": {"ratio": (1.243084e9 + 4.710656e6) / 1.235123281e9, "sha": "a8c77b0d95e41575",
                     "files": ["common.cuh", "decode_simt.cuh"]},
     "decode_tc": {"ratio": (701.80096e6 + 6.554368e6) / 701466464.0, "sha": "9917bd6aa78b9c79",
                   "files": ["common.cuh", "decode_simt.cuh", "decode_tc.cuh"]},
@@ -263,6 +263,31 @@ class Replica:
         self.lens = np.array(start_lens, dtype=np.int64)  # own copy per replica
 
 
+class StepMeta:
+    """One step's metadata in one pinned buffer (slots int64 [S], lengths int32 [S],
+    block tables int32 [S, MB]) and its device mirror, so one H2D copy moves it all."""
+
+    def __init__(self, S, MB, device):
+        import torch
+
+        nbytes = S * 8 + S * 4 + S * MB * 4
+        self.host = torch.empty(nbytes, dtype=torch.uint8).pin_memory()
+        self.dev = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        self.nbytes = nbytes
+
+        def views(buf):
+            slots = buf[: S * 8].view(torch.int64)
+            lens = buf[S * 8: S * 12].view(torch.int32)
+            tables = buf[S * 12:].view(torch.int32).view(S, MB)
+            return slots, lens, tables
+
+        self.slot_h, self.len_h, self.tab_h = views(self.host)
+        self.slot_d, self.len_d, self.tab_d = views(self.dev)
+
+    def upload(self):
+        self.dev.copy_(self.host, non_blocking=True)
+
+
 def to_dev(bits, dtype, device):
     import torch
 
@@ -314,13 +339,7 @@ def run_ours(args, world, rank, local):
     max_ctx_total = int(start.max()) + grow
     MB = -(-max_ctx_total // g.block_size)
     NBUF = 3
-    pin = lambda shape, dt: torch.empty(shape, dtype=dt, pin_memory=True)
-    slot_h = [pin((S,), torch.int64) for _ in range(NBUF)]
-    tab_h = [pin((S, MB), torch.int32) for _ in range(NBUF)]
-    len_h = [pin((S,), torch.int32) for _ in range(NBUF)]
-    slot_d = [torch.empty((S,), dtype=torch.int64, device=device) for _ in range(NBUF)]
-    tab_d = [torch.empty((S, MB), dtype=torch.int32, device=device) for _ in range(NBUF)]
-    len_d = [torch.empty((S,), dtype=torch.int32, device=device) for _ in range(NBUF)]
+    meta = [StepMeta(S, MB, device) for _ in range(NBUF)]
     done = [None] * NBUF
     out = torch.empty((S, g.num_q_heads, g.head_dim), dtype=qs[0].dtype, device=device)
     ws_bytes = kvp.decode_workspace_bytes(S, g.num_q_heads, g.head_dim, max_ctx_total, part)
@@ -335,26 +354,24 @@ def run_ours(args, world, rank, local):
         b = i % NBUF
         if done[b] is not None:
             done[b].synchronize()
-        slots_np = slot_h[b].numpy()
-        rep.pool.append_batch(rep.seqs, 1, out=slots_np)
+        m = meta[b]
+        rep.pool.append_batch(rep.seqs, 1, out=m.slot_h.numpy())
         copies = rep.pool.take_copies()
-        rep.pool.build_batch(rep.seqs, MB, tab_h[b].numpy(), len_h[b].numpy())
+        rep.pool.build_batch(rep.seqs, MB, m.tab_h.numpy(), m.len_h.numpy())
         rep.lens += 1
-        slot_d[b].copy_(slot_h[b], non_blocking=True)
-        tab_d[b].copy_(tab_h[b], non_blocking=True)
-        len_d[b].copy_(len_h[b], non_blocking=True)
+        m.upload()
         n_launch = 0
         if copies:
             pairs = torch.tensor(copies, dtype=torch.int32).to(device, non_blocking=True)
             kvp.copy_blocks(rep.k, rep.v, pairs)
             n_launch += 1
         j = i % NI
-        kvp.reshape_and_cache(kn[j], vn[j], rep.k, rep.v, slot_d[b])
+        kvp.reshape_and_cache(kn[j], vn[j], rep.k, rep.v, m.slot_d)
         n_launch += 1
         if timed:
             e0 = torch.cuda.Event(enable_timing=True)
             e0.record(stream)
-        kvp.paged_attention_decode(qs[j], rep.k, rep.v, tab_d[b], len_d[b], wl.scale, out,
+        kvp.paged_attention_decode(qs[j], rep.k, rep.v, m.tab_d, m.len_d, wl.scale, out,
                                    max_context_len=max_ctx_total, partition_size=part,
                                    workspace=ws)
         n_launch += 2 if (part and int(rep.lens.max()) > part) else 1
@@ -362,7 +379,7 @@ def run_ours(args, world, rank, local):
             e1 = torch.cuda.Event(enable_timing=True)
             e1.record(stream)
             ev_pairs.append((e0, e1))
-            packed = len_h[b].numpy()  # the lengths this step's kernels read
+            packed = m.len_h.numpy()  # the lengths this step's kernels read
             assert np.array_equal(packed, rep.lens)
             step_bytes.append(algorithmic_bytes(packed, g))
             step_tokens.append(int(packed.sum()))
@@ -474,18 +491,12 @@ def run_e2e(args, wl, reps, device, seed_rank, MB, max_ctx_total, part, ws, worl
     host_v = pin(torch.from_numpy(normal_bits(value_seed_words(seed_rank, V_STREAM, 999), (S, g.num_kv_heads, g.head_dim), g.dtype).view(np.int16)))
     tdt = torch.float16 if g.dtype == "f16" else torch.bfloat16
     host_out = torch.empty((S, g.num_q_heads, g.head_dim), dtype=torch.int16).pin_memory()
-    slot_h = torch.empty((S,), dtype=torch.int64).pin_memory()
-    tab_h = torch.empty((S, MB), dtype=torch.int32).pin_memory()
-    len_h = torch.empty((S,), dtype=torch.int32).pin_memory()
+    m = StepMeta(S, MB, device)
     q_d = torch.empty((S, g.num_q_heads, g.head_dim), dtype=tdt, device=device)
     k_d = torch.empty((S, g.num_kv_heads, g.head_dim), dtype=tdt, device=device)
     v_d = torch.empty_like(k_d)
     out = torch.empty_like(q_d)
-    slot_d = torch.empty((S,), dtype=torch.int64, device=device)
-    tab_d = torch.empty((S, MB), dtype=torch.int32, device=device)
-    len_d = torch.empty((S,), dtype=torch.int32, device=device)
-    h2d = (host_q.numel() + host_k.numel() + host_v.numel()) * 2 + slot_h.numel() * 8 + \
-        (tab_h.numel() + len_h.numel()) * 4
+    h2d = (host_q.numel() + host_k.numel() + host_v.numel()) * 2 + m.nbytes
     d2h = host_out.numel() * 2
     total_bytes = 0
     barrier(world)
@@ -493,24 +504,22 @@ def run_e2e(args, wl, reps, device, seed_rank, MB, max_ctx_total, part, ws, worl
     t = time.perf_counter()
     for i in range(K):
         rep = reps[i % R]
-        rep.pool.append_batch(rep.seqs, 1, out=slot_h.numpy())
+        rep.pool.append_batch(rep.seqs, 1, out=m.slot_h.numpy())
         copies = rep.pool.take_copies()
-        rep.pool.build_batch(rep.seqs, MB, tab_h.numpy(), len_h.numpy())
+        rep.pool.build_batch(rep.seqs, MB, m.tab_h.numpy(), m.len_h.numpy())
         rep.lens += 1
         q_d.view(torch.int16).copy_(host_q, non_blocking=True)
         k_d.view(torch.int16).copy_(host_k, non_blocking=True)
         v_d.view(torch.int16).copy_(host_v, non_blocking=True)
-        slot_d.copy_(slot_h, non_blocking=True)
-        tab_d.copy_(tab_h, non_blocking=True)
-        len_d.copy_(len_h, non_blocking=True)
+        m.upload()
         if copies:
             kvp.copy_blocks(rep.k, rep.v, torch.tensor(copies, dtype=torch.int32).to(device))
-        kvp.reshape_and_cache(k_d, v_d, rep.k, rep.v, slot_d)
-        kvp.paged_attention_decode(q_d, rep.k, rep.v, tab_d, len_d, wl.scale, out,
+        kvp.reshape_and_cache(k_d, v_d, rep.k, rep.v, m.slot_d)
+        kvp.paged_attention_decode(q_d, rep.k, rep.v, m.tab_d, m.len_d, wl.scale, out,
                                    max_context_len=max_ctx_total, partition_size=part, workspace=ws)
         host_out.copy_(out.view(torch.int16), non_blocking=True)
         torch.cuda.current_stream(device).synchronize()
-        total_bytes += algorithmic_bytes(len_h.numpy(), g)
+        total_bytes += algorithmic_bytes(m.len_h.numpy(), g)
     el = time.perf_counter() - t
     el = dist_max(el, world)
     total_bytes = dist_sum(float(total_bytes), world)

@@ -297,6 +297,15 @@ KVP_API int paged_attention_decode_noalloc(const void* q, const void* k_cache, c
  * out-of-range index since the last check (the message names the first). */
 KVP_API int kvp_check_device_error(kvp_stream_t stream);
 
+/* Diagnostic of the kernels' bounded waits: launches one CTA that waits, with
+ * the same bounded-wait code the decode kernels use but a limit of limit_ms
+ * (1..2000), for an mbarrier phase that nothing ever completes. The wait runs
+ * out, records a timeout in the device error word and the kernel returns; the
+ * next kvp_check_device_error() reports KVP_ERR_CUDA ("bounded wait timed
+ * out"), and the context stays usable. Asynchronous like the other device
+ * calls. */
+KVP_API int kvp_selftest_bounded_wait(int32_t limit_ms, kvp_stream_t stream);
+
 /* Description of the calling thread's last failure ("" if none). */
 KVP_API const char* kvp_last_error_message(void);
 

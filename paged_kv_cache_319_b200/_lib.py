@@ -75,6 +75,7 @@ SIGNATURES = {
     "paged_attention_decode_noalloc": (C.c_int, [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,
                                                  i32, i32, f32, i32, vp, i32, vp]),
     "kvp_check_device_error": (C.c_int, [vp]),
+    "kvp_selftest_bounded_wait": (C.c_int, [i32, vp]),
     "kvp_last_error_message": (C.c_char_p, []),
     "kvp_version": (C.c_char_p, []),
 }

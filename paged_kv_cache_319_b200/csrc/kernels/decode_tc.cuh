@@ -56,6 +56,9 @@ constexpr int kSCol = 0;                             // S buffers: [0, 128)
 constexpr int kOCol = 128;                           // O buffers: [128, 128 + 2 * kNPV)
 constexpr int kThreads = 192;
 constexpr int kSoftmaxThreads = 128;
+// Batches of up to this many sequences keep their context lengths in shared
+// memory, so no warp role waits on a global load when it moves to a new unit.
+constexpr int kCtxCacheMax = 4096;
 
 // Layout for a group width NG (query heads per KV head, padded to 4, 8 or 16).
 // P^T holds p split into a high part and a low part, both in the input type
@@ -75,12 +78,13 @@ struct Cfg {
   static constexpr int kOffRed = kOffBar + kNumBars * 8;     // [2 halves][4 warps][kN] maxima
   static constexpr int kOffRedL = kOffRed + 2 * 4 * kN * 4;  // [2 halves][4 warps][kN] sums
   static constexpr int kOffTmemPtr = kOffRedL + 2 * 4 * kN * 4;
-  static constexpr int kSmemBytes = 1024 + kOffTmemPtr + 16;
+  static constexpr int kOffCtx = kOffTmemPtr + 16;           // cached context lengths
+  static constexpr int kSmemBytes = 1024 + kOffCtx;          // + 4 bytes per cached length
   // The softmax warps wait for a chunk's last V tile (to zero rows past the
   // end of the sequence) before the PV MMAs free any stage of that chunk, so
   // the ring must hold a chunk's K tiles plus that V tile.
   static_assert(kStages >= kChunkTiles, "ring too shallow for one chunk");
-  static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
+  static_assert(kSmemBytes + 4 * kCtxCacheMax <= 227 * 1024, "shared memory budget");
   static_assert(kOCol + 2 * kNPV <= kTmemCols, "tensor memory budget");
 };
 
@@ -143,7 +147,10 @@ __device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, float (&v)[NG]) {
   for (int j = 0; j < NG; ++j) v[j] = __uint_as_float(r[j]);
 }
 
-// Work unit u -> (s, g, p) over the grid pmax x Hkv x S (p fastest).
+// Work unit u -> (s, p, g) over S x pmax x Hkv with the KV head fastest, so the
+// CTAs running at the same time read different heads of each block (different
+// offsets inside the blocks, spread over the HBM channels) rather than one head
+// of many blocks.
 struct Unit {
   int32_t s, g, p;
   int32_t tok_begin, tok_end;  // token range of the unit
@@ -151,13 +158,15 @@ struct Unit {
   int32_t nparts;
 };
 
-__device__ __forceinline__ bool decode_unit(const DecodeArgs& a, int64_t u, Unit& w) {
+// ctx_sm: the batch's clamped context lengths in shared memory, or null.
+__device__ __forceinline__ bool decode_unit(const DecodeArgs& a, int64_t u, Unit& w,
+                                            const int32_t* ctx_sm) {
   const int64_t per_seq = int64_t(a.pmax) * a.num_kv_heads;
   w.s = int32_t(u / per_seq);
   const int32_t rem = int32_t(u - int64_t(w.s) * per_seq);
-  w.g = rem / a.pmax;
-  w.p = rem - w.g * a.pmax;
-  w.ctx = load_ctx(a, w.s, false);
+  w.p = rem / a.num_kv_heads;
+  w.g = rem - w.p * a.num_kv_heads;
+  w.ctx = ctx_sm ? ctx_sm[w.s] : load_ctx(a, w.s, w.g == 0 && w.p == 0);
   w.nparts = (w.ctx + a.part_tokens - 1) / a.part_tokens;
   if (w.p > 0 && w.p >= w.nparts) return false;  // empty (p == 0 always runs)
   w.tok_begin = w.p * a.part_tokens;
@@ -174,6 +183,45 @@ __device__ __forceinline__ int32_t tiles_of(const Unit& w, int32_t c) {
   const int32_t c1 = min(w.tok_end, c0 + kChunkTok);
   return (c1 - c0 + kTileTok - 1) / kTileTok;
 }
+
+// The chunks a persistent CTA processes, in order: its units blockIdx.x,
+// blockIdx.x + gridDim.x, ... (empty partitions and units without tokens
+// skipped), each cut into chunks of up to kChunkTok tokens. Every warp role
+// walks the same stream.
+struct ChunkStream {
+  int64_t u, stride, num_units;
+  const int32_t* ctx_sm;
+  Unit w;
+  int32_t c, nch;
+  bool valid;
+
+  __device__ __forceinline__ void init(const DecodeArgs& a, int64_t first, int64_t step,
+                                       int64_t n, const int32_t* ctx_cache) {
+    ctx_sm = ctx_cache;
+    stride = step;
+    num_units = n;
+    u = first - step;
+    c = 0;
+    nch = 0;
+    valid = true;
+    next_unit(a);
+  }
+  __device__ __forceinline__ void next_unit(const DecodeArgs& a) {
+    for (u += stride; u < num_units; u += stride) {
+      if (decode_unit(a, u, w, ctx_sm) && (nch = chunks_of(w)) > 0) {
+        c = 0;
+        return;
+      }
+    }
+    valid = false;
+  }
+  __device__ __forceinline__ void advance(const DecodeArgs& a) {
+    if (++c >= nch) next_unit(a);
+  }
+  __device__ __forceinline__ int32_t tiles() const { return tiles_of(w, c); }
+  __device__ __forceinline__ bool first() const { return c == 0; }
+  __device__ __forceinline__ bool last() const { return c == nch - 1; }
+};
 
 }  // namespace tc
 
@@ -215,6 +263,12 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
   float* red = reinterpret_cast<float*>(smem + L::kOffRed);
   float* redl = reinterpret_cast<float*>(smem + L::kOffRedL);
   uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + L::kOffTmemPtr);
+  int32_t* ctx_cache = reinterpret_cast<int32_t*>(smem + L::kOffCtx);
+  const int32_t* ctx_sm = a.num_seqs <= kCtxCacheMax ? ctx_cache : nullptr;
+  if (ctx_sm) {
+    for (int i = threadIdx.x; i < a.num_seqs; i += blockDim.x)
+      ctx_cache[i] = load_ctx(a, i, blockIdx.x == 0);  // clamped; out-of-range reported once
+  }
   __shared__ int abort_flag;
 
   const int warp = threadIdx.x >> 5;
@@ -259,6 +313,8 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
+    // Ring order: K tiles of chunk 0, then for every chunk i: K tiles of chunk
+    // i + 1, V tiles of chunk i (the keys run one chunk ahead of the values).
     if (lane == 0) {
       prefetch_tensormap(&kmap);
       prefetch_tensormap(&vmap);
@@ -269,60 +325,76 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
     uint32_t ctr = 0;   // ring tiles issued
     uint32_t ucnt = 0;  // units started
     bool ok = true;
-    for (int64_t u = blockIdx.x; u < num_units && ok; u += gridDim.x) {
-      tc::Unit w;
-      if (!tc::decode_unit(a, u, w)) continue;
-      const int32_t nch = tc::chunks_of(w);
-      if (nch == 0) continue;
-      const uint32_t qb = ucnt & 1u;
-      if (lane == 0) {
-        ok = mbar_wait(&q_empty[qb], ((ucnt >> 1) & 1u) ^ 1u, 0x7100u);
-        if (ok) {
-          mbar_arrive_expect_tx(&q_full[qb], kQBytes);
-          const int32_t qrow = w.s * a.num_q_heads + w.g * G;
-          tma_load_2d(qbuf + qb * kQBytes, &qmap, &q_full[qb], 0, qrow, pol_q);
-          tma_load_2d(qbuf + qb * kQBytes + kN * 128, &qmap, &q_full[qb], 64, qrow, pol_q);
+    // Lane j's TMA row of block j of a chunk (one chunk = 512 / BS <= 32 blocks).
+    auto chunk_row = [&](const tc::ChunkStream& cs) -> int32_t {
+      const tc::Unit& w = cs.w;
+      const int32_t ntile = cs.tiles();
+      const int32_t blk0 = (w.tok_begin + cs.c * kChunkTok) / BS;
+      const int32_t nblk_seq = (w.ctx + BS - 1) / BS;
+      const int32_t bidx = blk0 + lane;
+      int32_t id = -1;
+      if (lane < ntile * kBlocksPerTile && bidx < nblk_seq) {
+        id = __ldg(a.block_tables + int64_t(w.s) * a.max_blocks_per_seq + bidx);
+        if (id < 0 || id >= a.num_blocks) {
+          record_error(KVP_DEVERR_BLOCK_ID, (uint64_t(w.s) << 32) | uint32_t(bidx));
+          id = -1;
         }
       }
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-      ++ucnt;
-      const int32_t* table = a.block_tables + int64_t(w.s) * a.max_blocks_per_seq;
-      for (int32_t c = 0; c < nch && ok; ++c) {
-        const int32_t ntile = tc::tiles_of(w, c);
-        const int32_t blk0 = (w.tok_begin + c * kChunkTok) / BS;
-        const int32_t nblk_seq = (w.ctx + BS - 1) / BS;
-        // lane j holds the id of block blk0 + j (one chunk = 512 / BS <= 32 blocks)
-        const int32_t bidx = blk0 + lane;
-        int32_t id = -1;
-        if (lane < ntile * kBlocksPerTile && bidx < nblk_seq) {
-          id = __ldg(table + bidx);
-          if (id < 0 || id >= a.num_blocks) {
-            record_error(KVP_DEVERR_BLOCK_ID, (uint64_t(w.s) << 32) | uint32_t(bidx));
-            id = -1;
-          }
+      return id < 0 ? rows_total : (id * a.num_kv_heads + w.g) * BS;
+    };
+    auto load_tiles = [&](const CUtensorMap* map, int32_t row, int32_t ntile) {
+      for (int32_t t = 0; t < ntile && ok; ++t, ++ctr) {
+        const uint32_t st = ctr % kStages;
+        if (lane == 0) {
+          ok = mbar_wait(&empty[st], ((ctr / kStages) & 1u) ^ 1u, 0x7200u);
+          if (ok) mbar_arrive_expect_tx(&full[st], kStageBytes);
         }
-        const int32_t row = id < 0 ? rows_total : (id * a.num_kv_heads + w.g) * BS;
-        for (int kv = 0; kv < 2 && ok; ++kv) {
-          const CUtensorMap* map = kv == 0 ? &kmap : &vmap;
-          for (int32_t t = 0; t < ntile && ok; ++t, ++ctr) {
-            const uint32_t st = ctr % kStages;
-            if (lane == 0) {
-              ok = mbar_wait(&empty[st], ((ctr / kStages) & 1u) ^ 1u, 0x7200u);
-              if (ok) mbar_arrive_expect_tx(&full[st], kStageBytes);
-            }
-            ok = __shfl_sync(0xffffffffu, ok, 0);
-            if (!ok) break;
-            const int j = lane - t * kBlocksPerTile;  // block j of this tile
-            if (j >= 0 && j < kBlocksPerTile) {
-              uint8_t* dst = ring + st * kStageBytes + j * BS * 128;
-              tma_load_2d(dst, map, &full[st], 0, row, pol_kv);
-              tma_load_2d(dst + kRegionBytes, map, &full[st], 64, row, pol_kv);
-            }
-            __syncwarp();
-          }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        const int j = lane - t * kBlocksPerTile;  // block j of this tile
+        if (j >= 0 && j < kBlocksPerTile) {
+          uint8_t* dst = ring + st * kStageBytes + j * BS * 128;
+          tma_load_2d(dst, map, &full[st], 0, row, pol_kv);
+          tma_load_2d(dst + kRegionBytes, map, &full[st], 64, row, pol_kv);
         }
+        __syncwarp();
       }
+    };
+    tc::ChunkStream cur;
+    cur.init(a, blockIdx.x, gridDim.x, num_units, ctx_sm);
+    int32_t pend_row = rows_total, pend_tiles = 0;
+    bool have_pend = false;
+    int32_t row = cur.valid ? chunk_row(cur) : rows_total;
+    while (cur.valid && ok) {
+      // the next chunk's block ids are loaded now and used one iteration later
+      tc::ChunkStream nxt = cur;
+      nxt.advance(a);
+      const int32_t row_next = nxt.valid ? chunk_row(nxt) : rows_total;
+      if (cur.first()) {
+        const uint32_t qb = ucnt & 1u;
+        if (lane == 0) {
+          ok = mbar_wait(&q_empty[qb], ((ucnt >> 1) & 1u) ^ 1u, 0x7100u);
+          if (ok) {
+            mbar_arrive_expect_tx(&q_full[qb], kQBytes);
+            const int32_t qrow = cur.w.s * a.num_q_heads + cur.w.g * G;
+            tma_load_2d(qbuf + qb * kQBytes, &qmap, &q_full[qb], 0, qrow, pol_q);
+            tma_load_2d(qbuf + qb * kQBytes + kN * 128, &qmap, &q_full[qb], 64, qrow, pol_q);
+          }
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        ++ucnt;
+        if (!ok) break;
+      }
+      const int32_t nt = cur.tiles();
+      load_tiles(&kmap, row, nt);
+      if (have_pend && ok) load_tiles(&vmap, pend_row, pend_tiles);
+      pend_row = row;
+      pend_tiles = nt;
+      have_pend = true;
+      row = row_next;
+      cur = nxt;
     }
+    if (have_pend && ok) load_tiles(&vmap, pend_row, pend_tiles);
     if (!ok) {
       atomicExch(&abort_flag, 1);
       if (lane == 0)  // drain the loads that may still be in flight
@@ -331,81 +403,123 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
+    // Issue order: S^T of chunk i + 1 before O^T of chunk i, so the tensor
+    // cores and the loads of the next keys run while chunk i's softmax runs.
     uint32_t ctr = 0, ucnt = 0, cc = 0;
     bool ok = true;
-    for (int64_t u = blockIdx.x; u < num_units && ok; u += gridDim.x) {
-      tc::Unit w;
-      if (!tc::decode_unit(a, u, w)) continue;
-      const int32_t nch = tc::chunks_of(w);
-      if (nch == 0) continue;  // nothing to multiply; the producer loads no Q for it
-      const uint32_t qb = ucnt & 1u;
-      if (lane == 0) ok = mbar_wait(&q_full[qb], (ucnt >> 1) & 1u, 0x7400u);
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-      const uint32_t q_addr = smem_u32(qbuf + qb * kQBytes);
-      for (int32_t c = 0; c < nch && ok; ++c, ++cc) {
-        const uint32_t b = cc & 1u;
-        const uint32_t use = cc >> 1;
-        const int32_t ntile = tc::tiles_of(w, c);
-        if (lane == 0) {
-          // ---- S^T = K Q^T, one tile of 128 tokens at a time
-          ok = mbar_wait(&s_free[b], (use & 1u) ^ 1u, 0x7500u);
-          tc_fence_after();
-          for (int32_t t = 0; t < ntile && ok; ++t, ++ctr) {
-            const uint32_t st = ctr % kStages;
-            ok = mbar_wait(&full[st], (ctr / kStages) & 1u, 0x7600u);
-            if (!ok) break;
-            tc_fence_after();
-            const uint32_t k_addr = smem_u32(ring + st * kStageBytes);
-            const uint32_t d_tmem = tmem_base + kSCol + b * (kChunkTiles * kN) + t * kN;
+    uint32_t q_addr = 0, qb = 0;
+    auto qk = [&](uint32_t b, uint32_t use, int32_t ntile) {  // lane 0
+      ok = mbar_wait(&s_free[b], (use & 1u) ^ 1u, 0x7500u);
+      tc_fence_after();
+      for (int32_t t = 0; t < ntile && ok; ++t, ++ctr) {
+        const uint32_t st = ctr % kStages;
+        ok = mbar_wait(&full[st], (ctr / kStages) & 1u, 0x7600u);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t k_addr = smem_u32(ring + st * kStageBytes);
+        const uint32_t d_tmem = tmem_base + kSCol + b * (kChunkTiles * kN) + t * kN;
 #pragma unroll
-            for (int kk = 0; kk < kD / 16; ++kk) {
-              const uint32_t off = (kk >> 2) * kRegionBytes + (kk & 3) * 32;
-              const uint32_t qoff = (kk >> 2) * (kN * 128) + (kk & 3) * 32;
-              umma_f16_ss(d_tmem, smem_desc(k_addr + off, 16, 1024, kLayoutSw128),
-                          smem_desc(q_addr + qoff, 16, 1024, kLayoutSw128), kIdescQK, kk > 0);
-            }
-            umma_commit(&empty[st]);
-          }
-          if (ok) {
-            umma_commit(&s_full[b]);
-            if (c == nch - 1) umma_commit(&q_empty[qb]);
-          }
-          // ---- O^T += V^T P^T
-          if (ok) ok = mbar_wait(&p_full[b], use & 1u, 0x7700u);
-          if (ok) ok = mbar_wait(&o_free[b], (use & 1u) ^ 1u, 0x7800u);
-          tc_fence_after();
-          const uint32_t p_addr = smem_u32(pbuf + b * kPBytes);
-          const uint32_t o_tmem = tmem_base + kOCol + b * kNPV;
-          for (int32_t t = 0; t < ntile && ok; ++t, ++ctr) {
-            const uint32_t st = ctr % kStages;
-            ok = mbar_wait(&full[st], (ctr / kStages) & 1u, 0x7900u);
-            if (!ok) break;
-            tc_fence_after();
-            const uint32_t v_addr = smem_u32(ring + st * kStageBytes);
-#pragma unroll
-            for (int kk = 0; kk < kTileTok / 16; ++kk) {
-              const uint32_t pk = (t * kTileTok + kk * 16) / 8 * L::kPLbo;
-              umma_f16_ss(o_tmem, smem_desc(v_addr + kk * 2048, kRegionBytes, 1024, kLayoutSw128),
-                          smem_desc(p_addr + pk, L::kPLbo, 128, kLayoutNone), kIdescPV,
-                          (t > 0 || kk > 0) ? 1u : 0u);
-            }
-            umma_commit(&empty[st]);
-          }
-          if (ok) {
-            umma_commit(&o_full[b]);
-            umma_commit(&p_free[b]);
-          }
+        for (int kk = 0; kk < kD / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * kRegionBytes + (kk & 3) * 32;
+          const uint32_t qoff = (kk >> 2) * (kN * 128) + (kk & 3) * 32;
+          umma_f16_ss(d_tmem, smem_desc(k_addr + off, 16, 1024, kLayoutSw128),
+                      smem_desc(q_addr + qoff, 16, 1024, kLayoutSw128), kIdescQK, kk > 0);
         }
-        ok = __shfl_sync(0xffffffffu, ok, 0);
+        umma_commit(&empty[st]);
       }
-      ++ucnt;
+      if (ok) umma_commit(&s_full[b]);
+    };
+    // O^T += V^T P^T for a chunk, run by the whole warp: lane 0 waits and
+    // issues; in the chunk's last tile the lanes first zero the V rows of
+    // tokens past the end of the sequence (rows >= zero_from), which hold
+    // whatever the pool had there: p is 0 for them, but 0 * inf is NaN.
+    auto pv = [&](uint32_t b, uint32_t use, int32_t ntile, int32_t zero_from) {
+      if (lane == 0) {
+        ok = mbar_wait(&p_full[b], use & 1u, 0x7700u);
+        if (ok) ok = mbar_wait(&o_free[b], (use & 1u) ^ 1u, 0x7800u);
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      tc_fence_after();
+      const uint32_t p_addr = smem_u32(pbuf + b * kPBytes);
+      const uint32_t o_tmem = tmem_base + kOCol + b * kNPV;
+      for (int32_t t = 0; t < ntile && ok; ++t, ++ctr) {
+        const uint32_t st = ctr % kStages;
+        if (lane == 0) ok = mbar_wait(&full[st], (ctr / kStages) & 1u, 0x7900u);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        tc_fence_after();
+        if (t == ntile - 1 && zero_from < kTileTok) {
+          uint8_t* tile = ring + st * kStageBytes;
+          for (int row = zero_from + lane; row < kTileTok; row += 32) {
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              reinterpret_cast<uint4*>(tile + row * 128)[q] = make_uint4(0, 0, 0, 0);
+              reinterpret_cast<uint4*>(tile + kRegionBytes + row * 128)[q] = make_uint4(0, 0, 0, 0);
+            }
+          }
+          fence_proxy_async_smem();
+        }
+        __syncwarp();
+        if (lane == 0) {
+          tc_fence_after();
+          const uint32_t v_addr = smem_u32(ring + st * kStageBytes);
+#pragma unroll
+          for (int kk = 0; kk < kTileTok / 16; ++kk) {
+            const uint32_t pk = (t * kTileTok + kk * 16) / 8 * L::kPLbo;
+            umma_f16_ss(o_tmem, smem_desc(v_addr + kk * 2048, kRegionBytes, 1024, kLayoutSw128),
+                        smem_desc(p_addr + pk, L::kPLbo, 128, kLayoutNone), kIdescPV,
+                        (t > 0 || kk > 0) ? 1u : 0u);
+          }
+          umma_commit(&empty[st]);
+        }
+        __syncwarp();
+      }
+      if (ok && lane == 0) {
+        umma_commit(&o_full[b]);
+        umma_commit(&p_free[b]);
+      }
+    };
+    tc::ChunkStream cur;
+    cur.init(a, blockIdx.x, gridDim.x, num_units, ctx_sm);
+    uint32_t pend_b = 0, pend_use = 0;
+    int32_t pend_tiles = 0, pend_zero = kTileTok;
+    bool have_pend = false;
+    while (cur.valid && ok) {
+      const uint32_t b = cc & 1u, use = cc >> 1;
+      const int32_t nt = cur.tiles();
+      if (lane == 0) {
+        if (cur.first()) {
+          qb = ucnt & 1u;
+          ok = mbar_wait(&q_full[qb], (ucnt >> 1) & 1u, 0x7400u);
+          q_addr = smem_u32(qbuf + qb * kQBytes);
+        }
+        if (ok) qk(b, use, nt);
+        if (ok && cur.last()) umma_commit(&q_empty[qb]);
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      ctr = __shfl_sync(0xffffffffu, ctr, 0);  // qk advanced the ring on lane 0 only
+      if (ok && have_pend) pv(pend_b, pend_use, pend_tiles, pend_zero);
+      if (cur.first()) ++ucnt;
+      // valid tokens in this chunk's last tile; rows from there on are zeroed
+      const int32_t ctok0 = cur.w.tok_begin + cur.c * kChunkTok;
+      const int32_t nvalid = min(cur.w.tok_end, ctok0 + kChunkTok) - ctok0;
+      pend_zero = nvalid - (nt - 1) * kTileTok;
+      pend_b = b;
+      pend_use = use;
+      pend_tiles = nt;
+      have_pend = true;
+      ++cc;
+      cur.advance(a);
     }
+    if (ok && have_pend) pv(pend_b, pend_use, pend_tiles, pend_zero);
     if (!ok) atomicExch(&abort_flag, 1);
   } else {
     // ------------------------------------------------------------ softmax + epilogue
     // All waits here are bounded mbarrier waits made warp-uniform; the four
     // warps exchange maxima and sums through shared memory guarded by count-4
-    // mbarriers on alternating halves (no unbounded named barriers).
+    // mbarriers on alternating halves (no unbounded named barriers). Order per
+    // chunk i: p of chunk i, then the merge of chunk i - 1's O (and the
+    // epilogue of its unit when it was the unit's last chunk).
     const int quarter = warp & 3;          // TMEM lanes 32*quarter .. +31
     const int r = quarter * 32 + lane;     // token row (S) / head-dim row (O)
     const uint32_t lane_addr = uint32_t(quarter * 32) << 16;
@@ -413,143 +527,49 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
     auto wait_all = [&](uint64_t* bar, uint32_t parity, uint32_t where) {
       return __all_sync(0xffffffffu, mbar_wait(bar, parity, where)) != 0;
     };
-    uint32_t ctr = 0, cc = 0, ucnt = 0;
-    bool ok = true;
-    for (int64_t u = blockIdx.x; u < num_units && ok; u += gridDim.x) {
+    // Units without tokens (context length 0) attend to nothing: zero rows.
+    for (int64_t u = blockIdx.x; u < num_units; u += gridDim.x) {
       tc::Unit w;
-      if (!tc::decode_unit(a, u, w)) continue;
-      float acc[NG], m_run[NG], l_thr[NG];
+      if (!tc::decode_unit(a, u, w, ctx_sm) || tc::chunks_of(w) > 0) continue;
+      for (int j = 0; j < G; ++j)
+        static_cast<uint16_t*>(a.out)[(int64_t(w.s) * a.num_q_heads + w.g * G + j) * kD + r] = 0;
+    }
+    float acc[NG], m_run[NG], l_thr[NG];
+#pragma unroll
+    for (int j = 0; j < NG; ++j) {
+      acc[j] = 0.f;
+      m_run[j] = -INFINITY;
+      l_thr[j] = 0.f;
+    }
+    // The chunk whose O is merged one step later.
+    tc::Unit pw{};
+    uint32_t pb_ = 0, puse = 0;
+    bool plast = false, have_pend = false;
+    float pmax_[NG], psum_[NG];
+    uint32_t cc = 0, ucnt = 0;
+    bool ok = true;
+
+    auto merge = [&]() {  // merge the pending chunk; epilogue when it ends its unit
+      ok = wait_all(&o_full[pb_], puse & 1u, 0x7d00u);
+      if (!ok) return;
+      tc_fence_after();
+      float ov2[2 * NG];  // [hi columns | lo columns]
+      tmem_ld_cols<2 * NG>(tmem_base + lane_addr + kOCol + pb_ * kNPV, ov2);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&o_free[pb_]);
 #pragma unroll
       for (int j = 0; j < NG; ++j) {
-        acc[j] = 0.f;
-        m_run[j] = -INFINITY;
-        l_thr[j] = 0.f;
+        const float ov = ov2[j] + ov2[NG + j];
+        const float mn = fmaxf(m_run[j], pmax_[j]);
+        const float fo = m_run[j] == -INFINITY ? 0.f : exp2f(m_run[j] - mn);
+        const float fc = pmax_[j] == -INFINITY ? 0.f : exp2f(pmax_[j] - mn);
+        acc[j] = acc[j] * fo + ov * fc;
+        l_thr[j] = l_thr[j] * fo + psum_[j] * fc;
+        m_run[j] = mn;
       }
-      const int32_t nch = tc::chunks_of(w);
-      for (int32_t c = 0; c < nch && ok; ++c, ++cc) {
-        const uint32_t b = cc & 1u;
-        const uint32_t use = cc >> 1;
-        const int32_t ntile = tc::tiles_of(w, c);
-        const int32_t ctok0 = w.tok_begin + c * kChunkTok;
-        const int32_t ctok1 = min(w.tok_end, ctok0 + kChunkTok);
-        // ---- scores of this thread's tokens (row r of each tile)
-        ok = wait_all(&s_full[b], use & 1u, 0x7a00u);
-        if (!ok) break;
-        tc_fence_after();
-        float sv[kChunkTiles][NG];
-#pragma unroll
-        for (int t = 0; t < kChunkTiles; ++t) {
-          if (t < ntile) {
-            tmem_ld_cols<NG>(tmem_base + lane_addr + kSCol + b * (kChunkTiles * kN) + t * kN,
-                             sv[t]);
-          } else {
-#pragma unroll
-            for (int j = 0; j < NG; ++j) sv[t][j] = -INFINITY;
-          }
-        }
-        tmem_ld_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&s_free[b]);
-        float cmax[NG];
-#pragma unroll
-        for (int j = 0; j < NG; ++j) cmax[j] = -INFINITY;
-#pragma unroll
-        for (int t = 0; t < kChunkTiles; ++t) {
-          const bool valid = t < ntile && ctok0 + t * kTileTok + r < ctok1;
-#pragma unroll
-          for (int j = 0; j < NG; ++j) {
-            sv[t][j] = valid ? sv[t][j] * a.scale_log2 : -INFINITY;
-            cmax[j] = fmaxf(cmax[j], sv[t][j]);
-          }
-        }
-        float* redm = red + b * 4 * kN;
-#pragma unroll
-        for (int j = 0; j < NG; ++j) {
-          cmax[j] = warp_max(cmax[j]);
-          if (lane == 0) redm[wi * kN + j] = cmax[j];
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&red_bar[b]);
-        ok = wait_all(&red_bar[b], use & 1u, 0x7a80u);
-        if (!ok) break;
-#pragma unroll
-        for (int j = 0; j < NG; ++j)
-          cmax[j] = fmaxf(fmaxf(redm[j], redm[kN + j]), fmaxf(redm[2 * kN + j], redm[3 * kN + j]));
-        // ---- p = 2^(s - m), rounded to the input type, into P^T (K-major, no swizzle)
-        ok = wait_all(&p_free[b], (use & 1u) ^ 1u, 0x7b00u);
-        if (!ok) break;
-        uint8_t* pb = pbuf + b * kPBytes;
-        float psum[NG];
-#pragma unroll
-        for (int j = 0; j < NG; ++j) psum[j] = 0.f;
-#pragma unroll
-        for (int t = 0; t < kChunkTiles; ++t) {
-          if (t < ntile) {
-            const int tok = t * kTileTok + r;  // token within the chunk
-            uint8_t* prow = pb + (tok >> 3) * L::kPLbo + (tok & 7) * 2;
-#pragma unroll
-            for (int j = 0; j < NG; ++j) {
-              const float pf = sv[t][j] == -INFINITY ? 0.f : exp2f(sv[t][j] - cmax[j]);
-              const uint16_t hi = Elem<T>::from_float(pf);
-              const float hf = Elem<T>::to_float2(uint32_t(hi)).x;
-              const uint16_t lo = Elem<T>::from_float(pf - hf);
-              psum[j] += hf + Elem<T>::to_float2(uint32_t(lo)).x;
-              const int jl = NG + j;
-              *reinterpret_cast<uint16_t*>(prow + (j >> 3) * 128 + (j & 7) * 16) = hi;
-              *reinterpret_cast<uint16_t*>(prow + (jl >> 3) * 128 + (jl & 7) * 16) = lo;
-            }
-          }
-        }
-        // Tokens past the end of the sequence in the chunk's last tile: their V
-        // rows hold whatever the pool had there; zero them before the PV MMA
-        // (p is already 0 for them, but 0 * inf would still be NaN).
-        {
-          const int32_t last_tile = (ctok1 - 1 - ctok0) / kTileTok;
-          const bool past_end = ctok0 + last_tile * kTileTok + r >= ctok1;
-          const uint32_t vctr = ctr + ntile + last_tile;
-          const uint32_t st = vctr % kStages;
-          if (__any_sync(0xffffffffu, past_end)) {
-            ok = wait_all(&full[st], (vctr / kStages) & 1u, 0x7c00u);
-            if (ok && past_end) {
-              uint8_t* vrow = ring + st * kStageBytes + r * 128;
-#pragma unroll
-              for (int q = 0; q < 8; ++q) {
-                reinterpret_cast<uint4*>(vrow)[q] = make_uint4(0, 0, 0, 0);
-                reinterpret_cast<uint4*>(vrow + kRegionBytes)[q] = make_uint4(0, 0, 0, 0);
-              }
-            }
-          }
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&p_full[b]);
-        if (!ok) break;
-        ctr += 2 * ntile;
-        // ---- merge this chunk's O into the running output
-        ok = wait_all(&o_full[b], use & 1u, 0x7d00u);
-        if (!ok) break;
-        tc_fence_after();
-        float ov2[2 * NG];  // [hi columns | lo columns]
-        tmem_ld_cols<2 * NG>(tmem_base + lane_addr + kOCol + b * kNPV, ov2);
-        float ov[NG];
-#pragma unroll
-        for (int j = 0; j < NG; ++j) ov[j] = ov2[j] + ov2[NG + j];
-        tmem_ld_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&o_free[b]);
-#pragma unroll
-        for (int j = 0; j < NG; ++j) {
-          const float mn = fmaxf(m_run[j], cmax[j]);
-          const float fo = m_run[j] == -INFINITY ? 0.f : exp2f(m_run[j] - mn);
-          const float fc = cmax[j] == -INFINITY ? 0.f : exp2f(cmax[j] - mn);
-          acc[j] = acc[j] * fo + ov[j] * fc;
-          l_thr[j] = l_thr[j] * fo + psum[j] * fc;
-          m_run[j] = mn;
-        }
-      }
-      if (!ok) break;
+      if (!plast) return;
       // ---- unit epilogue: l over all 128 rows, then write
       const uint32_t ub = ucnt & 1u;
       float* rl = redl + ub * 4 * kN;
@@ -564,26 +584,129 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
       if (lane == 0) mbar_arrive(&lred_bar[ub]);
       ok = wait_all(&lred_bar[ub], (ucnt >> 1) & 1u, 0x7e00u);
       ++ucnt;
-      if (!ok) break;
-      const int32_t h0 = w.g * G;
+      if (!ok) return;
+      const int32_t h0 = pw.g * G;
 #pragma unroll
       for (int j = 0; j < NG; ++j) {
-        const float L = (rl[j] + rl[kN + j]) + (rl[2 * kN + j] + rl[3 * kN + j]);
+        const float Lj = (rl[j] + rl[kN + j]) + (rl[2 * kN + j] + rl[3 * kN + j]);
         if (j < G) {
-          const int64_t row_sh = int64_t(w.s) * a.num_q_heads + h0 + j;
-          if (w.nparts <= 1) {
-            const float y = L > 0.f ? acc[j] / L : 0.f;
+          const int64_t row_sh = int64_t(pw.s) * a.num_q_heads + h0 + j;
+          if (pw.nparts <= 1) {
+            const float y = Lj > 0.f ? acc[j] / Lj : 0.f;
             static_cast<uint16_t*>(a.out)[row_sh * kD + r] = Elem<T>::from_float(y);
           } else {
-            a.ws_acc[(row_sh * a.pmax + w.p) * kD + r] = acc[j];
+            a.ws_acc[(row_sh * a.pmax + pw.p) * kD + r] = acc[j];
             if (r == 0) {
-              a.ws_ml[(row_sh * a.pmax + w.p) * 2 + 0] = m_run[j];
-              a.ws_ml[(row_sh * a.pmax + w.p) * 2 + 1] = L;
+              a.ws_ml[(row_sh * a.pmax + pw.p) * 2 + 0] = m_run[j];
+              a.ws_ml[(row_sh * a.pmax + pw.p) * 2 + 1] = Lj;
             }
           }
         }
+        acc[j] = 0.f;
+        m_run[j] = -INFINITY;
+        l_thr[j] = 0.f;
       }
+    };
+
+    tc::ChunkStream cur;
+    cur.init(a, blockIdx.x, gridDim.x, num_units, ctx_sm);
+    while (cur.valid && ok) {
+      const uint32_t b = cc & 1u;
+      const uint32_t use = cc >> 1;
+      const int32_t ntile = cur.tiles();
+      const int32_t ctok0 = cur.w.tok_begin + cur.c * kChunkTok;
+      const int32_t ctok1 = min(cur.w.tok_end, ctok0 + kChunkTok);
+      // ---- scores of this thread's tokens (row r of each tile)
+      ok = wait_all(&s_full[b], use & 1u, 0x7a00u);
+      if (!ok) break;
+      tc_fence_after();
+      float sv[kChunkTiles][NG];
+#pragma unroll
+      for (int t = 0; t < kChunkTiles; ++t) {
+        if (t < ntile) {
+          tmem_ld_cols<NG>(tmem_base + lane_addr + kSCol + b * (kChunkTiles * kN) + t * kN, sv[t]);
+        } else {
+#pragma unroll
+          for (int j = 0; j < NG; ++j) sv[t][j] = -INFINITY;
+        }
+      }
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_free[b]);
+      float cmax[NG];
+#pragma unroll
+      for (int j = 0; j < NG; ++j) cmax[j] = -INFINITY;
+#pragma unroll
+      for (int t = 0; t < kChunkTiles; ++t) {
+        const bool valid = t < ntile && ctok0 + t * kTileTok + r < ctok1;
+#pragma unroll
+        for (int j = 0; j < NG; ++j) {
+          sv[t][j] = valid ? sv[t][j] * a.scale_log2 : -INFINITY;
+          cmax[j] = fmaxf(cmax[j], sv[t][j]);
+        }
+      }
+      float* redm = red + b * 4 * kN;
+#pragma unroll
+      for (int j = 0; j < NG; ++j) {
+        cmax[j] = warp_max(cmax[j]);
+        if (lane == 0) redm[wi * kN + j] = cmax[j];
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&red_bar[b]);
+      ok = wait_all(&red_bar[b], use & 1u, 0x7a80u);
+      if (!ok) break;
+#pragma unroll
+      for (int j = 0; j < NG; ++j)
+        cmax[j] = fmaxf(fmaxf(redm[j], redm[kN + j]), fmaxf(redm[2 * kN + j], redm[3 * kN + j]));
+      // ---- p = 2^(s - m) as hi + lo parts in the input type, into P^T
+      ok = wait_all(&p_free[b], (use & 1u) ^ 1u, 0x7b00u);
+      if (!ok) break;
+      uint8_t* pbuf_b = pbuf + b * kPBytes;
+      float psum[NG];
+#pragma unroll
+      for (int j = 0; j < NG; ++j) psum[j] = 0.f;
+#pragma unroll
+      for (int t = 0; t < kChunkTiles; ++t) {
+        if (t < ntile) {
+          const int tok = t * kTileTok + r;  // token within the chunk
+          uint8_t* prow = pbuf_b + (tok >> 3) * L::kPLbo + (tok & 7) * 2;
+#pragma unroll
+          for (int j = 0; j < NG; ++j) {
+            const float pf = sv[t][j] == -INFINITY ? 0.f : exp2f(sv[t][j] - cmax[j]);
+            const uint16_t hi = Elem<T>::from_float(pf);
+            const float hf = Elem<T>::to_float2(uint32_t(hi)).x;
+            const uint16_t lo = Elem<T>::from_float(pf - hf);
+            psum[j] += hf + Elem<T>::to_float2(uint32_t(lo)).x;
+            const int jl = NG + j;
+            *reinterpret_cast<uint16_t*>(prow + (j >> 3) * 128 + (j & 7) * 16) = hi;
+            *reinterpret_cast<uint16_t*>(prow + (jl >> 3) * 128 + (jl & 7) * 16) = lo;
+          }
+        }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_full[b]);
+      if (!ok) break;
+      // ---- merge the previous chunk's O, now that this chunk's P is out
+      if (have_pend) {
+        merge();
+        if (!ok) break;
+      }
+      pw = cur.w;
+      pb_ = b;
+      puse = use;
+      plast = cur.last();
+#pragma unroll
+      for (int j = 0; j < NG; ++j) {
+        pmax_[j] = cmax[j];
+        psum_[j] = psum[j];
+      }
+      have_pend = true;
+      ++cc;
+      cur.advance(a);
     }
+    if (ok && have_pend) merge();
     if (!ok) atomicExch(&abort_flag, 1);
   }
 

@@ -159,8 +159,10 @@ template <typename T, int BS, int NG>
 int launch_tc(const CUtensorMap& km, const CUtensorMap& vm, const CUtensorMap& qm,
               const kvp::dev::DecodeArgs& a, cudaStream_t st) {
   auto k = kvp::dev::decode_tc_kernel<T, BS, NG>;
-  constexpr int smem = kvp::dev::tc::Cfg<NG>::kSmemBytes;
-  cudaError_t e = ensure_smem(k, smem);
+  // context lengths of small batches are cached in shared memory
+  const int ctx_bytes = a.num_seqs <= kvp::dev::tc::kCtxCacheMax ? 4 * a.num_seqs : 0;
+  const int smem = kvp::dev::tc::Cfg<NG>::kSmemBytes + ctx_bytes;
+  cudaError_t e = ensure_smem(k, kvp::dev::tc::Cfg<NG>::kSmemBytes + 4 * kvp::dev::tc::kCtxCacheMax);
   if (e != cudaSuccess) return cuda_fail(e, "decode (tensor cores): smem attribute");
   const int64_t units = int64_t(a.num_seqs) * a.num_kv_heads * a.pmax;
   const int grid = int(units < sm_count() ? units : sm_count());
@@ -369,6 +371,31 @@ int paged_attention_decode(const void* q, const void* k_cache, const void* v_cac
   if (head_dim == 128)
     return dtype == KVP_F16 ? launch_reduce<__half, 128>(a, st) : launch_reduce<__nv_bfloat16, 128>(a, st);
   return dtype == KVP_F16 ? launch_reduce<__half, 64>(a, st) : launch_reduce<__nv_bfloat16, 64>(a, st);
+}
+
+}  // extern "C"
+
+// One thread waits, with the decode kernels' bounded wait, for a phase of an
+// mbarrier that nothing arrives on: the wait runs out and records a status.
+__global__ void selftest_bounded_wait_kernel(uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    kvp::dev::mbar_init(&bar, 1);
+    kvp::dev::fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) kvp::dev::mbar_wait(&bar, 0, 0xFFFFu, limit_ns);
+}
+
+extern "C" {
+
+int kvp_selftest_bounded_wait(int32_t limit_ms, kvp_stream_t stream) {
+  if (limit_ms < 1 || limit_ms > 2000)
+    return fail(KVP_ERR_INVALID, "kvp_selftest_bounded_wait: limit_ms must be in [1, 2000]");
+  selftest_bounded_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+      uint64_t(limit_ms) * 1000000ull);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? KVP_OK : cuda_fail(e, "kvp_selftest_bounded_wait: launch");
 }
 
 int kvp_check_device_error(kvp_stream_t stream) {
