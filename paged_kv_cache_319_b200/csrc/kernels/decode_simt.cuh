@@ -9,9 +9,10 @@
 // GPU was mostly empty", section "The OS already solved this in the 1960s"].
 //
 // How: each warp of the CTA owns every NW-th block of the partition and runs
-// its own TMA pipeline of NST stages: one elected lane issues two 2-D tensor
-// loads (K tile, V tile: block_size rows x head_dim, 128-byte swizzled) per
-// block onto the stage's mbarrier. A (block, KV head) tile is one contiguous
+// its own TMA pipeline of NST stages: one elected lane issues two tensor loads
+// (K tile, V tile: block_size rows x head_dim, 128-byte swizzled; for 128 dims
+// one 3-D box {64 dims, rows, 2 halves} each, so a tile costs one TMA
+// operation) per block onto the stage's mbarrier. A (block, KV head) tile is one contiguous
 // block_size * head_dim run of the cache, so every load is one dense 2-4 KiB
 // burst. The warp keeps a running max m, a per-lane exponent sum and an fp32
 // accumulator (online softmax in the log2 domain, q pre-scaled by
@@ -152,10 +153,13 @@ __global__ void __launch_bounds__(NW * 32) decode_simt_kernel(
       row = (id * a.num_kv_heads + g) * BS;
     }
     mbar_arrive_expect_tx(&my_bars[stage], 2 * C::kTileBytes);
-#pragma unroll
-    for (int r = 0; r < C::kRegions; ++r) {
-      tma_load_2d(kt + r * BS * 128, &kmap, &my_bars[stage], r * 64, row, policy);
-      tma_load_2d(vt + r * BS * 128, &vmap, &my_bars[stage], r * 64, row, policy);
+    if constexpr (C::kRegions == 2) {
+      // one 3-D box {64 dims, BS rows, 2 halves} per tile: smem [half][row][64]
+      tma_load_3d(kt, &kmap, &my_bars[stage], 0, row, 0, policy);
+      tma_load_3d(vt, &vmap, &my_bars[stage], 0, row, 0, policy);
+    } else {
+      tma_load_2d(kt, &kmap, &my_bars[stage], 0, row, policy);
+      tma_load_2d(vt, &vmap, &my_bars[stage], 0, row, policy);
     }
   };
 

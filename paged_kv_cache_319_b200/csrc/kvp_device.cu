@@ -117,6 +117,26 @@ int make_map(CUtensorMap* map, const void* base, int32_t dtype, uint64_t rows, u
   return KVP_OK;
 }
 
+// 3-D view of [rows][128] 2-byte elements as {64 dims, rows, 2 halves} (strides
+// 256 and 128 bytes) with a {64, box_rows, 2} box: one load brings a whole
+// (block, head) tile as [half][row][64], 128-byte swizzled.
+int make_map_halves(CUtensorMap* map, const void* base, int32_t dtype, uint64_t rows,
+                    uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return fail(KVP_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  cuuint64_t dims[3] = {64, rows, 2};
+  cuuint64_t strides[2] = {256, 128};
+  cuuint32_t box[3] = {64, box_rows, 2};
+  cuuint32_t estr[3] = {1, 1, 1};
+  const CUtensorMapDataType dt =
+      dtype == KVP_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  CUresult r = fn(map, dt, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(KVP_ERR_CUDA, "cuTensorMapEncodeTiled (3-D) failed (%d)", int(r));
+  return KVP_OK;
+}
+
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
 int ilog2(int64_t v) {
@@ -348,9 +368,16 @@ int paged_attention_decode(const void* q, const void* k_cache, const void* v_cac
 
   const uint64_t rows = uint64_t(num_blocks) * num_kv_heads * block_size;
   CUtensorMap km, vm;
-  int rc = make_map(&km, k_cache, dtype, rows, head_dim, block_size);
-  if (rc) return rc;
-  rc = make_map(&vm, v_cache, dtype, rows, head_dim, block_size);
+  int rc;
+  if (!tensor_cores && head_dim == 128) {  // CUDA-core kernel: one 3-D box per tile
+    rc = make_map_halves(&km, k_cache, dtype, rows, block_size);
+    if (rc) return rc;
+    rc = make_map_halves(&vm, v_cache, dtype, rows, block_size);
+  } else {
+    rc = make_map(&km, k_cache, dtype, rows, head_dim, block_size);
+    if (rc) return rc;
+    rc = make_map(&vm, v_cache, dtype, rows, head_dim, block_size);
+  }
   if (rc) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
 
