@@ -47,6 +47,8 @@ import workloads  # noqa: E402
 from workloads.values import K_STREAM, Q_STREAM, V_STREAM, normal_bits, value_seed_words  # noqa: E402
 
 METRIC = "paged decode attention: KV GB/s (% of HBM peak) and seq-tokens/s per layer"
+# Workloads whose batch changes every step; measured by replaying their schedule.
+SCHEDULE_WORKLOADS = ("llama13b_churn", "sharing_A", "sharing_B", "beam")
 UNIT = "GB/s"
 
 
@@ -346,7 +348,7 @@ def run_ours(args, world, rank, local):
     ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=device)
     stream = torch.cuda.current_stream(device)
 
-    step_bytes, step_tokens, launches = [], [], []
+    step_bytes, step_tokens, launches, host_us = [], [], [], []
     ev_pairs = []
 
     def step(i, timed):
@@ -355,9 +357,12 @@ def run_ours(args, world, rank, local):
         if done[b] is not None:
             done[b].synchronize()
         m = meta[b]
+        th = time.perf_counter()
         rep.pool.append_batch(rep.seqs, 1, out=m.slot_h.numpy())
         copies = rep.pool.take_copies()
         rep.pool.build_batch(rep.seqs, MB, m.tab_h.numpy(), m.len_h.numpy())
+        if timed:
+            host_us.append((time.perf_counter() - th) * 1e6)
         rep.lens += 1
         m.upload()
         n_launch = 0
@@ -416,6 +421,7 @@ def run_ours(args, world, rank, local):
     achieved = dec_bytes_avg / (dec_avg_ms * 1e-3) / 1e9
 
     # ---- end to end through the public API with host buffers
+    rows = measure_rows(wl, reps[0], device, kn[0], vn[0], host_us)
     e2e = run_e2e(args, wl, reps, device, seed_rank, MB, max_ctx_total, part, ws, world)
 
     peak, peak_kind = peaks()
@@ -467,12 +473,82 @@ def run_ours(args, world, rank, local):
             "algorithmic_bytes_per_launch": int(dec_bytes_avg),
         },
         "e2e": e2e,
+        "rows": rows,
         "clocks": clk.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         res["cpu_baseline"] = cpu_baseline(wl, budget_s=args.cpu_seconds)
     if rank == 0:
         print(json.dumps(res), flush=True)
+
+
+def measure_rows(wl, rep, device, k_step, v_step, host_us):
+    """The other rows of the hot path, each against its own roofline: host
+    bookkeeping per step (a1), copy_blocks (a2) and reshape_and_cache (a3).
+    Copies and scatters target free blocks of the pool, so no live sequence
+    changes."""
+    import torch
+    import paged_kv_cache_319_b200 as kvp
+
+    g = wl.geometry
+    peak, _ = peaks()
+    stream = torch.cuda.current_stream(device)
+    free = np.asarray(rep.pool.free_list(), dtype=np.int64)
+    used = np.setdiff1d(np.arange(wl.num_blocks), free)
+    block_bytes = 2 * g.num_kv_heads * g.block_size * g.head_dim * g.elem_bytes
+
+    def timed(fn, reps=20):
+        """Device time per call: the calls are captured in a CUDA graph and the
+        graph replayed, so host launch overhead of small calls is not timed."""
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize(device)
+        graph = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream(device)
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            with torch.cuda.graph(graph, stream=side):
+                for _ in range(reps):
+                    fn()
+        stream.wait_stream(side)
+        graph.replay()
+        torch.cuda.synchronize(device)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        graph.replay()
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        del graph
+        return e0.elapsed_time(e1) / reps * 1e3  # us
+
+    out = {"a1_host_bookkeeping_us_per_step": round(float(np.median(host_us)), 1)}
+    # a2: copy-on-write copies, up to 1024 pairs (sources in use, destinations free)
+    n = int(min(1024, len(free), len(used)))
+    if n > 0:
+        pairs = torch.tensor(np.stack([used[:n], free[:n]], 1), dtype=torch.int32, device=device)
+        us = timed(lambda: kvp.copy_blocks(rep.k, rep.v, pairs))
+        moved = 2 * n * block_bytes  # read + write
+        out["a2_copy_blocks"] = {"pairs": n, "us": round(us, 2), "GBps": round(moved / us / 1e3, 1),
+                                 "frac": round(moved / us / 1e3 / peak, 3)}
+    # a3: one decode step's scatter (launch-bound) and a bulk prefill-sized scatter
+    S = k_step.shape[0]
+    slots = torch.tensor(free[:S] * g.block_size, dtype=torch.int64, device=device)
+    us = timed(lambda: kvp.reshape_and_cache(k_step, v_step, rep.k, rep.v, slots))
+    out["a3_reshape_and_cache_step"] = {"tokens": S, "us": round(us, 2)}
+    nb = int(min(len(free), 2048))
+    T = nb * g.block_size
+    bulk_slots = torch.from_numpy((free[:nb, None] * g.block_size +
+                                   np.arange(g.block_size)[None, :]).reshape(-1)).to(device)
+    kb = torch.randn((T, g.num_kv_heads, g.head_dim), dtype=k_step.dtype, device=device)
+    vb = torch.randn_like(kb)
+    us = timed(lambda: kvp.reshape_and_cache(kb, vb, rep.k, rep.v, bulk_slots), reps=10)
+    moved = 2 * 2 * T * g.num_kv_heads * g.head_dim * g.elem_bytes + 8 * T
+    out["a3_reshape_and_cache_bulk"] = {"tokens": T, "us": round(us, 1),
+                                        "GBps": round(moved / us / 1e3, 1),
+                                        "frac": round(moved / us / 1e3 / peak, 3)}
+    kvp.check_device_error(device)
+    return out
 
 
 def run_e2e(args, wl, reps, device, seed_rank, MB, max_ctx_total, part, ws, world):
@@ -561,6 +637,74 @@ def cpu_baseline(wl, budget_s=15.0, seqs_per_step=None):
                       f"{nbytes / 1e9:.3f} GB of K/V, {el:.1f} s"}
 
 
+def unique_bytes(tables, lens, g):
+    """Bytes of the distinct physical blocks a batch reads (each block's valid slots
+    counted once, however many sequences share it), plus q, out and metadata."""
+    valid = {}
+    bs = g.block_size
+    for row, L in zip(np.asarray(tables), np.asarray(lens)):
+        for i in range(-(-int(L) // bs)):
+            b = int(row[i])
+            valid[b] = max(valid.get(b, 0), min(bs, int(L) - i * bs))
+    kv = sum(valid.values()) * g.num_kv_heads * g.head_dim * g.elem_bytes * 2
+    qo = len(lens) * g.num_q_heads * g.head_dim * g.elem_bytes * 2
+    return kv + qo + 4 * int(np.sum(-(-np.asarray(lens) // bs))) + 4 * len(lens)
+
+
+def run_schedule(args):
+    """Workloads whose steps change the batch (churn, sharing, beam): the schedule is
+    replayed once through libkvp and every attention call is timed with CUDA events."""
+    import torch
+    import paged_kv_cache_319_b200 as kvp
+    from paged_kv_cache_319_b200.replay import DeviceReplay
+
+    device = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(device)
+    kw = {}
+    if args.workload in ("llama13b_churn", "beam"):
+        kw["steps"] = max(args.warmup + 1, min(args.steps + args.warmup, 32 if args.workload ==
+                                                "llama13b_churn" else 64))
+    wl = workloads.by_name(args.workload, **kw)
+    g = wl.geometry
+    rp = DeviceReplay(wl, device, keep_outputs=False, time_decode=True)
+    rp.run()
+    torch.cuda.synchronize(device)
+    kvp.check_device_error(device)
+    attends = {i: (t, l) for (i, _, t, l) in rp.attends}
+    rows = []
+    for n, (i, e0, e1) in enumerate(rp.decode_events):
+        t, l = attends[i]
+        ms = e0.elapsed_time(e1)
+        rows.append((ms, algorithmic_bytes(l, g), unique_bytes(t, l, g), int(np.sum(l))))
+    timed = rows[args.warmup:] if len(rows) > args.warmup else rows
+    ms = np.array([r[0] for r in timed])
+    logical = np.array([r[1] for r in timed], dtype=np.float64)
+    uniq = np.array([r[2] for r in timed], dtype=np.float64)
+    toks = np.array([r[3] for r in timed], dtype=np.float64)
+    peak, peak_kind = peaks()
+    kernel = "decode_tc" if g.num_q_heads > g.num_kv_heads else "decode_simt"
+    st = rp.pool.stats()
+    achieved_u = float(uniq.sum() / (ms.sum() * 1e-3) / 1e9)
+    res = {
+        "metric": METRIC, "value": round(float(logical.sum() / (ms.sum() * 1e-3) / 1e9), 2),
+        "unit": UNIT, "n_gpus": 1, "steps": len(timed), "warmup": len(rows) - len(timed),
+        "ms_per_step": round(float(ms.mean()), 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": g.dtype, "data": "synthetic",
+        "config": {"workload": wl.description, "name": wl.name, "timed": "attention calls only"},
+        "seq_tokens_per_s": round(float(toks.sum() / (ms.sum() * 1e-3)), 1),
+        "roofline": {"kernel": f"paged_attention_decode: {kernel} + decode_reduce_kernel",
+                     "bound": "hbm", "achieved_unique": round(achieved_u, 1),
+                     "achieved_logical": round(float(logical.sum() / (ms.sum() * 1e-3) / 1e9), 1),
+                     "peak": peak, "peak_source": peak_kind, "unit": "GB/s",
+                     "frac": round(achieved_u / peak, 4),
+                     "avg_launch_us": round(float(ms.mean() * 1e3), 2),
+                     "unique_bytes_per_launch": int(uniq.mean()),
+                     "logical_bytes_per_launch": int(logical.mean())},
+        "pool": {k: int(v) for k, v in st.items()},
+    }
+    print(json.dumps(res), flush=True)
+
+
 def run_reference(args, world, rank):
     """The oracle as the reference arm: each step is a bounded sample of the workload."""
     if rank != 0:
@@ -608,7 +752,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="opt13b",
-                    choices=["opt13b", "gqa_long_bs16", "gqa_long_bs32"])
+                    choices=["opt13b", "gqa_long_bs16", "gqa_long_bs32", "llama13b_churn",
+                             "sharing_A", "sharing_B", "beam"])
     ap.add_argument("--partition", type=int, default=None)
     ap.add_argument("--num-seqs", type=int, default=None,
                     help="smaller batch of the same workload (profiling small cases)")
@@ -616,12 +761,15 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--ref-seqs-per-step", type=int, default=1)
     args = ap.parse_args()
-    if args.warmup < 3:
+    if args.warmup < 3 and args.workload not in SCHEDULE_WORKLOADS:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
         # The oracle needs no GPU and no process group: rank 0 runs, the others exit.
         run_reference(args, int(os.environ.get("WORLD_SIZE", "1")),
                       int(os.environ.get("RANK", "0")))
+        return
+    if args.workload in SCHEDULE_WORKLOADS:
+        run_schedule(args)
         return
     world, rank, local = dist_setup()
     try:

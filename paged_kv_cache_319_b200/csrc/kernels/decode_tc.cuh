@@ -46,7 +46,12 @@ namespace tc {
 constexpr int kD = 128;             // head_dim
 constexpr int kN = 16;              // MMA N (query heads of a group, padded)
 constexpr int kTileTok = 128;       // MMA M: tokens per tile
-constexpr int kChunkTiles = 4;      // tiles per chunk (512 tokens)
+// Tiles per chunk (the unit of the softmax pipeline) and ring stages are
+// compile-time tunables; defaults: 4 tiles (512 tokens), 5 stages.
+#ifndef KVP_TC_CHUNK_TILES
+#define KVP_TC_CHUNK_TILES 4
+#endif
+constexpr int kChunkTiles = KVP_TC_CHUNK_TILES;  // tiles per chunk
 constexpr int kChunkTok = kTileTok * kChunkTiles;
 constexpr int kStageBytes = kTileTok * kD * 2;       // 32 KiB
 constexpr int kRegionBytes = kTileTok * 128;         // 16 KiB: 64 dims of 128 tokens
@@ -56,8 +61,9 @@ constexpr int kSCol = 0;                             // S buffers: [0, 128)
 constexpr int kOCol = 128;                           // O buffers: [128, 128 + 2 * kNPV)
 constexpr int kThreads = 192;
 constexpr int kSoftmaxThreads = 128;
-// Batches of up to this many sequences keep their context lengths in shared
-// memory, so no warp role waits on a global load when it moves to a new unit.
+// Batches of up to Cfg<NG>::kCtxCap sequences (at most kCtxCacheMax) keep their
+// context lengths in shared memory, so no warp role waits on a global load when
+// it moves to a new unit.
 constexpr int kCtxCacheMax = 4096;
 
 // Layout for a group width NG (query heads per KV head, padded to 4, 8 or 16).
@@ -67,7 +73,11 @@ constexpr int kCtxCacheMax = 4096;
 template <int NG>
 struct Cfg {
   static constexpr int kNPV = 2 * NG <= 16 ? 16 : 32;  // N of the PV MMA
-  static constexpr int kStages = NG <= 8 ? 5 : 4;
+#ifndef KVP_TC_STAGES
+#define KVP_TC_STAGES 5
+#endif
+  // groups of 16 need a P^T twice as wide, which costs one stage
+  static constexpr int kStages = NG <= 8 ? KVP_TC_STAGES : KVP_TC_STAGES - 1;
   static constexpr int kPBytes = kChunkTok * kNPV * 2;
   static constexpr int kPLbo = kNPV * 16;               // bytes between 8-token groups of P^T
   static constexpr int kOffRing = 0;
@@ -80,11 +90,10 @@ struct Cfg {
   static constexpr int kOffTmemPtr = kOffRedL + 2 * 4 * kN * 4;
   static constexpr int kOffCtx = kOffTmemPtr + 16;           // cached context lengths
   static constexpr int kSmemBytes = 1024 + kOffCtx;          // + 4 bytes per cached length
-  // The softmax warps wait for a chunk's last V tile (to zero rows past the
-  // end of the sequence) before the PV MMAs free any stage of that chunk, so
-  // the ring must hold a chunk's K tiles plus that V tile.
-  static_assert(kStages >= kChunkTiles, "ring too shallow for one chunk");
-  static_assert(kSmemBytes + 4 * kCtxCacheMax <= 227 * 1024, "shared memory budget");
+  static constexpr int kCtxCap =
+      (226 * 1024 - kSmemBytes) / 4 < kCtxCacheMax ? (226 * 1024 - kSmemBytes) / 4 : kCtxCacheMax;
+  static_assert(kStages >= 2, "ring stages");
+  static_assert(kCtxCap >= 0, "shared memory budget");
   static_assert(kOCol + 2 * kNPV <= kTmemCols, "tensor memory budget");
 };
 
@@ -264,7 +273,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
   float* redl = reinterpret_cast<float*>(smem + L::kOffRedL);
   uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + L::kOffTmemPtr);
   int32_t* ctx_cache = reinterpret_cast<int32_t*>(smem + L::kOffCtx);
-  const int32_t* ctx_sm = a.num_seqs <= kCtxCacheMax ? ctx_cache : nullptr;
+  const int32_t* ctx_sm = a.num_seqs <= L::kCtxCap ? ctx_cache : nullptr;
   if (ctx_sm) {
     for (int i = threadIdx.x; i < a.num_seqs; i += blockDim.x)
       ctx_cache[i] = load_ctx(a, i, blockIdx.x == 0);  // clamped; out-of-range reported once

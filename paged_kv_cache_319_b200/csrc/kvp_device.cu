@@ -180,9 +180,10 @@ int launch_tc(const CUtensorMap& km, const CUtensorMap& vm, const CUtensorMap& q
               const kvp::dev::DecodeArgs& a, cudaStream_t st) {
   auto k = kvp::dev::decode_tc_kernel<T, BS, NG>;
   // context lengths of small batches are cached in shared memory
-  const int ctx_bytes = a.num_seqs <= kvp::dev::tc::kCtxCacheMax ? 4 * a.num_seqs : 0;
-  const int smem = kvp::dev::tc::Cfg<NG>::kSmemBytes + ctx_bytes;
-  cudaError_t e = ensure_smem(k, kvp::dev::tc::Cfg<NG>::kSmemBytes + 4 * kvp::dev::tc::kCtxCacheMax);
+  using Cfg = kvp::dev::tc::Cfg<NG>;
+  const int ctx_bytes = a.num_seqs <= Cfg::kCtxCap ? 4 * a.num_seqs : 0;
+  const int smem = Cfg::kSmemBytes + ctx_bytes;
+  cudaError_t e = ensure_smem(k, Cfg::kSmemBytes + 4 * Cfg::kCtxCap);
   if (e != cudaSuccess) return cuda_fail(e, "decode (tensor cores): smem attribute");
   const int64_t units = int64_t(a.num_seqs) * a.num_kv_heads * a.pmax;
   const int grid = int(units < sm_count() ? units : sm_count());

@@ -31,7 +31,7 @@ def bits_to_tensor(bits: np.ndarray, dtype: str, device):
 
 
 class DeviceReplay:
-    def __init__(self, wl, device="cuda", keep_outputs: bool = True):
+    def __init__(self, wl, device="cuda", keep_outputs: bool = True, time_decode: bool = False):
         import torch
 
         g = wl.geometry
@@ -49,6 +49,8 @@ class DeviceReplay:
         self.attends = []          # (op_index, seq ids, tables, lens)
         self.outputs = {}          # op_index -> out tensor
         self.keep_outputs = keep_outputs
+        self.time_decode = time_decode
+        self.decode_events = []    # (op_index, start event, end event) around each decode call
         self.next_index = 0
 
     def kv_values(self, op_index: int, n: int):
@@ -119,9 +121,24 @@ class DeviceReplay:
             bt = torch.from_numpy(tables).to(self.device)
             cl = torch.from_numpy(lens).to(self.device)
             part = kw.get("partition_size", self.wl.partition_size)
+            if self.time_decode:
+                # an untimed call, then an L2-sized write, keep the stream busy while
+                # the timed call is issued (so the start event does not time the host's
+                # launch work) and leave none of the KV blocks in L2
+                paged_attention_decode(q, self.k_cache, self.v_cache, bt, cl, self.wl.scale,
+                                       max_context_len=int(lens.max()) if len(lens) else 0,
+                                       partition_size=part)
+                if not hasattr(self, "_l2_flush"):
+                    self._l2_flush = torch.empty(256 << 20, dtype=torch.uint8, device=self.device)
+                self._l2_flush.fill_(1)
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
             out = paged_attention_decode(q, self.k_cache, self.v_cache, bt, cl, self.wl.scale,
                                          max_context_len=int(lens.max()) if len(lens) else 0,
                                          partition_size=part)
+            if self.time_decode:
+                e1.record()
+                self.decode_events.append((i, e0, e1))
             if self.keep_outputs:
                 self.outputs[i] = out
         else:
