@@ -123,6 +123,23 @@ __device__ __forceinline__ uint64_t l2_policy_evict_first() {
   return p;
 }
 
+__device__ __forceinline__ uint64_t l2_policy_evict_normal() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+// L2 policy of the K/V tile loads (0: evict first, 1: normal, 2: evict last).
+#ifndef KVP_KV_L2_POLICY
+#define KVP_KV_L2_POLICY 0
+#endif
+__device__ __forceinline__ uint64_t l2_policy_evict_last();
+__device__ __forceinline__ uint64_t l2_policy_kv() {
+  if constexpr (KVP_KV_L2_POLICY == 1) return l2_policy_evict_normal();
+  if constexpr (KVP_KV_L2_POLICY == 2) return l2_policy_evict_last();
+  return l2_policy_evict_first();
+}
+
 __device__ __forceinline__ uint64_t l2_policy_evict_last() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));

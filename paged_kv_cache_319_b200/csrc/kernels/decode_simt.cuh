@@ -129,7 +129,7 @@ __global__ void __launch_bounds__(NW * 32) decode_simt_kernel(
   }
   __syncwarp();
 
-  const uint64_t policy = l2_policy_evict_first();
+  const uint64_t policy = l2_policy_kv();
   const int32_t rows_total = a.num_blocks * a.num_kv_heads * BS;
 
   // Register cache of 32 block ids: lane l holds id of index base + l.

@@ -329,7 +329,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
       prefetch_tensormap(&vmap);
       prefetch_tensormap(&qmap);
     }
-    const uint64_t pol_kv = l2_policy_evict_first();
+    const uint64_t pol_kv = l2_policy_kv();
     const uint64_t pol_q = l2_policy_evict_last();
     uint32_t ctr = 0;   // ring tiles issued
     uint32_t ucnt = 0;  // units started
