@@ -49,6 +49,9 @@ from workloads.values import K_STREAM, Q_STREAM, V_STREAM, normal_bits, value_se
 METRIC = "paged decode attention: KV GB/s (% of HBM peak) and seq-tokens/s per layer"
 # Workloads whose batch changes every step; measured by replaying their schedule.
 SCHEDULE_WORKLOADS = ("llama13b_churn", "sharing_A", "sharing_B", "beam")
+# batches of forked sequences: decoded by default through the grouped entry point,
+# which reads each shared block once per subgroup of the sequences holding it
+GROUPED_WORKLOADS = ("sharing_A", "sharing_B", "beam")
 UNIT = "GB/s"
 
 
@@ -666,15 +669,24 @@ def run_schedule(args):
                                                 "llama13b_churn" else 64))
     wl = workloads.by_name(args.workload, **kw)
     g = wl.geometry
-    rp = DeviceReplay(wl, device, keep_outputs=False, time_decode=True)
+    grouped = args.decode == "grouped" or (args.decode == "auto" and
+                                            args.workload in GROUPED_WORKLOADS)
+    # a workload with one attend op (sampling, beam) times that call `steps` times
+    n_att = sum(1 for op in wl.ops if op[0] == "attend")
+    reps = max(1, args.steps) if n_att == 1 else 1
+    rp = DeviceReplay(wl, device, keep_outputs=False, time_decode=True, grouped=grouped,
+                      time_reps=reps)
     rp.run()
     torch.cuda.synchronize(device)
     kvp.check_device_error(device)
     attends = {i: (t, l) for (i, _, t, l) in rp.attends}
+    per_op = {}
+    for i, e0, e1 in rp.decode_events:
+        per_op.setdefault(i, []).append(e0.elapsed_time(e1))
     rows = []
-    for n, (i, e0, e1) in enumerate(rp.decode_events):
+    for i in sorted(per_op):
         t, l = attends[i]
-        ms = e0.elapsed_time(e1)
+        ms = float(np.median(per_op[i]))  # median of the op's timed calls
         rows.append((ms, algorithmic_bytes(l, g), unique_bytes(t, l, g), int(np.sum(l))))
     timed = rows[args.warmup:] if len(rows) > args.warmup else rows
     ms = np.array([r[0] for r in timed])
@@ -682,7 +694,11 @@ def run_schedule(args):
     uniq = np.array([r[2] for r in timed], dtype=np.float64)
     toks = np.array([r[3] for r in timed], dtype=np.float64)
     peak, peak_kind = peaks()
-    kernel = "decode_tc" if g.num_q_heads > g.num_kv_heads else "decode_simt"
+    if grouped:
+        kernel = "paged_attention_decode_grouped: group_plan_kernel + decode_tc (grouped)"
+    else:
+        kernel = "paged_attention_decode: " + (
+            "decode_tc" if g.num_q_heads > g.num_kv_heads else "decode_simt")
     st = rp.pool.stats()
     achieved_u = float(uniq.sum() / (ms.sum() * 1e-3) / 1e9)
     res = {
@@ -690,9 +706,12 @@ def run_schedule(args):
         "unit": UNIT, "n_gpus": 1, "steps": len(timed), "warmup": len(rows) - len(timed),
         "ms_per_step": round(float(ms.mean()), 4), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": g.dtype, "data": "synthetic",
-        "config": {"workload": wl.description, "name": wl.name, "timed": "attention calls only"},
+        "config": {"workload": wl.description, "name": wl.name,
+                   "timed": "attention calls only" + (
+                       f" (median of {reps} calls, L2 flushed before each)" if reps > 1 else ""),
+                   "decode": "grouped" if grouped else "per-sequence"},
         "seq_tokens_per_s": round(float(toks.sum() / (ms.sum() * 1e-3)), 1),
-        "roofline": {"kernel": f"paged_attention_decode: {kernel} + decode_reduce_kernel",
+        "roofline": {"kernel": f"{kernel} + decode_reduce_kernel",
                      "bound": "hbm", "achieved_unique": round(achieved_u, 1),
                      "achieved_logical": round(float(logical.sum() / (ms.sum() * 1e-3) / 1e9), 1),
                      "peak": peak, "peak_source": peak_kind, "unit": "GB/s",
@@ -760,6 +779,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--ref-seqs-per-step", type=int, default=1)
+    ap.add_argument("--decode", choices=["auto", "plain", "grouped"], default="auto",
+                    help="decode entry point of the schedule workloads (auto: grouped for "
+                         "the sampling and beam workloads)")
     args = ap.parse_args()
     if args.warmup < 3 and args.workload not in SCHEDULE_WORKLOADS:
         ap.error("--warmup must be >= 3")

@@ -260,6 +260,52 @@ KVP_API int paged_attention_decode(const void* q, const void* k_cache, const voi
                            int32_t partition_size, void* workspace, size_t workspace_bytes,
                            void* out, int32_t dtype, kvp_stream_t stream);
 
+/* Bytes of device workspace paged_attention_decode_grouped needs for this
+ * batch shape: 0 when partition_size <= 0 (the call then runs as
+ * paged_attention_decode, unsplit); else room for num_seqs * num_q_heads *
+ * (P + 1) partial slots of (head_dim + 2) fp32 values, P = ceil(max(
+ * max_context_len, 1) / partition_size), plus the grouping plan (about
+ * 84 bytes per sequence). Always at least kvp_decode_workspace_bytes(...). */
+KVP_API size_t kvp_decode_grouped_workspace_bytes(int32_t num_seqs, int32_t num_q_heads,
+                                          int32_t head_dim, int32_t max_context_len,
+                                          int32_t partition_size);
+
+/* Decode attention for batches whose sequences share cache blocks: the same
+ * arguments and the same result (to fp32 rounding) as paged_attention_decode,
+ * but each run of leading blocks that several sequences hold is read from HBM
+ * once per subgroup of them instead of once per sequence.
+ * Why: sequences forked from one parent (parallel samples of a prompt, beams)
+ * share the physical blocks of their common prefix, stored once with a
+ * reference count ["Your GPU was mostly empty", section "Paging's second gift:
+ * copy-on-write"; "vLLM and PagedAttention", section on parallel sampling and
+ * beam search]. The pages' decode kernel still reads a shared block once per
+ * sequence that attends to it; this entry point, which the pages do not
+ * describe, reads it once per subgroup.
+ * How: a one-CTA kernel groups the sequences by their first block id (only
+ * sequences whose context holds a full block), cuts each group, in sequence
+ * order, into subgroups of up to M members (M = 8 for one query head per KV
+ * head, else 16 / G) and finds each subgroup's shared prefix c: the leading
+ * block-table entries equal across its members, capped at every member's
+ * full blocks. The tensor-core kernel then attends, per KV head, with all the
+ * members' queries of a subgroup as the columns of one contraction over the c
+ * shared blocks, and per sequence over its blocks from c on; both ranges are
+ * split into partitions of partition_size tokens and a log-sum-exp merge
+ * writes every output row.
+ * Needs head_dim 128, block_size 16 or 32, a group G = num_q_heads /
+ * num_kv_heads with 16 / G >= 2 (G <= 8), partition_size > 0 and a multiple
+ * of 128, and num_seqs <= 4096; other batches (and max_context_len == 0) are
+ * decoded by paged_attention_decode with the same workspace, so the call is
+ * valid for every batch paged_attention_decode accepts.
+ * workspace: device, >= kvp_decode_grouped_workspace_bytes(...) bytes,
+ * 256-byte aligned, contents ignored. Errors: those of paged_attention_decode. */
+KVP_API int paged_attention_decode_grouped(const void* q, const void* k_cache, const void* v_cache,
+                           const int32_t* block_tables, const int32_t* context_lens,
+                           int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
+                           int32_t head_dim, int32_t block_size, int32_t num_blocks,
+                           int32_t max_blocks_per_seq, int32_t max_context_len, float scale,
+                           int32_t partition_size, void* workspace, size_t workspace_bytes,
+                           void* out, int32_t dtype, kvp_stream_t stream);
+
 /* Largest split-context scratch, in bytes, that paged_attention_decode_noalloc
  * can serve from its built-in area (40 MiB). */
 #define KVP_STATIC_SCRATCH_BYTES (40u * 1024u * 1024u)

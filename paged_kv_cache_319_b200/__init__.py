@@ -21,7 +21,8 @@ from ._lib import (KVP_BF16, KVP_F16, KvpError, P_i32, P_i64, PoolStats, check, 
 
 __all__ = [
     "BlockPool", "KvpError", "reshape_and_cache", "copy_blocks", "paged_attention_decode",
-    "decode_workspace_bytes", "check_device_error", "kv_bytes_per_token", "version",
+    "decode_workspace_bytes", "decode_grouped_workspace_bytes", "check_device_error",
+    "kv_bytes_per_token", "version",
     "KVP_F16", "KVP_BF16",
 ]
 
@@ -231,14 +232,22 @@ def decode_workspace_bytes(num_seqs: int, num_q_heads: int, head_dim: int, max_c
                                                 partition_size))
 
 
+def decode_grouped_workspace_bytes(num_seqs: int, num_q_heads: int, head_dim: int,
+                                   max_context_len: int, partition_size: int) -> int:
+    return int(lib().kvp_decode_grouped_workspace_bytes(num_seqs, num_q_heads, head_dim,
+                                                        max_context_len, partition_size))
+
+
 def paged_attention_decode(q, k_cache, v_cache, block_tables, context_lens, scale: float,
                            out=None, *, max_context_len: int | None = None,
-                           partition_size: int = 0, workspace=None):
+                           partition_size: int = 0, workspace=None, grouped: bool = False):
     """Decode attention over the paged cache; returns ``out [S, Hq, D]`` (dtype of q).
 
     ``max_context_len`` bounds every ``context_lens`` entry (default: the
     block-table capacity); ``partition_size > 0`` selects the split-context
-    kernel pair. A workspace is allocated with torch when needed and none is given.
+    kernel pair. ``grouped`` calls ``paged_attention_decode_grouped``, which
+    reads blocks shared by several sequences once per subgroup of them. A
+    workspace is allocated with torch when needed and none is given.
     """
     torch = _torch()
     dev = _cuda(q, k_cache, v_cache, block_tables, context_lens)
@@ -258,18 +267,18 @@ def paged_attention_decode(q, k_cache, v_cache, block_tables, context_lens, scal
         _cuda(out)
         if out.shape != q.shape or out.dtype != q.dtype:
             raise ValueError("out mismatch")
-    need = decode_workspace_bytes(S, Hq, D, mcl, partition_size)
+    size_fn = decode_grouped_workspace_bytes if grouped else decode_workspace_bytes
+    need = size_fn(S, Hq, D, mcl, partition_size)
     ws_ptr, ws_bytes = None, 0
     if need:
         if workspace is None:
             workspace = torch.empty(need, dtype=torch.uint8, device=dev)
         _cuda(workspace)
         ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()
-    check(lib().paged_attention_decode(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
-                                       block_tables.data_ptr(), context_lens.data_ptr(), S, Hq,
-                                       Hkv, D, bs, NB, max(MB, 1), mcl, float(scale),
-                                       int(partition_size), ws_ptr, ws_bytes, out.data_ptr(),
-                                       _code(q), _stream(dev)))
+    fn = lib().paged_attention_decode_grouped if grouped else lib().paged_attention_decode
+    check(fn(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), block_tables.data_ptr(),
+             context_lens.data_ptr(), S, Hq, Hkv, D, bs, NB, max(MB, 1), mcl, float(scale),
+             int(partition_size), ws_ptr, ws_bytes, out.data_ptr(), _code(q), _stream(dev)))
     return out
 
 

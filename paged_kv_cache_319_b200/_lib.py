@@ -72,6 +72,9 @@ SIGNATURES = {
     "kvp_decode_workspace_bytes": (sz, [i32, i32, i32, i32, i32]),
     "paged_attention_decode": (C.c_int, [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32,
                                          i32, f32, i32, vp, sz, vp, i32, vp]),
+    "kvp_decode_grouped_workspace_bytes": (sz, [i32, i32, i32, i32, i32]),
+    "paged_attention_decode_grouped": (C.c_int, [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,
+                                                 i32, i32, f32, i32, vp, sz, vp, i32, vp]),
     "paged_attention_decode_noalloc": (C.c_int, [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,
                                                  i32, i32, f32, i32, vp, i32, vp]),
     "kvp_check_device_error": (C.c_int, [vp]),

@@ -107,6 +107,16 @@ __device__ __forceinline__ void pdl_trigger() {
 
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
+// Coherent load of a word that an earlier kernel of the stream wrote while
+// this one may already have been running (programmatic dependent launch):
+// issued after pdl_wait(), never through the read-only (.nc) path, whose loads
+// the compiler may treat as invariant and move above the wait.
+__device__ __forceinline__ int32_t ld_relaxed_gpu(const int32_t* p) {
+  int32_t v;
+  asm volatile("ld.relaxed.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
 // ---- proxies, named barriers -----------------------------------------------
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");

@@ -31,13 +31,17 @@
 namespace kvp {
 namespace dev {
 
+// Grouped decode: word of the plan where the per-sequence shared-prefix block
+// counts start (the plan's layout is described in decode_group.cuh).
+constexpr int kPlanSeqWord = 8;
+
 struct DecodeArgs {
   const void* q;                // [S][Hq][D]
   void* out;                    // [S][Hq][D]
   const int32_t* block_tables;  // [S][max_blocks_per_seq]
   const int32_t* context_lens;  // [S]
-  float* ws_ml;                 // [S][Hq][pmax][2] = (m in log2 units, l)
-  float* ws_acc;                // [S][Hq][pmax][D], unnormalised
+  float* ws_ml;                 // [S][Hq][ws_slots][2] = (m in log2 units, l)
+  float* ws_acc;                // [S][Hq][ws_slots][D], unnormalised
   int32_t num_seqs;
   int32_t num_q_heads;
   int32_t num_kv_heads;
@@ -46,8 +50,14 @@ struct DecodeArgs {
   int32_t max_context_len;
   int32_t part_blocks;  // partition length in blocks (whole context when unsplit)
   int32_t part_tokens;  // part_blocks * block_size
-  int32_t pmax;         // partitions per (sequence, head) in grid and workspace
+  int32_t pmax;         // partitions per (sequence, head) in the grid
+  int32_t ws_slots;     // partial slots per (sequence, head) in the workspace
   float scale_log2;     // scale * log2(e)
+  // Grouped decode only (null otherwise): the grouping plan of
+  // decode_group.cuh. Every (sequence, head) then has ceil(c * bs / P) slots
+  // for its shared prefix followed by the slots of its own range, and the
+  // reduce writes every output row.
+  const int32_t* plan;
 };
 
 __device__ __forceinline__ uint8_t* align_1024(uint8_t* p) {
@@ -104,12 +114,26 @@ __global__ void __launch_bounds__(NW * 32) decode_simt_kernel(
   // The split-context reduce may be scheduled as soon as every CTA of this grid
   // has started; it waits for this grid to complete before reading partials.
   pdl_trigger();
+  // Grouped decode: this kernel attends to each sequence's own blocks, from
+  // the end of its shared prefix on, and was launched while the shared-prefix
+  // kernel ahead of it may still run (every CTA of that kernel had passed its
+  // wait for the plan). One CTA waits for that kernel, so this grid completes
+  // after it and the reduce's wait covers both.
+  const bool grouped = a.plan != nullptr;
+  if (grouped && p == 0 && h == 0 && s == 0) pdl_wait();
   const int32_t ctx = load_ctx(a, s, p == 0 && h == 0 && threadIdx.x == 0);
   const int32_t nblk = (ctx + BS - 1) / BS;
-  const int32_t nparts = (nblk + a.part_blocks - 1) / a.part_blocks;
-  const int32_t b0 = p * a.part_blocks;
-  if (p > 0 && b0 >= nblk) return;  // empty partition (p == 0 always writes its row)
+  int32_t b_first = 0, slot = p;
+  if (grouped) {
+    b_first = ld_relaxed_gpu(a.plan + kPlanSeqWord + s);
+    slot = (b_first + a.part_blocks - 1) / a.part_blocks + p;  // after the shared slots
+  }
+  const int32_t b0 = b_first + p * a.part_blocks;
+  // empty partition (p == 0 always writes its row, except in the grouped decode)
+  if ((p > 0 || grouped) && b0 >= nblk) return;
   const int32_t b1 = min(nblk, b0 + a.part_blocks);
+  // partials go to the workspace for split sequences and in the grouped decode
+  const bool to_ws = grouped || nblk > a.part_blocks;
   const int32_t g = h / (a.num_q_heads / a.num_kv_heads);
   const int32_t* table = a.block_tables + int64_t(s) * a.max_blocks_per_seq;
 
@@ -343,23 +367,24 @@ __global__ void __launch_bounds__(NW * 32) decode_simt_kernel(
     float o = 0.f;
 #pragma unroll
     for (int w = 0; w < NW; ++w) o = fmaf(mg_acc[w * D + t], wgt[w], o);
-    if (nparts <= 1) {
+    if (!to_ws) {
       const float y = (L > 0.f && !any_abort) ? o / L : 0.f;
       static_cast<uint16_t*>(a.out)[row_sh * D + t] = Elem<T>::from_float(y);
     } else {
-      a.ws_acc[(row_sh * a.pmax + p) * D + t] = o;
+      a.ws_acc[(row_sh * a.ws_slots + slot) * D + t] = o;
     }
   }
-  if (nparts > 1 && threadIdx.x == 0) {
-    a.ws_ml[(row_sh * a.pmax + p) * 2 + 0] = any_abort ? -INFINITY : M;
-    a.ws_ml[(row_sh * a.pmax + p) * 2 + 1] = any_abort ? 0.f : L;
+  if (to_ws && threadIdx.x == 0) {
+    a.ws_ml[(row_sh * a.ws_slots + slot) * 2 + 0] = any_abort ? -INFINITY : M;
+    a.ws_ml[(row_sh * a.ws_slots + slot) * 2 + 1] = any_abort ? 0.f : L;
   }
 }
 
 // Log-sum-exp merge of the partitions of split sequences: M = max_p m_p,
 // L = sum_p l_p 2^(m_p - M), out = sum_p 2^(m_p - M) acc_p / L.
 // grid (Hq, S), D threads; sequences with a single partition were written by
-// the partition kernel and are skipped.
+// the partition kernel and are skipped, except in the grouped decode, where
+// this kernel writes every row (a row without tokens is zero).
 template <typename T, int D>
 __global__ void __launch_bounds__(D) decode_reduce_kernel(const DecodeArgs a) {
   extern __shared__ float wsh[];  // [pmax] weights
@@ -367,10 +392,17 @@ __global__ void __launch_bounds__(D) decode_reduce_kernel(const DecodeArgs a) {
   const int h = blockIdx.x;
   const int s = blockIdx.y;
   const int32_t ctx = load_ctx(a, s, false);
-  const int32_t nparts = (ctx + a.part_tokens - 1) / a.part_tokens;
-  if (nparts <= 1) return;
+  int32_t nparts;
+  if (a.plan) {  // grouped: shared-prefix slots, then the sequence's own
+    const int32_t shared = a.plan[kPlanSeqWord + s] * (a.part_tokens / a.part_blocks);
+    nparts = (shared + a.part_tokens - 1) / a.part_tokens +
+             (ctx > shared ? (ctx - shared + a.part_tokens - 1) / a.part_tokens : 0);
+  } else {
+    nparts = (ctx + a.part_tokens - 1) / a.part_tokens;
+    if (nparts <= 1) return;
+  }
   const int64_t row_sh = int64_t(s) * a.num_q_heads + h;
-  const float* ml = a.ws_ml + row_sh * a.pmax * 2;
+  const float* ml = a.ws_ml + row_sh * a.ws_slots * 2;
   __shared__ float red[2];
   if (threadIdx.x == 0) {
     float M = -INFINITY;
@@ -385,7 +417,7 @@ __global__ void __launch_bounds__(D) decode_reduce_kernel(const DecodeArgs a) {
   }
   __syncthreads();
   const float L = red[0];
-  const float* acc = a.ws_acc + row_sh * a.pmax * D;
+  const float* acc = a.ws_acc + row_sh * a.ws_slots * D;
   for (int t = threadIdx.x; t < D; t += blockDim.x) {
     float o = 0.f;
     for (int p = 0; p < nparts; ++p) o = fmaf(acc[int64_t(p) * D + t], wsh[p], o);

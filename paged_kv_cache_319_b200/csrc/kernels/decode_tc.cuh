@@ -36,10 +36,13 @@
 #include <type_traits>
 
 #include "common.cuh"
+#include "decode_group.cuh"
 #include "decode_simt.cuh"
 
 namespace kvp {
 namespace dev {
+
+static_assert(grp::kHdrWords == kPlanSeqWord, "plan layout");
 
 namespace tc {
 
@@ -92,6 +95,10 @@ struct Cfg {
   static constexpr int kSmemBytes = 1024 + kOffCtx;          // + 4 bytes per cached length
   static constexpr int kCtxCap =
       (226 * 1024 - kSmemBytes) / 4 < kCtxCacheMax ? (226 * 1024 - kSmemBytes) / 4 : kCtxCacheMax;
+  // Grouped decode: batches of up to kPlanCap sequences keep their context
+  // lengths and the grouping plan (per-sequence prefix blocks, subgroup table)
+  // in shared memory: 48 bytes per sequence + 80.
+  static constexpr int kPlanCap = (226 * 1024 - kSmemBytes - 80) / 48;
   static_assert(kStages >= 2, "ring stages");
   static_assert(kCtxCap >= 0, "shared memory budget");
   static_assert(kOCol + 2 * kNPV <= kTmemCols, "tensor memory budget");
@@ -163,8 +170,10 @@ __device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, float (&v)[NG]) {
 struct Unit {
   int32_t s, g, p;
   int32_t tok_begin, tok_end;  // token range of the unit
-  int32_t ctx;
+  int32_t ctx;                 // tokens of the block-table row s that the unit may read
   int32_t nparts;
+  int32_t sg;                  // grouped decode: subgroup of a shared-prefix unit, else -1
+  int32_t slot;                // workspace slot of the unit's partial
 };
 
 // ctx_sm: the batch's clamped context lengths in shared memory, or null.
@@ -181,6 +190,63 @@ __device__ __forceinline__ bool decode_unit(const DecodeArgs& a, int64_t u, Unit
   w.tok_begin = w.p * a.part_tokens;
   w.tok_end = min(w.ctx, w.tok_begin + a.part_tokens);
   if (w.tok_end < w.tok_begin) w.tok_end = w.tok_begin;
+  w.sg = -1;
+  w.slot = w.p;
+  return true;
+}
+
+// Grouped decode: units [0, shared_units) are (subgroup, partition of the
+// shared prefix, KV head), the rest (sequence, partition of the sequence's
+// own range from block c on, KV head); KV head fastest in both.
+struct GroupHdr {
+  int64_t shared_units;
+  int32_t psh;          // most shared partitions of any subgroup
+  const int32_t* cblk;  // per sequence: shared-prefix blocks
+  const int32_t* subs;  // subgroup table
+  bool in_smem;         // cblk and subs point at the CTA's shared-memory copy
+};
+
+__device__ __forceinline__ int32_t plan_at(const GroupHdr& gh, const int32_t* p) {
+  return gh.in_smem ? *p : ld_relaxed_gpu(p);
+}
+__device__ __forceinline__ const int32_t* sub_entry(const GroupHdr& gh, int32_t sg) {
+  return gh.subs + int64_t(sg) * grp::kSubWords;
+}
+
+template <int BS>
+__device__ __forceinline__ bool decode_unit_grp(const DecodeArgs& a, int64_t u, Unit& w,
+                                                const int32_t* ctx_sm, const GroupHdr& gh) {
+  if (u < gh.shared_units) {
+    const int64_t per = int64_t(gh.psh) * a.num_kv_heads;
+    w.sg = int32_t(u / per);
+    const int32_t rem = int32_t(u - int64_t(w.sg) * per);
+    w.p = rem / a.num_kv_heads;
+    w.g = rem - w.p * a.num_kv_heads;
+    const int32_t* e = sub_entry(gh, w.sg);
+    const int32_t shared = plan_at(gh, e) * BS;
+    w.tok_begin = w.p * a.part_tokens;
+    if (w.tok_begin >= shared) return false;
+    w.tok_end = min(shared, w.tok_begin + a.part_tokens);
+    w.s = plan_at(gh, e + 4);  // every member holds the same blocks here
+    w.ctx = shared;
+    w.nparts = 0;
+    w.slot = w.p;
+    return true;
+  }
+  u -= gh.shared_units;
+  const int64_t per_seq = int64_t(a.pmax) * a.num_kv_heads;
+  w.s = int32_t(u / per_seq);
+  const int32_t rem = int32_t(u - int64_t(w.s) * per_seq);
+  w.p = rem / a.num_kv_heads;
+  w.g = rem - w.p * a.num_kv_heads;
+  w.ctx = ctx_sm ? ctx_sm[w.s] : load_ctx(a, w.s, w.g == 0 && w.p == 0);
+  const int32_t shared = plan_at(gh, gh.cblk + w.s) * BS;
+  w.tok_begin = shared + w.p * a.part_tokens;
+  if (w.tok_begin >= w.ctx) return false;
+  w.tok_end = min(w.ctx, w.tok_begin + a.part_tokens);
+  w.nparts = 0;
+  w.sg = -1;
+  w.slot = (shared + a.part_tokens - 1) / a.part_tokens + w.p;
   return true;
 }
 
@@ -197,16 +263,19 @@ __device__ __forceinline__ int32_t tiles_of(const Unit& w, int32_t c) {
 // blockIdx.x + gridDim.x, ... (empty partitions and units without tokens
 // skipped), each cut into chunks of up to kChunkTok tokens. Every warp role
 // walks the same stream.
+template <bool GRP, int BS>
 struct ChunkStream {
   int64_t u, stride, num_units;
   const int32_t* ctx_sm;
+  GroupHdr gh;
   Unit w;
   int32_t c, nch;
   bool valid;
 
   __device__ __forceinline__ void init(const DecodeArgs& a, int64_t first, int64_t step,
-                                       int64_t n, const int32_t* ctx_cache) {
+                                       int64_t n, const int32_t* ctx_cache, const GroupHdr& g) {
     ctx_sm = ctx_cache;
+    gh = g;
     stride = step;
     num_units = n;
     u = first - step;
@@ -217,7 +286,8 @@ struct ChunkStream {
   }
   __device__ __forceinline__ void next_unit(const DecodeArgs& a) {
     for (u += stride; u < num_units; u += stride) {
-      if (decode_unit(a, u, w, ctx_sm) && (nch = chunks_of(w)) > 0) {
+      const bool has = GRP ? decode_unit_grp<BS>(a, u, w, ctx_sm, gh) : decode_unit(a, u, w, ctx_sm);
+      if (has && (nch = chunks_of(w)) > 0) {
         c = 0;
         return;
       }
@@ -234,7 +304,11 @@ struct ChunkStream {
 
 }  // namespace tc
 
-template <typename T, int BS, int NG>
+// GRP: grouped decode (a.plan set; launched after the plan kernel with
+// programmatic serialisation). num_units then counts the per-sequence units
+// (0 when the CUDA-core kernel takes them); the shared-prefix units are read
+// from the plan.
+template <typename T, int BS, int NG, bool GRP>
 __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
     const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
     const __grid_constant__ CUtensorMap qmap, const DecodeArgs a, int64_t num_units) {
@@ -274,6 +348,8 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
   uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + L::kOffTmemPtr);
   int32_t* ctx_cache = reinterpret_cast<int32_t*>(smem + L::kOffCtx);
   const int32_t* ctx_sm = a.num_seqs <= L::kCtxCap ? ctx_cache : nullptr;
+  // grouped decode: plan copy after the context lengths (when it fits)
+  const bool plan_sm = GRP && a.num_seqs <= L::kPlanCap;
   if (ctx_sm) {
     for (int i = threadIdx.x; i < a.num_seqs; i += blockDim.x)
       ctx_cache[i] = load_ctx(a, i, blockIdx.x == 0);  // clamped; out-of-range reported once
@@ -282,7 +358,9 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  pdl_trigger();  // the split-context reduce waits for this grid to complete
+  // the split-context reduce waits for this grid to complete; in the grouped
+  // decode the trigger comes after the wait for the plan (below)
+  if constexpr (!GRP) pdl_trigger();
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStages; ++i) {
@@ -319,6 +397,34 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
 
   const int32_t G = a.num_q_heads / a.num_kv_heads;
   const int32_t rows_total = a.num_blocks * a.num_kv_heads * BS;
+  tc::GroupHdr gh{0, 0, nullptr, nullptr, false};
+  if constexpr (GRP) {
+    pdl_wait();  // the plan kernel has completed and its writes are visible
+    // The kernel launched next (the CUDA-core kernel for the sequences' own
+    // ranges, or the reduce) may start once every CTA is past this point, so
+    // it may read the plan without a wait of its own.
+    pdl_trigger();
+    const int32_t n_sub = ld_relaxed_gpu(a.plan);
+    gh.psh = ld_relaxed_gpu(a.plan + 1);
+    gh.shared_units = int64_t(n_sub) * gh.psh * a.num_kv_heads;
+    num_units += gh.shared_units;
+    const int32_t* g_cblk = a.plan + kPlanSeqWord;
+    const int32_t* g_subs = a.plan + grp::sub_offset(a.num_seqs);
+    if (plan_sm) {
+      int32_t* c_sm = ctx_cache + a.num_seqs;
+      int32_t* s_sm = c_sm + a.num_seqs;
+      for (int i = threadIdx.x; i < a.num_seqs; i += blockDim.x) c_sm[i] = ld_relaxed_gpu(g_cblk + i);
+      for (int i = threadIdx.x; i < n_sub * grp::kSubWords; i += blockDim.x)
+        s_sm[i] = ld_relaxed_gpu(g_subs + i);
+      __syncthreads();
+      gh.cblk = c_sm;
+      gh.subs = s_sm;
+      gh.in_smem = true;
+    } else {
+      gh.cblk = g_cblk;
+      gh.subs = g_subs;
+    }
+  }
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -335,7 +441,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
     uint32_t ucnt = 0;  // units started
     bool ok = true;
     // Lane j's TMA row of block j of a chunk (one chunk = 512 / BS <= 32 blocks).
-    auto chunk_row = [&](const tc::ChunkStream& cs) -> int32_t {
+    auto chunk_row = [&](const tc::ChunkStream<GRP, BS>& cs) -> int32_t {
       const tc::Unit& w = cs.w;
       const int32_t ntile = cs.tiles();
       const int32_t blk0 = (w.tok_begin + cs.c * kChunkTok) / BS;
@@ -369,28 +475,56 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
         __syncwarp();
       }
     };
-    tc::ChunkStream cur;
-    cur.init(a, blockIdx.x, gridDim.x, num_units, ctx_sm);
+    tc::ChunkStream<GRP, BS> cur;
+    cur.init(a, blockIdx.x, gridDim.x, num_units, ctx_sm, gh);
     int32_t pend_row = rows_total, pend_tiles = 0;
     bool have_pend = false;
     int32_t row = cur.valid ? chunk_row(cur) : rows_total;
     while (cur.valid && ok) {
       // the next chunk's block ids are loaded now and used one iteration later
-      tc::ChunkStream nxt = cur;
+      tc::ChunkStream<GRP, BS> nxt = cur;
       nxt.advance(a);
       const int32_t row_next = nxt.valid ? chunk_row(nxt) : rows_total;
       if (cur.first()) {
         const uint32_t qb = ucnt & 1u;
-        if (lane == 0) {
-          ok = mbar_wait(&q_empty[qb], ((ucnt >> 1) & 1u) ^ 1u, 0x7100u);
+        if (GRP && cur.w.sg >= 0) {
+          // shared-prefix unit: column j is query head g * G + j % G of member
+          // j / G; the warp gathers the rows into the 128-byte-swizzled layout
+          // a TMA load would produce (chunk c of row j at (c ^ (j & 7)) * 16)
+          if (lane == 0) ok = mbar_wait(&q_empty[qb], ((ucnt >> 1) & 1u) ^ 1u, 0x7100u);
+          ok = __shfl_sync(0xffffffffu, ok, 0);
           if (ok) {
-            mbar_arrive_expect_tx(&q_full[qb], kQBytes);
-            const int32_t qrow = cur.w.s * a.num_q_heads + cur.w.g * G;
-            tma_load_2d(qbuf + qb * kQBytes, &qmap, &q_full[qb], 0, qrow, pol_q);
-            tma_load_2d(qbuf + qb * kQBytes + kN * 128, &qmap, &q_full[qb], 64, qrow, pol_q);
+            const int32_t* e = tc::sub_entry(gh, cur.w.sg);
+            const int32_t ncol = tc::plan_at(gh, e + 1) * G;
+            uint8_t* qdst = qbuf + qb * kQBytes;
+            for (int idx = lane; idx < kN * 16; idx += 32) {
+              const int j = idx >> 4, ch = idx & 15;
+              uint4 v = make_uint4(0, 0, 0, 0);
+              if (j < ncol) {
+                const int32_t m = j / G;
+                const int64_t qrow =
+                    int64_t(tc::plan_at(gh, e + 4 + m)) * a.num_q_heads + cur.w.g * G + (j - m * G);
+                v = __ldg(reinterpret_cast<const uint4*>(static_cast<const T*>(a.q) + qrow * kD) + ch);
+              }
+              *reinterpret_cast<uint4*>(qdst + (ch >> 3) * (kN * 128) + j * 128 +
+                                        (((ch & 7) ^ (j & 7)) << 4)) = v;
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&q_full[qb]);
           }
+        } else {
+          if (lane == 0) {
+            ok = mbar_wait(&q_empty[qb], ((ucnt >> 1) & 1u) ^ 1u, 0x7100u);
+            if (ok) {
+              mbar_arrive_expect_tx(&q_full[qb], kQBytes);
+              const int32_t qrow = cur.w.s * a.num_q_heads + cur.w.g * G;
+              tma_load_2d(qbuf + qb * kQBytes, &qmap, &q_full[qb], 0, qrow, pol_q);
+              tma_load_2d(qbuf + qb * kQBytes + kN * 128, &qmap, &q_full[qb], 64, qrow, pol_q);
+            }
+          }
+          ok = __shfl_sync(0xffffffffu, ok, 0);
         }
-        ok = __shfl_sync(0xffffffffu, ok, 0);
         ++ucnt;
         if (!ok) break;
       }
@@ -488,8 +622,8 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
         umma_commit(&p_free[b]);
       }
     };
-    tc::ChunkStream cur;
-    cur.init(a, blockIdx.x, gridDim.x, num_units, ctx_sm);
+    tc::ChunkStream<GRP, BS> cur;
+    cur.init(a, blockIdx.x, gridDim.x, num_units, ctx_sm, gh);
     uint32_t pend_b = 0, pend_use = 0;
     int32_t pend_tiles = 0, pend_zero = kTileTok;
     bool have_pend = false;
@@ -536,8 +670,9 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
     auto wait_all = [&](uint64_t* bar, uint32_t parity, uint32_t where) {
       return __all_sync(0xffffffffu, mbar_wait(bar, parity, where)) != 0;
     };
-    // Units without tokens (context length 0) attend to nothing: zero rows.
-    for (int64_t u = blockIdx.x; u < num_units; u += gridDim.x) {
+    // Units without tokens (context length 0) attend to nothing: zero rows
+    // (written by the reduce in the grouped decode).
+    for (int64_t u = blockIdx.x; !GRP && u < num_units; u += gridDim.x) {
       tc::Unit w;
       if (!tc::decode_unit(a, u, w, ctx_sm) || tc::chunks_of(w) > 0) continue;
       for (int j = 0; j < G; ++j)
@@ -595,19 +730,26 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
       ++ucnt;
       if (!ok) return;
       const int32_t h0 = pw.g * G;
+      // grouped decode: a shared-prefix unit's columns are its members' heads
+      const int32_t* ge = (GRP && pw.sg >= 0) ? tc::sub_entry(gh, pw.sg) : nullptr;
+      const int32_t ncol = ge ? tc::plan_at(gh, ge + 1) * G : G;
 #pragma unroll
       for (int j = 0; j < NG; ++j) {
         const float Lj = (rl[j] + rl[kN + j]) + (rl[2 * kN + j] + rl[3 * kN + j]);
-        if (j < G) {
-          const int64_t row_sh = int64_t(pw.s) * a.num_q_heads + h0 + j;
-          if (pw.nparts <= 1) {
+        if (j < ncol) {
+          int64_t row_sh = int64_t(pw.s) * a.num_q_heads + h0 + j;
+          if (ge) {
+            const int32_t m = j / G;
+            row_sh = int64_t(tc::plan_at(gh, ge + 4 + m)) * a.num_q_heads + h0 + (j - m * G);
+          }
+          if (!GRP && pw.nparts <= 1) {
             const float y = Lj > 0.f ? acc[j] / Lj : 0.f;
             static_cast<uint16_t*>(a.out)[row_sh * kD + r] = Elem<T>::from_float(y);
           } else {
-            a.ws_acc[(row_sh * a.pmax + pw.p) * kD + r] = acc[j];
+            a.ws_acc[(row_sh * a.ws_slots + pw.slot) * kD + r] = acc[j];
             if (r == 0) {
-              a.ws_ml[(row_sh * a.pmax + pw.p) * 2 + 0] = m_run[j];
-              a.ws_ml[(row_sh * a.pmax + pw.p) * 2 + 1] = Lj;
+              a.ws_ml[(row_sh * a.ws_slots + pw.slot) * 2 + 0] = m_run[j];
+              a.ws_ml[(row_sh * a.ws_slots + pw.slot) * 2 + 1] = Lj;
             }
           }
         }
@@ -617,8 +759,8 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
       }
     };
 
-    tc::ChunkStream cur;
-    cur.init(a, blockIdx.x, gridDim.x, num_units, ctx_sm);
+    tc::ChunkStream<GRP, BS> cur;
+    cur.init(a, blockIdx.x, gridDim.x, num_units, ctx_sm, gh);
     while (cur.valid && ok) {
       const uint32_t b = cc & 1u;
       const uint32_t use = cc >> 1;

@@ -8,6 +8,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstdint>
@@ -17,6 +18,7 @@
 
 #include "kernels/cache_ops.cuh"
 #include "kernels/common.cuh"
+#include "kernels/decode_group.cuh"
 #include "kernels/decode_simt.cuh"
 #include "kernels/decode_tc.cuh"
 #include "status.h"
@@ -159,10 +161,29 @@ Workspace ws_layout(int64_t S, int64_t Hq, int64_t D, int64_t pmax) {
   return w;
 }
 
+// Grouped decode: [ml][acc][plan], with pmax + 1 slots per (sequence, head)
+// (a sequence's shared prefix and its own range may each end in a partial
+// partition) and the grouping plan.
+struct GroupWorkspace {
+  size_t ml_bytes, acc_bytes, plan_bytes, total;
+};
+
+GroupWorkspace group_ws_layout(int64_t S, int64_t Hq, int64_t D, int64_t pmax) {
+  auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
+  GroupWorkspace w{};
+  w.ml_bytes = up(size_t(S * Hq * (pmax + 1) * 2 * 4));
+  w.acc_bytes = up(size_t(S * Hq * (pmax + 1) * D * 4));
+  w.plan_bytes = up(size_t(kvp::dev::grp::plan_words(S) * 4));
+  w.total = w.ml_bytes + w.acc_bytes + w.plan_bytes;
+  return w;
+}
+
 // ---- decode launches ----------------------------------------------------------
+// programmatic: launched with programmatic stream serialisation (the grouped
+// decode, after the shared-prefix kernel).
 template <typename T, int D, int BS>
 int launch_simt(const CUtensorMap& km, const CUtensorMap& vm, const kvp::dev::DecodeArgs& a,
-                cudaStream_t st) {
+                cudaStream_t st, bool programmatic = false) {
   constexpr int NW = (BS * D * 2 >= 8192 && KVP_SIMT_WARPS > 1) ? KVP_SIMT_WARPS / 2 : KVP_SIMT_WARPS;
   constexpr int NST = KVP_SIMT_STAGES;
   using C = kvp::dev::SimtCfg<T, D, BS, NW, NST>;
@@ -170,7 +191,22 @@ int launch_simt(const CUtensorMap& km, const CUtensorMap& vm, const kvp::dev::De
   cudaError_t e = ensure_smem(k, C::kSmemBytes);
   if (e != cudaSuccess) return cuda_fail(e, "decode (CUDA cores): smem attribute");
   dim3 grid(a.pmax, a.num_q_heads, a.num_seqs);
-  k<<<grid, NW * 32, C::kSmemBytes, st>>>(km, vm, a);
+  if (!programmatic) {
+    k<<<grid, NW * 32, C::kSmemBytes, st>>>(km, vm, a);
+  } else {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(NW * 32);
+    cfg.dynamicSmemBytes = size_t(C::kSmemBytes);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, k, km, vm, a);
+    if (e != cudaSuccess) return cuda_fail(e, "decode (CUDA cores): launch");
+  }
   e = cudaGetLastError();
   return e == cudaSuccess ? KVP_OK : cuda_fail(e, "decode (CUDA cores): launch");
 }
@@ -178,7 +214,7 @@ int launch_simt(const CUtensorMap& km, const CUtensorMap& vm, const kvp::dev::De
 template <typename T, int BS, int NG>
 int launch_tc(const CUtensorMap& km, const CUtensorMap& vm, const CUtensorMap& qm,
               const kvp::dev::DecodeArgs& a, cudaStream_t st) {
-  auto k = kvp::dev::decode_tc_kernel<T, BS, NG>;
+  auto k = kvp::dev::decode_tc_kernel<T, BS, NG, false>;
   // context lengths of small batches are cached in shared memory
   using Cfg = kvp::dev::tc::Cfg<NG>;
   const int ctx_bytes = a.num_seqs <= Cfg::kCtxCap ? 4 * a.num_seqs : 0;
@@ -199,7 +235,7 @@ int launch_reduce(const kvp::dev::DecodeArgs& a, cudaStream_t st) {
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(a.num_q_heads, a.num_seqs);
   cfg.blockDim = dim3(D);
-  cfg.dynamicSmemBytes = size_t(a.pmax) * 4;
+  cfg.dynamicSmemBytes = size_t(a.ws_slots) * 4;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -222,6 +258,53 @@ int simt_by_bs(int bs, const CUtensorMap& km, const CUtensorMap& vm, const kvp::
   return fail(KVP_ERR_INVALID, "block_size %d not supported", bs);
 }
 
+// Grouped decode, tensor-core kernel: launched right after the plan kernel
+// with programmatic serialisation; its CTAs set up while the plan is built and
+// wait for it (griddepcontrol.wait) before reading it.
+// with_private: the kernel also takes every sequence's own range (else the
+// CUDA-core kernel launched after it does).
+template <typename T, int BS, int NG>
+int launch_tc_grouped(const CUtensorMap& km, const CUtensorMap& vm, const CUtensorMap& qm,
+                      const kvp::dev::DecodeArgs& a, cudaStream_t st, bool with_private) {
+  auto k = kvp::dev::decode_tc_kernel<T, BS, NG, true>;
+  using Cfg = kvp::dev::tc::Cfg<NG>;
+  // shared-memory tail: context lengths, per-sequence prefix blocks and the
+  // subgroup table when they fit (S <= kPlanCap), else the context lengths alone
+  auto plan_bytes = [](int S) { return 8 * S + (S / 2 + 1) * kvp::dev::grp::kSubWords * 4; };
+  const int S = a.num_seqs;
+  const int ctx_bytes = S <= Cfg::kPlanCap ? plan_bytes(S) : (S <= Cfg::kCtxCap ? 4 * S : 0);
+  const int tail_max = std::max(4 * Cfg::kCtxCap, plan_bytes(Cfg::kPlanCap));
+  cudaError_t e = ensure_smem(k, Cfg::kSmemBytes + tail_max);
+  if (e != cudaSuccess) return cuda_fail(e, "grouped decode: smem attribute");
+  const int64_t units = with_private ? int64_t(a.num_seqs) * a.num_kv_heads * a.pmax : 0;
+  // at most S / 2 subgroups of at most pmax shared partitions each
+  const int64_t bound = std::max<int64_t>(
+      1, units + int64_t(a.num_seqs / 2) * a.num_kv_heads * a.pmax);
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(unsigned(bound < sm_count() ? bound : sm_count()));
+  cfg.blockDim = dim3(kvp::dev::tc::kThreads);
+  cfg.dynamicSmemBytes = size_t(Cfg::kSmemBytes + ctx_bytes);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, k, km, vm, qm, a, units);
+  if (e == cudaSuccess) e = cudaGetLastError();
+  return e == cudaSuccess ? KVP_OK : cuda_fail(e, "grouped decode: launch");
+}
+
+template <typename T>
+int tc_grouped_dispatch(int bs, int ng, const CUtensorMap& km, const CUtensorMap& vm,
+                        const CUtensorMap& qm, const kvp::dev::DecodeArgs& a, cudaStream_t st,
+                        bool with_private) {
+  if (bs == 16) return ng == 8 ? launch_tc_grouped<T, 16, 8>(km, vm, qm, a, st, with_private)
+                               : launch_tc_grouped<T, 16, 16>(km, vm, qm, a, st, with_private);
+  return ng == 8 ? launch_tc_grouped<T, 32, 8>(km, vm, qm, a, st, with_private)
+                 : launch_tc_grouped<T, 32, 16>(km, vm, qm, a, st, with_private);
+}
+
 template <typename T>
 int tc_dispatch(int bs, int G, const CUtensorMap& km, const CUtensorMap& vm, const CUtensorMap& qm,
                 const kvp::dev::DecodeArgs& a, cudaStream_t st) {
@@ -234,6 +317,40 @@ int tc_dispatch(int bs, int G, const CUtensorMap& km, const CUtensorMap& vm, con
   if (ng == 4) return launch_tc<T, 32, 4>(km, vm, qm, a, st);
   if (ng == 8) return launch_tc<T, 32, 8>(km, vm, qm, a, st);
   return launch_tc<T, 32, 16>(km, vm, qm, a, st);
+}
+
+// Argument checks of the decode entry points (fn names the caller in the
+// messages); *empty is set when there is nothing to do (no sequences).
+int check_decode(const char* fn, const void* q, const void* k_cache, const void* v_cache,
+                 const int32_t* block_tables, const int32_t* context_lens, int32_t num_seqs,
+                 int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                 int32_t num_blocks, int32_t max_blocks_per_seq, int32_t max_context_len,
+                 float scale, int32_t partition_size, const void* out, int32_t dtype, bool* empty) {
+  *empty = false;
+  if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_blocks <= 0 ||
+      max_blocks_per_seq <= 0 || max_context_len < 0 || partition_size < 0)
+    return fail(KVP_ERR_INVALID, "%s: bad sizes", fn);
+  if (num_q_heads % num_kv_heads) return fail(KVP_ERR_INVALID, "%s: num_q_heads %% num_kv_heads != 0", fn);
+  if (head_dim != 64 && head_dim != 128) return fail(KVP_ERR_INVALID, "%s: head_dim must be 64 or 128", fn);
+  if (block_size != 8 && block_size != 16 && block_size != 32)
+    return fail(KVP_ERR_INVALID, "%s: block_size must be 8, 16 or 32", fn);
+  if (dtype != KVP_F16 && dtype != KVP_BF16) return fail(KVP_ERR_INVALID, "%s: bad dtype", fn);
+  if (int64_t(max_context_len) > int64_t(max_blocks_per_seq) * block_size)
+    return fail(KVP_ERR_INVALID, "%s: max_context_len > max_blocks_per_seq * block_size", fn);
+  if (int64_t(num_blocks) * num_kv_heads * block_size >= (int64_t(1) << 31))
+    return fail(KVP_ERR_INVALID, "%s: pool too large for 32-bit row coordinates", fn);
+  if (partition_size % block_size) return fail(KVP_ERR_INVALID, "%s: partition_size must be a multiple of block_size", fn);
+  if (!std::isfinite(scale)) return fail(KVP_ERR_INVALID, "%s: scale not finite", fn);
+  if (num_seqs == 0) {
+    *empty = true;
+    return KVP_OK;
+  }
+  if (!q || !k_cache || !v_cache || !block_tables || !context_lens || !out)
+    return fail(KVP_ERR_INVALID, "%s: NULL pointer", fn);
+  if (!aligned(q, 16) || !aligned(out, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
+      !aligned(block_tables, 4) || !aligned(context_lens, 4))
+    return fail(KVP_ERR_INVALID, "%s: misaligned pointer", fn);
+  return KVP_OK;
 }
 
 }  // namespace
@@ -307,26 +424,12 @@ int paged_attention_decode(const void* q, const void* k_cache, const void* v_cac
                            int32_t max_blocks_per_seq, int32_t max_context_len, float scale,
                            int32_t partition_size, void* workspace, size_t workspace_bytes,
                            void* out, int32_t dtype, kvp_stream_t stream) {
-  if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_blocks <= 0 ||
-      max_blocks_per_seq <= 0 || max_context_len < 0 || partition_size < 0)
-    return fail(KVP_ERR_INVALID, "paged_attention_decode: bad sizes");
-  if (num_q_heads % num_kv_heads) return fail(KVP_ERR_INVALID, "paged_attention_decode: num_q_heads %% num_kv_heads != 0");
-  if (head_dim != 64 && head_dim != 128) return fail(KVP_ERR_INVALID, "paged_attention_decode: head_dim must be 64 or 128");
-  if (block_size != 8 && block_size != 16 && block_size != 32)
-    return fail(KVP_ERR_INVALID, "paged_attention_decode: block_size must be 8, 16 or 32");
-  if (dtype != KVP_F16 && dtype != KVP_BF16) return fail(KVP_ERR_INVALID, "paged_attention_decode: bad dtype");
-  if (int64_t(max_context_len) > int64_t(max_blocks_per_seq) * block_size)
-    return fail(KVP_ERR_INVALID, "paged_attention_decode: max_context_len > max_blocks_per_seq * block_size");
-  if (int64_t(num_blocks) * num_kv_heads * block_size >= (int64_t(1) << 31))
-    return fail(KVP_ERR_INVALID, "paged_attention_decode: pool too large for 32-bit row coordinates");
-  if (partition_size % block_size) return fail(KVP_ERR_INVALID, "paged_attention_decode: partition_size must be a multiple of block_size");
-  if (!std::isfinite(scale)) return fail(KVP_ERR_INVALID, "paged_attention_decode: scale not finite");
-  if (num_seqs == 0) return KVP_OK;
-  if (!q || !k_cache || !v_cache || !block_tables || !context_lens || !out)
-    return fail(KVP_ERR_INVALID, "paged_attention_decode: NULL pointer");
-  if (!aligned(q, 16) || !aligned(out, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
-      !aligned(block_tables, 4) || !aligned(context_lens, 4))
-    return fail(KVP_ERR_INVALID, "paged_attention_decode: misaligned pointer");
+  bool empty = false;
+  const int crc = check_decode("paged_attention_decode", q, k_cache, v_cache, block_tables,
+                               context_lens, num_seqs, num_q_heads, num_kv_heads, head_dim,
+                               block_size, num_blocks, max_blocks_per_seq, max_context_len, scale,
+                               partition_size, out, dtype, &empty);
+  if (crc || empty) return crc;
 
   const int G = num_q_heads / num_kv_heads;
   const bool tensor_cores = G > 1 && G <= 16 && head_dim == 128 && (block_size == 16 || block_size == 32);
@@ -365,6 +468,7 @@ int paged_attention_decode(const void* q, const void* k_cache, const void* v_cac
   a.part_blocks = part_tokens / block_size;
   a.part_tokens = part_tokens;
   a.pmax = pmax;
+  a.ws_slots = pmax;
   a.scale_log2 = scale * 1.4426950408889634f;
 
   const uint64_t rows = uint64_t(num_blocks) * num_kv_heads * block_size;
@@ -399,6 +503,115 @@ int paged_attention_decode(const void* q, const void* k_cache, const void* v_cac
   if (head_dim == 128)
     return dtype == KVP_F16 ? launch_reduce<__half, 128>(a, st) : launch_reduce<__nv_bfloat16, 128>(a, st);
   return dtype == KVP_F16 ? launch_reduce<__half, 64>(a, st) : launch_reduce<__nv_bfloat16, 64>(a, st);
+}
+
+size_t kvp_decode_grouped_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, int32_t head_dim,
+                                          int32_t max_context_len, int32_t partition_size) {
+  if (partition_size <= 0 || num_seqs <= 0 || num_q_heads <= 0 || head_dim <= 0 || max_context_len < 0)
+    return 0;
+  const int64_t ctx = max_context_len > 0 ? max_context_len : 1;
+  const int64_t pmax = (ctx + partition_size - 1) / partition_size;
+  // covers paged_attention_decode's own layout too (pmax slots, no plan)
+  return group_ws_layout(num_seqs, num_q_heads, head_dim, pmax).total;
+}
+
+int paged_attention_decode_grouped(const void* q, const void* k_cache, const void* v_cache,
+                                   const int32_t* block_tables, const int32_t* context_lens,
+                                   int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
+                                   int32_t head_dim, int32_t block_size, int32_t num_blocks,
+                                   int32_t max_blocks_per_seq, int32_t max_context_len, float scale,
+                                   int32_t partition_size, void* workspace, size_t workspace_bytes,
+                                   void* out, int32_t dtype, kvp_stream_t stream) {
+  bool empty = false;
+  const int crc = check_decode("paged_attention_decode_grouped", q, k_cache, v_cache, block_tables,
+                               context_lens, num_seqs, num_q_heads, num_kv_heads, head_dim,
+                               block_size, num_blocks, max_blocks_per_seq, max_context_len, scale,
+                               partition_size, out, dtype, &empty);
+  if (crc || empty) return crc;
+  // Columns of the tensor-core contraction: 8 for one query head per KV head
+  // (up to 8 members per subgroup), else 16 (16 / G members).
+  const int G = num_q_heads / num_kv_heads;
+  const int ng = G == 1 ? 8 : 16;
+  const int mmax = ng / G;
+  const bool grouped = head_dim == 128 && (block_size == 16 || block_size == 32) && G <= 16 &&
+                       mmax >= 2 && partition_size > 0 && partition_size % 128 == 0 &&
+                       num_seqs <= kvp::dev::grp::kMaxSeqs && max_context_len > 0;
+  if (!grouped)
+    return paged_attention_decode(q, k_cache, v_cache, block_tables, context_lens, num_seqs,
+                                  num_q_heads, num_kv_heads, head_dim, block_size, num_blocks,
+                                  max_blocks_per_seq, max_context_len, scale, partition_size,
+                                  workspace, workspace_bytes, out, dtype, stream);
+
+  const int32_t pmax = (max_context_len + partition_size - 1) / partition_size;
+  const GroupWorkspace wl = group_ws_layout(num_seqs, num_q_heads, head_dim, pmax);
+  if (!workspace || workspace_bytes < wl.total)
+    return fail(KVP_ERR_INVALID, "paged_attention_decode_grouped: workspace of %zu bytes needed", wl.total);
+  if (!aligned(workspace, 256))
+    return fail(KVP_ERR_INVALID, "paged_attention_decode_grouped: workspace not 256-byte aligned");
+
+  char* ws = static_cast<char*>(workspace);
+  int32_t* plan = reinterpret_cast<int32_t*>(ws + wl.ml_bytes + wl.acc_bytes);
+  kvp::dev::DecodeArgs a{};
+  a.q = q;
+  a.out = out;
+  a.block_tables = block_tables;
+  a.context_lens = context_lens;
+  a.ws_ml = reinterpret_cast<float*>(ws);
+  a.ws_acc = reinterpret_cast<float*>(ws + wl.ml_bytes);
+  a.num_seqs = num_seqs;
+  a.num_q_heads = num_q_heads;
+  a.num_kv_heads = num_kv_heads;
+  a.num_blocks = num_blocks;
+  a.max_blocks_per_seq = max_blocks_per_seq;
+  a.max_context_len = max_context_len;
+  a.part_blocks = partition_size / block_size;
+  a.part_tokens = partition_size;
+  a.pmax = pmax;
+  a.ws_slots = pmax + 1;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.plan = plan;
+
+  // One query head per KV head: the CUDA-core kernel takes the sequences' own
+  // ranges (short, many: its independent per-warp pipelines suit them); with
+  // grouped-query heads the tensor-core kernel takes both.
+  const bool simt_private = G == 1;
+  const uint64_t rows = uint64_t(num_blocks) * num_kv_heads * block_size;
+  CUtensorMap km, vm, qm, km3, vm3;
+  int rc = make_map(&km, k_cache, dtype, rows, head_dim, block_size);
+  if (!rc) rc = make_map(&vm, v_cache, dtype, rows, head_dim, block_size);
+  if (!rc) rc = make_map(&qm, q, dtype, uint64_t(num_seqs) * num_q_heads, head_dim, kvp::dev::tc::kN);
+  if (!rc && simt_private) rc = make_map_halves(&km3, k_cache, dtype, rows, block_size);
+  if (!rc && simt_private) rc = make_map_halves(&vm3, v_cache, dtype, rows, block_size);
+  if (rc) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+  // 1. the plan (one CTA)
+  using namespace kvp::dev;
+  cudaError_t e = ensure_smem(group_plan_kernel, int(grp::plan_smem_bytes(grp::kMaxSeqs)));
+  if (e != cudaSuccess) return cuda_fail(e, "grouped decode: plan smem attribute");
+  group_plan_kernel<<<1, grp::plan_threads(grp::sort_len(num_seqs)), grp::plan_smem_bytes(num_seqs),
+                      st>>>(block_tables, context_lens, num_seqs, max_blocks_per_seq,
+                            max_context_len, block_size, partition_size, mmax, num_blocks, plan);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "grouped decode: plan launch");
+  // 2. shared prefixes once per subgroup (and, with grouped-query heads, every
+  // sequence's own range) on the tensor cores
+  rc = dtype == KVP_F16
+           ? tc_grouped_dispatch<__half>(block_size, ng, km, vm, qm, a, st, !simt_private)
+           : tc_grouped_dispatch<__nv_bfloat16>(block_size, ng, km, vm, qm, a, st, !simt_private);
+  if (rc) return rc;
+  // 2b. every sequence's own range on the CUDA cores, overlapping the tail of 2
+  if (simt_private) {
+    if (block_size == 16)
+      rc = dtype == KVP_F16 ? launch_simt<__half, 128, 16>(km3, vm3, a, st, true)
+                            : launch_simt<__nv_bfloat16, 128, 16>(km3, vm3, a, st, true);
+    else
+      rc = dtype == KVP_F16 ? launch_simt<__half, 128, 32>(km3, vm3, a, st, true)
+                            : launch_simt<__nv_bfloat16, 128, 32>(km3, vm3, a, st, true);
+    if (rc) return rc;
+  }
+  // 3. the log-sum-exp merge of every row
+  return dtype == KVP_F16 ? launch_reduce<__half, 128>(a, st) : launch_reduce<__nv_bfloat16, 128>(a, st);
 }
 
 }  // extern "C"

@@ -5,7 +5,7 @@ release into block tables, slots and copy-on-write pairs; at each ``sync``
 the pending copies run (``copy_blocks``) and then every token appended since
 the previous sync is written to its slot (``reshape_and_cache``); at each
 ``attend`` the batch's block tables and lengths go to the device and
-``paged_attention_decode`` runs. Per-step order: copies, then scatter, then
+``paged_attention_decode`` (or, with ``grouped``, ``paged_attention_decode_grouped``) runs. Per-step order: copies, then scatter, then
 attention, because a new token may land in a block copied in the same step.
 
 Inputs (K/V of appended tokens, q of each attend) are drawn from
@@ -31,7 +31,8 @@ def bits_to_tensor(bits: np.ndarray, dtype: str, device):
 
 
 class DeviceReplay:
-    def __init__(self, wl, device="cuda", keep_outputs: bool = True, time_decode: bool = False):
+    def __init__(self, wl, device="cuda", keep_outputs: bool = True, time_decode: bool = False,
+                 grouped: bool = False, time_reps: int = 1):
         import torch
 
         g = wl.geometry
@@ -50,6 +51,8 @@ class DeviceReplay:
         self.outputs = {}          # op_index -> out tensor
         self.keep_outputs = keep_outputs
         self.time_decode = time_decode
+        self.grouped = grouped     # decode through paged_attention_decode_grouped
+        self.time_reps = max(1, int(time_reps))  # timed calls per attend op (time_decode)
         self.decode_events = []    # (op_index, start event, end event) around each decode call
         self.next_index = 0
 
@@ -121,24 +124,32 @@ class DeviceReplay:
             bt = torch.from_numpy(tables).to(self.device)
             cl = torch.from_numpy(lens).to(self.device)
             part = kw.get("partition_size", self.wl.partition_size)
+            grouped = kw.get("grouped", self.grouped)
+            mcl = int(lens.max()) if len(lens) else 0
+            call = lambda: paged_attention_decode(q, self.k_cache, self.v_cache, bt, cl,  # noqa: E731
+                                                  self.wl.scale, max_context_len=mcl,
+                                                  partition_size=part, grouped=grouped)
             if self.time_decode:
-                # an untimed call, then an L2-sized write, keep the stream busy while
-                # the timed call is issued (so the start event does not time the host's
-                # launch work) and leave none of the KV blocks in L2
-                paged_attention_decode(q, self.k_cache, self.v_cache, bt, cl, self.wl.scale,
-                                       max_context_len=int(lens.max()) if len(lens) else 0,
-                                       partition_size=part)
+                # an untimed call, then before each timed call an L2 flush: a
+                # 256 MB write, then a 256 MB read of another buffer, which writes
+                # the dirty lines back before the timed region (a write alone would
+                # leave L2 full of dirty lines that the timed call's reads evict,
+                # adding up to L2's size of write-back to its traffic); the flush
+                # also keeps the stream busy while the timed call is issued
+                call()
                 if not hasattr(self, "_l2_flush"):
                     self._l2_flush = torch.empty(256 << 20, dtype=torch.uint8, device=self.device)
-                self._l2_flush.fill_(1)
-                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                e0.record()
-            out = paged_attention_decode(q, self.k_cache, self.v_cache, bt, cl, self.wl.scale,
-                                         max_context_len=int(lens.max()) if len(lens) else 0,
-                                         partition_size=part)
-            if self.time_decode:
-                e1.record()
-                self.decode_events.append((i, e0, e1))
+                    self._l2_clean = torch.ones(256 << 20, dtype=torch.uint8, device=self.device)
+                for _ in range(self.time_reps):
+                    self._l2_flush.fill_(1)
+                    self._l2_clean.amax()
+                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    e0.record()
+                    out = call()
+                    e1.record()
+                    self.decode_events.append((i, e0, e1))
+            else:
+                out = call()
             if self.keep_outputs:
                 self.outputs[i] = out
         else:

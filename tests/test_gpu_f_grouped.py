@@ -1,0 +1,183 @@
+"""paged_attention_decode_grouped against the oracle and against paged_attention_decode.
+
+The grouped entry point reads blocks held by several sequences once per
+subgroup of them; the oracle decodes every sequence on its own, so agreement
+shows the sharing changes nothing but the traffic. Batches are built with
+explicit sharing: the members of a group hold the same physical blocks for a
+leading run, then blocks of their own, in a shuffled batch order. The cases
+cover groups larger than one subgroup (with a leftover member of one), a
+member whose partial last block another member holds in full (the shared
+prefix stops at full blocks), whole-sequence duplicates, sequences that share
+only their first block, sequences shorter than a block, empty sequences,
+shared prefixes that end inside a partition, grouped-query heads, and
+batches the entry point hands to paged_attention_decode (unsplit, a query
+group too wide for two members, a head size the tensor cores do not take,
+more sequences than the plan takes).
+"""
+
+import math
+
+import numpy as np
+import pytest
+
+from oracle import attention
+from oracle.numerics import to_f64
+from parity import ATOL, check_close, from_bits, to_bits
+import workloads
+
+pytestmark = pytest.mark.gpu
+
+
+def shared_batch(seed, groups, Hq, Hkv, D, bs, dtype, extra_blocks=5):
+    """groups: list of (shared_blocks, member lengths). Each member's first
+    min(shared_blocks, its own blocks) blocks are the group's; the rest are its own.
+    Returns (q, k, v bits, tables int32 [S, MB], lens int32 [S])."""
+    rng = np.random.default_rng(seed)
+    members = [(gi, L) for gi, (_, lens) in enumerate(groups) for L in lens]
+    need = [-(-L // bs) for _, L in members]
+    n_shared = [sb for sb, _ in groups]
+    nb = sum(n_shared) + sum(max(0, n - n_shared[gi]) for (gi, _), n in zip(members, need))
+    nb += extra_blocks
+    perm = rng.permutation(nb).astype(np.int32)
+    pos = 0
+    shared_ids = []
+    for sb in n_shared:
+        shared_ids.append(perm[pos:pos + sb])
+        pos += sb
+    order = rng.permutation(len(members))
+    S = len(members)
+    mb = max(1, max(need))
+    tables = np.full((S, mb), -1, np.int32)
+    lens = np.zeros(S, np.int32)
+    for row, mi in enumerate(order):
+        gi, L = members[mi]
+        n = need[mi]
+        k = min(n, n_shared[gi])
+        tables[row, :k] = shared_ids[gi][:k]
+        tables[row, k:n] = perm[pos:pos + n - k]
+        pos += n - k
+        lens[row] = L
+    q = workloads.normal_bits([seed, 11], (S, Hq, D), dtype)
+    k = workloads.normal_bits([seed, 12], (nb, Hkv, bs, D), dtype)
+    v = workloads.normal_bits([seed, 13], (nb, Hkv, bs, D), dtype)
+    return q, k, v, tables, lens
+
+
+def run(q, k, v, tables, lens, dtype, scale, partition, grouped, workspace=None):
+    import torch
+    import paged_kv_cache_319_b200 as kvp
+
+    out = kvp.paged_attention_decode(
+        from_bits(q, dtype), from_bits(k, dtype), from_bits(v, dtype),
+        torch.from_numpy(tables).cuda(), torch.from_numpy(lens).cuda(), scale,
+        max_context_len=int(max(lens.max(), 1)), partition_size=partition, grouped=grouped,
+        workspace=workspace)
+    kvp.check_device_error()
+    return to_bits(out)
+
+
+def oracle(q, k, v, tables, lens, dtype, scale, bs):
+    return attention.paged_decode(to_f64(q, dtype), k, v, tables, lens, scale, bs, dtype=dtype)
+
+
+# One query head per KV head: subgroups of up to 8.
+GROUPS_MHA = [
+    (31, [600, 700, 511, 767, 520, 530, 540, 550]),  # one subgroup of 8, prefix 31 blocks
+    (40, [700] * 9),          # identical lengths: a subgroup of 8 and a leftover decoded alone
+    (4, [50, 100, 64]),       # the 50-token member holds block 3 partly: prefix 3 blocks
+    (2, [16, 16]),            # one full block each, nothing of their own
+    (3, [40, 40]),            # duplicates whose last block is partial: prefix 2 blocks
+    (1, [300, 900]),          # only the first block in common
+    (0, [0]), (0, [5]), (0, [1500]),
+    (20, [272] * 17),         # 17 members: 8 + 8 + a leftover
+]
+
+CASES = [
+    # (name, Hq, Hkv, bs, dtype, partition, groups)
+    ("mha_f16_bs16_p512", 8, 8, 16, "f16", 512, GROUPS_MHA),
+    ("mha_bf16_bs32_p128", 4, 4, 32, "bf16", 128, GROUPS_MHA),
+    ("mha_f16_bs16_p256", 2, 2, 16, "f16", 256, GROUPS_MHA),
+    ("gqa4_bf16_bs16_p512", 16, 4, 16, "bf16", 512,
+     [(31, [600, 700, 511, 767, 520]), (8, [128, 300, 129]), (0, [0]), (0, [7]), (0, [2000])]),
+    ("gqa2_f16_bs32_p256", 8, 4, 32, "f16", 256,
+     [(12, [400, 390, 500, 385, 1000, 386, 387, 388, 389]), (1, [33, 64]), (0, [1])]),
+    ("gqa5_f16_bs16_p128", 10, 2, 16, "f16", 128,
+     [(9, [150, 160, 170, 180]), (2, [20, 40]), (0, [300])]),
+    ("gqa8_bf16_bs16_p512", 16, 2, 16, "bf16", 512,
+     [(20, [400, 500, 600]), (30, [480, 480]), (0, [64])]),
+    # handed to paged_attention_decode: a 16-wide query group, unsplit, 64-dim heads
+    ("gqa16_fallback", 16, 1, 16, "bf16", 512, [(10, [200, 300]), (0, [50])]),
+    ("unsplit_fallback", 4, 4, 16, "f16", 0, [(5, [100, 120]), (0, [30])]),
+]
+
+
+@pytest.mark.parametrize("name,Hq,Hkv,bs,dtype,partition,groups", CASES, ids=[c[0] for c in CASES])
+def test_grouped_matches_oracle(name, Hq, Hkv, bs, dtype, partition, groups):
+    seed = sum(map(ord, name))
+    q, k, v, t, l = shared_batch(seed, groups, Hq, Hkv, 128, bs, dtype)
+    scale = 1 / math.sqrt(128)
+    got = run(q, k, v, t, l, dtype, scale, partition, grouped=True)
+    ref = oracle(q, k, v, t, l, dtype, scale, bs)
+    check_close(got, ref, dtype, allow_ulp=(dtype == "bf16"))
+
+
+def test_head_dim_64_is_handed_on():
+    q, k, v, t, l = shared_batch(5, [(6, [100, 130, 140]), (0, [20])], 4, 4, 64, 16, "f16")
+    got = run(q, k, v, t, l, "f16", 0.125, 512, grouped=True)
+    check_close(got, oracle(q, k, v, t, l, "f16", 0.125, 16), "f16")
+
+
+def test_grouped_agrees_with_the_ungrouped_entry():
+    q, k, v, t, l = shared_batch(21, GROUPS_MHA, 8, 8, 128, 16, "f16")
+    a = to_f64(run(q, k, v, t, l, "f16", 0.088, 512, grouped=True), "f16")
+    b = to_f64(run(q, k, v, t, l, "f16", 0.088, 512, grouped=False), "f16")
+    assert np.abs(a - b).max() <= ATOL
+
+
+def test_reused_workspace_two_batches_in_a_row():
+    """The plan and partial slots left in the workspace by one call must not leak into the next."""
+    import torch
+    import paged_kv_cache_319_b200 as kvp
+
+    ws = torch.empty(kvp.decode_grouped_workspace_bytes(64, 8, 128, 2048, 512), dtype=torch.uint8,
+                     device="cuda")
+    ws.fill_(0xFF)  # NaN bit patterns everywhere
+    for seed, groups in ((1, GROUPS_MHA), (2, [(2, [40, 2000, 700]), (0, [900]), (9, [150] * 5)])):
+        q, k, v, t, l = shared_batch(seed, groups, 8, 8, 128, 16, "f16")
+        assert l.max() <= 2048 and len(l) <= 64
+        got = run(q, k, v, t, l, "f16", 0.09, 512, grouped=True, workspace=ws)
+        check_close(got, oracle(q, k, v, t, l, "f16", 0.09, 16), "f16")
+
+
+@pytest.mark.parametrize("S", [4096, 4100])
+def test_batch_size_limit_of_the_plan(S):
+    """4096 sequences are grouped (the plan's limit); 4100 go through paged_attention_decode."""
+    rng = np.random.default_rng(S)
+    groups, n = [], 0
+    while n < S:
+        m = int(min(S - n, rng.integers(1, 12)))
+        groups.append((int(rng.integers(1, 4)), rng.integers(1, 60, size=m).tolist()))
+        n += m
+    q, k, v, t, l = shared_batch(S, groups, 1, 1, 128, 16, "f16")
+    got = run(q, k, v, t, l, "f16", 0.09, 128, grouped=True)
+    check_close(got, oracle(q, k, v, t, l, "f16", 0.09, 16), "f16")
+
+
+@pytest.mark.parametrize("name,kw", [("sharing_A", {}), ("sharing_B", {}), ("beam", {"steps": 16})])
+def test_fork_workloads_grouped_every_output(name, kw):
+    """The sampling and beam workloads (blocks shared through fork and copy-on-write),
+    decoded through the grouped entry point at every attend op."""
+    from oracle.replay import OracleReplay
+    from paged_kv_cache_319_b200.replay import DeviceReplay
+    import paged_kv_cache_319_b200 as kvp
+
+    wl = workloads.by_name(name, **kw)
+    dev = DeviceReplay(wl, "cuda", grouped=True)
+    dev.run()
+    kvp.check_device_error()
+    ora = OracleReplay(wl)
+    refs = {}
+    ora.run(attend=lambda i, seqs, tables, lens: refs.__setitem__(i, ora.decode(i, tables, lens.tolist())))
+    assert refs
+    for i, ref in refs.items():
+        check_close(to_bits(dev.outputs[i]), ref, wl.geometry.dtype)
