@@ -281,30 +281,72 @@ KVP_API size_t kvp_decode_grouped_workspace_bytes(int32_t num_seqs, int32_t num_
  * beam search]. The pages' decode kernel still reads a shared block once per
  * sequence that attends to it; this entry point, which the pages do not
  * describe, reads it once per subgroup.
- * How: a one-CTA kernel groups the sequences by their first block id (only
- * sequences whose context holds a full block), cuts each group, in sequence
- * order, into subgroups of up to M members (M = 8 for one query head per KV
- * head, else 16 / G) and finds each subgroup's shared prefix c: the leading
- * block-table entries equal across its members, capped at every member's
- * full blocks. The tensor-core kernel then attends, per KV head, with all the
- * members' queries of a subgroup as the columns of one contraction over the c
- * shared blocks, and per sequence over its blocks from c on; both ranges are
- * split into partitions of partition_size tokens and a log-sum-exp merge
- * writes every output row.
+ * How: a grouping plan (the rule is kv_decode_group_plan's) names subgroups of
+ * up to M sequences (M = 8 for one query head per KV head, else 16 / G) and
+ * each subgroup's shared prefix of c full blocks. The tensor-core kernel
+ * attends, per KV head, with all the members' queries of a subgroup as the
+ * columns of one contraction over the c shared blocks; each sequence's blocks
+ * from c on go to the CUDA-core kernel (one query head per KV head) or to the
+ * tensor-core kernel (grouped-query heads). Both ranges are split into
+ * partitions of partition_size tokens and a log-sum-exp merge writes every
+ * output row.
+ * host_plan: NULL, and a one-CTA kernel builds the plan on the GPU; or the
+ * plan kv_decode_group_plan built from these same block tables and lengths
+ * (host memory, kvp_decode_group_plan_words(num_seqs) words). The kernels read
+ * the plan from device memory: device_plan, a copy of host_plan that the
+ * caller has placed there (for example uploaded together with its block
+ * tables; 4-byte aligned, read-only to the call), or, when device_plan is
+ * NULL, a copy the call makes into the workspace by cudaMemcpyAsync on
+ * `stream` (pageable host memory may be reused once the call returns;
+ * page-locked memory, whose copy runs in stream order, must stay unchanged
+ * until the stream has reached this call). device_plan without host_plan is
+ * rejected. A host
+ * plan also lets the call give the tensor-core kernel only its share of the
+ * SMs and run the CUDA-core kernel beside it. A plan from other tables gives
+ * wrong results; one whose header does not fit the batch is rejected.
  * Needs head_dim 128, block_size 16 or 32, a group G = num_q_heads /
  * num_kv_heads with 16 / G >= 2 (G <= 8), partition_size > 0 and a multiple
  * of 128, and num_seqs <= 4096; other batches (and max_context_len == 0) are
- * decoded by paged_attention_decode with the same workspace, so the call is
- * valid for every batch paged_attention_decode accepts.
+ * decoded by paged_attention_decode with the same workspace (host_plan
+ * ignored), so the call is valid for every batch paged_attention_decode
+ * accepts.
  * workspace: device, >= kvp_decode_grouped_workspace_bytes(...) bytes,
- * 256-byte aligned, contents ignored. Errors: those of paged_attention_decode. */
+ * 256-byte aligned, contents ignored. Errors: those of paged_attention_decode,
+ * and KVP_ERR_INVALID for a host plan that does not fit. */
 KVP_API int paged_attention_decode_grouped(const void* q, const void* k_cache, const void* v_cache,
                            const int32_t* block_tables, const int32_t* context_lens,
                            int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
                            int32_t head_dim, int32_t block_size, int32_t num_blocks,
                            int32_t max_blocks_per_seq, int32_t max_context_len, float scale,
-                           int32_t partition_size, void* workspace, size_t workspace_bytes,
+                           int32_t partition_size, const int32_t* host_plan,
+                           const int32_t* device_plan, void* workspace, size_t workspace_bytes,
                            void* out, int32_t dtype, kvp_stream_t stream);
+
+/* Words of the grouping plan of a batch of num_seqs sequences (0 if
+ * num_seqs <= 0): 8 + num_seqs + (num_seqs / 2 + 1) * 20. */
+KVP_API size_t kvp_decode_group_plan_words(int32_t num_seqs);
+
+/* Builds on the host the grouping plan of paged_attention_decode_grouped
+ * from host copies of the batch's block tables ([num_seqs][max_blocks_per_seq])
+ * and context lengths (clamped to [0, max_context_len]). Rule: a sequence
+ * whose context holds a full block and whose first table entry is a valid id
+ * is keyed by that id; sorted by (key, sequence index), each run of equal keys
+ * is cut in order into subgroups of up to M members (M as above, from
+ * num_q_heads / num_kv_heads; a subgroup of one is dropped); a subgroup's
+ * shared prefix c is the number of leading entries equal across its members,
+ * capped at every member's full blocks. Layout of `plan` (int32 words):
+ * [0] subgroups, [1] most partitions of a shared prefix, [2] most partitions
+ * of a sequence's own range (from block c on), [3] sum of c over subgroups,
+ * [4] blocks of all own ranges, [5..8) zero; [8, 8 + num_seqs) c of each
+ * sequence's subgroup (0 if none); then per subgroup 20 words {c, members,
+ * 0, 0, member indices [16]}. The GPU plan kernel builds the same words.
+ * num_seqs in [1, 4096]; plan_words >= kvp_decode_group_plan_words(num_seqs).
+ * Errors: KVP_ERR_INVALID. */
+KVP_API int kv_decode_group_plan(const int32_t* block_tables, const int32_t* context_lens,
+                         int32_t num_seqs, int32_t max_blocks_per_seq, int32_t max_context_len,
+                         int32_t block_size, int32_t partition_size, int32_t num_q_heads,
+                         int32_t num_kv_heads, int32_t num_blocks, int32_t* plan,
+                         size_t plan_words);
 
 /* Largest split-context scratch, in bytes, that paged_attention_decode_noalloc
  * can serve from its built-in area (40 MiB). */

@@ -21,7 +21,7 @@ from ._lib import (KVP_BF16, KVP_F16, KvpError, P_i32, P_i64, PoolStats, check, 
 
 __all__ = [
     "BlockPool", "KvpError", "reshape_and_cache", "copy_blocks", "paged_attention_decode",
-    "decode_workspace_bytes", "decode_grouped_workspace_bytes", "check_device_error",
+    "decode_workspace_bytes", "decode_grouped_workspace_bytes", "group_plan", "check_device_error",
     "kv_bytes_per_token", "version",
     "KVP_F16", "KVP_BF16",
 ]
@@ -238,16 +238,37 @@ def decode_grouped_workspace_bytes(num_seqs: int, num_q_heads: int, head_dim: in
                                                         max_context_len, partition_size))
 
 
+def group_plan(block_tables: np.ndarray, context_lens: np.ndarray, *, block_size: int,
+               partition_size: int, num_q_heads: int, num_kv_heads: int, num_blocks: int,
+               max_context_len: int | None = None) -> np.ndarray:
+    """The grouping plan of ``paged_attention_decode_grouped``, built on the host
+    (``kv_decode_group_plan``) from host block tables [S, MB] and lengths [S]."""
+    t = np.ascontiguousarray(block_tables, dtype=np.int32)
+    l = np.ascontiguousarray(context_lens, dtype=np.int32)
+    S, MB = t.shape
+    mcl = MB * block_size if max_context_len is None else int(max_context_len)
+    n = int(lib().kvp_decode_group_plan_words(S))
+    plan = np.zeros(max(n, 1), np.int32)
+    check(lib().kv_decode_group_plan(_i32p(t), _i32p(l), S, max(MB, 1), mcl, block_size,
+                                     partition_size, num_q_heads, num_kv_heads, num_blocks,
+                                     _i32p(plan), n))
+    return plan
+
+
 def paged_attention_decode(q, k_cache, v_cache, block_tables, context_lens, scale: float,
                            out=None, *, max_context_len: int | None = None,
-                           partition_size: int = 0, workspace=None, grouped: bool = False):
+                           partition_size: int = 0, workspace=None, grouped: bool = False,
+                           host_plan: np.ndarray | None = None, device_plan=None):
     """Decode attention over the paged cache; returns ``out [S, Hq, D]`` (dtype of q).
 
     ``max_context_len`` bounds every ``context_lens`` entry (default: the
     block-table capacity); ``partition_size > 0`` selects the split-context
     kernel pair. ``grouped`` calls ``paged_attention_decode_grouped``, which
-    reads blocks shared by several sequences once per subgroup of them. A
-    workspace is allocated with torch when needed and none is given.
+    reads blocks shared by several sequences once per subgroup of them, with
+    ``host_plan`` (from :func:`group_plan` on the same tables; ``device_plan``,
+    an int32 CUDA tensor holding a copy of it, saves the call its upload) or a
+    plan built on the GPU. A workspace is allocated with torch when needed and
+    none is given.
     """
     torch = _torch()
     dev = _cuda(q, k_cache, v_cache, block_tables, context_lens)
@@ -275,10 +296,22 @@ def paged_attention_decode(q, k_cache, v_cache, block_tables, context_lens, scal
             workspace = torch.empty(need, dtype=torch.uint8, device=dev)
         _cuda(workspace)
         ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()
-    fn = lib().paged_attention_decode_grouped if grouped else lib().paged_attention_decode
-    check(fn(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), block_tables.data_ptr(),
-             context_lens.data_ptr(), S, Hq, Hkv, D, bs, NB, max(MB, 1), mcl, float(scale),
-             int(partition_size), ws_ptr, ws_bytes, out.data_ptr(), _code(q), _stream(dev)))
+    args = [q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), block_tables.data_ptr(),
+            context_lens.data_ptr(), S, Hq, Hkv, D, bs, NB, max(MB, 1), mcl, float(scale),
+            int(partition_size), ws_ptr, ws_bytes, out.data_ptr(), _code(q), _stream(dev)]
+    if grouped:
+        if host_plan is not None:
+            host_plan = np.ascontiguousarray(host_plan, dtype=np.int32)
+        dp = None
+        if device_plan is not None:
+            _cuda(device_plan)
+            if device_plan.dtype != torch.int32:
+                raise TypeError("device_plan must be int32")
+            dp = device_plan.data_ptr()
+        args[15:15] = [host_plan.ctypes.data if host_plan is not None else None, dp]
+        check(lib().paged_attention_decode_grouped(*args))
+    else:
+        check(lib().paged_attention_decode(*args))
     return out
 
 

@@ -74,7 +74,10 @@ SIGNATURES = {
                                          i32, f32, i32, vp, sz, vp, i32, vp]),
     "kvp_decode_grouped_workspace_bytes": (sz, [i32, i32, i32, i32, i32]),
     "paged_attention_decode_grouped": (C.c_int, [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,
-                                                 i32, i32, f32, i32, vp, sz, vp, i32, vp]),
+                                                 i32, i32, f32, i32, vp, vp, vp, sz, vp, i32, vp]),
+    "kvp_decode_group_plan_words": (sz, [i32]),
+    "kv_decode_group_plan": (C.c_int, [P_i32, P_i32, i32, i32, i32, i32, i32, i32, i32, i32, P_i32,
+                                       sz]),
     "paged_attention_decode_noalloc": (C.c_int, [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,
                                                  i32, i32, f32, i32, vp, i32, vp]),
     "kvp_check_device_error": (C.c_int, [vp]),

@@ -1,69 +1,38 @@
-// Grouping of the sequences of a decode batch that hold the same leading
-// cache blocks (the samples of one prompt, the beams of one request), for the
-// grouped decode.
-//
-// With paged memory, sequences forked from one parent share the physical
-// blocks of their common prefix, each block stored once with a reference
-// count ["Your GPU was mostly empty", section "Paging's second gift:
-// copy-on-write"; "vLLM and PagedAttention", section on parallel sampling and
-// beam search]. A decode kernel that works sequence by sequence still reads
-// such a block once per sequence. The grouped decode reads it once per
-// subgroup of up to `mmax` sequences, with their queries side by side as the
-// columns of one tensor-core contraction; this kernel decides the subgroups.
-//
-// Rule. A sequence whose context holds at least one full block is keyed by
-// its first block id; the batch is sorted by (key, sequence index) and every
-// run of equal keys is cut, in that order, into subgroups of up to mmax
-// members (a subgroup of one is dropped: its member is decoded alone). The
-// shared prefix of a subgroup is its first c blocks, c = the number of leading
-// block-table entries that are equal across all members, capped at every
-// member's number of full blocks; every member therefore attends to every one
-// of the c * block_size shared tokens, and from block c on to its own.
-//
-// Plan (int32 words, in the caller's workspace):
-//   [0]             n_sub: number of subgroups
-//   [1]             most shared partitions of any subgroup
-//   [2, 8)          unused
-//   [8, 8 + S)      per sequence: c of its subgroup (first block of its own
-//                   range), 0 for a sequence in no subgroup
-//   [8 + S, ...)    per subgroup, kSubWords words:
-//                   {c, n_members, 0, 0, member sequence indices [kMaxMembers]}
+// The grouping plan of the grouped decode, built on the GPU: the rule and
+// the plan's layout are in group_layout.h (the host planner,
+// host/group_plan.cpp, builds the same plan word for word). One CTA sorts
+// the batch's (first block id, sequence) keys (bitonic sort in shared memory),
+// finds the runs of equal keys and their subgroups with prefix scans, and
+// compares the members' block tables, one warp per subgroup.
 #pragma once
 
 #include "common.cuh"
+#include "group_layout.h"
 
 namespace kvp {
-namespace dev {
-
 namespace grp {
 
-constexpr int kMaxSeqs = 4096;     // larger batches are decoded without grouping
-constexpr int kMaxMembers = 16;    // columns of the tensor-core contraction
-constexpr int kHdrWords = 8;
-constexpr int kSubWords = 4 + kMaxMembers;
 constexpr int kMaxThreads = 1024;
 
-__host__ __device__ constexpr int64_t sub_offset(int64_t S) { return kHdrWords + S; }
-__host__ __device__ constexpr int64_t plan_words(int64_t S) {
-  return kHdrWords + S + (S / 2 + 1) * kSubWords;
-}
 // Sort length: a power of two >= S (and >= 2).
-__host__ __device__ constexpr int sort_len(int S) {
+KVP_HD constexpr int sort_len(int S) {
   int n = 2;
   while (n < S) n <<= 1;
   return n;
 }
 // at least 8 warps: one warp per subgroup compares block tables
-__host__ __device__ constexpr int plan_threads(int N) {
+KVP_HD constexpr int plan_threads(int N) {
   return N < 256 ? 256 : (N > kMaxThreads ? kMaxThreads : N);
 }
 // Shared memory of the plan kernel: sort keys, three scan arrays, per-sequence
 // context and subgroup, per-subgroup head position, size and prefix.
-__host__ __device__ constexpr size_t plan_smem_bytes(int S) {
+KVP_HD constexpr size_t plan_smem_bytes(int S) {
   return size_t(sort_len(S)) * (8 + 3 * 4) + size_t(S) * 2 * 4 + size_t(S / 2 + 1) * 3 * 4;
 }
 
 }  // namespace grp
+
+namespace dev {
 
 // One CTA. tables: [S][MB]; lens: [S] (clamped to [0, max_ctx] as the decode
 // kernels do); plan: grp::plan_words(S) words.
@@ -83,13 +52,18 @@ __global__ void __launch_bounds__(grp::kMaxThreads, 1) group_plan_kernel(
   int32_t* sub_head = sub_of + S;
   int32_t* sub_nm = sub_head + (S / 2 + 1);
   int32_t* sub_c = sub_nm + (S / 2 + 1);
-  __shared__ int32_t psh_sh;
+  __shared__ int32_t psh_sh, pown_sh, shared_blk_sh, own_blk_sh;
 
   // the decode kernel launched after this one prepares while this one runs
   pdl_trigger();
   const int tid = threadIdx.x, nt = blockDim.x;
   constexpr uint32_t kNoKey = 0xFFFFFFFFu;
-  if (tid == 0) psh_sh = 0;
+  if (tid == 0) {
+    psh_sh = 0;
+    pown_sh = 0;
+    shared_blk_sh = 0;
+    own_blk_sh = 0;
+  }
   for (int i = tid; i < N; i += nt) {
     uint64_t k = ~0ull;
     if (i < S) {
@@ -242,15 +216,28 @@ __global__ void __launch_bounds__(grp::kMaxThreads, 1) group_plan_kernel(
       e[2] = 0;
       e[3] = 0;
       atomicMax(&psh_sh, (c * bs + part_tokens - 1) / part_tokens);
+      atomicAdd(&shared_blk_sh, c);
     }
   }
   __syncthreads();
-  for (int s = tid; s < S; s += nt) plan[grp::kHdrWords + s] = sub_of[s] >= 0 ? sub_c[sub_of[s]] : 0;
+  for (int s = tid; s < S; s += nt) {
+    const int32_t c = sub_of[s] >= 0 ? sub_c[sub_of[s]] : 0;
+    plan[grp::kHdrWords + s] = c;
+    const int32_t own = ctxs[s] - c * bs;  // tokens of the sequence's own range
+    if (own > 0) {
+      atomicMax(&pown_sh, (own + part_tokens - 1) / part_tokens);
+      atomicAdd(&own_blk_sh, (own + bs - 1) / bs);
+    }
+  }
+  __syncthreads();
   if (tid == 0) {
-    plan[0] = n_sub;
-    plan[1] = psh_sh;
+    plan[grp::kNumSub] = n_sub;
+    plan[grp::kSharedParts] = psh_sh;
+    plan[grp::kOwnParts] = pown_sh;
+    plan[grp::kSharedBlocks] = shared_blk_sh;
+    plan[grp::kOwnBlocks] = own_blk_sh;
 #pragma unroll
-    for (int i = 2; i < grp::kHdrWords; ++i) plan[i] = 0;
+    for (int i = 5; i < grp::kHdrWords; ++i) plan[i] = 0;
   }
 }
 

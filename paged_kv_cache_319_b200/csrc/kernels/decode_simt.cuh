@@ -92,7 +92,12 @@ struct SimtCfg {
   static_assert(NST >= 1 && NST <= 32, "stages");
 };
 
-template <typename T, int D, int BS, int NW, int NST>
+// PH (per-head warps): grid (partition, ceil(Hq / NW), sequence); warp w takes
+// query head blockIdx.y * NW + w over the whole partition and writes its own
+// partial, with no merge across warps. For short ranges (a few blocks per
+// (sequence, head)), where splitting a range over the warps would leave each
+// warp one or two blocks, this keeps every warp's pipeline busy.
+template <typename T, int D, int BS, int NW, int NST, bool PH = false>
 __global__ void __launch_bounds__(NW * 32) decode_simt_kernel(
     const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
     const DecodeArgs a) {
@@ -108,7 +113,7 @@ __global__ void __launch_bounds__(NW * 32) decode_simt_kernel(
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int p = blockIdx.x;
-  const int h = blockIdx.y;
+  const int h = PH ? int(blockIdx.y) * NW + warp : int(blockIdx.y);
   const int s = blockIdx.z;
 
   // The split-context reduce may be scheduled as soon as every CTA of this grid
@@ -120,14 +125,14 @@ __global__ void __launch_bounds__(NW * 32) decode_simt_kernel(
   // wait for the plan). One CTA waits for that kernel, so this grid completes
   // after it and the reduce's wait covers both.
   const bool grouped = a.plan != nullptr;
-  if (grouped && p == 0 && h == 0 && s == 0) pdl_wait();
-  const int32_t ctx = load_ctx(a, s, p == 0 && h == 0 && threadIdx.x == 0);
+  if (grouped && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0) pdl_wait();
+  if (PH && h >= a.num_q_heads) return;  // a warp past the last head (no CTA-wide sync follows)
+  // the plan word and the context length are loaded together
+  int32_t b_first = grouped ? ld_relaxed_gpu(a.plan + kPlanSeqWord + s) : 0;
+  const int32_t ctx = load_ctx(a, s, p == 0 && blockIdx.y == 0 && threadIdx.x == 0);
   const int32_t nblk = (ctx + BS - 1) / BS;
-  int32_t b_first = 0, slot = p;
-  if (grouped) {
-    b_first = ld_relaxed_gpu(a.plan + kPlanSeqWord + s);
-    slot = (b_first + a.part_blocks - 1) / a.part_blocks + p;  // after the shared slots
-  }
+  int32_t slot = p;
+  if (grouped) slot = (b_first + a.part_blocks - 1) / a.part_blocks + p;  // after the shared slots
   const int32_t b0 = b_first + p * a.part_blocks;
   // empty partition (p == 0 always writes its row, except in the grouped decode)
   if ((p > 0 || grouped) && b0 >= nblk) return;
@@ -137,9 +142,11 @@ __global__ void __launch_bounds__(NW * 32) decode_simt_kernel(
   const int32_t g = h / (a.num_q_heads / a.num_kv_heads);
   const int32_t* table = a.block_tables + int64_t(s) * a.max_blocks_per_seq;
 
-  // Blocks of this warp: b0 + warp + NW * i, i < nw.
+  // Blocks of this warp: b0 + warp + NW * i, i < nw (PH: b0 + i, i < span).
   const int32_t span = b1 - b0;
-  const int32_t nw = span > warp ? (span - warp + NW - 1) / NW : 0;
+  constexpr int kStride = PH ? 1 : NW;
+  const int32_t wfirst = PH ? 0 : warp;
+  const int32_t nw = span > wfirst ? (span - wfirst + kStride - 1) / kStride : 0;
 
   uint64_t* my_bars = bars + warp * NST;
   uint8_t* my_tiles = tiles + size_t(warp) * NST * 2 * C::kTileBytes;
@@ -161,7 +168,7 @@ __global__ void __launch_bounds__(NW * 32) decode_simt_kernel(
   int32_t my_id = -1;
   auto load_ids = [&](int32_t base) {
     const int32_t idx = base + lane;
-    my_id = idx < nw ? __ldg(table + b0 + warp + NW * idx) : -1;
+    my_id = idx < nw ? __ldg(table + b0 + wfirst + kStride * idx) : -1;
   };
   load_ids(0);
 
@@ -171,7 +178,7 @@ __global__ void __launch_bounds__(NW * 32) decode_simt_kernel(
     uint8_t* vt = kt + C::kTileBytes;
     int32_t row;
     if (id < 0 || id >= a.num_blocks) {
-      record_error(KVP_DEVERR_BLOCK_ID, (uint64_t(s) << 32) | uint32_t(b0 + warp + NW * i));
+      record_error(KVP_DEVERR_BLOCK_ID, (uint64_t(s) << 32) | uint32_t(b0 + wfirst + kStride * i));
       row = rows_total;  // out of the tensor: the load fills zeros
     } else {
       row = (id * a.num_kv_heads + g) * BS;
@@ -233,7 +240,7 @@ __global__ void __launch_bounds__(NW * 32) decode_simt_kernel(
     }
     const uint8_t* kt = my_tiles + size_t(stage) * 2 * C::kTileBytes;
     const uint8_t* vt = kt + C::kTileBytes;
-    const int32_t tok0 = (b0 + warp + NW * i) * BS;
+    const int32_t tok0 = (b0 + wfirst + kStride * i) * BS;
     const int32_t nvalid = min(BS, ctx - tok0);
 
     // ---- scores: row r = pass * 16 + (lane & 15), half `part` of its chunks
@@ -341,42 +348,64 @@ __global__ void __launch_bounds__(NW * 32) decode_simt_kernel(
     m_run = -INFINITY;
   }
 
-  // ---- merge the warps
+  if constexpr (PH) {
+    // ---- this warp's partial (no merge across warps)
 #pragma unroll
-  for (int o = 8; o >= 1; o >>= 1) l_lane += __shfl_xor_sync(0xffffffffu, l_lane, o);
-  if (lane == 0) {
-    mg_m[warp] = m_run;
-    mg_l[warp] = l_lane;
-  }
+    for (int o = 8; o >= 1; o >>= 1) l_lane += __shfl_xor_sync(0xffffffffu, l_lane, o);
+    const float L = __shfl_sync(0xffffffffu, l_lane, 0);
+    const int64_t row_sh = int64_t(s) * a.num_q_heads + h;
 #pragma unroll
-  for (int e = 0; e < C::kDimsPerLane; ++e) mg_acc[warp * D + lane * C::kDimsPerLane + e] = acc[e];
-  const int any_abort = __syncthreads_or(aborted ? 1 : 0);
-
-  const int64_t row_sh = int64_t(s) * a.num_q_heads + h;
-  float M = -INFINITY;
-#pragma unroll
-  for (int w = 0; w < NW; ++w) M = fmaxf(M, mg_m[w]);
-  float wgt[NW];
-  float L = 0.f;
-#pragma unroll
-  for (int w = 0; w < NW; ++w) {
-    wgt[w] = (mg_m[w] == -INFINITY || M == -INFINITY) ? 0.f : exp2f(mg_m[w] - M);
-    L += mg_l[w] * wgt[w];
-  }
-  for (int t = threadIdx.x; t < D; t += NW * 32) {
-    float o = 0.f;
-#pragma unroll
-    for (int w = 0; w < NW; ++w) o = fmaf(mg_acc[w * D + t], wgt[w], o);
-    if (!to_ws) {
-      const float y = (L > 0.f && !any_abort) ? o / L : 0.f;
-      static_cast<uint16_t*>(a.out)[row_sh * D + t] = Elem<T>::from_float(y);
-    } else {
-      a.ws_acc[(row_sh * a.ws_slots + slot) * D + t] = o;
+    for (int e = 0; e < C::kDimsPerLane; ++e) {
+      const int t = lane * C::kDimsPerLane + e;
+      if (!to_ws) {
+        const float y = (L > 0.f && !aborted) ? acc[e] / L : 0.f;
+        static_cast<uint16_t*>(a.out)[row_sh * D + t] = Elem<T>::from_float(y);
+      } else {
+        a.ws_acc[(row_sh * a.ws_slots + slot) * D + t] = acc[e];
+      }
     }
-  }
-  if (to_ws && threadIdx.x == 0) {
-    a.ws_ml[(row_sh * a.ws_slots + slot) * 2 + 0] = any_abort ? -INFINITY : M;
-    a.ws_ml[(row_sh * a.ws_slots + slot) * 2 + 1] = any_abort ? 0.f : L;
+    if (to_ws && lane == 0) {
+      a.ws_ml[(row_sh * a.ws_slots + slot) * 2 + 0] = aborted ? -INFINITY : m_run;
+      a.ws_ml[(row_sh * a.ws_slots + slot) * 2 + 1] = aborted ? 0.f : L;
+    }
+  } else {
+    // ---- merge the warps
+#pragma unroll
+    for (int o = 8; o >= 1; o >>= 1) l_lane += __shfl_xor_sync(0xffffffffu, l_lane, o);
+    if (lane == 0) {
+      mg_m[warp] = m_run;
+      mg_l[warp] = l_lane;
+    }
+#pragma unroll
+    for (int e = 0; e < C::kDimsPerLane; ++e) mg_acc[warp * D + lane * C::kDimsPerLane + e] = acc[e];
+    const int any_abort = __syncthreads_or(aborted ? 1 : 0);
+
+    const int64_t row_sh = int64_t(s) * a.num_q_heads + h;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) M = fmaxf(M, mg_m[w]);
+    float wgt[NW];
+    float L = 0.f;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) {
+      wgt[w] = (mg_m[w] == -INFINITY || M == -INFINITY) ? 0.f : exp2f(mg_m[w] - M);
+      L += mg_l[w] * wgt[w];
+    }
+    for (int t = threadIdx.x; t < D; t += NW * 32) {
+      float o = 0.f;
+#pragma unroll
+      for (int w = 0; w < NW; ++w) o = fmaf(mg_acc[w * D + t], wgt[w], o);
+      if (!to_ws) {
+        const float y = (L > 0.f && !any_abort) ? o / L : 0.f;
+        static_cast<uint16_t*>(a.out)[row_sh * D + t] = Elem<T>::from_float(y);
+      } else {
+        a.ws_acc[(row_sh * a.ws_slots + slot) * D + t] = o;
+      }
+    }
+    if (to_ws && threadIdx.x == 0) {
+      a.ws_ml[(row_sh * a.ws_slots + slot) * 2 + 0] = any_abort ? -INFINITY : M;
+      a.ws_ml[(row_sh * a.ws_slots + slot) * 2 + 1] = any_abort ? 0.f : L;
+    }
   }
 }
 

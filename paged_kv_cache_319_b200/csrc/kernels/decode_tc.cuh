@@ -16,10 +16,12 @@
 // Structure: a persistent CTA per SM walks its share of work units
 // (sequence, KV head, partition); a unit is cut into chunks of up to 512
 // tokens (4 M-tiles). Warp roles:
-//   warp 0  producer: 2-D TMA loads (128-byte swizzle) of Q (per unit) and of
+//   warp 0  producer: TMA loads (128-byte swizzle) of Q (per unit) and of
 //           K then V tiles (per chunk) into a 5-stage ring of 32 KiB stages;
-//           a stage is 128 tokens = 128 / block_size cache blocks, each block
-//           tile landing at its rows of the stage.
+//           a stage is 128 tokens = 128 / block_size cache blocks: a K block
+//           lands as two 2-D boxes at its rows of the stage's two 64-dim
+//           regions (the QK MMA's 128 token rows need one 8-row stride), a V
+//           block as one 3-D box [half][rows][64] that PV reads in place.
 //   warp 1  MMA issuer (one thread) and tensor-memory owner: per chunk, QK^T
 //           into a double-buffered S region, then PV into a double-buffered O
 //           region; tcgen05.commit releases ring stages and signals softmax.
@@ -404,8 +406,8 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
     // ranges, or the reduce) may start once every CTA is past this point, so
     // it may read the plan without a wait of its own.
     pdl_trigger();
-    const int32_t n_sub = ld_relaxed_gpu(a.plan);
-    gh.psh = ld_relaxed_gpu(a.plan + 1);
+    const int32_t n_sub = ld_relaxed_gpu(a.plan + grp::kNumSub);
+    gh.psh = ld_relaxed_gpu(a.plan + grp::kSharedParts);
     gh.shared_units = int64_t(n_sub) * gh.psh * a.num_kv_heads;
     num_units += gh.shared_units;
     const int32_t* g_cblk = a.plan + kPlanSeqWord;
@@ -440,24 +442,32 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
     uint32_t ctr = 0;   // ring tiles issued
     uint32_t ucnt = 0;  // units started
     bool ok = true;
-    // Lane j's TMA row of block j of a chunk (one chunk = 512 / BS <= 32 blocks).
-    auto chunk_row = [&](const tc::ChunkStream<GRP, BS>& cs) -> int32_t {
+    // Lane j's block of a chunk (one chunk = 512 / BS <= 32 blocks): its table
+    // entry is loaded a chunk ahead (chunk_id, not waited on) and turned into a
+    // TMA row, range-checked, when the chunk's tiles are issued (id_row).
+    auto lane_has_block = [&](const tc::ChunkStream<GRP, BS>& cs, int32_t& bidx) {
       const tc::Unit& w = cs.w;
-      const int32_t ntile = cs.tiles();
-      const int32_t blk0 = (w.tok_begin + cs.c * kChunkTok) / BS;
-      const int32_t nblk_seq = (w.ctx + BS - 1) / BS;
-      const int32_t bidx = blk0 + lane;
-      int32_t id = -1;
-      if (lane < ntile * kBlocksPerTile && bidx < nblk_seq) {
-        id = __ldg(a.block_tables + int64_t(w.s) * a.max_blocks_per_seq + bidx);
-        if (id < 0 || id >= a.num_blocks) {
-          record_error(KVP_DEVERR_BLOCK_ID, (uint64_t(w.s) << 32) | uint32_t(bidx));
-          id = -1;
-        }
-      }
-      return id < 0 ? rows_total : (id * a.num_kv_heads + w.g) * BS;
+      bidx = (w.tok_begin + cs.c * kChunkTok) / BS + lane;
+      return lane < cs.tiles() * kBlocksPerTile && bidx < (w.ctx + BS - 1) / BS;
     };
-    auto load_tiles = [&](const CUtensorMap* map, int32_t row, int32_t ntile) {
+    auto chunk_id = [&](const tc::ChunkStream<GRP, BS>& cs) -> int32_t {
+      int32_t bidx;
+      if (!lane_has_block(cs, bidx)) return -1;
+      return __ldg(a.block_tables + int64_t(cs.w.s) * a.max_blocks_per_seq + bidx);
+    };
+    auto id_row = [&](const tc::ChunkStream<GRP, BS>& cs, int32_t id) -> int32_t {
+      int32_t bidx;
+      if (!lane_has_block(cs, bidx)) return rows_total;  // past the sequence: zeros
+      if (id < 0 || id >= a.num_blocks) {
+        record_error(KVP_DEVERR_BLOCK_ID, (uint64_t(cs.w.s) << 32) | uint32_t(bidx));
+        return rows_total;
+      }
+      return (id * a.num_kv_heads + cs.w.g) * BS;
+    };
+    // Key tiles: two 2-D boxes per block (its rows of each 64-dim region of the
+    // stage). Value tiles: one 3-D box per block ([half][BS rows][64], 256 * BS
+    // bytes at block j's offset), which the PV descriptors read in place.
+    auto load_tiles = [&](const CUtensorMap* map, int32_t row, int32_t ntile, bool values) {
       for (int32_t t = 0; t < ntile && ok; ++t, ++ctr) {
         const uint32_t st = ctr % kStages;
         if (lane == 0) {
@@ -468,76 +478,100 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
         if (!ok) break;
         const int j = lane - t * kBlocksPerTile;  // block j of this tile
         if (j >= 0 && j < kBlocksPerTile) {
-          uint8_t* dst = ring + st * kStageBytes + j * BS * 128;
-          tma_load_2d(dst, map, &full[st], 0, row, pol_kv);
-          tma_load_2d(dst + kRegionBytes, map, &full[st], 64, row, pol_kv);
+          if (values) {
+            tma_load_3d(ring + st * kStageBytes + j * BS * 256, map, &full[st], 0, row, 0, pol_kv);
+          } else {
+            uint8_t* dst = ring + st * kStageBytes + j * BS * 128;
+            tma_load_2d(dst, map, &full[st], 0, row, pol_kv);
+            tma_load_2d(dst + kRegionBytes, map, &full[st], 64, row, pol_kv);
+          }
         }
         __syncwarp();
+      }
+    };
+    // Shared-prefix units (grouped decode): column j of Q is query head
+    // g * G + j % G of member j / G. The warp loads a unit's rows into
+    // registers one iteration ahead and stores them, when the unit starts, in
+    // the 128-byte-swizzled layout a TMA load would produce (16-byte chunk c of
+    // row j at (c ^ (j & 7)) * 16): before the unit's key tiles and so before
+    // the previous unit's value tiles, since the MMA needs this Q before it
+    // frees the ring stages those wait for.
+    constexpr int kQChunksPerLane = kN * 16 / 32;
+    auto is_gather = [&](const tc::ChunkStream<GRP, BS>& cs) {
+      return GRP && cs.valid && cs.first() && cs.w.sg >= 0;
+    };
+    auto gather_q = [&](const tc::ChunkStream<GRP, BS>& cs, uint4 (&v)[kQChunksPerLane]) {
+      const int32_t* e = tc::sub_entry(gh, cs.w.sg);
+      const int32_t ncol = tc::plan_at(gh, e + 1) * G;
+#pragma unroll
+      for (int i = 0; i < kQChunksPerLane; ++i) {
+        const int idx = lane + 32 * i;
+        const int j = idx >> 4, ch = idx & 15;
+        v[i] = make_uint4(0, 0, 0, 0);
+        if (j < ncol) {
+          const int32_t m = j / G;
+          const int64_t qrow =
+              int64_t(tc::plan_at(gh, e + 4 + m)) * a.num_q_heads + cs.w.g * G + (j - m * G);
+          v[i] = __ldg(reinterpret_cast<const uint4*>(static_cast<const T*>(a.q) + qrow * kD) + ch);
+        }
       }
     };
     tc::ChunkStream<GRP, BS> cur;
     cur.init(a, blockIdx.x, gridDim.x, num_units, ctx_sm, gh);
     int32_t pend_row = rows_total, pend_tiles = 0;
     bool have_pend = false;
-    int32_t row = cur.valid ? chunk_row(cur) : rows_total;
+    int32_t id = cur.valid ? chunk_id(cur) : -1;
+    uint4 qv[kQChunksPerLane];
+    if (is_gather(cur)) gather_q(cur, qv);
     while (cur.valid && ok) {
-      // the next chunk's block ids are loaded now and used one iteration later
+      // the next chunk's block ids (and a grouped unit's Q rows) are loaded now
+      // and used one iteration later
       tc::ChunkStream<GRP, BS> nxt = cur;
       nxt.advance(a);
-      const int32_t row_next = nxt.valid ? chunk_row(nxt) : rows_total;
+      const int32_t id_next = nxt.valid ? chunk_id(nxt) : -1;
+      uint4 qn[kQChunksPerLane];
+      const bool gather_next = is_gather(nxt);
+      if (gather_next) gather_q(nxt, qn);
+      const int32_t row = id_row(cur, id);
       if (cur.first()) {
         const uint32_t qb = ucnt & 1u;
-        if (GRP && cur.w.sg >= 0) {
-          // shared-prefix unit: column j is query head g * G + j % G of member
-          // j / G; the warp gathers the rows into the 128-byte-swizzled layout
-          // a TMA load would produce (chunk c of row j at (c ^ (j & 7)) * 16)
-          if (lane == 0) ok = mbar_wait(&q_empty[qb], ((ucnt >> 1) & 1u) ^ 1u, 0x7100u);
-          ok = __shfl_sync(0xffffffffu, ok, 0);
-          if (ok) {
-            const int32_t* e = tc::sub_entry(gh, cur.w.sg);
-            const int32_t ncol = tc::plan_at(gh, e + 1) * G;
-            uint8_t* qdst = qbuf + qb * kQBytes;
-            for (int idx = lane; idx < kN * 16; idx += 32) {
-              const int j = idx >> 4, ch = idx & 15;
-              uint4 v = make_uint4(0, 0, 0, 0);
-              if (j < ncol) {
-                const int32_t m = j / G;
-                const int64_t qrow =
-                    int64_t(tc::plan_at(gh, e + 4 + m)) * a.num_q_heads + cur.w.g * G + (j - m * G);
-                v = __ldg(reinterpret_cast<const uint4*>(static_cast<const T*>(a.q) + qrow * kD) + ch);
-              }
-              *reinterpret_cast<uint4*>(qdst + (ch >> 3) * (kN * 128) + j * 128 +
-                                        (((ch & 7) ^ (j & 7)) << 4)) = v;
-            }
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&q_full[qb]);
+        if (lane == 0) ok = mbar_wait(&q_empty[qb], ((ucnt >> 1) & 1u) ^ 1u, 0x7100u);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        if (is_gather(cur)) {
+          uint8_t* qdst = qbuf + qb * kQBytes;
+#pragma unroll
+          for (int i = 0; i < kQChunksPerLane; ++i) {
+            const int idx = lane + 32 * i;
+            const int j = idx >> 4, ch = idx & 15;
+            *reinterpret_cast<uint4*>(qdst + (ch >> 3) * (kN * 128) + j * 128 +
+                                      (((ch & 7) ^ (j & 7)) << 4)) = qv[i];
           }
-        } else {
-          if (lane == 0) {
-            ok = mbar_wait(&q_empty[qb], ((ucnt >> 1) & 1u) ^ 1u, 0x7100u);
-            if (ok) {
-              mbar_arrive_expect_tx(&q_full[qb], kQBytes);
-              const int32_t qrow = cur.w.s * a.num_q_heads + cur.w.g * G;
-              tma_load_2d(qbuf + qb * kQBytes, &qmap, &q_full[qb], 0, qrow, pol_q);
-              tma_load_2d(qbuf + qb * kQBytes + kN * 128, &qmap, &q_full[qb], 64, qrow, pol_q);
-            }
-          }
-          ok = __shfl_sync(0xffffffffu, ok, 0);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&q_full[qb]);
+        } else if (lane == 0) {
+          mbar_arrive_expect_tx(&q_full[qb], kQBytes);
+          const int32_t qrow = cur.w.s * a.num_q_heads + cur.w.g * G;
+          tma_load_2d(qbuf + qb * kQBytes, &qmap, &q_full[qb], 0, qrow, pol_q);
+          tma_load_2d(qbuf + qb * kQBytes + kN * 128, &qmap, &q_full[qb], 64, qrow, pol_q);
         }
         ++ucnt;
-        if (!ok) break;
       }
       const int32_t nt = cur.tiles();
-      load_tiles(&kmap, row, nt);
-      if (have_pend && ok) load_tiles(&vmap, pend_row, pend_tiles);
+      load_tiles(&kmap, row, nt, false);
+      if (have_pend && ok) load_tiles(&vmap, pend_row, pend_tiles, true);
       pend_row = row;
       pend_tiles = nt;
       have_pend = true;
-      row = row_next;
+      id = id_next;
+      if (gather_next) {
+#pragma unroll
+        for (int i = 0; i < kQChunksPerLane; ++i) qv[i] = qn[i];
+      }
       cur = nxt;
     }
-    if (have_pend && ok) load_tiles(&vmap, pend_row, pend_tiles);
+    if (have_pend && ok) load_tiles(&vmap, pend_row, pend_tiles, true);
     if (!ok) {
       atomicExch(&abort_flag, 1);
       if (lane == 0)  // drain the loads that may still be in flight
@@ -594,10 +628,12 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
         if (t == ntile - 1 && zero_from < kTileTok) {
           uint8_t* tile = ring + st * kStageBytes;
           for (int row = zero_from + lane; row < kTileTok; row += 32) {
+            // token row of block row / BS: [half][BS rows][128 bytes]
+            uint8_t* r0 = tile + (row / BS) * (BS * 256) + (row % BS) * 128;
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
-              reinterpret_cast<uint4*>(tile + row * 128)[q] = make_uint4(0, 0, 0, 0);
-              reinterpret_cast<uint4*>(tile + kRegionBytes + row * 128)[q] = make_uint4(0, 0, 0, 0);
+              reinterpret_cast<uint4*>(r0)[q] = make_uint4(0, 0, 0, 0);
+              reinterpret_cast<uint4*>(r0 + BS * 128)[q] = make_uint4(0, 0, 0, 0);
             }
           }
           fence_proxy_async_smem();
@@ -609,7 +645,10 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
 #pragma unroll
           for (int kk = 0; kk < kTileTok / 16; ++kk) {
             const uint32_t pk = (t * kTileTok + kk * 16) / 8 * L::kPLbo;
-            umma_f16_ss(o_tmem, smem_desc(v_addr + kk * 2048, kRegionBytes, 1024, kLayoutSw128),
+            // V^T, MN-major: tokens kk*16.. of block (kk*16)/BS; the two 64-dim
+            // halves BS*128 bytes apart (LBO), 8-token groups 1024 apart (SBO)
+            const uint32_t va = v_addr + ((kk * 16) / BS) * (BS * 256) + ((kk * 16) % BS) * 128;
+            umma_f16_ss(o_tmem, smem_desc(va, BS * 128, 1024, kLayoutSw128),
                         smem_desc(p_addr + pk, L::kPLbo, 128, kLayoutNone), kIdescPV,
                         (t > 0 || kk > 0) ? 1u : 0u);
           }

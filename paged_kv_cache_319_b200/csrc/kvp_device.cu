@@ -37,6 +37,22 @@ using kvp::fail;
 #ifndef KVP_SIMT_STAGES
 #define KVP_SIMT_STAGES 2
 #endif
+// Grouped decode with a host plan: the tensor-core kernel's per-SM rate on
+// shared blocks, in percent of the CUDA-core kernel's rate on a sequence's own
+// blocks; it sets the tensor-core kernel's share of the SMs.
+#ifndef KVP_GROUP_TC_RATE
+#define KVP_GROUP_TC_RATE 70
+#endif
+// Grouped decode: the CUDA-core kernel on the sequences' own ranges. Ranges
+// that average fewer than KVP_GROUP_PER_HEAD_BELOW blocks per sequence (beams,
+// a block or two each) run with per-head warps (each warp one query head's
+// whole range, 4 warps x 3 stages); longer ones as in the plain decode (warps
+// split a range's blocks). On the OPT-13B geometry: 8 parallel samples with
+// about 9 own blocks each, 70.7 us split against 74.9 us per-head; beams of
+// about 1 own block, 54.3 us split against 50.1 us per-head.
+#ifndef KVP_GROUP_PER_HEAD_BELOW
+#define KVP_GROUP_PER_HEAD_BELOW 4
+#endif
 
 namespace {
 
@@ -173,7 +189,7 @@ GroupWorkspace group_ws_layout(int64_t S, int64_t Hq, int64_t D, int64_t pmax) {
   GroupWorkspace w{};
   w.ml_bytes = up(size_t(S * Hq * (pmax + 1) * 2 * 4));
   w.acc_bytes = up(size_t(S * Hq * (pmax + 1) * D * 4));
-  w.plan_bytes = up(size_t(kvp::dev::grp::plan_words(S) * 4));
+  w.plan_bytes = up(size_t(kvp::grp::plan_words(S) * 4));
   w.total = w.ml_bytes + w.acc_bytes + w.plan_bytes;
   return w;
 }
@@ -181,16 +197,17 @@ GroupWorkspace group_ws_layout(int64_t S, int64_t Hq, int64_t D, int64_t pmax) {
 // ---- decode launches ----------------------------------------------------------
 // programmatic: launched with programmatic stream serialisation (the grouped
 // decode, after the shared-prefix kernel).
-template <typename T, int D, int BS>
+template <typename T, int D, int BS, int W = KVP_SIMT_WARPS, int NST = KVP_SIMT_STAGES,
+          bool PH = false>
 int launch_simt(const CUtensorMap& km, const CUtensorMap& vm, const kvp::dev::DecodeArgs& a,
-                cudaStream_t st, bool programmatic = false) {
-  constexpr int NW = (BS * D * 2 >= 8192 && KVP_SIMT_WARPS > 1) ? KVP_SIMT_WARPS / 2 : KVP_SIMT_WARPS;
-  constexpr int NST = KVP_SIMT_STAGES;
+                cudaStream_t st, bool programmatic = false, int grid_x = 0) {
+  constexpr int NW = (BS * D * 2 >= 8192 && W > 1) ? W / 2 : W;
   using C = kvp::dev::SimtCfg<T, D, BS, NW, NST>;
-  auto k = kvp::dev::decode_simt_kernel<T, D, BS, NW, NST>;
+  auto k = kvp::dev::decode_simt_kernel<T, D, BS, NW, NST, PH>;
   cudaError_t e = ensure_smem(k, C::kSmemBytes);
   if (e != cudaSuccess) return cuda_fail(e, "decode (CUDA cores): smem attribute");
-  dim3 grid(a.pmax, a.num_q_heads, a.num_seqs);
+  dim3 grid(grid_x > 0 ? grid_x : a.pmax, PH ? (a.num_q_heads + NW - 1) / NW : a.num_q_heads,
+            a.num_seqs);
   if (!programmatic) {
     k<<<grid, NW * 32, C::kSmemBytes, st>>>(km, vm, a);
   } else {
@@ -263,14 +280,17 @@ int simt_by_bs(int bs, const CUtensorMap& km, const CUtensorMap& vm, const kvp::
 // wait for it (griddepcontrol.wait) before reading it.
 // with_private: the kernel also takes every sequence's own range (else the
 // CUDA-core kernel launched after it does).
+// grid_ctas > 0 sets the grid (else one CTA per SM, at most one per unit);
+// programmatic: launched right after the plan kernel, overlapping it.
 template <typename T, int BS, int NG>
 int launch_tc_grouped(const CUtensorMap& km, const CUtensorMap& vm, const CUtensorMap& qm,
-                      const kvp::dev::DecodeArgs& a, cudaStream_t st, bool with_private) {
+                      const kvp::dev::DecodeArgs& a, cudaStream_t st, bool with_private,
+                      int grid_ctas, bool programmatic) {
   auto k = kvp::dev::decode_tc_kernel<T, BS, NG, true>;
   using Cfg = kvp::dev::tc::Cfg<NG>;
   // shared-memory tail: context lengths, per-sequence prefix blocks and the
   // subgroup table when they fit (S <= kPlanCap), else the context lengths alone
-  auto plan_bytes = [](int S) { return 8 * S + (S / 2 + 1) * kvp::dev::grp::kSubWords * 4; };
+  auto plan_bytes = [](int S) { return 8 * S + (S / 2 + 1) * kvp::grp::kSubWords * 4; };
   const int S = a.num_seqs;
   const int ctx_bytes = S <= Cfg::kPlanCap ? plan_bytes(S) : (S <= Cfg::kCtxCap ? 4 * S : 0);
   const int tail_max = std::max(4 * Cfg::kCtxCap, plan_bytes(Cfg::kPlanCap));
@@ -281,7 +301,7 @@ int launch_tc_grouped(const CUtensorMap& km, const CUtensorMap& vm, const CUtens
   const int64_t bound = std::max<int64_t>(
       1, units + int64_t(a.num_seqs / 2) * a.num_kv_heads * a.pmax);
   cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3(unsigned(bound < sm_count() ? bound : sm_count()));
+  cfg.gridDim = dim3(unsigned(grid_ctas > 0 ? grid_ctas : (bound < sm_count() ? bound : sm_count())));
   cfg.blockDim = dim3(kvp::dev::tc::kThreads);
   cfg.dynamicSmemBytes = size_t(Cfg::kSmemBytes + ctx_bytes);
   cfg.stream = st;
@@ -289,7 +309,7 @@ int launch_tc_grouped(const CUtensorMap& km, const CUtensorMap& vm, const CUtens
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = programmatic ? 1 : 0;
   e = cudaLaunchKernelEx(&cfg, k, km, vm, qm, a, units);
   if (e == cudaSuccess) e = cudaGetLastError();
   return e == cudaSuccess ? KVP_OK : cuda_fail(e, "grouped decode: launch");
@@ -298,11 +318,35 @@ int launch_tc_grouped(const CUtensorMap& km, const CUtensorMap& vm, const CUtens
 template <typename T>
 int tc_grouped_dispatch(int bs, int ng, const CUtensorMap& km, const CUtensorMap& vm,
                         const CUtensorMap& qm, const kvp::dev::DecodeArgs& a, cudaStream_t st,
-                        bool with_private) {
-  if (bs == 16) return ng == 8 ? launch_tc_grouped<T, 16, 8>(km, vm, qm, a, st, with_private)
-                               : launch_tc_grouped<T, 16, 16>(km, vm, qm, a, st, with_private);
-  return ng == 8 ? launch_tc_grouped<T, 32, 8>(km, vm, qm, a, st, with_private)
-                 : launch_tc_grouped<T, 32, 16>(km, vm, qm, a, st, with_private);
+                        bool with_private, int grid_ctas, bool programmatic) {
+  if (bs == 16)
+    return ng == 8 ? launch_tc_grouped<T, 16, 8>(km, vm, qm, a, st, with_private, grid_ctas, programmatic)
+                   : launch_tc_grouped<T, 16, 16>(km, vm, qm, a, st, with_private, grid_ctas, programmatic);
+  return ng == 8 ? launch_tc_grouped<T, 32, 8>(km, vm, qm, a, st, with_private, grid_ctas, programmatic)
+                 : launch_tc_grouped<T, 32, 16>(km, vm, qm, a, st, with_private, grid_ctas, programmatic);
+}
+
+// Grouped decode: the CUDA-core kernel over the sequences' own ranges
+// (grid_x partitions; 0: all).
+int launch_own_ranges(int bs, int32_t dtype, bool per_head, const CUtensorMap& km,
+                      const CUtensorMap& vm, const kvp::dev::DecodeArgs& a, cudaStream_t st,
+                      bool programmatic, int grid_x) {
+  using H = __half;
+  using B = __nv_bfloat16;
+  constexpr int W = KVP_SIMT_WARPS, N = KVP_SIMT_STAGES;
+  const bool f16 = dtype == KVP_F16;
+  if (per_head) {
+    if (bs == 16)
+      return f16 ? launch_simt<H, 128, 16, 4, 3, true>(km, vm, a, st, programmatic, grid_x)
+                 : launch_simt<B, 128, 16, 4, 3, true>(km, vm, a, st, programmatic, grid_x);
+    return f16 ? launch_simt<H, 128, 32, 4, 3, true>(km, vm, a, st, programmatic, grid_x)
+               : launch_simt<B, 128, 32, 4, 3, true>(km, vm, a, st, programmatic, grid_x);
+  }
+  if (bs == 16)
+    return f16 ? launch_simt<H, 128, 16, W, N>(km, vm, a, st, programmatic, grid_x)
+               : launch_simt<B, 128, 16, W, N>(km, vm, a, st, programmatic, grid_x);
+  return f16 ? launch_simt<H, 128, 32, W, N>(km, vm, a, st, programmatic, grid_x)
+             : launch_simt<B, 128, 32, W, N>(km, vm, a, st, programmatic, grid_x);
 }
 
 template <typename T>
@@ -478,6 +522,10 @@ int paged_attention_decode(const void* q, const void* k_cache, const void* v_cac
     rc = make_map_halves(&km, k_cache, dtype, rows, block_size);
     if (rc) return rc;
     rc = make_map_halves(&vm, v_cache, dtype, rows, block_size);
+  } else if (tensor_cores) {  // K as 2-D boxes per 64-dim half, V as one 3-D box per block
+    rc = make_map(&km, k_cache, dtype, rows, head_dim, block_size);
+    if (rc) return rc;
+    rc = make_map_halves(&vm, v_cache, dtype, rows, block_size);
   } else {
     rc = make_map(&km, k_cache, dtype, rows, head_dim, block_size);
     if (rc) return rc;
@@ -520,8 +568,10 @@ int paged_attention_decode_grouped(const void* q, const void* k_cache, const voi
                                    int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
                                    int32_t head_dim, int32_t block_size, int32_t num_blocks,
                                    int32_t max_blocks_per_seq, int32_t max_context_len, float scale,
-                                   int32_t partition_size, void* workspace, size_t workspace_bytes,
-                                   void* out, int32_t dtype, kvp_stream_t stream) {
+                                   int32_t partition_size, const int32_t* host_plan,
+                                   const int32_t* device_plan, void* workspace,
+                                   size_t workspace_bytes, void* out, int32_t dtype,
+                                   kvp_stream_t stream) {
   bool empty = false;
   const int crc = check_decode("paged_attention_decode_grouped", q, k_cache, v_cache, block_tables,
                                context_lens, num_seqs, num_q_heads, num_kv_heads, head_dim,
@@ -531,11 +581,11 @@ int paged_attention_decode_grouped(const void* q, const void* k_cache, const voi
   // Columns of the tensor-core contraction: 8 for one query head per KV head
   // (up to 8 members per subgroup), else 16 (16 / G members).
   const int G = num_q_heads / num_kv_heads;
-  const int ng = G == 1 ? 8 : 16;
-  const int mmax = ng / G;
+  const int ng = kvp::grp::plan_columns(G);
+  const int mmax = kvp::grp::members_per_subgroup(G);
   const bool grouped = head_dim == 128 && (block_size == 16 || block_size == 32) && G <= 16 &&
                        mmax >= 2 && partition_size > 0 && partition_size % 128 == 0 &&
-                       num_seqs <= kvp::dev::grp::kMaxSeqs && max_context_len > 0;
+                       num_seqs <= kvp::grp::kMaxSeqs && max_context_len > 0;
   if (!grouped)
     return paged_attention_decode(q, k_cache, v_cache, block_tables, context_lens, num_seqs,
                                   num_q_heads, num_kv_heads, head_dim, block_size, num_blocks,
@@ -549,8 +599,13 @@ int paged_attention_decode_grouped(const void* q, const void* k_cache, const voi
   if (!aligned(workspace, 256))
     return fail(KVP_ERR_INVALID, "paged_attention_decode_grouped: workspace not 256-byte aligned");
 
+  if (device_plan && !host_plan)
+    return fail(KVP_ERR_INVALID, "paged_attention_decode_grouped: device_plan needs host_plan");
+  if (device_plan && !aligned(device_plan, 4))
+    return fail(KVP_ERR_INVALID, "paged_attention_decode_grouped: misaligned device_plan");
   char* ws = static_cast<char*>(workspace);
-  int32_t* plan = reinterpret_cast<int32_t*>(ws + wl.ml_bytes + wl.acc_bytes);
+  int32_t* plan = device_plan ? const_cast<int32_t*>(device_plan)
+                              : reinterpret_cast<int32_t*>(ws + wl.ml_bytes + wl.acc_bytes);
   kvp::dev::DecodeArgs a{};
   a.q = q;
   a.out = out;
@@ -576,39 +631,82 @@ int paged_attention_decode_grouped(const void* q, const void* k_cache, const voi
   // grouped-query heads the tensor-core kernel takes both.
   const bool simt_private = G == 1;
   const uint64_t rows = uint64_t(num_blocks) * num_kv_heads * block_size;
-  CUtensorMap km, vm, qm, km3, vm3;
+  // tensor cores: K as 2-D boxes, V as 3-D boxes; CUDA cores: both 3-D
+  CUtensorMap km, vm3, qm, km3;
   int rc = make_map(&km, k_cache, dtype, rows, head_dim, block_size);
-  if (!rc) rc = make_map(&vm, v_cache, dtype, rows, head_dim, block_size);
+  if (!rc) rc = make_map_halves(&vm3, v_cache, dtype, rows, block_size);
   if (!rc) rc = make_map(&qm, q, dtype, uint64_t(num_seqs) * num_q_heads, head_dim, kvp::dev::tc::kN);
   if (!rc && simt_private) rc = make_map_halves(&km3, k_cache, dtype, rows, block_size);
-  if (!rc && simt_private) rc = make_map_halves(&vm3, v_cache, dtype, rows, block_size);
   if (rc) return rc;
+  const CUtensorMap& vm = vm3;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
 
-  // 1. the plan (one CTA)
   using namespace kvp::dev;
-  cudaError_t e = ensure_smem(group_plan_kernel, int(grp::plan_smem_bytes(grp::kMaxSeqs)));
-  if (e != cudaSuccess) return cuda_fail(e, "grouped decode: plan smem attribute");
-  group_plan_kernel<<<1, grp::plan_threads(grp::sort_len(num_seqs)), grp::plan_smem_bytes(num_seqs),
-                      st>>>(block_tables, context_lens, num_seqs, max_blocks_per_seq,
-                            max_context_len, block_size, partition_size, mmax, num_blocks, plan);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return cuda_fail(e, "grouped decode: plan launch");
-  // 2. shared prefixes once per subgroup (and, with grouped-query heads, every
-  // sequence's own range) on the tensor cores
-  rc = dtype == KVP_F16
-           ? tc_grouped_dispatch<__half>(block_size, ng, km, vm, qm, a, st, !simt_private)
-           : tc_grouped_dispatch<__nv_bfloat16>(block_size, ng, km, vm, qm, a, st, !simt_private);
-  if (rc) return rc;
-  // 2b. every sequence's own range on the CUDA cores, overlapping the tail of 2
-  if (simt_private) {
-    if (block_size == 16)
-      rc = dtype == KVP_F16 ? launch_simt<__half, 128, 16>(km3, vm3, a, st, true)
-                            : launch_simt<__nv_bfloat16, 128, 16>(km3, vm3, a, st, true);
-    else
-      rc = dtype == KVP_F16 ? launch_simt<__half, 128, 32>(km3, vm3, a, st, true)
-                            : launch_simt<__nv_bfloat16, 128, 32>(km3, vm3, a, st, true);
+  const int sms = sm_count();
+  bool after_kernel = false;  // the tensor-core kernel precedes the CUDA-core one
+  if (host_plan) {
+    // 1. the caller's plan (host memory) into the workspace; its header sizes
+    // the launches: the tensor-core kernel gets a share of the SMs by the
+    // estimated times of the shared blocks and of the sequences' own blocks,
+    // and the CUDA-core kernel, launched right after it, the rest
+    namespace g = kvp::grp;
+    const int32_t n_sub = host_plan[g::kNumSub], psh = host_plan[g::kSharedParts];
+    const int32_t pown = host_plan[g::kOwnParts];
+    const int32_t sblk = host_plan[g::kSharedBlocks], oblk = host_plan[g::kOwnBlocks];
+    if (n_sub < 0 || n_sub > num_seqs / 2 || psh < 0 || psh > pmax || pown < 0 || pown > pmax ||
+        sblk < 0 || oblk < 0)
+      return fail(KVP_ERR_INVALID, "paged_attention_decode_grouped: host_plan does not fit this batch");
+    if (!device_plan) {
+      cudaError_t e = cudaMemcpyAsync(plan, host_plan, size_t(g::plan_words(num_seqs)) * 4,
+                                      cudaMemcpyHostToDevice, st);
+      if (e != cudaSuccess) return cuda_fail(e, "grouped decode: plan copy");
+    }
+    if (simt_private) {
+      const int64_t shared_units = int64_t(n_sub) * psh * num_kv_heads;
+      if (shared_units > 0) {
+        const double ts = double(sblk) * 100.0 / KVP_GROUP_TC_RATE, to = double(oblk);
+        int64_t grid = std::llround(sms * ts / (ts + to));
+        grid = std::max<int64_t>(1, std::min<int64_t>(grid, std::min<int64_t>(sms, shared_units)));
+        rc = dtype == KVP_F16
+                 ? tc_grouped_dispatch<__half>(block_size, ng, km, vm, qm, a, st, false, int(grid), false)
+                 : tc_grouped_dispatch<__nv_bfloat16>(block_size, ng, km, vm, qm, a, st, false, int(grid), false);
+        if (rc) return rc;
+        after_kernel = true;
+      }
+      if (pown > 0) {
+        const bool per_head = int64_t(oblk) < int64_t(KVP_GROUP_PER_HEAD_BELOW) * num_seqs;
+        rc = launch_own_ranges(block_size, dtype, per_head, km3, vm3, a, st, after_kernel, pown);
+        if (rc) return rc;
+      }
+    } else {
+      const int64_t units = int64_t(num_seqs) * num_kv_heads * pmax + int64_t(n_sub) * psh * num_kv_heads;
+      const int grid = int(std::max<int64_t>(1, std::min<int64_t>(units, sms)));
+      rc = dtype == KVP_F16
+               ? tc_grouped_dispatch<__half>(block_size, ng, km, vm, qm, a, st, true, grid, false)
+               : tc_grouped_dispatch<__nv_bfloat16>(block_size, ng, km, vm, qm, a, st, true, grid, false);
+      if (rc) return rc;
+    }
+  } else {
+    // 1. the plan (one CTA)
+    cudaError_t e = ensure_smem(group_plan_kernel, int(kvp::grp::plan_smem_bytes(kvp::grp::kMaxSeqs)));
+    if (e != cudaSuccess) return cuda_fail(e, "grouped decode: plan smem attribute");
+    group_plan_kernel<<<1, kvp::grp::plan_threads(kvp::grp::sort_len(num_seqs)),
+                        kvp::grp::plan_smem_bytes(num_seqs), st>>>(
+        block_tables, context_lens, num_seqs, max_blocks_per_seq, max_context_len, block_size,
+        partition_size, mmax, num_blocks, plan);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "grouped decode: plan launch");
+    // 2. shared prefixes once per subgroup (and, with grouped-query heads, every
+    // sequence's own range) on the tensor cores, overlapping the plan kernel
+    rc = dtype == KVP_F16
+             ? tc_grouped_dispatch<__half>(block_size, ng, km, vm, qm, a, st, !simt_private, 0, true)
+             : tc_grouped_dispatch<__nv_bfloat16>(block_size, ng, km, vm, qm, a, st, !simt_private, 0, true);
     if (rc) return rc;
+    // 2b. every sequence's own range on the CUDA cores, overlapping the tail of 2
+    if (simt_private) {
+      rc = launch_own_ranges(block_size, dtype, false, km3, vm3, a, st, true, 0);
+      if (rc) return rc;
+    }
   }
   // 3. the log-sum-exp merge of every row
   return dtype == KVP_F16 ? launch_reduce<__half, 128>(a, st) : launch_reduce<__nv_bfloat16, 128>(a, st);

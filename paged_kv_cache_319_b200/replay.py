@@ -19,7 +19,9 @@ import numpy as np
 
 from workloads.values import K_STREAM, Q_STREAM, V_STREAM, normal_bits, value_seed_words
 
-from . import BlockPool, copy_blocks, paged_attention_decode, reshape_and_cache
+import time
+
+from . import BlockPool, copy_blocks, group_plan, paged_attention_decode, reshape_and_cache
 
 
 def bits_to_tensor(bits: np.ndarray, dtype: str, device):
@@ -32,7 +34,7 @@ def bits_to_tensor(bits: np.ndarray, dtype: str, device):
 
 class DeviceReplay:
     def __init__(self, wl, device="cuda", keep_outputs: bool = True, time_decode: bool = False,
-                 grouped: bool = False, time_reps: int = 1):
+                 grouped: bool = False, time_reps: int = 1, plan_on: str = "host"):
         import torch
 
         g = wl.geometry
@@ -52,6 +54,8 @@ class DeviceReplay:
         self.keep_outputs = keep_outputs
         self.time_decode = time_decode
         self.grouped = grouped     # decode through paged_attention_decode_grouped
+        self.plan_on = plan_on     # grouped: "host" (kv_decode_group_plan) or "device"
+        self.plan_us = []          # host time of each grouping plan
         self.time_reps = max(1, int(time_reps))  # timed calls per attend op (time_decode)
         self.decode_events = []    # (op_index, start event, end event) around each decode call
         self.next_index = 0
@@ -126,9 +130,19 @@ class DeviceReplay:
             part = kw.get("partition_size", self.wl.partition_size)
             grouped = kw.get("grouped", self.grouped)
             mcl = int(lens.max()) if len(lens) else 0
+            plan = dplan = None
+            if grouped and self.plan_on == "host" and part > 0 and len(lens):
+                t0 = time.perf_counter()
+                plan = group_plan(tables, lens, block_size=bs, partition_size=part,
+                                  num_q_heads=self.g.num_q_heads, num_kv_heads=self.g.num_kv_heads,
+                                  num_blocks=self.wl.num_blocks, max_context_len=mcl)
+                self.plan_us.append((time.perf_counter() - t0) * 1e6)
+                # uploaded with the block tables, as an engine would
+                dplan = torch.from_numpy(plan).to(self.device)
             call = lambda: paged_attention_decode(q, self.k_cache, self.v_cache, bt, cl,  # noqa: E731
                                                   self.wl.scale, max_context_len=mcl,
-                                                  partition_size=part, grouped=grouped)
+                                                  partition_size=part, grouped=grouped,
+                                                  host_plan=plan, device_plan=dplan)
             if self.time_decode:
                 # an untimed call, then before each timed call an L2 flush: a
                 # 256 MB write, then a 256 MB read of another buffer, which writes

@@ -9,7 +9,8 @@ cover groups larger than one subgroup (with a leftover member of one), a
 member whose partial last block another member holds in full (the shared
 prefix stops at full blocks), whole-sequence duplicates, sequences that share
 only their first block, sequences shorter than a block, empty sequences,
-shared prefixes that end inside a partition, grouped-query heads, and
+shared prefixes that end inside a partition, own ranges of a block or two
+(per-head warps), grouped-query heads, and
 batches the entry point hands to paged_attention_decode (unsplit, a query
 group too wide for two members, a head size the tensor cores do not take,
 more sequences than the plan takes).
@@ -63,15 +64,26 @@ def shared_batch(seed, groups, Hq, Hkv, D, bs, dtype, extra_blocks=5):
     return q, k, v, tables, lens
 
 
-def run(q, k, v, tables, lens, dtype, scale, partition, grouped, workspace=None):
+def host_plan(tables, lens, Hq, Hkv, bs, partition, num_blocks):
+    import paged_kv_cache_319_b200 as kvp
+
+    return kvp.group_plan(tables, lens, block_size=bs, partition_size=partition, num_q_heads=Hq,
+                          num_kv_heads=Hkv, num_blocks=num_blocks,
+                          max_context_len=int(max(lens.max(), 1)))
+
+
+def run(q, k, v, tables, lens, dtype, scale, partition, grouped, workspace=None, plan=None,
+        upload=False):
+    """upload: also pass a device copy of the host plan (the call then copies nothing)."""
     import torch
     import paged_kv_cache_319_b200 as kvp
 
+    dplan = torch.from_numpy(plan).cuda() if upload and plan is not None else None
     out = kvp.paged_attention_decode(
         from_bits(q, dtype), from_bits(k, dtype), from_bits(v, dtype),
         torch.from_numpy(tables).cuda(), torch.from_numpy(lens).cuda(), scale,
         max_context_len=int(max(lens.max(), 1)), partition_size=partition, grouped=grouped,
-        workspace=workspace)
+        workspace=workspace, host_plan=plan, device_plan=dplan)
     kvp.check_device_error()
     return to_bits(out)
 
@@ -97,6 +109,11 @@ CASES = [
     ("mha_f16_bs16_p512", 8, 8, 16, "f16", 512, GROUPS_MHA),
     ("mha_bf16_bs32_p128", 4, 4, 32, "bf16", 128, GROUPS_MHA),
     ("mha_f16_bs16_p256", 2, 2, 16, "f16", 256, GROUPS_MHA),
+    # own ranges of a block or two (beams): per-head warps on the CUDA cores
+    ("mha_short_own_f16_bs16", 8, 8, 16, "f16", 512,
+     [(30, [480, 481, 482, 490, 500, 495]), (20, [320, 321, 322]), (2, [33, 40]), (0, [9])]),
+    ("mha_short_own_bf16_bs32", 6, 6, 32, "bf16", 256,
+     [(15, [480, 481, 482, 500]), (9, [288, 300]), (0, [40])]),
     ("gqa4_bf16_bs16_p512", 16, 4, 16, "bf16", 512,
      [(31, [600, 700, 511, 767, 520]), (8, [128, 300, 129]), (0, [0]), (0, [7]), (0, [2000])]),
     ("gqa2_f16_bs32_p256", 8, 4, 32, "f16", 256,
@@ -111,14 +128,48 @@ CASES = [
 ]
 
 
+@pytest.mark.parametrize("plan_on", ["device", "host", "host+upload"])
 @pytest.mark.parametrize("name,Hq,Hkv,bs,dtype,partition,groups", CASES, ids=[c[0] for c in CASES])
-def test_grouped_matches_oracle(name, Hq, Hkv, bs, dtype, partition, groups):
+def test_grouped_matches_oracle(name, Hq, Hkv, bs, dtype, partition, groups, plan_on):
     seed = sum(map(ord, name))
     q, k, v, t, l = shared_batch(seed, groups, Hq, Hkv, 128, bs, dtype)
     scale = 1 / math.sqrt(128)
-    got = run(q, k, v, t, l, dtype, scale, partition, grouped=True)
+    plan = None
+    if plan_on.startswith("host") and partition:
+        plan = host_plan(t, l, Hq, Hkv, bs, partition, k.shape[0])
+    got = run(q, k, v, t, l, dtype, scale, partition, grouped=True, plan=plan,
+              upload=plan_on.endswith("upload"))
     ref = oracle(q, k, v, t, l, dtype, scale, bs)
     check_close(got, ref, dtype, allow_ulp=(dtype == "bf16"))
+
+
+@pytest.mark.parametrize("name,Hq,Hkv,bs,dtype,partition,groups",
+                         [c for c in CASES if c[5] and c[1] // c[2] < 16],
+                         ids=[c[0] for c in CASES if c[5] and c[1] // c[2] < 16])
+def test_device_plan_equals_host_plan(name, Hq, Hkv, bs, dtype, partition, groups):
+    """The GPU plan kernel and the host planner build the same plan, word for word."""
+    import torch
+
+    q, k, v, t, l = shared_batch(sum(map(ord, name)), groups, Hq, Hkv, 128, bs, dtype)
+    S, mcl = len(l), int(l.max())
+    import paged_kv_cache_319_b200 as kvp
+
+    need = kvp.decode_grouped_workspace_bytes(S, Hq, 128, mcl, partition)
+    ws = torch.full((need,), 0x7F, dtype=torch.uint8, device="cuda")
+    run(q, k, v, t, l, dtype, 0.09, partition, grouped=True, workspace=ws)
+    pmax = -(-mcl // partition)
+    up = lambda x: (x + 255) // 256 * 256  # noqa: E731
+    off = up(S * Hq * (pmax + 1) * 8) + up(S * Hq * (pmax + 1) * 128 * 4)
+    ref = host_plan(t, l, Hq, Hkv, bs, partition, k.shape[0])
+    dev = ws[off:off + 4 * len(ref)].cpu().numpy().view(np.int32)
+    # member slots past a subgroup's size are not written by the GPU kernel
+    n_sub = int(ref[0])
+    mask = np.ones(len(ref), bool)
+    for i in range(n_sub):
+        e = 8 + S + i * 20
+        mask[e + 4 + ref[e + 1]:e + 20] = False
+    mask[8 + S + n_sub * 20:] = False
+    assert np.array_equal(dev[mask], ref[mask])
 
 
 def test_head_dim_64_is_handed_on():
@@ -145,12 +196,37 @@ def test_reused_workspace_two_batches_in_a_row():
     for seed, groups in ((1, GROUPS_MHA), (2, [(2, [40, 2000, 700]), (0, [900]), (9, [150] * 5)])):
         q, k, v, t, l = shared_batch(seed, groups, 8, 8, 128, 16, "f16")
         assert l.max() <= 2048 and len(l) <= 64
-        got = run(q, k, v, t, l, "f16", 0.09, 512, grouped=True, workspace=ws)
-        check_close(got, oracle(q, k, v, t, l, "f16", 0.09, 16), "f16")
+        for plan in (None, host_plan(t, l, 8, 8, 16, 512, k.shape[0])):
+            got = run(q, k, v, t, l, "f16", 0.09, 512, grouped=True, workspace=ws, plan=plan)
+            check_close(got, oracle(q, k, v, t, l, "f16", 0.09, 16), "f16")
 
 
+def test_host_plan_of_another_batch_is_rejected():
+    import torch
+    import paged_kv_cache_319_b200 as kvp
+    from paged_kv_cache_319_b200._lib import KvpError
+
+    q, k, v, t, l = shared_batch(3, [(4, [100, 120]), (0, [30])], 8, 8, 128, 16, "f16")
+    plan = host_plan(t, l, 8, 8, 16, 512, k.shape[0])
+    bad = plan.copy()
+    bad[0] = 99  # more subgroups than the batch can have
+    with pytest.raises(KvpError) as e:
+        run(q, k, v, t, l, "f16", 0.09, 512, grouped=True, plan=bad)
+    assert e.value.kind == "invalid"
+    # a device copy without the host plan it copies is rejected too
+    with pytest.raises(KvpError) as e:
+        kvp.paged_attention_decode(
+            from_bits(q, "f16"), from_bits(k, "f16"), from_bits(v, "f16"),
+            torch.from_numpy(t).cuda(), torch.from_numpy(l).cuda(), 0.09,
+            max_context_len=int(l.max()), partition_size=512, grouped=True,
+            device_plan=torch.from_numpy(plan).cuda())
+    assert e.value.kind == "invalid"
+    torch.cuda.synchronize()
+
+
+@pytest.mark.parametrize("plan_on", ["device", "host"])
 @pytest.mark.parametrize("S", [4096, 4100])
-def test_batch_size_limit_of_the_plan(S):
+def test_batch_size_limit_of_the_plan(S, plan_on):
     """4096 sequences are grouped (the plan's limit); 4100 go through paged_attention_decode."""
     rng = np.random.default_rng(S)
     groups, n = [], 0
@@ -159,12 +235,14 @@ def test_batch_size_limit_of_the_plan(S):
         groups.append((int(rng.integers(1, 4)), rng.integers(1, 60, size=m).tolist()))
         n += m
     q, k, v, t, l = shared_batch(S, groups, 1, 1, 128, 16, "f16")
-    got = run(q, k, v, t, l, "f16", 0.09, 128, grouped=True)
+    plan = host_plan(t, l, 1, 1, 16, 128, k.shape[0]) if plan_on == "host" and S <= 4096 else None
+    got = run(q, k, v, t, l, "f16", 0.09, 128, grouped=True, plan=plan)
     check_close(got, oracle(q, k, v, t, l, "f16", 0.09, 16), "f16")
 
 
+@pytest.mark.parametrize("plan_on", ["device", "host"])
 @pytest.mark.parametrize("name,kw", [("sharing_A", {}), ("sharing_B", {}), ("beam", {"steps": 16})])
-def test_fork_workloads_grouped_every_output(name, kw):
+def test_fork_workloads_grouped_every_output(name, kw, plan_on):
     """The sampling and beam workloads (blocks shared through fork and copy-on-write),
     decoded through the grouped entry point at every attend op."""
     from oracle.replay import OracleReplay
@@ -172,7 +250,7 @@ def test_fork_workloads_grouped_every_output(name, kw):
     import paged_kv_cache_319_b200 as kvp
 
     wl = workloads.by_name(name, **kw)
-    dev = DeviceReplay(wl, "cuda", grouped=True)
+    dev = DeviceReplay(wl, "cuda", grouped=True, plan_on=plan_on)
     dev.run()
     kvp.check_device_error()
     ora = OracleReplay(wl)
