@@ -411,15 +411,21 @@ __global__ void __launch_bounds__(NW * 32) decode_simt_kernel(
 
 // Log-sum-exp merge of the partitions of split sequences: M = max_p m_p,
 // L = sum_p l_p 2^(m_p - M), out = sum_p 2^(m_p - M) acc_p / L.
-// grid (Hq, S), D threads; sequences with a single partition were written by
-// the partition kernel and are skipped, except in the grouped decode, where
-// this kernel writes every row (a row without tokens is zero).
+// grid (ceil(Hq / kReduceHeads), S), kReduceHeads * D threads: a CTA merges
+// kReduceHeads heads of one sequence, thread (i, t) output dim t of head i
+// (few CTAs, so that they are resident, waiting, while the partition kernels
+// run). Sequences with a single partition were written by the partition
+// kernel and are skipped, except in the grouped decode, where this kernel
+// writes every row (a row without tokens is zero).
+constexpr int kReduceHeads = 8;
+
 template <typename T, int D>
-__global__ void __launch_bounds__(D) decode_reduce_kernel(const DecodeArgs a) {
-  extern __shared__ float wsh[];  // [pmax] weights
+__global__ void __launch_bounds__(kReduceHeads * D) decode_reduce_kernel(const DecodeArgs a) {
+  extern __shared__ float wsh[];  // [kReduceHeads][ws_slots] weights, then [kReduceHeads] sums
   pdl_wait();  // launched programmatically: the partition kernel must be complete
-  const int h = blockIdx.x;
+  const int h0 = blockIdx.x * kReduceHeads;
   const int s = blockIdx.y;
+  const int i = threadIdx.x / D, t = threadIdx.x % D;
   const int32_t ctx = load_ctx(a, s, false);
   int32_t nparts;
   if (a.plan) {  // grouped: shared-prefix slots, then the sequence's own
@@ -430,29 +436,29 @@ __global__ void __launch_bounds__(D) decode_reduce_kernel(const DecodeArgs a) {
     nparts = (ctx + a.part_tokens - 1) / a.part_tokens;
     if (nparts <= 1) return;
   }
-  const int64_t row_sh = int64_t(s) * a.num_q_heads + h;
-  const float* ml = a.ws_ml + row_sh * a.ws_slots * 2;
-  __shared__ float red[2];
-  if (threadIdx.x == 0) {
+  const bool head = h0 + i < a.num_q_heads;
+  const int64_t row_sh = int64_t(s) * a.num_q_heads + h0 + i;
+  float* lsh = wsh + kReduceHeads * a.ws_slots;
+  if (head && t == 0) {  // the weights of head h0 + i
+    const float* ml = a.ws_ml + row_sh * a.ws_slots * 2;
     float M = -INFINITY;
     for (int p = 0; p < nparts; ++p) M = fmaxf(M, ml[2 * p]);
     float L = 0.f;
     for (int p = 0; p < nparts; ++p) {
       const float w = (ml[2 * p] == -INFINITY || M == -INFINITY) ? 0.f : exp2f(ml[2 * p] - M);
-      wsh[p] = w;
+      wsh[i * a.ws_slots + p] = w;
       L += ml[2 * p + 1] * w;
     }
-    red[0] = L;
+    lsh[i] = L;
   }
   __syncthreads();
-  const float L = red[0];
+  if (!head) return;
   const float* acc = a.ws_acc + row_sh * a.ws_slots * D;
-  for (int t = threadIdx.x; t < D; t += blockDim.x) {
-    float o = 0.f;
-    for (int p = 0; p < nparts; ++p) o = fmaf(acc[int64_t(p) * D + t], wsh[p], o);
-    const float y = L > 0.f ? o / L : 0.f;
-    static_cast<uint16_t*>(a.out)[row_sh * D + t] = Elem<T>::from_float(y);
-  }
+  float o = 0.f;
+  for (int p = 0; p < nparts; ++p) o = fmaf(acc[int64_t(p) * D + t], wsh[i * a.ws_slots + p], o);
+  const float L = lsh[i];
+  const float y = L > 0.f ? o / L : 0.f;
+  static_cast<uint16_t*>(a.out)[row_sh * D + t] = Elem<T>::from_float(y);
 }
 
 }  // namespace dev

@@ -250,9 +250,17 @@ int launch_reduce(const kvp::dev::DecodeArgs& a, cudaStream_t st) {
   // Programmatic dependent launch: the reduce's launch overlaps the tail of the
   // partition kernel; the kernel itself waits (griddepcontrol.wait) for it.
   cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3(a.num_q_heads, a.num_seqs);
-  cfg.blockDim = dim3(D);
-  cfg.dynamicSmemBytes = size_t(a.ws_slots) * 4;
+  constexpr int HR = kvp::dev::kReduceHeads;
+  const size_t smem = size_t(HR) * (a.ws_slots + 1) * 4;
+  if (smem > 200u * 1024u)
+    return fail(KVP_ERR_INVALID, "decode reduce: %d partitions per sequence is too many", a.ws_slots);
+  if (smem > 48u * 1024u) {
+    cudaError_t e = ensure_smem(kvp::dev::decode_reduce_kernel<T, D>, int(200u * 1024u));
+    if (e != cudaSuccess) return cuda_fail(e, "decode reduce: smem attribute");
+  }
+  cfg.gridDim = dim3((a.num_q_heads + HR - 1) / HR, a.num_seqs);
+  cfg.blockDim = dim3(HR * D);
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
