@@ -92,6 +92,110 @@ struct SimtCfg {
   static_assert(NST >= 1 && NST <= 32, "stages");
 };
 
+// Per-lane shapes of a (block, KV head) tile in the CUDA-core kernels.
+template <int D, int BS>
+struct TileShape {
+  static constexpr int kChunksPerLane = D / 16;  // 16-byte chunks of q / a key row per lane
+  static constexpr int kPasses = (BS + 15) / 16;  // 16 key rows per QK pass
+  static constexpr int kDimsPerLane = D / 32;     // output dims per lane
+};
+
+// Folds one tile of keys and values ([region][row][64], 128-byte swizzled,
+// rows r < nvalid valid) into a warp's online-softmax state (log2 domain):
+// running max m_run, per-lane exponent sum l_lane (lanes 0..15), and the
+// lane's kDimsPerLane output dims acc. qf: the lane's half of q, pre-scaled.
+// QK: two lanes per key row, swizzled 16-byte shared loads, one shuffle; row
+// max by one integer max-reduction; PV: p broadcast by shuffle.
+template <typename T, int D, int BS>
+__device__ __forceinline__ void simt_tile(const uint8_t* kt, const uint8_t* vt, int32_t nvalid,
+                                          const float (&qf)[TileShape<D, BS>::kChunksPerLane * 8],
+                                          float& m_run, float& l_lane,
+                                          float (&acc)[TileShape<D, BS>::kDimsPerLane], int lane) {
+  using TC_ = TileShape<D, BS>;
+  const int part = lane >> 4;
+  // ---- scores: row r = pass * 16 + (lane & 15), half `part` of its chunks
+  float sc[TC_::kPasses];
+#pragma unroll
+  for (int ps = 0; ps < TC_::kPasses; ++ps) {
+    const int r = ps * 16 + (lane & 15);
+    float d0 = 0.f, d1 = 0.f, d2 = 0.f, d3 = 0.f;
+    if (r < BS) {
+#pragma unroll
+      for (int c = 0; c < TC_::kChunksPerLane; ++c) {
+        const int lc = part * TC_::kChunksPerLane + c;
+        const int region = lc >> 3;
+        const int cc = lc & 7;
+        const uint4 kv = *reinterpret_cast<const uint4*>(kt + region * BS * 128 + r * 128 +
+                                                         ((cc ^ (r & 7)) << 4));
+        const float2 f0 = Elem<T>::to_float2(kv.x);
+        const float2 f1 = Elem<T>::to_float2(kv.y);
+        const float2 f2 = Elem<T>::to_float2(kv.z);
+        const float2 f3 = Elem<T>::to_float2(kv.w);
+        d0 = fmaf(qf[c * 8 + 0], f0.x, d0);
+        d1 = fmaf(qf[c * 8 + 1], f0.y, d1);
+        d2 = fmaf(qf[c * 8 + 2], f1.x, d2);
+        d3 = fmaf(qf[c * 8 + 3], f1.y, d3);
+        d0 = fmaf(qf[c * 8 + 4], f2.x, d0);
+        d1 = fmaf(qf[c * 8 + 5], f2.y, d1);
+        d2 = fmaf(qf[c * 8 + 6], f3.x, d2);
+        d3 = fmaf(qf[c * 8 + 7], f3.y, d3);
+      }
+    }
+    float dot = (d0 + d1) + (d2 + d3);
+    dot += __shfl_xor_sync(0xffffffffu, dot, 16);
+    sc[ps] = r < nvalid ? dot : -INFINITY;
+  }
+
+  // ---- online softmax update (log2 domain)
+  float tmax = sc[0];
+#pragma unroll
+  for (int ps = 1; ps < TC_::kPasses; ++ps) tmax = fmaxf(tmax, sc[ps]);
+  tmax = warp_max(tmax);
+  const float m_new = fmaxf(m_run, tmax);
+  const float alpha = m_run == -INFINITY ? 0.f : exp2f(m_run - m_new);
+  float pr[TC_::kPasses];
+  float psum = 0.f;
+#pragma unroll
+  for (int ps = 0; ps < TC_::kPasses; ++ps) {
+    pr[ps] = sc[ps] == -INFINITY ? 0.f : exp2f(sc[ps] - m_new);
+    psum += pr[ps];
+  }
+  l_lane = l_lane * alpha + (lane < 16 ? psum : 0.f);
+#pragma unroll
+  for (int e = 0; e < TC_::kDimsPerLane; ++e) acc[e] *= alpha;
+  m_run = m_new;
+
+  // ---- acc += p V: lane owns dims [lane * kDimsPerLane, +kDimsPerLane)
+  {
+    constexpr int DPL = TC_::kDimsPerLane;
+    const int d0 = lane * DPL;
+    const int region = d0 >> 6;
+    const int cc = (d0 & 63) >> 3;
+    const int pos = d0 & 7;
+#pragma unroll
+    for (int r = 0; r < BS; ++r) {
+      const float pv = __shfl_sync(0xffffffffu, pr[r >> 4], r & 15);
+      if (r < nvalid) {
+        const uint8_t* src = vt + region * BS * 128 + r * 128 + ((cc ^ (r & 7)) << 4) + pos * 2;
+        if constexpr (DPL == 4) {
+          const uint2 v = *reinterpret_cast<const uint2*>(src);
+          const float2 f0 = Elem<T>::to_float2(v.x);
+          const float2 f1 = Elem<T>::to_float2(v.y);
+          acc[0] = fmaf(pv, f0.x, acc[0]);
+          acc[1] = fmaf(pv, f0.y, acc[1]);
+          acc[2] = fmaf(pv, f1.x, acc[2]);
+          acc[3] = fmaf(pv, f1.y, acc[3]);
+        } else {
+          const uint32_t v = *reinterpret_cast<const uint32_t*>(src);
+          const float2 f0 = Elem<T>::to_float2(v);
+          acc[0] = fmaf(pv, f0.x, acc[0]);
+          acc[1] = fmaf(pv, f0.y, acc[1]);
+        }
+      }
+    }
+  }
+}
+
 // PH (per-head warps): grid (partition, ceil(Hq / NW), sequence); warp w takes
 // query head blockIdx.y * NW + w over the whole partition and writes its own
 // partial, with no merge across warps. For short ranges (a few blocks per
@@ -243,87 +347,7 @@ __global__ void __launch_bounds__(NW * 32) decode_simt_kernel(
     const int32_t tok0 = (b0 + wfirst + kStride * i) * BS;
     const int32_t nvalid = min(BS, ctx - tok0);
 
-    // ---- scores: row r = pass * 16 + (lane & 15), half `part` of its chunks
-    float sc[C::kPasses];
-#pragma unroll
-    for (int ps = 0; ps < C::kPasses; ++ps) {
-      const int r = ps * 16 + (lane & 15);
-      float d0 = 0.f, d1 = 0.f, d2 = 0.f, d3 = 0.f;
-      if (r < BS) {
-#pragma unroll
-        for (int c = 0; c < C::kChunksPerLane; ++c) {
-          const int lc = part * C::kChunksPerLane + c;
-          const int region = lc >> 3;
-          const int cc = lc & 7;
-          const uint4 kv = *reinterpret_cast<const uint4*>(kt + region * BS * 128 + r * 128 +
-                                                           ((cc ^ (r & 7)) << 4));
-          const float2 f0 = Elem<T>::to_float2(kv.x);
-          const float2 f1 = Elem<T>::to_float2(kv.y);
-          const float2 f2 = Elem<T>::to_float2(kv.z);
-          const float2 f3 = Elem<T>::to_float2(kv.w);
-          d0 = fmaf(qf[c * 8 + 0], f0.x, d0);
-          d1 = fmaf(qf[c * 8 + 1], f0.y, d1);
-          d2 = fmaf(qf[c * 8 + 2], f1.x, d2);
-          d3 = fmaf(qf[c * 8 + 3], f1.y, d3);
-          d0 = fmaf(qf[c * 8 + 4], f2.x, d0);
-          d1 = fmaf(qf[c * 8 + 5], f2.y, d1);
-          d2 = fmaf(qf[c * 8 + 6], f3.x, d2);
-          d3 = fmaf(qf[c * 8 + 7], f3.y, d3);
-        }
-      }
-      float dot = (d0 + d1) + (d2 + d3);
-      dot += __shfl_xor_sync(0xffffffffu, dot, 16);
-      sc[ps] = r < nvalid ? dot : -INFINITY;
-    }
-
-    // ---- online softmax update (log2 domain)
-    float tmax = sc[0];
-#pragma unroll
-    for (int ps = 1; ps < C::kPasses; ++ps) tmax = fmaxf(tmax, sc[ps]);
-    tmax = warp_max(tmax);
-    const float m_new = fmaxf(m_run, tmax);
-    const float alpha = m_run == -INFINITY ? 0.f : exp2f(m_run - m_new);
-    float pr[C::kPasses];
-    float psum = 0.f;
-#pragma unroll
-    for (int ps = 0; ps < C::kPasses; ++ps) {
-      pr[ps] = sc[ps] == -INFINITY ? 0.f : exp2f(sc[ps] - m_new);
-      psum += pr[ps];
-    }
-    l_lane = l_lane * alpha + (lane < 16 ? psum : 0.f);
-#pragma unroll
-    for (int e = 0; e < C::kDimsPerLane; ++e) acc[e] *= alpha;
-    m_run = m_new;
-
-    // ---- acc += p V: lane owns dims [lane * kDimsPerLane, +kDimsPerLane)
-    {
-      constexpr int DPL = C::kDimsPerLane;
-      const int d0 = lane * DPL;
-      const int region = d0 >> 6;
-      const int cc = (d0 & 63) >> 3;
-      const int pos = d0 & 7;
-#pragma unroll
-      for (int r = 0; r < BS; ++r) {
-        const float pv = __shfl_sync(0xffffffffu, pr[r >> 4], r & 15);
-        if (r < nvalid) {
-          const uint8_t* src = vt + region * BS * 128 + r * 128 + ((cc ^ (r & 7)) << 4) + pos * 2;
-          if constexpr (DPL == 4) {
-            const uint2 v = *reinterpret_cast<const uint2*>(src);
-            const float2 f0 = Elem<T>::to_float2(v.x);
-            const float2 f1 = Elem<T>::to_float2(v.y);
-            acc[0] = fmaf(pv, f0.x, acc[0]);
-            acc[1] = fmaf(pv, f0.y, acc[1]);
-            acc[2] = fmaf(pv, f1.x, acc[2]);
-            acc[3] = fmaf(pv, f1.y, acc[3]);
-          } else {
-            const uint32_t v = *reinterpret_cast<const uint32_t*>(src);
-            const float2 f0 = Elem<T>::to_float2(v);
-            acc[0] = fmaf(pv, f0.x, acc[0]);
-            acc[1] = fmaf(pv, f0.y, acc[1]);
-          }
-        }
-      }
-    }
+    simt_tile<T, D, BS>(kt, vt, nvalid, qf, m_run, l_lane, acc, lane);
 
     // ---- refill this stage with block i + NST
     const int32_t nxt = i + NST;
@@ -417,7 +441,10 @@ __global__ void __launch_bounds__(NW * 32) decode_simt_kernel(
 // run). Sequences with a single partition were written by the partition
 // kernel and are skipped, except in the grouped decode, where this kernel
 // writes every row (a row without tokens is zero).
-constexpr int kReduceHeads = 8;
+#ifndef KVP_REDUCE_HEADS
+#define KVP_REDUCE_HEADS 4
+#endif
+constexpr int kReduceHeads = KVP_REDUCE_HEADS;
 
 template <typename T, int D>
 __global__ void __launch_bounds__(kReduceHeads * D) decode_reduce_kernel(const DecodeArgs a) {

@@ -491,11 +491,10 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
     };
     // Shared-prefix units (grouped decode): column j of Q is query head
     // g * G + j % G of member j / G. The warp loads a unit's rows into
-    // registers one iteration ahead and stores them, when the unit starts, in
-    // the 128-byte-swizzled layout a TMA load would produce (16-byte chunk c of
-    // row j at (c ^ (j & 7)) * 16): before the unit's key tiles and so before
-    // the previous unit's value tiles, since the MMA needs this Q before it
-    // frees the ring stages those wait for.
+    // registers one iteration ahead and stores them in the 128-byte-swizzled
+    // layout a TMA load would produce (16-byte chunk c of row j at
+    // (c ^ (j & 7)) * 16) before the previous unit's value tiles, since the MMA
+    // needs this Q before it frees the ring stages those wait for.
     constexpr int kQChunksPerLane = kN * 16 / 32;
     auto is_gather = [&](const tc::ChunkStream<GRP, BS>& cs) {
       return GRP && cs.valid && cs.first() && cs.w.sg >= 0;
@@ -533,12 +532,19 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
       const bool gather_next = is_gather(nxt);
       if (gather_next) gather_q(nxt, qn);
       const int32_t row = id_row(cur, id);
-      if (cur.first()) {
+      const int32_t nt = cur.tiles();
+      // A unit's Q goes in before its key tiles when a TMA load brings it, and
+      // right after them when the warp stores gathered rows (their loads then
+      // overlap the key tiles' issue); either way before the previous unit's
+      // value tiles.
+      const bool gather = is_gather(cur);
+      if (gather) load_tiles(&kmap, row, nt, false);
+      if (cur.first() && ok) {
         const uint32_t qb = ucnt & 1u;
         if (lane == 0) ok = mbar_wait(&q_empty[qb], ((ucnt >> 1) & 1u) ^ 1u, 0x7100u);
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) break;
-        if (is_gather(cur)) {
+        if (gather) {
           uint8_t* qdst = qbuf + qb * kQBytes;
 #pragma unroll
           for (int i = 0; i < kQChunksPerLane; ++i) {
@@ -558,8 +564,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
         }
         ++ucnt;
       }
-      const int32_t nt = cur.tiles();
-      load_tiles(&kmap, row, nt, false);
+      if (!gather && ok) load_tiles(&kmap, row, nt, false);
       if (have_pend && ok) load_tiles(&vmap, pend_row, pend_tiles, true);
       pend_row = row;
       pend_tiles = nt;
