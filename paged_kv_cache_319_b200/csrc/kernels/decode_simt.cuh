@@ -459,6 +459,10 @@ __global__ void __launch_bounds__(kReduceHeads * D) decode_reduce_kernel(const D
     const int32_t shared = a.plan[kPlanSeqWord + s] * (a.part_tokens / a.part_blocks);
     nparts = (shared + a.part_tokens - 1) / a.part_tokens +
              (ctx > shared ? (ctx - shared + a.part_tokens - 1) / a.part_tokens : 0);
+    if (nparts > a.ws_slots) {  // a prefix longer than the context: a plan of other tables
+      if (threadIdx.x == 0 && blockIdx.x == 0) record_error(KVP_DEVERR_CTX, uint64_t(s));
+      nparts = a.ws_slots;
+    }
   } else {
     nparts = (ctx + a.part_tokens - 1) / a.part_tokens;
     if (nparts <= 1) return;

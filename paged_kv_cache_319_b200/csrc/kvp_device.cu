@@ -15,6 +15,7 @@
 #include <cstring>
 #include <mutex>
 #include <unordered_map>
+#include <vector>
 
 #include "kernels/cache_ops.cuh"
 #include "kernels/common.cuh"
@@ -371,6 +372,40 @@ int tc_dispatch(int bs, int G, const CUtensorMap& km, const CUtensorMap& vm, con
   return launch_tc<T, 32, 16>(km, vm, qm, a, st);
 }
 
+// A caller's grouping plan, checked word by word before any kernel reads it:
+// counts in range, every index inside the batch and every shared prefix inside
+// the block tables, members distinct and in one subgroup each, per-sequence
+// prefixes equal to their subgroup's, and the header's partition counts. (A
+// plan built from other tables that passes still gives wrong results; only
+// its shape is checked.)
+bool host_plan_fits(const int32_t* plan, int32_t S, int32_t MB, int32_t max_ctx, int32_t bs,
+                    int32_t part, int mmax, int32_t pmax) {
+  namespace g = kvp::grp;
+  const int32_t n_sub = plan[g::kNumSub], psh = plan[g::kSharedParts], pown = plan[g::kOwnParts];
+  if (n_sub < 0 || n_sub > S / 2 || psh < 0 || psh > pmax || pown < 0 || pown > pmax ||
+      plan[g::kSharedBlocks] < 0 || plan[g::kOwnBlocks] < 0)
+    return false;
+  const int32_t cap = max_ctx / bs;  // a shared prefix is made of full blocks
+  const int32_t* cblk = plan + g::kHdrWords;
+  const int32_t* subs = plan + g::sub_offset(S);
+  std::vector<int32_t> owner(size_t(S), -1);
+  int32_t most = 0;
+  for (int32_t i = 0; i < n_sub; ++i) {
+    const int32_t* e = subs + int64_t(i) * g::kSubWords;
+    const int32_t c = e[0], nm = e[1];
+    if (c < 1 || c > cap || c > MB || nm < 2 || nm > mmax) return false;
+    most = std::max(most, (c * bs + part - 1) / part);
+    for (int m = 0; m < nm; ++m) {
+      const int32_t s = e[4 + m];
+      if (s < 0 || s >= S || owner[size_t(s)] >= 0 || cblk[s] != c) return false;
+      owner[size_t(s)] = i;
+    }
+  }
+  for (int32_t s = 0; s < S; ++s)
+    if (owner[size_t(s)] < 0 && cblk[s] != 0) return false;
+  return most == psh;
+}
+
 // Argument checks of the decode entry points (fn names the caller in the
 // messages); *empty is set when there is nothing to do (no sequences).
 int check_decode(const char* fn, const void* q, const void* k_cache, const void* v_cache,
@@ -661,8 +696,8 @@ int paged_attention_decode_grouped(const void* q, const void* k_cache, const voi
     const int32_t n_sub = host_plan[g::kNumSub], psh = host_plan[g::kSharedParts];
     const int32_t pown = host_plan[g::kOwnParts];
     const int32_t sblk = host_plan[g::kSharedBlocks], oblk = host_plan[g::kOwnBlocks];
-    if (n_sub < 0 || n_sub > num_seqs / 2 || psh < 0 || psh > pmax || pown < 0 || pown > pmax ||
-        sblk < 0 || oblk < 0)
+    if (!host_plan_fits(host_plan, num_seqs, max_blocks_per_seq, max_context_len, block_size,
+                        partition_size, mmax, pmax))
       return fail(KVP_ERR_INVALID, "paged_attention_decode_grouped: host_plan does not fit this batch");
     if (!device_plan) {
       cudaError_t e = cudaMemcpyAsync(plan, host_plan, size_t(g::plan_words(num_seqs)) * 4,

@@ -201,18 +201,38 @@ def test_reused_workspace_two_batches_in_a_row():
             check_close(got, oracle(q, k, v, t, l, "f16", 0.09, 16), "f16")
 
 
-def test_host_plan_of_another_batch_is_rejected():
+def test_malformed_host_plans_are_rejected():
+    """Every index and count of a caller's plan is checked on the host before a kernel reads it."""
     import torch
     import paged_kv_cache_319_b200 as kvp
     from paged_kv_cache_319_b200._lib import KvpError
 
     q, k, v, t, l = shared_batch(3, [(4, [100, 120]), (0, [30])], 8, 8, 128, 16, "f16")
     plan = host_plan(t, l, 8, 8, 16, 512, k.shape[0])
-    bad = plan.copy()
-    bad[0] = 99  # more subgroups than the batch can have
-    with pytest.raises(KvpError) as e:
-        run(q, k, v, t, l, "f16", 0.09, 512, grouped=True, plan=bad)
-    assert e.value.kind == "invalid"
+    S = len(l)
+    sub0 = 8 + S  # first subgroup entry
+    assert plan[0] == 1 and plan[sub0 + 1] == 2
+    members = plan[sub0 + 4:sub0 + 6].tolist()
+    other = next(x for x in range(S) if x not in members)
+
+    def corrupt(fn):
+        bad = plan.copy()
+        fn(bad)
+        return bad
+
+    malformed = [
+        corrupt(lambda b: b.__setitem__(0, 99)),                 # more subgroups than the batch holds
+        corrupt(lambda b: b.__setitem__(sub0 + 4, S)),           # member index outside the batch
+        corrupt(lambda b: b.__setitem__(sub0 + 5, members[0])),  # a member twice
+        corrupt(lambda b: b.__setitem__(sub0, 500)),             # prefix past every table
+        corrupt(lambda b: b.__setitem__(8 + other, 3)),          # a prefix for a sequence in no subgroup
+        corrupt(lambda b: b.__setitem__(sub0 + 1, 17)),          # more members than columns
+        corrupt(lambda b: b.__setitem__(1, 2)),                  # shared partition count off
+    ]
+    for bad in malformed:
+        with pytest.raises(KvpError) as e:
+            run(q, k, v, t, l, "f16", 0.09, 512, grouped=True, plan=bad)
+        assert e.value.kind == "invalid"
     # a device copy without the host plan it copies is rejected too
     with pytest.raises(KvpError) as e:
         kvp.paged_attention_decode(
