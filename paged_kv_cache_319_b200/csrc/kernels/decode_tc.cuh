@@ -533,12 +533,9 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
       if (gather_next) gather_q(nxt, qn);
       const int32_t row = id_row(cur, id);
       const int32_t nt = cur.tiles();
-      // A unit's Q goes in before its key tiles when a TMA load brings it, and
-      // right after them when the warp stores gathered rows (their loads then
-      // overlap the key tiles' issue); either way before the previous unit's
-      // value tiles.
+      // A unit's Q goes in before its key tiles (gathered rows were loaded an
+      // iteration ago), so the MMA can start on the first key tile that lands.
       const bool gather = is_gather(cur);
-      if (gather) load_tiles(&kmap, row, nt, false);
       if (cur.first() && ok) {
         const uint32_t qb = ucnt & 1u;
         if (lane == 0) ok = mbar_wait(&q_empty[qb], ((ucnt >> 1) & 1u) ^ 1u, 0x7100u);
@@ -564,7 +561,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
         }
         ++ucnt;
       }
-      if (!gather && ok) load_tiles(&kmap, row, nt, false);
+      if (ok) load_tiles(&kmap, row, nt, false);
       if (have_pend && ok) load_tiles(&vmap, pend_row, pend_tiles, true);
       pend_row = row;
       pend_tiles = nt;

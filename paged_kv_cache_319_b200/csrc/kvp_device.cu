@@ -54,6 +54,13 @@ using kvp::fail;
 #ifndef KVP_GROUP_PER_HEAD_BELOW
 #define KVP_GROUP_PER_HEAD_BELOW 4
 #endif
+// Warps and stages of the CUDA-core kernel on longer own ranges.
+#ifndef KVP_GROUP_SPLIT_WARPS
+#define KVP_GROUP_SPLIT_WARPS KVP_SIMT_WARPS
+#endif
+#ifndef KVP_GROUP_SPLIT_STAGES
+#define KVP_GROUP_SPLIT_STAGES KVP_SIMT_STAGES
+#endif
 
 namespace {
 
@@ -342,7 +349,7 @@ int launch_own_ranges(int bs, int32_t dtype, bool per_head, const CUtensorMap& k
                       bool programmatic, int grid_x) {
   using H = __half;
   using B = __nv_bfloat16;
-  constexpr int W = KVP_SIMT_WARPS, N = KVP_SIMT_STAGES;
+  constexpr int W = KVP_GROUP_SPLIT_WARPS, N = KVP_GROUP_SPLIT_STAGES;
   const bool f16 = dtype == KVP_F16;
   if (per_head) {
     if (bs == 16)
