@@ -85,6 +85,39 @@ def paged_decode(q: np.ndarray, k_cache: np.ndarray, v_cache: np.ndarray, block_
     return out
 
 
+def paged_prefill(q: np.ndarray, k_cache: np.ndarray, v_cache: np.ndarray, block_tables,
+                  context_lens, scale: float, block_size: int, dtype=None) -> np.ndarray:
+    """Attention of a chunk of ``T`` new tokens per sequence over the paged cache,
+    causal within the chunk: the prefill of a prompt, or a chunk of it, whose keys
+    and values are already in the sequence's blocks ("PagedAttention: KV cache
+    memory management", section "A request lifecycle": prefill creates the
+    cache state through the block table). Reading (the pages leave it open): query
+    ``i`` of sequence ``s`` sits at position ``ctx_s - T + i`` and attends to the
+    tokens ``j <= ctx_s - T + i``, where ``context_lens[s]`` counts the chunk; a
+    query with no such token (``ctx_s < T - i``) gives a zero row.
+
+    ``q``: float64 ``[S, T, Hq, D]``; caches and ``dtype`` as for
+    :func:`paged_decode`; returns float64 ``[S, T, Hq, D]``.
+    """
+    S, T, Hq, D = q.shape
+    Hkv = k_cache.shape[1]
+    if Hq % Hkv:
+        raise ValueError("num_q_heads must be a multiple of num_kv_heads")
+    G = Hq // Hkv
+    out = np.zeros((S, T, Hq, D), dtype=np.float64)
+    for s in range(S):
+        ctx = int(context_lens[s])
+        for g in range(Hkv):
+            K = _rows(k_cache, block_tables[s], ctx, g, block_size, dtype)
+            V = _rows(v_cache, block_tables[s], ctx, g, block_size, dtype)
+            for i in range(T):
+                vis = ctx - T + i + 1
+                if vis > 0:
+                    out[s, i, g * G:(g + 1) * G] = attend(q[s, i, g * G:(g + 1) * G], K[:vis], V[:vis],
+                                                          scale)
+    return out
+
+
 def partition_partials(q: np.ndarray, K: np.ndarray, V: np.ndarray, scale: float,
                        partition_size: int):
     """Per-partition ``(m_p, l_p, acc_p)`` for one query row over contiguous K/V."""

@@ -230,3 +230,76 @@ def test_bf16_decoding():
     assert to_f64(bits, "bf16").tolist() == [1.0, -2.0, 0.5, 2.0**-126]
     bits = np.array([0x3C00, 0xC000, 0x3800, 0x0400], np.uint16)
     assert to_f64(bits, "f16").tolist() == [1.0, -2.0, 0.5, 2.0**-14]
+
+
+# ---- paged prefill (a chunk of T new tokens per sequence, causal within the chunk)
+
+def _prefill_batch(seed, lens, T, Hq=4, Hkv=2, D=16, bs=4):
+    rng = np.random.default_rng(seed)
+    need = [-(-L // bs) for L in lens]
+    nb = sum(need) + 3
+    perm = rng.permutation(nb)
+    tables = np.full((len(lens), max(need)), -1, np.int64)
+    i = 0
+    for s, n in enumerate(need):
+        tables[s, :n] = perm[i:i + n]
+        i += n
+    k = rng.standard_normal((nb, Hkv, bs, D))
+    v = rng.standard_normal((nb, Hkv, bs, D))
+    q = rng.standard_normal((len(lens), T, Hq, D))
+    return q, k, v, tables, np.asarray(lens)
+
+
+def test_prefill_of_one_token_is_decode():
+    q, k, v, t, l = _prefill_batch(1, [5, 17, 9], T=1)
+    a = attention.paged_prefill(q, k, v, t, l, 0.3, 4)
+    b = attention.paged_decode(q[:, 0], k, v, t, l, 0.3, 4)
+    assert np.array_equal(a[:, 0], b)
+
+
+def test_prefill_rows_are_the_decodes_of_their_prefixes():
+    """Query i of a chunk attends exactly what a decode step at length ctx - T + i + 1 would."""
+    T = 6
+    q, k, v, t, l = _prefill_batch(2, [6, 11, 23], T=T)
+    out = attention.paged_prefill(q, k, v, t, l, 0.25, 4)
+    for i in range(T):
+        lens_i = l - T + i + 1
+        ref = attention.paged_decode(q[:, i], k, v, t, lens_i, 0.25, 4)
+        assert np.allclose(out[:, i], ref, atol=1e-12, rtol=0)
+
+
+def test_prefill_matches_sdpa_with_an_explicit_causal_mask():
+    """torch fp64 scaled_dot_product_attention on the gathered contiguous K/V, with the
+    bottom-right causal mask (query i at position L - T + i) built as a boolean matrix."""
+    torch = pytest.importorskip("torch")
+    T, Hq, Hkv = 5, 4, 2
+    q, k, v, t, l = _prefill_batch(3, [5, 9, 20], T=T, Hq=Hq, Hkv=Hkv)
+    out = attention.paged_prefill(q, k, v, t, l, 0.2, 4)
+    for s, L in enumerate(l):
+        for g in range(Hkv):
+            K = torch.from_numpy(attention.gather(k, t[s], L, g, 4))
+            V = torch.from_numpy(attention.gather(v, t[s], L, g, 4))
+            mask = torch.arange(L)[None, :] <= (L - T + torch.arange(T))[:, None]
+            for hh in range(g * (Hq // Hkv), (g + 1) * (Hq // Hkv)):
+                Q = torch.from_numpy(q[s, :, hh])
+                ref = torch.nn.functional.scaled_dot_product_attention(
+                    Q[None], K[None], V[None], attn_mask=mask[None], scale=0.2)[0].numpy()
+                assert np.allclose(out[s, :, hh], ref, atol=1e-12, rtol=0)
+
+
+def test_prefill_closed_forms():
+    """A whole prompt (ctx = T): row 0 is v_0 exactly; zero queries give the mean of the
+    visible values, a different mean for every row; queries with no visible token give 0."""
+    T = 7
+    q, k, v, t, l = _prefill_batch(4, [7, 3], T=T, Hq=2, Hkv=2)
+    out = attention.paged_prefill(q, k, v, t, l, 0.5, 4)
+    V0 = attention.gather(v, t[0], 7, 0, 4)
+    assert np.array_equal(out[0, 0, 0], V0[0])
+    qz = np.zeros_like(q)
+    outz = attention.paged_prefill(qz, k, v, t, l, 0.5, 4)
+    for i in range(T):
+        assert np.allclose(outz[0, i, 0], V0[:i + 1].mean(axis=0), atol=1e-13)
+    # sequence 1 holds 3 tokens but the chunk has 7: queries 0..3 see nothing
+    assert not outz[1, :4].any()
+    V1 = attention.gather(v, t[1], 3, 1, 4)
+    assert np.allclose(outz[1, 6, 1], V1.mean(axis=0), atol=1e-13)
