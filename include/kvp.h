@@ -348,6 +348,39 @@ KVP_API int kv_decode_group_plan(const int32_t* block_tables, const int32_t* con
                          int32_t num_kv_heads, int32_t num_blocks, int32_t* plan,
                          size_t plan_words);
 
+/* Bytes of device workspace paged_attention_prefill needs: that of
+ * paged_attention_decode for num_seqs * q_len rows (0 if q_len <= 0). */
+KVP_API size_t kvp_prefill_workspace_bytes(int32_t num_seqs, int32_t q_len, int32_t num_q_heads,
+                                   int32_t head_dim, int32_t max_context_len,
+                                   int32_t partition_size);
+
+/* Attention of a chunk of q_len new tokens per sequence over the paged cache,
+ * causal within the chunk: the prefill of a prompt (or of a chunk of it)
+ * whose keys and values reshape_and_cache has already written to the
+ * sequence's blocks ["PagedAttention: KV cache memory management", section "A
+ * request lifecycle": prefill creates the cache state through the block
+ * table]. context_lens[s] counts the chunk; query i of sequence s sits at
+ * position ctx_s - q_len + i and attends to the tokens j <= ctx_s - q_len + i
+ * (a query with none gives a zero row):
+ *   out[s][i][h] = sum_j softmax_j(scale * q[s][i][h] . key j) * value j.
+ * q, out: device [num_seqs][q_len][num_q_heads][head_dim]; the other arguments
+ * as for paged_attention_decode (context_lens[s] <= max_context_len).
+ * q_len == 1 is paged_attention_decode. Longer chunks run on the tensor
+ * cores, up to 16 / G queries of every sequence per launch (G = num_q_heads /
+ * num_kv_heads), each launch reading the sequences' keys and values once, so
+ * a whole prompt of T tokens reads them ceil(T * G / 16) times; needs head_dim
+ * 128, block_size 16 or 32, G <= 16, partition_size a multiple of 128 (or 0).
+ * workspace: >= kvp_prefill_workspace_bytes(...) bytes, 256-byte aligned.
+ * Errors: those of paged_attention_decode. */
+KVP_API int paged_attention_prefill(const void* q, const void* k_cache, const void* v_cache,
+                            const int32_t* block_tables, const int32_t* context_lens,
+                            int32_t num_seqs, int32_t q_len, int32_t num_q_heads,
+                            int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                            int32_t num_blocks, int32_t max_blocks_per_seq,
+                            int32_t max_context_len, float scale, int32_t partition_size,
+                            void* workspace, size_t workspace_bytes, void* out, int32_t dtype,
+                            kvp_stream_t stream);
+
 /* Largest split-context scratch, in bytes, that paged_attention_decode_noalloc
  * can serve from its built-in area (40 MiB). */
 #define KVP_STATIC_SCRATCH_BYTES (40u * 1024u * 1024u)

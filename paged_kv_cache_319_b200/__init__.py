@@ -21,6 +21,7 @@ from ._lib import (KVP_BF16, KVP_F16, KvpError, P_i32, P_i64, PoolStats, check, 
 
 __all__ = [
     "BlockPool", "KvpError", "reshape_and_cache", "copy_blocks", "paged_attention_decode",
+    "paged_attention_prefill",
     "decode_workspace_bytes", "decode_grouped_workspace_bytes", "group_plan", "check_device_error",
     "kv_bytes_per_token", "version",
     "KVP_F16", "KVP_BF16",
@@ -312,6 +313,45 @@ def paged_attention_decode(q, k_cache, v_cache, block_tables, context_lens, scal
         check(lib().paged_attention_decode_grouped(*args))
     else:
         check(lib().paged_attention_decode(*args))
+    return out
+
+
+def paged_attention_prefill(q, k_cache, v_cache, block_tables, context_lens, scale: float,
+                            out=None, *, max_context_len: int | None = None,
+                            partition_size: int = 0, workspace=None):
+    """Attention of a chunk of T new tokens per sequence, causal within the chunk;
+    ``q [S, T, Hq, D]`` (dtype of the cache), returns ``out`` of the same shape.
+    ``context_lens[s]`` counts the chunk, whose K/V must already be in the cache."""
+    torch = _torch()
+    dev = _cuda(q, k_cache, v_cache, block_tables, context_lens)
+    if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32:
+        raise TypeError("block_tables and context_lens must be int32")
+    S, T, Hq, D = q.shape
+    NB, Hkv, bs, D2 = k_cache.shape
+    if D2 != D or v_cache.shape != k_cache.shape or q.dtype != k_cache.dtype:
+        raise ValueError("q / cache mismatch")
+    MB = block_tables.shape[1] if block_tables.dim() == 2 else 0
+    if block_tables.shape[0] != S or context_lens.shape != (S,):
+        raise ValueError("batch metadata mismatch")
+    mcl = MB * bs if max_context_len is None else int(max_context_len)
+    if out is None:
+        out = torch.empty_like(q)
+    else:
+        _cuda(out)
+        if out.shape != q.shape or out.dtype != q.dtype:
+            raise ValueError("out mismatch")
+    need = int(lib().kvp_prefill_workspace_bytes(S, T, Hq, D, mcl, partition_size))
+    ws_ptr, ws_bytes = None, 0
+    if need:
+        if workspace is None:
+            workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+        _cuda(workspace)
+        ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()
+    check(lib().paged_attention_prefill(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
+                                        block_tables.data_ptr(), context_lens.data_ptr(), S, T,
+                                        Hq, Hkv, D, bs, NB, max(MB, 1), mcl, float(scale),
+                                        int(partition_size), ws_ptr, ws_bytes, out.data_ptr(),
+                                        _code(q), _stream(dev)))
     return out
 
 

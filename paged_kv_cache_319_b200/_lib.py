@@ -76,6 +76,9 @@ SIGNATURES = {
     "paged_attention_decode_grouped": (C.c_int, [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,
                                                  i32, i32, f32, i32, vp, vp, vp, sz, vp, i32, vp]),
     "kvp_decode_group_plan_words": (sz, [i32]),
+    "kvp_prefill_workspace_bytes": (sz, [i32, i32, i32, i32, i32, i32]),
+    "paged_attention_prefill": (C.c_int, [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32,
+                                          i32, i32, f32, i32, vp, sz, vp, i32, vp]),
     "kv_decode_group_plan": (C.c_int, [P_i32, P_i32, i32, i32, i32, i32, i32, i32, i32, i32, P_i32,
                                        sz]),
     "paged_attention_decode_noalloc": (C.c_int, [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,

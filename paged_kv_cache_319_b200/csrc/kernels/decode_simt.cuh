@@ -53,6 +53,9 @@ struct DecodeArgs {
   int32_t pmax;         // partitions per (sequence, head) in the grid
   int32_t ws_slots;     // partial slots per (sequence, head) in the workspace
   float scale_log2;     // scale * log2(e)
+  // Multi-query (prefill) chunks: q and out hold q_len rows per sequence; a
+  // launch takes queries [q_first, q_first + q_count) of each. Decode: 1, 0, 1.
+  int32_t q_len, q_first, q_count;
   // Grouped decode only (null otherwise): the grouping plan of
   // decode_group.cuh. Every (sequence, head) then has ceil(c * bs / P) slots
   // for its shared prefix followed by the slots of its own range, and the
@@ -435,8 +438,9 @@ __global__ void __launch_bounds__(NW * 32) decode_simt_kernel(
 
 // Log-sum-exp merge of the partitions of split sequences: M = max_p m_p,
 // L = sum_p l_p 2^(m_p - M), out = sum_p 2^(m_p - M) acc_p / L.
-// grid (ceil(Hq / kReduceHeads), S), kReduceHeads * D threads: a CTA merges
-// kReduceHeads heads of one sequence, thread (i, t) output dim t of head i
+// grid (ceil(Hq / kReduceHeads), S * q_len), kReduceHeads * D threads: a CTA
+// merges kReduceHeads heads of one row (a sequence, or one query row of a
+// multi-query chunk), thread (i, t) output dim t of head i
 // (few CTAs, so that they are resident, waiting, while the partition kernels
 // run). Sequences with a single partition were written by the partition
 // kernel and are skipped, except in the grouped decode, where this kernel
@@ -451,7 +455,8 @@ __global__ void __launch_bounds__(kReduceHeads * D) decode_reduce_kernel(const D
   extern __shared__ float wsh[];  // [kReduceHeads][ws_slots] weights, then [kReduceHeads] sums
   pdl_wait();  // launched programmatically: the partition kernel must be complete
   const int h0 = blockIdx.x * kReduceHeads;
-  const int s = blockIdx.y;
+  const int row = blockIdx.y;          // a sequence, or one of its q_len query rows
+  const int s = row / a.q_len;
   const int i = threadIdx.x / D, t = threadIdx.x % D;
   const int32_t ctx = load_ctx(a, s, false);
   int32_t nparts;
@@ -468,7 +473,7 @@ __global__ void __launch_bounds__(kReduceHeads * D) decode_reduce_kernel(const D
     if (nparts <= 1) return;
   }
   const bool head = h0 + i < a.num_q_heads;
-  const int64_t row_sh = int64_t(s) * a.num_q_heads + h0 + i;
+  const int64_t row_sh = int64_t(row) * a.num_q_heads + h0 + i;
   float* lsh = wsh + kReduceHeads * a.ws_slots;
   if (head && t == 0) {  // the weights of head h0 + i
     const float* ml = a.ws_ml + row_sh * a.ws_slots * 2;

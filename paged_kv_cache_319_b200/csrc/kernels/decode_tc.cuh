@@ -48,6 +48,8 @@ static_assert(grp::kHdrWords == kPlanSeqWord, "plan layout");
 
 namespace tc {
 
+enum Mode : int { kPlain = 0, kGrouped = 1, kMultiQuery = 2 };
+
 constexpr int kD = 128;             // head_dim
 constexpr int kN = 16;              // MMA N (query heads of a group, padded)
 constexpr int kTileTok = 128;       // MMA M: tokens per tile
@@ -306,15 +308,21 @@ struct ChunkStream {
 
 }  // namespace tc
 
-// GRP: grouped decode (a.plan set; launched after the plan kernel with
-// programmatic serialisation). num_units then counts the per-sequence units
-// (0 when the CUDA-core kernel takes them); the shared-prefix units are read
-// from the plan.
-template <typename T, int BS, int NG, bool GRP>
+// MODE tc::kPlain: decode. MODE tc::kGrouped: grouped decode (a.plan set;
+// launched after the plan kernel with programmatic serialisation); num_units
+// then counts the per-sequence units (0 when the CUDA-core kernel takes them)
+// and the shared-prefix units are read from the plan. MODE tc::kMultiQuery:
+// a chunk of a.q_count query tokens per sequence (tokens a.q_first.. of an
+// a.q_len-token chunk, rows s * q_len + i of q and out), causal within the
+// chunk: column j is query a.q_first + j / G at head g * G + j % G and sees
+// the tokens before ctx - q_len + q_first + j / G + 1.
+template <typename T, int BS, int NG, int MODE>
 __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
     const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
     const __grid_constant__ CUtensorMap qmap, const DecodeArgs a, int64_t num_units) {
   using namespace tc;
+  constexpr bool GRP = MODE == kGrouped;
+  constexpr bool MQ = MODE == kMultiQuery;
   static_assert(BS == 16 || BS == 32, "block_size 16 or 32");
   using L = tc::Cfg<NG>;
   constexpr int kStages = L::kStages;
@@ -497,20 +505,21 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
     // needs this Q before it frees the ring stages those wait for.
     constexpr int kQChunksPerLane = kN * 16 / 32;
     auto is_gather = [&](const tc::ChunkStream<GRP, BS>& cs) {
-      return GRP && cs.valid && cs.first() && cs.w.sg >= 0;
+      return cs.valid && cs.first() && ((GRP && cs.w.sg >= 0) || MQ);
     };
     auto gather_q = [&](const tc::ChunkStream<GRP, BS>& cs, uint4 (&v)[kQChunksPerLane]) {
-      const int32_t* e = tc::sub_entry(gh, cs.w.sg);
-      const int32_t ncol = tc::plan_at(gh, e + 1) * G;
+      const int32_t* e = GRP ? tc::sub_entry(gh, cs.w.sg) : nullptr;
+      const int32_t ncol = GRP ? tc::plan_at(gh, e + 1) * G : a.q_count * G;
 #pragma unroll
       for (int i = 0; i < kQChunksPerLane; ++i) {
         const int idx = lane + 32 * i;
         const int j = idx >> 4, ch = idx & 15;
         v[i] = make_uint4(0, 0, 0, 0);
         if (j < ncol) {
-          const int32_t m = j / G;
-          const int64_t qrow =
-              int64_t(tc::plan_at(gh, e + 4 + m)) * a.num_q_heads + cs.w.g * G + (j - m * G);
+          const int32_t m = j / G;  // member (grouped) or query token (multi-query)
+          const int64_t seq_row = GRP ? int64_t(tc::plan_at(gh, e + 4 + m))
+                                      : int64_t(cs.w.s) * a.q_len + a.q_first + m;
+          const int64_t qrow = seq_row * a.num_q_heads + cs.w.g * G + (j - m * G);
           v[i] = __ldg(reinterpret_cast<const uint4*>(static_cast<const T*>(a.q) + qrow * kD) + ch);
         }
       }
@@ -711,13 +720,20 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
     auto wait_all = [&](uint64_t* bar, uint32_t parity, uint32_t where) {
       return __all_sync(0xffffffffu, mbar_wait(bar, parity, where)) != 0;
     };
+    int32_t col_q[NG];  // multi-query: the query token of column j within the launch
+#pragma unroll
+    for (int j = 0; j < NG; ++j) col_q[j] = j / G;
     // Units without tokens (context length 0) attend to nothing: zero rows
     // (written by the reduce in the grouped decode).
     for (int64_t u = blockIdx.x; !GRP && u < num_units; u += gridDim.x) {
       tc::Unit w;
       if (!tc::decode_unit(a, u, w, ctx_sm) || tc::chunks_of(w) > 0) continue;
-      for (int j = 0; j < G; ++j)
-        static_cast<uint16_t*>(a.out)[(int64_t(w.s) * a.num_q_heads + w.g * G + j) * kD + r] = 0;
+      const int32_t nq = MQ ? a.q_count : 1;
+      for (int i = 0; i < nq; ++i) {
+        const int64_t row = MQ ? int64_t(w.s) * a.q_len + a.q_first + i : int64_t(w.s);
+        for (int j = 0; j < G; ++j)
+          static_cast<uint16_t*>(a.out)[(row * a.num_q_heads + w.g * G + j) * kD + r] = 0;
+      }
     }
     float acc[NG], m_run[NG], l_thr[NG];
 #pragma unroll
@@ -773,7 +789,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
       const int32_t h0 = pw.g * G;
       // grouped decode: a shared-prefix unit's columns are its members' heads
       const int32_t* ge = (GRP && pw.sg >= 0) ? tc::sub_entry(gh, pw.sg) : nullptr;
-      const int32_t ncol = ge ? tc::plan_at(gh, ge + 1) * G : G;
+      const int32_t ncol = ge ? tc::plan_at(gh, ge + 1) * G : (MQ ? a.q_count * G : G);
 #pragma unroll
       for (int j = 0; j < NG; ++j) {
         const float Lj = (rl[j] + rl[kN + j]) + (rl[2 * kN + j] + rl[3 * kN + j]);
@@ -782,6 +798,9 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
           if (ge) {
             const int32_t m = j / G;
             row_sh = int64_t(tc::plan_at(gh, ge + 4 + m)) * a.num_q_heads + h0 + (j - m * G);
+          } else if (MQ) {
+            const int32_t i = col_q[j];
+            row_sh = (int64_t(pw.s) * a.q_len + a.q_first + i) * a.num_q_heads + h0 + (j - i * G);
           }
           if (!GRP && pw.nparts <= 1) {
             const float y = Lj > 0.f ? acc[j] / Lj : 0.f;
@@ -829,12 +848,16 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
       float cmax[NG];
 #pragma unroll
       for (int j = 0; j < NG; ++j) cmax[j] = -INFINITY;
+      // multi-query: column j sees the tokens before lim0 + j / G
+      const int32_t lim0 = MQ ? cur.w.ctx - a.q_len + a.q_first + 1 : 0;
 #pragma unroll
       for (int t = 0; t < kChunkTiles; ++t) {
-        const bool valid = t < ntile && ctok0 + t * kTileTok + r < ctok1;
+        const int32_t tok = ctok0 + t * kTileTok + r;
+        const bool valid = t < ntile && tok < ctok1;
 #pragma unroll
         for (int j = 0; j < NG; ++j) {
-          sv[t][j] = valid ? sv[t][j] * a.scale_log2 : -INFINITY;
+          const bool vis = valid && (!MQ || tok < lim0 + col_q[j]);
+          sv[t][j] = vis ? sv[t][j] * a.scale_log2 : -INFINITY;
           cmax[j] = fmaxf(cmax[j], sv[t][j]);
         }
       }

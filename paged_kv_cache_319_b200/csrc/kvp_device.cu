@@ -239,7 +239,7 @@ int launch_simt(const CUtensorMap& km, const CUtensorMap& vm, const kvp::dev::De
 template <typename T, int BS, int NG>
 int launch_tc(const CUtensorMap& km, const CUtensorMap& vm, const CUtensorMap& qm,
               const kvp::dev::DecodeArgs& a, cudaStream_t st) {
-  auto k = kvp::dev::decode_tc_kernel<T, BS, NG, false>;
+  auto k = kvp::dev::decode_tc_kernel<T, BS, NG, kvp::dev::tc::kPlain>;
   // context lengths of small batches are cached in shared memory
   using Cfg = kvp::dev::tc::Cfg<NG>;
   const int ctx_bytes = a.num_seqs <= Cfg::kCtxCap ? 4 * a.num_seqs : 0;
@@ -266,7 +266,7 @@ int launch_reduce(const kvp::dev::DecodeArgs& a, cudaStream_t st) {
     cudaError_t e = ensure_smem(kvp::dev::decode_reduce_kernel<T, D>, int(200u * 1024u));
     if (e != cudaSuccess) return cuda_fail(e, "decode reduce: smem attribute");
   }
-  cfg.gridDim = dim3((a.num_q_heads + HR - 1) / HR, a.num_seqs);
+  cfg.gridDim = dim3((a.num_q_heads + HR - 1) / HR, a.num_seqs * a.q_len);
   cfg.blockDim = dim3(HR * D);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
@@ -302,7 +302,7 @@ template <typename T, int BS, int NG>
 int launch_tc_grouped(const CUtensorMap& km, const CUtensorMap& vm, const CUtensorMap& qm,
                       const kvp::dev::DecodeArgs& a, cudaStream_t st, bool with_private,
                       int grid_ctas, bool programmatic) {
-  auto k = kvp::dev::decode_tc_kernel<T, BS, NG, true>;
+  auto k = kvp::dev::decode_tc_kernel<T, BS, NG, kvp::dev::tc::kGrouped>;
   using Cfg = kvp::dev::tc::Cfg<NG>;
   // shared-memory tail: context lengths, per-sequence prefix blocks and the
   // subgroup table when they fit (S <= kPlanCap), else the context lengths alone
@@ -363,6 +363,32 @@ int launch_own_ranges(int bs, int32_t dtype, bool per_head, const CUtensorMap& k
                : launch_simt<B, 128, 16, W, N>(km, vm, a, st, programmatic, grid_x);
   return f16 ? launch_simt<H, 128, 32, W, N>(km, vm, a, st, programmatic, grid_x)
              : launch_simt<B, 128, 32, W, N>(km, vm, a, st, programmatic, grid_x);
+}
+
+// Multi-query (prefill) chunk on the tensor cores: one launch per a.q_count
+// queries of every sequence.
+template <typename T, int BS, int NG>
+int launch_tc_mq(const CUtensorMap& km, const CUtensorMap& vm, const CUtensorMap& qm,
+                 const kvp::dev::DecodeArgs& a, cudaStream_t st) {
+  auto k = kvp::dev::decode_tc_kernel<T, BS, NG, kvp::dev::tc::kMultiQuery>;
+  using Cfg = kvp::dev::tc::Cfg<NG>;
+  const int ctx_bytes = a.num_seqs <= Cfg::kCtxCap ? 4 * a.num_seqs : 0;
+  cudaError_t e = ensure_smem(k, Cfg::kSmemBytes + 4 * Cfg::kCtxCap);
+  if (e != cudaSuccess) return cuda_fail(e, "prefill (tensor cores): smem attribute");
+  const int64_t units = int64_t(a.num_seqs) * a.num_kv_heads * a.pmax;
+  const int grid = int(units < sm_count() ? units : sm_count());
+  k<<<grid, kvp::dev::tc::kThreads, Cfg::kSmemBytes + ctx_bytes, st>>>(km, vm, qm, a, units);
+  e = cudaGetLastError();
+  return e == cudaSuccess ? KVP_OK : cuda_fail(e, "prefill (tensor cores): launch");
+}
+
+template <typename T>
+int tc_mq_dispatch(int bs, int ng, const CUtensorMap& km, const CUtensorMap& vm,
+                   const CUtensorMap& qm, const kvp::dev::DecodeArgs& a, cudaStream_t st) {
+  if (bs == 16) return ng == 8 ? launch_tc_mq<T, 16, 8>(km, vm, qm, a, st)
+                               : launch_tc_mq<T, 16, 16>(km, vm, qm, a, st);
+  return ng == 8 ? launch_tc_mq<T, 32, 8>(km, vm, qm, a, st)
+                 : launch_tc_mq<T, 32, 16>(km, vm, qm, a, st);
 }
 
 template <typename T>
@@ -564,6 +590,9 @@ int paged_attention_decode(const void* q, const void* k_cache, const void* v_cac
   a.pmax = pmax;
   a.ws_slots = pmax;
   a.scale_log2 = scale * 1.4426950408889634f;
+  a.q_len = 1;
+  a.q_first = 0;
+  a.q_count = 1;
 
   const uint64_t rows = uint64_t(num_blocks) * num_kv_heads * block_size;
   CUtensorMap km, vm;
@@ -601,6 +630,98 @@ int paged_attention_decode(const void* q, const void* k_cache, const void* v_cac
   if (head_dim == 128)
     return dtype == KVP_F16 ? launch_reduce<__half, 128>(a, st) : launch_reduce<__nv_bfloat16, 128>(a, st);
   return dtype == KVP_F16 ? launch_reduce<__half, 64>(a, st) : launch_reduce<__nv_bfloat16, 64>(a, st);
+}
+
+size_t kvp_prefill_workspace_bytes(int32_t num_seqs, int32_t q_len, int32_t num_q_heads,
+                                   int32_t head_dim, int32_t max_context_len,
+                                   int32_t partition_size) {
+  if (q_len <= 0 || num_seqs <= 0 || int64_t(num_seqs) * q_len > 0x7FFFFFFF) return 0;
+  return kvp_decode_workspace_bytes(num_seqs * q_len, num_q_heads, head_dim, max_context_len,
+                                    partition_size);
+}
+
+int paged_attention_prefill(const void* q, const void* k_cache, const void* v_cache,
+                            const int32_t* block_tables, const int32_t* context_lens,
+                            int32_t num_seqs, int32_t q_len, int32_t num_q_heads,
+                            int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                            int32_t num_blocks, int32_t max_blocks_per_seq,
+                            int32_t max_context_len, float scale, int32_t partition_size,
+                            void* workspace, size_t workspace_bytes, void* out, int32_t dtype,
+                            kvp_stream_t stream) {
+  bool empty = false;
+  const int crc = check_decode("paged_attention_prefill", q, k_cache, v_cache, block_tables,
+                               context_lens, num_seqs, num_q_heads, num_kv_heads, head_dim,
+                               block_size, num_blocks, max_blocks_per_seq, max_context_len, scale,
+                               partition_size, out, dtype, &empty);
+  if (crc || empty) return crc;
+  if (q_len < 1 || int64_t(num_seqs) * q_len > 0x7FFFFFFF)
+    return fail(KVP_ERR_INVALID, "paged_attention_prefill: bad q_len");
+  if (q_len == 1)
+    return paged_attention_decode(q, k_cache, v_cache, block_tables, context_lens, num_seqs,
+                                  num_q_heads, num_kv_heads, head_dim, block_size, num_blocks,
+                                  max_blocks_per_seq, max_context_len, scale, partition_size,
+                                  workspace, workspace_bytes, out, dtype, stream);
+  const int G = num_q_heads / num_kv_heads;
+  if (head_dim != 128 || (block_size != 16 && block_size != 32) || G > 16)
+    return fail(KVP_ERR_INVALID,
+                "paged_attention_prefill: needs head_dim 128, block_size 16 or 32, and at most 16 "
+                "query heads per KV head");
+  if (partition_size % 128)
+    return fail(KVP_ERR_INVALID, "paged_attention_prefill: partition_size must be a multiple of 128");
+  const int32_t ctx_cap = max_context_len > 0 ? max_context_len : 1;
+  int32_t part_tokens, pmax;
+  if (partition_size > 0) {
+    part_tokens = partition_size;
+    pmax = (ctx_cap + partition_size - 1) / partition_size;
+  } else {
+    part_tokens = ((ctx_cap + block_size - 1) / block_size) * block_size;
+    pmax = 1;
+  }
+  const Workspace wl = ws_layout(int64_t(num_seqs) * q_len, num_q_heads, head_dim, pmax);
+  if (wl.total) {
+    if (!workspace || workspace_bytes < wl.total)
+      return fail(KVP_ERR_INVALID, "paged_attention_prefill: workspace of %zu bytes needed", wl.total);
+    if (!aligned(workspace, 256)) return fail(KVP_ERR_INVALID, "paged_attention_prefill: workspace not 256-byte aligned");
+  }
+  kvp::dev::DecodeArgs a{};
+  a.q = q;
+  a.out = out;
+  a.block_tables = block_tables;
+  a.context_lens = context_lens;
+  a.ws_ml = wl.total ? static_cast<float*>(workspace) : nullptr;
+  a.ws_acc = wl.total ? reinterpret_cast<float*>(static_cast<char*>(workspace) + wl.ml_bytes) : nullptr;
+  a.num_seqs = num_seqs;
+  a.num_q_heads = num_q_heads;
+  a.num_kv_heads = num_kv_heads;
+  a.num_blocks = num_blocks;
+  a.max_blocks_per_seq = max_blocks_per_seq;
+  a.max_context_len = max_context_len;
+  a.part_blocks = part_tokens / block_size;
+  a.part_tokens = part_tokens;
+  a.pmax = pmax;
+  a.ws_slots = pmax;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.q_len = q_len;
+  const uint64_t rows = uint64_t(num_blocks) * num_kv_heads * block_size;
+  CUtensorMap km, vm, qm;
+  int rc = make_map(&km, k_cache, dtype, rows, head_dim, block_size);
+  if (!rc) rc = make_map_halves(&vm, v_cache, dtype, rows, block_size);
+  if (!rc)
+    rc = make_map(&qm, q, dtype, uint64_t(num_seqs) * q_len * num_q_heads, head_dim, kvp::dev::tc::kN);
+  if (rc) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // up to 16 columns per launch: 16 / G query tokens of every sequence
+  const int per_launch = std::max(1, kvp::dev::tc::kN / G);
+  for (int32_t c0 = 0; c0 < q_len; c0 += per_launch) {
+    a.q_first = c0;
+    a.q_count = std::min(per_launch, q_len - c0);
+    const int ng = a.q_count * G <= 8 ? 8 : 16;
+    rc = dtype == KVP_F16 ? tc_mq_dispatch<__half>(block_size, ng, km, vm, qm, a, st)
+                          : tc_mq_dispatch<__nv_bfloat16>(block_size, ng, km, vm, qm, a, st);
+    if (rc) return rc;
+  }
+  if (pmax <= 1) return KVP_OK;
+  return dtype == KVP_F16 ? launch_reduce<__half, 128>(a, st) : launch_reduce<__nv_bfloat16, 128>(a, st);
 }
 
 size_t kvp_decode_grouped_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, int32_t head_dim,
@@ -674,6 +795,9 @@ int paged_attention_decode_grouped(const void* q, const void* k_cache, const voi
   a.pmax = pmax;
   a.ws_slots = pmax + 1;
   a.scale_log2 = scale * 1.4426950408889634f;
+  a.q_len = 1;
+  a.q_first = 0;
+  a.q_count = 1;
   a.plan = plan;
 
   // One query head per KV head: the CUDA-core kernel takes the sequences' own
