@@ -760,6 +760,106 @@ def run_schedule(args):
     print(json.dumps(res), flush=True)
 
 
+# Paged prefill workloads: a chunk of T new tokens per sequence, causal within
+# the chunk, over a pool already holding every context (chunk included).
+PREFILL_WORKLOADS = {
+    "prefill_opt13b_t16": ("opt13b", 16),        # OPT-13B batch, 16-token chunks
+    "prefill_gqa_bs16_t4": ("gqa_long_bs16", 4),  # long-context GQA, 4-token chunks
+    "prefill_prompt512": ("prompt512", 512),     # 64 whole prompts of 512 tokens
+}
+
+
+def run_prefill(args):
+    """paged_attention_prefill, timed with CUDA events (median of --steps calls, L2
+    flushed before each); roofline on algorithmic bytes: K/V of every context token
+    read once, q, out, block tables and lengths."""
+    import torch
+    import paged_kv_cache_319_b200 as kvp
+
+    device = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(device)
+    base, T = PREFILL_WORKLOADS[args.workload]
+    if base == "prompt512":
+        g = workloads.Geometry(40, 40, 128, 16, "f16")
+        lens = np.full(64, 512, np.int64)
+        part, desc = 512, "OPT-13B geometry, 64 prompts of 512 tokens prefilled whole (ctx = T = 512)"
+    else:
+        wl = workloads.by_name(base)
+        g = wl.geometry
+        lens = np.asarray(wl.info["context_lens"], np.int64)
+        part, desc = wl.partition_size, f"{wl.description}; a chunk of the last {T} tokens per sequence"
+    S, Hq, Hkv, D, bs = len(lens), g.num_q_heads, g.num_kv_heads, g.head_dim, g.block_size
+    rng = np.random.default_rng(3001)
+    need = -(-lens // bs)
+    NB = int(need.sum()) + 8
+    perm = rng.permutation(NB).astype(np.int32)
+    tables = np.full((S, int(need.max())), -1, np.int32)
+    i = 0
+    for s_, n in enumerate(need):
+        tables[s_, :n] = perm[i:i + n]
+        i += n
+    tdt = torch.float16 if g.dtype == "f16" else torch.bfloat16
+    gen = torch.Generator(device=device).manual_seed(3002)
+    k = torch.randn((NB, Hkv, bs, D), generator=gen, device=device, dtype=torch.float32).to(tdt)
+    v = torch.randn((NB, Hkv, bs, D), generator=gen, device=device, dtype=torch.float32).to(tdt)
+    q = torch.randn((S, T, Hq, D), generator=gen, device=device, dtype=torch.float32).to(tdt)
+    tt = torch.from_numpy(tables).to(device)
+    cl = torch.from_numpy(lens.astype(np.int32)).to(device)
+    mcl = int(lens.max())
+    out = torch.empty_like(q)
+    ws = torch.empty(max(1, kvp.lib().kvp_prefill_workspace_bytes(S, T, Hq, D, mcl, part)),
+                     dtype=torch.uint8, device=device)
+    call = lambda: kvp.paged_attention_prefill(q, k, v, tt, cl, 1 / math.sqrt(D), out,  # noqa: E731
+                                               max_context_len=mcl, partition_size=part,
+                                               workspace=ws)
+    for _ in range(max(3, args.warmup)):
+        call()
+    kvp.check_device_error(device)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    clean = torch.ones(256 << 20, dtype=torch.uint8, device=device)
+    pairs = []
+    with ClockSampler(device) as clk:
+        for _ in range(max(1, args.steps)):
+            flush.fill_(1)
+            clean.amax()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            call()
+            e1.record()
+            pairs.append((e0, e1))
+        torch.cuda.synchronize(device)
+    ms = float(np.median([a.elapsed_time(b) for a, b in pairs]))
+    kv = float(lens.sum()) * Hkv * D * g.elem_bytes * 2
+    alg = kv + S * T * Hq * D * g.elem_bytes * 2 + 4 * float(need.sum()) + 4 * S
+    G = Hq // Hkv
+    launches = -(-T // max(1, 16 // G)) if T > 1 else 1
+    vis = np.clip(lens[:, None] - T + np.arange(T)[None, :] + 1, 0, None)  # visible tokens per query
+    flops = 4.0 * float(vis.sum()) * D * Hq
+    peak, peak_kind = peaks()
+    achieved = alg / (ms * 1e-3) / 1e9
+    res = {
+        "metric": METRIC, "value": round(achieved, 2), "unit": UNIT, "n_gpus": 1,
+        "steps": len(pairs), "warmup": max(3, args.warmup), "ms_per_step": round(ms, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": g.dtype,
+        "data": "synthetic (seeded normal q/K/V on the device)",
+        "config": {"workload": desc, "name": args.workload, "chunk_tokens": T,
+                   "launches_per_call": launches, "partition_size": part,
+                   "timed": f"paged_attention_prefill (median of {len(pairs)} calls, L2 "
+                            "flushed before each)"},
+        "query_tokens_per_s": round(S * T / (ms * 1e-3), 1),
+        "attention_tflops": round(flops / (ms * 1e-3) / 1e12, 2),
+        "roofline": {"kernel": "paged_attention_prefill: decode_tc (multi-query) + decode_reduce_kernel",
+                     "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
+                     "peak_source": peak_kind, "unit": "GB/s", "frac": round(achieved / peak, 4),
+                     "algorithmic_bytes_per_launch": int(alg),
+                     "note": f"algorithmic bytes count the keys and values once per call; "
+                             f"each of the call's {launches} launch(es) reads the contexts again",
+                     "avg_launch_us": round(ms * 1e3, 2)},
+        "clocks": clk.summary(),
+    }
+    print(json.dumps(res), flush=True)
+
+
 def run_reference(args, world, rank):
     """The oracle as the reference arm: each step is a bounded sample of the workload."""
     if rank != 0:
@@ -808,7 +908,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="opt13b",
                     choices=["opt13b", "gqa_long_bs16", "gqa_long_bs32", "llama13b_churn",
-                             "sharing_A", "sharing_B", "beam"])
+                             "sharing_A", "sharing_B", "beam"] + list(PREFILL_WORKLOADS))
     ap.add_argument("--partition", type=int, default=None)
     ap.add_argument("--num-seqs", type=int, default=None,
                     help="smaller batch of the same workload (profiling small cases)")
@@ -819,7 +919,7 @@ def main():
                     help="decode entry point of the schedule workloads (auto: grouped for "
                          "the sampling and beam workloads)")
     args = ap.parse_args()
-    if args.warmup < 3 and args.workload not in SCHEDULE_WORKLOADS:
+    if args.warmup < 3 and args.workload not in SCHEDULE_WORKLOADS + tuple(PREFILL_WORKLOADS):
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
         # The oracle needs no GPU and no process group: rank 0 runs, the others exit.
@@ -828,6 +928,9 @@ def main():
         return
     if args.workload in SCHEDULE_WORKLOADS:
         run_schedule(args)
+        return
+    if args.workload in PREFILL_WORKLOADS:
+        run_prefill(args)
         return
     world, rank, local = dist_setup()
     try:
