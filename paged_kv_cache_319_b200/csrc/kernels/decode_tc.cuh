@@ -75,8 +75,13 @@ constexpr int kCtxCacheMax = 4096;
 
 // Layout for a group width NG (query heads per KV head, padded to 4, 8 or 16).
 // P^T holds p split into a high part and a low part, both in the input type
-// (rows [0, NG) and [NG, 2 NG)): the PV MMA multiplies V by hi + lo, which
+// (columns [0, NG) and [NG, 2 NG)): the PV MMA multiplies V by hi + lo, which
 // carries p to about 16 significant bits instead of the 8 of one bf16.
+// P^T is the MMA's B operand in the MN-major layout without swizzle: the 8
+// columns [8g, 8g + 8) of a token are 16 contiguous bytes, tokens follow each
+// other every 16 bytes, and column groups are kPSbo bytes apart. A softmax
+// thread owns one token, so it writes its columns with 16-byte stores, and a
+// warp's 32 tokens fill 512 contiguous bytes.
 template <int NG>
 struct Cfg {
   static constexpr int kNPV = 2 * NG <= 16 ? 16 : 32;  // N of the PV MMA
@@ -86,7 +91,7 @@ struct Cfg {
   // groups of 16 need a P^T twice as wide, which costs one stage
   static constexpr int kStages = NG <= 8 ? KVP_TC_STAGES : KVP_TC_STAGES - 1;
   static constexpr int kPBytes = kChunkTok * kNPV * 2;
-  static constexpr int kPLbo = kNPV * 16;               // bytes between 8-token groups of P^T
+  static constexpr int kPSbo = kChunkTok * 16;          // bytes between 8-column groups of P^T
   static constexpr int kOffRing = 0;
   static constexpr int kOffQ = kOffRing + kStages * kStageBytes;
   static constexpr int kOffP = kOffQ + 2 * kQBytes;
@@ -333,7 +338,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
   // A = K (K-major), B = Q (K-major), N = 16
   constexpr uint32_t kIdescQK = idesc_f16(kFmt, 0, 0, kN);
   // A = V^T (MN-major), B = P^T (K-major, hi and lo rows), N = kNPV
-  constexpr uint32_t kIdescPV = idesc_f16(kFmt, 1, 0, kNPV);
+  constexpr uint32_t kIdescPV = idesc_f16(kFmt, 1, 1, kNPV);
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align_1024(smem_raw);
@@ -655,12 +660,12 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
           const uint32_t v_addr = smem_u32(ring + st * kStageBytes);
 #pragma unroll
           for (int kk = 0; kk < kTileTok / 16; ++kk) {
-            const uint32_t pk = (t * kTileTok + kk * 16) / 8 * L::kPLbo;
+            const uint32_t pk = (t * kTileTok + kk * 16) * 16;
             // V^T, MN-major: tokens kk*16.. of block (kk*16)/BS; the two 64-dim
             // halves BS*128 bytes apart (LBO), 8-token groups 1024 apart (SBO)
             const uint32_t va = v_addr + ((kk * 16) / BS) * (BS * 256) + ((kk * 16) % BS) * 128;
             umma_f16_ss(o_tmem, smem_desc(va, BS * 128, 1024, kLayoutSw128),
-                        smem_desc(p_addr + pk, L::kPLbo, 128, kLayoutNone), kIdescPV,
+                        smem_desc(p_addr + pk, 128, L::kPSbo, kLayoutNone), kIdescPV,
                         (t > 0 || kk > 0) ? 1u : 0u);
           }
           umma_commit(&empty[st]);
@@ -885,17 +890,35 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
       for (int t = 0; t < kChunkTiles; ++t) {
         if (t < ntile) {
           const int tok = t * kTileTok + r;  // token within the chunk
-          uint8_t* prow = pbuf_b + (tok >> 3) * L::kPLbo + (tok & 7) * 2;
+          uint8_t* prow = pbuf_b + tok * 16;
+          // p of columns [j0, j0 + 2n) as packed hi and lo pairs
+          auto p_pairs = [&](int j0, uint32_t* hw, uint32_t* lw, int n) {
 #pragma unroll
-          for (int j = 0; j < NG; ++j) {
-            const float pf = sv[t][j] == -INFINITY ? 0.f : exp2f(sv[t][j] - cmax[j]);
-            const uint16_t hi = Elem<T>::from_float(pf);
-            const float hf = Elem<T>::to_float2(uint32_t(hi)).x;
-            const uint16_t lo = Elem<T>::from_float(pf - hf);
-            psum[j] += hf + Elem<T>::to_float2(uint32_t(lo)).x;
-            const int jl = NG + j;
-            *reinterpret_cast<uint16_t*>(prow + (j >> 3) * 128 + (j & 7) * 16) = hi;
-            *reinterpret_cast<uint16_t*>(prow + (jl >> 3) * 128 + (jl & 7) * 16) = lo;
+            for (int i = 0; i < n; ++i) {
+              const int j = j0 + 2 * i;
+              const float p0 = sv[t][j] == -INFINITY ? 0.f : exp2f(sv[t][j] - cmax[j]);
+              const float p1 = sv[t][j + 1] == -INFINITY ? 0.f : exp2f(sv[t][j + 1] - cmax[j + 1]);
+              hw[i] = Elem<T>::pack2(p0, p1);
+              const float2 hf = Elem<T>::to_float2(hw[i]);
+              lw[i] = Elem<T>::pack2(p0 - hf.x, p1 - hf.y);
+              const float2 lf = Elem<T>::to_float2(lw[i]);
+              psum[j] += hf.x + lf.x;
+              psum[j + 1] += hf.y + lf.y;
+            }
+          };
+          if constexpr (NG == 4) {  // hi and lo share one 8-column group
+            uint32_t hw[2], lw[2];
+            p_pairs(0, hw, lw, 2);
+            *reinterpret_cast<uint4*>(prow) = make_uint4(hw[0], hw[1], lw[0], lw[1]);
+          } else {
+#pragma unroll
+            for (int g = 0; g < NG / 8; ++g) {
+              uint32_t hw[4], lw[4];
+              p_pairs(8 * g, hw, lw, 4);
+              *reinterpret_cast<uint4*>(prow + g * L::kPSbo) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+              *reinterpret_cast<uint4*>(prow + (NG / 8 + g) * L::kPSbo) =
+                  make_uint4(lw[0], lw[1], lw[2], lw[3]);
+            }
           }
         }
       }
