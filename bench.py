@@ -712,8 +712,9 @@ def run_schedule(args):
     reps = max(1, args.steps) if n_att == 1 else 1
     rp = DeviceReplay(wl, device, keep_outputs=False, time_decode=True, grouped=grouped,
                       time_reps=reps)
-    rp.run()
-    torch.cuda.synchronize(device)
+    with ClockSampler(device) as clk:
+        rp.run()
+        torch.cuda.synchronize(device)
     kvp.check_device_error(device)
     attends = {i: (t, l) for (i, _, t, l) in rp.attends}
     per_op = {}
@@ -731,7 +732,9 @@ def run_schedule(args):
     toks = np.array([r[3] for r in timed], dtype=np.float64)
     peak, peak_kind = peaks()
     if grouped:
-        kernel = "paged_attention_decode_grouped: group_plan_kernel + decode_tc (grouped)"
+        kernel = ("paged_attention_decode_grouped (plan built on the host): decode_tc (grouped, "
+                  "shared prefixes) + " + ("decode_tc (own ranges)" if g.num_q_heads > g.num_kv_heads
+                                           else "decode_simt (own ranges)"))
     else:
         kernel = "paged_attention_decode: " + (
             "decode_tc" if g.num_q_heads > g.num_kv_heads else "decode_simt")
@@ -756,6 +759,7 @@ def run_schedule(args):
                      "unique_bytes_per_launch": int(uniq.mean()),
                      "logical_bytes_per_launch": int(logical.mean())},
         "pool": {k: int(v) for k, v in st.items()},
+        "clocks": clk.summary(),
     }
     print(json.dumps(res), flush=True)
 
