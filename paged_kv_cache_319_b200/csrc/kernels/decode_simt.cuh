@@ -470,7 +470,11 @@ __global__ void __launch_bounds__(kReduceHeads * D) decode_reduce_kernel(const D
     }
   } else {
     nparts = (ctx + a.part_tokens - 1) / a.part_tokens;
-    if (nparts <= 1) return;
+    if (nparts <= 1) return;  // pass 1 wrote the output
+    if (a.q_len > 1) {  // query row i of a chunk sees ctx - q_len + i + 1 tokens
+      const int32_t vis = min(ctx, max(0, ctx - a.q_len + row % a.q_len + 1));
+      nparts = (vis + a.part_tokens - 1) / a.part_tokens;
+    }
   }
   const bool head = h0 + i < a.num_q_heads;
   const int64_t row_sh = int64_t(row) * a.num_q_heads + h0 + i;

@@ -113,6 +113,15 @@ struct Cfg {
   static_assert(kOCol + 2 * kNPV <= kTmemCols, "tensor memory budget");
 };
 
+// 2^x by the PTX instruction ex2.approx.ftz.f32. For p = 2^(s - m) with
+// s <= m, flushing a subnormal result to zero drops only weights below 2^-126
+// of the chunk's largest, far under the resolution of p in fp16 or bf16.
+__device__ __forceinline__ float ex2_ftz(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // tcgen05 instruction descriptor, kind::f16, fp32 accumulate, M = 128.
 __host__ __device__ constexpr uint32_t idesc_f16(uint32_t ab_fmt, uint32_t a_mn, uint32_t b_mn,
                                                  uint32_t n) {
@@ -198,6 +207,11 @@ __device__ __forceinline__ bool decode_unit(const DecodeArgs& a, int64_t u, Unit
   if (w.p > 0 && w.p >= w.nparts) return false;  // empty (p == 0 always runs)
   w.tok_begin = w.p * a.part_tokens;
   w.tok_end = min(w.ctx, w.tok_begin + a.part_tokens);
+  if (a.q_len > 1) {  // multi-query: no query of the launch sees a token from vis_end on
+    const int32_t vis_end = w.ctx - a.q_len + a.q_first + a.q_count;
+    if (w.tok_end > vis_end) w.tok_end = vis_end;
+    if (w.p > 0 && w.tok_end <= w.tok_begin) return false;
+  }
   if (w.tok_end < w.tok_begin) w.tok_end = w.tok_begin;
   w.sg = -1;
   w.slot = w.p;
@@ -896,8 +910,8 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
 #pragma unroll
             for (int i = 0; i < n; ++i) {
               const int j = j0 + 2 * i;
-              const float p0 = sv[t][j] == -INFINITY ? 0.f : exp2f(sv[t][j] - cmax[j]);
-              const float p1 = sv[t][j + 1] == -INFINITY ? 0.f : exp2f(sv[t][j + 1] - cmax[j + 1]);
+              const float p0 = sv[t][j] == -INFINITY ? 0.f : ex2_ftz(sv[t][j] - cmax[j]);
+              const float p1 = sv[t][j + 1] == -INFINITY ? 0.f : ex2_ftz(sv[t][j + 1] - cmax[j + 1]);
               hw[i] = Elem<T>::pack2(p0, p1);
               const float2 hf = Elem<T>::to_float2(hw[i]);
               lw[i] = Elem<T>::pack2(p0 - hf.x, p1 - hf.y);

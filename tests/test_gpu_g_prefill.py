@@ -4,7 +4,8 @@ The cases cover chunks that fit one launch (T * G <= 16 columns) and chunks cut
 into several launches (a whole prompt), sequences holding fewer tokens than
 the chunk (their first queries see nothing), a whole prompt (ctx == T),
 grouped-query heads (G = 4 and 16), block sizes 16 and 32, split and unsplit
-partitions, and T = 1 (the decode path).
+partitions, launches that stop at the last token their queries see, and T = 1
+(the decode path).
 """
 
 import math
@@ -41,6 +42,12 @@ CASES = [
     (16, 4, 16, [9, 300, 1200], 10, "bf16", 0),          # 4 + 4 + 2, unsplit, ctx 9 < T
     (16, 1, 32, [50, 700], 3, "bf16", 256),              # G = 16: one query per launch
     (8, 8, 16, [1, 33, 900], 1, "f16", 512),             # T = 1: decode
+    # 13 launches; each reads only the tokens its last query sees, and the
+    # reduce merges each row's visible partitions: ctx 150 < T with two
+    # partitions (the first 50 rows see nothing), partition boundaries inside
+    # the launches' ranges
+    (4, 4, 16, [150, 300, 700], 200, "f16", 128),
+    (16, 4, 32, [90, 520, 1000], 24, "bf16", 128),       # G = 4: 6 launches of 4 queries
 ]
 
 
