@@ -872,6 +872,125 @@ def run_prefill(args):
     print(json.dumps(res), flush=True)
 
 
+FP8_WORKLOADS = ("opt13b_fp8",)
+
+
+def run_fp8(args):
+    """paged_attention_decode_fp8 on the OPT-13B batch with an E4M3 cache, timed with
+    CUDA events (median of --steps calls, L2 flushed before each), beside the 16-bit
+    decode of the same batch; roofline on the E4M3 algorithmic bytes."""
+    import torch
+    import paged_kv_cache_319_b200 as kvp
+
+    device = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(device)
+    wl = workloads.by_name("opt13b")
+    g = wl.geometry
+    lens = np.asarray(wl.info["context_lens"], np.int64)
+    S, Hq, Hkv, D, bs, part = len(lens), g.num_q_heads, g.num_kv_heads, g.head_dim, g.block_size, 512
+    rng = np.random.default_rng(4001)
+    need = -(-lens // bs)
+    NB = int(np.ceil(1.25 * need.sum()))
+    perm = rng.permutation(NB).astype(np.int32)
+    tables = np.full((S, int(need.max())), -1, np.int32)
+    i = 0
+    for s_, n in enumerate(need):
+        tables[s_, :n] = perm[i:i + n]
+        i += n
+    gen = torch.Generator(device=device).manual_seed(4002)
+
+    def codes():  # uniform E4M3 codes without the two NaN codes
+        c = torch.randint(0, 256, (NB, Hkv, bs, D), generator=gen, device=device, dtype=torch.uint8)
+        return torch.where((c & 0x7F) == 0x7F, c & 0xBF, c)
+
+    kc, vc = codes(), codes()
+    ks = torch.linspace(1 / 448, 2 / 448, Hkv, device=device, dtype=torch.float32)
+    vs = torch.linspace(1 / 448, 4 / 448, Hkv, device=device, dtype=torch.float32)
+    q = torch.randn((S, Hq, D), generator=gen, device=device, dtype=torch.float32).half()
+    tt = torch.from_numpy(tables).to(device)
+    cl = torch.from_numpy(lens.astype(np.int32)).to(device)
+    mcl = int(lens.max())
+    out = torch.empty_like(q)
+    ws = torch.empty(max(1, kvp.decode_workspace_bytes(S, Hq, D, mcl, part)), dtype=torch.uint8,
+                     device=device)
+    scale = 1 / math.sqrt(D)
+    call = lambda: kvp.paged_attention_decode_fp8(q, kc, vc, ks, vs, tt, cl, scale, out,  # noqa: E731
+                                                  max_context_len=mcl, partition_size=part,
+                                                  workspace=ws)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    clean = torch.ones(256 << 20, dtype=torch.uint8, device=device)
+
+    def timed(fn, n):
+        pairs = []
+        for _ in range(n):
+            flush.fill_(1)
+            clean.amax()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            pairs.append((e0, e1))
+        torch.cuda.synchronize(device)
+        return float(np.median([a.elapsed_time(b) for a, b in pairs]))
+
+    for _ in range(max(3, args.warmup)):
+        call()
+    kvp.check_device_error(device)
+    steps = max(1, args.steps)
+    with ClockSampler(device) as clk:
+        ms = timed(call, steps)
+    # the new token of every sequence, quantised into the cache (one decode step's scatter)
+    kn = torch.randn((S, Hkv, D), generator=gen, device=device, dtype=torch.float32).half()
+    vn = torch.randn((S, Hkv, D), generator=gen, device=device, dtype=torch.float32).half()
+    slots = torch.from_numpy((tables[np.arange(S), (lens - 1) // bs].astype(np.int64) * bs
+                              + (lens - 1) % bs)).to(device)
+    scatter = lambda: kvp.reshape_and_cache_fp8(kn, vn, kc, vc, slots, ks, vs)  # noqa: E731
+    for _ in range(3):
+        scatter()
+    scatter_ms = timed(scatter, steps)
+    kvp.check_device_error(device)
+    # the 16-bit decode of the same batch (fp16 K/V of the same shape)
+    del kc, vc
+    k16 = torch.randn((NB, Hkv, bs, D), generator=gen, device=device, dtype=torch.float32).half()
+    v16 = torch.randn((NB, Hkv, bs, D), generator=gen, device=device, dtype=torch.float32).half()
+    call16 = lambda: kvp.paged_attention_decode(q, k16, v16, tt, cl, scale, out,  # noqa: E731
+                                                max_context_len=mcl, partition_size=part,
+                                                workspace=ws)
+    for _ in range(3):
+        call16()
+    ms16 = timed(call16, steps)
+    kvp.check_device_error(device)
+
+    kv = float(lens.sum()) * Hkv * D * 1 * 2
+    alg = kv + S * Hq * D * 2 * 2 + 4 * float(need.sum()) + 4 * S
+    peak, peak_kind = peaks()
+    achieved = alg / (ms * 1e-3) / 1e9
+    res = {
+        "metric": METRIC, "value": round(achieved, 2), "unit": UNIT, "n_gpus": 1,
+        "steps": steps, "warmup": max(3, args.warmup), "ms_per_step": round(ms, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "e4m3 (K/V cache), f16 (q, out), fp32 accumulation",
+        "data": "synthetic (uniform E4M3 codes, per-KV-head scales; seeded N(0,1) q)",
+        "config": {"workload": "OPT-13B geometry, one layer: 64 seqs, 40 heads x 128, block 16, "
+                               "ctx U[1,2048], E4M3 cache with per-KV-head scales, partitions of 512",
+                   "name": args.workload,
+                   "timed": f"paged_attention_decode_fp8 (median of {steps} calls, L2 flushed "
+                            "before each)"},
+        "seq_tokens_per_s": round(float(lens.sum()) / (ms * 1e-3), 1),
+        "f16_cache_same_batch": {"call_us": round(ms16 * 1e3, 2),
+                                 "seq_tokens_per_s": round(float(lens.sum()) / (ms16 * 1e-3), 1),
+                                 "speedup_of_e4m3": round(ms16 / ms, 3)},
+        "rows": {"reshape_and_cache_fp8_step": {"tokens": S, "us": round(scatter_ms * 1e3, 2)}},
+        "roofline": {"kernel": "paged_attention_decode_fp8: decode_simt (E4M3) + decode_reduce_kernel",
+                     "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
+                     "peak_source": peak_kind, "unit": "GB/s", "frac": round(achieved / peak, 4),
+                     "algorithmic_bytes_per_launch": int(alg), "avg_launch_us": round(ms * 1e3, 2),
+                     "traffic": None},
+        "clocks": clk.summary(),
+    }
+    print(json.dumps(res), flush=True)
+
+
 def run_reference(args, world, rank):
     """The oracle as the reference arm: each step is a bounded sample of the workload."""
     if rank != 0:
@@ -920,7 +1039,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="opt13b",
                     choices=["opt13b", "gqa_long_bs16", "gqa_long_bs32", "llama13b_churn",
-                             "sharing_A", "sharing_B", "beam"] + list(PREFILL_WORKLOADS))
+                             "sharing_A", "sharing_B", "beam"] + list(PREFILL_WORKLOADS)
+                    + list(FP8_WORKLOADS))
     ap.add_argument("--partition", type=int, default=None)
     ap.add_argument("--num-seqs", type=int, default=None,
                     help="smaller batch of the same workload (profiling small cases)")
@@ -943,6 +1063,9 @@ def main():
         return
     if args.workload in PREFILL_WORKLOADS:
         run_prefill(args)
+        return
+    if args.workload in FP8_WORKLOADS:
+        run_fp8(args)
         return
     world, rank, local = dist_setup()
     try:

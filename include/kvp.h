@@ -71,6 +71,10 @@ extern "C" {
 /* ---- element types ------------------------------------------------------ */
 #define KVP_F16 0
 #define KVP_BF16 1
+/* E4M3 codes (1 sign, 4 exponent, 3 mantissa bits, bias 7, largest 448, no
+ * infinities) with per-KV-head fp32 scales: a pool of this type is written by
+ * reshape_and_cache_fp8 and read by paged_attention_decode_fp8. */
+#define KVP_FP8_E4M3 2
 
 typedef struct kvp_pool kvp_pool;
 typedef void* kvp_stream_t; /* a cudaStream_t */
@@ -208,8 +212,8 @@ KVP_API int reshape_and_cache(const void* k_new, const void* v_new, void* k_cach
  * distinct and no destination may be a source. Out-of-range ids are skipped
  * and set KVP_ERR_BOUNDS in the device error word. ["Your GPU was mostly
  * empty", section "Paging's second gift: copy-on-write"]
- * pairs: device int32 [num_pairs][2]. block_elems * 2 bytes must be a
- * multiple of 16. */
+ * pairs: device int32 [num_pairs][2]. block_elems * (bytes per element: 2,
+ * or 1 for KVP_FP8_E4M3) must be a multiple of 16. */
 KVP_API int copy_blocks(void* k_cache, void* v_cache, const int32_t* pairs, int32_t num_pairs,
                 int32_t num_blocks, int64_t block_elems, int32_t dtype, kvp_stream_t stream);
 
@@ -380,6 +384,51 @@ KVP_API int paged_attention_prefill(const void* q, const void* k_cache, const vo
                             int32_t max_context_len, float scale, int32_t partition_size,
                             void* workspace, size_t workspace_bytes, void* out, int32_t dtype,
                             kvp_stream_t stream);
+
+/* ---- FP8 (E4M3) KV cache ------------------------------------------------
+ * Cached keys and values as E4M3 codes, one byte per element, with one fp32
+ * scale per KV head for K and one for V: code c of KV head g stands for
+ * value(c) * scale[g]. Quantisation keeps the cached state in a
+ * lower-precision representation, and it combines with paging, which only
+ * decides where the blocks live ["PagedAttention: KV cache memory
+ * management", section "PagedAttention vs KV-cache quantization vs prefix
+ * caching"]. The pool layout is that of the 16-bit cache with 1-byte
+ * elements: [num_blocks][num_kv_heads][block_size][head_dim]. copy_blocks
+ * copies its blocks with dtype KVP_FP8_E4M3. */
+
+/* reshape_and_cache into an E4M3 cache: element x of KV head h of token t is
+ * stored at slot slot_mapping[t] as the code of x / k_scale[h] (values: of
+ * x / v_scale[h]), the division correctly rounded in fp32, the quotient
+ * rounded to the nearest E4M3 value (ties to even) and saturated to +-448;
+ * a negative slot is skipped, a slot past the pool is skipped and recorded
+ * (KVP_ERR_BOUNDS from kvp_check_device_error).
+ * k_new, v_new: device [num_tokens][num_kv_heads][head_dim] of dtype
+ * (KVP_F16 or KVP_BF16), 16-byte aligned; k_cache, v_cache: device uint8
+ * pools; slot_mapping: device int64 [num_tokens]; k_scale, v_scale: device
+ * fp32 [num_kv_heads]. head_dim / 16 and block_size must be powers of two.
+ * Errors: KVP_ERR_INVALID (sizes, dtype, NULL or misaligned pointers). */
+KVP_API int reshape_and_cache_fp8(const void* k_new, const void* v_new, void* k_cache,
+                                  void* v_cache, const int64_t* slot_mapping, const float* k_scale,
+                                  const float* v_scale, int32_t num_tokens, int32_t num_kv_heads,
+                                  int32_t head_dim, int32_t block_size, int32_t num_blocks,
+                                  int32_t dtype, kvp_stream_t stream);
+
+/* paged_attention_decode over an E4M3 cache: key j of KV head g is
+ * value(code) * k_scale[g] and value j is value(code) * v_scale[g]; the
+ * output is the softmax-weighted sum as in paged_attention_decode. q and out
+ * are of dtype (KVP_F16 or KVP_BF16); the other arguments, the workspace
+ * (kvp_decode_workspace_bytes) and the errors are those of
+ * paged_attention_decode. Runs on the CUDA cores for every query head (any
+ * num_q_heads / num_kv_heads); needs head_dim 128. */
+KVP_API int paged_attention_decode_fp8(const void* q, const void* k_cache, const void* v_cache,
+                                       const float* k_scale, const float* v_scale,
+                                       const int32_t* block_tables, const int32_t* context_lens,
+                                       int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
+                                       int32_t head_dim, int32_t block_size, int32_t num_blocks,
+                                       int32_t max_blocks_per_seq, int32_t max_context_len,
+                                       float scale, int32_t partition_size, void* workspace,
+                                       size_t workspace_bytes, void* out, int32_t dtype,
+                                       kvp_stream_t stream);
 
 /* Largest split-context scratch, in bytes, that paged_attention_decode_noalloc
  * can serve from its built-in area (40 MiB). */

@@ -17,17 +17,18 @@ import ctypes as C
 
 import numpy as np
 
-from ._lib import (KVP_BF16, KVP_F16, KvpError, P_i32, P_i64, PoolStats, check, lib)
+from ._lib import (KVP_BF16, KVP_F16, KVP_FP8_E4M3, KvpError, P_i32, P_i64, PoolStats, check,
+                   lib)
 
 __all__ = [
     "BlockPool", "KvpError", "reshape_and_cache", "copy_blocks", "paged_attention_decode",
-    "paged_attention_prefill",
+    "paged_attention_prefill", "reshape_and_cache_fp8", "paged_attention_decode_fp8",
     "decode_workspace_bytes", "decode_grouped_workspace_bytes", "group_plan", "check_device_error",
     "kv_bytes_per_token", "version",
-    "KVP_F16", "KVP_BF16",
+    "KVP_F16", "KVP_BF16", "KVP_FP8_E4M3",
 ]
 
-_DTYPES = {"f16": KVP_F16, "bf16": KVP_BF16}
+_DTYPES = {"f16": KVP_F16, "bf16": KVP_BF16, "fp8_e4m3": KVP_FP8_E4M3}
 
 
 def version() -> str:
@@ -184,6 +185,12 @@ def _code(t) -> int:
     raise TypeError(f"unsupported dtype {t.dtype}")
 
 
+def _is_e4m3(t) -> bool:
+    """An E4M3 cache: uint8 codes, or torch's float8_e4m3fn over the same bytes."""
+    torch = _torch()
+    return t.dtype == torch.uint8 or t.dtype == getattr(torch, "float8_e4m3fn", None)
+
+
 def _cuda(*ts):
     dev = ts[0].device
     for t in ts:
@@ -223,8 +230,11 @@ def copy_blocks(k_cache, v_cache, pairs) -> None:
         raise TypeError("pairs must be int32 [n, 2]")
     NB = k_cache.shape[0]
     elems = k_cache[0].numel()
+    code = KVP_FP8_E4M3 if _is_e4m3(k_cache) else _code(k_cache)
+    if k_cache.dtype != v_cache.dtype:
+        raise TypeError("dtype mismatch")
     check(lib().copy_blocks(k_cache.data_ptr(), v_cache.data_ptr(), pairs.data_ptr(),
-                            pairs.shape[0], NB, elems, _code(k_cache), _stream(dev)))
+                            pairs.shape[0], NB, elems, code, _stream(dev)))
 
 
 def decode_workspace_bytes(num_seqs: int, num_q_heads: int, head_dim: int, max_context_len: int,
@@ -352,6 +362,75 @@ def paged_attention_prefill(q, k_cache, v_cache, block_tables, context_lens, sca
                                         Hq, Hkv, D, bs, NB, max(MB, 1), mcl, float(scale),
                                         int(partition_size), ws_ptr, ws_bytes, out.data_ptr(),
                                         _code(q), _stream(dev)))
+    return out
+
+
+def _fp8_scales(k_scale, v_scale, Hkv, dev):
+    torch = _torch()
+    for t in (k_scale, v_scale):
+        _cuda(t)
+        if t.device != dev or t.dtype != torch.float32 or t.shape != (Hkv,):
+            raise ValueError("k_scale / v_scale must be CUDA float32 [num_kv_heads] on the cache's device")
+
+
+def reshape_and_cache_fp8(k_new, v_new, k_cache, v_cache, slot_mapping, k_scale, v_scale) -> None:
+    """Quantises ``k_new/v_new [T, Hkv, D]`` (fp16 / bf16) into the E4M3 caches
+    ``k_cache/v_cache [NB, Hkv, bs, D]`` (uint8 or float8_e4m3fn) at
+    ``slot_mapping [T]``: KV head h is divided by ``k_scale[h]`` (values:
+    ``v_scale[h]``, CUDA float32 ``[Hkv]``) and rounded to E4M3."""
+    torch = _torch()
+    dev = _cuda(k_new, v_new, k_cache, v_cache, slot_mapping)
+    if slot_mapping.dtype != torch.int64:
+        raise TypeError("slot_mapping must be int64")
+    T, Hkv, D = k_new.shape
+    NB, Hkv2, bs, D2 = k_cache.shape
+    if (Hkv, D) != (Hkv2, D2) or v_new.shape != k_new.shape or v_cache.shape != k_cache.shape:
+        raise ValueError("shape mismatch")
+    if k_new.dtype != v_new.dtype or not (_is_e4m3(k_cache) and _is_e4m3(v_cache)):
+        raise TypeError("k_new/v_new must share a 16-bit dtype and the caches must be E4M3 (uint8)")
+    _fp8_scales(k_scale, v_scale, Hkv, dev)
+    check(lib().reshape_and_cache_fp8(k_new.data_ptr(), v_new.data_ptr(), k_cache.data_ptr(),
+                                      v_cache.data_ptr(), slot_mapping.data_ptr(), k_scale.data_ptr(),
+                                      v_scale.data_ptr(), T, Hkv, D, bs, NB, _code(k_new),
+                                      _stream(dev)))
+
+
+def paged_attention_decode_fp8(q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens,
+                               scale: float, out=None, *, max_context_len: int | None = None,
+                               partition_size: int = 0, workspace=None):
+    """Decode attention over E4M3 caches (uint8 or float8_e4m3fn ``[NB, Hkv, bs, D]``)
+    with per-KV-head scales; q and ``out [S, Hq, D]`` are fp16 / bf16. The other
+    arguments as for :func:`paged_attention_decode`."""
+    torch = _torch()
+    dev = _cuda(q, k_cache, v_cache, block_tables, context_lens)
+    if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32:
+        raise TypeError("block_tables and context_lens must be int32")
+    S, Hq, D = q.shape
+    NB, Hkv, bs, D2 = k_cache.shape
+    if D2 != D or v_cache.shape != k_cache.shape or not (_is_e4m3(k_cache) and _is_e4m3(v_cache)):
+        raise ValueError("q / cache mismatch")
+    _fp8_scales(k_scale, v_scale, Hkv, dev)
+    MB = block_tables.shape[1] if block_tables.dim() == 2 else 0
+    if block_tables.shape[0] != S or context_lens.shape != (S,):
+        raise ValueError("batch metadata mismatch")
+    mcl = MB * bs if max_context_len is None else int(max_context_len)
+    if out is None:
+        out = torch.empty_like(q)
+    else:
+        _cuda(out)
+        if out.shape != q.shape or out.dtype != q.dtype:
+            raise ValueError("out mismatch")
+    need = decode_workspace_bytes(S, Hq, D, mcl, partition_size)
+    ws_ptr, ws_bytes = None, 0
+    if need:
+        if workspace is None:
+            workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+        _cuda(workspace)
+        ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()
+    check(lib().paged_attention_decode_fp8(
+        q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), k_scale.data_ptr(), v_scale.data_ptr(),
+        block_tables.data_ptr(), context_lens.data_ptr(), S, Hq, Hkv, D, bs, NB, max(MB, 1), mcl,
+        float(scale), int(partition_size), ws_ptr, ws_bytes, out.data_ptr(), _code(q), _stream(dev)))
     return out
 
 

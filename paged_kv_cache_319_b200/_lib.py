@@ -17,6 +17,7 @@ KVP_ERR_BOUNDS = -5
 KVP_ERR_CAPACITY = -6
 KVP_F16 = 0
 KVP_BF16 = 1
+KVP_FP8_E4M3 = 2
 KVP_STATIC_SCRATCH_BYTES = 40 * 1024 * 1024  # include/kvp.h
 
 ERROR_KINDS = {
@@ -79,6 +80,10 @@ SIGNATURES = {
     "kvp_prefill_workspace_bytes": (sz, [i32, i32, i32, i32, i32, i32]),
     "paged_attention_prefill": (C.c_int, [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32,
                                           i32, i32, f32, i32, vp, sz, vp, i32, vp]),
+    "reshape_and_cache_fp8": (C.c_int, [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,
+                                        vp]),
+    "paged_attention_decode_fp8": (C.c_int, [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32,
+                                             i32, i32, i32, f32, i32, vp, sz, vp, i32, vp]),
     "kv_decode_group_plan": (C.c_int, [P_i32, P_i32, i32, i32, i32, i32, i32, i32, i32, i32, P_i32,
                                        sz]),
     "paged_attention_decode_noalloc": (C.c_int, [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,

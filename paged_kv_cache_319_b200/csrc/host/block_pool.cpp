@@ -113,8 +113,8 @@ int kv_pool_create(int32_t num_blocks, int32_t block_size, int32_t num_kv_heads,
   if (!out) return fail(KVP_ERR_INVALID, "kv_pool_create: out is NULL");
   if (num_blocks <= 0 || block_size <= 0 || num_kv_heads <= 0 || head_dim <= 0)
     return fail(KVP_ERR_INVALID, "kv_pool_create: sizes must be positive");
-  if (dtype != KVP_F16 && dtype != KVP_BF16)
-    return fail(KVP_ERR_INVALID, "kv_pool_create: dtype must be KVP_F16 or KVP_BF16");
+  if (dtype != KVP_F16 && dtype != KVP_BF16 && dtype != KVP_FP8_E4M3)
+    return fail(KVP_ERR_INVALID, "kv_pool_create: dtype must be KVP_F16, KVP_BF16 or KVP_FP8_E4M3");
   if (int64_t(num_blocks) * block_size > (int64_t(1) << 40))
     return fail(KVP_ERR_INVALID, "kv_pool_create: pool too large");
   kvp_pool* p = new (std::nothrow) kvp_pool();

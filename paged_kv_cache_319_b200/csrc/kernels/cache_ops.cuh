@@ -44,6 +44,58 @@ __global__ void __launch_bounds__(256) reshape_and_cache_kernel(
   }
 }
 
+// FP8 cache: the new tokens' K and V rows quantised into their slots, KV head
+// h with its own scales: code = E4M3(x / scale[h]), the division correctly
+// rounded in fp32, then rounded to the nearest E4M3 value (ties to even) and
+// saturated to +-448. Quantised cached values are a lower-precision
+// representation of the same state ["PagedAttention: KV cache memory
+// management", section "PagedAttention vs KV-cache quantization vs prefix
+// caching"]. k_new/v_new: [T][Hkv][D] of T; cache: [NB][Hkv][bs][D] bytes.
+// Thread-iteration c writes the 16-byte chunk j = c % cpr (16 codes) of row
+// (t, h) = c / cpr, cpr = D / 16.
+template <typename T>
+__global__ void __launch_bounds__(256) reshape_and_cache_fp8_kernel(
+    const uint4* __restrict__ k_new, const uint4* __restrict__ v_new, uint4* __restrict__ k_cache,
+    uint4* __restrict__ v_cache, const int64_t* __restrict__ slot_mapping,
+    const float* __restrict__ k_scale, const float* __restrict__ v_scale, uint32_t num_chunks,
+    uint32_t num_kv_heads, uint32_t log2_cpr, uint32_t log2_bs, int64_t num_slots) {
+  const uint32_t stride = gridDim.x * blockDim.x;
+  const uint32_t cpr_mask = (1u << log2_cpr) - 1u;
+  auto quantize = [](uint4 a, uint4 b, float s) {  // 16 values -> 16 codes
+    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 f0 = Elem<T>::to_float2(w[2 * i]);
+      const float2 f1 = Elem<T>::to_float2(w[2 * i + 1]);
+      const uint32_t c0 = float2_to_e4m3x2(__fdiv_rn(f0.x, s), __fdiv_rn(f0.y, s));
+      const uint32_t c1 = float2_to_e4m3x2(__fdiv_rn(f1.x, s), __fdiv_rn(f1.y, s));
+      o[i] = c0 | (c1 << 16);
+    }
+    return make_uint4(o[0], o[1], o[2], o[3]);
+  };
+  for (uint32_t c = blockIdx.x * blockDim.x + threadIdx.x; c < num_chunks; c += stride) {
+    const uint32_t row = c >> log2_cpr;
+    const uint32_t j = c & cpr_mask;
+    const uint32_t t = row / num_kv_heads;
+    const uint32_t h = row - t * num_kv_heads;
+    const int64_t s = __ldg(slot_mapping + t);
+    if (s < 0) continue;  // padding token
+    if (s >= num_slots) {
+      if (h == 0 && j == 0) record_error(KVP_DEVERR_SLOT, uint64_t(t));
+      continue;
+    }
+    const int64_t blk = s >> log2_bs;
+    const int64_t off = s & ((int64_t(1) << log2_bs) - 1);
+    const int64_t dst = (((blk * num_kv_heads + h) << log2_bs) + off) * (int64_t(1) << log2_cpr) + j;
+    // source: 16 elements of T = two 16-byte vectors
+    const uint4 k0 = __ldg(k_new + 2 * int64_t(c)), k1 = __ldg(k_new + 2 * int64_t(c) + 1);
+    const uint4 v0 = __ldg(v_new + 2 * int64_t(c)), v1 = __ldg(v_new + 2 * int64_t(c) + 1);
+    k_cache[dst] = quantize(k0, k1, __ldg(k_scale + h));
+    v_cache[dst] = quantize(v0, v1, __ldg(v_scale + h));
+  }
+}
+
 // Block-level copy-on-write: block dst of K and V becomes a copy of block src
 // ["Your GPU was mostly empty", section "Paging's second gift: copy-on-write"].
 // grid.y = pair, grid.z = 0 (K) / 1 (V); grid.x strides over the block's chunks.

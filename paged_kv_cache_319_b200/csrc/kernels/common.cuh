@@ -272,6 +272,23 @@ struct Elem<__nv_bfloat16> {
   }
 };
 
+// E4M3 (8-bit float: 1 sign, 4 exponent, 3 mantissa bits, bias 7, largest
+// finite 448) by the PTX conversions of sm_89 and later. Two codes per 16 bits,
+// the lower byte first.
+// Two codes -> their exact values (every E4M3 value is an fp16 value).
+__device__ __forceinline__ float2 e4m3x2_to_float2(uint32_t two_codes) {
+  uint32_t h2;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(static_cast<uint16_t>(two_codes)));
+  return __half22float2(*reinterpret_cast<const __half2*>(&h2));
+}
+// Two fp32 values -> their codes: round to nearest even, saturated to +-448
+// (infinities too), NaN to NaN; lo goes to the lower byte.
+__device__ __forceinline__ uint32_t float2_to_e4m3x2(float lo, float hi) {
+  uint16_t d;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(d) : "f"(hi), "f"(lo));
+  return d;
+}
+
 // Order-preserving map of fp32 to int32 (for integer max reductions).
 __device__ __forceinline__ int32_t float_to_ordered(float f) {
   const int32_t i = __float_as_int(f);

@@ -61,6 +61,10 @@ struct DecodeArgs {
   // for its shared prefix followed by the slots of its own range, and the
   // reduce writes every output row.
   const int32_t* plan;
+  // FP8 cache only (null otherwise): per KV head, the scales of the E4M3 keys
+  // and values (a cached code c of head g stands for value(c) * scale[g]).
+  const float* k_scale;
+  const float* v_scale;
 };
 
 __device__ __forceinline__ uint8_t* align_1024(uint8_t* p) {
@@ -78,10 +82,11 @@ __device__ __forceinline__ int32_t load_ctx(const DecodeArgs& a, int32_t s, bool
   return ctx;
 }
 
-template <typename T, int D, int BS, int NW, int NST>
+// EB: bytes per cached element (2: fp16 / bf16; 1: E4M3).
+template <typename T, int D, int BS, int NW, int NST, int EB = 2>
 struct SimtCfg {
-  static constexpr int kRegions = D / 64;          // 128-byte row regions (1 or 2)
-  static constexpr int kTileBytes = BS * D * 2;    // one (block, KV head) tile
+  static constexpr int kRegions = D * EB / 128;    // 128-byte row regions (1 or 2)
+  static constexpr int kTileBytes = BS * D * EB;   // one (block, KV head) tile
   static constexpr int kChunksPerRow = D / 8;      // 16-byte chunks per row
   static constexpr int kChunksPerLane = kChunksPerRow / 2;
   static constexpr int kPasses = (BS + 15) / 16;   // 16 rows per QK pass
@@ -93,6 +98,7 @@ struct SimtCfg {
   static_assert(D == 64 || D == 128, "head_dim 64 or 128");
   static_assert(BS == 8 || BS == 16 || BS == 32, "block_size 8, 16 or 32");
   static_assert(NST >= 1 && NST <= 32, "stages");
+  static_assert(EB == 2 || D == 128, "E4M3 caches: head_dim 128 (one 128-byte row)");
 };
 
 // Per-lane shapes of a (block, KV head) tile in the CUDA-core kernels.
@@ -199,16 +205,125 @@ __device__ __forceinline__ void simt_tile(const uint8_t* kt, const uint8_t* vt, 
   }
 }
 
+// simt_tile for an E4M3 cache (head_dim 128: a tile row is 128 codes, one
+// 128-byte swizzled region). Same lanes and steps as simt_tile: a QK lane
+// covers 64 dims of its key row as four 16-byte chunks of 16 codes; a PV lane
+// owns 4 output dims (4 codes of each value row). Codes convert exactly to
+// fp16 (cvt.rn.f16x2.e4m3x2, two per instruction). With half the bytes of a
+// 16-bit cache per token the kernel is bound by instructions, not HBM, so the
+// QK products of an fp16 q take the fp16 keys directly in sm_100's mixed-
+// precision fma (fp16 x fp16 + fp32; the products are exact in fp32), with
+// the scales applied to the dot. On the OPT-13B batch this took the call from
+// 142 us (keys widened to fp32 first) to 118 us; widening by shifts and masks
+// instead of cvt was slower (167 us). A bf16 q, and the PV products (p is
+// fp32), use fp32 FMAs. The value scale is applied by the caller to the
+// finished accumulator.
+#ifndef KVP_FP8_MIXED
+#define KVP_FP8_MIXED 1  // 0: widen fp16 keys to fp32 for the QK products as well
+#endif
+// d0 += lo(q2) * lo(k2), d1 += hi(q2) * hi(k2): fp16 products accumulated in
+// fp32 by sm_100's mixed-precision fma (no conversion of k to fp32).
+__device__ __forceinline__ void fma2_f16_f32(float& d0, float& d1, uint32_t q2, uint32_t k2) {
+  asm("{\n\t.reg .f16 ql, qh, kl, kh;\n\t"
+      "mov.b32 {ql, qh}, %2;\n\t"
+      "mov.b32 {kl, kh}, %3;\n\t"
+      "fma.rn.f32.f16 %0, ql, kl, %0;\n\t"
+      "fma.rn.f32.f16 %1, qh, kh, %1;\n\t}"
+      : "+f"(d0), "+f"(d1)
+      : "r"(q2), "r"(k2));
+}
+
+// MX: q is fp16 and arrives as 32 packed pairs in qh (qf unused), unscaled; the
+// score is dot * q_mul.
+template <int BS, bool MX = false>
+__device__ __forceinline__ void simt_tile_fp8(const uint8_t* kt, const uint8_t* vt, int32_t nvalid,
+                                              const float (&qf)[64], const uint32_t (&qh)[32],
+                                              float q_mul, float& m_run, float& l_lane,
+                                              float (&acc)[4], int lane) {
+  constexpr int kPasses = (BS + 15) / 16;
+  const int part = lane >> 4;
+  float sc[kPasses];
+#pragma unroll
+  for (int ps = 0; ps < kPasses; ++ps) {
+    const int r = ps * 16 + (lane & 15);
+    float d0 = 0.f, d1 = 0.f, d2 = 0.f, d3 = 0.f;
+    if (r < BS) {
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const int lc = part * 4 + c;  // 16-byte chunk of the row: dims lc * 16 ..
+        const uint4 kv = *reinterpret_cast<const uint4*>(kt + r * 128 + ((lc ^ (r & 7)) << 4));
+        const uint32_t w[4] = {kv.x, kv.y, kv.z, kv.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          if constexpr (MX) {
+            uint32_t k01, k23;
+            asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(k01) : "h"(static_cast<uint16_t>(w[e])));
+            asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(k23) : "h"(static_cast<uint16_t>(w[e] >> 16)));
+            fma2_f16_f32(d0, d1, qh[c * 8 + 2 * e], k01);
+            fma2_f16_f32(d2, d3, qh[c * 8 + 2 * e + 1], k23);
+          } else {
+            const float2 f0 = e4m3x2_to_float2(w[e]);
+            const float2 f1 = e4m3x2_to_float2(w[e] >> 16);
+            d0 = fmaf(qf[c * 16 + 4 * e + 0], f0.x, d0);
+            d1 = fmaf(qf[c * 16 + 4 * e + 1], f0.y, d1);
+            d2 = fmaf(qf[c * 16 + 4 * e + 2], f1.x, d2);
+            d3 = fmaf(qf[c * 16 + 4 * e + 3], f1.y, d3);
+          }
+        }
+      }
+    }
+    float dot = (d0 + d1) + (d2 + d3);
+    if constexpr (MX) dot *= q_mul;
+    dot += __shfl_xor_sync(0xffffffffu, dot, 16);
+    sc[ps] = r < nvalid ? dot : -INFINITY;
+  }
+  float tmax = sc[0];
+#pragma unroll
+  for (int ps = 1; ps < kPasses; ++ps) tmax = fmaxf(tmax, sc[ps]);
+  tmax = warp_max(tmax);
+  const float m_new = fmaxf(m_run, tmax);
+  const float alpha = m_run == -INFINITY ? 0.f : exp2f(m_run - m_new);
+  float pr[kPasses];
+  float psum = 0.f;
+#pragma unroll
+  for (int ps = 0; ps < kPasses; ++ps) {
+    pr[ps] = sc[ps] == -INFINITY ? 0.f : exp2f(sc[ps] - m_new);
+    psum += pr[ps];
+  }
+  l_lane = l_lane * alpha + (lane < 16 ? psum : 0.f);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) acc[e] *= alpha;
+  m_run = m_new;
+  // acc += p V: dims lane * 4 .. + 3 are bytes (lane & 3) * 4 .. of chunk lane / 4
+  const int cc = lane >> 2;
+  const int pos = (lane & 3) * 4;
+#pragma unroll
+  for (int r = 0; r < BS; ++r) {
+    const float pv = __shfl_sync(0xffffffffu, pr[r >> 4], r & 15);
+    if (r < nvalid) {
+      const uint32_t v = *reinterpret_cast<const uint32_t*>(vt + r * 128 + ((cc ^ (r & 7)) << 4) + pos);
+      const float2 f0 = e4m3x2_to_float2(v);
+      const float2 f1 = e4m3x2_to_float2(v >> 16);
+      acc[0] = fmaf(pv, f0.x, acc[0]);
+      acc[1] = fmaf(pv, f0.y, acc[1]);
+      acc[2] = fmaf(pv, f1.x, acc[2]);
+      acc[3] = fmaf(pv, f1.y, acc[3]);
+    }
+  }
+}
+
 // PH (per-head warps): grid (partition, ceil(Hq / NW), sequence); warp w takes
 // query head blockIdx.y * NW + w over the whole partition and writes its own
 // partial, with no merge across warps. For short ranges (a few blocks per
 // (sequence, head)), where splitting a range over the warps would leave each
 // warp one or two blocks, this keeps every warp's pipeline busy.
-template <typename T, int D, int BS, int NW, int NST, bool PH = false>
+// F8: the cache holds E4M3 codes (a.k_scale / a.v_scale set; head_dim 128);
+// q and out stay in T.
+template <typename T, int D, int BS, int NW, int NST, bool PH = false, bool F8 = false>
 __global__ void __launch_bounds__(NW * 32) decode_simt_kernel(
     const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
     const DecodeArgs a) {
-  using C = SimtCfg<T, D, BS, NW, NST>;
+  using C = SimtCfg<T, D, BS, NW, NST, F8 ? 1 : 2>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align_1024(smem_raw);
   uint8_t* tiles = smem;
@@ -291,7 +406,11 @@ __global__ void __launch_bounds__(NW * 32) decode_simt_kernel(
       row = (id * a.num_kv_heads + g) * BS;
     }
     mbar_arrive_expect_tx(&my_bars[stage], 2 * C::kTileBytes);
-    if constexpr (C::kRegions == 2) {
+    if constexpr (F8) {
+      // one 2-D box {128 codes, BS rows} per tile: smem [row][128]
+      tma_load_2d(kt, &kmap, &my_bars[stage], 0, row, policy);
+      tma_load_2d(vt, &vmap, &my_bars[stage], 0, row, policy);
+    } else if constexpr (C::kRegions == 2) {
       // one 3-D box {64 dims, BS rows, 2 halves} per tile: smem [half][row][64]
       tma_load_3d(kt, &kmap, &my_bars[stage], 0, row, 0, policy);
       tma_load_3d(vt, &vmap, &my_bars[stage], 0, row, 0, policy);
@@ -313,7 +432,22 @@ __global__ void __launch_bounds__(NW * 32) decode_simt_kernel(
   // [part * kChunksPerLane, (part + 1) * kChunksPerLane) of the row.
   const int part = lane >> 4;
   float qf[C::kChunksPerLane * 8];
-  {
+  float q_mul = a.scale_log2;
+  if constexpr (F8) q_mul *= __ldg(a.k_scale + g);
+  constexpr bool kMixed = F8 && KVP_FP8_MIXED && std::is_same<T, __half>::value;
+  uint32_t qh[32];  // kMixed: this lane's 64 dims of q as fp16 pairs
+  if constexpr (kMixed) {
+    const uint4* qrow = reinterpret_cast<const uint4*>(static_cast<const T*>(a.q) +
+                                                       (int64_t(s) * a.num_q_heads + h) * D);
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const uint4 v = __ldg(qrow + part * 8 + c);
+      qh[4 * c] = v.x;
+      qh[4 * c + 1] = v.y;
+      qh[4 * c + 2] = v.z;
+      qh[4 * c + 3] = v.w;
+    }
+  } else {
     const uint4* qrow = reinterpret_cast<const uint4*>(static_cast<const T*>(a.q) +
                                                        (int64_t(s) * a.num_q_heads + h) * D);
 #pragma unroll
@@ -323,8 +457,8 @@ __global__ void __launch_bounds__(NW * 32) decode_simt_kernel(
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const float2 f = Elem<T>::to_float2(w[e]);
-        qf[c * 8 + 2 * e] = f.x * a.scale_log2;
-        qf[c * 8 + 2 * e + 1] = f.y * a.scale_log2;
+        qf[c * 8 + 2 * e] = f.x * q_mul;
+        qf[c * 8 + 2 * e + 1] = f.y * q_mul;
       }
     }
   }
@@ -350,7 +484,11 @@ __global__ void __launch_bounds__(NW * 32) decode_simt_kernel(
     const int32_t tok0 = (b0 + wfirst + kStride * i) * BS;
     const int32_t nvalid = min(BS, ctx - tok0);
 
-    simt_tile<T, D, BS>(kt, vt, nvalid, qf, m_run, l_lane, acc, lane);
+    if constexpr (F8) {
+      simt_tile_fp8<BS, kMixed>(kt, vt, nvalid, qf, qh, q_mul, m_run, l_lane, acc, lane);
+    } else {
+      simt_tile<T, D, BS>(kt, vt, nvalid, qf, m_run, l_lane, acc, lane);
+    }
 
     // ---- refill this stage with block i + NST
     const int32_t nxt = i + NST;
@@ -366,6 +504,11 @@ __global__ void __launch_bounds__(NW * 32) decode_simt_kernel(
     }
   }
 
+  if constexpr (F8) {  // the values' scale, once, on the finished sums
+    const float vs = __ldg(a.v_scale + g);
+#pragma unroll
+    for (int e = 0; e < C::kDimsPerLane; ++e) acc[e] *= vs;
+  }
   if (aborted) {
     // Drain this warp's loads still in flight before the CTA exits.
     if (lane == 0) {

@@ -67,3 +67,13 @@ def random_paged_batch(seed, S, Hq, Hkv, D, bs, lens, dtype, extra_blocks=7):
     k = workloads.normal_bits([seed, 2], (nb, Hkv, bs, D), dtype)
     v = workloads.normal_bits([seed, 3], (nb, Hkv, bs, D), dtype)
     return q, k, v, tables, np.asarray(lens, np.int32)
+
+
+def random_e4m3_codes(seed, shape) -> np.ndarray:
+    """Seeded uniform E4M3 codes (uint8) with the two NaN codes replaced by +-1.875
+    (0x3F / 0xBF): a cache of every finite magnitude from 2^-9 to 448."""
+    rng = np.random.default_rng(seed)
+    c = rng.integers(0, 256, size=shape, dtype=np.uint8)
+    nan = (c & 0x7F) == 0x7F
+    c[nan] = c[nan] & 0xBF
+    return c
