@@ -69,12 +69,15 @@ def peaks():
 # its algorithmic bytes, from the ncu captures summarised in profiles/; valid only
 # while the kernel source hashes to the value it had when captured.
 PROFILED_TRAFFIC = {
-    # profiles/decode_simt_opt13b.md: 614.78 MB read + 4.49 MB written, 610.45 MB algorithmic
-    "decode_simt": {"ratio": (614.783232e6 + 4.493312e6) / 610454988.0, "sha": "c223337b324668bc",
+    # profiles/decode_simt_opt13b.md: 614.77 MB read + 4.34 MB written, 610.45 MB algorithmic
+    "decode_simt": {"ratio": (614.76992e6 + 4.34048e6) / 610454988.0, "sha": "5459ca24c585c329",
                     "files": ["common.cuh", "decode_simt.cuh"]},
-    # profiles/decode_tc_gqa_long_bs16.md: 334.34 MB read + 5.07 MB written, 334.13 MB algorithmic
-    "decode_tc": {"ratio": (334.336512e6 + 5.07264e6) / 334131132.0, "sha": "d219218fe69cafb4",
+    # profiles/decode_tc_gqa_long_bs16.md: 334.32 MB read + 4.82 MB written, 334.13 MB algorithmic
+    "decode_tc": {"ratio": (334.321408e6 + 4.816384e6) / 334131132.0, "sha": "e7bb48ce13b9f527",
                   "files": ["common.cuh", "decode_group.cuh", "decode_simt.cuh", "decode_tc.cuh"]},
+    # profiles/decode_simt_fp8_opt13b.md: 621.82 MB read + 4.93 MB written, 617.57 MB algorithmic
+    "decode_simt_fp8": {"ratio": (621.820928e6 + 4.93184e6) / 617569340.0, "sha": "5459ca24c585c329",
+                        "files": ["common.cuh", "decode_simt.cuh"]},
 }
 
 
@@ -179,13 +182,23 @@ class ClockSampler:
             pass
         self._p.join(timeout=10)
 
-    def summary(self):
+    def summary(self, min_samples: int = 3):
+        """Median SM clock and the throttle reasons seen inside the timed window. A
+        window shorter than a few NVML queries is widened 25 ms at a time on both
+        sides (the warm-up just before it runs the same work) until it holds
+        ``min_samples`` samples, at most 0.5 s; ``window_padded_ms`` says by how much."""
         t0, t1 = self.window
+        pad = 0.0
         inside = [(c, r) for t, c, r in self.samples if t0 <= t <= t1]
+        while len(inside) < min_samples and pad < 0.5:
+            pad += 0.025
+            inside = [(c, r) for t, c, r in self.samples if t0 - pad <= t <= t1 + pad]
         reasons = sorted({n for _, r in inside for n, b in REASON_BITS.items() if r & b})
         res = {"sm_mhz": float(statistics.median([c for c, _ in inside])) if inside else None,
                "sm_max_mhz": self.max_mhz, "reasons": reasons, "samples": len(inside),
                "window_ms": round((t1 - t0) * 1e3, 1)}
+        if pad:
+            res["window_padded_ms"] = round(pad * 1e3, 1)
         if self.error:
             res["error"] = self.error
         return res
@@ -985,7 +998,7 @@ def run_fp8(args):
                      "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
                      "peak_source": peak_kind, "unit": "GB/s", "frac": round(achieved / peak, 4),
                      "algorithmic_bytes_per_launch": int(alg), "avg_launch_us": round(ms * 1e3, 2),
-                     "traffic": None},
+                     "traffic": traffic_per_launch("decode_simt_fp8", alg)},
         "clocks": clk.summary(),
     }
     print(json.dumps(res), flush=True)
