@@ -220,3 +220,162 @@ class BlockManager:
     def _check(self, seq: int) -> None:
         if seq not in self._tables:
             raise NoSuchSequence(f"no live sequence {seq}")
+
+
+class PrefixCachingBlockManager(BlockManager):
+    """The block manager with prefix caching across requests: full blocks keep the
+    keys and values of a token prefix that a later request with the same prefix
+    reuses instead of recomputing ("PagedAttention: KV cache memory management",
+    section "PagedAttention vs KV-cache quantization vs prefix caching"; sharing
+    across requests: "vLLM and PagedAttention", section "Key claims from the
+    paper"). The pages give no policy; this oracle pins one (readings 7-13, on top
+    of 1-6 of the module doc):
+
+    7. A full block is cached under the key (parent, tokens): ``parent`` is the
+       physical block before it in the table that filled it (-1 for a first
+       block), ``tokens`` its ``block_size`` token ids. Keys are compared
+       exactly, so a match means the whole token prefix up to that block is
+       equal (by induction over the parents).
+    8. ``append_tokens(seq, tokens)`` is ``append`` with the token ids given;
+       whenever a token fills a block, that block is registered under its key
+       unless the key is taken (another request computed the same prefix: the
+       first registration stays) or the block is registered already. A plain
+       ``append`` on a sequence stops its registration for good (its later
+       tokens are unknown).
+    9. ``create_prefixed(tokens)`` creates a sequence holding the longest run of
+       leading cached blocks of ``tokens`` whose tokens end before the prompt's
+       last one (the last prompt token is always computed): each matched block
+       gains a reference. It returns (sequence, cached tokens); the caller
+       appends ``tokens[cached:]`` with ``append_tokens``.
+    10. ``release`` drops references in logical order; a block reaching zero goes
+        to the free stack if it is not registered, else it becomes evictable.
+        The blocks of one release become evictable from the last logical block
+        to the first, so the deepest blocks of a prefix are evicted first.
+    11. A new block comes from the free stack; when it is empty, the evictable
+        block released longest ago is evicted (its key dropped) and used.
+        Capacity checks count free and evictable blocks.
+    12. A lookup that matches an evictable block takes it back (it leaves the
+        evictable list).
+    13. ``fork`` copies the parent's tokens and registration state.
+    """
+
+    def __init__(self, num_blocks: int, block_size: int, free_order=None):
+        super().__init__(num_blocks, block_size, free_order)
+        self._key_of: dict[int, tuple] = {}     # registered block -> key
+        self._block_of: dict[tuple, int] = {}   # key -> registered block
+        self._evictable: list[int] = []         # front = evicted next
+        self._tokens: dict[int, list[int]] = {}  # tracked sequences' token ids
+        self.hit_tokens = 0
+
+    # ---- queries -----------------------------------------------------------
+    def evictable(self) -> list[int]:
+        return list(self._evictable)
+
+    def cached_blocks(self) -> int:
+        return len(self._key_of)
+
+    def available(self) -> int:
+        return len(self._free) + len(self._evictable)
+
+    # ---- mutations ---------------------------------------------------------
+    def _take(self) -> int:
+        if self._free:
+            return self._free.pop()
+        b = self._evictable.pop(0)
+        del self._block_of[self._key_of.pop(b)]
+        return b
+
+    def create(self) -> int:
+        seq = super().create()
+        self._tokens[seq] = []
+        return seq
+
+    def create_prefixed(self, tokens) -> tuple[int, int]:
+        tokens = [int(t) for t in tokens]
+        seq = self.create()
+        bs = self.block_size
+        table = self._tables[seq]
+        parent = -1
+        i = 0
+        while (i + 1) * bs <= len(tokens) - 1:
+            b = self._block_of.get((parent, tuple(tokens[i * bs:(i + 1) * bs])))
+            if b is None:
+                break
+            if self.rc[b] == 0:
+                self._evictable.remove(b)
+            self.rc[b] += 1
+            table.append(b)
+            parent = b
+            i += 1
+        self._lens[seq] = i * bs
+        self._tokens[seq] = tokens[:i * bs]
+        self.hit_tokens += i * bs
+        return seq, i * bs
+
+    def blocks_needed(self, seq: int, n: int) -> int:
+        return super().blocks_needed(seq, n)
+
+    def append_tokens(self, seq: int, tokens) -> list[int]:
+        tokens = [int(t) for t in tokens]
+        return self._append(seq, len(tokens), tokens)
+
+    def append(self, seq: int, n: int) -> list[int]:
+        return self._append(seq, n, None)
+
+    def _append(self, seq, n, tokens):
+        self._check(seq)
+        if n < 0:
+            raise InvalidArgument("n must be >= 0")
+        if self.blocks_needed(seq, n) > self.available():
+            raise OutOfBlocks("not enough free blocks")
+        if tokens is None:
+            self._tokens.pop(seq, None)  # reading 8: registration stops
+        table = self._tables[seq]
+        bs = self.block_size
+        slots = []
+        for k in range(n):
+            pos = self._lens[seq]
+            if pos % bs == 0:
+                b = self._take()
+                self.rc[b] = 1
+                table.append(b)
+            elif self.rc[table[-1]] > 1:
+                src = table[-1]
+                dst = self._take()
+                self._pending.append((src, dst))
+                self._cow_total += 1
+                self.rc[src] -= 1
+                self.rc[dst] = 1
+                table[-1] = dst
+            slots.append(table[pos // bs] * bs + pos % bs)
+            self._lens[seq] = pos + 1
+            if seq in self._tokens:
+                self._tokens[seq].append(tokens[k])
+                if (pos + 1) % bs == 0:
+                    blk = table[pos // bs]
+                    parent = table[pos // bs - 1] if pos // bs > 0 else -1
+                    key = (parent, tuple(self._tokens[seq][pos + 1 - bs:pos + 1]))
+                    if key not in self._block_of and blk not in self._key_of:
+                        self._block_of[key] = blk
+                        self._key_of[blk] = key
+        return slots
+
+    def fork(self, parent: int) -> int:
+        child = super().fork(parent)
+        if parent in self._tokens:
+            self._tokens[child] = list(self._tokens[parent])
+        return child
+
+    def release(self, seq: int) -> None:
+        self._check(seq)
+        newly = []
+        for b in self._tables.pop(seq):
+            self.rc[b] -= 1
+            if self.rc[b] == 0:
+                if b in self._key_of:
+                    newly.append(b)
+                else:
+                    self._free.append(b)
+        self._evictable.extend(reversed(newly))
+        del self._lens[seq]
+        self._tokens.pop(seq, None)
