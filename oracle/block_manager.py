@@ -231,15 +231,18 @@ class PrefixCachingBlockManager(BlockManager):
     paper"). The pages give no policy; this oracle pins one (readings 7-13, on top
     of 1-6 of the module doc):
 
-    7. A full block is cached under the key (parent, tokens): ``parent`` is the
-       physical block before it in the table that filled it (-1 for a first
-       block), ``tokens`` its ``block_size`` token ids. Keys are compared
-       exactly, so a match means the whole token prefix up to that block is
-       equal (by induction over the parents).
+    7. A full block is cached under the key (parent, tokens): ``tokens`` are its
+       ``block_size`` token ids and ``parent`` is the registration number of the
+       block before it in the table that filled it (-1 for a first block).
+       Registrations are numbered 0, 1, 2, ... and numbers are never reused, so
+       a key names one exact token prefix: a match means the whole prefix up to
+       that block is equal (by induction over the parents), even after a parent
+       block was evicted and its physical block reused.
     8. ``append_tokens(seq, tokens)`` is ``append`` with the token ids given;
        whenever a token fills a block, that block is registered under its key
        unless the key is taken (another request computed the same prefix: the
-       first registration stays) or the block is registered already. A plain
+       first registration stays), the block is registered already, or the block
+       before it is not registered (then no lookup can reach it). A plain
        ``append`` on a sequence stops its registration for good (its later
        tokens are unknown).
     9. ``create_prefixed(tokens)`` creates a sequence holding the longest run of
@@ -263,6 +266,8 @@ class PrefixCachingBlockManager(BlockManager):
         super().__init__(num_blocks, block_size, free_order)
         self._key_of: dict[int, tuple] = {}     # registered block -> key
         self._block_of: dict[tuple, int] = {}   # key -> registered block
+        self._reg_of: dict[int, int] = {}       # registered block -> registration number
+        self._next_reg = 0
         self._evictable: list[int] = []         # front = evicted next
         self._tokens: dict[int, list[int]] = {}  # tracked sequences' token ids
         self.hit_tokens = 0
@@ -283,6 +288,7 @@ class PrefixCachingBlockManager(BlockManager):
             return self._free.pop()
         b = self._evictable.pop(0)
         del self._block_of[self._key_of.pop(b)]
+        del self._reg_of[b]
         return b
 
     def create(self) -> int:
@@ -305,7 +311,7 @@ class PrefixCachingBlockManager(BlockManager):
                 self._evictable.remove(b)
             self.rc[b] += 1
             table.append(b)
-            parent = b
+            parent = self._reg_of[b]
             i += 1
         self._lens[seq] = i * bs
         self._tokens[seq] = tokens[:i * bs]
@@ -353,11 +359,14 @@ class PrefixCachingBlockManager(BlockManager):
                 self._tokens[seq].append(tokens[k])
                 if (pos + 1) % bs == 0:
                     blk = table[pos // bs]
-                    parent = table[pos // bs - 1] if pos // bs > 0 else -1
+                    prev = table[pos // bs - 1] if pos // bs > 0 else None
+                    parent = -1 if prev is None else self._reg_of.get(prev)
                     key = (parent, tuple(self._tokens[seq][pos + 1 - bs:pos + 1]))
-                    if key not in self._block_of and blk not in self._key_of:
+                    if parent is not None and key not in self._block_of and blk not in self._key_of:
                         self._block_of[key] = blk
                         self._key_of[blk] = key
+                        self._reg_of[blk] = self._next_reg
+                        self._next_reg += 1
         return slots
 
     def fork(self, parent: int) -> int:

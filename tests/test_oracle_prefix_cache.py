@@ -47,6 +47,21 @@ def test_eviction_takes_the_deepest_block_released_longest_ago():
         m.append_tokens(c, [3, 4, 9, 9, 9])  # needs 3 blocks, none free or evictable
 
 
+def test_a_block_after_an_unregistered_one_is_not_registered():
+    """Two requests fill the same prefix at once: the first keeps the cache entry, the
+    second's copy stays private, and so does every block after it."""
+    m = PrefixCachingBlockManager(8, 2)
+    a, b = m.create(), m.create()
+    m.append_tokens(a, [1, 2])
+    m.append_tokens(b, [1, 2, 3, 4])  # b's first block duplicates a's: not registered
+    m.append_tokens(a, [3, 4])
+    assert m.cached_blocks() == 2 and set(m._key_of) == set(m.block_table(a))
+    m.release(b)  # b's blocks were private: straight to the free stack
+    assert m.evictable() == [] and m.num_free() == 6
+    c, hit = m.create_prefixed([1, 2, 3, 4, 5])
+    assert hit == 4 and m.block_table(c) == m.block_table(a)
+
+
 def test_plain_append_stops_registration():
     m = PrefixCachingBlockManager(6, 2)
     s = m.create()
@@ -135,3 +150,4 @@ def test_bookkeeping_invariants(seed):
             assert b in m._key_of  # only registered blocks wait for reuse
         for b, (parent, toks) in m._key_of.items():
             assert [int(x) for x in content[b * bs:(b + 1) * bs]] == list(toks)
+            assert parent == -1 or parent < m._reg_of[b]  # parents were registered first
