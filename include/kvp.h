@@ -170,6 +170,60 @@ KVP_API int kv_pool_take_copies(kvp_pool* pool, int32_t* pairs, int32_t cap, int
 /* Like kv_pool_take_copies but leaves the queue as it is. */
 KVP_API int kv_pool_pending_copies(const kvp_pool* pool, int32_t* pairs, int32_t cap, int32_t* n);
 
+/* ---- prefix caching across requests -------------------------------------
+ * Full blocks keep the keys and values of a token prefix, and a later request
+ * whose prompt starts with the same tokens reuses them instead of recomputing
+ * them ["PagedAttention: KV cache memory management", section "PagedAttention
+ * vs KV-cache quantization vs prefix caching"; sharing across requests: "vLLM
+ * and PagedAttention", section "Key claims from the paper"]. Off unless
+ * turned on. Policy:
+ *  - a block that fills during kv_seq_append_tokens is registered under the
+ *    key (registration number of the block before it, or -1 for a first
+ *    block; its block_size token ids), unless the key is taken (the first
+ *    registration stays), the block is registered, or the block before it is
+ *    not registered; registration numbers are never reused, so a key names
+ *    one exact token prefix. A kv_seq_append (token ids unknown) ends the
+ *    sequence's registrations;
+ *  - kv_seq_create_prefixed attaches the longest run of leading registered
+ *    blocks of a prompt that ends before the prompt's last token;
+ *  - a registered block whose reference count reaches zero becomes evictable
+ *    (the blocks of one release from the last logical block to the first)
+ *    instead of free; a block taken back by a lookup leaves the evictable list;
+ *  - a new block comes from the free stack, and when it is empty from evicting
+ *    the evictable block released longest ago (its key dropped); appends
+ *    check their need against free plus evictable blocks. */
+
+/* Turns prefix caching on (enable != 0; only while no sequence is live) or
+ * off (every registration dropped, evictable blocks pushed to the free stack
+ * in eviction order, live sequences no longer registered).
+ * Errors: KVP_ERR_INVALID (NULL pool, turning it on with live sequences). */
+KVP_API int kv_pool_set_prefix_caching(kvp_pool* pool, int32_t enable);
+
+/* Creates a sequence for a prompt of n_tokens token ids: its table starts
+ * with the longest run of cached leading blocks of the prompt ending before
+ * its last token (each gains a reference), and its length is that run's
+ * tokens, returned in *cached_tokens. The caller appends
+ * tokens[*cached_tokens:] with kv_seq_append_tokens and writes only their
+ * keys and values. Errors: KVP_ERR_INVALID (NULL arguments, n_tokens < 0,
+ * prefix caching off), KVP_ERR_OOM (host allocation). */
+KVP_API int kv_seq_create_prefixed(kvp_pool* pool, const int32_t* tokens, int32_t n_tokens,
+                                   int64_t* seq_id, int32_t* cached_tokens);
+
+/* kv_seq_append with the token ids given (tokens: host int32 [n_tokens]); on a
+ * pool with prefix caching, blocks that fill are registered (policy above).
+ * Errors: those of kv_seq_append. */
+KVP_API int kv_seq_append_tokens(kvp_pool* pool, int64_t seq, const int32_t* tokens,
+                                 int32_t n_tokens, int64_t* slots_out);
+
+/* The evictable blocks, the one evicted next first. Errors: KVP_ERR_INVALID,
+ * KVP_ERR_CAPACITY (cap too small; *n is set). */
+KVP_API int kv_pool_evictable_list(const kvp_pool* pool, int32_t* out, int32_t cap, int32_t* n);
+
+/* Registered blocks, evictable blocks, and prompt tokens served from the
+ * cache so far. Errors: KVP_ERR_INVALID (NULL argument). */
+KVP_API int kv_pool_prefix_stats(const kvp_pool* pool, int64_t* registered, int64_t* evictable,
+                                 int64_t* hit_tokens);
+
 /* Packs the batch metadata the decode kernels read: block_tables is
  * [num_seqs][max_blocks] (row i = table of seqs[i], padded with -1) and
  * context_lens[i] = length of seqs[i]. Host buffers; copy them to the device.

@@ -92,6 +92,38 @@ class BlockPool:
         check(lib().kv_seq_append_batch(self._h, _i64p(s), len(s), int(n_each), _i64p(out)))
         return out
 
+    def append_tokens(self, seq: int, tokens) -> list[int]:
+        """``append`` with the token ids given (registers filled blocks when prefix
+        caching is on)."""
+        t = np.ascontiguousarray(np.asarray(tokens, dtype=np.int32).reshape(-1))
+        out = np.empty(len(t), dtype=np.int64)
+        check(lib().kv_seq_append_tokens(self._h, seq, _i32p(t) if len(t) else None, len(t),
+                                         _i64p(out) if len(t) else None))
+        return out.tolist()
+
+    # ---- prefix caching ---------------------------------------------------------
+    def set_prefix_caching(self, enable: bool = True) -> None:
+        check(lib().kv_pool_set_prefix_caching(self._h, 1 if enable else 0))
+
+    def create_prefixed(self, tokens) -> tuple[int, int]:
+        """A sequence holding the longest cached prefix of ``tokens``: (id, cached tokens)."""
+        t = np.ascontiguousarray(np.asarray(tokens, dtype=np.int32).reshape(-1))
+        sid, cached = C.c_int64(), C.c_int32()
+        check(lib().kv_seq_create_prefixed(self._h, _i32p(t) if len(t) else None, len(t),
+                                           C.byref(sid), C.byref(cached)))
+        return sid.value, cached.value
+
+    def evictable(self) -> list[int]:
+        out = np.empty(self.num_blocks, dtype=np.int32)
+        n = C.c_int32()
+        check(lib().kv_pool_evictable_list(self._h, _i32p(out), self.num_blocks, C.byref(n)))
+        return out[:n.value].tolist()
+
+    def prefix_stats(self) -> dict:
+        r, e, h = C.c_int64(), C.c_int64(), C.c_int64()
+        check(lib().kv_pool_prefix_stats(self._h, C.byref(r), C.byref(e), C.byref(h)))
+        return {"registered": r.value, "evictable": e.value, "hit_tokens": h.value}
+
     def fork(self, parent: int) -> int:
         cid = C.c_int64()
         check(lib().kv_seq_fork(self._h, parent, C.byref(cid)))

@@ -84,6 +84,11 @@ SIGNATURES = {
                                         vp]),
     "paged_attention_decode_fp8": (C.c_int, [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32,
                                              i32, i32, i32, f32, i32, vp, sz, vp, i32, vp]),
+    "kv_pool_set_prefix_caching": (C.c_int, [vp, i32]),
+    "kv_seq_create_prefixed": (C.c_int, [vp, P_i32, i32, P_i64, P_i32]),
+    "kv_seq_append_tokens": (C.c_int, [vp, i64, P_i32, i32, P_i64]),
+    "kv_pool_evictable_list": (C.c_int, [vp, P_i32, i32, P_i32]),
+    "kv_pool_prefix_stats": (C.c_int, [vp, P_i64, P_i64, P_i64]),
     "kv_decode_group_plan": (C.c_int, [P_i32, P_i32, i32, i32, i32, i32, i32, i32, i32, i32, P_i32,
                                        sz]),
     "paged_attention_decode_noalloc": (C.c_int, [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,

@@ -19,9 +19,27 @@
 //
 // Every mutating call first checks that it can succeed (block need vs free
 // count, ids), then mutates, so a failed call changes nothing.
+//
+// Prefix caching across requests (off unless kv_pool_set_prefix_caching turns
+// it on): full blocks keep the keys and values of a token prefix that a later
+// request with the same prefix reuses ["PagedAttention: KV cache memory
+// management", section "PagedAttention vs KV-cache quantization vs prefix
+// caching"; sharing across requests: "vLLM and PagedAttention", section "Key
+// claims from the paper"]. Policy: a block that fills during
+// kv_seq_append_tokens is registered under the key (registration number of
+// the block before it, or -1; its token ids), unless the key is taken, the
+// block is registered or the block before it is not; registration numbers
+// are never reused, so a key names one exact token prefix. kv_seq_create_prefixed
+// attaches the longest run of leading registered blocks that ends before the
+// prompt's last token. A registered block whose count reaches zero becomes
+// evictable (the blocks of one release from the last logical one to the
+// first) instead of free; a new block comes from the free stack, else from
+// evicting the evictable block released longest ago.
 
 #include <cstdint>
 #include <cstring>
+#include <iterator>
+#include <list>
 #include <new>
 #include <unordered_map>
 #include <utility>
@@ -40,11 +58,96 @@ struct kvp_pool {
   struct Seq {
     std::vector<int32_t> table;
     int32_t len = 0;
+    // prefix caching: the token ids appended so far, while every append gave them
+    std::vector<int32_t> tokens;
+    bool tracked = true;
   };
   std::unordered_map<int64_t, Seq> seqs;
   std::vector<std::pair<int32_t, int32_t>> pending;  // (src, dst) copy-on-write pairs
   int64_t next_seq = 0;
   int64_t cow_total = 0;
+
+  // ---- prefix caching
+  struct KeyHash {
+    size_t operator()(const std::vector<int64_t>& k) const noexcept {
+      uint64_t h = 1469598103934665603ull;  // FNV-1a over the words
+      for (int64_t w : k) {
+        h ^= uint64_t(w);
+        h *= 1099511628211ull;
+      }
+      return size_t(h);
+    }
+  };
+  bool prefix_caching = false;
+  std::unordered_map<std::vector<int64_t>, int32_t, KeyHash> block_of;  // key -> block
+  std::vector<std::vector<int64_t>> key_of;   // per block: its key, empty if unregistered
+  std::vector<int64_t> reg_of;                // per block: registration number, -1 if none
+  int64_t next_reg = 0;
+  std::list<int32_t> evictable;               // front: evicted next
+  std::vector<std::list<int32_t>::iterator> evict_pos;
+  std::vector<char> in_evict;
+  int64_t hit_tokens = 0;
+
+  int64_t available() const { return int64_t(free_stack.size()) + int64_t(evictable.size()); }
+
+  // A block for a new table entry: the free stack first, else the evictable
+  // block released longest ago (its key dropped).
+  int32_t take_block() {
+    if (!free_stack.empty()) {
+      const int32_t b = free_stack.back();
+      free_stack.pop_back();
+      return b;
+    }
+    const int32_t b = evictable.front();
+    evictable.pop_front();
+    in_evict[b] = 0;
+    block_of.erase(key_of[b]);
+    key_of[b].clear();
+    key_of[b].shrink_to_fit();
+    reg_of[b] = -1;
+    return b;
+  }
+
+  // Block bi of s has just filled: register it (policy above). Registration is
+  // a cache, so a host allocation failure here only skips it.
+  void maybe_register(const Seq& s, int32_t bi) {
+    const int32_t blk = s.table[bi];
+    if (reg_of[blk] >= 0) return;
+    const int64_t parent = bi == 0 ? -1 : reg_of[s.table[bi - 1]];
+    if (bi > 0 && parent < 0) return;
+    try {
+      std::vector<int64_t> key;
+      key.reserve(size_t(block_size) + 1);
+      key.push_back(parent);
+      for (int32_t i = 0; i < block_size; ++i) key.push_back(s.tokens[size_t(bi) * block_size + i]);
+      if (block_of.count(key)) return;
+      key_of[blk] = key;
+      block_of.emplace(std::move(key), blk);
+      reg_of[blk] = next_reg++;
+    } catch (...) {
+      key_of[blk].clear();
+    }
+  }
+
+  // Drops one reference of each block of a released table (logical order);
+  // blocks reaching zero go to the free stack, or become evictable if
+  // registered. Everything that allocates happens first (it may throw), then
+  // the pool changes without allocating.
+  void drop_table(const std::vector<int32_t>& table) {
+    std::list<int32_t> newly;  // the blocks to become evictable, last logical block first
+    for (int32_t b : table)
+      if (rc[b] == 1 && prefix_caching && reg_of[b] >= 0) newly.push_front(b);
+    free_stack.reserve(free_stack.size() + table.size());
+    for (int32_t b : table) {
+      if (--rc[b] != 0) continue;
+      if (!(prefix_caching && reg_of[b] >= 0)) free_stack.push_back(b);
+    }
+    if (newly.empty()) return;
+    for (int32_t b : newly) in_evict[b] = 1;
+    auto first = newly.begin();  // stays valid: splice moves the nodes
+    evictable.splice(evictable.end(), newly);
+    for (auto it = first; it != evictable.end(); ++it) evict_pos[*it] = it;
+  }
 
   Seq* find(int64_t id) {
     auto it = seqs.find(id);
@@ -64,19 +167,23 @@ struct kvp_pool {
     return need;
   }
 
-  // Appends n tokens; the caller has checked that the free list suffices.
-  void append_unchecked(Seq& s, int32_t n, int64_t* slots) {
+  // Appends n tokens (their ids, or null if unknown); the caller has checked
+  // that free and evictable blocks suffice and reserved s.tokens when given.
+  void append_unchecked(Seq& s, int32_t n, int64_t* slots, const int32_t* ids = nullptr) {
+    const bool track = prefix_caching && s.tracked && ids;
+    if (prefix_caching && !ids) {  // later tokens unknown: no more registrations
+      s.tracked = false;
+      s.tokens.clear();
+    }
     for (int32_t i = 0; i < n; ++i) {
       const int32_t pos = s.len;
       if (pos % block_size == 0) {
-        const int32_t b = free_stack.back();
-        free_stack.pop_back();
+        const int32_t b = take_block();
         rc[b] = 1;
         s.table.push_back(b);
       } else if (rc[s.table.back()] > 1) {
         const int32_t src = s.table.back();
-        const int32_t dst = free_stack.back();
-        free_stack.pop_back();
+        const int32_t dst = take_block();
         pending.emplace_back(src, dst);
         ++cow_total;
         rc[src] -= 1;
@@ -85,6 +192,10 @@ struct kvp_pool {
       }
       slots[i] = int64_t(s.table[pos / block_size]) * block_size + pos % block_size;
       s.len = pos + 1;
+      if (track) {
+        s.tokens.push_back(ids[i]);
+        if (s.len % block_size == 0) maybe_register(s, pos / block_size);
+      }
     }
   }
 };
@@ -127,6 +238,10 @@ int kv_pool_create(int32_t num_blocks, int32_t block_size, int32_t num_kv_heads,
     p->dtype = dtype;
     p->rc.assign(num_blocks, 0);
     p->free_stack.resize(num_blocks);
+    p->key_of.resize(num_blocks);
+    p->reg_of.assign(num_blocks, -1);
+    p->evict_pos.resize(num_blocks);
+    p->in_evict.assign(num_blocks, 0);
     if (free_order) {
       std::vector<char> seen(num_blocks, 0);
       for (int32_t i = 0; i < num_blocks; ++i) {
@@ -220,9 +335,9 @@ int kv_seq_append(kvp_pool* pool, int64_t seq, int32_t n_tokens, int64_t* slots_
   if (int64_t(s->len) + n_tokens > INT32_MAX) return fail(KVP_ERR_INVALID, "kv_seq_append: length overflow");
   const int32_t last_rc = s->table.empty() ? 0 : pool->rc[s->table.back()];
   const int64_t need = pool->need_for(*s, n_tokens, last_rc);
-  if (need > int64_t(pool->free_stack.size()))
-    return fail(KVP_ERR_OOM, "kv_seq_append: need %lld blocks, %zu free", (long long)need,
-                pool->free_stack.size());
+  if (need > pool->available())
+    return fail(KVP_ERR_OOM, "kv_seq_append: need %lld blocks, %lld free or evictable",
+                (long long)need, (long long)pool->available());
   try {
     s->table.reserve(s->table.size() + size_t(need));
     pool->pending.reserve(pool->pending.size() + 1);
@@ -230,6 +345,126 @@ int kv_seq_append(kvp_pool* pool, int64_t seq, int32_t n_tokens, int64_t* slots_
     return fail(KVP_ERR_OOM, "kv_seq_append: host allocation failed");
   }
   pool->append_unchecked(*s, n_tokens, slots_out);
+  return KVP_OK;
+}
+
+int kv_seq_append_tokens(kvp_pool* pool, int64_t seq, const int32_t* tokens, int32_t n_tokens,
+                         int64_t* slots_out) {
+  if (!pool) return fail(KVP_ERR_INVALID, "kv_seq_append_tokens: NULL pool");
+  kvp_pool::Seq* s = pool->find(seq);
+  if (!s) return fail(KVP_ERR_NO_SEQ, "kv_seq_append_tokens: no live sequence %lld", (long long)seq);
+  if (n_tokens < 0) return fail(KVP_ERR_INVALID, "kv_seq_append_tokens: n_tokens < 0");
+  if (n_tokens > 0 && (!slots_out || !tokens))
+    return fail(KVP_ERR_INVALID, "kv_seq_append_tokens: NULL argument");
+  if (int64_t(s->len) + n_tokens > INT32_MAX)
+    return fail(KVP_ERR_INVALID, "kv_seq_append_tokens: length overflow");
+  const int32_t last_rc = s->table.empty() ? 0 : pool->rc[s->table.back()];
+  const int64_t need = pool->need_for(*s, n_tokens, last_rc);
+  if (need > pool->available())
+    return fail(KVP_ERR_OOM, "kv_seq_append_tokens: need %lld blocks, %lld free or evictable",
+                (long long)need, (long long)pool->available());
+  try {
+    s->table.reserve(s->table.size() + size_t(need));
+    pool->pending.reserve(pool->pending.size() + 1);
+    if (pool->prefix_caching && s->tracked) s->tokens.reserve(s->tokens.size() + size_t(n_tokens));
+  } catch (...) {
+    return fail(KVP_ERR_OOM, "kv_seq_append_tokens: host allocation failed");
+  }
+  static const int32_t kNone = 0;
+  pool->append_unchecked(*s, n_tokens, slots_out, tokens ? tokens : &kNone);
+  return KVP_OK;
+}
+
+int kv_pool_set_prefix_caching(kvp_pool* pool, int32_t enable) {
+  if (!pool) return fail(KVP_ERR_INVALID, "kv_pool_set_prefix_caching: NULL pool");
+  if (enable) {
+    if (!pool->prefix_caching && !pool->seqs.empty())
+      return fail(KVP_ERR_INVALID, "kv_pool_set_prefix_caching: turn it on while no sequence is live");
+    pool->prefix_caching = true;
+    return KVP_OK;
+  }
+  // off: every registration is dropped; evictable blocks become free (front first)
+  try {
+    pool->free_stack.reserve(pool->free_stack.size() + pool->evictable.size());
+  } catch (...) {
+    return fail(KVP_ERR_OOM, "kv_pool_set_prefix_caching: host allocation failed");
+  }
+  for (int32_t b : pool->evictable) {
+    pool->free_stack.push_back(b);
+    pool->in_evict[b] = 0;
+  }
+  pool->evictable.clear();
+  pool->block_of.clear();
+  for (int32_t b = 0; b < pool->num_blocks; ++b) {
+    pool->key_of[b].clear();
+    pool->reg_of[b] = -1;
+  }
+  for (auto& kv : pool->seqs) {
+    kv.second.tracked = false;
+    kv.second.tokens.clear();
+  }
+  pool->prefix_caching = false;
+  return KVP_OK;
+}
+
+int kv_seq_create_prefixed(kvp_pool* pool, const int32_t* tokens, int32_t n_tokens, int64_t* seq_id,
+                           int32_t* cached_tokens) {
+  if (!pool || !seq_id || !cached_tokens)
+    return fail(KVP_ERR_INVALID, "kv_seq_create_prefixed: NULL argument");
+  if (n_tokens < 0 || (n_tokens > 0 && !tokens))
+    return fail(KVP_ERR_INVALID, "kv_seq_create_prefixed: bad tokens");
+  if (!pool->prefix_caching) return fail(KVP_ERR_INVALID, "kv_seq_create_prefixed: prefix caching is off");
+  const int32_t bs = pool->block_size;
+  kvp_pool::Seq s;
+  try {
+    std::vector<int64_t> key(size_t(bs) + 1);
+    int64_t parent = -1;
+    for (int32_t i = 0; int64_t(i + 1) * bs <= int64_t(n_tokens) - 1; ++i) {
+      key[0] = parent;
+      for (int32_t j = 0; j < bs; ++j) key[size_t(j) + 1] = tokens[int64_t(i) * bs + j];
+      auto it = pool->block_of.find(key);
+      if (it == pool->block_of.end()) break;
+      s.table.push_back(it->second);
+      parent = pool->reg_of[it->second];
+    }
+    s.len = int32_t(s.table.size()) * bs;
+    s.tokens.assign(tokens, tokens + s.len);
+    pool->seqs.emplace(pool->next_seq, std::move(s));
+  } catch (...) {
+    return fail(KVP_ERR_OOM, "kv_seq_create_prefixed: host allocation failed");
+  }
+  const kvp_pool::Seq& made = pool->seqs[pool->next_seq];
+  for (int32_t b : made.table) {
+    if (pool->rc[b] == 0 && pool->in_evict[b]) {
+      pool->evictable.erase(pool->evict_pos[b]);
+      pool->in_evict[b] = 0;
+    }
+    pool->rc[b] += 1;
+  }
+  pool->hit_tokens += made.len;
+  *cached_tokens = made.len;
+  *seq_id = pool->next_seq++;
+  return KVP_OK;
+}
+
+int kv_pool_evictable_list(const kvp_pool* pool, int32_t* out, int32_t cap, int32_t* n) {
+  if (!pool || !n) return fail(KVP_ERR_INVALID, "kv_pool_evictable_list: NULL argument");
+  const int32_t cnt = int32_t(pool->evictable.size());
+  *n = cnt;
+  if (cap < cnt || (cnt && !out))
+    return fail(KVP_ERR_CAPACITY, "kv_pool_evictable_list: cap %d < %d", cap, cnt);
+  int32_t i = 0;
+  for (int32_t b : pool->evictable) out[i++] = b;
+  return KVP_OK;
+}
+
+int kv_pool_prefix_stats(const kvp_pool* pool, int64_t* registered, int64_t* evictable,
+                         int64_t* hit_tokens) {
+  if (!pool || !registered || !evictable || !hit_tokens)
+    return fail(KVP_ERR_INVALID, "kv_pool_prefix_stats: NULL argument");
+  *registered = int64_t(pool->block_of.size());
+  *evictable = int64_t(pool->evictable.size());
+  *hit_tokens = pool->hit_tokens;
   return KVP_OK;
 }
 
@@ -260,9 +495,9 @@ int kv_seq_append_batch(kvp_pool* pool, const int64_t* seqs, int32_t num_seqs, i
     }
     need += pool->need_for(*s, n_each, last_rc);
   }
-  if (need > int64_t(pool->free_stack.size()))
-    return fail(KVP_ERR_OOM, "kv_seq_append_batch: need %lld blocks, %zu free", (long long)need,
-                pool->free_stack.size());
+  if (need > pool->available())
+    return fail(KVP_ERR_OOM, "kv_seq_append_batch: need %lld blocks, %lld free or evictable",
+                (long long)need, (long long)pool->available());
   for (int32_t i = 0; i < num_seqs; ++i)
     pool->append_unchecked(*ptrs[i], n_each, slots_out + int64_t(i) * n_each);
   return KVP_OK;
@@ -287,8 +522,10 @@ int kv_seq_release(kvp_pool* pool, int64_t seq) {
   if (!pool) return fail(KVP_ERR_INVALID, "kv_seq_release: NULL pool");
   auto it = pool->seqs.find(seq);
   if (it == pool->seqs.end()) return fail(KVP_ERR_NO_SEQ, "kv_seq_release: no live sequence %lld", (long long)seq);
-  for (int32_t b : it->second.table) {
-    if (--pool->rc[b] == 0) pool->free_stack.push_back(b);
+  try {
+    pool->drop_table(it->second.table);
+  } catch (...) {
+    return fail(KVP_ERR_OOM, "kv_seq_release: host allocation failed");
   }
   pool->seqs.erase(it);
   return KVP_OK;
