@@ -1004,9 +1004,82 @@ def run_fp8(args):
     print(json.dumps(res), flush=True)
 
 
+def run_reference_sampled(args, world):
+    """Reference arm of the prefill and E4M3 workloads: the matching oracle
+    (``attention.paged_prefill`` / ``fp8.paged_decode``) on one sequence of the
+    workload per step, longest first, inputs drawn before the timed region."""
+    from oracle import attention, fp8
+
+    fp8_case = args.workload in FP8_WORKLOADS
+    base, T = ("opt13b", 1) if fp8_case else PREFILL_WORKLOADS[args.workload]
+    if base == "prompt512":
+        g = workloads.Geometry(40, 40, 128, 16, "f16")
+        lens = np.full(64, 512, np.int64)
+    else:
+        wl = workloads.by_name(base)
+        g = wl.geometry
+        lens = np.asarray(wl.info["context_lens"], np.int64)
+    Hq, Hkv, D, bs = g.num_q_heads, g.num_kv_heads, g.head_dim, g.block_size
+    rng = np.random.default_rng(6001)
+    order = np.argsort(lens)[::-1]
+    n = args.warmup + args.steps
+    cases = []
+    for k in range(n):
+        L = int(lens[order[k % len(order)]])
+        nb = -(-L // bs)
+        table = np.arange(nb, dtype=np.int32)[None]
+        if fp8_case:
+            kc = rng.integers(0, 256, (nb, Hkv, bs, D), dtype=np.uint8)
+            vc = rng.integers(0, 256, (nb, Hkv, bs, D), dtype=np.uint8)
+            kc[(kc & 0x7F) == 0x7F] = 0x3F
+            vc[(vc & 0x7F) == 0x7F] = 0x3F
+            nbytes = L * Hkv * D * 2 + Hq * D * 4 + 4 * nb + 4
+        else:
+            kc = rng.standard_normal((nb, Hkv, bs, D))
+            vc = rng.standard_normal((nb, Hkv, bs, D))
+            nbytes = L * Hkv * D * g.elem_bytes * 2 + T * Hq * D * g.elem_bytes * 2 + 4 * nb + 4
+        q = rng.standard_normal((1, T, Hq, D) if not fp8_case else (1, Hq, D))
+        cases.append((L, table, kc, vc, q, nbytes))
+    ks = np.full(Hkv, 1 / 448, np.float32)
+    vs = np.full(Hkv, 2 / 448, np.float32)
+    scale = 1 / math.sqrt(D)
+
+    def one(c):
+        L, table, kc, vc, q, nbytes = c
+        if fp8_case:
+            fp8.paged_decode(q, kc, vc, table, [L], scale, bs, ks, vs)
+        else:
+            attention.paged_prefill(q, kc, vc, table, [L], scale, bs)
+        return nbytes
+
+    for c in cases[:args.warmup]:
+        one(c)
+    t0 = time.perf_counter()
+    nbytes = sum(one(c) for c in cases[args.warmup:])
+    el = time.perf_counter() - t0
+    value = nbytes / el / 1e9
+    what = "one sequence's E4M3 decode" if fp8_case else f"one sequence's {T}-token prefill"
+    res = {
+        "metric": METRIC, "value": round(value, 4), "unit": UNIT, "impl": "reference",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(el * 1e3 / max(1, args.steps), 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": args.workload, "name": args.workload},
+        "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "kind": "oracle",
+                         "cores": len(os.sched_getaffinity(0)), "blas_threads": cpu_threads(),
+                         "sample": f"{what} per step (longest contexts first)"},
+        "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(res), flush=True)
+
+
 def run_reference(args, world, rank):
     """The oracle as the reference arm: each step is a bounded sample of the workload."""
     if rank != 0:
+        return
+    if args.workload in FP8_WORKLOADS or args.workload in PREFILL_WORKLOADS:
+        run_reference_sampled(args, world)
         return
     from oracle.replay import OracleReplay
 
