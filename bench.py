@@ -1144,6 +1144,10 @@ def main():
         run_reference(args, int(os.environ.get("WORLD_SIZE", "1")),
                       int(os.environ.get("RANK", "0")))
         return
+    single_gpu = args.workload in SCHEDULE_WORKLOADS or args.workload in PREFILL_WORKLOADS \
+        or args.workload in FP8_WORKLOADS
+    if single_gpu and int(os.environ.get("RANK", "0")) != 0:
+        return  # one-GPU workloads: rank 0 runs and prints, the other ranks do nothing
     if args.workload in SCHEDULE_WORKLOADS:
         run_schedule(args)
         return
