@@ -215,6 +215,14 @@ KVP_API int kv_seq_create_prefixed(kvp_pool* pool, const int32_t* tokens, int32_
 KVP_API int kv_seq_append_tokens(kvp_pool* pool, int64_t seq, const int32_t* tokens,
                                  int32_t n_tokens, int64_t* slots_out);
 
+/* kv_seq_append_batch with token ids: tokens is host int32 [num_seqs][n_each],
+ * row i for seqs[i]; the appends run in batch order, as num_seqs calls of
+ * kv_seq_append_tokens would, after one check of the whole batch's need. The
+ * decode steps of a serving loop use it so that generated blocks are
+ * registered too. Errors: those of kv_seq_append_batch. */
+KVP_API int kv_seq_append_tokens_batch(kvp_pool* pool, const int64_t* seqs, int32_t num_seqs,
+                                       int32_t n_each, const int32_t* tokens, int64_t* slots_out);
+
 /* The evictable blocks, the one evicted next first. Errors: KVP_ERR_INVALID,
  * KVP_ERR_CAPACITY (cap too small; *n is set). */
 KVP_API int kv_pool_evictable_list(const kvp_pool* pool, int32_t* out, int32_t cap, int32_t* n);

@@ -101,6 +101,17 @@ class BlockPool:
                                          _i64p(out) if len(t) else None))
         return out.tolist()
 
+    def append_tokens_batch(self, seqs, tokens, out: np.ndarray | None = None) -> np.ndarray:
+        """``append_batch`` with token ids ``tokens [len(seqs), n_each]``."""
+        s = np.ascontiguousarray(np.asarray(seqs, dtype=np.int64))
+        t = np.ascontiguousarray(np.asarray(tokens, dtype=np.int32).reshape(len(s), -1))
+        n_each = t.shape[1] if len(s) else 0
+        if out is None:
+            out = np.empty(len(s) * n_each, dtype=np.int64)
+        check(lib().kv_seq_append_tokens_batch(self._h, _i64p(s), len(s), int(n_each), _i32p(t),
+                                               _i64p(out)))
+        return out
+
     # ---- prefix caching ---------------------------------------------------------
     def set_prefix_caching(self, enable: bool = True) -> None:
         check(lib().kv_pool_set_prefix_caching(self._h, 1 if enable else 0))

@@ -87,6 +87,7 @@ SIGNATURES = {
     "kv_pool_set_prefix_caching": (C.c_int, [vp, i32]),
     "kv_seq_create_prefixed": (C.c_int, [vp, P_i32, i32, P_i64, P_i32]),
     "kv_seq_append_tokens": (C.c_int, [vp, i64, P_i32, i32, P_i64]),
+    "kv_seq_append_tokens_batch": (C.c_int, [vp, P_i64, i32, i32, P_i32, P_i64]),
     "kv_pool_evictable_list": (C.c_int, [vp, P_i32, i32, P_i32]),
     "kv_pool_prefix_stats": (C.c_int, [vp, P_i64, P_i64, P_i64]),
     "kv_decode_group_plan": (C.c_int, [P_i32, P_i32, i32, i32, i32, i32, i32, i32, i32, i32, P_i32,

@@ -468,12 +468,15 @@ int kv_pool_prefix_stats(const kvp_pool* pool, int64_t* registered, int64_t* evi
   return KVP_OK;
 }
 
-int kv_seq_append_batch(kvp_pool* pool, const int64_t* seqs, int32_t num_seqs, int32_t n_each,
-                        int64_t* slots_out) {
-  if (!pool) return fail(KVP_ERR_INVALID, "kv_seq_append_batch: NULL pool");
-  if (num_seqs < 0 || n_each < 0) return fail(KVP_ERR_INVALID, "kv_seq_append_batch: negative size");
+// kv_seq_append_batch and kv_seq_append_tokens_batch: one check of the whole
+// batch's block need, then the appends in order (ids: null, or n_each token
+// ids per sequence).
+static int append_batch_impl(kvp_pool* pool, const int64_t* seqs, int32_t num_seqs, int32_t n_each,
+                             const int32_t* ids, int64_t* slots_out, const char* who) {
+  if (!pool) return fail(KVP_ERR_INVALID, "%s: NULL pool", who);
+  if (num_seqs < 0 || n_each < 0) return fail(KVP_ERR_INVALID, "%s: negative size", who);
   if (num_seqs == 0 || n_each == 0) return KVP_OK;
-  if (!seqs || !slots_out) return fail(KVP_ERR_INVALID, "kv_seq_append_batch: NULL argument");
+  if (!seqs || !slots_out) return fail(KVP_ERR_INVALID, "%s: NULL argument", who);
   // Exact block need of the whole batch: a copy-on-write by an earlier
   // sequence lowers the count a later sharer of the same last block sees.
   std::unordered_map<int32_t, int32_t> rc_after;
@@ -481,11 +484,11 @@ int kv_seq_append_batch(kvp_pool* pool, const int64_t* seqs, int32_t num_seqs, i
   int64_t need = 0;
   for (int32_t i = 0; i < num_seqs; ++i) {
     kvp_pool::Seq* s = pool->find(seqs[i]);
-    if (!s) return fail(KVP_ERR_NO_SEQ, "kv_seq_append_batch: no live sequence %lld", (long long)seqs[i]);
+    if (!s) return fail(KVP_ERR_NO_SEQ, "%s: no live sequence %lld", who, (long long)seqs[i]);
     for (int32_t j = 0; j < i; ++j)
-      if (ptrs[j] == s) return fail(KVP_ERR_INVALID, "kv_seq_append_batch: duplicate sequence");
+      if (ptrs[j] == s) return fail(KVP_ERR_INVALID, "%s: duplicate sequence", who);
     ptrs[i] = s;
-    if (int64_t(s->len) + n_each > INT32_MAX) return fail(KVP_ERR_INVALID, "kv_seq_append_batch: overflow");
+    if (int64_t(s->len) + n_each > INT32_MAX) return fail(KVP_ERR_INVALID, "%s: overflow", who);
     int32_t last_rc = 0;
     if (!s->table.empty()) {
       const int32_t last = s->table.back();
@@ -496,11 +499,35 @@ int kv_seq_append_batch(kvp_pool* pool, const int64_t* seqs, int32_t num_seqs, i
     need += pool->need_for(*s, n_each, last_rc);
   }
   if (need > pool->available())
-    return fail(KVP_ERR_OOM, "kv_seq_append_batch: need %lld blocks, %lld free or evictable",
-                (long long)need, (long long)pool->available());
+    return fail(KVP_ERR_OOM, "%s: need %lld blocks, %lld free or evictable", who, (long long)need,
+                (long long)pool->available());
+  try {
+    for (int32_t i = 0; i < num_seqs; ++i) {
+      ptrs[i]->table.reserve(ptrs[i]->table.size() + size_t(n_each / pool->block_size + 2));
+      if (ids && pool->prefix_caching && ptrs[i]->tracked)
+        ptrs[i]->tokens.reserve(ptrs[i]->tokens.size() + size_t(n_each));
+    }
+    pool->pending.reserve(pool->pending.size() + size_t(num_seqs));
+  } catch (...) {
+    return fail(KVP_ERR_OOM, "%s: host allocation failed", who);
+  }
   for (int32_t i = 0; i < num_seqs; ++i)
-    pool->append_unchecked(*ptrs[i], n_each, slots_out + int64_t(i) * n_each);
+    pool->append_unchecked(*ptrs[i], n_each, slots_out + int64_t(i) * n_each,
+                           ids ? ids + int64_t(i) * n_each : nullptr);
   return KVP_OK;
+}
+
+int kv_seq_append_batch(kvp_pool* pool, const int64_t* seqs, int32_t num_seqs, int32_t n_each,
+                        int64_t* slots_out) {
+  return append_batch_impl(pool, seqs, num_seqs, n_each, nullptr, slots_out, "kv_seq_append_batch");
+}
+
+int kv_seq_append_tokens_batch(kvp_pool* pool, const int64_t* seqs, int32_t num_seqs,
+                               int32_t n_each, const int32_t* tokens, int64_t* slots_out) {
+  if (num_seqs > 0 && n_each > 0 && !tokens)
+    return fail(KVP_ERR_INVALID, "kv_seq_append_tokens_batch: NULL tokens");
+  return append_batch_impl(pool, seqs, num_seqs, n_each, tokens, slots_out,
+                           "kv_seq_append_tokens_batch");
 }
 
 int kv_seq_fork(kvp_pool* pool, int64_t parent, int64_t* child) {

@@ -1,9 +1,11 @@
 """The library's prefix caching (kv_pool_set_prefix_caching, kv_seq_create_prefixed,
-kv_seq_append_tokens, evictable blocks) against the oracle's PrefixCachingBlockManager,
+kv_seq_append_tokens and its batch form, evictable blocks) against the oracle's PrefixCachingBlockManager,
 operation by operation on random request streams: block tables, slots, reference
 counts, the free stack, the evictable list, copy-on-write pairs and the cached-token
 counts must agree exactly. Also: the switch's rules, and that a pool without prefix
 caching behaves as before."""
+
+import copy
 
 import numpy as np
 import pytest
@@ -66,6 +68,20 @@ def test_random_streams_match_the_oracle(seed, NB, bs):
                     lib.append(s, len(tok)) if plain else lib.append_tokens(s, tok)
             else:
                 assert (lib.append(s, len(tok)) if plain else lib.append_tokens(s, tok)) == sl1
+        elif op < 0.64:  # a decode step of several sequences at once
+            pick = sorted(rng.choice(live, size=min(len(live), int(rng.integers(1, 5))),
+                                     replace=False).tolist())
+            n_each = int(rng.integers(1, 3))
+            tok = rng.integers(0, 4, size=(len(pick), n_each))
+            trial = copy.deepcopy(ora)
+            try:
+                want = [x for s, t in zip(pick, tok) for x in trial.append_tokens(s, t.tolist())]
+            except OutOfBlocks:
+                with pytest.raises(kvp.KvpError):
+                    lib.append_tokens_batch(pick, tok)
+            else:
+                assert lib.append_tokens_batch(pick, tok).tolist() == want
+                ora = trial
         elif op < 0.68:
             s = live[int(rng.integers(0, len(live)))]
             assert lib.fork(s) == ora.fork(s)
