@@ -47,6 +47,14 @@
 
 #include "../status.h"
 
+// Room for `extra` more elements, growing the capacity at least twofold, so a
+// vector that gains a few elements per call is not copied on every call.
+template <typename V>
+static void reserve_more(V& v, size_t extra) {
+  const size_t want = v.size() + extra;
+  if (v.capacity() < want) v.reserve(want > 2 * v.capacity() ? want : 2 * v.capacity());
+}
+
 struct kvp_pool {
   int32_t num_blocks = 0;
   int32_t block_size = 0;
@@ -339,8 +347,8 @@ int kv_seq_append(kvp_pool* pool, int64_t seq, int32_t n_tokens, int64_t* slots_
     return fail(KVP_ERR_OOM, "kv_seq_append: need %lld blocks, %lld free or evictable",
                 (long long)need, (long long)pool->available());
   try {
-    s->table.reserve(s->table.size() + size_t(need));
-    pool->pending.reserve(pool->pending.size() + 1);
+    reserve_more(s->table, size_t(need));
+    reserve_more(pool->pending, 1);
   } catch (...) {
     return fail(KVP_ERR_OOM, "kv_seq_append: host allocation failed");
   }
@@ -364,9 +372,9 @@ int kv_seq_append_tokens(kvp_pool* pool, int64_t seq, const int32_t* tokens, int
     return fail(KVP_ERR_OOM, "kv_seq_append_tokens: need %lld blocks, %lld free or evictable",
                 (long long)need, (long long)pool->available());
   try {
-    s->table.reserve(s->table.size() + size_t(need));
-    pool->pending.reserve(pool->pending.size() + 1);
-    if (pool->prefix_caching && s->tracked) s->tokens.reserve(s->tokens.size() + size_t(n_tokens));
+    reserve_more(s->table, size_t(need));
+    reserve_more(pool->pending, 1);
+    if (pool->prefix_caching && s->tracked) reserve_more(s->tokens, size_t(n_tokens));
   } catch (...) {
     return fail(KVP_ERR_OOM, "kv_seq_append_tokens: host allocation failed");
   }
@@ -503,11 +511,10 @@ static int append_batch_impl(kvp_pool* pool, const int64_t* seqs, int32_t num_se
                 (long long)pool->available());
   try {
     for (int32_t i = 0; i < num_seqs; ++i) {
-      ptrs[i]->table.reserve(ptrs[i]->table.size() + size_t(n_each / pool->block_size + 2));
-      if (ids && pool->prefix_caching && ptrs[i]->tracked)
-        ptrs[i]->tokens.reserve(ptrs[i]->tokens.size() + size_t(n_each));
+      reserve_more(ptrs[i]->table, size_t(n_each / pool->block_size + 2));
+      if (ids && pool->prefix_caching && ptrs[i]->tracked) reserve_more(ptrs[i]->tokens, size_t(n_each));
     }
-    pool->pending.reserve(pool->pending.size() + size_t(num_seqs));
+    reserve_more(pool->pending, size_t(num_seqs));
   } catch (...) {
     return fail(KVP_ERR_OOM, "%s: host allocation failed", who);
   }
