@@ -140,7 +140,9 @@ KVP_API int kv_seq_create(kvp_pool* pool, int64_t* seq_id);
 KVP_API int kv_seq_append(kvp_pool* pool, int64_t seq, int32_t n_tokens, int64_t* slots_out);
 
 /* Appends n_each tokens to every sequence of seqs[0..num_seqs), in that order;
- * the result equals num_seqs successive kv_seq_append calls.
+ * the result equals num_seqs successive kv_seq_append calls (with prefix
+ * caching on, that ends the sequences' registrations: the token-carrying form
+ * is kv_seq_append_tokens_batch).
  * slots_out[i*n_each + j] is token j of seqs[i]. All or nothing: on
  * KVP_ERR_OOM / KVP_ERR_NO_SEQ nothing changes. */
 KVP_API int kv_seq_append_batch(kvp_pool* pool, const int64_t* seqs, int32_t num_seqs,
@@ -151,7 +153,8 @@ KVP_API int kv_seq_append_batch(kvp_pool* pool, const int64_t* seqs, int32_t num
 KVP_API int kv_seq_fork(kvp_pool* pool, int64_t parent, int64_t* child);
 
 /* Ends `seq`: each block of its table, in logical order, loses one reference;
- * a block that reaches zero is pushed onto the free list. */
+ * a block that reaches zero is pushed onto the free list (with prefix caching
+ * on, a registered block becomes evictable instead: see below). */
 KVP_API int kv_seq_release(kvp_pool* pool, int64_t seq);
 
 /* Length (tokens) of `seq`. */
