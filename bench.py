@@ -498,8 +498,164 @@ def run_ours(args, world, rank, local):
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         res["cpu_baseline"] = cpu_baseline(wl, budget_s=args.cpu_seconds)
+    if rank == 0 and world == 1 and not args.headline_only:
+        del reps, qs, kn, vn, ws, out
+        release_memory()
+        # the same decode call over a window long enough for the clock sampler, and
+        # one record per other workload, each measured as its own --workload run is
+        res["decode_window"] = decode_record(wl.name, device, calls=DECODE_WINDOW_CALLS)
+        release_memory()
+        res["workloads"] = workload_records(args, device)
     if rank == 0:
         print(json.dumps(res), flush=True)
+
+
+def release_memory():
+    import gc
+
+    import torch
+
+    gc.collect()
+    torch.cuda.empty_cache()
+
+
+def l2_flusher(device):
+    """Before each timed call: a 256 MB write, then a 256 MB read of another buffer,
+    which writes the dirty lines back before the timed region."""
+    import torch
+
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    clean = torch.ones(256 << 20, dtype=torch.uint8, device=device)
+
+    def run():
+        flush.fill_(1)
+        clean.amax()
+    return run
+
+
+DECODE_WINDOW_CALLS = 400
+
+
+def decode_record(name, device, calls=DECODE_WINDOW_CALLS):
+    """paged_attention_decode alone on one workload's batch (its configured lengths
+    and placement; keys, values and q drawn on the device), `calls` calls each after
+    an L2 flush, timed with CUDA events: a window of tens to hundreds of
+    milliseconds, so the clock sampler sees it under load."""
+    import torch
+    import paged_kv_cache_319_b200 as kvp
+
+    wl = workloads.by_name(name)
+    g = wl.geometry
+    lens = np.asarray(wl.info["context_lens"], np.int64)
+    S, bs = len(lens), g.block_size
+    pool = kvp.BlockPool(wl.num_blocks, bs, g.num_kv_heads, g.head_dim, g.dtype, wl.free_order)
+    seqs = np.array([pool.create() for _ in lens], dtype=np.int64)
+    slots = np.concatenate([np.asarray(pool.append(int(s), int(L)), np.int64)
+                            for s, L in zip(seqs, lens)])
+    tdt = torch.float16 if g.dtype == "f16" else torch.bfloat16
+    shape = (wl.num_blocks, g.num_kv_heads, bs, g.head_dim)
+    k = torch.zeros(shape, dtype=tdt, device=device)
+    v = torch.zeros(shape, dtype=tdt, device=device)
+    gen = torch.Generator(device=device).manual_seed(5001)
+    st = torch.from_numpy(slots).to(device)
+    for t0 in range(0, len(slots), 65536):  # fill in chunks (fp32 draws, then rounded)
+        n = min(65536, len(slots) - t0)
+        kn = torch.randn((n, g.num_kv_heads, g.head_dim), generator=gen, device=device).to(tdt)
+        vn = torch.randn((n, g.num_kv_heads, g.head_dim), generator=gen, device=device).to(tdt)
+        kvp.reshape_and_cache(kn, vn, k, v, st[t0:t0 + n])
+    MB = int(-(-lens.max() // bs))
+    tables, cl = pool.build_batch(list(seqs), MB)
+    tt = torch.from_numpy(tables).to(device)
+    ct = torch.from_numpy(cl).to(device)
+    q = torch.randn((S, g.num_q_heads, g.head_dim), generator=gen, device=device).to(tdt)
+    out = torch.empty_like(q)
+    part = wl.partition_size
+    mcl = int(lens.max())
+    ws = torch.empty(max(256, kvp.decode_workspace_bytes(S, g.num_q_heads, g.head_dim, mcl, part)),
+                     dtype=torch.uint8, device=device)
+    call = lambda: kvp.paged_attention_decode(q, k, v, tt, ct, wl.scale, out,  # noqa: E731
+                                              max_context_len=mcl, partition_size=part,
+                                              workspace=ws)
+    flush = l2_flusher(device)
+    for _ in range(5):
+        call()
+    kvp.check_device_error(device)
+    stream = torch.cuda.current_stream(device)
+    pairs = []
+    with ClockSampler(device) as clk:
+        for _ in range(calls):
+            flush()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            call()
+            e1.record(stream)
+            pairs.append((e0, e1))
+        torch.cuda.synchronize(device)
+    kvp.check_device_error(device)
+    ms = np.array([a.elapsed_time(b) for a, b in pairs])
+    alg = algorithmic_bytes(cl, g)
+    peak, peak_kind = peaks()
+    achieved = alg / (float(np.median(ms)) * 1e-3) / 1e9
+    kernel = "decode_tc" if g.num_q_heads > g.num_kv_heads else "decode_simt"
+    pool.close()
+    return {"name": wl.name, "workload": wl.description, "calls": calls,
+            "timed": f"paged_attention_decode alone, {calls} calls, L2 flushed before each",
+            "call_us_median": round(float(np.median(ms)) * 1e3, 2),
+            "call_us_mean": round(float(ms.mean()) * 1e3, 2),
+            "seq_tokens_per_s": round(float(lens.sum()) / (float(np.median(ms)) * 1e-3), 1),
+            "roofline": {"kernel": f"paged_attention_decode: {kernel} + decode_reduce_kernel",
+                         "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
+                         "peak_source": peak_kind, "unit": "GB/s",
+                         "frac": round(achieved / peak, 4),
+                         "frac_of_nominal_8tbs": round(achieved / 8000.0, 4),
+                         "algorithmic_bytes_per_launch": int(alg)},
+            "clocks": clk.summary(min_samples=20)}
+
+
+# Workloads measured after the headline in the default run, each as its own
+# --workload run measures it (calls: timed calls of a single-call workload).
+OTHER_WORKLOADS = [
+    ("gqa_long_bs16", "decode", 0), ("gqa_long_bs32", "decode", 0),
+    ("llama13b_churn", "schedule", 0), ("sharing_A", "schedule", 200),
+    ("sharing_B", "schedule", 200), ("beam", "schedule", 200),
+    ("opt13b_fp8", "fp8", 200), ("prefill_opt13b_t16", "prefill", 200),
+    ("prefill_gqa_bs16_t4", "prefill", 200), ("prefill_prompt512", "prefill", 50),
+]
+
+
+def _summary(rec):
+    """The parts of a workload's line that the default line carries."""
+    keep = ("value", "unit", "steps", "warmup", "ms_per_step", "dtype", "config", "roofline",
+            "clocks", "seq_tokens_per_s", "query_tokens_per_s", "attention_tflops",
+            "f16_cache_same_batch", "rows", "call_us_median", "call_us_mean", "calls", "timed",
+            "workload", "name")
+    return {k: v for k, v in rec.items() if k in keep}
+
+
+def workload_records(args, device):
+    import types
+
+    out = {}
+    for name, kind, calls in OTHER_WORKLOADS:
+        t0 = time.perf_counter()
+        try:
+            if kind == "decode":
+                rec = decode_record(name, device)
+            else:
+                a = types.SimpleNamespace(**vars(args))
+                a.workload, a.partition, a.num_seqs, a.decode = name, None, None, "auto"
+                if calls:
+                    a.steps = calls
+                a.warmup = max(3, args.warmup)
+                rec = {"schedule": schedule_record, "fp8": fp8_record,
+                       "prefill": prefill_record}[kind](a)
+            rec = _summary(rec)
+        except Exception as exc:  # one workload's failure must not lose the others
+            rec = {"error": repr(exc)[:300]}
+        rec["wall_s"] = round(time.perf_counter() - t0, 1)
+        out[name] = rec
+        release_memory()
+    return out
 
 
 def measure_rows(wl, rep, device, k_step, v_step, host_us):
@@ -703,9 +859,10 @@ def unique_bytes(tables, lens, g):
     return kv + qo + 4 * int(np.sum(-(-np.asarray(lens) // bs))) + 4 * len(lens)
 
 
-def run_schedule(args):
+def schedule_record(args):
     """Workloads whose steps change the batch (churn, sharing, beam): the schedule is
-    replayed once through libkvp and every attention call is timed with CUDA events."""
+    replayed once through libkvp and every attention call is timed with CUDA events.
+    Values are drawn on the device (the parity tests replay the seeded host draws)."""
     import torch
     import paged_kv_cache_319_b200 as kvp
     from paged_kv_cache_319_b200.replay import DeviceReplay
@@ -724,7 +881,7 @@ def run_schedule(args):
     n_att = sum(1 for op in wl.ops if op[0] == "attend")
     reps = max(1, args.steps) if n_att == 1 else 1
     rp = DeviceReplay(wl, device, keep_outputs=False, time_decode=True, grouped=grouped,
-                      time_reps=reps)
+                      time_reps=reps, device_values=True)
     with ClockSampler(device) as clk:
         rp.run()
         torch.cuda.synchronize(device)
@@ -774,7 +931,7 @@ def run_schedule(args):
         "pool": {k: int(v) for k, v in st.items()},
         "clocks": clk.summary(),
     }
-    print(json.dumps(res), flush=True)
+    return res
 
 
 # Paged prefill workloads: a chunk of T new tokens per sequence, causal within
@@ -791,7 +948,7 @@ PREFILL_WORKLOADS = {
 }
 
 
-def run_prefill(args):
+def prefill_record(args):
     """paged_attention_prefill, timed with CUDA events (median of --steps calls, L2
     flushed before each); roofline on algorithmic bytes: K/V of every context token
     read once, q, out, block tables and lengths."""
@@ -882,13 +1039,13 @@ def run_prefill(args):
                      "avg_launch_us": round(ms * 1e3, 2)},
         "clocks": clk.summary(),
     }
-    print(json.dumps(res), flush=True)
+    return res
 
 
 FP8_WORKLOADS = ("opt13b_fp8",)
 
 
-def run_fp8(args):
+def fp8_record(args):
     """paged_attention_decode_fp8 on the OPT-13B batch with an E4M3 cache, timed with
     CUDA events (median of --steps calls, L2 flushed before each), beside the 16-bit
     decode of the same batch; roofline on the E4M3 algorithmic bytes."""
@@ -1001,7 +1158,7 @@ def run_fp8(args):
                      "traffic": traffic_per_launch("decode_simt_fp8", alg)},
         "clocks": clk.summary(),
     }
-    print(json.dumps(res), flush=True)
+    return res
 
 
 def run_reference_sampled(args, world):
@@ -1133,6 +1290,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--ref-seqs-per-step", type=int, default=1)
+    ap.add_argument("--headline-only", action="store_true",
+                    help="skip the decode window and the other workloads' records of the "
+                         "default line")
     ap.add_argument("--decode", choices=["auto", "plain", "grouped"], default="auto",
                     help="decode entry point of the schedule workloads (auto: grouped for "
                          "the sampling and beam workloads)")
@@ -1149,13 +1309,13 @@ def main():
     if single_gpu and int(os.environ.get("RANK", "0")) != 0:
         return  # one-GPU workloads: rank 0 runs and prints, the other ranks do nothing
     if args.workload in SCHEDULE_WORKLOADS:
-        run_schedule(args)
+        print(json.dumps(schedule_record(args)), flush=True)
         return
     if args.workload in PREFILL_WORKLOADS:
-        run_prefill(args)
+        print(json.dumps(prefill_record(args)), flush=True)
         return
     if args.workload in FP8_WORKLOADS:
-        run_fp8(args)
+        print(json.dumps(fp8_record(args)), flush=True)
         return
     world, rank, local = dist_setup()
     try:

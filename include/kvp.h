@@ -96,7 +96,10 @@ typedef struct kvp_pool_stats {
 
 /* Creates a pool of `num_blocks` physical blocks of `block_size` token slots
  * for a layer group with `num_kv_heads` KV heads of `head_dim` elements of
- * `dtype`. The free list is a stack: the first block handed out is
+ * `dtype`: the shared pool of fixed-size physical blocks that sequences take
+ * blocks from ["vLLM and PagedAttention", section "Architecture, step by
+ * step", step 1; "Your GPU was mostly empty", section "The OS already solved
+ * this in the 1960s"]. The free list is a stack: the first block handed out is
  * free_order[0], then free_order[1], ... `free_order` must be a permutation of
  * 0..num_blocks-1 (it is copied); NULL means 0, 1, 2, ... Block placement is
  * then fully determined by the call sequence.
@@ -130,7 +133,13 @@ KVP_API int kv_seq_create(kvp_pool* pool, int64_t* seq_id);
 
 /* Appends n_tokens >= 0 tokens to `seq`, one after another, and writes each
  * token's flat slot (physical_block * block_size + offset) to slots_out
- * (may be NULL when n_tokens == 0). A token at a block boundary takes a new
+ * (may be NULL when n_tokens == 0). Blocks are taken only as the sequence
+ * grows into them and mapped through its block table ["vLLM and
+ * PagedAttention", section "Architecture, step by step", steps 1-2;
+ * "PagedAttention: KV cache memory management", section "A request lifecycle":
+ * a full block makes the runtime take another]; a write into a shared block
+ * copies it first ["Your GPU was mostly empty", section "Paging's second gift:
+ * copy-on-write"]. A token at a block boundary takes a new
  * block from the free list; a token that lands in a partly filled last block
  * that other sequences also reference first takes a private copy: a new block
  * is taken, the pair (old, new) is queued for copy_blocks, the old block loses
@@ -149,12 +158,17 @@ KVP_API int kv_seq_append_batch(kvp_pool* pool, const int64_t* seqs, int32_t num
                         int32_t n_each, int64_t* slots_out);
 
 /* New sequence sharing every block of `parent` (each block gains one
- * reference); the child has the parent's length. */
+ * reference); the child has the parent's length. Parallel samples and beams
+ * share their common blocks by reference count, as fork() shares pages ["Your
+ * GPU was mostly empty", section "Paging's second gift: copy-on-write"]. */
 KVP_API int kv_seq_fork(kvp_pool* pool, int64_t parent, int64_t* child);
 
 /* Ends `seq`: each block of its table, in logical order, loses one reference;
  * a block that reaches zero is pushed onto the free list (with prefix caching
- * on, a registered block becomes evictable instead: see below). */
+ * on, a registered block becomes evictable instead: see below). A finished
+ * request's blocks go back to the shared pool ["vLLM and PagedAttention",
+ * section "Architecture, step by step", step 4; "PagedAttention: KV cache
+ * memory management", section "A request lifecycle": release]. */
 KVP_API int kv_seq_release(kvp_pool* pool, int64_t seq);
 
 /* Length (tokens) of `seq`. */
@@ -166,7 +180,9 @@ KVP_API int kv_seq_block_table(const kvp_pool* pool, int64_t seq, int32_t* out, 
                        int32_t* n);
 
 /* Moves the queued copy-on-write pairs, in creation order, into
- * pairs[2*i] = src, pairs[2*i+1] = dst, and clears the queue. KVP_ERR_CAPACITY
+ * pairs[2*i] = src, pairs[2*i+1] = dst, and clears the queue: the block copies
+ * that copy-on-write owes, for copy_blocks to make on the device ["Your GPU
+ * was mostly empty", section "Paging's second gift: copy-on-write"]. KVP_ERR_CAPACITY
  * (with *n set, queue kept) if cap (pairs) is too small. */
 KVP_API int kv_pool_take_copies(kvp_pool* pool, int32_t* pairs, int32_t cap, int32_t* n);
 
@@ -237,7 +253,11 @@ KVP_API int kv_pool_prefix_stats(const kvp_pool* pool, int64_t* registered, int6
 
 /* Packs the batch metadata the decode kernels read: block_tables is
  * [num_seqs][max_blocks] (row i = table of seqs[i], padded with -1) and
- * context_lens[i] = length of seqs[i]. Host buffers; copy them to the device.
+ * context_lens[i] = length of seqs[i]: the logical-to-physical map the
+ * attention kernel follows ["vLLM and PagedAttention", section "Architecture,
+ * step by step", steps 2-3; "PagedAttention: KV cache memory management",
+ * section "Operational trade-offs and limits": the runtime keeps the block
+ * metadata]. Host buffers; copy them to the device.
  * KVP_ERR_CAPACITY if a table is longer than max_blocks. */
 KVP_API int kv_build_batch(const kvp_pool* pool, const int64_t* seqs, int32_t num_seqs,
                    int32_t max_blocks, int32_t* block_tables, int32_t* context_lens);
@@ -368,8 +388,10 @@ KVP_API size_t kvp_decode_grouped_workspace_bytes(int32_t num_seqs, int32_t num_
  * NULL, a copy the call makes into the workspace by cudaMemcpyAsync on
  * `stream` (pageable host memory may be reused once the call returns;
  * page-locked memory, whose copy runs in stream order, must stay unchanged
- * until the stream has reached this call). device_plan without host_plan is
- * rejected. A host
+ * until the stream has reached this call). A call captured into a CUDA graph
+ * needs device_plan, or a host_plan in page-locked memory that stays valid for
+ * every replay: a copy from pageable memory cannot be captured.
+ * device_plan without host_plan is rejected. A host
  * plan also lets the call give the tensor-core kernel only its share of the
  * SMs and run the CUDA-core kernel beside it. A plan from other tables gives
  * wrong results; one whose header does not fit the batch is rejected.
@@ -511,7 +533,10 @@ KVP_API int paged_attention_decode_fp8(const void* q, const void* k_cache, const
  * nothing: inputs and outputs are the caller's, as for
  * paged_attention_decode, and the arguments and results are the same.
  * The first call on a device looks up the array's device address on that
- * device (with it current); make that first call before any stream capture.
+ * device (with it current), and so does the first call after the device's
+ * context changes (cudaDeviceReset, or a thread bound to another context);
+ * make those calls before any stream capture: a lookup while `stream` is
+ * capturing is refused with KVP_ERR_INVALID.
  * All calls share the one array and it keeps the last call's contents;
  * nothing in it needs to start at zero (each call writes every partial it
  * later reads), but calls whose kernels overlap on the GPU (different streams,

@@ -69,11 +69,19 @@ struct kvp_pool {
     // prefix caching: the token ids appended so far, while every append gave them
     std::vector<int32_t> tokens;
     bool tracked = true;
+    uint64_t batch_mark = 0;  // epoch of the last batch append that listed this sequence
   };
   std::unordered_map<int64_t, Seq> seqs;
   std::vector<std::pair<int32_t, int32_t>> pending;  // (src, dst) copy-on-write pairs
   int64_t next_seq = 0;
   int64_t cow_total = 0;
+  // batch appends: an epoch per call (duplicates found in one pass), per block
+  // the reference count left after the batch's earlier copies (-1: untouched),
+  // and the blocks whose entry a call set, so it can put them back
+  uint64_t batch_epoch = 0;
+  std::vector<int32_t> rc_seen;
+  std::vector<int32_t> rc_touched;
+  std::vector<Seq*> batch_ptrs;
 
   // ---- prefix caching
   struct KeyHash {
@@ -245,6 +253,7 @@ int kv_pool_create(int32_t num_blocks, int32_t block_size, int32_t num_kv_heads,
     p->head_dim = head_dim;
     p->dtype = dtype;
     p->rc.assign(num_blocks, 0);
+    p->rc_seen.assign(num_blocks, -1);
     p->free_stack.resize(num_blocks);
     p->key_of.resize(num_blocks);
     p->reg_of.assign(num_blocks, -1);
@@ -487,28 +496,48 @@ static int append_batch_impl(kvp_pool* pool, const int64_t* seqs, int32_t num_se
   if (!seqs || !slots_out) return fail(KVP_ERR_INVALID, "%s: NULL argument", who);
   // Exact block need of the whole batch: a copy-on-write by an earlier
   // sequence lowers the count a later sharer of the same last block sees.
-  std::unordered_map<int32_t, int32_t> rc_after;
-  std::vector<kvp_pool::Seq*> ptrs(num_seqs);
+  // Linear in the batch: sequences are marked with this call's epoch, and the
+  // lowered counts live in the pool's per-block scratch, reset on every exit.
+  try {
+    reserve_more(pool->batch_ptrs, size_t(num_seqs));
+    reserve_more(pool->rc_touched, size_t(num_seqs));
+  } catch (...) {
+    return fail(KVP_ERR_OOM, "%s: host allocation failed", who);
+  }
+  pool->batch_ptrs.clear();
+  pool->rc_touched.clear();
+  struct Restore {
+    kvp_pool* p;
+    ~Restore() {
+      for (int32_t b : p->rc_touched) p->rc_seen[b] = -1;
+      p->rc_touched.clear();
+    }
+  } restore{pool};
+  const uint64_t epoch = ++pool->batch_epoch;
   int64_t need = 0;
   for (int32_t i = 0; i < num_seqs; ++i) {
     kvp_pool::Seq* s = pool->find(seqs[i]);
     if (!s) return fail(KVP_ERR_NO_SEQ, "%s: no live sequence %lld", who, (long long)seqs[i]);
-    for (int32_t j = 0; j < i; ++j)
-      if (ptrs[j] == s) return fail(KVP_ERR_INVALID, "%s: duplicate sequence", who);
-    ptrs[i] = s;
+    if (s->batch_mark == epoch) return fail(KVP_ERR_INVALID, "%s: duplicate sequence", who);
+    s->batch_mark = epoch;
+    pool->batch_ptrs.push_back(s);
     if (int64_t(s->len) + n_each > INT32_MAX) return fail(KVP_ERR_INVALID, "%s: overflow", who);
     int32_t last_rc = 0;
     if (!s->table.empty()) {
       const int32_t last = s->table.back();
-      auto it = rc_after.find(last);
-      last_rc = it == rc_after.end() ? pool->rc[last] : it->second;
-      if (s->len % pool->block_size != 0 && last_rc > 1) rc_after[last] = last_rc - 1;
+      const int32_t seen = pool->rc_seen[last];
+      last_rc = seen >= 0 ? seen : pool->rc[last];
+      if (s->len % pool->block_size != 0 && last_rc > 1) {
+        if (seen < 0) pool->rc_touched.push_back(last);
+        pool->rc_seen[last] = last_rc - 1;
+      }
     }
     need += pool->need_for(*s, n_each, last_rc);
   }
   if (need > pool->available())
     return fail(KVP_ERR_OOM, "%s: need %lld blocks, %lld free or evictable", who, (long long)need,
                 (long long)pool->available());
+  std::vector<kvp_pool::Seq*>& ptrs = pool->batch_ptrs;
   try {
     for (int32_t i = 0; i < num_seqs; ++i) {
       reserve_more(ptrs[i]->table, size_t(n_each / pool->block_size + 2));

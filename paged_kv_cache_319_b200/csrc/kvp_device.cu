@@ -1084,22 +1084,59 @@ static __device__ __align__(256) unsigned char g_static_decode_scratch[KVP_STATI
 
 namespace {
 
+// The static scratch's device address, per device, with the context it was
+// taken in: a device reset (cudaDeviceReset) or a thread bound to another
+// context makes a cached address stale, so a call whose current context
+// differs looks the address up again.
+struct ScratchAddr {
+  CUcontext ctx;
+  void* ptr;
+};
 std::mutex g_static_scratch_mu;
-void* g_static_scratch_ptr[kMaxDevices] = {};
+ScratchAddr g_static_scratch[kMaxDevices] = {};
 
-// Device address of the static scratch on the current device (looked up on the
-// first call for each device, with that device current).
-int static_scratch_address(void** out) {
+CUcontext current_context() {
+  static PFN_cuCtxGetCurrent_v4000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &p, 4000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+  });
+  CUcontext c = nullptr;
+  if (!fn || fn(&c) != CUDA_SUCCESS) return nullptr;
+  return c;
+}
+
+// Device address of the static scratch in the current context. The lookup
+// (cudaGetSymbolAddress, with the device current) runs on the first call per
+// device and context; it may load the module, which a stream capture does not
+// allow, so a lookup while `stream` is capturing is refused.
+int static_scratch_address(cudaStream_t stream, void** out) {
   const int d = current_device();
   if (d < 0 || d >= kMaxDevices) return fail(KVP_ERR_INVALID, "device index %d out of range", d);
   std::lock_guard<std::mutex> g(g_static_scratch_mu);
-  if (!g_static_scratch_ptr[d]) {
-    void* p = nullptr;
-    cudaError_t e = cudaGetSymbolAddress(&p, g_static_decode_scratch);
-    if (e != cudaSuccess) return cuda_fail(e, "paged_attention_decode_noalloc: scratch address");
-    g_static_scratch_ptr[d] = p;
+  ScratchAddr& slot = g_static_scratch[d];
+  const CUcontext ctx = current_context();
+  if (slot.ptr && ctx && slot.ctx == ctx) {
+    *out = slot.ptr;
+    return KVP_OK;
   }
-  *out = g_static_scratch_ptr[d];
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(stream, &cs) == cudaSuccess && cs != cudaStreamCaptureStatusNone)
+    return fail(KVP_ERR_INVALID,
+                "paged_attention_decode_noalloc: the first call on a device (and the first after "
+                "a device reset) looks up the static scratch and must come before any stream "
+                "capture");
+  void* p = nullptr;
+  cudaError_t e = cudaGetSymbolAddress(&p, g_static_decode_scratch);
+  if (e != cudaSuccess) return cuda_fail(e, "paged_attention_decode_noalloc: scratch address");
+  slot.ptr = p;
+  slot.ctx = current_context();
+  *out = p;
   return KVP_OK;
 }
 
@@ -1120,7 +1157,7 @@ extern "C" int paged_attention_decode_noalloc(
                 need, size_t(KVP_STATIC_SCRATCH_BYTES));
   void* ws = nullptr;
   if (need > 0) {
-    const int rc = static_scratch_address(&ws);
+    const int rc = static_scratch_address(static_cast<cudaStream_t>(stream), &ws);
     if (rc) return rc;
   }
   return paged_attention_decode(q, k_cache, v_cache, block_tables, context_lens, num_seqs,

@@ -10,7 +10,10 @@ attention, because a new token may land in a block copied in the same step.
 
 Inputs (K/V of appended tokens, q of each attend) are drawn from
 :mod:`workloads` keyed by the op's index, the same draws any other consumer
-of the schedule sees.
+of the schedule sees. With ``device_values`` they are drawn on the GPU
+instead (seeded by the op's index, normal, rounded to the cache type): the
+same shapes and distribution without the host draws, for timing runs that do
+not compare with the oracle.
 """
 
 from __future__ import annotations
@@ -34,7 +37,8 @@ def bits_to_tensor(bits: np.ndarray, dtype: str, device):
 
 class DeviceReplay:
     def __init__(self, wl, device="cuda", keep_outputs: bool = True, time_decode: bool = False,
-                 grouped: bool = False, time_reps: int = 1, plan_on: str = "host"):
+                 grouped: bool = False, time_reps: int = 1, plan_on: str = "host",
+                 device_values: bool = False):
         import torch
 
         g = wl.geometry
@@ -59,9 +63,22 @@ class DeviceReplay:
         self.time_reps = max(1, int(time_reps))  # timed calls per attend op (time_decode)
         self.decode_events = []    # (op_index, start event, end event) around each decode call
         self.next_index = 0
+        self.device_values = device_values
+
+    def _device_normal(self, stream: int, op_index: int, shape):
+        import torch
+
+        gen = torch.Generator(device=self.device)
+        gen.manual_seed((int(self.wl.value_seed) * 1000003 + stream) * 1000003 + int(op_index))
+        return torch.randn(shape, generator=gen, device=self.device,
+                           dtype=torch.float32).to(self.tdtype)
 
     def kv_values(self, op_index: int, n: int):
         g = self.g
+        if self.device_values:
+            shape = (n, g.num_kv_heads, g.head_dim)
+            return (self._device_normal(K_STREAM, op_index, shape),
+                    self._device_normal(V_STREAM, op_index, shape))
         shape = (n, g.num_kv_heads, g.head_dim)
         k = normal_bits(value_seed_words(self.wl.value_seed, K_STREAM, op_index), shape, g.dtype)
         v = normal_bits(value_seed_words(self.wl.value_seed, V_STREAM, op_index), shape, g.dtype)
@@ -70,6 +87,8 @@ class DeviceReplay:
     def q_values(self, op_index: int, num_seqs: int):
         g = self.g
         shape = (num_seqs, g.num_q_heads, g.head_dim)
+        if self.device_values:
+            return self._device_normal(Q_STREAM, op_index, shape)
         return normal_bits(value_seed_words(self.wl.value_seed, Q_STREAM, op_index), shape, g.dtype)
 
     def run(self, ops=None, start_index=None, attend_kwargs=None):
@@ -112,8 +131,11 @@ class DeviceReplay:
                     ks.append(k)
                     vs.append(v)
                     sl.extend(slots)
-                k_new = bits_to_tensor(np.concatenate(ks), self.g.dtype, self.device)
-                v_new = bits_to_tensor(np.concatenate(vs), self.g.dtype, self.device)
+                if self.device_values:
+                    k_new, v_new = torch.cat(ks), torch.cat(vs)
+                else:
+                    k_new = bits_to_tensor(np.concatenate(ks), self.g.dtype, self.device)
+                    v_new = bits_to_tensor(np.concatenate(vs), self.g.dtype, self.device)
                 slot_t = torch.tensor(sl, dtype=torch.int64, device=self.device)
                 reshape_and_cache(k_new, v_new, self.k_cache, self.v_cache, slot_t)
             self._pending = []
@@ -124,7 +146,9 @@ class DeviceReplay:
             max_blocks = max(1, max(-(-L // bs) for L in lens_host))
             tables, lens = pool.build_batch(seqs, max_blocks)
             self.attends.append((i, seqs, tables, lens))
-            q = bits_to_tensor(self.q_values(i, len(seqs)), self.g.dtype, self.device)
+            q = self.q_values(i, len(seqs))
+            if not self.device_values:
+                q = bits_to_tensor(q, self.g.dtype, self.device)
             bt = torch.from_numpy(tables).to(self.device)
             cl = torch.from_numpy(lens).to(self.device)
             part = kw.get("partition_size", self.wl.partition_size)

@@ -82,6 +82,40 @@ def test_batch_append_equals_sequential_and_is_atomic():
     assert e.value.kind == "invalid"
 
 
+def test_rejected_duplicate_batch_leaves_no_trace():
+    # The batch check lowers a shared last block's count for each earlier sharer
+    # it has seen; a batch rejected part-way (a duplicate) must leave later
+    # batches computing the same need as sequential appends.
+    import paged_kv_cache_319_b200 as kvp
+
+    pools = [kvp.BlockPool(16, 4, 1, 8, "f16", list(range(16))) for _ in range(2)]
+    seqs = []
+    for p in pools:
+        s = p.create()
+        p.append(s, 5)                     # block 1 partial
+        seqs = [s, p.fork(s), p.fork(s)]   # three sharers of it
+    p1, p2 = pools
+    with pytest.raises(kvp.KvpError) as e:
+        p1.append_batch([seqs[1], seqs[2], seqs[1]], 1)
+    assert e.value.kind == "invalid"
+    assert p1.refcounts() == p2.refcounts() and p1.free_list() == p2.free_list()
+    got = p1.append_batch([seqs[1], seqs[2], seqs[0]], 1)
+    want = [p2.append(s, 1)[0] for s in (seqs[1], seqs[2], seqs[0])]
+    assert got.tolist() == want
+    assert p1.pending_copies() == p2.pending_copies() == [(1, 2), (1, 3)]
+    # exactly enough blocks for a batch whose sharers copy in turn
+    q1, q2 = (kvp.BlockPool(6, 4, 1, 8, "f16", list(range(6))) for _ in range(2))
+    for q in (q1, q2):
+        a = q.create()
+        q.append(a, 2)
+        b, c = q.fork(a), q.fork(a)
+    assert q1.num_free() == 5
+    q1.append_batch([a, b, c], 3)          # two copies (a, b) + c in place, 3 more for growth
+    for s in (a, b, c):
+        q2.append(s, 3)
+    assert q1.refcounts() == q2.refcounts() and q1.free_list() == q2.free_list()
+
+
 def test_errors_and_capacity():
     import paged_kv_cache_319_b200 as kvp
 
