@@ -338,7 +338,7 @@ def run_ours(args, world, rank, local):
     R = max(1, min(r_cap, math.ceil((W + K + K_e2e) / 64)))
     shift = math.ceil(W / R) + math.ceil(K / R) // 2
     start = np.maximum(ctx - shift, 1)
-    grow = math.ceil((W + K + K_e2e) / R) + 1
+    grow = math.ceil((W + K + K_e2e) / R) + 8  # + the e2e breakdown's few steps
     need_end = int(np.sum(-(-(start + grow) // g.block_size)))
     if need_end > wl.num_blocks:
         raise SystemExit(f"pool of {wl.num_blocks} blocks too small for {W + K} steps")
@@ -612,6 +612,149 @@ def decode_record(name, device, calls=DECODE_WINDOW_CALLS):
             "clocks": clk.summary(min_samples=20)}
 
 
+def vcache_record(name, device, calls=200, grow_steps=256):
+    """A/B of the block table's translation cost: the same batch (a workload's
+    lengths; keys, values and q drawn once on the device and written to both
+    caches) decoded from the paged pool and from the virtually contiguous cache
+    (CUDA virtual memory management), each `calls` calls after an L2 flush, at
+    equal algorithmic bytes. Host side: the growth of every sequence by one
+    token per step over `grow_steps` steps, kv_seq_append_batch + kv_build_batch
+    (paged) against kv_vcache_reserve_batch (contiguous: no table), and the cost
+    of mapping a physical chunk."""
+    import torch
+    import paged_kv_cache_319_b200 as kvp
+
+    wl = workloads.by_name(name)
+    g = wl.geometry
+    lens = np.asarray(wl.info["context_lens"], np.int64)
+    S, bs, Hkv, D = len(lens), g.block_size, g.num_kv_heads, g.head_dim
+    tdt = torch.float16 if g.dtype == "f16" else torch.bfloat16
+    max_tokens = int(lens.max()) + grow_steps + 16
+    # paged pool, sized for the growth steps too
+    nb = int(np.sum(-(-(lens + grow_steps) // bs))) + 16
+    free_order = np.random.default_rng(wl.value_seed).permutation(nb).astype(np.int32)
+    pool = kvp.BlockPool(nb, bs, Hkv, D, g.dtype, free_order)
+    seqs = np.array([pool.create() for _ in lens], dtype=np.int64)
+    slots = np.concatenate([np.asarray(pool.append(int(s), int(L)), np.int64)
+                            for s, L in zip(seqs, lens)])
+    k = torch.zeros((nb, Hkv, bs, D), dtype=tdt, device=device)
+    v = torch.zeros_like(k)
+    vc = kvp.VCache(S, max_tokens, Hkv, D, g.dtype)
+    stream = torch.cuda.current_stream(device)
+    torch.cuda.synchronize(device)
+    t0 = time.perf_counter()
+    vc.reserve_batch(np.arange(S), lens)
+    torch.cuda.synchronize(device)
+    map_s = time.perf_counter() - t0
+    st_map = vc.stats()
+    vslot = torch.from_numpy(np.repeat(np.arange(S), lens).astype(np.int32)).to(device)
+    vpos = torch.from_numpy(np.concatenate([np.arange(L) for L in lens]).astype(np.int32)).to(device)
+    st = torch.from_numpy(slots).to(device)
+    gen = torch.Generator(device=device).manual_seed(5101)
+    for t0_ in range(0, len(slots), 65536):
+        n = min(65536, len(slots) - t0_)
+        kn = torch.randn((n, Hkv, D), generator=gen, device=device).to(tdt)
+        vn = torch.randn((n, Hkv, D), generator=gen, device=device).to(tdt)
+        kvp.reshape_and_cache(kn, vn, k, v, st[t0_:t0_ + n])
+        kvp.reshape_and_cache_vcache(kn, vn, vc, vslot[t0_:t0_ + n], vpos[t0_:t0_ + n])
+    MB = int(-(-lens.max() // bs))
+    tables, cl = pool.build_batch(list(seqs), MB)
+    tt = torch.from_numpy(tables).to(device)
+    ct = torch.from_numpy(cl).to(device)
+    sl = torch.arange(S, dtype=torch.int32, device=device)
+    q = torch.randn((S, g.num_q_heads, D), generator=gen, device=device).to(tdt)
+    out_p, out_c = torch.empty_like(q), torch.empty_like(q)
+    part = wl.partition_size
+    mcl = int(lens.max())
+    ws = torch.empty(max(256, kvp.decode_workspace_bytes(S, g.num_q_heads, D, mcl, part)),
+                     dtype=torch.uint8, device=device)
+    paged = lambda: kvp.paged_attention_decode(q, k, v, tt, ct, wl.scale, out_p,  # noqa: E731
+                                               max_context_len=mcl, partition_size=part,
+                                               workspace=ws)
+    contig = lambda: kvp.attention_decode_vcache(q, vc, sl, ct, wl.scale, out_c,  # noqa: E731
+                                                 max_context_len=mcl, partition_size=part,
+                                                 workspace=ws)
+    flush = l2_flusher(device)
+
+    def timed(fn):
+        for _ in range(5):
+            fn()
+        pairs = []
+        for _ in range(calls):
+            flush()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            pairs.append((e0, e1))
+        torch.cuda.synchronize(device)
+        return float(np.median([a.elapsed_time(b) for a, b in pairs]))
+
+    with ClockSampler(device) as clk:
+        ms_p = timed(paged)
+        ms_c = timed(contig)
+    kvp.check_device_error(device)
+    same_bits = bool(torch.equal(out_p.view(torch.int16), out_c.view(torch.int16)))
+    err = float((out_p.float() - out_c.float()).abs().max())
+    alg = algorithmic_bytes(cl, g)
+    # the contiguous call reads a slot index per sequence instead of table entries
+    alg_c = alg - 4 * int(np.sum(-(-lens // bs))) + 4 * S
+    peak, peak_kind = peaks()
+    # host: one token per sequence per step
+    cur = lens.copy()
+    slot_buf = np.empty(S, np.int64)
+    tab_buf = np.empty((S, MB + grow_steps // bs + 2), np.int32)
+    len_buf = np.empty(S, np.int32)
+    t_paged, t_vc = [], []
+    maps_before = vc.stats()["map_calls"]
+    all_slots = np.arange(S, dtype=np.int32)
+    for _ in range(grow_steps):
+        t0 = time.perf_counter()
+        pool.append_batch(seqs, 1, out=slot_buf)
+        pool.build_batch(seqs, tab_buf.shape[1], tab_buf, len_buf)
+        t_paged.append(time.perf_counter() - t0)
+        cur += 1
+        t0 = time.perf_counter()
+        vc.reserve_batch(all_slots, cur)
+        t_vc.append(time.perf_counter() - t0)
+    torch.cuda.synchronize(device)
+    st_end = vc.stats()
+    grow_maps = st_end["map_calls"] - maps_before
+    paged_bytes = 2 * int(np.sum(-(-lens // bs))) * Hkv * bs * D * g.elem_bytes
+    res = {
+        "name": f"vcache_{name}", "workload": wl.description,
+        "timed": f"paged_attention_decode and attention_decode_vcache on the same batch and data, "
+                 f"{calls} calls each, L2 flushed before each",
+        "paged_call_us": round(ms_p * 1e3, 2), "contiguous_call_us": round(ms_c * 1e3, 2),
+        "translation_cost": round(ms_p / ms_c, 4),
+        "outputs_bit_identical": same_bits, "outputs_max_abs_diff": err,
+        "roofline": {"kernel": "attention_decode_vcache: " + (
+            "decode_tc (contiguous, 128-token boxes)" if g.num_q_heads > Hkv else
+            "decode_simt (contiguous, 16-token boxes)") + " + decode_reduce_kernel",
+            "bound": "hbm", "achieved": round(alg_c / (ms_c * 1e-3) / 1e9, 1),
+            "achieved_paged": round(alg / (ms_p * 1e-3) / 1e9, 1), "peak": peak,
+            "peak_source": peak_kind, "unit": "GB/s",
+            "frac": round(alg_c / (ms_c * 1e-3) / 1e9 / peak, 4),
+            "frac_paged": round(alg / (ms_p * 1e-3) / 1e9 / peak, 4),
+            "algorithmic_bytes_per_launch": int(alg_c)},
+        "memory": {"chunk_bytes": st_map["chunk_bytes"],
+                   "vcache_mapped_bytes": st_map["mapped_bytes"],
+                   "paged_block_bytes": paged_bytes,
+                   "vcache_over_paged": round(st_map["mapped_bytes"] / paged_bytes, 4)},
+        "host": {"initial_map_ms": round(map_s * 1e3, 2), "initial_chunks": st_map["map_calls"],
+                 "us_per_chunk_mapped": round(map_s * 1e6 / max(1, st_map["map_calls"]), 2),
+                 "grow_steps": grow_steps,
+                 "paged_append_batch_and_build_us_per_step": round(float(np.median(t_paged)) * 1e6, 2),
+                 "vcache_reserve_batch_us_per_step_median": round(float(np.median(t_vc)) * 1e6, 2),
+                 "vcache_reserve_batch_us_per_step_mean": round(float(np.mean(t_vc)) * 1e6, 2),
+                 "chunks_mapped_while_growing": int(grow_maps)},
+        "clocks": clk.summary(min_samples=20),
+    }
+    vc.close()
+    pool.close()
+    return res
+
+
 # Workloads measured after the headline in the default run, each as its own
 # --workload run measures it (calls: timed calls of a single-call workload).
 OTHER_WORKLOADS = [
@@ -620,6 +763,7 @@ OTHER_WORKLOADS = [
     ("sharing_B", "schedule", 200), ("beam", "schedule", 200),
     ("opt13b_fp8", "fp8", 200), ("prefill_opt13b_t16", "prefill", 200),
     ("prefill_gqa_bs16_t4", "prefill", 200), ("prefill_prompt512", "prefill", 50),
+    ("vcache_opt13b", "vcache", 200), ("vcache_gqa_long_bs16", "vcache", 100),
 ]
 
 
@@ -628,7 +772,8 @@ def _summary(rec):
     keep = ("value", "unit", "steps", "warmup", "ms_per_step", "dtype", "config", "roofline",
             "clocks", "seq_tokens_per_s", "query_tokens_per_s", "attention_tflops",
             "f16_cache_same_batch", "rows", "call_us_median", "call_us_mean", "calls", "timed",
-            "workload", "name")
+            "workload", "name", "paged_call_us", "contiguous_call_us", "translation_cost",
+            "outputs_bit_identical", "outputs_max_abs_diff", "memory", "host")
     return {k: v for k, v in rec.items() if k in keep}
 
 
@@ -641,6 +786,8 @@ def workload_records(args, device):
         try:
             if kind == "decode":
                 rec = decode_record(name, device)
+            elif kind == "vcache":
+                rec = vcache_record(name[len("vcache_"):], device, calls=calls)
             else:
                 a = types.SimpleNamespace(**vars(args))
                 a.workload, a.partition, a.num_seqs, a.decode = name, None, None, "auto"
@@ -729,7 +876,10 @@ def measure_rows(wl, rep, device, k_step, v_step, host_us):
 
 def run_e2e(args, wl, reps, device, seed_rank, MB, max_ctx_total, part, ws, world):
     """Same metric with host inputs: per step, pinned host -> device copies of q, the
-    new K/V and the metadata, the kernels, and the output copied back, synchronised."""
+    new K/V and the metadata, the kernels, and the output copied back, synchronised.
+    The host bookkeeping of step i + 1 (appends, block tables) runs while the GPU
+    runs step i (two pinned metadata buffers), as an engine's scheduler would; the
+    inputs go up, the result comes down and the host waits for it every step."""
     import torch
     import paged_kv_cache_319_b200 as kvp
 
@@ -743,72 +893,132 @@ def run_e2e(args, wl, reps, device, seed_rank, MB, max_ctx_total, part, ws, worl
     host_v = pin(torch.from_numpy(normal_bits(value_seed_words(seed_rank, V_STREAM, 999), (S, g.num_kv_heads, g.head_dim), g.dtype).view(np.int16)))
     tdt = torch.float16 if g.dtype == "f16" else torch.bfloat16
     host_out = torch.empty((S, g.num_q_heads, g.head_dim), dtype=torch.int16).pin_memory()
-    m = StepMeta(S, MB, device)
+    metas = [StepMeta(S, MB, device), StepMeta(S, MB, device)]
     q_d = torch.empty((S, g.num_q_heads, g.head_dim), dtype=tdt, device=device)
     k_d = torch.empty((S, g.num_kv_heads, g.head_dim), dtype=tdt, device=device)
     v_d = torch.empty_like(k_d)
     out = torch.empty_like(q_d)
-    h2d = (host_q.numel() + host_k.numel() + host_v.numel()) * 2 + m.nbytes
+    h2d = (host_q.numel() + host_k.numel() + host_v.numel()) * 2 + metas[0].nbytes
     d2h = host_out.numel() * 2
+    stream = torch.cuda.current_stream(device)
 
-    def device_part(rep):
-        """One step's stream work: inputs up, scatter, decode, result down."""
+    def up(m):
         q_d.view(torch.int16).copy_(host_q, non_blocking=True)
         k_d.view(torch.int16).copy_(host_k, non_blocking=True)
         v_d.view(torch.int16).copy_(host_v, non_blocking=True)
         m.upload()
+
+    def kernels(rep, m):
         kvp.reshape_and_cache(k_d, v_d, rep.k, rep.v, m.slot_d)
         kvp.paged_attention_decode(q_d, rep.k, rep.v, m.tab_d, m.len_d, wl.scale, out,
                                    max_context_len=max_ctx_total, partition_size=part, workspace=ws)
+
+    def down():
         host_out.copy_(out.view(torch.int16), non_blocking=True)
 
-    # Each replica's step as one CUDA graph (captured once; it reads the pinned
-    # buffers the host bookkeeping fills in every step). A step with
-    # copy-on-write pairs runs eagerly.
-    graphs = []
+    def device_part(rep, m):
+        """One step's stream work: inputs up, scatter, decode, result down."""
+        up(m)
+        kernels(rep, m)
+        down()
+
+    def book(rep, m):
+        """Host bookkeeping of a step into a pinned metadata buffer; CoW pairs."""
+        rep.pool.append_batch(rep.seqs, 1, out=m.slot_h.numpy())
+        copies = rep.pool.take_copies()
+        rep.pool.build_batch(rep.seqs, MB, m.tab_h.numpy(), m.len_h.numpy())
+        rep.lens += 1
+        return copies
+
+    # One CUDA graph per (replica, metadata buffer), captured once; it reads the
+    # pinned buffers the bookkeeping fills in. A step with copy-on-write pairs runs
+    # eagerly.
+    graphs = {}
     try:
         side = torch.cuda.Stream(device)
-        side.wait_stream(torch.cuda.current_stream(device))
+        side.wait_stream(stream)
         with torch.cuda.stream(side):
-            for rep in reps:
-                gr = torch.cuda.CUDAGraph()
-                with torch.cuda.graph(gr, stream=side):
-                    device_part(rep)
-                graphs.append(gr)
-        torch.cuda.current_stream(device).wait_stream(side)
+            for ri, rep in enumerate(reps):
+                for b, m in enumerate(metas):
+                    gr = torch.cuda.CUDAGraph()
+                    with torch.cuda.graph(gr, stream=side):
+                        device_part(rep, m)
+                    graphs[(ri, b)] = gr
+        stream.wait_stream(side)
         torch.cuda.synchronize(device)
     except Exception as exc:  # capture unsupported here: eager steps
-        graphs = []
+        graphs = {}
         print(f"e2e: CUDA graph capture failed ({exc}); eager steps", file=sys.stderr)
     total_bytes = 0
     barrier(world)
     torch.cuda.synchronize(device)
     t = time.perf_counter()
     eager = 0
+    copies = book(reps[0], metas[0])
     for i in range(K):
-        rep = reps[i % R]
-        rep.pool.append_batch(rep.seqs, 1, out=m.slot_h.numpy())
-        copies = rep.pool.take_copies()
-        rep.pool.build_batch(rep.seqs, MB, m.tab_h.numpy(), m.len_h.numpy())
-        rep.lens += 1
+        rep, b = reps[i % R], i % 2
+        m = metas[b]
         if copies or not graphs:
             if copies:
                 kvp.copy_blocks(rep.k, rep.v, torch.tensor(copies, dtype=torch.int32).to(device))
-            device_part(rep)
+            device_part(rep, m)
             eager += 1
         else:
-            graphs[i % R].replay()
-        torch.cuda.current_stream(device).synchronize()
-        total_bytes += algorithmic_bytes(m.len_h.numpy(), g)
+            graphs[(i % R, b)].replay()
+        step_bytes = algorithmic_bytes(m.len_h.numpy(), g)
+        if i + 1 < K:  # the next step's bookkeeping, while this one runs
+            copies = book(reps[(i + 1) % R], metas[(i + 1) % 2])
+        stream.synchronize()  # this step's result is on the host
+        total_bytes += step_bytes
     el = time.perf_counter() - t
     el = dist_max(el, world)
     total_bytes = dist_sum(float(total_bytes), world)
-    del graphs
+    # Where a step's time goes (not part of the timed loop): host bookkeeping,
+    # and each piece of the device work timed alone with CUDA events.
+    brk = {}
+    try:
+        rep, m = reps[0], metas[0]
+        hb = []
+        for _ in range(5):
+            t0 = time.perf_counter()
+            book(rep, m)
+            hb.append(time.perf_counter() - t0)
+        rep.pool.take_copies()
+
+        def ev_time(fn, n=10):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            fn()
+            e0.record(stream)
+            for _ in range(n):
+                fn()
+            e1.record(stream)
+            torch.cuda.synchronize(device)
+            return e0.elapsed_time(e1) / n * 1e3
+
+        def wall(fn, n=10):
+            fn()
+            torch.cuda.synchronize(device)
+            t0 = time.perf_counter()
+            for _ in range(n):
+                fn()
+                stream.synchronize()
+            return (time.perf_counter() - t0) / n * 1e6
+
+        brk = {"host_bookkeeping_us": round(float(np.median(hb)) * 1e6, 1),
+               "h2d_us": round(ev_time(lambda: up(m)), 1),
+               "kernels_us": round(ev_time(lambda: kernels(rep, m)), 1),
+               "d2h_us": round(ev_time(down), 1),
+               "graph_step_wall_us": round(wall(lambda: graphs[(0, 0)].replay()), 1) if graphs else None,
+               "step_us_in_timed_loop": round(el / K * 1e6, 1)}
+    except Exception as exc:  # pragma: no cover - diagnostics only
+        brk = {"error": repr(exc)[:200]}
+    graphs.clear()
     return {"value": round(total_bytes / el / 1e9, 2), "unit": UNIT, "steps": K,
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-            "how": "per step: host bookkeeping, then one CUDA graph replay (inputs from pinned "
-                   "host memory up, scatter, decode, result down) and a synchronize"
-                   + (f"; {eager} steps eager" if eager else "")}
+            "how": "per step: one CUDA graph replay (inputs from pinned host memory up, scatter, "
+                   "decode, result down) and a synchronize; the next step's host bookkeeping "
+                   "runs while the graph runs" + (f"; {eager} steps eager" if eager else ""),
+            "breakdown": brk}
 
 
 # ---------------------------------------------------------------- CPU oracle
@@ -875,13 +1085,14 @@ def schedule_record(args):
                                                 "llama13b_churn" else 64))
     wl = workloads.by_name(args.workload, **kw)
     g = wl.geometry
+    packed = args.decode == "packed"
     grouped = args.decode == "grouped" or (args.decode == "auto" and
                                             args.workload in GROUPED_WORKLOADS)
     # a workload with one attend op (sampling, beam) times that call `steps` times
     n_att = sum(1 for op in wl.ops if op[0] == "attend")
     reps = max(1, args.steps) if n_att == 1 else 1
-    rp = DeviceReplay(wl, device, keep_outputs=False, time_decode=True, grouped=grouped,
-                      time_reps=reps, device_values=True)
+    rp = DeviceReplay(wl, device, keep_outputs=False, time_decode=True, grouped=grouped and not packed,
+                      time_reps=reps, device_values=True, packed=packed)
     with ClockSampler(device) as clk:
         rp.run()
         torch.cuda.synchronize(device)
@@ -901,7 +1112,10 @@ def schedule_record(args):
     uniq = np.array([r[2] for r in timed], dtype=np.float64)
     toks = np.array([r[3] for r in timed], dtype=np.float64)
     peak, peak_kind = peaks()
-    if grouped:
+    if packed:
+        kernel = ("paged_attention_decode_packed (plan built on the host): decode_tc (packed: "
+                  "shared prefixes and own blocks in one stream per group)")
+    elif grouped:
         kernel = ("paged_attention_decode_grouped (plan built on the host): decode_tc (grouped, "
                   "shared prefixes) + " + ("decode_tc (own ranges)" if g.num_q_heads > g.num_kv_heads
                                            else "decode_simt (own ranges)"))
@@ -918,7 +1132,7 @@ def schedule_record(args):
         "config": {"workload": wl.description, "name": wl.name,
                    "timed": "attention calls only" + (
                        f" (median of {reps} calls, L2 flushed before each)" if reps > 1 else ""),
-                   "decode": "grouped" if grouped else "per-sequence"},
+                   "decode": "packed" if packed else ("grouped" if grouped else "per-sequence")},
         "seq_tokens_per_s": round(float(toks.sum() / (ms.sum() * 1e-3)), 1),
         "roofline": {"kernel": f"{kernel} + decode_reduce_kernel",
                      "bound": "hbm", "achieved_unique": round(achieved_u, 1),
@@ -1043,6 +1257,8 @@ def prefill_record(args):
 
 
 FP8_WORKLOADS = ("opt13b_fp8",)
+# the virtually contiguous cache against the paged one, on a workload's batch
+VCACHE_WORKLOADS = {"vcache_opt13b": "opt13b", "vcache_gqa_long_bs16": "gqa_long_bs16"}
 
 
 def fp8_record(args):
@@ -1283,7 +1499,7 @@ def main():
     ap.add_argument("--workload", default="opt13b",
                     choices=["opt13b", "gqa_long_bs16", "gqa_long_bs32", "llama13b_churn",
                              "sharing_A", "sharing_B", "beam"] + list(PREFILL_WORKLOADS)
-                    + list(FP8_WORKLOADS))
+                    + list(FP8_WORKLOADS) + list(VCACHE_WORKLOADS))
     ap.add_argument("--partition", type=int, default=None)
     ap.add_argument("--num-seqs", type=int, default=None,
                     help="smaller batch of the same workload (profiling small cases)")
@@ -1293,7 +1509,7 @@ def main():
     ap.add_argument("--headline-only", action="store_true",
                     help="skip the decode window and the other workloads' records of the "
                          "default line")
-    ap.add_argument("--decode", choices=["auto", "plain", "grouped"], default="auto",
+    ap.add_argument("--decode", choices=["auto", "plain", "grouped", "packed"], default="auto",
                     help="decode entry point of the schedule workloads (auto: grouped for "
                          "the sampling and beam workloads)")
     args = ap.parse_args()
@@ -1305,7 +1521,7 @@ def main():
                       int(os.environ.get("RANK", "0")))
         return
     single_gpu = args.workload in SCHEDULE_WORKLOADS or args.workload in PREFILL_WORKLOADS \
-        or args.workload in FP8_WORKLOADS
+        or args.workload in FP8_WORKLOADS or args.workload in VCACHE_WORKLOADS
     if single_gpu and int(os.environ.get("RANK", "0")) != 0:
         return  # one-GPU workloads: rank 0 runs and prints, the other ranks do nothing
     if args.workload in SCHEDULE_WORKLOADS:
@@ -1316,6 +1532,14 @@ def main():
         return
     if args.workload in FP8_WORKLOADS:
         print(json.dumps(fp8_record(args)), flush=True)
+        return
+    if args.workload in VCACHE_WORKLOADS:
+        import torch
+
+        device = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+        torch.cuda.set_device(device)
+        print(json.dumps(vcache_record(VCACHE_WORKLOADS[args.workload], device,
+                                       calls=max(1, args.steps))), flush=True)
         return
     world, rank, local = dist_setup()
     try:

@@ -439,6 +439,75 @@ KVP_API int kv_decode_group_plan(const int32_t* block_tables, const int32_t* con
                          int32_t num_kv_heads, int32_t num_blocks, int32_t* plan,
                          size_t plan_words);
 
+/* ---- packed grouped decode ------------------------------------------------
+ * Decode attention for batches whose sequences share cache blocks (forked
+ * samples, beams), reading every block once per group of the sequences that
+ * hold it ["Your GPU was mostly empty", section "Paging's second gift:
+ * copy-on-write": forked sequences share their common blocks]; the pages'
+ * decode reads a shared block once per sequence, and this entry point, which
+ * the pages do not describe, is an optimisation of the same result. Groups
+ * follow kv_decode_group_plan's rule; a sequence in no subgroup is a group of
+ * one. Each group's blocks form one stream - the shared prefix, then each
+ * member's own blocks - cut into chunks of 512 tokens; one persistent
+ * tensor-core kernel takes the chunks (longest first) with the members' query
+ * heads as the columns of the contraction, a column counting only the tokens
+ * of its member's blocks, and a log-sum-exp merge writes every output row.
+ * Unlike paged_attention_decode_grouped (two kernels: shared prefixes on the
+ * tensor cores, own ranges on the CUDA cores), short own ranges share key tiles
+ * with other members and the shared prefix, so no kernel pays a sequence's
+ * dependent loads alone. */
+
+/* Words a packed plan of num_seqs sequences with up to max_blocks_per_seq
+ * blocks each may take (an upper bound; 0 for non-positive sizes). */
+KVP_API size_t kvp_decode_pack_plan_words(int32_t num_seqs, int32_t max_blocks_per_seq);
+
+/* Builds on the host the packed plan of a batch from host copies of its block
+ * tables ([num_seqs][max_blocks_per_seq]) and context lengths (clamped to
+ * [0, max_context_len]). Layout (int32 words): [0] groups, [1] units per KV
+ * head, [2] entries, [3] most chunks of any group, [4] block size, [5] blocks
+ * per chunk (512 / block_size), [6] offset of the unit table, [7] offset of
+ * the entries; [8, 8 + S) each sequence's group; per group 20 words {first
+ * entry, members, entries, chunks, member sequences [16]}; per unit 4 words
+ * {group, first entry, entries, chunk}, longest first; per entry 2 words
+ * {block id, column mask << 8 | valid tokens of the block}. Column j of a group
+ * is query head g * G + j % G of member j / G.
+ * Needs block_size 16 or 32, num_seqs in [1, 4096], at most 16 query heads
+ * per KV head, plan_words >= kvp_decode_pack_plan_words(...). Errors:
+ * KVP_ERR_INVALID. */
+KVP_API int kv_decode_pack_plan(const int32_t* block_tables, const int32_t* context_lens,
+                                int32_t num_seqs, int32_t max_blocks_per_seq,
+                                int32_t max_context_len, int32_t block_size, int32_t num_q_heads,
+                                int32_t num_kv_heads, int32_t num_blocks, int32_t* plan,
+                                size_t plan_words);
+
+/* Bytes of device workspace paged_attention_decode_packed needs for this
+ * host plan: per (sequence, query head) one partial slot of head_dim + 2 fp32
+ * values per chunk of the longest group stream, plus room for a copy of the
+ * plan. 0 for a NULL plan or non-positive sizes. */
+KVP_API size_t kvp_decode_packed_workspace_bytes(const int32_t* host_plan, int32_t num_seqs,
+                                                 int32_t num_q_heads, int32_t head_dim);
+
+/* The packed grouped decode: the result of paged_attention_decode (to fp32
+ * rounding) for the batch the plan was built from. host_plan (required) is
+ * kv_decode_pack_plan's plan of these sequences, checked word by word against
+ * the batch (KVP_ERR_INVALID if its shape does not fit); the kernels read it
+ * from device_plan, a copy the caller placed in device memory (4-byte aligned,
+ * read-only to the call), or, when device_plan is NULL, from a copy the call
+ * makes into the workspace by cudaMemcpyAsync on `stream` (see
+ * paged_attention_decode_grouped for host memory and graph capture). The block
+ * ids are the plan's: the device block tables are not read. context_lens:
+ * device int32 [num_seqs]. Needs head_dim 128, block_size 16 or 32, at most 16
+ * query heads per KV head. workspace: >= kvp_decode_packed_workspace_bytes(...),
+ * 256-byte aligned. Errors: those of paged_attention_decode. */
+KVP_API int paged_attention_decode_packed(const void* q, const void* k_cache, const void* v_cache,
+                                          const int32_t* context_lens, int32_t num_seqs,
+                                          int32_t num_q_heads, int32_t num_kv_heads,
+                                          int32_t head_dim, int32_t block_size, int32_t num_blocks,
+                                          int32_t max_context_len, float scale,
+                                          const int32_t* host_plan, const int32_t* device_plan,
+                                          void* workspace, size_t workspace_bytes, void* out,
+                                          int32_t dtype, kvp_stream_t stream);
+
 /* Bytes of device workspace paged_attention_prefill needs: that of
  * paged_attention_decode for num_seqs * q_len rows (0 if q_len <= 0). */
 KVP_API size_t kvp_prefill_workspace_bytes(int32_t num_seqs, int32_t q_len, int32_t num_q_heads,
@@ -516,6 +585,123 @@ KVP_API int paged_attention_decode_fp8(const void* q, const void* k_cache, const
                                        float scale, int32_t partition_size, void* workspace,
                                        size_t workspace_bytes, void* out, int32_t dtype,
                                        kvp_stream_t stream);
+
+/* ---- virtually contiguous KV cache (CUDA virtual memory management) --------
+ * The alternative the pages name to block tables: keep each sequence's cache
+ * contiguous in virtual memory and back it with physical pages on demand
+ * through CUDA's virtual memory management, so the attention kernel computes
+ * addresses instead of dereferencing a block table ["Your GPU was mostly
+ * empty", section "The tradeoff: you just wrote a virtual memory subsystem in
+ * userspace": translation in the kernel (block tables) or in CUDA's VMM].
+ * Here it serves as an A/B of the block table's translation cost: the same
+ * decode kernels, tiles and math, with the address of a tile computed from
+ * (slot, token) instead of looked up.
+ *
+ * A cache has num_slots sequence slots of up to max_tokens tokens. Each slot
+ * is one reserved virtual range per cache (K, V), token-major:
+ *   K of token j of slot s, KV head g = k_base[((s * slot_tokens + j) *
+ *   num_kv_heads + g) * head_dim .. + head_dim)
+ * (slot_tokens from kv_vcache_layout: >= max_tokens plus a mapped tail, a whole
+ * number of physical chunks). Physical chunks (the device's allocation
+ * granularity, 2 MiB on B200) are mapped at the end of a slot's range as its
+ * capacity grows (kv_vcache_reserve) and unmapped only by kv_vcache_trim; a
+ * finished request's slot keeps its chunks for the next request. A slot's
+ * capacity is the tokens the kernels may touch; at least 256 more tokens are
+ * always mapped past it, so no kernel tile that starts inside the capacity
+ * reaches unmapped memory, and the kernels clamp every context length to the
+ * capacity of its slot (device copy, updated in stream order). Only head_dim
+ * 128 and 16-bit elements; one device (the current one at creation). Host
+ * calls are not thread-safe per cache. */
+typedef struct kvp_vcache kvp_vcache;
+
+typedef struct kvp_vcache_stats {
+  int64_t chunk_bytes;     /* physical mapping granularity                 */
+  int64_t mapped_chunks;   /* chunks mapped now, K and V together          */
+  int64_t spare_chunks;    /* unmapped chunks kept for reuse               */
+  int64_t mapped_bytes;    /* mapped_chunks * chunk_bytes                  */
+  int64_t reserved_bytes;  /* virtual bytes reserved, K and V together     */
+  int64_t map_calls;       /* chunk mappings made since creation           */
+  int64_t create_calls;    /* physical chunks created since creation       */
+  int64_t slot_tokens;     /* token stride between slots                   */
+} kvp_vcache_stats;
+
+/* Reserves the virtual ranges of a cache of num_slots slots of up to
+ * max_tokens tokens of num_kv_heads x head_dim elements of dtype (KVP_F16 or
+ * KVP_BF16; head_dim 128) on the current device; no physical memory is mapped
+ * yet (every capacity is 0). Errors: KVP_ERR_INVALID (sizes, dtype, more than
+ * 2^31 tokens in all), KVP_ERR_CUDA (VMM unavailable, reservation failed),
+ * KVP_ERR_OOM. */
+KVP_API int kv_vcache_create(int32_t num_slots, int32_t max_tokens, int32_t num_kv_heads,
+                             int32_t head_dim, int32_t dtype, kvp_vcache** out);
+
+/* Synchronises the device, unmaps and frees every chunk, releases the
+ * reservations. NULL is accepted. */
+KVP_API int kv_vcache_destroy(kvp_vcache* vc);
+
+/* Grows the capacity of `slot` to at least `tokens` (<= max_tokens) by mapping
+ * chunks at the end of its range; the device copy of the capacity is updated
+ * by a one-thread kernel on `stream`, so kernels launched after this call on
+ * that stream see it. No-op if the capacity suffices. On failure (KVP_ERR_OOM
+ * when the device has no memory for a chunk, KVP_ERR_CUDA) the call's own
+ * mappings are undone and nothing changes. */
+KVP_API int kv_vcache_reserve(kvp_vcache* vc, int32_t slot, int32_t tokens, kvp_stream_t stream);
+
+/* kv_vcache_reserve for n slots (host int32 arrays slots[n], tokens[n]), in
+ * order, as one call: a decode step's growth of the whole batch. All or
+ * nothing: if one slot cannot grow, the slots the call grew before it are
+ * returned to their earlier capacity (their chunks kept as spares). */
+KVP_API int kv_vcache_reserve_batch(kvp_vcache* vc, const int32_t* slots, const int32_t* tokens,
+                                    int32_t n, kvp_stream_t stream);
+
+/* Shrinks the capacity of `slot` to what `tokens` needs: the capacity drops on
+ * `stream`, the whole device is synchronised (no kernel may still read the
+ * chunks), then the chunks past it are unmapped and kept as spares for later
+ * reserves. tokens == 0 unmaps the slot entirely. */
+KVP_API int kv_vcache_trim(kvp_vcache* vc, int32_t slot, int32_t tokens, kvp_stream_t stream);
+
+/* Returns the spare chunks to the driver. */
+KVP_API int kv_vcache_release_spares(kvp_vcache* vc);
+
+/* Capacity (tokens) of `slot`. */
+KVP_API int kv_vcache_capacity(const kvp_vcache* vc, int32_t slot, int32_t* tokens);
+
+/* Base device addresses of the K and V ranges and the token stride between
+ * slots (see the layout above). Only the mapped part of a slot
+ * (kv_vcache_capacity tokens) may be read or written. */
+KVP_API int kv_vcache_layout(const kvp_vcache* vc, void** k_base, void** v_base,
+                             int32_t* slot_tokens);
+
+/* Counters (see kvp_vcache_stats). */
+KVP_API int kv_vcache_stats(const kvp_vcache* vc, kvp_vcache_stats* out);
+
+/* reshape_and_cache into a virtually contiguous cache: for t < num_tokens,
+ * token t's keys and values (k_new, v_new: device [num_tokens][num_kv_heads]
+ * [head_dim] of the cache's dtype, 16-byte aligned) go to position
+ * positions[t] of slot slots[t] (device int32 arrays). A negative slot is
+ * padding and skipped; a slot >= num_slots or a position outside [0, capacity)
+ * is skipped and recorded (KVP_ERR_BOUNDS from kvp_check_device_error), so no
+ * write reaches unmapped memory. Errors: KVP_ERR_INVALID. */
+KVP_API int reshape_and_cache_vcache(const void* k_new, const void* v_new, kvp_vcache* vc,
+                                     const int32_t* slots, const int32_t* positions,
+                                     int32_t num_tokens, kvp_stream_t stream);
+
+/* paged_attention_decode over a virtually contiguous cache: sequence s reads
+ * slot seq_slots[s] (device int32 [num_seqs]) through context_lens[s] tokens,
+ * each clamped to max_context_len and to the slot's capacity (a length or a
+ * slot out of range is recorded; an invalid slot reads nothing). Same result
+ * as paged_attention_decode with the block table of the slot's tokens. q, out
+ * [num_seqs][num_q_heads][head_dim] of the cache's dtype; num_q_heads a
+ * multiple of the cache's num_kv_heads (grouped-query heads, G <= 16, run on
+ * the tensor cores and need partition_size % 128 == 0); partition_size and
+ * workspace as for paged_attention_decode (kvp_decode_workspace_bytes). One
+ * query head per KV head reads 16-token tiles, grouped-query heads 128-token
+ * tiles, each one TMA load per tile (per 64-dim half for the keys).
+ * Errors: those of paged_attention_decode. */
+KVP_API int attention_decode_vcache(const void* q, const kvp_vcache* vc, const int32_t* seq_slots,
+                                    const int32_t* context_lens, int32_t num_seqs,
+                                    int32_t num_q_heads, int32_t max_context_len, float scale,
+                                    int32_t partition_size, void* workspace,
+                                    size_t workspace_bytes, void* out, kvp_stream_t stream);
 
 /* Largest split-context scratch, in bytes, that paged_attention_decode_noalloc
  * can serve from its built-in area (40 MiB). */

@@ -17,13 +17,15 @@ import ctypes as C
 
 import numpy as np
 
-from ._lib import (KVP_BF16, KVP_F16, KVP_FP8_E4M3, KvpError, P_i32, P_i64, PoolStats, check,
-                   lib)
+from ._lib import (KVP_BF16, KVP_F16, KVP_FP8_E4M3, KvpError, P_i32, P_i64, PoolStats,
+                   VCacheStats, check, lib)
 
 __all__ = [
     "BlockPool", "KvpError", "reshape_and_cache", "copy_blocks", "paged_attention_decode",
     "paged_attention_prefill", "reshape_and_cache_fp8", "paged_attention_decode_fp8",
     "decode_workspace_bytes", "decode_grouped_workspace_bytes", "group_plan", "check_device_error",
+    "VCache", "reshape_and_cache_vcache", "attention_decode_vcache", "pack_plan",
+    "paged_attention_decode_packed",
     "kv_bytes_per_token", "version",
     "KVP_F16", "KVP_BF16", "KVP_FP8_E4M3",
 ]
@@ -309,6 +311,56 @@ def group_plan(block_tables: np.ndarray, context_lens: np.ndarray, *, block_size
     return plan
 
 
+def pack_plan(block_tables: np.ndarray, context_lens: np.ndarray, *, block_size: int,
+              num_q_heads: int, num_kv_heads: int, num_blocks: int,
+              max_context_len: int | None = None) -> np.ndarray:
+    """The packed plan of ``paged_attention_decode_packed`` (``kv_decode_pack_plan``),
+    built on the host from host block tables [S, MB] and lengths [S]; trimmed to the
+    words its header says it uses."""
+    t = np.ascontiguousarray(block_tables, dtype=np.int32)
+    l = np.ascontiguousarray(context_lens, dtype=np.int32)
+    S, MB = t.shape
+    mcl = MB * block_size if max_context_len is None else int(max_context_len)
+    n = int(lib().kvp_decode_pack_plan_words(S, max(MB, 1)))
+    plan = np.zeros(max(n, 1), np.int32)
+    check(lib().kv_decode_pack_plan(_i32p(t), _i32p(l), S, max(MB, 1), mcl, block_size,
+                                    num_q_heads, num_kv_heads, num_blocks, _i32p(plan), n))
+    used = int(plan[7]) + 2 * int(plan[2])
+    return plan[:used].copy()
+
+
+def paged_attention_decode_packed(q, k_cache, v_cache, context_lens, scale: float, host_plan,
+                                  out=None, *, max_context_len: int | None = None,
+                                  device_plan=None, workspace=None):
+    """Decode attention of forked sequences through the packed grouped decode (every
+    shared block read once per group); ``host_plan`` from :func:`pack_plan`."""
+    torch = _torch()
+    dev = _cuda(q, k_cache, v_cache, context_lens)
+    if context_lens.dtype != torch.int32:
+        raise TypeError("context_lens must be int32")
+    S, Hq, D = q.shape
+    NB, Hkv, bs, D2 = k_cache.shape
+    if D2 != D or v_cache.shape != k_cache.shape:
+        raise ValueError("shape mismatch")
+    plan = np.ascontiguousarray(host_plan, dtype=np.int32)
+    mcl = int(context_lens.max().item()) if max_context_len is None else int(max_context_len)
+    if out is None:
+        out = torch.empty_like(q)
+    need = int(lib().kvp_decode_packed_workspace_bytes(_i32p(plan), S, Hq, D))
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    _cuda(out, workspace)
+    dp = None
+    if device_plan is not None:
+        _cuda(device_plan)
+        dp = device_plan.data_ptr()
+    check(lib().paged_attention_decode_packed(
+        q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), context_lens.data_ptr(), S, Hq, Hkv,
+        D, bs, NB, mcl, float(scale), _i32p(plan), dp, workspace.data_ptr(),
+        workspace.numel() * workspace.element_size(), out.data_ptr(), _code(q), _stream(dev)))
+    return out
+
+
 def paged_attention_decode(q, k_cache, v_cache, block_tables, context_lens, scale: float,
                            out=None, *, max_context_len: int | None = None,
                            partition_size: int = 0, workspace=None, grouped: bool = False,
@@ -474,6 +526,143 @@ def paged_attention_decode_fp8(q, k_cache, v_cache, k_scale, v_scale, block_tabl
         q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), k_scale.data_ptr(), v_scale.data_ptr(),
         block_tables.data_ptr(), context_lens.data_ptr(), S, Hq, Hkv, D, bs, NB, max(MB, 1), mcl,
         float(scale), int(partition_size), ws_ptr, ws_bytes, out.data_ptr(), _code(q), _stream(dev)))
+    return out
+
+
+class VCache:
+    """A virtually contiguous KV cache (``kv_vcache_*``): per sequence slot one
+    reserved virtual range of K and of V, token-major ``[slot][token][Hkv][D]``,
+    backed by physical chunks mapped as the slot's capacity grows. Created on
+    the current CUDA device."""
+
+    def __init__(self, num_slots: int, max_tokens: int, num_kv_heads: int, head_dim: int,
+                 dtype: str):
+        h = C.c_void_p()
+        check(lib().kv_vcache_create(num_slots, max_tokens, num_kv_heads, head_dim, _DTYPES[dtype],
+                                     C.byref(h)))
+        self._h = h
+        self.num_slots, self.max_tokens = num_slots, max_tokens
+        self.num_kv_heads, self.head_dim, self.dtype = num_kv_heads, head_dim, dtype
+        kb, vb, st = C.c_void_p(), C.c_void_p(), C.c_int32()
+        check(lib().kv_vcache_layout(h, C.byref(kb), C.byref(vb), C.byref(st)))
+        self.k_base, self.v_base, self.slot_tokens = kb.value, vb.value, st.value
+
+    @property
+    def handle(self):
+        if self._h is None:
+            raise RuntimeError("cache destroyed")
+        return self._h
+
+    def close(self):
+        if getattr(self, "_h", None) is not None:
+            lib().kv_vcache_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:  # pragma: no cover - interpreter shutdown
+            pass
+
+    def reserve(self, slot: int, tokens: int) -> None:
+        """Capacity of ``slot`` >= ``tokens`` (maps chunks; the device copy is updated
+        on the current stream)."""
+        torch = _torch()
+        check(lib().kv_vcache_reserve(self.handle, slot, tokens,
+                                      _stream(torch.device("cuda", torch.cuda.current_device()))))
+
+    def reserve_batch(self, slots: np.ndarray, tokens: np.ndarray) -> None:
+        """reserve() for every (slot, tokens) pair in one call (all or nothing)."""
+        torch = _torch()
+        sl = np.ascontiguousarray(slots, dtype=np.int32)
+        tk = np.ascontiguousarray(tokens, dtype=np.int32)
+        if sl.shape != tk.shape:
+            raise ValueError("one token count per slot")
+        check(lib().kv_vcache_reserve_batch(self.handle, _i32p(sl), _i32p(tk), sl.size,
+                                            _stream(torch.device("cuda", torch.cuda.current_device()))))
+
+    def trim(self, slot: int, tokens: int) -> None:
+        torch = _torch()
+        check(lib().kv_vcache_trim(self.handle, slot, tokens,
+                                   _stream(torch.device("cuda", torch.cuda.current_device()))))
+
+    def release_spares(self) -> None:
+        check(lib().kv_vcache_release_spares(self.handle))
+
+    def capacity(self, slot: int) -> int:
+        n = C.c_int32()
+        check(lib().kv_vcache_capacity(self.handle, slot, C.byref(n)))
+        return n.value
+
+    def stats(self) -> dict:
+        st = VCacheStats()
+        check(lib().kv_vcache_stats(self.handle, C.byref(st)))
+        return {name: getattr(st, name) for name, _ in VCacheStats._fields_}
+
+    def view(self, which: str, slot: int, tokens: int):
+        """A torch view ``[tokens, Hkv, D]`` of the first ``tokens`` tokens of a slot's
+        K or V range; refused beyond the slot's capacity (unmapped memory)."""
+        torch = _torch()
+        if not 0 <= slot < self.num_slots or not 0 <= tokens <= self.capacity(slot):
+            raise ValueError("view outside the slot's mapped capacity")
+        base = self.k_base if which == "k" else self.v_base
+        elem = 2
+        row = self.num_kv_heads * self.head_dim
+        ptr = base + slot * self.slot_tokens * row * elem
+
+        class _Arr:
+            __cuda_array_interface__ = {"shape": (tokens, self.num_kv_heads, self.head_dim),
+                                        "typestr": "<f2", "data": (ptr, False), "version": 3,
+                                        "strides": None}
+        t = torch.as_tensor(_Arr(), device=torch.device("cuda", torch.cuda.current_device()))
+        return t.view(torch.float16 if self.dtype == "f16" else torch.bfloat16)
+
+
+def reshape_and_cache_vcache(k_new, v_new, vc: VCache, slots, positions) -> None:
+    """Writes ``k_new/v_new [T, Hkv, D]`` to position ``positions[t]`` of slot ``slots[t]``
+    (CUDA int32 [T]) of a virtually contiguous cache."""
+    torch = _torch()
+    dev = _cuda(k_new, v_new, slots, positions)
+    if slots.dtype != torch.int32 or positions.dtype != torch.int32:
+        raise TypeError("slots and positions must be int32")
+    T = k_new.shape[0]
+    if tuple(k_new.shape) != (T, vc.num_kv_heads, vc.head_dim) or v_new.shape != k_new.shape:
+        raise ValueError("shape mismatch")
+    if slots.numel() != T or positions.numel() != T:
+        raise ValueError("one slot and one position per token")
+    if _code(k_new) != _DTYPES[vc.dtype] or v_new.dtype != k_new.dtype:
+        raise TypeError("dtype mismatch")
+    check(lib().reshape_and_cache_vcache(k_new.data_ptr(), v_new.data_ptr(), vc.handle,
+                                         slots.data_ptr(), positions.data_ptr(), T, _stream(dev)))
+
+
+def attention_decode_vcache(q, vc: VCache, seq_slots, context_lens, scale: float, out=None, *,
+                            max_context_len: int | None = None, partition_size: int = 0,
+                            workspace=None):
+    """Decode attention over a virtually contiguous cache: sequence s reads slot
+    ``seq_slots[s]``; returns ``out [S, Hq, D]``."""
+    torch = _torch()
+    dev = _cuda(q, seq_slots, context_lens)
+    if seq_slots.dtype != torch.int32 or context_lens.dtype != torch.int32:
+        raise TypeError("seq_slots and context_lens must be int32")
+    S, Hq, D = q.shape
+    if D != vc.head_dim or _code(q) != _DTYPES[vc.dtype]:
+        raise ValueError("q does not match the cache")
+    mcl = vc.max_tokens if max_context_len is None else int(max_context_len)
+    if out is None:
+        out = torch.empty_like(q)
+    _cuda(out)
+    ws_ptr, ws_bytes = None, 0
+    need = decode_workspace_bytes(S, Hq, D, mcl, partition_size)
+    if need:
+        if workspace is None:
+            workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+        _cuda(workspace)
+        ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()
+    check(lib().attention_decode_vcache(q.data_ptr(), vc.handle, seq_slots.data_ptr(),
+                                        context_lens.data_ptr(), S, Hq, mcl, float(scale),
+                                        int(partition_size), ws_ptr, ws_bytes, out.data_ptr(),
+                                        _stream(dev)))
     return out
 
 

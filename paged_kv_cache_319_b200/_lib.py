@@ -44,6 +44,12 @@ class PoolStats(C.Structure):
                                          "waste_slots", "cow_copies_total", "num_seqs")]
 
 
+class VCacheStats(C.Structure):
+    _fields_ = [(n, C.c_int64) for n in ("chunk_bytes", "mapped_chunks", "spare_chunks",
+                                         "mapped_bytes", "reserved_bytes", "map_calls",
+                                         "create_calls", "slot_tokens")]
+
+
 i32, i64, u64, f32 = C.c_int32, C.c_int64, C.c_uint64, C.c_float
 vp, sz = C.c_void_p, C.c_size_t
 P_i32, P_i64 = C.POINTER(C.c_int32), C.POINTER(C.c_int64)
@@ -94,6 +100,23 @@ SIGNATURES = {
                                        sz]),
     "paged_attention_decode_noalloc": (C.c_int, [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,
                                                  i32, i32, f32, i32, vp, i32, vp]),
+    "kv_vcache_create": (C.c_int, [i32, i32, i32, i32, i32, C.POINTER(vp)]),
+    "kv_vcache_destroy": (C.c_int, [vp]),
+    "kv_vcache_reserve": (C.c_int, [vp, i32, i32, vp]),
+    "kv_vcache_reserve_batch": (C.c_int, [vp, P_i32, P_i32, i32, vp]),
+    "kv_vcache_trim": (C.c_int, [vp, i32, i32, vp]),
+    "kv_vcache_release_spares": (C.c_int, [vp]),
+    "kv_vcache_capacity": (C.c_int, [vp, i32, P_i32]),
+    "kv_vcache_layout": (C.c_int, [vp, C.POINTER(vp), C.POINTER(vp), P_i32]),
+    "kv_vcache_stats": (C.c_int, [vp, C.POINTER(VCacheStats)]),
+    "reshape_and_cache_vcache": (C.c_int, [vp, vp, vp, vp, vp, i32, vp]),
+    "attention_decode_vcache": (C.c_int, [vp, vp, vp, vp, i32, i32, i32, f32, i32, vp, sz, vp,
+                                          vp]),
+    "kvp_decode_pack_plan_words": (sz, [i32, i32]),
+    "kv_decode_pack_plan": (C.c_int, [P_i32, P_i32, i32, i32, i32, i32, i32, i32, i32, P_i32, sz]),
+    "kvp_decode_packed_workspace_bytes": (sz, [P_i32, i32, i32, i32]),
+    "paged_attention_decode_packed": (C.c_int, [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32,
+                                                f32, P_i32, vp, vp, sz, vp, i32, vp]),
     "kvp_check_device_error": (C.c_int, [vp]),
     "kvp_selftest_bounded_wait": (C.c_int, [i32, vp]),
     "kvp_last_error_message": (C.c_char_p, []),

@@ -23,6 +23,7 @@ BUILD_DIR = os.path.join(PKG, "_build")
 SOURCES = [
     os.path.join(CSRC, "host", "block_pool.cpp"),
     os.path.join(CSRC, "host", "group_plan.cpp"),
+    os.path.join(CSRC, "host", "vcache.cpp"),
     os.path.join(CSRC, "kvp_device.cu"),
 ]
 

@@ -44,6 +44,43 @@ __global__ void __launch_bounds__(256) reshape_and_cache_kernel(
   }
 }
 
+// Virtually contiguous cache: token t's K and V rows go to position pos[t] of
+// slot slots[t], i.e. row (slot * slot_tokens + pos) * Hkv + h of the
+// token-major ranges. A position outside [0, cap[slot]) (the slot's mapped
+// capacity) or a slot >= num_slots is skipped and recorded, so no store
+// reaches an unmapped address; a negative slot is padding. Chunks as in
+// reshape_and_cache_kernel: c moves chunk c % cpr of row c / cpr.
+__global__ void __launch_bounds__(256) vcache_write_kernel(
+    const uint4* __restrict__ k_new, const uint4* __restrict__ v_new, uint4* __restrict__ k_base,
+    uint4* __restrict__ v_base, const int32_t* __restrict__ slots, const int32_t* __restrict__ pos,
+    const int32_t* __restrict__ cap, uint32_t num_chunks, uint32_t num_kv_heads, uint32_t log2_cpr,
+    int32_t num_slots, int64_t slot_tokens) {
+  const uint32_t stride = gridDim.x * blockDim.x;
+  const uint32_t cpr_mask = (1u << log2_cpr) - 1u;
+  for (uint32_t c = blockIdx.x * blockDim.x + threadIdx.x; c < num_chunks; c += stride) {
+    const uint32_t row = c >> log2_cpr;
+    const uint32_t j = c & cpr_mask;
+    const uint32_t t = row / num_kv_heads;
+    const uint32_t h = row - t * num_kv_heads;
+    const int32_t s = __ldg(slots + t);
+    if (s < 0) continue;  // padding token
+    const int32_t p = __ldg(pos + t);
+    if (s >= num_slots || p < 0 || p >= __ldg(cap + s)) {
+      if (h == 0 && j == 0) record_error(KVP_DEVERR_SLOT, uint64_t(t));
+      continue;
+    }
+    const int64_t dst = ((int64_t(s) * slot_tokens + p) * num_kv_heads + h) * (int64_t(1) << log2_cpr) + j;
+    k_base[dst] = __ldg(k_new + c);
+    v_base[dst] = __ldg(v_new + c);
+  }
+}
+
+// One slot's capacity in the device copy, in stream order with the kernels
+// that read it.
+__global__ void vcache_set_cap_kernel(int32_t* cap, int32_t slot, int32_t value) {
+  if (threadIdx.x == 0 && blockIdx.x == 0) cap[slot] = value;
+}
+
 // FP8 cache: the new tokens' K and V rows quantised into their slots, KV head
 // h with its own scales: code = E4M3(x / scale[h]), the division correctly
 // rounded in fp32, then rounded to the nearest E4M3 value (ties to even) and
@@ -98,7 +135,12 @@ __global__ void __launch_bounds__(256) reshape_and_cache_fp8_kernel(
 
 // Block-level copy-on-write: block dst of K and V becomes a copy of block src
 // ["Your GPU was mostly empty", section "Paging's second gift: copy-on-write"].
-// grid.y = pair, grid.z = 0 (K) / 1 (V); grid.x strides over the block's chunks.
+// grid.y = pair, grid.z = 0 (K) / 1 (V); grid.x strides over the block's chunks,
+// each thread keeping kCopyUnroll 16-byte loads in flight before its stores
+// (destinations are distinct and never sources, so the loads may take the
+// read-only path).
+constexpr int kCopyUnroll = 4;
+
 __global__ void __launch_bounds__(256) copy_blocks_kernel(uint4* __restrict__ k_cache,
                                                           uint4* __restrict__ v_cache,
                                                           const int32_t* __restrict__ pairs,
@@ -116,9 +158,20 @@ __global__ void __launch_bounds__(256) copy_blocks_kernel(uint4* __restrict__ k_
   const uint4* s = base + int64_t(src) * chunks_per_block;
   uint4* d = base + int64_t(dst) * chunks_per_block;
   const int64_t stride = int64_t(gridDim.x) * blockDim.x;
-  for (int64_t c = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; c < chunks_per_block;
-       c += stride)
-    d[c] = s[c];
+  for (int64_t c0 = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; c0 < chunks_per_block;
+       c0 += stride * kCopyUnroll) {
+    uint4 r[kCopyUnroll];
+#pragma unroll
+    for (int u = 0; u < kCopyUnroll; ++u) {
+      const int64_t c = c0 + u * stride;
+      if (c < chunks_per_block) r[u] = __ldg(s + c);
+    }
+#pragma unroll
+    for (int u = 0; u < kCopyUnroll; ++u) {
+      const int64_t c = c0 + u * stride;
+      if (c < chunks_per_block) d[c] = r[u];
+    }
+  }
 }
 
 }  // namespace dev

@@ -26,6 +26,7 @@
 
 #include <math.h>
 
+#include "../pack_layout.h"
 #include "common.cuh"
 
 namespace kvp {
@@ -65,6 +66,16 @@ struct DecodeArgs {
   // and values (a cached code c of head g stands for value(c) * scale[g]).
   const float* k_scale;
   const float* v_scale;
+  // Virtually contiguous cache only (null otherwise): the slot of each
+  // sequence and each slot's mapped capacity; a tile of sequence s starting at
+  // token j has the token coordinate vc_seq_slots[s] * vc_slot_tokens + j.
+  const int32_t* vc_seq_slots;
+  const int32_t* vc_cap;
+  int32_t vc_slot_tokens;
+  int32_t vc_num_slots;
+  // Packed grouped decode: `plan` is a packed plan (pack_layout.h); every
+  // (sequence, head) has one partial per chunk of its group's block stream.
+  int32_t plan_packed;
 };
 
 __device__ __forceinline__ uint8_t* align_1024(uint8_t* p) {
@@ -80,6 +91,34 @@ __device__ __forceinline__ int32_t load_ctx(const DecodeArgs& a, int32_t s, bool
     ctx = ctx < 0 ? 0 : a.max_context_len;
   }
   return ctx;
+}
+
+// Context length of sequence s as every kernel of a call reads it: clamped as
+// by load_ctx and, over a virtually contiguous cache, to the mapped capacity
+// of the sequence's slot (a slot out of range reads nothing), so no tile ever
+// reaches an unmapped address.
+__device__ __forceinline__ int32_t seq_ctx(const DecodeArgs& a, int32_t s, bool report) {
+  int32_t ctx = load_ctx(a, s, report);
+  if (a.vc_cap) {
+    const int32_t slot = __ldg(a.vc_seq_slots + s);
+    if (slot < 0 || slot >= a.vc_num_slots) {
+      if (report) record_error(KVP_DEVERR_BLOCK_ID, (uint64_t(s) << 32) | 0xFFFFFFFFu);
+      return 0;
+    }
+    const int32_t cap = __ldg(a.vc_cap + slot);
+    if (ctx > cap) {
+      if (report) record_error(KVP_DEVERR_CTX, uint64_t(s));
+      ctx = cap;
+    }
+  }
+  return ctx;
+}
+
+// Token coordinate of the first token of sequence s's slot (virtually
+// contiguous cache; 0 for a slot out of range, whose context is 0).
+__device__ __forceinline__ int32_t vc_base(const DecodeArgs& a, int32_t s) {
+  const int32_t slot = __ldg(a.vc_seq_slots + s);
+  return (slot >= 0 && slot < a.vc_num_slots) ? slot * a.vc_slot_tokens : 0;
 }
 
 // EB: bytes per cached element (2: fp16 / bf16; 1: E4M3).
@@ -319,7 +358,12 @@ __device__ __forceinline__ void simt_tile_fp8(const uint8_t* kt, const uint8_t* 
 // warp one or two blocks, this keeps every warp's pipeline busy.
 // F8: the cache holds E4M3 codes (a.k_scale / a.v_scale set; head_dim 128);
 // q and out stay in T.
-template <typename T, int D, int BS, int NW, int NST, bool PH = false, bool F8 = false>
+// VC: a virtually contiguous cache (a.vc_* set; head_dim 128): a tile is BS
+// consecutive tokens of the sequence's slot, one 4-D box {64 dims, BS tokens,
+// 2 halves, 1 head} at the computed token coordinate, in place of a block
+// table lookup; everything else is the paged kernel's.
+template <typename T, int D, int BS, int NW, int NST, bool PH = false, bool F8 = false,
+          bool VC = false>
 __global__ void __launch_bounds__(NW * 32) decode_simt_kernel(
     const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
     const DecodeArgs a) {
@@ -351,7 +395,7 @@ __global__ void __launch_bounds__(NW * 32) decode_simt_kernel(
   if (PH && h >= a.num_q_heads) return;  // a warp past the last head (no CTA-wide sync follows)
   // the plan word and the context length are loaded together
   int32_t b_first = grouped ? ld_relaxed_gpu(a.plan + kPlanSeqWord + s) : 0;
-  const int32_t ctx = load_ctx(a, s, p == 0 && blockIdx.y == 0 && threadIdx.x == 0);
+  const int32_t ctx = seq_ctx(a, s, p == 0 && blockIdx.y == 0 && threadIdx.x == 0);
   const int32_t nblk = (ctx + BS - 1) / BS;
   int32_t slot = p;
   if (grouped) slot = (b_first + a.part_blocks - 1) / a.part_blocks + p;  // after the shared slots
@@ -385,12 +429,16 @@ __global__ void __launch_bounds__(NW * 32) decode_simt_kernel(
   const uint64_t policy = l2_policy_kv();
   const int32_t rows_total = a.num_blocks * a.num_kv_heads * BS;
 
-  // Register cache of 32 block ids: lane l holds id of index base + l.
+  // Register cache of 32 block ids: lane l holds id of index base + l (a
+  // virtually contiguous cache has no ids: the tile coordinate is computed).
   int32_t id_base = 0;
   int32_t my_id = -1;
+  const int32_t tok_base = VC ? vc_base(a, s) : 0;
   auto load_ids = [&](int32_t base) {
-    const int32_t idx = base + lane;
-    my_id = idx < nw ? __ldg(table + b0 + wfirst + kStride * idx) : -1;
+    if constexpr (!VC) {
+      const int32_t idx = base + lane;
+      my_id = idx < nw ? __ldg(table + b0 + wfirst + kStride * idx) : -1;
+    }
   };
   load_ids(0);
 
@@ -398,6 +446,14 @@ __global__ void __launch_bounds__(NW * 32) decode_simt_kernel(
     const int stage = i % NST;
     uint8_t* kt = my_tiles + size_t(stage) * 2 * C::kTileBytes;
     uint8_t* vt = kt + C::kTileBytes;
+    if constexpr (VC) {
+      // tokens [j, j + BS) of the slot, all inside its mapped range (j < ctx <= cap)
+      const int32_t tok = tok_base + (b0 + wfirst + kStride * i) * BS;
+      mbar_arrive_expect_tx(&my_bars[stage], 2 * C::kTileBytes);
+      tma_load_4d(kt, &kmap, &my_bars[stage], 0, tok, 0, g, policy);
+      tma_load_4d(vt, &vmap, &my_bars[stage], 0, tok, 0, g, policy);
+      return;
+    }
     int32_t row;
     if (id < 0 || id >= a.num_blocks) {
       record_error(KVP_DEVERR_BLOCK_ID, (uint64_t(s) << 32) | uint32_t(b0 + wfirst + kStride * i));
@@ -601,9 +657,16 @@ __global__ void __launch_bounds__(kReduceHeads * D) decode_reduce_kernel(const D
   const int row = blockIdx.y;          // a sequence, or one of its q_len query rows
   const int s = row / a.q_len;
   const int i = threadIdx.x / D, t = threadIdx.x % D;
-  const int32_t ctx = load_ctx(a, s, false);
+  const int32_t ctx = seq_ctx(a, s, false);
   int32_t nparts;
-  if (a.plan) {  // grouped: shared-prefix slots, then the sequence's own
+  if (a.plan && a.plan_packed) {  // packed: one slot per chunk of the sequence's group
+    const int32_t gid = a.plan[pack::kHdrWords + s];
+    nparts = a.plan[pack::group_offset(a.num_seqs) + int64_t(gid) * pack::kGroupWords + 3];
+    if (nparts > a.ws_slots) {
+      if (threadIdx.x == 0 && blockIdx.x == 0) record_error(KVP_DEVERR_CTX, uint64_t(s));
+      nparts = a.ws_slots;
+    }
+  } else if (a.plan) {  // grouped: shared-prefix slots, then the sequence's own
     const int32_t shared = a.plan[kPlanSeqWord + s] * (a.part_tokens / a.part_blocks);
     nparts = (shared + a.part_tokens - 1) / a.part_tokens +
              (ctx > shared ? (ctx - shared + a.part_tokens - 1) / a.part_tokens : 0);

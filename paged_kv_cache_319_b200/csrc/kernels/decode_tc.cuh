@@ -37,6 +37,7 @@
 
 #include <type_traits>
 
+#include "../pack_layout.h"
 #include "common.cuh"
 #include "decode_group.cuh"
 #include "decode_simt.cuh"
@@ -48,7 +49,7 @@ static_assert(grp::kHdrWords == kPlanSeqWord, "plan layout");
 
 namespace tc {
 
-enum Mode : int { kPlain = 0, kGrouped = 1, kMultiQuery = 2 };
+enum Mode : int { kPlain = 0, kGrouped = 1, kMultiQuery = 2, kContig = 3, kPacked = 4 };
 
 constexpr int kD = 128;             // head_dim
 constexpr int kN = 16;              // MMA N (query heads of a group, padded)
@@ -192,9 +193,20 @@ struct Unit {
   int32_t nparts;
   int32_t sg;                  // grouped decode: subgroup of a shared-prefix unit, else -1
   int32_t slot;                // workspace slot of the unit's partial
+  int32_t vbase;               // virtually contiguous cache: token coordinate of the slot
+  int32_t e0;                  // packed decode: the chunk's first entry
 };
 
+// Context length of sequence s as the tensor-core kernel reads it (VC: over a
+// virtually contiguous cache, clamped to the slot's capacity).
+template <bool VC>
+__device__ __forceinline__ int32_t ctx_of(const DecodeArgs& a, int32_t s, bool report) {
+  if constexpr (VC) return seq_ctx(a, s, report);
+  return load_ctx(a, s, report);
+}
+
 // ctx_sm: the batch's clamped context lengths in shared memory, or null.
+template <bool VC = false>
 __device__ __forceinline__ bool decode_unit(const DecodeArgs& a, int64_t u, Unit& w,
                                             const int32_t* ctx_sm) {
   const int64_t per_seq = int64_t(a.pmax) * a.num_kv_heads;
@@ -202,7 +214,8 @@ __device__ __forceinline__ bool decode_unit(const DecodeArgs& a, int64_t u, Unit
   const int32_t rem = int32_t(u - int64_t(w.s) * per_seq);
   w.p = rem / a.num_kv_heads;
   w.g = rem - w.p * a.num_kv_heads;
-  w.ctx = ctx_sm ? ctx_sm[w.s] : load_ctx(a, w.s, w.g == 0 && w.p == 0);
+  w.ctx = ctx_sm ? ctx_sm[w.s] : ctx_of<VC>(a, w.s, w.g == 0 && w.p == 0);
+  w.vbase = VC ? vc_base(a, w.s) : 0;
   w.nparts = (w.ctx + a.part_tokens - 1) / a.part_tokens;
   if (w.p > 0 && w.p >= w.nparts) return false;  // empty (p == 0 always runs)
   w.tok_begin = w.p * a.part_tokens;
@@ -225,8 +238,10 @@ struct GroupHdr {
   int64_t shared_units;
   int32_t psh;          // most shared partitions of any subgroup
   const int32_t* cblk;  // per sequence: shared-prefix blocks
-  const int32_t* subs;  // subgroup table
+  const int32_t* subs;  // subgroup table (packed decode: the group table)
   bool in_smem;         // cblk and subs point at the CTA's shared-memory copy
+  const int32_t* units; // packed decode: the unit table
+  const int32_t* ents;  // packed decode: the entries
 };
 
 __device__ __forceinline__ int32_t plan_at(const GroupHdr& gh, const int32_t* p) {
@@ -252,6 +267,7 @@ __device__ __forceinline__ bool decode_unit_grp(const DecodeArgs& a, int64_t u, 
     w.tok_end = min(shared, w.tok_begin + a.part_tokens);
     w.s = plan_at(gh, e + 4);  // every member holds the same blocks here
     w.ctx = shared;
+    w.vbase = 0;
     w.nparts = 0;
     w.slot = w.p;
     return true;
@@ -263,6 +279,7 @@ __device__ __forceinline__ bool decode_unit_grp(const DecodeArgs& a, int64_t u, 
   w.p = rem / a.num_kv_heads;
   w.g = rem - w.p * a.num_kv_heads;
   w.ctx = ctx_sm ? ctx_sm[w.s] : load_ctx(a, w.s, w.g == 0 && w.p == 0);
+  w.vbase = 0;
   const int32_t shared = plan_at(gh, gh.cblk + w.s) * BS;
   w.tok_begin = shared + w.p * a.part_tokens;
   if (w.tok_begin >= w.ctx) return false;
@@ -271,6 +288,29 @@ __device__ __forceinline__ bool decode_unit_grp(const DecodeArgs& a, int64_t u, 
   w.sg = -1;
   w.slot = (shared + a.part_tokens - 1) / a.part_tokens + w.p;
   return true;
+}
+
+// Packed decode: unit u is (unit record u / Hkv, KV head u % Hkv); its tokens
+// are the blocks of one chunk of its group's stream (n * BS token rows, which
+// the entries' column masks and valid counts qualify).
+template <int BS>
+__device__ __forceinline__ bool decode_unit_pack(const DecodeArgs& a, int64_t u, Unit& w,
+                                                 const GroupHdr& gh) {
+  const int64_t ui = u / a.num_kv_heads;
+  w.g = int32_t(u - ui * a.num_kv_heads);
+  const int32_t* ur = gh.units + ui * pack::kUnitWords;
+  w.sg = __ldg(ur + 0);
+  w.e0 = __ldg(ur + 1);
+  const int32_t n = __ldg(ur + 2);
+  w.slot = __ldg(ur + 3);
+  w.p = w.slot;
+  w.tok_begin = 0;
+  w.tok_end = n * BS;
+  w.ctx = n * BS;
+  w.s = __ldg(gh.subs + int64_t(w.sg) * pack::kGroupWords + 4);
+  w.nparts = 0;
+  w.vbase = 0;
+  return n > 0;
 }
 
 __device__ __forceinline__ int32_t chunks_of(const Unit& w) {
@@ -286,8 +326,10 @@ __device__ __forceinline__ int32_t tiles_of(const Unit& w, int32_t c) {
 // blockIdx.x + gridDim.x, ... (empty partitions and units without tokens
 // skipped), each cut into chunks of up to kChunkTok tokens. Every warp role
 // walks the same stream.
-template <bool GRP, int BS>
+template <int MODE, int BS>
 struct ChunkStream {
+  static constexpr bool GRP = MODE == kGrouped;
+  static constexpr bool PK = MODE == kPacked;
   int64_t u, stride, num_units;
   const int32_t* ctx_sm;
   GroupHdr gh;
@@ -309,7 +351,9 @@ struct ChunkStream {
   }
   __device__ __forceinline__ void next_unit(const DecodeArgs& a) {
     for (u += stride; u < num_units; u += stride) {
-      const bool has = GRP ? decode_unit_grp<BS>(a, u, w, ctx_sm, gh) : decode_unit(a, u, w, ctx_sm);
+      const bool has = PK    ? decode_unit_pack<BS>(a, u, w, gh)
+                       : GRP ? decode_unit_grp<BS>(a, u, w, ctx_sm, gh)
+                             : decode_unit<BS == kTileTok>(a, u, w, ctx_sm);
       if (has && (nch = chunks_of(w)) > 0) {
         c = 0;
         return;
@@ -327,7 +371,10 @@ struct ChunkStream {
 
 }  // namespace tc
 
-// MODE tc::kPlain: decode. MODE tc::kGrouped: grouped decode (a.plan set;
+// MODE tc::kContig: decode over a virtually contiguous cache (a.vc_* set,
+// BS = 128): a tile is 128 consecutive tokens of the sequence's slot, loaded
+// as one 4-D box per 64-dim half of K and one for V at the computed token
+// coordinate, with no block table. MODE tc::kPlain: decode. MODE tc::kGrouped: grouped decode (a.plan set;
 // launched after the plan kernel with programmatic serialisation); num_units
 // then counts the per-sequence units (0 when the CUDA-core kernel takes them)
 // and the shared-prefix units are read from the plan. MODE tc::kMultiQuery:
@@ -342,7 +389,9 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
   using namespace tc;
   constexpr bool GRP = MODE == kGrouped;
   constexpr bool MQ = MODE == kMultiQuery;
-  static_assert(BS == 16 || BS == 32, "block_size 16 or 32");
+  constexpr bool VC = MODE == kContig;
+  constexpr bool PK = MODE == kPacked;
+  static_assert(VC ? BS == kTileTok : (BS == 16 || BS == 32), "block_size 16 or 32");
   using L = tc::Cfg<NG>;
   constexpr int kStages = L::kStages;
   constexpr int kPBytes = L::kPBytes;
@@ -381,7 +430,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
   const bool plan_sm = GRP && a.num_seqs <= L::kPlanCap;
   if (ctx_sm) {
     for (int i = threadIdx.x; i < a.num_seqs; i += blockDim.x)
-      ctx_cache[i] = load_ctx(a, i, blockIdx.x == 0);  // clamped; out-of-range reported once
+      ctx_cache[i] = tc::ctx_of<VC>(a, i, blockIdx.x == 0);  // clamped; out-of-range reported once
   }
   __shared__ int abort_flag;
 
@@ -425,7 +474,9 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
   const uint32_t tmem_base = *tmem_ptr;
 
   const int32_t G = a.num_q_heads / a.num_kv_heads;
-  const int32_t rows_total = a.num_blocks * a.num_kv_heads * BS;
+  // the coordinate of a tile past the tensor (read as zeros): paged rows, or
+  // the virtually contiguous cache's tokens
+  const int32_t rows_total = VC ? a.vc_num_slots * a.vc_slot_tokens : a.num_blocks * a.num_kv_heads * BS;
   tc::GroupHdr gh{0, 0, nullptr, nullptr, false};
   if constexpr (GRP) {
     pdl_wait();  // the plan kernel has completed and its writes are visible
@@ -455,6 +506,12 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
     }
   }
 
+  if constexpr (PK) {  // the packed plan: uploaded before the launch, read-only here
+    gh.subs = a.plan + pack::group_offset(a.num_seqs);
+    gh.units = a.plan + __ldg(a.plan + pack::kUnitOffset);
+    gh.ents = a.plan + __ldg(a.plan + pack::kEntryOffset);
+  }
+
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     // Ring order: K tiles of chunk 0, then for every chunk i: K tiles of chunk
@@ -472,19 +529,22 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
     // Lane j's block of a chunk (one chunk = 512 / BS <= 32 blocks): its table
     // entry is loaded a chunk ahead (chunk_id, not waited on) and turned into a
     // TMA row, range-checked, when the chunk's tiles are issued (id_row).
-    auto lane_has_block = [&](const tc::ChunkStream<GRP, BS>& cs, int32_t& bidx) {
+    auto lane_has_block = [&](const tc::ChunkStream<MODE, BS>& cs, int32_t& bidx) {
       const tc::Unit& w = cs.w;
       bidx = (w.tok_begin + cs.c * kChunkTok) / BS + lane;
       return lane < cs.tiles() * kBlocksPerTile && bidx < (w.ctx + BS - 1) / BS;
     };
-    auto chunk_id = [&](const tc::ChunkStream<GRP, BS>& cs) -> int32_t {
+    auto chunk_id = [&](const tc::ChunkStream<MODE, BS>& cs) -> int32_t {
       int32_t bidx;
       if (!lane_has_block(cs, bidx)) return -1;
+      if constexpr (VC) return 0;  // no table: the coordinate is computed
+      if constexpr (PK) return __ldg(gh.ents + 2 * (int64_t(cs.w.e0) + bidx));
       return __ldg(a.block_tables + int64_t(cs.w.s) * a.max_blocks_per_seq + bidx);
     };
-    auto id_row = [&](const tc::ChunkStream<GRP, BS>& cs, int32_t id) -> int32_t {
+    auto id_row = [&](const tc::ChunkStream<MODE, BS>& cs, int32_t id) -> int32_t {
       int32_t bidx;
       if (!lane_has_block(cs, bidx)) return rows_total;  // past the sequence: zeros
+      if constexpr (VC) return cs.w.vbase + bidx * kTileTok;  // inside the slot's capacity
       if (id < 0 || id >= a.num_blocks) {
         record_error(KVP_DEVERR_BLOCK_ID, (uint64_t(cs.w.s) << 32) | uint32_t(bidx));
         return rows_total;
@@ -494,7 +554,8 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
     // Key tiles: two 2-D boxes per block (its rows of each 64-dim region of the
     // stage). Value tiles: one 3-D box per block ([half][BS rows][64], 256 * BS
     // bytes at block j's offset), which the PV descriptors read in place.
-    auto load_tiles = [&](const CUtensorMap* map, int32_t row, int32_t ntile, bool values) {
+    auto load_tiles = [&](const CUtensorMap* map, int32_t row, int32_t head, int32_t ntile,
+                          bool values) {
       for (int32_t t = 0; t < ntile && ok; ++t, ++ctr) {
         const uint32_t st = ctr % kStages;
         if (lane == 0) {
@@ -504,7 +565,16 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) break;
         const int j = lane - t * kBlocksPerTile;  // block j of this tile
-        if (j >= 0 && j < kBlocksPerTile) {
+        if (VC && j == 0) {
+          // one box {64, 128 tokens, halves, 1 head}: K one per 64-dim region, V both halves
+          uint8_t* dst = ring + st * kStageBytes;
+          if (values) {
+            tma_load_4d(dst, map, &full[st], 0, row, 0, head, pol_kv);
+          } else {
+            tma_load_4d(dst, map, &full[st], 0, row, 0, head, pol_kv);
+            tma_load_4d(dst + kRegionBytes, map, &full[st], 0, row, 1, head, pol_kv);
+          }
+        } else if (!VC && j >= 0 && j < kBlocksPerTile) {
           if (values) {
             tma_load_3d(ring + st * kStageBytes + j * BS * 256, map, &full[st], 0, row, 0, pol_kv);
           } else {
@@ -523,12 +593,12 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
     // (c ^ (j & 7)) * 16) before the previous unit's value tiles, since the MMA
     // needs this Q before it frees the ring stages those wait for.
     constexpr int kQChunksPerLane = kN * 16 / 32;
-    auto is_gather = [&](const tc::ChunkStream<GRP, BS>& cs) {
-      return cs.valid && cs.first() && ((GRP && cs.w.sg >= 0) || MQ);
+    auto is_gather = [&](const tc::ChunkStream<MODE, BS>& cs) {
+      return cs.valid && cs.first() && ((GRP && cs.w.sg >= 0) || MQ || PK);
     };
-    auto gather_q = [&](const tc::ChunkStream<GRP, BS>& cs, uint4 (&v)[kQChunksPerLane]) {
-      const int32_t* e = GRP ? tc::sub_entry(gh, cs.w.sg) : nullptr;
-      const int32_t ncol = GRP ? tc::plan_at(gh, e + 1) * G : a.q_count * G;
+    auto gather_q = [&](const tc::ChunkStream<MODE, BS>& cs, uint4 (&v)[kQChunksPerLane]) {
+      const int32_t* e = (GRP || PK) ? tc::sub_entry(gh, cs.w.sg) : nullptr;
+      const int32_t ncol = (GRP || PK) ? tc::plan_at(gh, e + 1) * G : a.q_count * G;
 #pragma unroll
       for (int i = 0; i < kQChunksPerLane; ++i) {
         const int idx = lane + 32 * i;
@@ -536,16 +606,16 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
         v[i] = make_uint4(0, 0, 0, 0);
         if (j < ncol) {
           const int32_t m = j / G;  // member (grouped) or query token (multi-query)
-          const int64_t seq_row = GRP ? int64_t(tc::plan_at(gh, e + 4 + m))
+          const int64_t seq_row = (GRP || PK) ? int64_t(tc::plan_at(gh, e + 4 + m))
                                       : int64_t(cs.w.s) * a.q_len + a.q_first + m;
           const int64_t qrow = seq_row * a.num_q_heads + cs.w.g * G + (j - m * G);
           v[i] = __ldg(reinterpret_cast<const uint4*>(static_cast<const T*>(a.q) + qrow * kD) + ch);
         }
       }
     };
-    tc::ChunkStream<GRP, BS> cur;
+    tc::ChunkStream<MODE, BS> cur;
     cur.init(a, blockIdx.x, gridDim.x, num_units, ctx_sm, gh);
-    int32_t pend_row = rows_total, pend_tiles = 0;
+    int32_t pend_row = rows_total, pend_tiles = 0, pend_head = 0;
     bool have_pend = false;
     int32_t id = cur.valid ? chunk_id(cur) : -1;
     uint4 qv[kQChunksPerLane];
@@ -553,7 +623,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
     while (cur.valid && ok) {
       // the next chunk's block ids (and a grouped unit's Q rows) are loaded now
       // and used one iteration later
-      tc::ChunkStream<GRP, BS> nxt = cur;
+      tc::ChunkStream<MODE, BS> nxt = cur;
       nxt.advance(a);
       const int32_t id_next = nxt.valid ? chunk_id(nxt) : -1;
       uint4 qn[kQChunksPerLane];
@@ -589,9 +659,10 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
         }
         ++ucnt;
       }
-      if (ok) load_tiles(&kmap, row, nt, false);
-      if (have_pend && ok) load_tiles(&vmap, pend_row, pend_tiles, true);
+      if (ok) load_tiles(&kmap, row, cur.w.g, nt, false);
+      if (have_pend && ok) load_tiles(&vmap, pend_row, pend_head, pend_tiles, true);
       pend_row = row;
+      pend_head = cur.w.g;
       pend_tiles = nt;
       have_pend = true;
       id = id_next;
@@ -601,7 +672,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
       }
       cur = nxt;
     }
-    if (have_pend && ok) load_tiles(&vmap, pend_row, pend_tiles, true);
+    if (have_pend && ok) load_tiles(&vmap, pend_row, pend_head, pend_tiles, true);
     if (!ok) {
       atomicExch(&abort_flag, 1);
       if (lane == 0)  // drain the loads that may still be in flight
@@ -640,7 +711,10 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
     // issues; in the chunk's last tile the lanes first zero the V rows of
     // tokens past the end of the sequence (rows >= zero_from), which hold
     // whatever the pool had there: p is 0 for them, but 0 * inf is NaN.
-    auto pv = [&](uint32_t b, uint32_t use, int32_t ntile, int32_t zero_from) {
+    // Packed decode: nv is the valid tokens of this lane's block of the chunk
+    // (lane j holds block j); rows past them (a member's last block) are zeroed
+    // the same way.
+    auto pv = [&](uint32_t b, uint32_t use, int32_t ntile, int32_t zero_from, int32_t nv) {
       if (lane == 0) {
         ok = mbar_wait(&p_full[b], use & 1u, 0x7700u);
         if (ok) ok = mbar_wait(&o_free[b], (use & 1u) ^ 1u, 0x7800u);
@@ -668,6 +742,21 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
           }
           fence_proxy_async_smem();
         }
+        if constexpr (PK) {
+          const int jb = lane - t * kBlocksPerTile;  // this lane's block within the tile
+          if (jb >= 0 && jb < kBlocksPerTile && nv < BS) {
+            uint8_t* tile = ring + st * kStageBytes;
+            for (int rr = nv; rr < BS; ++rr) {
+              uint8_t* r0 = tile + jb * (BS * 256) + rr * 128;
+#pragma unroll
+              for (int q = 0; q < 8; ++q) {
+                reinterpret_cast<uint4*>(r0)[q] = make_uint4(0, 0, 0, 0);
+                reinterpret_cast<uint4*>(r0 + BS * 128)[q] = make_uint4(0, 0, 0, 0);
+              }
+            }
+            fence_proxy_async_smem();
+          }
+        }
         __syncwarp();
         if (lane == 0) {
           tc_fence_after();
@@ -691,14 +780,19 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
         umma_commit(&p_free[b]);
       }
     };
-    tc::ChunkStream<GRP, BS> cur;
+    tc::ChunkStream<MODE, BS> cur;
     cur.init(a, blockIdx.x, gridDim.x, num_units, ctx_sm, gh);
     uint32_t pend_b = 0, pend_use = 0;
-    int32_t pend_tiles = 0, pend_zero = kTileTok;
+    int32_t pend_tiles = 0, pend_zero = kTileTok, pend_nv = BS;
     bool have_pend = false;
     while (cur.valid && ok) {
       const uint32_t b = cc & 1u, use = cc >> 1;
       const int32_t nt = cur.tiles();
+      int32_t nv_cur = BS;  // packed decode: valid tokens of this lane's block of the chunk
+      if constexpr (PK) {
+        if (lane < (cur.w.ctx + BS - 1) / BS)
+          nv_cur = __ldg(gh.ents + 2 * (int64_t(cur.w.e0) + lane) + 1) & 0xFF;
+      }
       if (lane == 0) {
         if (cur.first()) {
           qb = ucnt & 1u;
@@ -710,7 +804,8 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
       }
       ok = __shfl_sync(0xffffffffu, ok, 0);
       ctr = __shfl_sync(0xffffffffu, ctr, 0);  // qk advanced the ring on lane 0 only
-      if (ok && have_pend) pv(pend_b, pend_use, pend_tiles, pend_zero);
+      if (ok && have_pend) pv(pend_b, pend_use, pend_tiles, pend_zero, pend_nv);
+      pend_nv = nv_cur;
       if (cur.first()) ++ucnt;
       // valid tokens in this chunk's last tile; rows from there on are zeroed
       const int32_t ctok0 = cur.w.tok_begin + cur.c * kChunkTok;
@@ -723,7 +818,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
       ++cc;
       cur.advance(a);
     }
-    if (ok && have_pend) pv(pend_b, pend_use, pend_tiles, pend_zero);
+    if (ok && have_pend) pv(pend_b, pend_use, pend_tiles, pend_zero, pend_nv);
     if (!ok) atomicExch(&abort_flag, 1);
   } else {
     // ------------------------------------------------------------ softmax + epilogue
@@ -744,9 +839,9 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
     for (int j = 0; j < NG; ++j) col_q[j] = j / G;
     // Units without tokens (context length 0) attend to nothing: zero rows
     // (written by the reduce in the grouped decode).
-    for (int64_t u = blockIdx.x; !GRP && u < num_units; u += gridDim.x) {
+    for (int64_t u = blockIdx.x; !GRP && !PK && u < num_units; u += gridDim.x) {
       tc::Unit w;
-      if (!tc::decode_unit(a, u, w, ctx_sm) || tc::chunks_of(w) > 0) continue;
+      if (!tc::decode_unit<VC>(a, u, w, ctx_sm) || tc::chunks_of(w) > 0) continue;
       const int32_t nq = MQ ? a.q_count : 1;
       for (int i = 0; i < nq; ++i) {
         const int64_t row = MQ ? int64_t(w.s) * a.q_len + a.q_first + i : int64_t(w.s);
@@ -807,7 +902,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
       if (!ok) return;
       const int32_t h0 = pw.g * G;
       // grouped decode: a shared-prefix unit's columns are its members' heads
-      const int32_t* ge = (GRP && pw.sg >= 0) ? tc::sub_entry(gh, pw.sg) : nullptr;
+      const int32_t* ge = ((GRP && pw.sg >= 0) || PK) ? tc::sub_entry(gh, pw.sg) : nullptr;
       const int32_t ncol = ge ? tc::plan_at(gh, ge + 1) * G : (MQ ? a.q_count * G : G);
 #pragma unroll
       for (int j = 0; j < NG; ++j) {
@@ -821,7 +916,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
             const int32_t i = col_q[j];
             row_sh = (int64_t(pw.s) * a.q_len + a.q_first + i) * a.num_q_heads + h0 + (j - i * G);
           }
-          if (!GRP && pw.nparts <= 1) {
+          if (!GRP && !PK && pw.nparts <= 1) {
             const float y = Lj > 0.f ? acc[j] / Lj : 0.f;
             static_cast<uint16_t*>(a.out)[row_sh * kD + r] = Elem<T>::from_float(y);
           } else {
@@ -838,12 +933,29 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
       }
     };
 
-    tc::ChunkStream<GRP, BS> cur;
+    tc::ChunkStream<MODE, BS> cur;
     cur.init(a, blockIdx.x, gridDim.x, num_units, ctx_sm, gh);
     while (cur.valid && ok) {
       const uint32_t b = cc & 1u;
       const uint32_t use = cc >> 1;
       const int32_t ntile = cur.tiles();
+      // packed decode: per tile, the columns that take this thread's token row
+      // (its block's column mask, none past the block's valid tokens)
+      uint32_t pm[kChunkTiles];
+#pragma unroll
+      for (int t = 0; t < kChunkTiles; ++t) pm[t] = 0xFFFFFFFFu;
+      if constexpr (PK) {
+        const int32_t nblk = (cur.w.ctx + BS - 1) / BS;
+#pragma unroll
+        for (int t = 0; t < kChunkTiles; ++t) {
+          const int32_t blk = t * kBlocksPerTile + r / BS;
+          pm[t] = 0;
+          if (blk < nblk) {
+            const uint32_t wd = uint32_t(__ldg(gh.ents + 2 * (int64_t(cur.w.e0) + blk) + 1));
+            pm[t] = (r % BS) < int32_t(wd & 0xFFu) ? (wd >> 8) : 0u;
+          }
+        }
+      }
       const int32_t ctok0 = cur.w.tok_begin + cur.c * kChunkTok;
       const int32_t ctok1 = min(cur.w.tok_end, ctok0 + kChunkTok);
       // ---- scores of this thread's tokens (row r of each tile)
@@ -875,7 +987,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
         const bool valid = t < ntile && tok < ctok1;
 #pragma unroll
         for (int j = 0; j < NG; ++j) {
-          const bool vis = valid && (!MQ || tok < lim0 + col_q[j]);
+          const bool vis = valid && (!MQ || tok < lim0 + col_q[j]) && (!PK || ((pm[t] >> j) & 1u));
           sv[t][j] = vis ? sv[t][j] * a.scale_log2 : -INFINITY;
           cmax[j] = fmaxf(cmax[j], sv[t][j]);
         }

@@ -22,7 +22,10 @@
 #include "kernels/decode_group.cuh"
 #include "kernels/decode_simt.cuh"
 #include "kernels/decode_tc.cuh"
+#include "kernels/prefill_tc.cuh"
+#include "pack_layout.h"
 #include "status.h"
+#include "vcache.h"
 
 using kvp::fail;
 
@@ -184,6 +187,60 @@ int make_map_u8(CUtensorMap* map, const void* base, uint64_t rows, uint32_t box_
   return KVP_OK;
 }
 
+// 4-D view of a virtually contiguous cache, {64 dims, tokens, 2 halves, KV
+// heads} with strides (Hkv * 256, 128, 256) bytes, and a {64, box_tokens,
+// box_halves, 1} box: one load brings box_tokens consecutive tokens of one
+// head as [half][token][64], 128-byte swizzled (the paged tiles' layout).
+int make_map_vcache(CUtensorMap* map, const void* base, int32_t dtype, uint64_t tokens,
+                    uint32_t heads, uint32_t box_tokens, uint32_t box_halves) {
+  auto fn = encode_fn();
+  if (!fn) return fail(KVP_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  cuuint64_t dims[4] = {64, tokens, 2, heads};
+  cuuint64_t strides[3] = {uint64_t(heads) * 256, 128, 256};
+  cuuint32_t box[4] = {64, box_tokens, box_halves, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUtensorMapDataType dt =
+      dtype == KVP_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  CUresult r = fn(map, dt, 4, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(KVP_ERR_CUDA, "cuTensorMapEncodeTiled (4-D) failed (%d)", int(r));
+  return KVP_OK;
+}
+
+// q of a prefill chunk as 3-D {128 dims, heads, tokens} (strides 256 and
+// heads * 256 bytes) with a {64, G, 128 / G} box: 128 rows (token, head of the
+// group), 128-byte swizzled, per 64-dim half.
+int make_map_prefill_q(CUtensorMap* map, const void* base, int32_t dtype, uint32_t heads,
+                       uint64_t tokens, uint32_t G) {
+  auto fn = encode_fn();
+  if (!fn) return fail(KVP_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  cuuint64_t dims[3] = {128, heads, tokens};
+  cuuint64_t strides[2] = {256, uint64_t(heads) * 256};
+  cuuint32_t box[3] = {64, G, 128 / G};
+  cuuint32_t estr[3] = {1, 1, 1};
+  const CUtensorMapDataType dt =
+      dtype == KVP_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  CUresult r = fn(map, dt, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(KVP_ERR_CUDA, "cuTensorMapEncodeTiled (prefill q) failed (%d)", int(r));
+  return KVP_OK;
+}
+
+// Prefill chunks with at least this many query rows (q_len x query heads per
+// KV head, a power of two) run on the prompt-shaped kernel (128 query rows per
+// tensor-core tile); shorter ones on the decode-shaped kernel, 16 columns per
+// launch, which suits a few tokens per sequence.
+#ifndef KVP_PREFILL_TILE_MIN_ROWS
+#define KVP_PREFILL_TILE_MIN_ROWS 64
+#endif
+
+// Tokens per tile of the CUDA-core decode over a virtually contiguous cache.
+#ifndef KVP_VCACHE_SIMT_TILE
+#define KVP_VCACHE_SIMT_TILE 16
+#endif
+
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
 int ilog2(int64_t v) {
@@ -227,13 +284,13 @@ GroupWorkspace group_ws_layout(int64_t S, int64_t Hq, int64_t D, int64_t pmax) {
 // programmatic: launched with programmatic stream serialisation (the grouped
 // decode, after the shared-prefix kernel).
 template <typename T, int D, int BS, int W = KVP_SIMT_WARPS, int NST = KVP_SIMT_STAGES,
-          bool PH = false, bool F8 = false>
+          bool PH = false, bool F8 = false, bool VC = false>
 int launch_simt(const CUtensorMap& km, const CUtensorMap& vm, const kvp::dev::DecodeArgs& a,
                 cudaStream_t st, bool programmatic = false, int grid_x = 0) {
   constexpr int EB = F8 ? 1 : 2;
   constexpr int NW = (BS * D * EB >= 8192 && W > 1) ? W / 2 : W;
   using C = kvp::dev::SimtCfg<T, D, BS, NW, NST, EB>;
-  auto k = kvp::dev::decode_simt_kernel<T, D, BS, NW, NST, PH, F8>;
+  auto k = kvp::dev::decode_simt_kernel<T, D, BS, NW, NST, PH, F8, VC>;
   cudaError_t e = ensure_smem(k, C::kSmemBytes);
   if (e != cudaSuccess) return cuda_fail(e, "decode (CUDA cores): smem attribute");
   dim3 grid(grid_x > 0 ? grid_x : a.pmax, PH ? (a.num_q_heads + NW - 1) / NW : a.num_q_heads,
@@ -258,10 +315,10 @@ int launch_simt(const CUtensorMap& km, const CUtensorMap& vm, const kvp::dev::De
   return e == cudaSuccess ? KVP_OK : cuda_fail(e, "decode (CUDA cores): launch");
 }
 
-template <typename T, int BS, int NG>
+template <typename T, int BS, int NG, int MODE = kvp::dev::tc::kPlain>
 int launch_tc(const CUtensorMap& km, const CUtensorMap& vm, const CUtensorMap& qm,
               const kvp::dev::DecodeArgs& a, cudaStream_t st) {
-  auto k = kvp::dev::decode_tc_kernel<T, BS, NG, kvp::dev::tc::kPlain>;
+  auto k = kvp::dev::decode_tc_kernel<T, BS, NG, MODE>;
   // context lengths of small batches are cached in shared memory
   using Cfg = kvp::dev::tc::Cfg<NG>;
   const int ctx_bytes = a.num_seqs <= Cfg::kCtxCap ? 4 * a.num_seqs : 0;
@@ -376,6 +433,21 @@ int tc_grouped_dispatch(int bs, int ng, const CUtensorMap& km, const CUtensorMap
                  : launch_tc_grouped<T, 32, 16>(km, vm, qm, a, st, with_private, grid_ctas, programmatic);
 }
 
+// Packed grouped decode: one persistent tensor-core launch over units x KV heads.
+template <typename T, int BS, int NG>
+int launch_tc_packed(const CUtensorMap& km, const CUtensorMap& vm, const CUtensorMap& qm,
+                     const kvp::dev::DecodeArgs& a, int64_t units, cudaStream_t st) {
+  auto k = kvp::dev::decode_tc_kernel<T, BS, NG, kvp::dev::tc::kPacked>;
+  using Cfg = kvp::dev::tc::Cfg<NG>;
+  const int ctx_bytes = a.num_seqs <= Cfg::kCtxCap ? 4 * a.num_seqs : 0;
+  cudaError_t e = ensure_smem(k, Cfg::kSmemBytes + 4 * Cfg::kCtxCap);
+  if (e != cudaSuccess) return cuda_fail(e, "packed decode: smem attribute");
+  const int grid = int(units < sm_count() ? units : sm_count());
+  k<<<grid, kvp::dev::tc::kThreads, Cfg::kSmemBytes + ctx_bytes, st>>>(km, vm, qm, a, units);
+  e = cudaGetLastError();
+  return e == cudaSuccess ? KVP_OK : cuda_fail(e, "packed decode: launch");
+}
+
 // Grouped decode: the CUDA-core kernel over the sequences' own ranges
 // (grid_x partitions; 0: all).
 int launch_own_ranges(int bs, int32_t dtype, bool per_head, const CUtensorMap& km,
@@ -414,6 +486,19 @@ int launch_tc_mq(const CUtensorMap& km, const CUtensorMap& vm, const CUtensorMap
   k<<<grid, kvp::dev::tc::kThreads, Cfg::kSmemBytes + ctx_bytes, st>>>(km, vm, qm, a, units);
   e = cudaGetLastError();
   return e == cudaSuccess ? KVP_OK : cuda_fail(e, "prefill (tensor cores): launch");
+}
+
+template <typename T, int BS>
+int launch_prefill_tc(const CUtensorMap& km, const CUtensorMap& vm, const CUtensorMap& qm,
+                      const kvp::dev::DecodeArgs& a, int32_t qtiles, cudaStream_t st) {
+  auto k = kvp::dev::prefill_tc_kernel<T, BS>;
+  cudaError_t e = ensure_smem(k, kvp::dev::pf::kSmemBytes);
+  if (e != cudaSuccess) return cuda_fail(e, "prefill (prompt tiles): smem attribute");
+  const int64_t units = int64_t(a.num_seqs) * a.num_kv_heads * qtiles * a.pmax;
+  const int grid = int(units < sm_count() ? units : sm_count());
+  k<<<grid, kvp::dev::pf::kThreads, kvp::dev::pf::kSmemBytes, st>>>(km, vm, qm, a, qtiles, units);
+  e = cudaGetLastError();
+  return e == cudaSuccess ? KVP_OK : cuda_fail(e, "prefill (prompt tiles): launch");
 }
 
 template <typename T>
@@ -471,6 +556,84 @@ bool host_plan_fits(const int32_t* plan, int32_t S, int32_t MB, int32_t max_ctx,
   for (int32_t s = 0; s < S; ++s)
     if (owner[size_t(s)] < 0 && cblk[s] != 0) return false;
   return most == psh;
+}
+
+// Packed decode workspace: (m, l) and acc with one slot per chunk of the
+// longest group stream, then room for a copy of the plan.
+struct PackWorkspace {
+  size_t ml_bytes, acc_bytes, plan_bytes, total;
+};
+
+PackWorkspace pack_ws_layout(int64_t S, int64_t Hq, int64_t D, int64_t slots, int64_t plan_words) {
+  auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
+  PackWorkspace w{};
+  w.ml_bytes = up(size_t(S * Hq * slots * 2 * 4));
+  w.acc_bytes = up(size_t(S * Hq * slots * D * 4));
+  w.plan_bytes = up(size_t(plan_words * 4));
+  w.total = w.ml_bytes + w.acc_bytes + w.plan_bytes;
+  return w;
+}
+
+// Words of a packed plan as its header gives them (header, groups, units, entries).
+int64_t pack_plan_used_words(const int32_t* plan) {
+  namespace pk = kvp::pack;
+  return int64_t(plan[pk::kEntryOffset]) + 2 * int64_t(plan[pk::kEntries]);
+}
+
+// A caller's packed plan, checked word by word before any kernel reads it:
+// header and offsets consistent, every group's members distinct sequences of
+// the batch whose group word names it, every sequence in one group, every
+// group's entries inside the entry table with column masks inside its columns
+// and valid counts in [1, block_size], every (group, chunk) covered by exactly
+// one unit record with its entries. (A plan of other tables that passes still
+// gives wrong results; only its shape is checked.)
+bool pack_plan_fits(const int32_t* plan, int32_t S, int32_t bs, int32_t G, int mmax) {
+  namespace pk = kvp::pack;
+  const int32_t ngr = plan[pk::kGroups], nu = plan[pk::kUnits], ne = plan[pk::kEntries];
+  const int32_t mc = plan[pk::kMaxChunks], bpc = plan[pk::kChunkBlocks];
+  if (plan[pk::kBlockSize] != bs || bpc != 512 / bs) return false;
+  if (ngr < 0 || ngr > S || nu < 0 || ne < 0 || mc < 0) return false;
+  if (int64_t(plan[pk::kUnitOffset]) != pk::group_offset(S) + int64_t(ngr) * pk::kGroupWords) return false;
+  if (int64_t(plan[pk::kEntryOffset]) != int64_t(plan[pk::kUnitOffset]) + int64_t(nu) * pk::kUnitWords)
+    return false;
+  std::vector<int32_t> owner(size_t(S), -1);
+  std::vector<int32_t> chunk_base(size_t(ngr) + 1, 0);
+  const int32_t* ents = plan + plan[pk::kEntryOffset];
+  for (int32_t g = 0; g < ngr; ++g) {
+    const int32_t* e = plan + pk::group_offset(S) + int64_t(g) * pk::kGroupWords;
+    const int32_t first = e[0], nm = e[1], n = e[2], ch = e[3];
+    if (nm < 1 || nm > mmax || first < 0 || n < 0 || int64_t(first) + n > ne) return false;
+    if (ch != (n + bpc - 1) / bpc || ch > mc) return false;
+    chunk_base[size_t(g) + 1] = chunk_base[size_t(g)] + ch;
+    for (int m = 0; m < nm; ++m) {
+      const int32_t sq = e[4 + m];
+      if (sq < 0 || sq >= S || owner[size_t(sq)] >= 0 || plan[pk::kHdrWords + sq] != g) return false;
+      owner[size_t(sq)] = g;
+    }
+    const uint32_t cols = nm * G >= 32 ? 0xFFFFFFFFu : ((1u << (nm * G)) - 1u);
+    for (int32_t i = first; i < first + n; ++i) {
+      const uint32_t w = uint32_t(ents[2 * int64_t(i) + 1]);
+      const int32_t valid = int32_t(w & 0xFFu);
+      if (((w >> 8) & ~cols) != 0 || valid < 1 || valid > bs) return false;
+    }
+  }
+  for (int32_t sq = 0; sq < S; ++sq)
+    if (owner[size_t(sq)] < 0) return false;
+  if (chunk_base[size_t(ngr)] != nu) return false;
+  std::vector<char> seen(size_t(nu), 0);
+  const int32_t* u = plan + plan[pk::kUnitOffset];
+  for (int32_t i = 0; i < nu; ++i, u += pk::kUnitWords) {
+    const int32_t g = u[0], first = u[1], n = u[2], chunk = u[3];
+    if (g < 0 || g >= ngr) return false;
+    const int32_t* e = plan + pk::group_offset(S) + int64_t(g) * pk::kGroupWords;
+    if (chunk < 0 || chunk >= e[3] || first != e[0] + chunk * bpc ||
+        n != std::min(bpc, e[2] - chunk * bpc))
+      return false;
+    char& sn = seen[size_t(chunk_base[size_t(g)] + chunk)];
+    if (sn) return false;
+    sn = 1;
+  }
+  return true;
 }
 
 // Argument checks of the decode entry points (fn names the caller in the
@@ -556,7 +719,8 @@ int copy_blocks(void* k_cache, void* v_cache, const int32_t* pairs, int32_t num_
   if (!aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(pairs, 4))
     return fail(KVP_ERR_INVALID, "copy_blocks: misaligned pointer");
   const int64_t chunks = block_elems * eb / 16;
-  int gx = int((chunks + 255) / 256);
+  constexpr int64_t per_cta = 256 * kvp::dev::kCopyUnroll;
+  int gx = int((chunks + per_cta - 1) / per_cta);
   if (gx > 64) gx = 64;
   dim3 grid(gx, num_pairs, 2);
   kvp::dev::copy_blocks_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
@@ -705,12 +869,15 @@ int paged_attention_prefill(const void* q, const void* k_cache, const void* v_ca
   if (partition_size % 128)
     return fail(KVP_ERR_INVALID, "paged_attention_prefill: partition_size must be a multiple of 128");
   const int32_t ctx_cap = max_context_len > 0 ? max_context_len : 1;
+  // prompt-shaped chunks: 128 query rows per tile (G a power of two)
+  const bool prompt_tiles = (G & (G - 1)) == 0 && int64_t(q_len) * G >= KVP_PREFILL_TILE_MIN_ROWS;
+  const int32_t round = prompt_tiles ? 128 : block_size;
   int32_t part_tokens, pmax;
   if (partition_size > 0) {
     part_tokens = partition_size;
     pmax = (ctx_cap + partition_size - 1) / partition_size;
   } else {
-    part_tokens = ((ctx_cap + block_size - 1) / block_size) * block_size;
+    part_tokens = ((ctx_cap + round - 1) / round) * round;
     pmax = 1;
   }
   const Workspace wl = ws_layout(int64_t(num_seqs) * q_len, num_q_heads, head_dim, pmax);
@@ -742,10 +909,29 @@ int paged_attention_prefill(const void* q, const void* k_cache, const void* v_ca
   CUtensorMap km, vm, qm;
   int rc = make_map(&km, k_cache, dtype, rows, head_dim, block_size);
   if (!rc) rc = make_map_halves(&vm, v_cache, dtype, rows, block_size);
-  if (!rc)
-    rc = make_map(&qm, q, dtype, uint64_t(num_seqs) * q_len * num_q_heads, head_dim, kvp::dev::tc::kN);
   if (rc) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (prompt_tiles) {
+    rc = make_map_prefill_q(&qm, q, dtype, uint32_t(num_q_heads), uint64_t(num_seqs) * q_len,
+                            uint32_t(G));
+    if (rc) return rc;
+    const int32_t qtiles = (q_len + 128 / G - 1) / (128 / G);
+    a.q_first = 0;
+    a.q_count = q_len;
+    const bool f16 = dtype == KVP_F16;
+    using H = __half;
+    using B = __nv_bfloat16;
+    if (block_size == 16)
+      rc = f16 ? launch_prefill_tc<H, 16>(km, vm, qm, a, qtiles, st)
+               : launch_prefill_tc<B, 16>(km, vm, qm, a, qtiles, st);
+    else
+      rc = f16 ? launch_prefill_tc<H, 32>(km, vm, qm, a, qtiles, st)
+               : launch_prefill_tc<B, 32>(km, vm, qm, a, qtiles, st);
+    if (rc || pmax <= 1) return rc;
+    return f16 ? launch_reduce<H, 128>(a, st) : launch_reduce<B, 128>(a, st);
+  }
+  rc = make_map(&qm, q, dtype, uint64_t(num_seqs) * q_len * num_q_heads, head_dim, kvp::dev::tc::kN);
+  if (rc) return rc;
   // up to 16 columns per launch: 16 / G query tokens of every sequence
   const int per_launch = std::max(1, kvp::dev::tc::kN / G);
   for (int32_t c0 = 0; c0 < q_len; c0 += per_launch) {
@@ -1026,7 +1212,239 @@ int paged_attention_decode_grouped(const void* q, const void* k_cache, const voi
   return dtype == KVP_F16 ? launch_reduce<__half, 128>(a, st) : launch_reduce<__nv_bfloat16, 128>(a, st);
 }
 
+int reshape_and_cache_vcache(const void* k_new, const void* v_new, kvp_vcache* vc,
+                             const int32_t* slots, const int32_t* positions, int32_t num_tokens,
+                             kvp_stream_t stream) {
+  if (!vc) return fail(KVP_ERR_INVALID, "reshape_and_cache_vcache: NULL cache");
+  if (num_tokens < 0) return fail(KVP_ERR_INVALID, "reshape_and_cache_vcache: bad sizes");
+  if (num_tokens == 0) return KVP_OK;
+  if (!k_new || !v_new || !slots || !positions)
+    return fail(KVP_ERR_INVALID, "reshape_and_cache_vcache: NULL pointer");
+  if (!aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(slots, 4) || !aligned(positions, 4))
+    return fail(KVP_ERR_INVALID, "reshape_and_cache_vcache: misaligned pointer");
+  const int lcpr = ilog2(vc->head_dim / 8);
+  const int64_t chunks = int64_t(num_tokens) * vc->num_kv_heads * (vc->head_dim / 8);
+  if (lcpr < 0 || chunks >= (int64_t(1) << 31))
+    return fail(KVP_ERR_INVALID, "reshape_and_cache_vcache: too many tokens in one call");
+  const int threads = 256;
+  int64_t blocks = (chunks + threads - 1) / threads;
+  const int64_t cap = int64_t(sm_count()) * 16;
+  if (blocks > cap) blocks = cap;
+  kvp::dev::vcache_write_kernel<<<int(blocks), threads, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new),
+      reinterpret_cast<uint4*>(vc->k_base), reinterpret_cast<uint4*>(vc->v_base), slots, positions,
+      vc->cap_dev, uint32_t(chunks), uint32_t(vc->num_kv_heads), uint32_t(lcpr), vc->num_slots,
+      int64_t(vc->slot_tokens));
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? KVP_OK : cuda_fail(e, "reshape_and_cache_vcache: launch");
+}
+
+int attention_decode_vcache(const void* q, const kvp_vcache* vc, const int32_t* seq_slots,
+                            const int32_t* context_lens, int32_t num_seqs, int32_t num_q_heads,
+                            int32_t max_context_len, float scale, int32_t partition_size,
+                            void* workspace, size_t workspace_bytes, void* out,
+                            kvp_stream_t stream) {
+  if (!vc) return fail(KVP_ERR_INVALID, "attention_decode_vcache: NULL cache");
+  const int32_t Hkv = vc->num_kv_heads, D = vc->head_dim, dtype = vc->dtype;
+  if (num_seqs < 0 || num_q_heads <= 0 || max_context_len < 0 || partition_size < 0)
+    return fail(KVP_ERR_INVALID, "attention_decode_vcache: bad sizes");
+  if (num_q_heads % Hkv) return fail(KVP_ERR_INVALID, "attention_decode_vcache: num_q_heads %% num_kv_heads != 0");
+  if (max_context_len > vc->max_tokens)
+    return fail(KVP_ERR_INVALID, "attention_decode_vcache: max_context_len > the cache's max_tokens");
+  if (!std::isfinite(scale)) return fail(KVP_ERR_INVALID, "attention_decode_vcache: scale not finite");
+  if (num_seqs == 0) return KVP_OK;
+  if (!q || !seq_slots || !context_lens || !out)
+    return fail(KVP_ERR_INVALID, "attention_decode_vcache: NULL pointer");
+  if (!aligned(q, 16) || !aligned(out, 16) || !aligned(seq_slots, 4) || !aligned(context_lens, 4))
+    return fail(KVP_ERR_INVALID, "attention_decode_vcache: misaligned pointer");
+  const int G = num_q_heads / Hkv;
+  if (G > 16) return fail(KVP_ERR_INVALID, "attention_decode_vcache: more than 16 query heads per KV head");
+  const bool tensor_cores = G > 1;
+  constexpr int kSimtTile = KVP_VCACHE_SIMT_TILE;
+  const int tile = tensor_cores ? kvp::dev::tc::kTileTok : kSimtTile;
+  if (partition_size % tile)
+    return fail(KVP_ERR_INVALID, "attention_decode_vcache: partition_size must be a multiple of %d", tile);
+  const int32_t ctx_cap = max_context_len > 0 ? max_context_len : 1;
+  int32_t part_tokens, pmax;
+  if (partition_size > 0) {
+    part_tokens = partition_size;
+    pmax = (ctx_cap + partition_size - 1) / partition_size;
+  } else {
+    part_tokens = ((ctx_cap + tile - 1) / tile) * tile;
+    pmax = 1;
+  }
+  const Workspace wl = ws_layout(num_seqs, num_q_heads, D, pmax);
+  if (wl.total) {
+    if (!workspace || workspace_bytes < wl.total)
+      return fail(KVP_ERR_INVALID, "attention_decode_vcache: workspace of %zu bytes needed", wl.total);
+    if (!aligned(workspace, 256)) return fail(KVP_ERR_INVALID, "attention_decode_vcache: workspace not 256-byte aligned");
+  }
+  kvp::dev::DecodeArgs a{};
+  a.q = q;
+  a.out = out;
+  a.block_tables = nullptr;
+  a.context_lens = context_lens;
+  a.ws_ml = wl.total ? static_cast<float*>(workspace) : nullptr;
+  a.ws_acc = wl.total ? reinterpret_cast<float*>(static_cast<char*>(workspace) + wl.ml_bytes) : nullptr;
+  a.num_seqs = num_seqs;
+  a.num_q_heads = num_q_heads;
+  a.num_kv_heads = Hkv;
+  a.num_blocks = 1;
+  a.max_blocks_per_seq = 1;
+  a.max_context_len = max_context_len;
+  a.part_blocks = part_tokens / tile;
+  a.part_tokens = part_tokens;
+  a.pmax = pmax;
+  a.ws_slots = pmax;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.q_len = 1;
+  a.q_first = 0;
+  a.q_count = 1;
+  a.vc_seq_slots = seq_slots;
+  a.vc_cap = vc->cap_dev;
+  a.vc_slot_tokens = vc->slot_tokens;
+  a.vc_num_slots = vc->num_slots;
+  const uint64_t tokens = uint64_t(vc->num_slots) * uint64_t(vc->slot_tokens);
+  const void* kb = reinterpret_cast<const void*>(vc->k_base);
+  const void* vb = reinterpret_cast<const void*>(vc->v_base);
+  CUtensorMap km, vm;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int rc;
+  if (tensor_cores) {
+    rc = make_map_vcache(&km, kb, dtype, tokens, uint32_t(Hkv), kvp::dev::tc::kTileTok, 1);
+    if (!rc) rc = make_map_vcache(&vm, vb, dtype, tokens, uint32_t(Hkv), kvp::dev::tc::kTileTok, 2);
+    CUtensorMap qm;
+    if (!rc) rc = make_map(&qm, q, dtype, uint64_t(num_seqs) * num_q_heads, D, kvp::dev::tc::kN);
+    if (rc) return rc;
+    constexpr int M = kvp::dev::tc::kContig, TT = kvp::dev::tc::kTileTok;
+    using H = __half;
+    using B = __nv_bfloat16;
+    const bool f16 = dtype == KVP_F16;
+    if (G <= 4)
+      rc = f16 ? launch_tc<H, TT, 4, M>(km, vm, qm, a, st) : launch_tc<B, TT, 4, M>(km, vm, qm, a, st);
+    else if (G <= 8)
+      rc = f16 ? launch_tc<H, TT, 8, M>(km, vm, qm, a, st) : launch_tc<B, TT, 8, M>(km, vm, qm, a, st);
+    else
+      rc = f16 ? launch_tc<H, TT, 16, M>(km, vm, qm, a, st) : launch_tc<B, TT, 16, M>(km, vm, qm, a, st);
+  } else {
+    rc = make_map_vcache(&km, kb, dtype, tokens, uint32_t(Hkv), kSimtTile, 2);
+    if (!rc) rc = make_map_vcache(&vm, vb, dtype, tokens, uint32_t(Hkv), kSimtTile, 2);
+    if (rc) return rc;
+    constexpr int W = KVP_SIMT_WARPS, N = KVP_SIMT_STAGES;
+    rc = dtype == KVP_F16
+             ? launch_simt<__half, 128, kSimtTile, W, N, false, false, true>(km, vm, a, st)
+             : launch_simt<__nv_bfloat16, 128, kSimtTile, W, N, false, false, true>(km, vm, a, st);
+  }
+  if (rc || pmax <= 1) return rc;
+  return dtype == KVP_F16 ? launch_reduce<__half, 128>(a, st) : launch_reduce<__nv_bfloat16, 128>(a, st);
+}
+
+size_t kvp_decode_packed_workspace_bytes(const int32_t* host_plan, int32_t num_seqs,
+                                         int32_t num_q_heads, int32_t head_dim) {
+  if (!host_plan || num_seqs <= 0 || num_q_heads <= 0 || head_dim <= 0) return 0;
+  const int64_t slots = std::max<int32_t>(1, host_plan[kvp::pack::kMaxChunks]);
+  return pack_ws_layout(num_seqs, num_q_heads, head_dim, slots, pack_plan_used_words(host_plan)).total;
+}
+
+int paged_attention_decode_packed(const void* q, const void* k_cache, const void* v_cache,
+                                  const int32_t* context_lens, int32_t num_seqs,
+                                  int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                  int32_t block_size, int32_t num_blocks, int32_t max_context_len,
+                                  float scale, const int32_t* host_plan, const int32_t* device_plan,
+                                  void* workspace, size_t workspace_bytes, void* out,
+                                  int32_t dtype, kvp_stream_t stream) {
+  const char* fn = "paged_attention_decode_packed";
+  if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_blocks <= 0 || max_context_len < 0)
+    return fail(KVP_ERR_INVALID, "%s: bad sizes", fn);
+  if (num_q_heads % num_kv_heads) return fail(KVP_ERR_INVALID, "%s: num_q_heads %% num_kv_heads != 0", fn);
+  const int G = num_q_heads / num_kv_heads;
+  if (head_dim != 128 || (block_size != 16 && block_size != 32) || G > 16)
+    return fail(KVP_ERR_INVALID, "%s: needs head_dim 128, block_size 16 or 32, at most 16 query heads per KV head", fn);
+  if (dtype != KVP_F16 && dtype != KVP_BF16) return fail(KVP_ERR_INVALID, "%s: bad dtype", fn);
+  if (num_seqs > kvp::grp::kMaxSeqs) return fail(KVP_ERR_INVALID, "%s: more than %d sequences", fn, kvp::grp::kMaxSeqs);
+  if (int64_t(num_blocks) * num_kv_heads * block_size >= (int64_t(1) << 31))
+    return fail(KVP_ERR_INVALID, "%s: pool too large for 32-bit row coordinates", fn);
+  if (!std::isfinite(scale)) return fail(KVP_ERR_INVALID, "%s: scale not finite", fn);
+  if (num_seqs == 0) return KVP_OK;
+  if (!q || !k_cache || !v_cache || !context_lens || !out || !host_plan || !workspace)
+    return fail(KVP_ERR_INVALID, "%s: NULL pointer", fn);
+  if (!aligned(q, 16) || !aligned(out, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
+      !aligned(context_lens, 4) || !aligned(workspace, 256) || (device_plan && !aligned(device_plan, 4)))
+    return fail(KVP_ERR_INVALID, "%s: misaligned pointer", fn);
+  const int mmax = kvp::grp::members_per_subgroup(G);
+  if (!pack_plan_fits(host_plan, num_seqs, block_size, G, mmax))
+    return fail(KVP_ERR_INVALID, "%s: host_plan does not fit this batch", fn);
+  const int64_t plan_words = pack_plan_used_words(host_plan);
+  const int32_t slots = std::max<int32_t>(1, host_plan[kvp::pack::kMaxChunks]);
+  const PackWorkspace wl = pack_ws_layout(num_seqs, num_q_heads, head_dim, slots, plan_words);
+  if (workspace_bytes < wl.total)
+    return fail(KVP_ERR_INVALID, "%s: workspace of %zu bytes needed", fn, wl.total);
+  char* ws = static_cast<char*>(workspace);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int32_t* plan = device_plan ? const_cast<int32_t*>(device_plan)
+                              : reinterpret_cast<int32_t*>(ws + wl.ml_bytes + wl.acc_bytes);
+  if (!device_plan) {
+    cudaError_t e = cudaMemcpyAsync(plan, host_plan, size_t(plan_words) * 4, cudaMemcpyHostToDevice, st);
+    if (e != cudaSuccess) return cuda_fail(e, "packed decode: plan copy");
+  }
+  kvp::dev::DecodeArgs a{};
+  a.q = q;
+  a.out = out;
+  a.block_tables = nullptr;
+  a.context_lens = context_lens;
+  a.ws_ml = reinterpret_cast<float*>(ws);
+  a.ws_acc = reinterpret_cast<float*>(ws + wl.ml_bytes);
+  a.num_seqs = num_seqs;
+  a.num_q_heads = num_q_heads;
+  a.num_kv_heads = num_kv_heads;
+  a.num_blocks = num_blocks;
+  a.max_blocks_per_seq = 1;
+  a.max_context_len = max_context_len;
+  a.part_tokens = 512;
+  a.part_blocks = 512 / block_size;
+  a.pmax = 1;
+  a.ws_slots = slots;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.q_len = 1;
+  a.q_first = 0;
+  a.q_count = 1;
+  a.plan = plan;
+  a.plan_packed = 1;
+  const uint64_t rows = uint64_t(num_blocks) * num_kv_heads * block_size;
+  CUtensorMap km, vm, qm;
+  int rc = make_map(&km, k_cache, dtype, rows, head_dim, block_size);
+  if (!rc) rc = make_map_halves(&vm, v_cache, dtype, rows, block_size);
+  if (!rc) rc = make_map(&qm, q, dtype, uint64_t(num_seqs) * num_q_heads, head_dim, kvp::dev::tc::kN);
+  if (rc) return rc;
+  const int64_t units = int64_t(host_plan[kvp::pack::kUnits]) * num_kv_heads;
+  if (units > 0) {
+    const int ng = kvp::grp::plan_columns(G);
+    const bool f16 = dtype == KVP_F16;
+    using H = __half;
+    using B = __nv_bfloat16;
+    if (block_size == 16)
+      rc = ng == 8 ? (f16 ? launch_tc_packed<H, 16, 8>(km, vm, qm, a, units, st)
+                          : launch_tc_packed<B, 16, 8>(km, vm, qm, a, units, st))
+                   : (f16 ? launch_tc_packed<H, 16, 16>(km, vm, qm, a, units, st)
+                          : launch_tc_packed<B, 16, 16>(km, vm, qm, a, units, st));
+    else
+      rc = ng == 8 ? (f16 ? launch_tc_packed<H, 32, 8>(km, vm, qm, a, units, st)
+                          : launch_tc_packed<B, 32, 8>(km, vm, qm, a, units, st))
+                   : (f16 ? launch_tc_packed<H, 32, 16>(km, vm, qm, a, units, st)
+                          : launch_tc_packed<B, 32, 16>(km, vm, qm, a, units, st));
+    if (rc) return rc;
+  }
+  // the log-sum-exp merge of every row (a sequence of no tokens gets zeros)
+  return dtype == KVP_F16 ? launch_reduce<__half, 128>(a, st) : launch_reduce<__nv_bfloat16, 128>(a, st);
+}
+
 }  // extern "C"
+
+int kvp_vcache_push_cap(int32_t* cap_dev, int32_t slot, int32_t value, void* stream) {
+  kvp::dev::vcache_set_cap_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(cap_dev, slot, value);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? KVP_OK : cuda_fail(e, "kv_vcache: capacity update");
+}
 
 // One thread waits, with the decode kernels' bounded wait, for a phase of an
 // mbarrier that nothing arrives on: the wait runs out and records a status.

@@ -24,7 +24,8 @@ from workloads.values import K_STREAM, Q_STREAM, V_STREAM, normal_bits, value_se
 
 import time
 
-from . import BlockPool, copy_blocks, group_plan, paged_attention_decode, reshape_and_cache
+from . import (BlockPool, copy_blocks, group_plan, pack_plan, paged_attention_decode,
+               paged_attention_decode_packed, reshape_and_cache)
 
 
 def bits_to_tensor(bits: np.ndarray, dtype: str, device):
@@ -38,7 +39,7 @@ def bits_to_tensor(bits: np.ndarray, dtype: str, device):
 class DeviceReplay:
     def __init__(self, wl, device="cuda", keep_outputs: bool = True, time_decode: bool = False,
                  grouped: bool = False, time_reps: int = 1, plan_on: str = "host",
-                 device_values: bool = False):
+                 device_values: bool = False, packed: bool = False):
         import torch
 
         g = wl.geometry
@@ -64,6 +65,7 @@ class DeviceReplay:
         self.decode_events = []    # (op_index, start event, end event) around each decode call
         self.next_index = 0
         self.device_values = device_values
+        self.packed = packed       # decode through paged_attention_decode_packed (host plan)
 
     def _device_normal(self, stream: int, op_index: int, shape):
         import torch
@@ -167,6 +169,16 @@ class DeviceReplay:
                                                   self.wl.scale, max_context_len=mcl,
                                                   partition_size=part, grouped=grouped,
                                                   host_plan=plan, device_plan=dplan)
+            if kw.get("packed", self.packed) and len(lens):
+                t0 = time.perf_counter()
+                pplan = pack_plan(tables, lens, block_size=bs, num_q_heads=self.g.num_q_heads,
+                                  num_kv_heads=self.g.num_kv_heads, num_blocks=self.wl.num_blocks,
+                                  max_context_len=max(mcl, 1))
+                self.plan_us.append((time.perf_counter() - t0) * 1e6)
+                dpp = torch.from_numpy(pplan).to(self.device)  # uploaded with the tables
+                call = lambda: paged_attention_decode_packed(  # noqa: E731
+                    q, self.k_cache, self.v_cache, cl, self.wl.scale, pplan,
+                    max_context_len=max(mcl, 1), device_plan=dpp)
             if self.time_decode:
                 # an untimed call, then before each timed call an L2 flush: a
                 # 256 MB write, then a 256 MB read of another buffer, which writes

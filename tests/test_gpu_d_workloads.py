@@ -61,11 +61,11 @@ def fingerprint_device(cache, chunk=256) -> np.ndarray:
 class Lockstep:
     """Device and oracle replays advanced one step (ops up to a sync) at a time."""
 
-    def __init__(self, wl, grouped=False, check_rows=lambda step: True):
+    def __init__(self, wl, grouped=False, check_rows=lambda step: True, packed=False):
         from paged_kv_cache_319_b200.replay import DeviceReplay
 
         self.wl = wl
-        self.dev = DeviceReplay(wl, "cuda", grouped=grouped)
+        self.dev = DeviceReplay(wl, "cuda", grouped=grouped, packed=packed)
         self.ora = OracleReplay(wl)
         self._values = {}
         draw = self.ora.kv_values  # the seeded draw of op j, before it is shared
@@ -124,9 +124,9 @@ class Lockstep:
         self.steps += 1
 
 
-def replay_pair(wl, grouped=False):
-    """Simple (non-lockstep) replay of both sides, every attend compared in full."""
-    ls = Lockstep(wl, grouped=grouped)
+def replay_pair(wl, grouped=False, packed=False):
+    """Both sides replayed in lockstep, every attend compared in full."""
+    ls = Lockstep(wl, grouped=grouped, packed=packed)
     ls.run()
     return ls.dev, ls.ora, ls.refs
 
@@ -170,11 +170,12 @@ def test_small_workloads_every_output(name, kw):
         check_close(to_bits(dev.outputs[i]), ref, wl.geometry.dtype)
 
 
-@pytest.mark.parametrize("name", ["sharing_B", "beam"])
-def test_shared_workloads_grouped_every_output(name):
-    # the bench decodes these through the grouped entry point
+@pytest.mark.parametrize("decode", ["grouped", "packed"])
+@pytest.mark.parametrize("name", ["sharing_A", "sharing_B", "beam"])
+def test_shared_workloads_grouped_every_output(name, decode):
+    # forked sequences through the entry points that read shared blocks once per group
     wl = workloads.by_name(name)
-    dev, ora, refs = replay_pair(wl, grouped=True)
+    dev, ora, refs = replay_pair(wl, grouped=decode == "grouped", packed=decode == "packed")
     bookkeeping_equal(dev, ora)
     pools_equal(dev, ora)
     assert refs

@@ -172,6 +172,59 @@ def test_device_plan_equals_host_plan(name, Hq, Hkv, bs, dtype, partition, group
     assert np.array_equal(dev[mask], ref[mask])
 
 
+def run_packed(q, k, v, tables, lens, dtype, scale, Hq, Hkv, bs, upload=False):
+    import torch
+    import paged_kv_cache_319_b200 as kvp
+
+    plan = kvp.pack_plan(tables, lens, block_size=bs, num_q_heads=Hq, num_kv_heads=Hkv,
+                         num_blocks=k.shape[0], max_context_len=int(max(lens.max(), 1)))
+    dplan = torch.from_numpy(plan).cuda() if upload else None
+    out = kvp.paged_attention_decode_packed(
+        from_bits(q, dtype), from_bits(k, dtype), from_bits(v, dtype),
+        torch.from_numpy(lens).cuda(), scale, plan, max_context_len=int(max(lens.max(), 1)),
+        device_plan=dplan)
+    kvp.check_device_error()
+    return to_bits(out)
+
+
+# the packed decode takes 128-dim heads, blocks of 16 or 32, up to 16 query heads per KV head
+PACKED_CASES = [c for c in CASES if c[0] not in ("unsplit_fallback",)]
+
+
+@pytest.mark.parametrize("upload", [False, True])
+@pytest.mark.parametrize("name,Hq,Hkv,bs,dtype,partition,groups", PACKED_CASES,
+                         ids=[c[0] for c in PACKED_CASES])
+def test_packed_matches_oracle(name, Hq, Hkv, bs, dtype, partition, groups, upload):
+    seed = sum(map(ord, name)) + 7
+    q, k, v, t, l = shared_batch(seed, groups, Hq, Hkv, 128, bs, dtype)
+    scale = 1 / math.sqrt(128)
+    got = run_packed(q, k, v, t, l, dtype, scale, Hq, Hkv, bs, upload=upload)
+    ref = oracle(q, k, v, t, l, dtype, scale, bs)
+    check_close(got, ref, dtype, allow_ulp=(dtype == "bf16"))
+
+
+def test_packed_rejects_a_plan_of_another_shape():
+    import torch
+    import paged_kv_cache_319_b200 as kvp
+
+    q, k, v, t, l = shared_batch(3, [(31, [600, 700, 520]), (0, [40])], 8, 8, 128, 16, "f16")
+    plan = kvp.pack_plan(t, l, block_size=16, num_q_heads=8, num_kv_heads=8, num_blocks=k.shape[0])
+    args = (from_bits(q, "f16"), from_bits(k, "f16"), from_bits(v, "f16"),
+            torch.from_numpy(l).cuda(), 0.09)
+    bad = plan.copy()
+    bad[int(plan[6]) + 2] += 1                         # a unit with one entry too many
+    with pytest.raises(kvp.KvpError):
+        kvp.paged_attention_decode_packed(*args, bad)
+    bad = plan.copy()
+    bad[8] = (bad[8] + 1) % int(plan[0])               # a sequence's group word
+    with pytest.raises(kvp.KvpError):
+        kvp.paged_attention_decode_packed(*args, bad)
+    bad = plan.copy()
+    bad[int(plan[7]) + 1] |= 1 << 30                   # an entry's columns past its group
+    with pytest.raises(kvp.KvpError):
+        kvp.paged_attention_decode_packed(*args, bad)
+
+
 def test_head_dim_64_is_handed_on():
     q, k, v, t, l = shared_batch(5, [(6, [100, 130, 140]), (0, [20])], 4, 4, 64, 16, "f16")
     got = run(q, k, v, t, l, "f16", 0.125, 512, grouped=True)

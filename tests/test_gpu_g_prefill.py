@@ -5,7 +5,10 @@ into several launches (a whole prompt), sequences holding fewer tokens than
 the chunk (their first queries see nothing), a whole prompt (ctx == T),
 grouped-query heads (G = 4 and 16), block sizes 16 and 32, split and unsplit
 partitions, launches that stop at the last token their queries see, and T = 1
-(the decode path).
+(the decode path). Chunks of at least 64 query rows (T x G, G a power of two)
+run on the prompt-shaped kernel (128 query rows per tensor-core tile): whole
+512-token prompts, grouped heads filling the rows (G = 2, 8, 16), a query
+tile cut short, long contexts split or not, and rows that see nothing.
 """
 
 import math
@@ -48,6 +51,15 @@ CASES = [
     # the launches' ranges
     (4, 4, 16, [150, 300, 700], 200, "f16", 128),
     (16, 4, 32, [90, 520, 1000], 24, "bf16", 128),       # G = 4: 6 launches of 4 queries
+    # prompt-shaped chunks (T x G >= 64 rows): 128 query rows per tensor-core tile
+    (8, 8, 16, [512, 512, 512], 512, "f16", 512),        # whole 512-token prompts, 4 tiles each
+    (8, 8, 16, [512, 512, 512], 512, "bf16", 512),
+    (64, 8, 16, [16, 200, 1000], 16, "bf16", 256),       # G = 8: 16 tokens x 8 heads
+    (32, 2, 32, [8, 50, 700], 8, "f16", 0),              # G = 16: 8 tokens x 16 heads, unsplit
+    (8, 8, 32, [130, 1000, 2500], 130, "bf16", 512),     # a tile of 128 and one of 2 tokens
+    (16, 8, 16, [64, 1500, 3000], 64, "f16", 0),         # G = 2, long contexts unsplit
+    (8, 8, 16, [40, 300], 100, "f16", 128),              # ctx 40 < T: 60 rows see nothing
+    (4, 4, 16, [1, 129, 1000], 300, "bf16", 128),        # ctx 1 < T; partitions cut the tiles
 ]
 
 

@@ -99,3 +99,23 @@ def test_prefix_cache_calls_refuse_bad_arguments(lib):
         assert lib.kv_pool_prefix_stats(pool, C.byref(r), C.byref(e), C.byref(h)) == _lib.KVP_OK
     finally:
         lib.kv_pool_destroy(pool)
+
+
+@pytest.mark.parametrize("bad", [dict(n=0), dict(mt=0), dict(hkv=0), dict(d=64), dict(dt=FP8),
+                                 dict(out=None)])
+def test_vcache_create_refuses(lib, bad):
+    a = dict(n=4, mt=1024, hkv=8, d=128, dt=F16, out=C.byref(C.c_void_p()))
+    a.update(bad)
+    assert lib.kv_vcache_create(a["n"], a["mt"], a["hkv"], a["d"], a["dt"], a["out"]) == INVALID
+
+
+def test_vcache_calls_refuse_a_null_cache(lib):
+    n = C.c_int32()
+    assert lib.kv_vcache_reserve(None, 0, 1, None) == INVALID
+    assert lib.kv_vcache_trim(None, 0, 0, None) == INVALID
+    assert lib.kv_vcache_capacity(None, 0, C.byref(n)) == INVALID
+    assert lib.kv_vcache_release_spares(None) == INVALID
+    assert lib.kv_vcache_destroy(None) == _lib.KVP_OK
+    assert lib.reshape_and_cache_vcache(FAKE, FAKE, None, FAKE, FAKE, 4, None) == INVALID
+    assert lib.attention_decode_vcache(FAKE, None, FAKE, FAKE, 2, 8, 16, 0.1, 0, None, 0, FAKE,
+                                       None) == INVALID

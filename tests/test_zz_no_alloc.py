@@ -8,7 +8,8 @@ caller-given workspace. These tests call that entry point through the C ABI
 and check, on two calls in a row (the second with different inputs, so stale
 scratch from the first would show), that its output matches the output of the
 workspace-taking entry point within the parity tolerance of the other tests,
-and that both match the fp64 oracle within that tolerance. Batches whose
+and that both match the fp64 oracle within that tolerance (for bf16, plus
+half a bf16 ulp of the reference, as the other short-context bf16 tests). Batches whose
 contexts fit one partition (or that do not split at all) need no scratch;
 they are checked the same way. This file is collected last on purpose.
 """
@@ -20,7 +21,7 @@ import pytest
 
 from oracle import attention
 from oracle.numerics import to_f64
-from parity import ATOL, RTOL_NORM, from_bits, random_paged_batch, to_bits
+from parity import ATOL, RTOL_NORM, check_close, from_bits, random_paged_batch, to_bits
 
 pytestmark = pytest.mark.gpu
 
@@ -84,7 +85,9 @@ def _run_both(lib, _lib, case, seed, part, expect_scratch):
     b = to_f64(to_bits(ref), dtype)
     _close(a, b)
     want = attention.paged_decode(to_f64(qb, dtype), kb, vb, tb, lb, SCALE, bs, dtype=dtype)
-    _close(a, want)
+    # short bf16 contexts give outputs near 1, which bf16 holds only to half an
+    # ulp: the parity tests' rule for them allows that on top of 2e-3
+    check_close(to_bits(got), want, dtype, allow_ulp=dtype == "bf16")
 
 
 def test_noalloc_matches_the_workspace_entry_on_two_calls_in_a_row():
