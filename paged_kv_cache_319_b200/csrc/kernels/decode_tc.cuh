@@ -242,10 +242,12 @@ struct GroupHdr {
   bool in_smem;         // cblk and subs point at the CTA's shared-memory copy
   const int32_t* units; // packed decode: the unit table
   const int32_t* ents;  // packed decode: the entries
+  bool ldg;             // global plan words read through the read-only path (packed decode:
+                        // the plan was written before the launch)
 };
 
 __device__ __forceinline__ int32_t plan_at(const GroupHdr& gh, const int32_t* p) {
-  return gh.in_smem ? *p : ld_relaxed_gpu(p);
+  return gh.in_smem ? *p : (gh.ldg ? __ldg(p) : ld_relaxed_gpu(p));
 }
 __device__ __forceinline__ const int32_t* sub_entry(const GroupHdr& gh, int32_t sg) {
   return gh.subs + int64_t(sg) * grp::kSubWords;
@@ -307,7 +309,7 @@ __device__ __forceinline__ bool decode_unit_pack(const DecodeArgs& a, int64_t u,
   w.tok_begin = 0;
   w.tok_end = n * BS;
   w.ctx = n * BS;
-  w.s = __ldg(gh.subs + int64_t(w.sg) * pack::kGroupWords + 4);
+  w.s = plan_at(gh, gh.subs + int64_t(w.sg) * pack::kGroupWords + 4);
   w.nparts = 0;
   w.vbase = 0;
   return n > 0;
@@ -507,9 +509,20 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
   }
 
   if constexpr (PK) {  // the packed plan: uploaded before the launch, read-only here
-    gh.subs = a.plan + pack::group_offset(a.num_seqs);
+    const int32_t* g_subs = a.plan + pack::group_offset(a.num_seqs);
     gh.units = a.plan + __ldg(a.plan + pack::kUnitOffset);
     gh.ents = a.plan + __ldg(a.plan + pack::kEntryOffset);
+    gh.ldg = true;
+    if (a.plan_packed == 2) {  // the launch made room for the group table after the lengths
+      int32_t* s_sm = ctx_cache + (ctx_sm ? a.num_seqs : 0);
+      const int32_t n = __ldg(a.plan + pack::kGroups) * pack::kGroupWords;
+      for (int i = threadIdx.x; i < n; i += blockDim.x) s_sm[i] = __ldg(g_subs + i);
+      __syncthreads();
+      gh.subs = s_sm;
+      gh.in_smem = true;
+    } else {
+      gh.subs = g_subs;
+    }
   }
 
   if (warp == 0) {
@@ -625,10 +638,16 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
       // and used one iteration later
       tc::ChunkStream<MODE, BS> nxt = cur;
       nxt.advance(a);
-      const int32_t id_next = nxt.valid ? chunk_id(nxt) : -1;
+      // (packed decode: the next unit's block ids and Q rows hang on its unit
+      // record, a global load, so they are loaded after this chunk's tiles are
+      // issued)
+      int32_t id_next = -1;
       uint4 qn[kQChunksPerLane];
       const bool gather_next = is_gather(nxt);
-      if (gather_next) gather_q(nxt, qn);
+      if constexpr (!PK) {
+        id_next = nxt.valid ? chunk_id(nxt) : -1;
+        if (gather_next) gather_q(nxt, qn);
+      }
       const int32_t row = id_row(cur, id);
       const int32_t nt = cur.tiles();
       // A unit's Q goes in before its key tiles (gathered rows were loaded an
@@ -661,6 +680,10 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
       }
       if (ok) load_tiles(&kmap, row, cur.w.g, nt, false);
       if (have_pend && ok) load_tiles(&vmap, pend_row, pend_head, pend_tiles, true);
+      if constexpr (PK) {
+        id_next = nxt.valid ? chunk_id(nxt) : -1;
+        if (gather_next) gather_q(nxt, qn);
+      }
       pend_row = row;
       pend_head = cur.w.g;
       pend_tiles = nt;
@@ -785,13 +808,23 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
     uint32_t pend_b = 0, pend_use = 0;
     int32_t pend_tiles = 0, pend_zero = kTileTok, pend_nv = BS;
     bool have_pend = false;
+    int32_t nv_cur = BS;  // packed decode: valid tokens of this lane's block of the chunk
+    if constexpr (PK) {
+      if (cur.valid && lane < (cur.w.ctx + BS - 1) / BS)
+        nv_cur = __ldg(gh.ents + 2 * (int64_t(cur.w.e0) + lane) + 1) & 0xFF;
+    }
     while (cur.valid && ok) {
       const uint32_t b = cc & 1u, use = cc >> 1;
       const int32_t nt = cur.tiles();
-      int32_t nv_cur = BS;  // packed decode: valid tokens of this lane's block of the chunk
+      // packed decode: the next unit is decoded now (its plan loads overlap this
+      // chunk), and nv_cur, this lane's block's valid tokens, was loaded a unit ago
+      tc::ChunkStream<MODE, BS> nxt;
+      int32_t nv_next = BS;
       if constexpr (PK) {
-        if (lane < (cur.w.ctx + BS - 1) / BS)
-          nv_cur = __ldg(gh.ents + 2 * (int64_t(cur.w.e0) + lane) + 1) & 0xFF;
+        nxt = cur;
+        nxt.advance(a);
+        if (nxt.valid && lane < (nxt.w.ctx + BS - 1) / BS)
+          nv_next = __ldg(gh.ents + 2 * (int64_t(nxt.w.e0) + lane) + 1) & 0xFF;
       }
       if (lane == 0) {
         if (cur.first()) {
@@ -816,7 +849,12 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
       pend_tiles = nt;
       have_pend = true;
       ++cc;
-      cur.advance(a);
+      if constexpr (PK) {
+        cur = nxt;
+        nv_cur = nv_next;
+      } else {
+        cur.advance(a);
+      }
     }
     if (ok && have_pend) pv(pend_b, pend_use, pend_tiles, pend_zero, pend_nv);
     if (!ok) atomicExch(&abort_flag, 1);
@@ -933,28 +971,38 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
       }
     };
 
+    // packed decode: per tile of a unit, the columns that take this thread's
+    // token row (its block's column mask, none past the block's valid tokens)
+    auto row_masks = [&](const tc::ChunkStream<MODE, BS>& cs, uint32_t (&m)[kChunkTiles]) {
+      const int32_t nblk = cs.valid ? (cs.w.ctx + BS - 1) / BS : 0;
+#pragma unroll
+      for (int t = 0; t < kChunkTiles; ++t) {
+        const int32_t blk = t * kBlocksPerTile + r / BS;
+        m[t] = 0;
+        if (blk < nblk) {
+          const uint32_t wd = uint32_t(__ldg(gh.ents + 2 * (int64_t(cs.w.e0) + blk) + 1));
+          m[t] = (r % BS) < int32_t(wd & 0xFFu) ? (wd >> 8) : 0u;
+        }
+      }
+    };
     tc::ChunkStream<MODE, BS> cur;
     cur.init(a, blockIdx.x, gridDim.x, num_units, ctx_sm, gh);
+    uint32_t pm[kChunkTiles];
+#pragma unroll
+    for (int t = 0; t < kChunkTiles; ++t) pm[t] = 0xFFFFFFFFu;
+    if constexpr (PK) row_masks(cur, pm);
     while (cur.valid && ok) {
       const uint32_t b = cc & 1u;
       const uint32_t use = cc >> 1;
       const int32_t ntile = cur.tiles();
-      // packed decode: per tile, the columns that take this thread's token row
-      // (its block's column mask, none past the block's valid tokens)
-      uint32_t pm[kChunkTiles];
-#pragma unroll
-      for (int t = 0; t < kChunkTiles; ++t) pm[t] = 0xFFFFFFFFu;
+      // packed decode: the next unit is decoded now and its row masks loaded (the
+      // loads overlap this chunk); pm holds this unit's, loaded a unit ago
+      tc::ChunkStream<MODE, BS> nxt;
+      uint32_t pm_next[kChunkTiles];
       if constexpr (PK) {
-        const int32_t nblk = (cur.w.ctx + BS - 1) / BS;
-#pragma unroll
-        for (int t = 0; t < kChunkTiles; ++t) {
-          const int32_t blk = t * kBlocksPerTile + r / BS;
-          pm[t] = 0;
-          if (blk < nblk) {
-            const uint32_t wd = uint32_t(__ldg(gh.ents + 2 * (int64_t(cur.w.e0) + blk) + 1));
-            pm[t] = (r % BS) < int32_t(wd & 0xFFu) ? (wd >> 8) : 0u;
-          }
-        }
+        nxt = cur;
+        nxt.advance(a);
+        row_masks(nxt, pm_next);
       }
       const int32_t ctok0 = cur.w.tok_begin + cur.c * kChunkTok;
       const int32_t ctok1 = min(cur.w.tok_end, ctok0 + kChunkTok);
@@ -1068,7 +1116,13 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
       }
       have_pend = true;
       ++cc;
-      cur.advance(a);
+      if constexpr (PK) {
+        cur = nxt;
+#pragma unroll
+        for (int t = 0; t < kChunkTiles; ++t) pm[t] = pm_next[t];
+      } else {
+        cur.advance(a);
+      }
     }
     if (ok && have_pend) merge();
     if (!ok) atomicExch(&abort_flag, 1);

@@ -15,8 +15,10 @@
 //   S [128 rows x 128 keys]  = Q [128 x 128 dims] . K^T            (TMEM)
 //   O [128 rows x 128 dims] += P [128 x 128 keys] . V [128 x 128]  (TMEM)
 //
-// with P held as a high and a low part in the input type (the product V.(hi
-// + lo) carries p to about 16 significant bits, as the decode kernel does).
+// with P held, for bf16 inputs, as a high and a low part (the product V.(hi +
+// lo) carries p to about 16 significant bits, as the decode kernel does); for
+// fp16 inputs one part of 11 significant bits suffices (on causal 512-token
+// prompts of N(0, 1) data the output moves by at most 3.8e-4 against exact p).
 //
 // Warp roles (192 threads, one CTA per SM, persistent over units):
 //   warp 0     producer: TMA loads of Q (a 3-D box {64 dims, G heads, 128 / G
@@ -26,12 +28,14 @@
 //              PV of tile n; S is double-buffered, O double-buffered by unit.
 //   warps 2-5  softmax and epilogue, thread = TMEM lane = row: per tile a
 //              masked row max (causal: key j visible to the row's position),
-//              p = 2^(s - m) into the shared P buffer, and at a unit's end the
+//              p = 2^(s - m) into shared memory, and at a unit's end the
 //              normalised row (or its partial for the split-context reduce).
+//              fp16 inputs: P is double-buffered (the softmax of tile n + 1
+//              runs while PV of tile n does); bf16: one buffer of hi + lo.
 // The running maximum m of a row moves only when a tile's maximum exceeds it
-// by more than 8 (log2 units); O and l are then rescaled in TMEM (after the
-// previous PV has completed, which the single P buffer waits for anyway), so
-// p <= 2^8 and (m, l, O) stay a consistent partial.
+// by more than 8 (log2 units); O and l are then rescaled in TMEM, once the
+// previous PV has completed, so p <= 2^8 and (m, l, O) stay a consistent
+// partial.
 #pragma once
 
 #include <type_traits>
@@ -64,7 +68,7 @@ constexpr int kOffRing = kOffQ + 2 * kTileBytes;        // kStages K/V stages
 constexpr int kOffPHi = kOffRing + kStages * kTileBytes;
 constexpr int kOffPLo = kOffPHi + kTileBytes;
 constexpr int kOffBar = kOffPLo + kTileBytes;
-constexpr int kNumBars = 2 * kStages + 2 * 6 + 2;
+constexpr int kNumBars = 2 * kStages + 2 * 7;
 constexpr int kOffTmemPtr = kOffBar + kNumBars * 8;
 constexpr int kSmemBytes = 1024 + kOffTmemPtr + 16;
 static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
@@ -168,6 +172,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_tc_kernel(
   static_assert(BS == 16 || BS == 32, "block_size 16 or 32");
   constexpr int kBlocksPerTile = kKeys / BS;
   constexpr uint32_t kFmt = std::is_same<T, __half>::value ? 0u : 1u;
+  constexpr bool kLo = !std::is_same<T, __half>::value;  // p's low part (bf16 inputs)
   constexpr uint32_t kIdescQK = tc::idesc_f16(kFmt, 0, 0, kKeys);  // Q, K both K-major
   constexpr uint32_t kIdescPV = tc::idesc_f16(kFmt, 0, 1, kD);     // P K-major, V MN-major
 
@@ -185,9 +190,12 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_tc_kernel(
   uint64_t* s_full = q_empty + 2;        // [2]
   uint64_t* s_free = s_full + 2;         // [2]
   uint64_t* o_free = s_free + 2;         // [2]
-  uint64_t* spare = o_free + 2;          // [2] (unused)
-  uint64_t* p_full = spare + 2;          // [1]
-  uint64_t* p_free = p_full + 1;         // [1]: a PV has completed (one phase per tile)
+  // P buffer b (fp16: tile parity; bf16: always 0): p_full[b] completes when the
+  // softmax has written it, p_free[b] when the PV that read it has completed.
+  // Each barrier is at most one phase ahead of its waiter: a buffer is written
+  // again only after its previous PV has been waited for.
+  uint64_t* p_full = o_free + 2;         // [2]
+  uint64_t* p_free = p_full + 2;         // [2]
   uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + kOffTmemPtr);
   __shared__ int abort_flag;
   const int32_t* ctx_sm = nullptr;  // context lengths are read per unit (L1-resident)
@@ -206,10 +214,9 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_tc_kernel(
       mbar_init(&s_full[i], 1);
       mbar_init(&s_free[i], 4);
       mbar_init(&o_free[i], 4);
-      mbar_init(&spare[i], 1);
+      mbar_init(&p_full[i], 4);
+      mbar_init(&p_free[i], 1);
     }
-    mbar_init(p_full, 4);
-    mbar_init(p_free, 1);
     abort_flag = 0;
     fence_mbar_init();
   }
@@ -277,6 +284,8 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_tc_kernel(
     bool have_pend = false;
     while (cur.valid && ok) {
       const Unit w = cur.w;
+      UnitStream nxt = cur;  // the next unit, decoded now (its loads overlap this one)
+      nxt.next(a);
       // Q of the unit
       const uint32_t qb = ucnt & 1u;
       if (lane == 0) {
@@ -300,7 +309,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_tc_kernel(
         have_pend = true;
         id = id_next;
       }
-      cur.next(a);
+      cur = nxt;
     }
     if (ok && have_pend) load_tile(&vmap, pend_row, true);
     if (!ok) {
@@ -323,8 +332,10 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_tc_kernel(
     // rows of tokens past the context (they hold whatever the pool had there;
     // p is 0 for them, but 0 * inf is NaN).
     auto pv = [&](const Pend& pd, uint32_t tile_n) {
+      const uint32_t pb = kLo ? 0u : (tile_n & 1u);          // P buffer of the tile
+      const uint32_t pphase = kLo ? tile_n : (tile_n >> 1);  // its use count
       if (lane == 0) {
-        ok = mbar_wait(p_full, tile_n & 1u, 0x8700u);
+        ok = mbar_wait(&p_full[pb], pphase & 1u, 0x8700u);
         if (ok && pd.first) ok = mbar_wait(&o_free[pd.ob], ((pd.ucnt >> 1) & 1u) ^ 1u, 0x8800u);
       }
       ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -352,8 +363,10 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_tc_kernel(
         const uint32_t v_addr = smem_u32(tile);
         const uint32_t o_tmem = tmem_base + kOCol + pd.ob * kD;
 #pragma unroll
-        for (int part = 0; part < 2; ++part) {
-          const uint32_t p_addr = smem_u32(part == 0 ? phi : plo);
+        for (int part = 0; part < (kLo ? 2 : 1); ++part) {
+          // bf16: the hi and lo parts; fp16: one part, buffer by tile parity
+          const uint32_t p_addr =
+              smem_u32(kLo ? (part == 0 ? phi : plo) : ((tile_n & 1u) ? plo : phi));
 #pragma unroll
           for (int kk = 0; kk < kKeys / 16; ++kk) {
             const uint32_t pa = p_addr + (kk >> 2) * kRegion + (kk & 3) * 32;
@@ -364,7 +377,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_tc_kernel(
           }
         }
         umma_commit(&empty[st]);
-        umma_commit(p_free);
+        umma_commit(&p_free[pb]);
       }
       __syncwarp();
       ++ctr;
@@ -373,6 +386,8 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_tc_kernel(
     cur.init(a, G, qtiles, num_units, ctx_sm);
     while (cur.valid && ok) {
       const Unit w = cur.w;
+      UnitStream nxt = cur;
+      nxt.next(a);
       const uint32_t qb = ucnt & 1u;
       if (lane == 0) ok = mbar_wait(&q_full[qb], (ucnt >> 1) & 1u, 0x8400u);
       ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -414,7 +429,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_tc_kernel(
         have_pend = true;
       }
       ++ucnt;
-      cur.next(a);
+      cur = nxt;
     }
     if (ok && have_pend) pv(pend, n - 1);
     if (!ok) atomicExch(&abort_flag, 1);
@@ -439,19 +454,25 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_tc_kernel(
         for (int c = 0; c < kD * 2 / 16; ++c) dst[c] = make_uint4(0, 0, 0, 0);
       }
     }
-    uint32_t n = 0, ucnt = 0, pv_seen = 0;
+    uint32_t n = 0, ucnt = 0;
+    uint32_t seen[2] = {0, 0};  // phases of p_free[b] consumed
     bool ok = true;
-    // waits until `count` PV products have completed (their phases in order)
-    auto wait_pv = [&](uint32_t count) {
-      while (ok && pv_seen < count) {
-        ok = wait_all(p_free, pv_seen & 1u, 0x8b00u);
-        ++pv_seen;
+    // waits until the PV of tile k has completed (and with it every earlier
+    // MMA), consuming its buffer's phases in order
+    auto wait_pv = [&](uint32_t k) {
+      const uint32_t b = kLo ? 0u : (k & 1u);
+      const uint32_t ph = kLo ? k : (k >> 1);
+      while (ok && seen[b] <= ph) {
+        ok = wait_all(&p_free[b], seen[b] & 1u, 0x8b00u);
+        ++seen[b];
       }
     };
     UnitStream cur;
     cur.init(a, G, qtiles, num_units, ctx_sm);
     while (cur.valid && ok) {
       const Unit w = cur.w;
+      UnitStream nxt = cur;
+      nxt.next(a);
       const int32_t ti = r / G;  // query token of the row within the tile
       const bool row_live = ti < w.nq;
       const int32_t pos = w.ctx - a.q_len + w.q0 + ti;   // the row sees keys j <= pos
@@ -466,16 +487,31 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_tc_kernel(
         if (!ok) break;
         tc_fence_after();
         const uint32_t s_taddr = tmem_base + lane_addr + kSCol + sb * kKeys;
-        // pass 1: the row's masked maximum over the tile
+        // every row of the warp sees the whole tile (all but the diagonal tiles):
+        // no per-key masks
+        const bool full = __all_sync(0xffffffffu, k0 + kKeys <= lim);
+        // pass 1: the row's largest scaled score over the tile (keys it sees)
         float mx = -INFINITY;
-#pragma unroll
+#pragma unroll 1
         for (int c = 0; c < kKeys / 32; ++c) {
           float sv[32];
           tc::tmem_ld_cols<32>(s_taddr + c * 32, sv);
           tmem_ld_wait();
+          float m0 = -INFINITY, m1 = -INFINITY;
+          if (full) {
 #pragma unroll
-          for (int e = 0; e < 32; ++e)
-            if (k0 + c * 32 + e < lim) mx = fmaxf(mx, sv[e] * a.scale_log2);
+            for (int e = 0; e < 32; e += 2) {
+              m0 = fmaxf(m0, sv[e] * a.scale_log2);
+              m1 = fmaxf(m1, sv[e + 1] * a.scale_log2);
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; e += 2) {
+              if (k0 + c * 32 + e < lim) m0 = fmaxf(m0, sv[e] * a.scale_log2);
+              if (k0 + c * 32 + e + 1 < lim) m1 = fmaxf(m1, sv[e + 1] * a.scale_log2);
+            }
+          }
+          mx = fmaxf(mx, fmaxf(m0, m1));
         }
         // the running maximum moves only by more than kLazy
         float factor = 1.f;
@@ -489,12 +525,15 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_tc_kernel(
             need = true;
           }
         }
-        // the single P buffer is free once the previous tile's PV has completed
-        wait_pv(n);
+        // P's buffer is free once the PV that last read it has completed (one
+        // buffer: the previous tile's; two: the one before)
+        if (kLo ? n >= 1 : n >= 2) wait_pv(kLo ? n - 1 : n - 2);
         if (!ok) break;
         if (__any_sync(0xffffffffu, need) && t > 0) {
+          wait_pv(n - 1);  // O holds every PV of the unit so far
+          if (!ok) break;
           tc_fence_after();
-#pragma unroll
+#pragma unroll 1
           for (int c = 0; c < kD / 32; ++c) {
             float ov[32];
             tc::tmem_ld_cols<32>(o_taddr + c * 32, ov);
@@ -506,34 +545,50 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_tc_kernel(
           tmem_st_wait();
         }
         l *= factor;
-        // pass 2: p = 2^(s - m) as hi + lo parts into P (row r, 128-byte swizzle)
-#pragma unroll
+        // pass 2: p = 2^(s - m) (bf16: as hi + lo parts) into P (row r, 128-byte
+        // swizzle); l sums the rounded p the MMA multiplies
+        const float nm = -m_ref;
+        uint8_t* pdst = kLo ? phi : ((n & 1u) ? plo : phi);
+#pragma unroll 1
         for (int c = 0; c < kKeys / 32; ++c) {
           float sv[32];
           tc::tmem_ld_cols<32>(s_taddr + c * 32, sv);
           tmem_ld_wait();
           uint32_t hw[16], lw[16];
+          float l0 = 0.f, l1 = 0.f;
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
             const int j = k0 + c * 32 + e;
-            const float p0 = j < lim ? tc::ex2_ftz(sv[e] * a.scale_log2 - m_ref) : 0.f;
-            const float p1 = j + 1 < lim ? tc::ex2_ftz(sv[e + 1] * a.scale_log2 - m_ref) : 0.f;
+            float p0 = tc::ex2_ftz(fmaf(sv[e], a.scale_log2, nm));
+            float p1 = tc::ex2_ftz(fmaf(sv[e + 1], a.scale_log2, nm));
+            if (!full) {  // keys the row does not see (select, not multiply: NaN scores)
+              p0 = j < lim ? p0 : 0.f;
+              p1 = j + 1 < lim ? p1 : 0.f;
+            }
             hw[e / 2] = Elem<T>::pack2(p0, p1);
             const float2 hf = Elem<T>::to_float2(hw[e / 2]);
-            lw[e / 2] = Elem<T>::pack2(p0 - hf.x, p1 - hf.y);
-            const float2 lf = Elem<T>::to_float2(lw[e / 2]);
-            l += (hf.x + lf.x) + (hf.y + lf.y);
+            if constexpr (kLo) {
+              lw[e / 2] = Elem<T>::pack2(p0 - hf.x, p1 - hf.y);
+              const float2 lf = Elem<T>::to_float2(lw[e / 2]);
+              l0 += hf.x + lf.x;
+              l1 += hf.y + lf.y;
+            } else {
+              l0 += hf.x;
+              l1 += hf.y;
+            }
           }
+          l += l0 + l1;
           // keys c*32 .. +32 of row r: four 16-byte chunks of region c / 2
           const int region = c >> 1;
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             const int chunk = (c & 1) * 4 + q;  // 16-byte chunk within the 128-byte row
             const uint32_t off = region * kRegion + r * 128 + ((chunk ^ (r & 7)) << 4);
-            *reinterpret_cast<uint4*>(phi + off) =
+            *reinterpret_cast<uint4*>(pdst + off) =
                 make_uint4(hw[4 * q], hw[4 * q + 1], hw[4 * q + 2], hw[4 * q + 3]);
-            *reinterpret_cast<uint4*>(plo + off) =
-                make_uint4(lw[4 * q], lw[4 * q + 1], lw[4 * q + 2], lw[4 * q + 3]);
+            if constexpr (kLo)
+              *reinterpret_cast<uint4*>(plo + off) =
+                  make_uint4(lw[4 * q], lw[4 * q + 1], lw[4 * q + 2], lw[4 * q + 3]);
           }
         }
         tc_fence_before();
@@ -541,16 +596,16 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_tc_kernel(
         __syncwarp();
         if (lane == 0) {
           mbar_arrive(&s_free[sb]);
-          mbar_arrive(p_full);
+          mbar_arrive(&p_full[kLo ? 0u : (n & 1u)]);
         }
         if (t == w.ntiles - 1) {
           // ---- epilogue: O of the unit once its last PV has completed
-          wait_pv(n + 1);
+          wait_pv(n);
           if (!ok) break;
           tc_fence_after();
           const int64_t qrow = (int64_t(w.s) * a.q_len + w.q0 + ti) * a.num_q_heads + w.g * G + r % G;
           const float inv = l > 0.f ? 1.f / l : 0.f;
-#pragma unroll
+#pragma unroll 1
           for (int c = 0; c < kD / 32; ++c) {
             float ov[32];
             tc::tmem_ld_cols<32>(o_taddr + c * 32, ov);
@@ -583,7 +638,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_tc_kernel(
         }
       }
       ++ucnt;
-      cur.next(a);
+      cur = nxt;
     }
     if (!ok) atomicExch(&abort_flag, 1);
   }

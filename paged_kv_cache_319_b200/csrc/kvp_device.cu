@@ -436,14 +436,24 @@ int tc_grouped_dispatch(int bs, int ng, const CUtensorMap& km, const CUtensorMap
 // Packed grouped decode: one persistent tensor-core launch over units x KV heads.
 template <typename T, int BS, int NG>
 int launch_tc_packed(const CUtensorMap& km, const CUtensorMap& vm, const CUtensorMap& qm,
-                     const kvp::dev::DecodeArgs& a, int64_t units, cudaStream_t st) {
+                     const kvp::dev::DecodeArgs& a, int64_t units, int32_t groups, cudaStream_t st) {
   auto k = kvp::dev::decode_tc_kernel<T, BS, NG, kvp::dev::tc::kPacked>;
   using Cfg = kvp::dev::tc::Cfg<NG>;
+  constexpr int kMax = 226 * 1024;
   const int ctx_bytes = a.num_seqs <= Cfg::kCtxCap ? 4 * a.num_seqs : 0;
-  cudaError_t e = ensure_smem(k, Cfg::kSmemBytes + 4 * Cfg::kCtxCap);
+  cudaError_t e = ensure_smem(k, kMax);
   if (e != cudaSuccess) return cuda_fail(e, "packed decode: smem attribute");
+  // the group table in shared memory when it fits (the Q gather and every
+  // unit read it), else read from the plan in global memory
+  kvp::dev::DecodeArgs a2 = a;
+  int smem = Cfg::kSmemBytes + ctx_bytes;
+  const int grp_bytes = groups * kvp::pack::kGroupWords * 4;
+  if (smem + grp_bytes <= kMax) {
+    smem += grp_bytes;
+    a2.plan_packed = 2;
+  }
   const int grid = int(units < sm_count() ? units : sm_count());
-  k<<<grid, kvp::dev::tc::kThreads, Cfg::kSmemBytes + ctx_bytes, st>>>(km, vm, qm, a, units);
+  k<<<grid, kvp::dev::tc::kThreads, smem, st>>>(km, vm, qm, a2, units);
   e = cudaGetLastError();
   return e == cudaSuccess ? KVP_OK : cuda_fail(e, "packed decode: launch");
 }
@@ -1417,21 +1427,22 @@ int paged_attention_decode_packed(const void* q, const void* k_cache, const void
   if (!rc) rc = make_map(&qm, q, dtype, uint64_t(num_seqs) * num_q_heads, head_dim, kvp::dev::tc::kN);
   if (rc) return rc;
   const int64_t units = int64_t(host_plan[kvp::pack::kUnits]) * num_kv_heads;
+  const int32_t ngroups = host_plan[kvp::pack::kGroups];
   if (units > 0) {
     const int ng = kvp::grp::plan_columns(G);
     const bool f16 = dtype == KVP_F16;
     using H = __half;
     using B = __nv_bfloat16;
     if (block_size == 16)
-      rc = ng == 8 ? (f16 ? launch_tc_packed<H, 16, 8>(km, vm, qm, a, units, st)
-                          : launch_tc_packed<B, 16, 8>(km, vm, qm, a, units, st))
-                   : (f16 ? launch_tc_packed<H, 16, 16>(km, vm, qm, a, units, st)
-                          : launch_tc_packed<B, 16, 16>(km, vm, qm, a, units, st));
+      rc = ng == 8 ? (f16 ? launch_tc_packed<H, 16, 8>(km, vm, qm, a, units, ngroups, st)
+                          : launch_tc_packed<B, 16, 8>(km, vm, qm, a, units, ngroups, st))
+                   : (f16 ? launch_tc_packed<H, 16, 16>(km, vm, qm, a, units, ngroups, st)
+                          : launch_tc_packed<B, 16, 16>(km, vm, qm, a, units, ngroups, st));
     else
-      rc = ng == 8 ? (f16 ? launch_tc_packed<H, 32, 8>(km, vm, qm, a, units, st)
-                          : launch_tc_packed<B, 32, 8>(km, vm, qm, a, units, st))
-                   : (f16 ? launch_tc_packed<H, 32, 16>(km, vm, qm, a, units, st)
-                          : launch_tc_packed<B, 32, 16>(km, vm, qm, a, units, st));
+      rc = ng == 8 ? (f16 ? launch_tc_packed<H, 32, 8>(km, vm, qm, a, units, ngroups, st)
+                          : launch_tc_packed<B, 32, 8>(km, vm, qm, a, units, ngroups, st))
+                   : (f16 ? launch_tc_packed<H, 32, 16>(km, vm, qm, a, units, ngroups, st)
+                          : launch_tc_packed<B, 32, 16>(km, vm, qm, a, units, ngroups, st));
     if (rc) return rc;
   }
   // the log-sum-exp merge of every row (a sequence of no tokens gets zeros)
