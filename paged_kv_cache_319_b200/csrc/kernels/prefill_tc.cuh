@@ -82,17 +82,23 @@ struct Unit {
   bool to_ws;                // partial to the workspace (the sequence is split)
 };
 
-// Units are ordered (sequence, KV head, query tile from the last, partition),
-// so the tiles of one (sequence, head) run at about the same time and share
-// their key and value tiles through L2, and the longest (last) query tiles of
-// causal prompts start first.
+// Units are ordered (sequence, KV head, query tile, partition), so the tiles
+// of one (sequence, head) run at about the same time and share their key and
+// value tiles through L2. CTAs take units round-robin; the query tiles of a
+// (sequence, head) are rotated by the round in which its first unit is dealt,
+// so a CTA meets every query tile in turn (a causal prompt's tile qt has qt + 1
+// key tiles; without the rotation a grid that is a multiple of the tile count
+// would hand each CTA one tile index throughout).
 __device__ __forceinline__ void unit_at(const DecodeArgs& a, int64_t u, int32_t G, int32_t qtiles,
                                         const int32_t* ctx_sm, Unit& w) {
   const int32_t tq = kRows / G;
-  w.p = int32_t(u % a.pmax);
-  int64_t rest = u / a.pmax;
-  const int32_t qt = qtiles - 1 - int32_t(rest % qtiles);
-  rest /= qtiles;
+  const int64_t per_head = int64_t(qtiles) * a.pmax;
+  const int64_t head_unit = u / per_head;  // (sequence, KV head)
+  const int32_t within = int32_t(u - head_unit * per_head);
+  const int32_t rot = int32_t(((head_unit * per_head) / gridDim.x) % qtiles);
+  w.p = within % a.pmax;
+  const int32_t qt = qtiles - 1 - (within / a.pmax + rot) % qtiles;
+  int64_t rest = head_unit;
   w.g = int32_t(rest % a.num_kv_heads);
   w.s = int32_t(rest / a.num_kv_heads);
   w.ctx = ctx_sm ? ctx_sm[w.s] : load_ctx(a, w.s, w.g == 0 && qt == 0 && w.p == 0);
@@ -160,14 +166,15 @@ __device__ __forceinline__ void tmem_st_wait() {
 }  // namespace pf
 
 // q map: 3-D {128 dims, num_q_heads, num_seqs * q_len} with a {64, G, 128 / G}
-// box; K map 2-D {128, rows} with a {64, BS} box; V map 3-D halves {64, rows,
+// box, o map the same over the output with a {64, G, 32 / G} box (each softmax
+// warp stores its 32 rows of an unsplit unit through it); K map 2-D {128, rows} with a {64, BS} box; V map 3-D halves {64, rows,
 // 2} with a {64, BS, 2} box (the decode kernel's maps). num_units = num_seqs
 // x num_kv_heads x query tiles x a.pmax.
 template <typename T, int BS>
 __global__ void __launch_bounds__(pf::kThreads, 1) prefill_tc_kernel(
     const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
-    const __grid_constant__ CUtensorMap qmap, const DecodeArgs a, int32_t qtiles,
-    int64_t num_units) {
+    const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap omap,
+    const DecodeArgs a, int32_t qtiles, int64_t num_units) {
   using namespace pf;
   static_assert(BS == 16 || BS == 32, "block_size 16 or 32");
   constexpr int kBlocksPerTile = kKeys / BS;
@@ -237,6 +244,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_tc_kernel(
       prefetch_tensormap(&kmap);
       prefetch_tensormap(&vmap);
       prefetch_tensormap(&qmap);
+      prefetch_tensormap(&omap);
     }
     const uint64_t pol_kv = l2_policy_evict_normal();  // a key tile serves every query tile
     const uint64_t pol_q = l2_policy_evict_first();
@@ -309,9 +317,11 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_tc_kernel(
         have_pend = true;
         id = id_next;
       }
+      // V of the unit's last tile: its PV is issued before the next unit's QK
+      if (ok && have_pend) load_tile(&vmap, pend_row, true);
+      have_pend = false;
       cur = nxt;
     }
-    if (ok && have_pend) load_tile(&vmap, pend_row, true);
     if (!ok) {
       atomicExch(&abort_flag, 1);
       if (lane == 0)
@@ -320,6 +330,8 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_tc_kernel(
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
+    // Order: QK(0), then per tile t > 0 QK(t) and PV(t - 1); a unit's last PV
+    // is issued at once, so its epilogue never waits for the next unit's Q.
     uint32_t ctr = 0, ucnt = 0, n = 0;
     bool ok = true;
     struct Pend {
@@ -428,10 +440,11 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_tc_kernel(
         pend.zero_from = w.ctx - k0;
         have_pend = true;
       }
+      if (ok && have_pend) pv(pend, n - 1);
+      have_pend = false;
       ++ucnt;
       cur = nxt;
     }
-    if (ok && have_pend) pv(pend, n - 1);
     if (!ok) atomicExch(&abort_flag, 1);
   } else {
     // ------------------------------------------------------------ softmax + epilogue
@@ -456,6 +469,8 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_tc_kernel(
     }
     uint32_t n = 0, ucnt = 0;
     uint32_t seen[2] = {0, 0};  // phases of p_free[b] consumed
+    // P buffer that this warp's last output store may still be reading
+    const uint8_t* store_src = nullptr;
     bool ok = true;
     // waits until the PV of tile k has completed (and with it every earlier
     // MMA), consuming its buffer's phases in order
@@ -549,6 +564,11 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_tc_kernel(
         // swizzle); l sums the rounded p the MMA multiplies
         const float nm = -m_ref;
         uint8_t* pdst = kLo ? phi : ((n & 1u) ? plo : phi);
+        if (store_src == pdst) {  // the warp's output rows staged there have been read
+          if (lane == 0) bulk_wait_read();
+          __syncwarp();
+          store_src = nullptr;
+        }
 #pragma unroll 1
         for (int c = 0; c < kKeys / 32; ++c) {
           float sv[32];
@@ -605,6 +625,12 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_tc_kernel(
           tc_fence_after();
           const int64_t qrow = (int64_t(w.s) * a.q_len + w.q0 + ti) * a.num_q_heads + w.g * G + r % G;
           const float inv = l > 0.f ? 1.f / l : 0.f;
+          // an unsplit unit's rows go out through the P buffer of tile n (its PV
+          // has completed) and one TMA store per 64-dim half, when every row of
+          // the warp is a token of the chunk
+          const int32_t tw = 32 / G;  // tokens of the warp's rows
+          const bool staged = !w.to_ws && (quarter + 1) * tw <= w.nq;
+          uint8_t* stage = kLo ? phi : ((n & 1u) ? plo : phi);
 #pragma unroll 1
           for (int c = 0; c < kD / 32; ++c) {
             float ov[32];
@@ -614,6 +640,20 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_tc_kernel(
               tc_fence_before();
               __syncwarp();
               if (lane == 0) mbar_arrive(&o_free[ob]);
+            }
+            if (staged) {
+              // dims c*32 .. +32 of row r: four 16-byte chunks of region c / 2
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                const int chunk = (c & 1) * 4 + q;
+                const uint32_t off = (c >> 1) * kRegion + r * 128 + ((chunk ^ (r & 7)) << 4);
+                *reinterpret_cast<uint4*>(stage + off) =
+                    make_uint4(Elem<T>::pack2(ov[8 * q] * inv, ov[8 * q + 1] * inv),
+                               Elem<T>::pack2(ov[8 * q + 2] * inv, ov[8 * q + 3] * inv),
+                               Elem<T>::pack2(ov[8 * q + 4] * inv, ov[8 * q + 5] * inv),
+                               Elem<T>::pack2(ov[8 * q + 6] * inv, ov[8 * q + 7] * inv));
+              }
+              continue;
             }
             if (!row_live) continue;
             if (!w.to_ws) {
@@ -635,11 +675,24 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_tc_kernel(
             a.ws_ml[(qrow * a.ws_slots + w.p) * 2 + 0] = m_ref;
             a.ws_ml[(qrow * a.ws_slots + w.p) * 2 + 1] = l;
           }
+          if (staged) {
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              const uint8_t* src = stage + quarter * 32 * 128;
+              const int32_t z = w.s * a.q_len + w.q0 + quarter * tw;
+              tma_store_3d(&omap, src, 0, w.g * G, z);
+              tma_store_3d(&omap, src + kRegion, 64, w.g * G, z);
+              bulk_commit();
+            }
+            store_src = stage;
+          }
         }
       }
       ++ucnt;
       cur = nxt;
     }
+    if (lane == 0) bulk_wait_all();  // the warp's output stores have completed
     if (!ok) atomicExch(&abort_flag, 1);
   }
 

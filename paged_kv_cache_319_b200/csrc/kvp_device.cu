@@ -211,13 +211,15 @@ int make_map_vcache(CUtensorMap* map, const void* base, int32_t dtype, uint64_t 
 // q of a prefill chunk as 3-D {128 dims, heads, tokens} (strides 256 and
 // heads * 256 bytes) with a {64, G, 128 / G} box: 128 rows (token, head of the
 // group), 128-byte swizzled, per 64-dim half.
+// Prefill queries or outputs [tokens, heads, 128]: box {64 dims, G heads,
+// rows / G tokens} (128 rows for a Q tile, 32 for one softmax warp's output).
 int make_map_prefill_q(CUtensorMap* map, const void* base, int32_t dtype, uint32_t heads,
-                       uint64_t tokens, uint32_t G) {
+                       uint64_t tokens, uint32_t G, uint32_t rows) {
   auto fn = encode_fn();
   if (!fn) return fail(KVP_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
   cuuint64_t dims[3] = {128, heads, tokens};
   cuuint64_t strides[2] = {256, uint64_t(heads) * 256};
-  cuuint32_t box[3] = {64, G, 128 / G};
+  cuuint32_t box[3] = {64, G, rows / G};
   cuuint32_t estr[3] = {1, 1, 1};
   const CUtensorMapDataType dt =
       dtype == KVP_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
@@ -500,13 +502,14 @@ int launch_tc_mq(const CUtensorMap& km, const CUtensorMap& vm, const CUtensorMap
 
 template <typename T, int BS>
 int launch_prefill_tc(const CUtensorMap& km, const CUtensorMap& vm, const CUtensorMap& qm,
-                      const kvp::dev::DecodeArgs& a, int32_t qtiles, cudaStream_t st) {
+                      const CUtensorMap& om, const kvp::dev::DecodeArgs& a, int32_t qtiles,
+                      cudaStream_t st) {
   auto k = kvp::dev::prefill_tc_kernel<T, BS>;
   cudaError_t e = ensure_smem(k, kvp::dev::pf::kSmemBytes);
   if (e != cudaSuccess) return cuda_fail(e, "prefill (prompt tiles): smem attribute");
   const int64_t units = int64_t(a.num_seqs) * a.num_kv_heads * qtiles * a.pmax;
   const int grid = int(units < sm_count() ? units : sm_count());
-  k<<<grid, kvp::dev::pf::kThreads, kvp::dev::pf::kSmemBytes, st>>>(km, vm, qm, a, qtiles, units);
+  k<<<grid, kvp::dev::pf::kThreads, kvp::dev::pf::kSmemBytes, st>>>(km, vm, qm, om, a, qtiles, units);
   e = cudaGetLastError();
   return e == cudaSuccess ? KVP_OK : cuda_fail(e, "prefill (prompt tiles): launch");
 }
@@ -922,8 +925,12 @@ int paged_attention_prefill(const void* q, const void* k_cache, const void* v_ca
   if (rc) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (prompt_tiles) {
+    CUtensorMap om;
     rc = make_map_prefill_q(&qm, q, dtype, uint32_t(num_q_heads), uint64_t(num_seqs) * q_len,
-                            uint32_t(G));
+                            uint32_t(G), 128);
+    if (!rc)
+      rc = make_map_prefill_q(&om, out, dtype, uint32_t(num_q_heads), uint64_t(num_seqs) * q_len,
+                              uint32_t(G), 32);
     if (rc) return rc;
     const int32_t qtiles = (q_len + 128 / G - 1) / (128 / G);
     a.q_first = 0;
@@ -932,11 +939,11 @@ int paged_attention_prefill(const void* q, const void* k_cache, const void* v_ca
     using H = __half;
     using B = __nv_bfloat16;
     if (block_size == 16)
-      rc = f16 ? launch_prefill_tc<H, 16>(km, vm, qm, a, qtiles, st)
-               : launch_prefill_tc<B, 16>(km, vm, qm, a, qtiles, st);
+      rc = f16 ? launch_prefill_tc<H, 16>(km, vm, qm, om, a, qtiles, st)
+               : launch_prefill_tc<B, 16>(km, vm, qm, om, a, qtiles, st);
     else
-      rc = f16 ? launch_prefill_tc<H, 32>(km, vm, qm, a, qtiles, st)
-               : launch_prefill_tc<B, 32>(km, vm, qm, a, qtiles, st);
+      rc = f16 ? launch_prefill_tc<H, 32>(km, vm, qm, om, a, qtiles, st)
+               : launch_prefill_tc<B, 32>(km, vm, qm, om, a, qtiles, st);
     if (rc || pmax <= 1) return rc;
     return f16 ? launch_reduce<H, 128>(a, st) : launch_reduce<B, 128>(a, st);
   }

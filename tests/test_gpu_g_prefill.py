@@ -8,7 +8,8 @@ partitions, launches that stop at the last token their queries see, and T = 1
 (the decode path). Chunks of at least 64 query rows (T x G, G a power of two)
 run on the prompt-shaped kernel (128 query rows per tensor-core tile): whole
 512-token prompts, grouped heads filling the rows (G = 2, 8, 16), a query
-tile cut short, long contexts split or not, and rows that see nothing.
+tile cut short (inside a warp's 32 rows too), long contexts split or not, and
+rows that see nothing.
 """
 
 import math
@@ -60,6 +61,10 @@ CASES = [
     (16, 8, 16, [64, 1500, 3000], 64, "f16", 0),         # G = 2, long contexts unsplit
     (8, 8, 16, [40, 300], 100, "f16", 128),              # ctx 40 < T: 60 rows see nothing
     (4, 4, 16, [1, 129, 1000], 300, "bf16", 128),        # ctx 1 < T; partitions cut the tiles
+    # unsplit, last tile cut inside a warp's rows: whole warps store through
+    # TMA, the rest row by row
+    (8, 8, 16, [200, 900], 200, "f16", 0),               # last tile: 72 tokens
+    (16, 4, 16, [72, 1000], 72, "bf16", 0),              # G = 4: last tile 8 tokens x 4 heads
 ]
 
 
