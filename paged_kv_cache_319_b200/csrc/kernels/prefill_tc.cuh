@@ -23,15 +23,19 @@
 // Warp roles (192 threads, one CTA per SM, persistent over units):
 //   warp 0     producer: TMA loads of Q (a 3-D box {64 dims, G heads, 128 / G
 //              tokens} per 64-dim half) and of K then V tiles (the decode
-//              kernel's per-block boxes) into a 3-stage ring.
-//   warp 1     MMA issuer and TMEM owner: QK of tile n + 1 is issued before
-//              PV of tile n; S is double-buffered, O double-buffered by unit.
+//              kernel's per-block boxes) into a 3-stage ring, in the order
+//              the MMAs take them (K of tile t, then V of tile t - 2).
+//   warp 1     MMA issuer and TMEM owner: QK of tile t, then PV of tile t - 2,
+//              and a unit's last two PVs at its end; S is double-buffered, O
+//              double-buffered by unit.
 //   warps 2-5  softmax and epilogue, thread = TMEM lane = row: per tile a
 //              masked row max (causal: key j visible to the row's position),
 //              p = 2^(s - m) into shared memory, and at a unit's end the
 //              normalised row (or its partial for the split-context reduce).
 //              fp16 inputs: P is double-buffered (the softmax of tile n + 1
-//              runs while PV of tile n does); bf16: one buffer of hi + lo.
+//              runs while PV of tile n does) and a unit's epilogue waits
+//              until after the next tile's softmax; bf16: one buffer of hi +
+//              lo, epilogue at once.
 // The running maximum m of a row moves only when a tile's maximum exceeds it
 // by more than 8 (log2 units); O and l are then rescaled in TMEM, once the
 // previous PV has completed, so p <= 2^8 and (m, l, O) stay a consistent
@@ -88,19 +92,21 @@ struct Unit {
 // (sequence, head) are rotated by the round in which its first unit is dealt,
 // so a CTA meets every query tile in turn (a causal prompt's tile qt has qt + 1
 // key tiles; without the rotation a grid that is a multiple of the tile count
-// would hand each CTA one tile index throughout).
-__device__ __forceinline__ void unit_at(const DecodeArgs& a, int64_t u, int32_t G, int32_t qtiles,
+// would hand each CTA one tile index throughout). Unit indices are below
+// kMaxUnits (the host's bound), so the arithmetic is 32-bit.
+constexpr uint32_t kMaxUnits = 0x7FF00000u;
+__device__ __forceinline__ void unit_at(const DecodeArgs& a, uint32_t u, uint32_t G, uint32_t qtiles,
                                         const int32_t* ctx_sm, Unit& w) {
-  const int32_t tq = kRows / G;
-  const int64_t per_head = int64_t(qtiles) * a.pmax;
-  const int64_t head_unit = u / per_head;  // (sequence, KV head)
-  const int32_t within = int32_t(u - head_unit * per_head);
-  const int32_t rot = int32_t(((head_unit * per_head) / gridDim.x) % qtiles);
-  w.p = within % a.pmax;
-  const int32_t qt = qtiles - 1 - (within / a.pmax + rot) % qtiles;
-  int64_t rest = head_unit;
-  w.g = int32_t(rest % a.num_kv_heads);
-  w.s = int32_t(rest / a.num_kv_heads);
+  const int32_t tq = kRows / int32_t(G);
+  const uint32_t pmax = uint32_t(a.pmax);
+  const uint32_t per_head = qtiles * pmax;
+  const uint32_t head_unit = u / per_head;  // (sequence, KV head)
+  const uint32_t within = u - head_unit * per_head;
+  const uint32_t rot = ((head_unit * per_head) / gridDim.x) % qtiles;
+  w.p = int32_t(within % pmax);
+  const int32_t qt = int32_t(qtiles - 1 - (within / pmax + rot) % qtiles);
+  w.g = int32_t(head_unit % uint32_t(a.num_kv_heads));
+  w.s = int32_t(head_unit / uint32_t(a.num_kv_heads));
   w.ctx = ctx_sm ? ctx_sm[w.s] : load_ctx(a, w.s, w.g == 0 && qt == 0 && w.p == 0);
   w.q0 = qt * tq;
   w.nq = min(tq, a.q_len - w.q0);
@@ -111,30 +117,44 @@ __device__ __forceinline__ void unit_at(const DecodeArgs& a, int64_t u, int32_t 
   w.to_ws = w.ctx > a.part_tokens;
 }
 
-// Units with at least one key tile, in a CTA's order: blockIdx.x, + gridDim.x, ...
+// Units with at least one key tile, in a CTA's order: blockIdx.x, + gridDim.x,
+// ... A unit without one is passed to on_empty as the stream steps over it.
 struct UnitStream {
-  int64_t u, stride, n;
-  int32_t G, qtiles;
+  uint32_t u, stride, n;
+  uint32_t G, qtiles;
   const int32_t* ctx_sm;
   Unit w;
   bool valid;
+  template <typename F>
   __device__ __forceinline__ void init(const DecodeArgs& a, int32_t G_, int32_t qtiles_,
-                                       int64_t num_units, const int32_t* ctx_cache) {
-    G = G_;
-    qtiles = qtiles_;
-    n = num_units;
+                                       int64_t num_units, const int32_t* ctx_cache, F on_empty) {
+    G = uint32_t(G_);
+    qtiles = uint32_t(qtiles_);
+    n = uint32_t(num_units);
     ctx_sm = ctx_cache;
     stride = gridDim.x;
-    u = int64_t(blockIdx.x) - stride;
-    next(a);
+    u = blockIdx.x;
+    seek(a, on_empty);
   }
-  __device__ __forceinline__ void next(const DecodeArgs& a) {
-    for (u += stride; u < n; u += stride) {
+  __device__ __forceinline__ void init(const DecodeArgs& a, int32_t G_, int32_t qtiles_,
+                                       int64_t num_units, const int32_t* ctx_cache) {
+    init(a, G_, qtiles_, num_units, ctx_cache, [](const Unit&) {});
+  }
+  template <typename F>
+  __device__ __forceinline__ void next(const DecodeArgs& a, F on_empty) {
+    u += stride;
+    seek(a, on_empty);
+  }
+  __device__ __forceinline__ void next(const DecodeArgs& a) { next(a, [](const Unit&) {}); }
+  template <typename F>
+  __device__ __forceinline__ void seek(const DecodeArgs& a, F on_empty) {
+    for (; u < n; u += stride) {
       unit_at(a, u, G, qtiles, ctx_sm, w);
       if (w.ntiles > 0) {
         valid = true;
         return;
       }
+      on_empty(w);
     }
     valid = false;
   }
@@ -288,8 +308,8 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_tc_kernel(
     };
     UnitStream cur;
     cur.init(a, G, qtiles, num_units, ctx_sm);
-    int32_t pend_row = rows_total;
-    bool have_pend = false;
+    uint32_t n = 0;                               // tiles of the CTA's stream so far
+    int32_t v_row[2] = {rows_total, rows_total};  // rows of tiles n - 2 and n - 1
     while (cur.valid && ok) {
       const Unit w = cur.w;
       UnitStream nxt = cur;  // the next unit, decoded now (its loads overlap this one)
@@ -308,20 +328,18 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_tc_kernel(
       ok = __shfl_sync(0xffffffffu, ok, 0);
       ++ucnt;
       int32_t id = ok ? tile_id(w, 0) : -2;
-      for (int32_t t = 0; t < w.ntiles && ok; ++t) {
+      for (int32_t t = 0; t < w.ntiles && ok; ++t, ++n) {
         const int32_t id_next = t + 1 < w.ntiles ? tile_id(w, t + 1) : -2;
         const int32_t row = id_row(w, t, id);
-        load_tile(&kmap, row, false);                 // K of tile t
-        if (ok && have_pend) load_tile(&vmap, pend_row, true);  // V of the tile before
-        pend_row = row;
-        have_pend = true;
+        load_tile(&kmap, row, false);                          // K of tile n
+        if (ok && n >= 2) load_tile(&vmap, v_row[n & 1], true);  // V of tile n - 2
+        v_row[n & 1] = row;
         id = id_next;
       }
-      // V of the unit's last tile: its PV is issued before the next unit's QK
-      if (ok && have_pend) load_tile(&vmap, pend_row, true);
-      have_pend = false;
       cur = nxt;
     }
+    // V of the stream's last two tiles
+    for (uint32_t k = n < 2 ? 0u : n - 2; k < n && ok; ++k) load_tile(&vmap, v_row[k & 1], true);
     if (!ok) {
       atomicExch(&abort_flag, 1);
       if (lane == 0)
@@ -330,16 +348,17 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_tc_kernel(
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    // Order: QK(0), then per tile t > 0 QK(t) and PV(t - 1); a unit's last PV
-    // is issued at once, so its epilogue never waits for the next unit's Q.
+    // Order over the CTA's stream of tiles (units one after another): QK(n),
+    // then PV(n - 2), both waiting for the softmax of tile n - 2, and the last
+    // two PVs at the end: S of a tile never waits behind a PV or a unit
+    // boundary.
     uint32_t ctr = 0, ucnt = 0, n = 0;
     bool ok = true;
     struct Pend {
       uint32_t ob, ucnt;
       int32_t zero_from;
       bool first;
-    } pend{};
-    bool have_pend = false;
+    } pend[2] = {};
     // O[ob] (+)= (P_hi + P_lo) . V for the pending tile; the warp zeroes the V
     // rows of tokens past the context (they hold whatever the pool had there;
     // p is 0 for them, but 0 * inf is NaN).
@@ -431,20 +450,18 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_tc_kernel(
         ok = __shfl_sync(0xffffffffu, ok, 0);
         ++ctr;
         if (!ok) break;
-        // PV of the tile before
-        if (have_pend) pv(pend, n - 1);
+        if (n >= 2) pv(pend[n & 1], n - 2);  // PV of tile n - 2
         const int32_t k0 = w.k_begin + t * kKeys;
-        pend.ob = ucnt & 1u;
-        pend.ucnt = ucnt;
-        pend.first = t == 0;
-        pend.zero_from = w.ctx - k0;
-        have_pend = true;
+        pend[n & 1].ob = ucnt & 1u;
+        pend[n & 1].ucnt = ucnt;
+        pend[n & 1].first = t == 0;
+        pend[n & 1].zero_from = w.ctx - k0;
       }
-      if (ok && have_pend) pv(pend, n - 1);
-      have_pend = false;
       ++ucnt;
       cur = nxt;
     }
+    // the last two PVs
+    for (uint32_t k = n < 2 ? 0u : n - 2; k < n && ok; ++k) pv(pend[k & 1], k);
     if (!ok) atomicExch(&abort_flag, 1);
   } else {
     // ------------------------------------------------------------ softmax + epilogue
@@ -455,18 +472,15 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_tc_kernel(
       return __all_sync(0xffffffffu, mbar_wait(bar, parity, where)) != 0;
     };
     // Rows of query tiles that see no key (a context shorter than its chunk)
-    // in a sequence that is not split: zero output rows.
-    for (int64_t u = blockIdx.x; u < num_units; u += gridDim.x) {
-      Unit w;
-      unit_at(a, u, G, qtiles, ctx_sm, w);
-      if (w.ntiles > 0 || w.to_ws || w.p > 0) continue;
-      if (r / G < w.nq) {
-        const int64_t row = (int64_t(w.s) * a.q_len + w.q0 + r / G) * a.num_q_heads + w.g * G + r % G;
-        uint4* dst = reinterpret_cast<uint4*>(static_cast<T*>(a.out) + row * kD);
+    // in a sequence that is not split: zero output rows, as the stream steps
+    // over their units.
+    auto zero_rows = [&](const Unit& w) {
+      if (w.to_ws || w.p > 0 || r / G >= w.nq) return;
+      const int64_t row = (int64_t(w.s) * a.q_len + w.q0 + r / G) * a.num_q_heads + w.g * G + r % G;
+      uint4* dst = reinterpret_cast<uint4*>(static_cast<T*>(a.out) + row * kD);
 #pragma unroll
-        for (int c = 0; c < kD * 2 / 16; ++c) dst[c] = make_uint4(0, 0, 0, 0);
-      }
-    }
+      for (int c = 0; c < kD * 2 / 16; ++c) dst[c] = make_uint4(0, 0, 0, 0);
+    };
     uint32_t n = 0, ucnt = 0;
     uint32_t seen[2] = {0, 0};  // phases of p_free[b] consumed
     // P buffer that this warp's last output store may still be reading
@@ -482,14 +496,96 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_tc_kernel(
         ++seen[b];
       }
     };
+    // ---- epilogue of unit w (last tile nl, O buffer ob): the normalised rows,
+    // or the partial (m, l, O) of a split sequence, once PV(nl) has completed
+    auto epilogue = [&](const Unit& w, float m_ref, float l, uint32_t nl, uint32_t ob) {
+      wait_pv(nl);
+      if (!ok) return;
+      tc_fence_after();
+      const int32_t ti = r / G;  // query token of the row within the tile
+      const bool row_live = ti < w.nq;
+      const uint32_t o_taddr = tmem_base + lane_addr + kOCol + ob * kD;
+      const int64_t qrow = (int64_t(w.s) * a.q_len + w.q0 + ti) * a.num_q_heads + w.g * G + r % G;
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      // an unsplit unit's rows go out through the P buffer of tile nl (its PV
+      // has completed) and one TMA store per 64-dim half, when every row of
+      // the warp is a token of the chunk
+      const int32_t tw = 32 / G;  // tokens of the warp's rows
+      const bool staged = !w.to_ws && (quarter + 1) * tw <= w.nq;
+      uint8_t* stage = kLo ? phi : ((nl & 1u) ? plo : phi);
+#pragma unroll 1
+      for (int c = 0; c < kD / 32; ++c) {
+        float ov[32];
+        tc::tmem_ld_cols<32>(o_taddr + c * 32, ov);
+        tmem_ld_wait();
+        if (c == kD / 32 - 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&o_free[ob]);
+        }
+        if (staged) {
+          // dims c*32 .. +32 of row r: four 16-byte chunks of region c / 2
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int chunk = (c & 1) * 4 + q;
+            const uint32_t off = (c >> 1) * kRegion + r * 128 + ((chunk ^ (r & 7)) << 4);
+            *reinterpret_cast<uint4*>(stage + off) =
+                make_uint4(Elem<T>::pack2(ov[8 * q] * inv, ov[8 * q + 1] * inv),
+                           Elem<T>::pack2(ov[8 * q + 2] * inv, ov[8 * q + 3] * inv),
+                           Elem<T>::pack2(ov[8 * q + 4] * inv, ov[8 * q + 5] * inv),
+                           Elem<T>::pack2(ov[8 * q + 6] * inv, ov[8 * q + 7] * inv));
+          }
+          continue;
+        }
+        if (!row_live) continue;
+        if (!w.to_ws) {
+          uint4* dst = reinterpret_cast<uint4*>(static_cast<T*>(a.out) + qrow * kD + c * 32);
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            dst[q] = make_uint4(Elem<T>::pack2(ov[8 * q] * inv, ov[8 * q + 1] * inv),
+                                Elem<T>::pack2(ov[8 * q + 2] * inv, ov[8 * q + 3] * inv),
+                                Elem<T>::pack2(ov[8 * q + 4] * inv, ov[8 * q + 5] * inv),
+                                Elem<T>::pack2(ov[8 * q + 6] * inv, ov[8 * q + 7] * inv));
+        } else {
+          float4* dst = reinterpret_cast<float4*>(a.ws_acc + (qrow * a.ws_slots + w.p) * kD + c * 32);
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            dst[q] = make_float4(ov[4 * q], ov[4 * q + 1], ov[4 * q + 2], ov[4 * q + 3]);
+        }
+      }
+      if (row_live && w.to_ws) {
+        a.ws_ml[(qrow * a.ws_slots + w.p) * 2 + 0] = m_ref;
+        a.ws_ml[(qrow * a.ws_slots + w.p) * 2 + 1] = l;
+      }
+      if (staged) {
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          const uint8_t* src = stage + quarter * 32 * 128;
+          const int32_t z = w.s * a.q_len + w.q0 + quarter * tw;
+          tma_store_3d(&omap, src, 0, w.g * G, z);
+          tma_store_3d(&omap, src + kRegion, 64, w.g * G, z);
+          bulk_commit();
+        }
+        store_src = stage;
+      }
+    };
+    // fp16: a unit's epilogue runs after the softmax of the next tile, by which
+    // time its last PV has completed (the P buffer of tile nl + 1 is the other
+    // one); bf16 P fills both buffers, so its epilogue runs at once.
+    struct Deferred {
+      Unit w;
+      float m, l;
+      uint32_t nl, ob;
+      bool valid;
+    } dfr{};
     UnitStream cur;
-    cur.init(a, G, qtiles, num_units, ctx_sm);
+    cur.init(a, G, qtiles, num_units, ctx_sm, zero_rows);
     while (cur.valid && ok) {
       const Unit w = cur.w;
       UnitStream nxt = cur;
-      nxt.next(a);
+      nxt.next(a, zero_rows);
       const int32_t ti = r / G;  // query token of the row within the tile
-      const bool row_live = ti < w.nq;
       const int32_t pos = w.ctx - a.q_len + w.q0 + ti;   // the row sees keys j <= pos
       const int32_t lim = min(pos + 1, w.k_end);          // exclusive end of its keys here
       float m_ref = -INFINITY, l = 0.f;
@@ -618,80 +714,28 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_tc_kernel(
           mbar_arrive(&s_free[sb]);
           mbar_arrive(&p_full[kLo ? 0u : (n & 1u)]);
         }
-        if (t == w.ntiles - 1) {
-          // ---- epilogue: O of the unit once its last PV has completed
-          wait_pv(n);
+        if (!kLo && dfr.valid) {
+          epilogue(dfr.w, dfr.m, dfr.l, dfr.nl, dfr.ob);
+          dfr.valid = false;
           if (!ok) break;
-          tc_fence_after();
-          const int64_t qrow = (int64_t(w.s) * a.q_len + w.q0 + ti) * a.num_q_heads + w.g * G + r % G;
-          const float inv = l > 0.f ? 1.f / l : 0.f;
-          // an unsplit unit's rows go out through the P buffer of tile n (its PV
-          // has completed) and one TMA store per 64-dim half, when every row of
-          // the warp is a token of the chunk
-          const int32_t tw = 32 / G;  // tokens of the warp's rows
-          const bool staged = !w.to_ws && (quarter + 1) * tw <= w.nq;
-          uint8_t* stage = kLo ? phi : ((n & 1u) ? plo : phi);
-#pragma unroll 1
-          for (int c = 0; c < kD / 32; ++c) {
-            float ov[32];
-            tc::tmem_ld_cols<32>(o_taddr + c * 32, ov);
-            tmem_ld_wait();
-            if (c == kD / 32 - 1) {
-              tc_fence_before();
-              __syncwarp();
-              if (lane == 0) mbar_arrive(&o_free[ob]);
-            }
-            if (staged) {
-              // dims c*32 .. +32 of row r: four 16-byte chunks of region c / 2
-#pragma unroll
-              for (int q = 0; q < 4; ++q) {
-                const int chunk = (c & 1) * 4 + q;
-                const uint32_t off = (c >> 1) * kRegion + r * 128 + ((chunk ^ (r & 7)) << 4);
-                *reinterpret_cast<uint4*>(stage + off) =
-                    make_uint4(Elem<T>::pack2(ov[8 * q] * inv, ov[8 * q + 1] * inv),
-                               Elem<T>::pack2(ov[8 * q + 2] * inv, ov[8 * q + 3] * inv),
-                               Elem<T>::pack2(ov[8 * q + 4] * inv, ov[8 * q + 5] * inv),
-                               Elem<T>::pack2(ov[8 * q + 6] * inv, ov[8 * q + 7] * inv));
-              }
-              continue;
-            }
-            if (!row_live) continue;
-            if (!w.to_ws) {
-              uint4* dst = reinterpret_cast<uint4*>(static_cast<T*>(a.out) + qrow * kD + c * 32);
-#pragma unroll
-              for (int q = 0; q < 4; ++q)
-                dst[q] = make_uint4(Elem<T>::pack2(ov[8 * q] * inv, ov[8 * q + 1] * inv),
-                                    Elem<T>::pack2(ov[8 * q + 2] * inv, ov[8 * q + 3] * inv),
-                                    Elem<T>::pack2(ov[8 * q + 4] * inv, ov[8 * q + 5] * inv),
-                                    Elem<T>::pack2(ov[8 * q + 6] * inv, ov[8 * q + 7] * inv));
-            } else {
-              float4* dst = reinterpret_cast<float4*>(a.ws_acc + (qrow * a.ws_slots + w.p) * kD + c * 32);
-#pragma unroll
-              for (int q = 0; q < 8; ++q)
-                dst[q] = make_float4(ov[4 * q], ov[4 * q + 1], ov[4 * q + 2], ov[4 * q + 3]);
-            }
-          }
-          if (row_live && w.to_ws) {
-            a.ws_ml[(qrow * a.ws_slots + w.p) * 2 + 0] = m_ref;
-            a.ws_ml[(qrow * a.ws_slots + w.p) * 2 + 1] = l;
-          }
-          if (staged) {
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) {
-              const uint8_t* src = stage + quarter * 32 * 128;
-              const int32_t z = w.s * a.q_len + w.q0 + quarter * tw;
-              tma_store_3d(&omap, src, 0, w.g * G, z);
-              tma_store_3d(&omap, src + kRegion, 64, w.g * G, z);
-              bulk_commit();
-            }
-            store_src = stage;
+        }
+        if (t == w.ntiles - 1) {
+          if (kLo) {
+            epilogue(w, m_ref, l, n, ob);
+          } else {
+            dfr.w = w;
+            dfr.m = m_ref;
+            dfr.l = l;
+            dfr.nl = n;
+            dfr.ob = ob;
+            dfr.valid = true;
           }
         }
       }
       ++ucnt;
       cur = nxt;
     }
+    if (ok && dfr.valid) epilogue(dfr.w, dfr.m, dfr.l, dfr.nl, dfr.ob);
     if (lane == 0) bulk_wait_all();  // the warp's output stores have completed
     if (!ok) atomicExch(&abort_flag, 1);
   }

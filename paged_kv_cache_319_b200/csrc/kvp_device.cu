@@ -508,6 +508,9 @@ int launch_prefill_tc(const CUtensorMap& km, const CUtensorMap& vm, const CUtens
   cudaError_t e = ensure_smem(k, kvp::dev::pf::kSmemBytes);
   if (e != cudaSuccess) return cuda_fail(e, "prefill (prompt tiles): smem attribute");
   const int64_t units = int64_t(a.num_seqs) * a.num_kv_heads * qtiles * a.pmax;
+  if (units >= int64_t(kvp::dev::pf::kMaxUnits))
+    return fail(KVP_ERR_INVALID, "paged_attention_prefill: %lld work units exceed the kernel's index range",
+                static_cast<long long>(units));
   const int grid = int(units < sm_count() ? units : sm_count());
   k<<<grid, kvp::dev::pf::kThreads, kvp::dev::pf::kSmemBytes, st>>>(km, vm, qm, om, a, qtiles, units);
   e = cudaGetLastError();
