@@ -179,6 +179,29 @@ __device__ __forceinline__ void tmem_st_x32(uint32_t taddr, const float (&v)[32]
       : "memory");
 }
 
+// Two fp32 lanes in one 64-bit register: packed FMA and add (each lane rounds
+// as its scalar instruction does).
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t d;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(lo), "f"(hi));
+  return d;
+}
+__device__ __forceinline__ float2 f2_unpack(uint64_t v) {
+  float2 r;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
 __device__ __forceinline__ void tmem_st_wait() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
@@ -601,7 +624,9 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_tc_kernel(
         // every row of the warp sees the whole tile (all but the diagonal tiles):
         // no per-key masks
         const bool full = __all_sync(0xffffffffu, k0 + kKeys <= lim);
-        // pass 1: the row's largest scaled score over the tile (keys it sees)
+        // pass 1: the row's largest score over the tile (keys it sees), scaled
+        // once (scaling by a positive factor commutes with the max, rounding
+        // included)
         float mx = -INFINITY;
 #pragma unroll 1
         for (int c = 0; c < kKeys / 32; ++c) {
@@ -612,18 +637,19 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_tc_kernel(
           if (full) {
 #pragma unroll
             for (int e = 0; e < 32; e += 2) {
-              m0 = fmaxf(m0, sv[e] * a.scale_log2);
-              m1 = fmaxf(m1, sv[e + 1] * a.scale_log2);
+              m0 = fmaxf(m0, sv[e]);
+              m1 = fmaxf(m1, sv[e + 1]);
             }
           } else {
 #pragma unroll
             for (int e = 0; e < 32; e += 2) {
-              if (k0 + c * 32 + e < lim) m0 = fmaxf(m0, sv[e] * a.scale_log2);
-              if (k0 + c * 32 + e + 1 < lim) m1 = fmaxf(m1, sv[e + 1] * a.scale_log2);
+              if (k0 + c * 32 + e < lim) m0 = fmaxf(m0, sv[e]);
+              if (k0 + c * 32 + e + 1 < lim) m1 = fmaxf(m1, sv[e + 1]);
             }
           }
           mx = fmaxf(mx, fmaxf(m0, m1));
         }
+        mx *= a.scale_log2;
         // the running maximum moves only by more than kLazy
         float factor = 1.f;
         bool need = false;
@@ -657,8 +683,10 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_tc_kernel(
         }
         l *= factor;
         // pass 2: p = 2^(s - m) (bf16: as hi + lo parts) into P (row r, 128-byte
-        // swizzle); l sums the rounded p the MMA multiplies
+        // swizzle); l sums p in fp32 (pairs of lanes per instruction)
         const float nm = -m_ref;
+        const uint64_t scale2 = f2_pack(a.scale_log2, a.scale_log2);
+        const uint64_t nm2 = f2_pack(nm, nm);
         uint8_t* pdst = kLo ? phi : ((n & 1u) ? plo : phi);
         if (store_src == pdst) {  // the warp's output rows staged there have been read
           if (lane == 0) bulk_wait_read();
@@ -671,29 +699,26 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_tc_kernel(
           tc::tmem_ld_cols<32>(s_taddr + c * 32, sv);
           tmem_ld_wait();
           uint32_t hw[16], lw[16];
-          float l0 = 0.f, l1 = 0.f;
+          uint64_t l2 = f2_pack(0.f, 0.f);
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
             const int j = k0 + c * 32 + e;
-            float p0 = tc::ex2_ftz(fmaf(sv[e], a.scale_log2, nm));
-            float p1 = tc::ex2_ftz(fmaf(sv[e + 1], a.scale_log2, nm));
+            const float2 x = f2_unpack(f2_fma(f2_pack(sv[e], sv[e + 1]), scale2, nm2));
+            float p0 = tc::ex2_ftz(x.x);
+            float p1 = tc::ex2_ftz(x.y);
             if (!full) {  // keys the row does not see (select, not multiply: NaN scores)
               p0 = j < lim ? p0 : 0.f;
               p1 = j + 1 < lim ? p1 : 0.f;
             }
             hw[e / 2] = Elem<T>::pack2(p0, p1);
-            const float2 hf = Elem<T>::to_float2(hw[e / 2]);
             if constexpr (kLo) {
+              const float2 hf = Elem<T>::to_float2(hw[e / 2]);
               lw[e / 2] = Elem<T>::pack2(p0 - hf.x, p1 - hf.y);
-              const float2 lf = Elem<T>::to_float2(lw[e / 2]);
-              l0 += hf.x + lf.x;
-              l1 += hf.y + lf.y;
-            } else {
-              l0 += hf.x;
-              l1 += hf.y;
             }
+            l2 = f2_add(l2, f2_pack(p0, p1));
           }
-          l += l0 + l1;
+          const float2 lp = f2_unpack(l2);
+          l += lp.x + lp.y;
           // keys c*32 .. +32 of row r: four 16-byte chunks of region c / 2
           const int region = c >> 1;
 #pragma unroll
