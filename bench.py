@@ -93,8 +93,8 @@ def kernel_sha(files):
 
 
 def traffic_per_launch(kernel, alg_bytes):
-    p = PROFILED_TRAFFIC[kernel]
-    if kernel_sha(p["files"]) != p["sha"]:
+    p = PROFILED_TRAFFIC.get(kernel)
+    if p is None or kernel_sha(p["files"]) != p["sha"]:
         return None
     return int(p["ratio"] * alg_bytes)
 
@@ -761,7 +761,8 @@ OTHER_WORKLOADS = [
     ("gqa_long_bs16", "decode", 0), ("gqa_long_bs32", "decode", 0),
     ("llama13b_churn", "schedule", 0), ("sharing_A", "schedule", 200),
     ("sharing_B", "schedule", 200), ("beam", "schedule", 200),
-    ("opt13b_fp8", "fp8", 200), ("prefill_opt13b_t16", "prefill", 200),
+    ("opt13b_fp8", "fp8", 200), ("gqa_long_bs16_fp8", "fp8", 100),
+    ("prefill_opt13b_t16", "prefill", 200),
     ("prefill_gqa_bs16_t4", "prefill", 200), ("prefill_prompt512", "prefill", 50),
     ("vcache_opt13b", "vcache", 200), ("vcache_gqa_long_bs16", "vcache", 100),
 ]
@@ -1256,22 +1257,25 @@ def prefill_record(args):
     return res
 
 
-FP8_WORKLOADS = ("opt13b_fp8",)
+FP8_WORKLOADS = ("opt13b_fp8", "gqa_long_bs16_fp8")
 # the virtually contiguous cache against the paged one, on a workload's batch
 VCACHE_WORKLOADS = {"vcache_opt13b": "opt13b", "vcache_gqa_long_bs16": "gqa_long_bs16"}
 
 
 def fp8_record(args):
-    """paged_attention_decode_fp8 on the OPT-13B batch with an E4M3 cache, timed with
-    CUDA events (median of --steps calls, L2 flushed before each), beside the 16-bit
-    decode of the same batch; roofline on the E4M3 algorithmic bytes."""
+    """paged_attention_decode_fp8 on a decode batch (OPT-13B, or long-context GQA)
+    with an E4M3 cache, timed with CUDA events (median of --steps calls, L2 flushed
+    before each), beside the 16-bit decode of the same batch; roofline on the E4M3
+    algorithmic bytes."""
     import torch
     import paged_kv_cache_319_b200 as kvp
 
     device = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
     torch.cuda.set_device(device)
-    wl = workloads.by_name("opt13b")
+    base = args.workload[:-len("_fp8")]
+    wl = workloads.by_name(base)
     g = wl.geometry
+    qdt = torch.float16 if g.dtype == "f16" else torch.bfloat16
     lens = np.asarray(wl.info["context_lens"], np.int64)
     S, Hq, Hkv, D, bs, part = len(lens), g.num_q_heads, g.num_kv_heads, g.head_dim, g.block_size, 512
     rng = np.random.default_rng(4001)
@@ -1292,7 +1296,7 @@ def fp8_record(args):
     kc, vc = codes(), codes()
     ks = torch.linspace(1 / 448, 2 / 448, Hkv, device=device, dtype=torch.float32)
     vs = torch.linspace(1 / 448, 4 / 448, Hkv, device=device, dtype=torch.float32)
-    q = torch.randn((S, Hq, D), generator=gen, device=device, dtype=torch.float32).half()
+    q = torch.randn((S, Hq, D), generator=gen, device=device, dtype=torch.float32).to(qdt)
     tt = torch.from_numpy(tables).to(device)
     cl = torch.from_numpy(lens.astype(np.int32)).to(device)
     mcl = int(lens.max())
@@ -1326,8 +1330,8 @@ def fp8_record(args):
     with ClockSampler(device) as clk:
         ms = timed(call, steps)
     # the new token of every sequence, quantised into the cache (one decode step's scatter)
-    kn = torch.randn((S, Hkv, D), generator=gen, device=device, dtype=torch.float32).half()
-    vn = torch.randn((S, Hkv, D), generator=gen, device=device, dtype=torch.float32).half()
+    kn = torch.randn((S, Hkv, D), generator=gen, device=device, dtype=torch.float32).to(qdt)
+    vn = torch.randn((S, Hkv, D), generator=gen, device=device, dtype=torch.float32).to(qdt)
     slots = torch.from_numpy((tables[np.arange(S), (lens - 1) // bs].astype(np.int64) * bs
                               + (lens - 1) % bs)).to(device)
     scatter = lambda: kvp.reshape_and_cache_fp8(kn, vn, kc, vc, slots, ks, vs)  # noqa: E731
@@ -1337,8 +1341,8 @@ def fp8_record(args):
     kvp.check_device_error(device)
     # the 16-bit decode of the same batch (fp16 K/V of the same shape)
     del kc, vc
-    k16 = torch.randn((NB, Hkv, bs, D), generator=gen, device=device, dtype=torch.float32).half()
-    v16 = torch.randn((NB, Hkv, bs, D), generator=gen, device=device, dtype=torch.float32).half()
+    k16 = torch.randn((NB, Hkv, bs, D), generator=gen, device=device, dtype=torch.float32).to(qdt)
+    v16 = torch.randn((NB, Hkv, bs, D), generator=gen, device=device, dtype=torch.float32).to(qdt)
     call16 = lambda: kvp.paged_attention_decode(q, k16, v16, tt, cl, scale, out,  # noqa: E731
                                                 max_context_len=mcl, partition_size=part,
                                                 workspace=ws)
@@ -1355,10 +1359,12 @@ def fp8_record(args):
         "metric": METRIC, "value": round(achieved, 2), "unit": UNIT, "n_gpus": 1,
         "steps": steps, "warmup": max(3, args.warmup), "ms_per_step": round(ms, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "e4m3 (K/V cache), f16 (q, out), fp32 accumulation",
+        "dtype": f"e4m3 (K/V cache), {g.dtype} (q, out), fp32 accumulation",
         "data": "synthetic (uniform E4M3 codes, per-KV-head scales; seeded N(0,1) q)",
-        "config": {"workload": "OPT-13B geometry, one layer: 64 seqs, 40 heads x 128, block 16, "
-                               "ctx U[1,2048], E4M3 cache with per-KV-head scales, partitions of 512",
+        "config": {"workload": (wl.description + ", E4M3 cache with per-KV-head scales"
+                                if base != "opt13b" else
+                                "OPT-13B geometry, one layer: 64 seqs, 40 heads x 128, block 16, "
+                                "ctx U[1,2048], E4M3 cache with per-KV-head scales, partitions of 512"),
                    "name": args.workload,
                    "timed": f"paged_attention_decode_fp8 (median of {steps} calls, L2 flushed "
                             "before each)"},
@@ -1367,11 +1373,14 @@ def fp8_record(args):
                                  "seq_tokens_per_s": round(float(lens.sum()) / (ms16 * 1e-3), 1),
                                  "speedup_of_e4m3": round(ms16 / ms, 3)},
         "rows": {"reshape_and_cache_fp8_step": {"tokens": S, "us": round(scatter_ms * 1e3, 2)}},
-        "roofline": {"kernel": "paged_attention_decode_fp8: decode_simt (E4M3) + decode_reduce_kernel",
+        "roofline": {"kernel": ("paged_attention_decode_fp8: decode_tc (E4M3 tiles widened in shared "
+                                "memory) + decode_reduce_kernel" if Hq > Hkv else
+                                "paged_attention_decode_fp8: decode_simt (E4M3) + decode_reduce_kernel"),
                      "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
                      "peak_source": peak_kind, "unit": "GB/s", "frac": round(achieved / peak, 4),
                      "algorithmic_bytes_per_launch": int(alg), "avg_launch_us": round(ms * 1e3, 2),
-                     "traffic": traffic_per_launch("decode_simt_fp8", alg)},
+                     "traffic": traffic_per_launch("decode_simt_fp8" if Hq == Hkv else "decode_tc_fp8",
+                                                   alg)},
         "clocks": clk.summary(),
     }
     return res
@@ -1384,7 +1393,7 @@ def run_reference_sampled(args, world):
     from oracle import attention, fp8
 
     fp8_case = args.workload in FP8_WORKLOADS
-    base, T = ("opt13b", 1) if fp8_case else PREFILL_WORKLOADS[args.workload]
+    base, T = (args.workload[:-len("_fp8")], 1) if fp8_case else PREFILL_WORKLOADS[args.workload]
     if base == "prompt512":
         g = workloads.Geometry(40, 40, 128, 16, "f16")
         lens = np.full(64, 512, np.int64)

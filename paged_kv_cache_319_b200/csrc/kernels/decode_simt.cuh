@@ -254,9 +254,10 @@ __device__ __forceinline__ void simt_tile(const uint8_t* kt, const uint8_t* vt, 
 // precision fma (fp16 x fp16 + fp32; the products are exact in fp32), with
 // the scales applied to the dot. On the OPT-13B batch this took the call from
 // 142 us (keys widened to fp32 first) to 118 us; widening by shifts and masks
-// instead of cvt was slower (167 us). A bf16 q, and the PV products (p is
-// fp32), use fp32 FMAs. The value scale is applied by the caller to the
-// finished accumulator.
+// instead of cvt was slower (167 us). A bf16 q uses fp32 FMAs for the QK
+// products. The PV products take p rounded to fp16 (p <= 1, relative error
+// at most 2^-12) and the fp16 codes in the same mixed-precision fma; the value
+// scale is applied by the caller to the finished accumulator.
 #ifndef KVP_FP8_MIXED
 #define KVP_FP8_MIXED 1  // 0: widen fp16 keys to fp32 for the QK products as well
 #endif
@@ -270,6 +271,25 @@ __device__ __forceinline__ void fma2_f16_f32(float& d0, float& d1, uint32_t q2, 
       "fma.rn.f32.f16 %1, qh, kh, %1;\n\t}"
       : "+f"(d0), "+f"(d1)
       : "r"(q2), "r"(k2));
+}
+
+// acc[0..3] += p * v[0..3] for four E4M3 codes of a value row (bytes of v4,
+// lowest first): the codes widen exactly to fp16 (two per cvt) and meet p,
+// rounded once to fp16, in the mixed-precision fma with fp32 accumulation.
+__device__ __forceinline__ void fma4_p16_e4m3(float (&acc)[4], uint32_t p16, uint32_t v4) {
+  uint32_t k01, k23;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(k01) : "h"(static_cast<uint16_t>(v4)));
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(k23) : "h"(static_cast<uint16_t>(v4 >> 16)));
+  asm("{\n\t.reg .f16 p, pz, a, b, c, d;\n\t"
+      "mov.b32 {p, pz}, %4;\n\t"
+      "mov.b32 {a, b}, %5;\n\t"
+      "mov.b32 {c, d}, %6;\n\t"
+      "fma.rn.f32.f16 %0, p, a, %0;\n\t"
+      "fma.rn.f32.f16 %1, p, b, %1;\n\t"
+      "fma.rn.f32.f16 %2, p, c, %2;\n\t"
+      "fma.rn.f32.f16 %3, p, d, %3;\n\t}"
+      : "+f"(acc[0]), "+f"(acc[1]), "+f"(acc[2]), "+f"(acc[3])
+      : "r"(p16), "r"(k01), "r"(k23));
 }
 
 // MX: q is fp16 and arrives as 32 packed pairs in qh (qf unused), unscaled; the
@@ -322,12 +342,13 @@ __device__ __forceinline__ void simt_tile_fp8(const uint8_t* kt, const uint8_t* 
   tmax = warp_max(tmax);
   const float m_new = fmaxf(m_run, tmax);
   const float alpha = m_run == -INFINITY ? 0.f : exp2f(m_run - m_new);
-  float pr[kPasses];
+  uint32_t p16[kPasses];  // p in fp16 (p <= 1) for the value products; l sums it in fp32
   float psum = 0.f;
 #pragma unroll
   for (int ps = 0; ps < kPasses; ++ps) {
-    pr[ps] = sc[ps] == -INFINITY ? 0.f : exp2f(sc[ps] - m_new);
-    psum += pr[ps];
+    const float p = sc[ps] == -INFINITY ? 0.f : exp2f(sc[ps] - m_new);
+    p16[ps] = __half_as_ushort(__float2half_rn(p));
+    psum += p;
   }
   l_lane = l_lane * alpha + (lane < 16 ? psum : 0.f);
 #pragma unroll
@@ -338,16 +359,10 @@ __device__ __forceinline__ void simt_tile_fp8(const uint8_t* kt, const uint8_t* 
   const int pos = (lane & 3) * 4;
 #pragma unroll
   for (int r = 0; r < BS; ++r) {
-    const float pv = __shfl_sync(0xffffffffu, pr[r >> 4], r & 15);
-    if (r < nvalid) {
-      const uint32_t v = *reinterpret_cast<const uint32_t*>(vt + r * 128 + ((cc ^ (r & 7)) << 4) + pos);
-      const float2 f0 = e4m3x2_to_float2(v);
-      const float2 f1 = e4m3x2_to_float2(v >> 16);
-      acc[0] = fmaf(pv, f0.x, acc[0]);
-      acc[1] = fmaf(pv, f0.y, acc[1]);
-      acc[2] = fmaf(pv, f1.x, acc[2]);
-      acc[3] = fmaf(pv, f1.y, acc[3]);
-    }
+    const uint32_t pv = __shfl_sync(0xffffffffu, p16[r >> 4], r & 15);
+    if (r < nvalid)
+      fma4_p16_e4m3(acc, pv,
+                    *reinterpret_cast<const uint32_t*>(vt + r * 128 + ((cc ^ (r & 7)) << 4) + pos));
   }
 }
 

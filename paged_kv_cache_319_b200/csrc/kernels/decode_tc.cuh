@@ -49,7 +49,9 @@ static_assert(grp::kHdrWords == kPlanSeqWord, "plan layout");
 
 namespace tc {
 
-enum Mode : int { kPlain = 0, kGrouped = 1, kMultiQuery = 2, kContig = 3, kPacked = 4 };
+// kPlainF8: kPlain over an E4M3 cache (codes widened to the query type in
+// shared memory by four converter warps; scales per KV head).
+enum Mode : int { kPlain = 0, kGrouped = 1, kMultiQuery = 2, kContig = 3, kPacked = 4, kPlainF8 = 5 };
 
 constexpr int kD = 128;             // head_dim
 constexpr int kN = 16;              // MMA N (query heads of a group, padded)
@@ -68,6 +70,9 @@ constexpr int kTmemCols = 256;
 constexpr int kSCol = 0;                             // S buffers: [0, 128)
 constexpr int kOCol = 128;                           // O buffers: [128, 128 + 2 * kNPV)
 constexpr int kThreads = 192;
+constexpr int kThreadsF8 = 320;          // + four converter warps (E4M3 cache)
+constexpr int kCodeBytes = 128 * 128;    // 16 KiB: E4M3 codes of one 128-token tile
+constexpr int kCodeOffset = 16 * 1024;   // where they land in a 32 KiB stage
 constexpr int kSoftmaxThreads = 128;
 // Batches of up to Cfg<NG>::kCtxCap sequences (at most kCtxCacheMax) keep their
 // context lengths in shared memory, so no warp role waits on a global load when
@@ -83,13 +88,15 @@ constexpr int kCtxCacheMax = 4096;
 // other every 16 bytes, and column groups are kPSbo bytes apart. A softmax
 // thread owns one token, so it writes its columns with 16-byte stores, and a
 // warp's 32 tokens fill 512 contiguous bytes.
-template <int NG>
+template <int NG, bool F8 = false>
 struct Cfg {
   static constexpr int kNPV = 2 * NG <= 16 ? 16 : 32;  // N of the PV MMA
 #ifndef KVP_TC_STAGES
 #define KVP_TC_STAGES 5
 #endif
-  // groups of 16 need a P^T twice as wide, which costs one stage
+  // groups of 16 need a P^T twice as wide, which costs one stage. An E4M3
+  // cache lands its codes in the upper half of a stage (kCodeOffset), where the
+  // converter warps widen them over the whole stage.
   static constexpr int kStages = NG <= 8 ? KVP_TC_STAGES : KVP_TC_STAGES - 1;
   static constexpr int kPBytes = kChunkTok * kNPV * 2;
   static constexpr int kPSbo = kChunkTok * 16;          // bytes between 8-column groups of P^T
@@ -97,11 +104,12 @@ struct Cfg {
   static constexpr int kOffQ = kOffRing + kStages * kStageBytes;
   static constexpr int kOffP = kOffQ + 2 * kQBytes;
   static constexpr int kOffBar = kOffP + 2 * kPBytes;
-  static constexpr int kNumBars = 2 * kStages + 2 * 10;
+  static constexpr int kNumBars = 2 * kStages + 2 * 10 + (F8 ? kStages : 0);
   static constexpr int kOffRed = kOffBar + kNumBars * 8;     // [2 halves][4 warps][kN] maxima
   static constexpr int kOffRedL = kOffRed + 2 * 4 * kN * 4;  // [2 halves][4 warps][kN] sums
   static constexpr int kOffTmemPtr = kOffRedL + 2 * 4 * kN * 4;
-  static constexpr int kOffCtx = kOffTmemPtr + 16;           // cached context lengths
+  static constexpr int kOffTags = kOffTmemPtr + 16;          // E4M3: K / V / end per code stage
+  static constexpr int kOffCtx = kOffTags + 32;              // cached context lengths
   static constexpr int kSmemBytes = 1024 + kOffCtx;          // + 4 bytes per cached length
   static constexpr int kCtxCap =
       (226 * 1024 - kSmemBytes) / 4 < kCtxCacheMax ? (226 * 1024 - kSmemBytes) / 4 : kCtxCacheMax;
@@ -110,6 +118,7 @@ struct Cfg {
   // in shared memory: 48 bytes per sequence + 80.
   static constexpr int kPlanCap = (226 * 1024 - kSmemBytes - 80) / 48;
   static_assert(kStages >= 2, "ring stages");
+  static_assert(!F8 || kStages <= 8, "a tag per stage in 32 bytes");
   static_assert(kCtxCap >= 0, "shared memory budget");
   static_assert(kOCol + 2 * kNPV <= kTmemCols, "tensor memory budget");
 };
@@ -385,7 +394,7 @@ struct ChunkStream {
 // chunk: column j is query a.q_first + j / G at head g * G + j % G and sees
 // the tokens before ctx - q_len + q_first + j / G + 1.
 template <typename T, int BS, int NG, int MODE>
-__global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
+__global__ void __launch_bounds__(MODE == tc::kPlainF8 ? tc::kThreadsF8 : tc::kThreads, 1) decode_tc_kernel(
     const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
     const __grid_constant__ CUtensorMap qmap, const DecodeArgs a, int64_t num_units) {
   using namespace tc;
@@ -393,13 +402,19 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
   constexpr bool MQ = MODE == kMultiQuery;
   constexpr bool VC = MODE == kContig;
   constexpr bool PK = MODE == kPacked;
+  constexpr bool F8 = MODE == kPlainF8;
   static_assert(VC ? BS == kTileTok : (BS == 16 || BS == 32), "block_size 16 or 32");
-  using L = tc::Cfg<NG>;
+  using L = tc::Cfg<NG, F8>;
   constexpr int kStages = L::kStages;
   constexpr int kPBytes = L::kPBytes;
   constexpr int kNPV = L::kNPV;
   constexpr int kBlocksPerTile = kTileTok / BS;
-  constexpr uint32_t kFmt = std::is_same<T, __half>::value ? 0u : 1u;
+  // the MMA operand type: T, except over an E4M3 cache, whose codes widen to
+  // fp16 in one instruction per pair (a bf16 q is converted to fp16 in shared
+  // memory, exactly for |q| in [2^-14, 65504]); outputs stay in T
+  using TM = typename std::conditional<F8, __half, T>::type;
+  constexpr bool kQToHalf = F8 && !std::is_same<T, __half>::value;
+  constexpr uint32_t kFmt = std::is_same<TM, __half>::value ? 0u : 1u;
   // A = K (K-major), B = Q (K-major), N = 16
   constexpr uint32_t kIdescQK = idesc_f16(kFmt, 0, 0, kN);
   // A = V^T (MN-major), B = P^T (K-major, hi and lo rows), N = kNPV
@@ -423,6 +438,11 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
   uint64_t* o_free = o_full + 2;           // [2]
   uint64_t* red_bar = o_free + 2;          // [2] chunk maxima of the 4 softmax warps
   uint64_t* lred_bar = red_bar + 2;        // [2] unit sums of the 4 softmax warps
+  // E4M3 cache: per stage, cfull completes when its codes have landed (TMA
+  // bytes); the stage's full barrier then completes on the arrival of the
+  // converter warp that widened them, instead of on TMA bytes
+  uint64_t* cfull = lred_bar + 2;          // [kStages] (E4M3)
+  int32_t* ctags = reinterpret_cast<int32_t*>(smem + L::kOffTags);
   float* red = reinterpret_cast<float*>(smem + L::kOffRed);
   float* redl = reinterpret_cast<float*>(smem + L::kOffRedL);
   uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + L::kOffTmemPtr);
@@ -447,6 +467,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], 1);
     }
+    for (int i = 0; F8 && i < kStages; ++i) mbar_init(&cfull[i], 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&q_full[i], 1);
       mbar_init(&q_empty[i], 1);
@@ -570,6 +591,26 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
     auto load_tiles = [&](const CUtensorMap* map, int32_t row, int32_t head, int32_t ntile,
                           bool values) {
       for (int32_t t = 0; t < ntile && ok; ++t, ++ctr) {
+        if constexpr (F8) {
+          // E4M3: one 2-D box {128 codes, BS rows} per block into the stage's
+          // upper half, tagged K or V for the converter warps
+          const uint32_t st = ctr % kStages;
+          if (lane == 0) {
+            ok = mbar_wait(&empty[st], ((ctr / kStages) & 1u) ^ 1u, 0x7f01u);
+            if (ok) {
+              ctags[st] = values ? 1 : 0;
+              mbar_arrive_expect_tx(&cfull[st], kCodeBytes);
+            }
+          }
+          ok = __shfl_sync(0xffffffffu, ok, 0);
+          if (!ok) break;
+          const int j = lane - t * kBlocksPerTile;
+          if (j >= 0 && j < kBlocksPerTile)
+            tma_load_2d(ring + st * kStageBytes + kCodeOffset + j * BS * 128, map, &cfull[st], 0,
+                        row, pol_kv);
+          __syncwarp();
+          continue;
+        }
         const uint32_t st = ctr % kStages;
         if (lane == 0) {
           ok = mbar_wait(&empty[st], ((ctr / kStages) & 1u) ^ 1u, 0x7200u);
@@ -696,11 +737,33 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
       cur = nxt;
     }
     if (have_pend && ok) load_tiles(&vmap, pend_row, pend_head, pend_tiles, true);
+    if constexpr (F8) {
+      // the end of the stream: the next four items (one for each converter
+      // warp, which takes every fourth) are stages tagged 2
+      for (int e = 0; e < 4 && ok; ++e) {
+        if (lane == 0) {
+          const uint32_t st = (ctr + e) % kStages;
+          ok = mbar_wait(&empty[st], (((ctr + e) / kStages) & 1u) ^ 1u, 0x7f02u);
+          if (ok) {
+            ctags[st] = 2;
+            mbar_arrive(&cfull[st]);
+          }
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+    }
     if (!ok) {
       atomicExch(&abort_flag, 1);
-      if (lane == 0)  // drain the loads that may still be in flight
-        for (uint32_t i = ctr > kStages ? ctr - kStages : 0; i < ctr; ++i)
-          mbar_wait(&full[i % kStages], (i / kStages) & 1u, 0x7300u);
+      if (lane == 0) {  // drain the loads that may still be in flight
+        if constexpr (F8) {
+          for (uint32_t i = ctr > kStages ? ctr - kStages : 0; i < ctr; ++i)
+            mbar_wait(&cfull[i % kStages], (i / kStages) & 1u, 0x7f05u);
+        } else {
+          for (uint32_t i = ctr > kStages ? ctr - kStages : 0; i < ctr; ++i)
+            mbar_wait(&full[i % kStages], (i / kStages) & 1u, 0x7300u);
+        }
+      }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -826,6 +889,29 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
         if (nxt.valid && lane < (nxt.w.ctx + BS - 1) / BS)
           nv_next = __ldg(gh.ents + 2 * (int64_t(nxt.w.e0) + lane) + 1) & 0xFF;
       }
+      if constexpr (kQToHalf) {
+        // a unit's bf16 Q tile, once landed, becomes fp16 in place (the whole warp)
+        if (cur.first()) {
+          const uint32_t qbc = ucnt & 1u;
+          if (lane == 0) ok = mbar_wait(&q_full[qbc], (ucnt >> 1) & 1u, 0x7f06u);
+          ok = __shfl_sync(0xffffffffu, ok, 0);
+          if (!ok) break;
+          uint4* qv = reinterpret_cast<uint4*>(qbuf + qbc * kQBytes);
+#pragma unroll
+          for (int i = 0; i < kQBytes / 16 / 32; ++i) {
+            uint4 v = qv[lane + 32 * i];
+            uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 f = Elem<T>::to_float2(w[e]);
+              w[e] = Elem<__half>::pack2(f.x, f.y);
+            }
+            qv[lane + 32 * i] = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+        }
+      }
       if (lane == 0) {
         if (cur.first()) {
           qb = ucnt & 1u;
@@ -857,6 +943,92 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
       }
     }
     if (ok && have_pend) pv(pend_b, pend_use, pend_tiles, pend_zero, pend_nv);
+    if (!ok) atomicExch(&abort_flag, 1);
+  } else if (F8 && warp >= 6) {
+    // ------------------------------------------------------------ E4M3 converters
+    // Converter warp w widens items w, w + 4, w + 8, ... of the stream (the
+    // producer's order); item k sits in stage k % kStages as codes in the
+    // upper half and is widened exactly to fp16 (integer and fp16 arithmetic,
+    // not the conversion instruction, whose throughput is low) over the whole stage, in the
+    // layout the TMA would have produced for a 16-bit cache: keys as two
+    // 64-dim regions of 128 rows, values per block as [half][BS rows][64]
+    // (128-byte swizzle on both). In place by one warp: rows go in ascending
+    // batches of 16, each read whole before it is written; a write of token
+    // row t lands on the codes of a row t' <= t (keys: region 1 row t is code
+    // row t; values: t' = t + (j + 1) BS - 128 for block j's second half,
+    // lower for its first), so no code is overwritten before it is read.
+    const int cw_ = warp - 6;  // 0 .. 3
+    bool ok = true;
+    for (uint32_t k = cw_;; k += 4) {
+      const uint32_t st = k % kStages;
+      if (lane == 0) ok = mbar_wait(&cfull[st], (k / kStages) & 1u, 0x7f03u);
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      const int32_t tag = ctags[st];
+      if (tag == 2) break;  // end of the stream
+      uint8_t* dst = ring + st * kStageBytes;
+      const uint8_t* src = dst + kCodeOffset;
+      const int c = lane & 7;  // 16 codes: dims 16c .. 16c + 15
+#pragma unroll 1
+      for (int r0 = 0; r0 < kTileTok; r0 += 16) {
+        uint4 wv[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int row = r0 + 4 * u + (lane >> 3);
+          wv[u] = *reinterpret_cast<const uint4*>(src + row * 128 + ((c ^ (row & 7)) << 4));
+        }
+        __syncwarp();  // the batch's codes are read before any of its writes
+        // a batch with a NaN code anywhere in the warp widens by cvt (exact
+        // NaNs); the others by the integer path, as straight-line code
+        uint32_t nanw = 0;
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          nanw |= e4m3x4_nan_bits(wv[u].x) | e4m3x4_nan_bits(wv[u].y) |
+                  e4m3x4_nan_bits(wv[u].z) | e4m3x4_nan_bits(wv[u].w);
+        uint32_t hv[4][8];
+        if (!__any_sync(0xffffffffu, nanw != 0)) {
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const uint32_t cw[4] = {wv[u].x, wv[u].y, wv[u].z, wv[u].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) e4m3x4_to_f16x2x2(cw[e], hv[u][2 * e], hv[u][2 * e + 1]);
+          }
+        } else {
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const uint32_t cw[4] = {wv[u].x, wv[u].y, wv[u].z, wv[u].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              hv[u][2 * e] = e4m3x2_to_x2<TM>(cw[e] & 0xFFFFu);
+              hv[u][2 * e + 1] = e4m3x2_to_x2<TM>(cw[e] >> 16);
+            }
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int row = r0 + 4 * u + (lane >> 3);
+          const uint32_t* h = hv[u];
+          uint8_t* base;
+          int sw;
+          if (tag == 0) {  // key row: region c / 4, row `row`
+            base = dst + (c >> 2) * kRegionBytes + row * 128;
+            sw = row & 7;
+          } else {  // value row: block row / BS, half c / 4, row row % BS
+            const int jb = row / BS, ib = row % BS;
+            base = dst + jb * BS * 256 + (c >> 2) * BS * 128 + ib * 128;
+            sw = ib & 7;
+          }
+          const int ch = 2 * (c & 3);  // 16-byte chunks ch, ch + 1 of the 128-byte row
+          *reinterpret_cast<uint4*>(base + ((ch ^ sw) << 4)) = make_uint4(h[0], h[1], h[2], h[3]);
+          *reinterpret_cast<uint4*>(base + (((ch + 1) ^ sw) << 4)) =
+              make_uint4(h[4], h[5], h[6], h[7]);
+        }
+        __syncwarp();  // this batch's writes precede the next batch's reads
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&full[st]);
+    }
     if (!ok) atomicExch(&abort_flag, 1);
   } else {
     // ------------------------------------------------------------ softmax + epilogue
@@ -939,6 +1111,8 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
       ++ucnt;
       if (!ok) return;
       const int32_t h0 = pw.g * G;
+      // E4M3: O was accumulated on codes; the value scale of the KV head applies
+      const float vsc = F8 ? __ldg(a.v_scale + pw.g) : 1.f;
       // grouped decode: a shared-prefix unit's columns are its members' heads
       const int32_t* ge = ((GRP && pw.sg >= 0) || PK) ? tc::sub_entry(gh, pw.sg) : nullptr;
       const int32_t ncol = ge ? tc::plan_at(gh, ge + 1) * G : (MQ ? a.q_count * G : G);
@@ -955,10 +1129,10 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
             row_sh = (int64_t(pw.s) * a.q_len + a.q_first + i) * a.num_q_heads + h0 + (j - i * G);
           }
           if (!GRP && !PK && pw.nparts <= 1) {
-            const float y = Lj > 0.f ? acc[j] / Lj : 0.f;
+            const float y = Lj > 0.f ? acc[j] * vsc / Lj : 0.f;
             static_cast<uint16_t*>(a.out)[row_sh * kD + r] = Elem<T>::from_float(y);
           } else {
-            a.ws_acc[(row_sh * a.ws_slots + pw.slot) * kD + r] = acc[j];
+            a.ws_acc[(row_sh * a.ws_slots + pw.slot) * kD + r] = acc[j] * vsc;
             if (r == 0) {
               a.ws_ml[(row_sh * a.ws_slots + pw.slot) * 2 + 0] = m_run[j];
               a.ws_ml[(row_sh * a.ws_slots + pw.slot) * 2 + 1] = Lj;
@@ -1029,6 +1203,9 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
       for (int j = 0; j < NG; ++j) cmax[j] = -INFINITY;
       // multi-query: column j sees the tokens before lim0 + j / G
       const int32_t lim0 = MQ ? cur.w.ctx - a.q_len + a.q_first + 1 : 0;
+      // E4M3: the scores were taken on codes; the key scale of the KV head joins
+      // the softmax scale
+      const float sc_log2 = F8 ? a.scale_log2 * __ldg(a.k_scale + cur.w.g) : a.scale_log2;
 #pragma unroll
       for (int t = 0; t < kChunkTiles; ++t) {
         const int32_t tok = ctok0 + t * kTileTok + r;
@@ -1036,7 +1213,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
 #pragma unroll
         for (int j = 0; j < NG; ++j) {
           const bool vis = valid && (!MQ || tok < lim0 + col_q[j]) && (!PK || ((pm[t] >> j) & 1u));
-          sv[t][j] = vis ? sv[t][j] * a.scale_log2 : -INFINITY;
+          sv[t][j] = vis ? sv[t][j] * sc_log2 : -INFINITY;
           cmax[j] = fmaxf(cmax[j], sv[t][j]);
         }
       }
@@ -1072,10 +1249,10 @@ __global__ void __launch_bounds__(tc::kThreads, 1) decode_tc_kernel(
               const int j = j0 + 2 * i;
               const float p0 = sv[t][j] == -INFINITY ? 0.f : ex2_ftz(sv[t][j] - cmax[j]);
               const float p1 = sv[t][j + 1] == -INFINITY ? 0.f : ex2_ftz(sv[t][j + 1] - cmax[j + 1]);
-              hw[i] = Elem<T>::pack2(p0, p1);
-              const float2 hf = Elem<T>::to_float2(hw[i]);
-              lw[i] = Elem<T>::pack2(p0 - hf.x, p1 - hf.y);
-              const float2 lf = Elem<T>::to_float2(lw[i]);
+              hw[i] = Elem<TM>::pack2(p0, p1);
+              const float2 hf = Elem<TM>::to_float2(hw[i]);
+              lw[i] = Elem<TM>::pack2(p0 - hf.x, p1 - hf.y);
+              const float2 lf = Elem<TM>::to_float2(lw[i]);
               psum[j] += hf.x + lf.x;
               psum[j + 1] += hf.y + lf.y;
             }

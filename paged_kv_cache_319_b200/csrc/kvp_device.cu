@@ -230,6 +230,12 @@ int make_map_prefill_q(CUtensorMap* map, const void* base, int32_t dtype, uint32
   return KVP_OK;
 }
 
+// E4M3 decode with at least this many query heads per KV head runs on the
+// tensor cores (E4M3 tiles widened in shared memory); fewer, on CUDA cores.
+#ifndef KVP_FP8_TC_MIN_G
+#define KVP_FP8_TC_MIN_G 2
+#endif
+
 // Prefill chunks with at least this many query rows (q_len x query heads per
 // KV head, a power of two) run on the prompt-shaped kernel (128 query rows per
 // tensor-core tile); shorter ones on the decode-shaped kernel, 16 columns per
@@ -321,15 +327,16 @@ template <typename T, int BS, int NG, int MODE = kvp::dev::tc::kPlain>
 int launch_tc(const CUtensorMap& km, const CUtensorMap& vm, const CUtensorMap& qm,
               const kvp::dev::DecodeArgs& a, cudaStream_t st) {
   auto k = kvp::dev::decode_tc_kernel<T, BS, NG, MODE>;
+  constexpr bool f8 = MODE == kvp::dev::tc::kPlainF8;
   // context lengths of small batches are cached in shared memory
-  using Cfg = kvp::dev::tc::Cfg<NG>;
+  using Cfg = kvp::dev::tc::Cfg<NG, f8>;
   const int ctx_bytes = a.num_seqs <= Cfg::kCtxCap ? 4 * a.num_seqs : 0;
   const int smem = Cfg::kSmemBytes + ctx_bytes;
   cudaError_t e = ensure_smem(k, Cfg::kSmemBytes + 4 * Cfg::kCtxCap);
   if (e != cudaSuccess) return cuda_fail(e, "decode (tensor cores): smem attribute");
   const int64_t units = int64_t(a.num_seqs) * a.num_kv_heads * a.pmax;
   const int grid = int(units < sm_count() ? units : sm_count());
-  k<<<grid, kvp::dev::tc::kThreads, smem, st>>>(km, vm, qm, a, units);
+  k<<<grid, f8 ? kvp::dev::tc::kThreadsF8 : kvp::dev::tc::kThreads, smem, st>>>(km, vm, qm, a, units);
   e = cudaGetLastError();
   return e == cudaSuccess ? KVP_OK : cuda_fail(e, "decode (tensor cores): launch");
 }
@@ -524,6 +531,22 @@ int tc_mq_dispatch(int bs, int ng, const CUtensorMap& km, const CUtensorMap& vm,
                                : launch_tc_mq<T, 16, 16>(km, vm, qm, a, st);
   return ng == 8 ? launch_tc_mq<T, 32, 8>(km, vm, qm, a, st)
                  : launch_tc_mq<T, 32, 16>(km, vm, qm, a, st);
+}
+
+// E4M3 cache, grouped-query heads: the tensor-core decode with converter warps.
+template <typename T>
+int tc_fp8_dispatch(int bs, int G, const CUtensorMap& km, const CUtensorMap& vm,
+                    const CUtensorMap& qm, const kvp::dev::DecodeArgs& a, cudaStream_t st) {
+  constexpr int M = kvp::dev::tc::kPlainF8;
+  const int ng = G <= 4 ? 4 : (G <= 8 ? 8 : 16);
+  if (bs == 16) {
+    if (ng == 4) return launch_tc<T, 16, 4, M>(km, vm, qm, a, st);
+    if (ng == 8) return launch_tc<T, 16, 8, M>(km, vm, qm, a, st);
+    return launch_tc<T, 16, 16, M>(km, vm, qm, a, st);
+  }
+  if (ng == 4) return launch_tc<T, 32, 4, M>(km, vm, qm, a, st);
+  if (ng == 8) return launch_tc<T, 32, 8, M>(km, vm, qm, a, st);
+  return launch_tc<T, 32, 16, M>(km, vm, qm, a, st);
 }
 
 template <typename T>
@@ -1064,8 +1087,18 @@ int paged_attention_decode_fp8(const void* q, const void* k_cache, const void* v
   if (!rc) rc = make_map_u8(&vm, v_cache, rows, block_size);
   if (rc) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  rc = dtype == KVP_F16 ? simt_fp8_by_bs<__half>(block_size, km, vm, a, st)
-                        : simt_fp8_by_bs<__nv_bfloat16>(block_size, km, vm, a, st);
+  const int G = num_q_heads / num_kv_heads;
+  if (G >= KVP_FP8_TC_MIN_G && G <= 16 && (block_size == 16 || block_size == 32)) {
+    // grouped-query heads: one widened tile serves the group's heads on the tensor cores
+    CUtensorMap qm;
+    rc = make_map(&qm, q, dtype, uint64_t(num_seqs) * num_q_heads, head_dim, kvp::dev::tc::kN);
+    if (rc) return rc;
+    rc = dtype == KVP_F16 ? tc_fp8_dispatch<__half>(block_size, G, km, vm, qm, a, st)
+                          : tc_fp8_dispatch<__nv_bfloat16>(block_size, G, km, vm, qm, a, st);
+  } else {
+    rc = dtype == KVP_F16 ? simt_fp8_by_bs<__half>(block_size, km, vm, a, st)
+                          : simt_fp8_by_bs<__nv_bfloat16>(block_size, km, vm, a, st);
+  }
   if (rc || pmax <= 1) return rc;
   return dtype == KVP_F16 ? launch_reduce<__half, 128>(a, st) : launch_reduce<__nv_bfloat16, 128>(a, st);
 }

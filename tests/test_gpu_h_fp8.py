@@ -7,8 +7,10 @@ bf16 inputs. paged_attention_decode_fp8 is held to the decode tolerance against
 fp64 attention over the dequantised cache, on caches of uniform codes (every
 magnitude from 2^-9 to 448) and on caches the oracle quantised from N(0, 1)
 data: block sizes 8, 16 and 32, split and unsplit partitions, contexts of 0, 1,
-a block and one past it, grouped-query heads, and the full OPT-13B batch
-(64 sequences, 40 heads, contexts U[1, 2048]) checked on sampled sequences.
+a block and one past it, grouped-query heads (G = 2 to 16, on the tensor
+cores), NaN codes in the slots past the contexts, the full OPT-13B batch (64
+sequences, 40 heads, contexts U[1, 2048]) and the long-context GQA batch (32
+sequences, 32 / 8 heads, contexts U[16384, 32768]), both on every row.
 copy_blocks copies E4M3 blocks byte for byte.
 """
 
@@ -105,6 +107,13 @@ CASES = [
     (8, 8, 32, [33, 1030, 2048], "f16", 256, "quantised"),
     (16, 4, 16, [0, 100, 900], "bf16", 512, "quantised"),   # G = 4, a context of 0
     (40, 40, 16, [2048, 1, 517], "f16", 512, "quantised"),  # OPT-13B heads
+    # grouped-query heads run on the tensor cores (codes widened in shared memory)
+    (16, 8, 16, [1, 2, 511, 512, 513, 3000], "f16", 512, "quantised"),  # G = 2
+    (32, 8, 32, [0, 31, 32, 33, 1025, 4000], "bf16", 512, "uniform"),   # G = 4, bs 32
+    (32, 4, 16, [7, 700, 2500], "f16", 0, "quantised"),                 # G = 8, unsplit
+    (32, 2, 16, [200, 1300], "bf16", 256, "quantised"),                 # G = 16
+    (32, 8, 16, [100, 900, 37], "f16", 512, "nan_tail"),                # NaN codes past the contexts
+    (32, 8, 32, [5, 1000], "bf16", 0, "nan_tail"),
 ]
 
 
@@ -116,6 +125,21 @@ def test_decode_fp8_matches_oracle(Hq, Hkv, bs, lens, dtype, partition, codes):
     if codes == "uniform":
         kc = random_e4m3_codes([seed, 1], (NB, Hkv, bs, D))
         vc = random_e4m3_codes([seed, 2], (NB, Hkv, bs, D))
+        ks = np.float32(np.linspace(1 / 448, 3 / 448, Hkv))
+        vs = np.float32(np.linspace(0.5 / 448, 2 / 448, Hkv))
+    elif codes == "nan_tail":
+        # finite codes where the sequences have tokens; the NaN code (0x7F) in
+        # the rest of each last block and in the spare blocks: p is 0 there, and
+        # 0 times NaN must not reach the output
+        kc = np.full((NB, Hkv, bs, D), 0x7F, np.uint8)
+        vc = np.full((NB, Hkv, bs, D), 0x7F, np.uint8)
+        kr = random_e4m3_codes([seed, 1], (NB, Hkv, bs, D))
+        vr = random_e4m3_codes([seed, 2], (NB, Hkv, bs, D))
+        for si, L in enumerate(lens):
+            for j in range(L):
+                b = t[si, j // bs]
+                kc[b, :, j % bs] = kr[b, :, j % bs]
+                vc[b, :, j % bs] = vr[b, :, j % bs]
         ks = np.float32(np.linspace(1 / 448, 3 / 448, Hkv))
         vs = np.float32(np.linspace(0.5 / 448, 2 / 448, Hkv))
     else:
@@ -132,9 +156,9 @@ def test_decode_fp8_matches_oracle(Hq, Hkv, bs, lens, dtype, partition, codes):
     check_close(got, ref, dtype, allow_ulp=(dtype == "bf16"))
 
 
-def test_decode_fp8_opt13b_batch_sampled():
+def test_decode_fp8_opt13b_batch_every_row():
     """The bench's workload: 64 sequences, 40 heads x 128, contexts U[1, 2048],
-    block size 16, partitions of 512; eight sequences checked against the oracle."""
+    block size 16, partitions of 512; every row checked against the oracle."""
     wl = workloads.opt13b()
     lens = np.asarray(wl.info["context_lens"], np.int32)
     bs, Hkv, D = 16, 40, 128
@@ -145,11 +169,26 @@ def test_decode_fp8_opt13b_batch_sampled():
     vs = np.float32(np.linspace(1 / 448, 4 / 448, Hkv))
     q = workloads.normal_bits([77, 3], (len(lens), Hkv, D), "f16")
     got = _run(q, kc, vc, ks, vs, t, lens.tolist(), "f16", 1 / math.sqrt(D), 512)
-    rows = np.random.default_rng(78).choice(len(lens), 8, replace=False)
-    rows = np.union1d(rows, [int(np.argmax(lens)), int(np.argmin(lens))])
-    ref = fp8.paged_decode(to_f64(q[rows], "f16"), kc, vc, t[rows], lens[rows], 1 / math.sqrt(D), bs,
-                           ks, vs)
-    check_close(got[rows], ref, "f16")
+    ref = fp8.paged_decode(to_f64(q, "f16"), kc, vc, t, lens, 1 / math.sqrt(D), bs, ks, vs)
+    check_close(got, ref, "f16")
+
+
+def test_decode_fp8_gqa_long_every_row():
+    """Long-context GQA over an E4M3 cache: 32 sequences, 32 query / 8 KV heads
+    x 128, block size 16, contexts U[16384, 32768], partitions of 512, bf16
+    queries; every row checked against the oracle."""
+    wl = workloads.gqa_long(16)
+    lens = np.asarray(wl.info["context_lens"], np.int32)
+    bs, Hq, Hkv, D = 16, 32, 8, 128
+    t, NB = _tables(4004, lens.tolist(), bs, extra=16)
+    kc = random_e4m3_codes([4004, 1], (NB, Hkv, bs, D))
+    vc = random_e4m3_codes([4004, 2], (NB, Hkv, bs, D))
+    ks = np.float32(np.linspace(1 / 448, 2 / 448, Hkv))
+    vs = np.float32(np.linspace(1 / 448, 4 / 448, Hkv))
+    q = workloads.normal_bits([4004, 3], (len(lens), Hq, D), "bf16")
+    got = _run(q, kc, vc, ks, vs, t, lens.tolist(), "bf16", 1 / math.sqrt(D), 512)
+    ref = fp8.paged_decode(to_f64(q, "bf16"), kc, vc, t, lens, 1 / math.sqrt(D), bs, ks, vs)
+    check_close(got, ref, "bf16", allow_ulp=True)
 
 
 def test_copy_blocks_fp8_byte_for_byte():
