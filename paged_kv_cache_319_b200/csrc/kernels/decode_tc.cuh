@@ -1018,10 +1018,17 @@ __global__ void __launch_bounds__(MODE == tc::kPlainF8 ? tc::kThreadsF8 : tc::kT
             base = dst + jb * BS * 256 + (c >> 2) * BS * 128 + ib * 128;
             sw = ib & 7;
           }
-          const int ch = 2 * (c & 3);  // 16-byte chunks ch, ch + 1 of the 128-byte row
-          *reinterpret_cast<uint4*>(base + ((ch ^ sw) << 4)) = make_uint4(h[0], h[1], h[2], h[3]);
-          *reinterpret_cast<uint4*>(base + (((ch + 1) ^ sw) << 4)) =
-              make_uint4(h[4], h[5], h[6], h[7]);
+          // 16-byte chunks ch, ch + 1 of the 128-byte row. A 16-byte store is
+          // served eight lanes at a time, and lanes c and c + 4 (same row, other
+          // region) would meet at the same bank positions: lanes of the second
+          // region store chunk ch + 1 first, so each group of eight covers all 32
+          // banks once.
+          const int ch = 2 * (c & 3);
+          const bool sec = c >= 4;
+          const uint4 d0 = make_uint4(h[0], h[1], h[2], h[3]);
+          const uint4 d1 = make_uint4(h[4], h[5], h[6], h[7]);
+          *reinterpret_cast<uint4*>(base + (((ch + (sec ? 1 : 0)) ^ sw) << 4)) = sec ? d1 : d0;
+          *reinterpret_cast<uint4*>(base + (((ch + (sec ? 0 : 1)) ^ sw) << 4)) = sec ? d0 : d1;
         }
         __syncwarp();  // this batch's writes precede the next batch's reads
       }
