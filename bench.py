@@ -65,6 +65,17 @@ def peaks():
         return 6650.0, "fallback"
 
 
+def tensor_peaks():
+    """Dense bf16 (= fp16) tensor throughput, TFLOP/s: (sustained, burst, source)."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["bf16_tflops_sustained"]), float(d["bf16_tflops"]), "measured"
+    except Exception:
+        return 1400.0, 1590.0, "fallback"
+
+
 # DRAM traffic (read + write) of one launch of each decode kernel, as a multiple of
 # its algorithmic bytes, from the ncu captures summarised in profiles/; valid only
 # while the kernel source hashes to the value it had when captured.
@@ -331,7 +342,7 @@ def run_ours(args, world, rank, local):
     # Replicas: none grows by more than ~64 tokens over warm-up, timing and the
     # end-to-end pass; each starts short by its warm-up steps plus half its
     # timed steps, so the timed lengths are centred on the configured ones.
-    K_e2e = max(1, min(K, 64))
+    K_e2e = max(1, min(K, 64)) + max(1, min(K, 32))  # graph-replay pass + eager pass
     pool_bytes = 2 * wl.num_blocks * g.num_kv_heads * g.block_size * g.head_dim * g.elem_bytes
     free_b = torch.cuda.mem_get_info(device)[0]
     r_cap = max(1, int(0.6 * free_b // pool_bytes))
@@ -772,7 +783,7 @@ def _summary(rec):
     """The parts of a workload's line that the default line carries."""
     keep = ("value", "unit", "steps", "warmup", "ms_per_step", "dtype", "config", "roofline",
             "clocks", "seq_tokens_per_s", "query_tokens_per_s", "attention_tflops",
-            "f16_cache_same_batch", "rows", "call_us_median", "call_us_mean", "calls", "timed",
+            "f16_cache_same_batch", "rows", "call_us_median", "call_us_mean", "calls", "timed", "hbm_view",
             "workload", "name", "paged_call_us", "contiguous_call_us", "translation_cost",
             "outputs_bit_identical", "outputs_max_abs_diff", "memory", "host")
     return {k: v for k, v in rec.items() if k in keep}
@@ -974,6 +985,26 @@ def run_e2e(args, wl, reps, device, seed_rank, MB, max_ctx_total, part, ws, worl
     el = time.perf_counter() - t
     el = dist_max(el, world)
     total_bytes = dist_sum(float(total_bytes), world)
+    # The same steps eagerly: every step calls the library (argument checks, tensor-map
+    # encoding, launches) through its binding, as a caller without graphs would.
+    K_eager = max(1, min(args.steps, 32))
+    eager_bytes = 0
+    barrier(world)
+    torch.cuda.synchronize(device)
+    t = time.perf_counter()
+    copies = book(reps[K % R], metas[K % 2])
+    for i in range(K, K + K_eager):
+        rep, m = reps[i % R], metas[i % 2]
+        if copies:
+            kvp.copy_blocks(rep.k, rep.v, torch.tensor(copies, dtype=torch.int32).to(device))
+        device_part(rep, m)
+        step_bytes = algorithmic_bytes(m.len_h.numpy(), g)
+        if i + 1 < K + K_eager:
+            copies = book(reps[(i + 1) % R], metas[(i + 1) % 2])
+        stream.synchronize()
+        eager_bytes += step_bytes
+    el_eager = dist_max(time.perf_counter() - t, world)
+    eager_bytes = dist_sum(float(eager_bytes), world)
     # Where a step's time goes (not part of the timed loop): host bookkeeping,
     # and each piece of the device work timed alone with CUDA events.
     brk = {}
@@ -1019,7 +1050,12 @@ def run_e2e(args, wl, reps, device, seed_rank, MB, max_ctx_total, part, ws, worl
             "how": "per step: one CUDA graph replay (inputs from pinned host memory up, scatter, "
                    "decode, result down) and a synchronize; the next step's host bookkeeping "
                    "runs while the graph runs" + (f"; {eager} steps eager" if eager else ""),
-            "breakdown": brk}
+            "breakdown": brk,
+            "eager": {"value": round(eager_bytes / el_eager / 1e9, 2), "unit": UNIT,
+                      "steps": K_eager, "step_us": round(el_eager / K_eager * 1e6, 1),
+                      "how": "the same steps without graphs: every step calls the C ABI through "
+                             "the binding (copies up, reshape_and_cache, paged_attention_decode, "
+                             "copy down) and synchronizes"}}
 
 
 # ---------------------------------------------------------------- CPU oracle
@@ -1184,6 +1220,9 @@ def prefill_record(args):
         part, desc = PREFILL_PARTITION, f"{wl.description}; a chunk of the last {T} tokens per sequence"
     if args.partition:
         part = args.partition
+    if getattr(args, "num_seqs", None):  # a smaller case of the same workload (profiling)
+        lens = lens[:args.num_seqs]
+        desc += f"; first {len(lens)} sequences"
     S, Hq, Hkv, D, bs = len(lens), g.num_q_heads, g.num_kv_heads, g.head_dim, g.block_size
     rng = np.random.default_rng(3001)
     need = -(-lens // bs)
@@ -1228,11 +1267,36 @@ def prefill_record(args):
     kv = float(lens.sum()) * Hkv * D * g.elem_bytes * 2
     alg = kv + S * T * Hq * D * g.elem_bytes * 2 + 4 * float(need.sum()) + 4 * S
     G = Hq // Hkv
-    launches = -(-T // max(1, 16 // G)) if T > 1 else 1
+    # the library's routing: chunks of at least 64 query rows (T x G, G a power of two) run on
+    # the prompt-shaped kernel in one launch, shorter ones 16 columns per launch
+    prompt_tiles = T > 1 and (G & (G - 1)) == 0 and T * G >= 64
+    launches = 1 if prompt_tiles else (-(-T // max(1, 16 // G)) if T > 1 else 1)
     vis = np.clip(lens[:, None] - T + np.arange(T)[None, :] + 1, 0, None)  # visible tokens per query
     flops = 4.0 * float(vis.sum()) * D * Hq
     peak, peak_kind = peaks()
     achieved = alg / (ms * 1e-3) / 1e9
+    tflops = flops / (ms * 1e-3) / 1e12
+    split = part < int(lens.max())
+    kname = ("paged_attention_prefill: prefill_tc (128 query rows x 128 keys per tcgen05 tile)"
+             if prompt_tiles else "paged_attention_prefill: decode_tc (multi-query)") + \
+        (" + decode_reduce_kernel" if split else "")
+    hbm_view = {"kernel": kname, "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
+                "peak_source": peak_kind, "unit": "GB/s", "frac": round(achieved / peak, 4),
+                "algorithmic_bytes_per_launch": int(alg),
+                "note": f"algorithmic bytes count the keys and values once per call; "
+                        f"each of the call's {launches} launch(es) reads the tokens that its "
+                        f"queries see",
+                "avg_launch_us": round(ms * 1e3, 2)}
+    if prompt_tiles:
+        sus, burst, tkind = tensor_peaks()
+        roofline = {"kernel": kname, "bound": "tensor", "achieved": round(tflops, 1), "peak": sus,
+                    "peak_source": tkind + " (bf16_tflops_sustained; fp16 has the same dense rate)",
+                    "unit": "TFLOP/s", "frac": round(tflops / sus, 4),
+                    "frac_of_burst": round(tflops / burst, 4),
+                    "flops_per_launch": flops, "flops": "4 * head_dim * Hq per visible (query, key) pair",
+                    "avg_launch_us": round(ms * 1e3, 2), "traffic": None}
+    else:
+        roofline = hbm_view
     res = {
         "metric": METRIC, "value": round(achieved, 2), "unit": UNIT, "n_gpus": 1,
         "steps": len(pairs), "warmup": max(3, args.warmup), "ms_per_step": round(ms, 4),
@@ -1243,15 +1307,9 @@ def prefill_record(args):
                    "timed": f"paged_attention_prefill (median of {len(pairs)} calls, L2 "
                             "flushed before each)"},
         "query_tokens_per_s": round(S * T / (ms * 1e-3), 1),
-        "attention_tflops": round(flops / (ms * 1e-3) / 1e12, 2),
-        "roofline": {"kernel": "paged_attention_prefill: decode_tc (multi-query) + decode_reduce_kernel",
-                     "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
-                     "peak_source": peak_kind, "unit": "GB/s", "frac": round(achieved / peak, 4),
-                     "algorithmic_bytes_per_launch": int(alg),
-                     "note": f"algorithmic bytes count the keys and values once per call; "
-                             f"each of the call's {launches} launch(es) reads the tokens that its "
-                             f"queries see",
-                     "avg_launch_us": round(ms * 1e3, 2)},
+        "attention_tflops": round(tflops, 2),
+        "roofline": roofline,
+        "hbm_view": hbm_view,
         "clocks": clk.summary(),
     }
     return res
@@ -1276,7 +1334,10 @@ def fp8_record(args):
     wl = workloads.by_name(base)
     g = wl.geometry
     qdt = torch.float16 if g.dtype == "f16" else torch.bfloat16
+    nsub = getattr(args, "num_seqs", None)  # a smaller case of the same workload (profiling)
     lens = np.asarray(wl.info["context_lens"], np.int64)
+    if nsub:
+        lens = lens[:nsub]
     S, Hq, Hkv, D, bs, part = len(lens), g.num_q_heads, g.num_kv_heads, g.head_dim, g.block_size, 512
     rng = np.random.default_rng(4001)
     need = -(-lens // bs)
