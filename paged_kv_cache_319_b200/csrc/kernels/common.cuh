@@ -332,28 +332,6 @@ __device__ __forceinline__ uint32_t e4m3x2_to_x2(uint32_t two_codes) {
     return *reinterpret_cast<const uint32_t*>(&b);
   }
 }
-// Four E4M3 codes (the bytes of w, lowest first) -> two fp16x2 words (codes
-// 0, 1 and codes 2, 3), exactly, on the integer and fp16 pipes. Byte b becomes
-// the fp16 bit pattern with b's sign at bit 15 and its seven magnitude bits at
-// bits 7..13, which read as fp16 is the code's value times 2^-8 (E4M3's
-// subnormals land on fp16 subnormals); one multiply by 2^8 is then exact. The
-// NaN codes (0x7F, 0xFF) would read as +-480 that way: callers test words
-// with e4m3x4_nan_bits first and convert those with the cvt instruction.
-__device__ __forceinline__ uint32_t e4m3x4_nan_bits(uint32_t w) {
-  return ((w & 0x7F7F7F7Fu) + 0x01010101u) & 0x80808080u;  // bit 7 of a byte: low seven set
-}
-__device__ __forceinline__ void e4m3x4_to_f16x2x2(uint32_t w, uint32_t& lo, uint32_t& hi) {
-  const uint32_t t0 = __byte_perm(w, 0u, 0x1404u);  // b1 << 24 | b0 << 8
-  const uint32_t t1 = __byte_perm(w, 0u, 0x3424u);  // b3 << 24 | b2 << 8
-  const uint32_t f0 = (t0 & 0x80008000u) | ((t0 >> 1) & 0x3F803F80u);
-  const uint32_t f1 = (t1 & 0x80008000u) | ((t1 >> 1) & 0x3F803F80u);
-  const __half2 k256 = __halves2half2(__ushort_as_half(0x5C00), __ushort_as_half(0x5C00));
-  const __half2 h0 = __hmul2(*reinterpret_cast<const __half2*>(&f0), k256);
-  const __half2 h1 = __hmul2(*reinterpret_cast<const __half2*>(&f1), k256);
-  lo = *reinterpret_cast<const uint32_t*>(&h0);
-  hi = *reinterpret_cast<const uint32_t*>(&h1);
-}
-
 // Two fp32 values -> their codes: round to nearest even, saturated to +-448
 // (infinities too), NaN to NaN; lo goes to the lower byte.
 __device__ __forceinline__ uint32_t float2_to_e4m3x2(float lo, float hi) {

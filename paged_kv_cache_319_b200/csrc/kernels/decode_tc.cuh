@@ -72,7 +72,6 @@ constexpr int kOCol = 128;                           // O buffers: [128, 128 + 2
 constexpr int kThreads = 192;
 constexpr int kThreadsF8 = 320;          // + four converter warps (E4M3 cache)
 constexpr int kCodeBytes = 128 * 128;    // 16 KiB: E4M3 codes of one 128-token tile
-constexpr int kCodeOffset = 16 * 1024;   // where they land in a 32 KiB stage
 constexpr int kSoftmaxThreads = 128;
 // Batches of up to Cfg<NG>::kCtxCap sequences (at most kCtxCacheMax) keep their
 // context lengths in shared memory, so no warp role waits on a global load when
@@ -95,16 +94,19 @@ struct Cfg {
 #define KVP_TC_STAGES 5
 #endif
   // groups of 16 need a P^T twice as wide, which costs one stage. An E4M3
-  // cache lands its codes in the upper half of a stage (kCodeOffset), where the
-  // converter warps widen them over the whole stage.
-  static constexpr int kStages = NG <= 8 ? KVP_TC_STAGES : KVP_TC_STAGES - 1;
+  // cache keeps its loads in flight as codes (4 stages of 16 KiB, 3 for groups
+  // of 16) besides 3 widened stages (measured on the long-context GQA batch:
+  // 3 + 4 and 4 + 3 626 us, 2 + 6 677 us, 4 + 2 725 us, 5 + 1 1261 us).
+  static constexpr int kStages = F8 ? 3 : (NG <= 8 ? KVP_TC_STAGES : KVP_TC_STAGES - 1);
+  static constexpr int kCodeStages = F8 ? (NG <= 8 ? 4 : 3) : 0;
   static constexpr int kPBytes = kChunkTok * kNPV * 2;
   static constexpr int kPSbo = kChunkTok * 16;          // bytes between 8-column groups of P^T
   static constexpr int kOffRing = 0;
-  static constexpr int kOffQ = kOffRing + kStages * kStageBytes;
+  static constexpr int kOffCodes = kOffRing + kStages * kStageBytes;
+  static constexpr int kOffQ = kOffCodes + kCodeStages * kCodeBytes;
   static constexpr int kOffP = kOffQ + 2 * kQBytes;
   static constexpr int kOffBar = kOffP + 2 * kPBytes;
-  static constexpr int kNumBars = 2 * kStages + 2 * 10 + (F8 ? kStages : 0);
+  static constexpr int kNumBars = 2 * kStages + 2 * 10 + 2 * kCodeStages;
   static constexpr int kOffRed = kOffBar + kNumBars * 8;     // [2 halves][4 warps][kN] maxima
   static constexpr int kOffRedL = kOffRed + 2 * 4 * kN * 4;  // [2 halves][4 warps][kN] sums
   static constexpr int kOffTmemPtr = kOffRedL + 2 * 4 * kN * 4;
@@ -118,7 +120,7 @@ struct Cfg {
   // in shared memory: 48 bytes per sequence + 80.
   static constexpr int kPlanCap = (226 * 1024 - kSmemBytes - 80) / 48;
   static_assert(kStages >= 2, "ring stages");
-  static_assert(!F8 || kStages <= 8, "a tag per stage in 32 bytes");
+  static_assert(kCodeStages <= 8, "a tag per code stage in 32 bytes");
   static_assert(kCtxCap >= 0, "shared memory budget");
   static_assert(kOCol + 2 * kNPV <= kTmemCols, "tensor memory budget");
 };
@@ -438,10 +440,12 @@ __global__ void __launch_bounds__(MODE == tc::kPlainF8 ? tc::kThreadsF8 : tc::kT
   uint64_t* o_free = o_full + 2;           // [2]
   uint64_t* red_bar = o_free + 2;          // [2] chunk maxima of the 4 softmax warps
   uint64_t* lred_bar = red_bar + 2;        // [2] unit sums of the 4 softmax warps
-  // E4M3 cache: per stage, cfull completes when its codes have landed (TMA
-  // bytes); the stage's full barrier then completes on the arrival of the
-  // converter warp that widened them, instead of on TMA bytes
-  uint64_t* cfull = lred_bar + 2;          // [kStages] (E4M3)
+  // E4M3 cache: code stages filled by TMA (cfull) and handed back by the four
+  // converter warps once read (cempty); a widened ring stage's full barrier
+  // counts the converter warps' writes instead of TMA bytes
+  uint64_t* cfull = lred_bar + 2;               // [kCodeStages]
+  uint64_t* cempty = cfull + L::kCodeStages;    // [kCodeStages]
+  uint8_t* codes = smem + L::kOffCodes;
   int32_t* ctags = reinterpret_cast<int32_t*>(smem + L::kOffTags);
   float* red = reinterpret_cast<float*>(smem + L::kOffRed);
   float* redl = reinterpret_cast<float*>(smem + L::kOffRedL);
@@ -464,10 +468,13 @@ __global__ void __launch_bounds__(MODE == tc::kPlainF8 ? tc::kThreadsF8 : tc::kT
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStages; ++i) {
-      mbar_init(&full[i], 1);
+      mbar_init(&full[i], F8 ? 4 : 1);
       mbar_init(&empty[i], 1);
     }
-    for (int i = 0; F8 && i < kStages; ++i) mbar_init(&cfull[i], 1);
+    for (int i = 0; i < L::kCodeStages; ++i) {
+      mbar_init(&cfull[i], 1);
+      mbar_init(&cempty[i], 4);
+    }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&q_full[i], 1);
       mbar_init(&q_empty[i], 1);
@@ -592,22 +599,21 @@ __global__ void __launch_bounds__(MODE == tc::kPlainF8 ? tc::kThreadsF8 : tc::kT
                           bool values) {
       for (int32_t t = 0; t < ntile && ok; ++t, ++ctr) {
         if constexpr (F8) {
-          // E4M3: one 2-D box {128 codes, BS rows} per block into the stage's
-          // upper half, tagged K or V for the converter warps
-          const uint32_t st = ctr % kStages;
+          // E4M3: one 2-D box {128 codes, BS rows} per block into a code stage,
+          // tagged K or V for the converter warps
+          const uint32_t cs = ctr % L::kCodeStages;
           if (lane == 0) {
-            ok = mbar_wait(&empty[st], ((ctr / kStages) & 1u) ^ 1u, 0x7f01u);
+            ok = mbar_wait(&cempty[cs], ((ctr / L::kCodeStages) & 1u) ^ 1u, 0x7f01u);
             if (ok) {
-              ctags[st] = values ? 1 : 0;
-              mbar_arrive_expect_tx(&cfull[st], kCodeBytes);
+              ctags[cs] = values ? 1 : 0;
+              mbar_arrive_expect_tx(&cfull[cs], kCodeBytes);
             }
           }
           ok = __shfl_sync(0xffffffffu, ok, 0);
           if (!ok) break;
           const int j = lane - t * kBlocksPerTile;
           if (j >= 0 && j < kBlocksPerTile)
-            tma_load_2d(ring + st * kStageBytes + kCodeOffset + j * BS * 128, map, &cfull[st], 0,
-                        row, pol_kv);
+            tma_load_2d(codes + cs * kCodeBytes + j * BS * 128, map, &cfull[cs], 0, row, pol_kv);
           __syncwarp();
           continue;
         }
@@ -738,27 +744,24 @@ __global__ void __launch_bounds__(MODE == tc::kPlainF8 ? tc::kThreadsF8 : tc::kT
     }
     if (have_pend && ok) load_tiles(&vmap, pend_row, pend_head, pend_tiles, true);
     if constexpr (F8) {
-      // the end of the stream: the next four items (one for each converter
-      // warp, which takes every fourth) are stages tagged 2
-      for (int e = 0; e < 4 && ok; ++e) {
-        if (lane == 0) {
-          const uint32_t st = (ctr + e) % kStages;
-          ok = mbar_wait(&empty[st], (((ctr + e) / kStages) & 1u) ^ 1u, 0x7f02u);
-          if (ok) {
-            ctags[st] = 2;
-            mbar_arrive(&cfull[st]);
-          }
+      // the end of the stream for the converter warps: a code stage tagged 2
+      if (ok && lane == 0) {
+        const uint32_t cs = ctr % L::kCodeStages;
+        ok = mbar_wait(&cempty[cs], ((ctr / L::kCodeStages) & 1u) ^ 1u, 0x7f02u);
+        if (ok) {
+          ctags[cs] = 2;
+          mbar_arrive(&cfull[cs]);
         }
-        ok = __shfl_sync(0xffffffffu, ok, 0);
       }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
       ok = __shfl_sync(0xffffffffu, ok, 0);
     }
     if (!ok) {
       atomicExch(&abort_flag, 1);
       if (lane == 0) {  // drain the loads that may still be in flight
         if constexpr (F8) {
-          for (uint32_t i = ctr > kStages ? ctr - kStages : 0; i < ctr; ++i)
-            mbar_wait(&cfull[i % kStages], (i / kStages) & 1u, 0x7f05u);
+          for (uint32_t i = ctr > L::kCodeStages ? ctr - L::kCodeStages : 0; i < ctr; ++i)
+            mbar_wait(&cfull[i % L::kCodeStages], (i / L::kCodeStages) & 1u, 0x7f05u);
         } else {
           for (uint32_t i = ctr > kStages ? ctr - kStages : 0; i < ctr; ++i)
             mbar_wait(&full[i % kStages], (i / kStages) & 1u, 0x7300u);
@@ -946,91 +949,70 @@ __global__ void __launch_bounds__(MODE == tc::kPlainF8 ? tc::kThreadsF8 : tc::kT
     if (!ok) atomicExch(&abort_flag, 1);
   } else if (F8 && warp >= 6) {
     // ------------------------------------------------------------ E4M3 converters
-    // Converter warp w widens items w, w + 4, w + 8, ... of the stream (the
-    // producer's order); item k sits in stage k % kStages as codes in the
-    // upper half and is widened exactly to fp16 (integer and fp16 arithmetic,
-    // not the conversion instruction, whose throughput is low) over the whole stage, in the
-    // layout the TMA would have produced for a 16-bit cache: keys as two
-    // 64-dim regions of 128 rows, values per block as [half][BS rows][64]
-    // (128-byte swizzle on both). In place by one warp: rows go in ascending
-    // batches of 16, each read whole before it is written; a write of token
-    // row t lands on the codes of a row t' <= t (keys: region 1 row t is code
-    // row t; values: t' = t + (j + 1) BS - 128 for block j's second half,
-    // lower for its first), so no code is overwritten before it is read.
-    const int cw_ = warp - 6;  // 0 .. 3
+    // Item k of the stream (the producer's order): code stage k % kCodeStages
+    // into ring stage k % kStages, widened exactly to fp16 (cvt.rn.f16x2.e4m3x2,
+    // two codes per instruction; NaN codes stay NaN) in the layout the TMA would
+    // have produced for a 16-bit cache:
+    // keys as two 64-dim regions of 128 rows, values per block as [half][BS
+    // rows][64] (128-byte swizzle on both). The four warps share each item:
+    // thread ct takes 16 codes (dims 16c .. 16c + 15, c = ct % 8) of token rows
+    // ct / 8 + 16u, reads them all, hands the code stage back, then writes.
+    const int ct = threadIdx.x - 6 * 32;  // 0 .. 127
+    const int c = ct & 7;
     bool ok = true;
-    for (uint32_t k = cw_;; k += 4) {
+    for (uint32_t k = 0;; ++k) {
+      const uint32_t cs = k % L::kCodeStages;
       const uint32_t st = k % kStages;
-      if (lane == 0) ok = mbar_wait(&cfull[st], (k / kStages) & 1u, 0x7f03u);
+      if (lane == 0) ok = mbar_wait(&cfull[cs], (k / L::kCodeStages) & 1u, 0x7f03u);
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
-      const int32_t tag = ctags[st];
+      const int32_t tag = ctags[cs];
       if (tag == 2) break;  // end of the stream
+      const uint8_t* src = codes + cs * kCodeBytes;
+      uint4 wv[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int row = (ct >> 3) + 16 * u;
+        wv[u] = *reinterpret_cast<const uint4*>(src + row * 128 + ((c ^ (row & 7)) << 4));
+      }
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&cempty[cs]);  // releases this warp's reads
+        ok = mbar_wait(&empty[st], ((k / kStages) & 1u) ^ 1u, 0x7f04u);
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
       uint8_t* dst = ring + st * kStageBytes;
-      const uint8_t* src = dst + kCodeOffset;
-      const int c = lane & 7;  // 16 codes: dims 16c .. 16c + 15
-#pragma unroll 1
-      for (int r0 = 0; r0 < kTileTok; r0 += 16) {
-        uint4 wv[4];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int row = r0 + 4 * u + (lane >> 3);
-          wv[u] = *reinterpret_cast<const uint4*>(src + row * 128 + ((c ^ (row & 7)) << 4));
+      for (int u = 0; u < 8; ++u) {
+        const int row = (ct >> 3) + 16 * u;
+        const uint32_t cw[4] = {wv[u].x, wv[u].y, wv[u].z, wv[u].w};
+        uint32_t h[8];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          h[2 * e] = e4m3x2_to_x2<TM>(cw[e] & 0xFFFFu);
+          h[2 * e + 1] = e4m3x2_to_x2<TM>(cw[e] >> 16);
         }
-        __syncwarp();  // the batch's codes are read before any of its writes
-        // a batch with a NaN code anywhere in the warp widens by cvt (exact
-        // NaNs); the others by the integer path, as straight-line code
-        uint32_t nanw = 0;
-#pragma unroll
-        for (int u = 0; u < 4; ++u)
-          nanw |= e4m3x4_nan_bits(wv[u].x) | e4m3x4_nan_bits(wv[u].y) |
-                  e4m3x4_nan_bits(wv[u].z) | e4m3x4_nan_bits(wv[u].w);
-        uint32_t hv[4][8];
-        if (!__any_sync(0xffffffffu, nanw != 0)) {
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const uint32_t cw[4] = {wv[u].x, wv[u].y, wv[u].z, wv[u].w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) e4m3x4_to_f16x2x2(cw[e], hv[u][2 * e], hv[u][2 * e + 1]);
-          }
-        } else {
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const uint32_t cw[4] = {wv[u].x, wv[u].y, wv[u].z, wv[u].w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              hv[u][2 * e] = e4m3x2_to_x2<TM>(cw[e] & 0xFFFFu);
-              hv[u][2 * e + 1] = e4m3x2_to_x2<TM>(cw[e] >> 16);
-            }
-          }
+        uint8_t* base;
+        int sw;
+        if (tag == 0) {  // key row: region c / 4, row `row`
+          base = dst + (c >> 2) * kRegionBytes + row * 128;
+          sw = row & 7;
+        } else {  // value row: block row / BS, half c / 4, row row % BS
+          const int jb = row / BS, ib = row % BS;
+          base = dst + jb * BS * 256 + (c >> 2) * BS * 128 + ib * 128;
+          sw = ib & 7;
         }
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int row = r0 + 4 * u + (lane >> 3);
-          const uint32_t* h = hv[u];
-          uint8_t* base;
-          int sw;
-          if (tag == 0) {  // key row: region c / 4, row `row`
-            base = dst + (c >> 2) * kRegionBytes + row * 128;
-            sw = row & 7;
-          } else {  // value row: block row / BS, half c / 4, row row % BS
-            const int jb = row / BS, ib = row % BS;
-            base = dst + jb * BS * 256 + (c >> 2) * BS * 128 + ib * 128;
-            sw = ib & 7;
-          }
-          // 16-byte chunks ch, ch + 1 of the 128-byte row. A 16-byte store is
-          // served eight lanes at a time, and lanes c and c + 4 (same row, other
-          // region) would meet at the same bank positions: lanes of the second
-          // region store chunk ch + 1 first, so each group of eight covers all 32
-          // banks once.
-          const int ch = 2 * (c & 3);
-          const bool sec = c >= 4;
-          const uint4 d0 = make_uint4(h[0], h[1], h[2], h[3]);
-          const uint4 d1 = make_uint4(h[4], h[5], h[6], h[7]);
-          *reinterpret_cast<uint4*>(base + (((ch + (sec ? 1 : 0)) ^ sw) << 4)) = sec ? d1 : d0;
-          *reinterpret_cast<uint4*>(base + (((ch + (sec ? 0 : 1)) ^ sw) << 4)) = sec ? d0 : d1;
-        }
-        __syncwarp();  // this batch's writes precede the next batch's reads
+        // 16-byte chunks ch, ch + 1 of the 128-byte row. A 16-byte store is served
+        // eight lanes at a time, and lanes c and c + 4 (same row, other region)
+        // would meet at the same bank positions: lanes of the second region store
+        // chunk ch + 1 first, so each group of eight covers all 32 banks once.
+        const int ch = 2 * (c & 3);
+        const bool sec = c >= 4;
+        const uint4 d0 = make_uint4(h[0], h[1], h[2], h[3]);
+        const uint4 d1 = make_uint4(h[4], h[5], h[6], h[7]);
+        *reinterpret_cast<uint4*>(base + (((ch + (sec ? 1 : 0)) ^ sw) << 4)) = sec ? d1 : d0;
+        *reinterpret_cast<uint4*>(base + (((ch + (sec ? 0 : 1)) ^ sw) << 4)) = sec ? d0 : d1;
       }
       fence_proxy_async_smem();
       __syncwarp();
