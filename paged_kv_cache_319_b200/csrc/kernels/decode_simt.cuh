@@ -667,7 +667,9 @@ constexpr int kReduceHeads = KVP_REDUCE_HEADS;
 template <typename T, int D>
 __global__ void __launch_bounds__(kReduceHeads * D) decode_reduce_kernel(const DecodeArgs a) {
   extern __shared__ float wsh[];  // [kReduceHeads][ws_slots] weights, then [kReduceHeads] sums
-  pdl_wait();  // launched programmatically: the partition kernel must be complete
+  // The context length and the plan words are the call's inputs, not pass 1's
+  // outputs: they are read before the wait for pass 1, so only the partials'
+  // loads follow it.
   const int h0 = blockIdx.x * kReduceHeads;
   const int row = blockIdx.y;          // a sequence, or one of its q_len query rows
   const int s = row / a.q_len;
@@ -691,26 +693,32 @@ __global__ void __launch_bounds__(kReduceHeads * D) decode_reduce_kernel(const D
     }
   } else {
     nparts = (ctx + a.part_tokens - 1) / a.part_tokens;
-    if (nparts <= 1) return;  // pass 1 wrote the output
-    if (a.q_len > 1) {  // query row i of a chunk sees ctx - q_len + i + 1 tokens
+    if (nparts > 1 && a.q_len > 1) {  // query row i of a chunk sees ctx - q_len + i + 1 tokens
       const int32_t vis = min(ctx, max(0, ctx - a.q_len + row % a.q_len + 1));
       nparts = (vis + a.part_tokens - 1) / a.part_tokens;
     }
   }
+  // every CTA waits, so that the grid completes only after the partition kernel
+  pdl_wait();  // launched programmatically: the partition kernel must be complete
+  if (!a.plan && (ctx + a.part_tokens - 1) / a.part_tokens <= 1) return;  // pass 1 wrote the output
   const bool head = h0 + i < a.num_q_heads;
   const int64_t row_sh = int64_t(row) * a.num_q_heads + h0 + i;
   float* lsh = wsh + kReduceHeads * a.ws_slots;
-  if (head && t == 0) {  // the weights of head h0 + i
+  if (head && t < 32) {  // the weights of head h0 + i, by its first warp: lane p takes
+                         // partitions p, p + 32, ... (their loads go out together)
     const float* ml = a.ws_ml + row_sh * a.ws_slots * 2;
     float M = -INFINITY;
-    for (int p = 0; p < nparts; ++p) M = fmaxf(M, ml[2 * p]);
+    for (int p = t; p < nparts; p += 32) M = fmaxf(M, ml[2 * p]);
+    M = warp_max(M);
     float L = 0.f;
-    for (int p = 0; p < nparts; ++p) {
+    for (int p = t; p < nparts; p += 32) {
       const float w = (ml[2 * p] == -INFINITY || M == -INFINITY) ? 0.f : exp2f(ml[2 * p] - M);
       wsh[i * a.ws_slots + p] = w;
       L += ml[2 * p + 1] * w;
     }
-    lsh[i] = L;
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+    if (t == 0) lsh[i] = L;
   }
   __syncthreads();
   if (!head) return;
