@@ -619,7 +619,8 @@ def decode_record(name, device, calls=DECODE_WINDOW_CALLS):
                          "peak_source": peak_kind, "unit": "GB/s",
                          "frac": round(achieved / peak, 4),
                          "frac_of_nominal_8tbs": round(achieved / 8000.0, 4),
-                         "algorithmic_bytes_per_launch": int(alg)},
+                         "algorithmic_bytes_per_launch": int(alg),
+                         "traffic": traffic_per_launch(kernel, alg)},
             "clocks": clk.summary(min_samples=20)}
 
 
