@@ -62,12 +62,15 @@ using kvp::fail;
 #ifndef KVP_GROUP_PER_HEAD_BELOW
 #define KVP_GROUP_PER_HEAD_BELOW 4
 #endif
-// Warps and stages of the CUDA-core kernel on longer own ranges.
+// Warps and stages of the CUDA-core kernel on longer own ranges. One stage per
+// warp: an own range is a few blocks per (sequence, head), so a deeper ring
+// buys little, and 32 KiB of tiles per CTA lets registers, not shared memory,
+// set the CTAs per SM (four at 4 warps).
 #ifndef KVP_GROUP_SPLIT_WARPS
 #define KVP_GROUP_SPLIT_WARPS KVP_SIMT_WARPS
 #endif
 #ifndef KVP_GROUP_SPLIT_STAGES
-#define KVP_GROUP_SPLIT_STAGES KVP_SIMT_STAGES
+#define KVP_GROUP_SPLIT_STAGES 1
 #endif
 
 namespace {
