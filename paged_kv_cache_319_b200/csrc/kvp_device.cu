@@ -1404,10 +1404,15 @@ int attention_decode_vcache(const void* q, const kvp_vcache* vc, const int32_t* 
     rc = make_map_vcache(&km, kb, dtype, tokens, uint32_t(Hkv), kSimtTile, 2);
     if (!rc) rc = make_map_vcache(&vm, vb, dtype, tokens, uint32_t(Hkv), kSimtTile, 2);
     if (rc) return rc;
+    // the paged decode's shapes, by the same batch-size rule, so the A/B compares like with like
     constexpr int W = KVP_SIMT_WARPS, N = KVP_SIMT_STAGES;
-    rc = dtype == KVP_F16
-             ? launch_simt<__half, 128, kSimtTile, W, N, false, false, true>(km, vm, a, st)
-             : launch_simt<__nv_bfloat16, 128, kSimtTile, W, N, false, false, true>(km, vm, a, st);
+    const bool f16 = dtype == KVP_F16;
+    if (num_seqs >= KVP_SIMT_ONE_STAGE_SEQS)
+      rc = f16 ? launch_simt<__half, 128, kSimtTile, W, 1, false, false, true>(km, vm, a, st)
+               : launch_simt<__nv_bfloat16, 128, kSimtTile, W, 1, false, false, true>(km, vm, a, st);
+    else
+      rc = f16 ? launch_simt<__half, 128, kSimtTile, W, N, false, false, true>(km, vm, a, st)
+               : launch_simt<__nv_bfloat16, 128, kSimtTile, W, N, false, false, true>(km, vm, a, st);
   }
   if (rc || pmax <= 1) return rc;
   return dtype == KVP_F16 ? launch_reduce<__half, 128>(a, st) : launch_reduce<__nv_bfloat16, 128>(a, st);

@@ -77,6 +77,8 @@ CASES = [
     (32, 8, [1, 100, 129, 5000, 9000], "bf16", 512),
     (16, 4, [7, 128, 256, 3000], "f16", 1024),
     (64, 4, [33, 1024, 2500], "bf16", 512),
+    # 130 sequences: the CUDA cores' one-stage shape for large batches
+    (8, 8, [1, 16, 17, 200, 511] * 26, "f16", 256),
 ]
 
 
@@ -130,15 +132,17 @@ def test_vcache_slots_in_any_order():
         vc.close()
 
 
-@pytest.mark.parametrize("part", [0, 512])
-def test_vcache_equals_paged_decode_bit_for_bit_on_the_cuda_cores(part):
+@pytest.mark.parametrize("part,lens", [(0, [1, 16, 17, 511, 1200, 2048]),
+                                       (512, [1, 16, 17, 511, 1200, 2048]),
+                                       # 130 sequences: both take the one-stage shape
+                                       (256, [1, 16, 17, 200, 511] * 26)])
+def test_vcache_equals_paged_decode_bit_for_bit_on_the_cuda_cores(part, lens):
     # same tiles (16 tokens), same warps, same order: only the address differs
     import torch
     import paged_kv_cache_319_b200 as kvp
 
-    lens = [1, 16, 17, 511, 1200, 2048]
     S, Hkv, bs = len(lens), 8, 16
-    vc = kvp.VCache(S, 2048, Hkv, D, "f16")
+    vc = kvp.VCache(S, max(lens), Hkv, D, "f16")
     try:
         kh, vh = _fill(vc, lens, Hkv, "f16", seed=23)
         need = [-(-n // bs) for n in lens]
@@ -160,9 +164,9 @@ def test_vcache_equals_paged_decode_bit_for_bit_on_the_cuda_cores(part):
         cl = torch.tensor(lens, dtype=torch.int32, device="cuda")
         paged = kvp.paged_attention_decode(q, from_bits(kp, "f16"), from_bits(vp, "f16"),
                                            torch.from_numpy(tables).cuda(), cl, 0.088,
-                                           max_context_len=2048, partition_size=part)
+                                           max_context_len=max(lens), partition_size=part)
         contig = kvp.attention_decode_vcache(q, vc, torch.arange(S, dtype=torch.int32, device="cuda"),
-                                             cl, 0.088, max_context_len=2048, partition_size=part)
+                                             cl, 0.088, max_context_len=max(lens), partition_size=part)
         kvp.check_device_error()
         assert np.array_equal(to_bits(paged), to_bits(contig))
     finally:
